@@ -1,0 +1,361 @@
+"""Pins of the fp64 oracle to things other than itself: the pages' worked
+numbers (tests/golden, each with its citation), closed forms, special cases
+that reduce to a library routine, and brute force on tiny inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from conftest import read_golden
+
+rng = np.random.default_rng(1234)
+
+
+# ---------------------------------------------------------------------------
+# step 1: pooling
+# ---------------------------------------------------------------------------
+def _worked_example_inputs(weight_on):
+    """m = 2, entry i = 1: a branch = tokens 2, 3, b branch = tokens 0, 1."""
+    g = read_golden("pooling_worked_example.txt")
+    a = [float(x) for x in g["a_content"][0]]
+    b = [float(x) for x in g["b_content"][0]]
+    ex = [float(x) for x in g["exp_logits"][0]]
+    Ca = np.zeros((4, 1)); Cb = np.zeros((4, 1)); Za = np.zeros((4, 1)); Zb = np.zeros((4, 1))
+    Ca[2, 0], Ca[3, 0] = a
+    Cb[0, 0], Cb[1, 0] = b
+    # logits whose exponentials are the printed (2, 1, 1, 1), in the given order
+    slots = {"a1": (Za, 2), "a2": (Za, 3), "b1": (Zb, 0), "b2": (Zb, 1)}
+    for name, e in zip(weight_on, ex):
+        arr, row = slots[name]
+        arr[row, 0] = math.log(e)
+    return Ca, Za, Cb, Zb, g
+
+
+def test_pooling_worked_example_listed_order():
+    Ca, Za, Cb, Zb, g = _worked_example_inputs(["a1", "a2", "b1", "b2"])
+    out = oracle.pool_overlap(Ca, Za, Cb, Zb, m=2)
+    assert out.shape == (2, 1)
+    assert out[1, 0] == pytest.approx(float(g["result_listed_order"][0][0]), abs=1e-12)
+
+
+def test_pooling_worked_example_chronological_order():
+    Ca, Za, Cb, Zb, g = _worked_example_inputs(["b1", "b2", "a1", "a2"])
+    out = oracle.pool_overlap(Ca, Za, Cb, Zb, m=2)
+    assert out[1, 0] == pytest.approx(float(g["result_chronological_order"][0][0]), abs=1e-12)
+
+
+def test_pooling_weights_printed():
+    g = read_golden("pooling_worked_example.txt")
+    ex = np.array([float(x) for x in g["exp_logits"][0]])
+    w = np.array([float(x) for x in g["weights"][0]])
+    # the oracle's pooling with content = one-hot picks out each weight
+    for j in range(4):
+        C = np.zeros((4, 1)); C[j, 0] = 1.0
+        Z = np.log(ex)[:, None]
+        assert oracle.pool_block(C, Z, m=4)[0, 0] == pytest.approx(w[j], abs=1e-12)
+
+
+def test_overlap_first_entry_closed_form():
+    """Entry 0 has no previous block: b branch masked, all weight on tokens
+    0..m-1 (Ch.5 'Receptive field versus compression stride').  Closed form:
+    logits (0, ln 3) on contents (4, 8) -> 0.25*4 + 0.75*8 = 7."""
+    Ca = np.array([[4.0], [8.0], [100.0], [100.0]])
+    Za = np.array([[0.0], [math.log(3.0)], [0.0], [0.0]])
+    Cb = np.full((4, 1), 1e6)   # must not leak into entry 0
+    Zb = np.full((4, 1), 50.0)
+    out = oracle.pool_overlap(Ca, Za, Cb, Zb, m=2)
+    assert out[0, 0] == pytest.approx(7.0, abs=1e-12)
+
+
+def test_overlap_m1_is_two_way_sigmoid():
+    """m = 1: entry i mixes token i (a) and token i-1 (b) with weight
+    sigmoid(za - zb) on the a side."""
+    N = 6
+    Ca, Za, Cb, Zb = (rng.standard_normal((N, 3)) for _ in range(4))
+    out = oracle.pool_overlap(Ca, Za, Cb, Zb, m=1)
+    for i in range(1, N):
+        wa = 1.0 / (1.0 + np.exp(Zb[i - 1] - Za[i]))
+        np.testing.assert_allclose(out[i], wa * Ca[i] + (1 - wa) * Cb[i - 1], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out[0], Ca[0], atol=1e-12)
+
+
+def test_overlap_b_branch_uses_previous_block_and_bias_positions():
+    """m = 2 with all logits equal except biases: Ba = (ln 3, 0), Bb = (0, ln 2)
+    give weights 3:1 on the a tokens and 1:2 on the b tokens."""
+    m = 2
+    Ca = np.array([[1.0], [2.0], [3.0], [4.0]])
+    Cb = np.array([[10.0], [20.0], [30.0], [40.0]])
+    Z = np.zeros((4, 1))
+    Ba = np.array([[math.log(3.0)], [0.0]])
+    Bb = np.array([[0.0], [math.log(2.0)]])
+    out = oracle.pool_overlap(Ca, Z, Cb, Z, m, Ba, Bb)
+    # entry 1: a = tokens 2,3 (weights 3,1), b = tokens 0,1 (weights 1,2); total 7
+    want = (3 * 3.0 + 1 * 4.0 + 1 * 10.0 + 2 * 20.0) / 7.0
+    assert out[1, 0] == pytest.approx(want, abs=1e-12)
+
+
+def test_block_bias_is_indexed_by_position_in_block():
+    m = 2
+    C = np.array([[1.0], [5.0], [7.0], [11.0], [13.0]])   # 5 tokens -> 2 entries
+    Z = np.zeros((5, 1))
+    B = np.array([[math.log(3.0)], [0.0]])
+    out = oracle.pool_block(C, Z, m, B)
+    assert out.shape == (2, 1)     # the trailing token makes no entry
+    np.testing.assert_allclose(out[:, 0], [(3 * 1 + 5) / 4, (3 * 7 + 11) / 4], atol=1e-12)
+
+
+def test_block_special_cases():
+    C = rng.standard_normal((12, 5))
+    Z = rng.standard_normal((12, 5))
+    np.testing.assert_allclose(oracle.pool_block(C, Z, m=1), C, atol=1e-15)          # identity
+    np.testing.assert_allclose(oracle.pool_block(C, np.zeros_like(Z), m=4),
+                               C.reshape(3, 4, 5).mean(axis=1), atol=1e-12)           # mean
+    np.testing.assert_allclose(oracle.pool_block(np.full_like(C, 2.5), Z, m=3),
+                               np.full((4, 5), 2.5), atol=1e-12)                      # sums to 1
+    Zbig = np.zeros_like(Z); Zbig[5] = 1000.0                                          # stability
+    out = oracle.pool_block(C, Zbig, m=4)
+    np.testing.assert_allclose(out[1], C[5], atol=1e-12)
+
+
+def test_coordinatewise_independence():
+    """Weights are computed per coordinate: coordinate 0 may favour token 0
+    while coordinate 1 favours token 3 (Ch.5 'Coordinate-wise softmax
+    pooling')."""
+    C = np.arange(8.0).reshape(4, 2)
+    Z = np.array([[50.0, 0.0], [0.0, 0.0], [0.0, 0.0], [0.0, 50.0]])
+    out = oracle.pool_block(C, Z, m=4)
+    np.testing.assert_allclose(out[0], [C[0, 0], C[3, 1]], atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# steps 2-3: indexer and top-k
+# ---------------------------------------------------------------------------
+def _toy_indexer():
+    g = read_golden("indexer_toy_example.txt")
+    table = {row[0]: [float(x) for x in row[1:]] for row in g["table"]}
+    names = ["A", "B", "C"]
+    # keys / queries with q_h . K_s = table[s][h]; q is not the identity so a
+    # transposed operand would change the numbers: q1 = (1, 1), q2 = (0, 1)
+    qI = np.array([[1.0, 1.0], [0.0, 1.0]])
+    KI = np.array([[table[n][0] - table[n][1], table[n][1]] for n in names])
+    np.testing.assert_allclose(KI @ qI.T, [table[n] for n in names])
+    return g, names, qI, KI
+
+
+def test_indexer_toy_scores():
+    g, names, qI, KI = _toy_indexer()
+    w = np.array([float(x) for x in g["w_second"][0]])
+    want = [float(x) for x in g["scores_second"][0]]
+    np.testing.assert_allclose(oracle.indexer_scores(qI, w, KI), want, atol=1e-12)
+    assert names[int(np.argmax(oracle.indexer_scores(qI, w, KI)))] == "B"
+
+
+def test_indexer_toy_ranking():
+    g, names, qI, KI = _toy_indexer()
+    w = np.array([float(x) for x in g["w_first"][0]])
+    sel = oracle.topk_select(oracle.indexer_scores(qI, w, KI), 2)
+    assert [names[i] for i in sel] == g["top2_first"][0]
+
+
+def test_indexer_relu_clips_each_head():
+    qI = np.array([[1.0, 0.0], [0.0, 1.0]])
+    KI = np.array([[-2.0, 3.0], [-1.0, -1.0]])
+    w = np.array([0.2, 0.8])
+    # head 1 negative -> 0; block 2 all heads negative -> exactly 0
+    np.testing.assert_allclose(oracle.indexer_scores(qI, w, KI), [0.8 * 3.0, 0.0], atol=0)
+
+
+def _brute_topk(scores, k):
+    """Element i is selected iff fewer than k elements beat it, where j beats
+    i when s_j > s_i or (s_j == s_i and j < i)."""
+    s = np.asarray(scores, dtype=np.float32)
+    n = s.shape[0]
+    sel = [i for i in range(n) if sum(1 for j in range(n) if s[j] > s[i] or (s[j] == s[i] and j < i)) < k]
+    return np.array(sel, dtype=np.int64)
+
+
+@pytest.mark.parametrize("n,k", [(1, 1), (5, 2), (17, 4), (40, 7), (64, 63), (9, 20)])
+def test_topk_matches_brute_force_with_ties(n, k):
+    for trial in range(5):
+        s = rng.integers(-3, 4, size=n).astype(np.float64)        # many exact ties
+        s[rng.random(n) < 0.2] = -0.0                               # signed zeros tie with +0
+        got = oracle.topk_select(s, k)
+        np.testing.assert_array_equal(got, _brute_topk(s, k))
+        assert np.all(np.diff(got) > 0)                             # ascending
+        assert got.shape[0] == min(n, k)
+
+
+def test_topk_decides_in_fp32():
+    """Scores equal after fp32 rounding are ties (lower index wins)."""
+    s = np.array([1.0, 1.0 + 1e-12, 0.5])
+    np.testing.assert_array_equal(oracle.topk_select(s, 1), [0])
+
+
+def test_causal_eligibility():
+    assert [oracle.eligible_entries(t, 4) for t in range(10)] == [0, 0, 0, 0, 1, 1, 1, 1, 2, 2]
+    L, m, k = 40, 4, 3
+    qI = rng.standard_normal((L, 2, 8)); w = rng.random((L, 2)); KI = rng.standard_normal((L // m, 8))
+    idx, cnt = oracle.csa_prefill_topk(qI, w, KI, m, k)
+    for t in range(L):
+        n = t // m
+        assert cnt[t] == min(k, n)
+        assert np.all(idx[t, :cnt[t]] < n) and np.all(idx[t, cnt[t]:] == -1)
+
+
+# ---------------------------------------------------------------------------
+# step 4: attention
+# ---------------------------------------------------------------------------
+def _sdpa_causal(q, kv, lam, bias=None):
+    """torch's scaled_dot_product_attention in float64, one shared KV head
+    serving as both K and V, causal."""
+    L, H, d = q.shape
+    qt = torch.from_numpy(q).permute(1, 0, 2)[None]                       # [1, H, L, d]
+    kt = torch.from_numpy(kv)[None, None].expand(1, H, L, d)
+    if bias is None:
+        o = F.scaled_dot_product_attention(qt, kt, kt, is_causal=True, scale=lam)
+    else:
+        o = F.scaled_dot_product_attention(qt, kt, kt, attn_mask=torch.from_numpy(bias), scale=lam)
+    return o[0].permute(1, 0, 2).numpy()
+
+
+def _csa_m1_inputs(L=24, H=3, d=16):
+    q = rng.standard_normal((L, H, d))
+    kv = rng.standard_normal((L, d))
+    Z = rng.standard_normal((L, d))
+    kI = rng.standard_normal((L, 8)); ZI = rng.standard_normal((L, 8))
+    qI = rng.standard_normal((L, 2, 8)); w = rng.random((L, 2))
+    return q, kv, Z, kI, ZI, qI, w
+
+
+def test_csa_m1_full_topk_window1_is_dense_causal():
+    """m = 1 pooling is the identity, k >= L selects every earlier token and a
+    window of 1 adds the current one: exactly dense causal MQA."""
+    q, kv, Z, kI, ZI, qI, w = _csa_m1_inputs()
+    L = q.shape[0]
+    lam = 0.37
+    # no bf16 storage rounding here: compare the definitions exactly
+    kv_comp = oracle.pool_block(kv, Z, 1)
+    idx, cnt = oracle.csa_prefill_topk(qI, w, oracle.pool_block(kI, ZI, 1), 1, L)
+    out, _ = oracle.csa_prefill_attention(q, kv_comp, kv, idx, cnt, 1, lam)
+    np.testing.assert_allclose(out, _sdpa_causal(q, kv, lam), atol=1e-12)
+
+
+def test_csa_m1_window_duplicates_closed_form():
+    """With W > 1 the tokens t-W+1 .. t-1 appear both as selected entries and
+    in the window; each duplicate adds ln 2 to that position's logit."""
+    q, kv, Z, kI, ZI, qI, w = _csa_m1_inputs()
+    L, W, lam = q.shape[0], 5, 0.2
+    idx, cnt = oracle.csa_prefill_topk(qI, w, kI, 1, L)
+    out, _ = oracle.csa_prefill_attention(q, kv, kv, idx, cnt, W, lam)
+    bias = np.full((L, L), -np.inf)
+    for t in range(L):
+        bias[t, : t + 1] = 0.0
+        bias[t, max(0, t - W + 1): t] = math.log(2.0)
+    np.testing.assert_allclose(out, _sdpa_causal(q, kv, lam, bias), atol=1e-12)
+
+
+def test_hca_m1_window1_is_dense_causal():
+    q, kv, *_ = _csa_m1_inputs()
+    lam = 0.5
+    out, _ = oracle.hca_prefill(q, kv, kv, 1, 1, lam)
+    np.testing.assert_allclose(out, _sdpa_causal(q, kv, lam), atol=1e-12)
+
+
+def test_decode_m1_is_last_row_of_dense_causal():
+    """Decode of token N with m = 1, k >= N and a window of 1 (the new token)
+    equals the last row of dense causal attention over N+1 tokens."""
+    N, H, d = 30, 4, 8
+    kv = rng.standard_normal((N + 1, d))
+    q = rng.standard_normal((N + 1, H, d))
+    qI = rng.standard_normal((1, 2, 8)); w = rng.random((1, 2)); kI = rng.standard_normal((N, 8))
+    out, _, idx, cnt = oracle.csa_decode(q[N:N + 1], [kv[:N]], [kI], qI, w, kv[None, N:N + 1],
+                                         [1], [N], 1, N, 0.3)
+    assert cnt[0] == N
+    np.testing.assert_allclose(out[0], _sdpa_causal(q, kv, 0.3)[N], atol=1e-12)
+    out_h, _ = oracle.hca_decode(q[N:N + 1], [kv[:N]], kv[None, N:N + 1], [1], [N], 1, 0.3)
+    np.testing.assert_allclose(out_h[0], out[0], atol=1e-12)
+
+
+def test_attention_weights_sum_to_one():
+    v = rng.standard_normal(6)
+    rows = np.tile(v, (9, 1))
+    o, _ = oracle.attend_shared_kv(rng.standard_normal((4, 6)), rows, 0.7)
+    np.testing.assert_allclose(o, np.tile(v, (4, 1)), atol=1e-12)
+
+
+def test_sink_worked_example():
+    g = read_golden("sink_example.txt")
+    real, sink, want = (float(g[k][0][0]) for k in ("real_mass", "sink_mass", "real_weight"))
+    # one real entry whose logit is ln(real): q . kv = ln(real) with lam = 1
+    kv = np.array([[math.log(real), 2.0]])
+    q = np.array([[1.0, 0.0]])
+    o, lse = oracle.attend_shared_kv(q, kv, 1.0, sink=np.array([math.log(sink)]))
+    np.testing.assert_allclose(o[0], want * kv[0], atol=1e-12)
+    assert lse[0] == pytest.approx(math.log(real + sink), abs=1e-12)
+
+
+def test_lse_without_sink():
+    q = rng.standard_normal((3, 5)); rows = rng.standard_normal((7, 5))
+    _, lse = oracle.attend_shared_kv(q, rows, 0.4)
+    np.testing.assert_allclose(lse, np.log(np.exp(0.4 * q @ rows.T).sum(1)), atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# storage rounding
+# ---------------------------------------------------------------------------
+def test_bf16_round_matches_torch():
+    x = rng.standard_normal(10000) * 10.0 ** rng.integers(-5, 5, 10000)
+    want = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(oracle.bf16_round(x), want)
+
+
+# ---------------------------------------------------------------------------
+# cost model (Ch.8)
+# ---------------------------------------------------------------------------
+def test_cost_model_matches_pages():
+    cm = oracle.cost_model
+    g = read_golden("cost_model.txt")
+    gqa_pro = cm.gqa8_cache_bytes(10**6, 61)
+    gqa_flash = cm.gqa8_cache_bytes(10**6, 43)
+    pro = cm.model_cache_bytes(10**6, 30, 31)
+    flash = cm.model_cache_bytes(10**6, 21, 20)
+    d_f, g_f = cm.grouped_out_proj_params(64, 512, 4096, 8, 1024)
+    d_p, g_p = cm.grouped_out_proj_params(128, 512, 7168, 16, 1024)
+    csa_fl = cm.attention_flops(128, 512, 1024 + 128)
+    got = {
+        "gqa8_bytes_per_token_layer": cm.gqa8_bytes_per_token_layer(),
+        "gqa8_layer_bytes_1M": cm.gqa8_cache_bytes(10**6, 1),
+        "gqa8_61_layers_1M": gqa_pro,
+        "gqa8_43_layers_1M": gqa_flash,
+        "entry_bytes": cm.v4_entry_bytes(),
+        "csa_main_bytes_per_token": cm.main_cache_bytes_per_token(4),
+        "hca_main_bytes_per_token": cm.main_cache_bytes_per_token(128),
+        "indexer_key_bytes": cm.indexer_key_bytes(),
+        "indexer_bytes_per_token": cm.indexer_key_bytes() / 4,
+        "csa_total_bytes_per_token": cm.csa_bytes_per_token(),
+        "pro_cache_1M_bytes": pro,
+        "flash_cache_1M_bytes": flash,
+        "pro_over_gqa8": pro / gqa_pro,
+        "flash_over_gqa8": flash / gqa_flash,
+        "fp4_scale_overhead": cm.fp4_scale_overhead(),
+        "csa_attention_flops": csa_fl,
+        "hca_attention_flops": cm.attention_flops(128, 512, cm.hca_entries(10**6)[0] + 128),
+        "indexer_ops": cm.indexer_ops(10**6, 4, 64, 128),
+        "indexer_over_csa_main": cm.indexer_ops(10**6, 4, 64, 128) / csa_fl,
+        "hca_entries_1M": cm.hca_entries(10**6)[0],
+        "hca_trailing_1M": cm.hca_entries(10**6)[1],
+        "flash_out_proj_ratio": g_f / d_f,
+        "pro_out_proj_ratio": g_p / d_p,
+        "pro_out_proj_saving": d_p - g_p,
+    }
+    assert set(got) == set(g)
+    for name, rows in g.items():
+        want, tol = float(rows[0][0]), float(rows[0][1])
+        v = float(got[name])
+        if tol == 0:
+            assert v == want, name
+        else:
+            assert abs(v - want) <= tol * abs(want), (name, v, want)

@@ -1,0 +1,13 @@
+"""B200-native (sm_100a) CSA / HCA hot path: block compression, lightning
+indexer + top-k, and sparse / dense shared-KV attention with a sliding window.
+
+The computation runs in the CUDA library ``_csa_b200.so`` (C ABI:
+include/csa.h); this package is its thin Python binding.
+"""
+from ._lib import (CsaError, KERNEL_ATTENTION, KERNEL_COMPRESS, KERNEL_INDEXER_SCORE,  # noqa: F401
+                   KERNEL_MERGE, KERNEL_TOPK_SELECT, load)
+from .api import (Cache, Workspace, compress_kv, hca_attn, indexer_topk, launch_count,  # noqa: F401
+                  set_timing_events, sparse_attn_decode, sparse_attn_prefill)
+
+__all__ = ["Cache", "Workspace", "CsaError", "compress_kv", "indexer_topk", "sparse_attn_prefill",
+           "sparse_attn_decode", "hca_attn", "launch_count", "set_timing_events", "load"]

@@ -1,0 +1,273 @@
+"""Python entry points with the names of the C ABI (include/csa.h).
+
+Arguments are torch CUDA tensors; results are written by the CUDA library on
+the current torch stream.  Shapes follow the header:
+
+    compress_kv          (step 1)    C, Z [N, dim] -> [N // m, dim]
+    indexer_topk         (steps 2-3) q_idx [T, H_I, c_I], w [T, H_I], keys -> idx [T, k], count [T]
+    sparse_attn_prefill  (step 4)    q [L, H, 128] over kv_comp[idx] + raw window
+    sparse_attn_decode   (step 4)    q [B, H, 128] over cache[idx] + window buffer
+    hca_attn             (step 4)    q [T, H, 128] over all eligible entries + window
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import CacheT, check, load
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype, ndim=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    return t
+
+
+@dataclass
+class Cache:
+    """A compressed cache: ``data`` [rows, dim] bf16, contiguous per sequence
+    (``seq_stride`` rows apart) or paged through ``page_table`` [n_seq,
+    max_pages] int32 with ``page_size`` rows per page."""
+    data: torch.Tensor
+    seq_stride: int = 0
+    page_table: Optional[torch.Tensor] = None
+    page_size: int = 0
+
+    @staticmethod
+    def contiguous(t):
+        """[n_seq, S, dim] -> one contiguous cache per sequence."""
+        return Cache(t.reshape(-1, t.shape[-1]), seq_stride=t.shape[-2] if t.dim() == 3 else 0)
+
+    @property
+    def dim(self):
+        return self.data.shape[-1]
+
+    def c(self):
+        _need(self.data, "cache.data", torch.bfloat16, 2)
+        if self.page_table is not None:
+            _need(self.page_table, "cache.page_table", torch.int32, 2)
+            return CacheT(self.data.data_ptr(), self.data.shape[0], 0, self.page_table.data_ptr(),
+                          self.page_size, self.page_table.shape[1])
+        return CacheT(self.data.data_ptr(), self.data.shape[0], self.seq_stride, None, 0, 0)
+
+
+class Workspace:
+    """Device scratch for the calls that take one; grows on demand.  The
+    header is zeroed at allocation (csa_workspace_init)."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device if device is not None else "cuda")
+        self.buf = None
+
+    def get(self, nbytes):
+        nbytes = max(int(nbytes), 256)
+        if self.buf is None or self.buf.numel() < nbytes + 256:
+            self.buf = torch.zeros(nbytes + 256, dtype=torch.uint8, device=self.device)
+        base = self.buf.data_ptr()
+        off = (-base) % 256
+        return C.c_void_p(base + off), self.buf.numel() - off
+
+    def check(self, stream=None):
+        """Synchronise and raise CsaError if a kernel recorded a device check."""
+        if self.buf is None:
+            return
+        ptr, _ = self.get(256)
+        check(load().csa_workspace_check(ptr, _stream(stream)))
+
+
+_default_ws = {}
+
+
+def _ws(ws, device):
+    if ws is not None:
+        return ws
+    key = torch.device(device).index
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+# ---------------------------------------------------------------------------
+def compress_kv(C_a, Z_a, m, *, C_b=None, Z_b=None, bias=None, overlap=False, out=None,
+                stream=None):
+    """Step 1: coordinate-wise softmax pooling of [N, dim] into [N // m, dim]."""
+    _need(C_a, "C_a", torch.bfloat16, 2)
+    _need(Z_a, "Z_a", torch.bfloat16, 2, C_a.device)
+    if Z_a.shape != C_a.shape:
+        raise ValueError("C_a and Z_a shapes differ")
+    N, dim = C_a.shape
+    for name, t in (("C_b", C_b), ("Z_b", Z_b)):
+        if t is not None:
+            _need(t, name, torch.bfloat16, 2, C_a.device)
+            if t.shape != C_a.shape:
+                raise ValueError(f"{name} shape differs from C_a")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, None, C_a.device)
+        want = (2, m, dim) if overlap else (m, dim)
+        if tuple(bias.shape) != want:
+            raise ValueError(f"bias must be {want}")
+    if out is None:
+        out = torch.empty((N // m, dim), dtype=torch.bfloat16, device=C_a.device)
+    _need(out, "out", torch.bfloat16, 2, C_a.device)
+    check(load().csa_compress_kv(_ptr(C_a), _ptr(Z_a), _ptr(C_b), _ptr(Z_b), _ptr(bias), N, dim,
+                                 m, int(bool(overlap)), _ptr(out), _stream(stream)))
+    return out
+
+
+def indexer_topk(q_idx, w, keys: Cache, m, top_k, *, seq_id=None, q_pos=None, max_entries=None,
+                 return_scores=False, ws=None, stream=None, out=None):
+    """Steps 2-3: lightning-indexer scores and exact top-k per query.
+    Returns (idx [T, top_k] int32, count [T] int32[, scores [T, top_k] fp32])."""
+    _need(q_idx, "q_idx", torch.bfloat16, 3)
+    T, H_I, c_I = q_idx.shape
+    dev = q_idx.device
+    _need(w, "w", torch.float32, 2, dev)
+    if tuple(w.shape) != (T, H_I):
+        raise ValueError("w must be [T, H_I]")
+    if keys.dim != c_I:
+        raise ValueError("indexer keys dim differs from c_I")
+    if seq_id is not None:
+        _need(seq_id, "seq_id", torch.int32, 1, dev)
+    if q_pos is not None:
+        _need(q_pos, "q_pos", torch.int64, 1, dev)
+    if max_entries is None:
+        if q_pos is None:
+            max_entries = max(T - 1, 0) // m
+        else:
+            raise ValueError("max_entries is required with q_pos")
+    if out is None:
+        idx = torch.empty((T, top_k), dtype=torch.int32, device=dev)
+        cnt = torch.empty((T,), dtype=torch.int32, device=dev)
+        sco = torch.empty((T, top_k), dtype=torch.float32, device=dev) if return_scores else None
+    else:
+        idx, cnt, sco = out
+    lib = load()
+    wsp, wsb = _ws(ws, dev).get(lib.csa_indexer_topk_workspace_size(T, max_entries, top_k))
+    kc = keys.c()
+    check(lib.csa_indexer_topk(_ptr(q_idx), _ptr(w), C.byref(kc), _ptr(seq_id), _ptr(q_pos), T,
+                               H_I, c_I, m, max_entries, top_k, _ptr(idx), _ptr(cnt), _ptr(sco),
+                               wsp, wsb, _stream(stream)))
+    return (idx, cnt, sco) if return_scores else (idx, cnt)
+
+
+def sparse_attn_prefill(q, kv_comp, kv_raw, idx, count, window, sm_scale, *, sink=None,
+                        return_lse=False, ws=None, stream=None, out=None):
+    """Step 4 (CSA prefill): query t attends to kv_comp[idx[t, :count[t]]]
+    and the raw window rows max(0, t-W+1) .. t."""
+    _need(q, "q", torch.bfloat16, 3)
+    L, H, d = q.shape
+    dev = q.device
+    _need(kv_comp, "kv_comp", torch.bfloat16, 2, dev)
+    _need(kv_raw, "kv_raw", torch.bfloat16, 2, dev)
+    _need(idx, "idx", torch.int32, 2, dev)
+    _need(count, "count", torch.int32, 1, dev)
+    if sink is not None:
+        _need(sink, "sink", torch.float32, 1, dev)
+    top_k = idx.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((L, H), dtype=torch.float32, device=dev) if return_lse else None
+    lib = load()
+    wsp, wsb = _ws(ws, dev).get(lib.csa_sparse_attn_prefill_workspace_size(L, H, d))
+    check(lib.csa_sparse_attn_prefill(_ptr(q), _ptr(kv_comp), kv_comp.shape[0], _ptr(kv_raw),
+                                      _ptr(idx), _ptr(count), L, H, d, top_k, window,
+                                      float(sm_scale), _ptr(sink), _ptr(out), _ptr(lse), wsp, wsb,
+                                      _stream(stream)))
+    return (out, lse) if return_lse else out
+
+
+def sparse_attn_decode(q, kv: Cache, win, win_len, idx, count, sm_scale, *, sink=None,
+                       return_lse=False, ws=None, stream=None, out=None):
+    """Step 4 (CSA decode): query b attends to entries idx[b, :count[b]] of
+    sequence b of `kv` and its window buffer win[b, :win_len[b]]."""
+    _need(q, "q", torch.bfloat16, 3)
+    B, H, d = q.shape
+    dev = q.device
+    _need(win, "win", torch.bfloat16, 3, dev)
+    _need(win_len, "win_len", torch.int32, 1, dev)
+    _need(idx, "idx", torch.int32, 2, dev)
+    _need(count, "count", torch.int32, 1, dev)
+    if sink is not None:
+        _need(sink, "sink", torch.float32, 1, dev)
+    top_k, window = idx.shape[1], win.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev) if return_lse else None
+    lib = load()
+    wsp, wsb = _ws(ws, dev).get(
+        lib.csa_sparse_attn_decode_workspace_size(B, H, d, top_k, window))
+    kc = kv.c()
+    check(lib.csa_sparse_attn_decode(_ptr(q), C.byref(kc), _ptr(win), _ptr(win_len), _ptr(idx),
+                                     _ptr(count), B, H, d, top_k, window, float(sm_scale),
+                                     _ptr(sink), _ptr(out), _ptr(lse), wsp, wsb, _stream(stream)))
+    return (out, lse) if return_lse else out
+
+
+def hca_attn(q, kv: Cache, kv_win, m, window, sm_scale, *, win_len=None, q_pos=None,
+             max_entries=None, sink=None, return_lse=False, ws=None, stream=None, out=None):
+    """Step 4 (HCA): dense attention over every entry s < floor(t/m) plus the
+    window.  Decode when `win_len` is given (kv_win [T, window, d]); prefill of
+    sequence 0 otherwise (kv_win = raw tokens [*, d])."""
+    _need(q, "q", torch.bfloat16, 3)
+    T, H, d = q.shape
+    dev = q.device
+    if win_len is not None:
+        _need(win_len, "win_len", torch.int32, 1, dev)
+        _need(kv_win, "kv_win", torch.bfloat16, 3, dev)
+    else:
+        _need(kv_win, "kv_win", torch.bfloat16, 2, dev)
+    if q_pos is not None:
+        _need(q_pos, "q_pos", torch.int64, 1, dev)
+    if sink is not None:
+        _need(sink, "sink", torch.float32, 1, dev)
+    if max_entries is None:
+        if q_pos is None:
+            max_entries = max(T - 1, 0) // m
+        else:
+            raise ValueError("max_entries is required with q_pos")
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((T, H), dtype=torch.float32, device=dev) if return_lse else None
+    lib = load()
+    wsp, wsb = _ws(ws, dev).get(lib.hca_attn_workspace_size(T, H, d, max_entries, window))
+    kc = kv.c()
+    check(lib.hca_attn(_ptr(q), C.byref(kc), _ptr(kv_win), _ptr(win_len), _ptr(q_pos), T, H, d, m,
+                       max_entries, window, float(sm_scale), _ptr(sink), _ptr(out), _ptr(lse), wsp,
+                       wsb, _stream(stream)))
+    return (out, lse) if return_lse else out
+
+
+def launch_count():
+    """Kernels launched by the library since it was loaded."""
+    return int(load().csa_launch_count())
+
+
+def set_timing_events(kernel_id, begin=None, end=None):
+    """Attach torch.cuda.Event objects (enable_timing=True) around every launch
+    of one library kernel; pass None to detach."""
+    b = C.c_void_p(begin.cuda_event) if begin is not None else None
+    e = C.c_void_p(end.cuda_event) if end is not None else None
+    check(load().csa_set_timing_events(kernel_id, b, e))

@@ -1,0 +1,462 @@
+// C-ABI entry points: argument validation, workspace layout, dispatch.
+//
+// Nothing here computes any part of the method; every step runs in the
+// kernels.  Validation happens before anything is enqueued, so an argument
+// error leaves the stream untouched.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "kernels.h"
+
+namespace csa {
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_launches{0};
+struct EventPair {
+  cudaEvent_t begin = nullptr, end = nullptr;
+};
+EventPair g_events[kNumKernelIds];
+
+csa_status_t fail(csa_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+csa_status_t cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return CSA_OK;
+  return fail(CSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kNumSMs = 148;           // B200: workspace layouts are sized for it
+constexpr int kAttnTargetCtas = 2 * kNumSMs;
+constexpr int kD = 128;
+constexpr int kMaxWindow = 1024;
+constexpr size_t kIndexerChunkBytes = size_t(512) << 20;   // score scratch per chunk of queries
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int64_t score_stride(int64_t max_entries) { return (max_entries + 63) / 64 * 64; }
+
+int64_t indexer_chunk(int64_t T, int64_t max_entries) {
+  const int64_t per_query = score_stride(max_entries) * (int64_t)sizeof(float);
+  int64_t c = per_query > 0 ? (int64_t)(kIndexerChunkBytes / per_query) : T;
+  if (c < 1) c = 1;
+  if (c > 65535) c = 65535;
+  return c < T ? c : T;
+}
+
+struct Split {
+  int n, len;
+};
+// Split-KV layout for T queries whose row lists hold at most total_max rows.
+Split attn_split(int64_t T, int64_t total_max, int H) {
+  const int64_t hgroups = (H + 63) / 64;
+  const int64_t ctas = T * hgroups;
+  int64_t max_split = (total_max + 63) / 64;
+  if (max_split < 1) max_split = 1;
+  int64_t n = (kAttnTargetCtas + ctas - 1) / ctas;
+  if (n > max_split) n = max_split;
+  if (n < 1) n = 1;
+  int64_t len = (total_max + n - 1) / n;
+  len = (len + 63) / 64 * 64;
+  if (len < 64) len = 64;
+  n = (total_max + len - 1) / len;
+  if (n < 1) n = 1;
+  return Split{(int)n, (int)len};
+}
+
+size_t attn_ws_bytes(int64_t T, int H, int64_t total_max) {
+  const Split sp = attn_split(T, total_max, H);
+  if (sp.n == 1) return kWsHeader;
+  const size_t acc = (size_t)T * sp.n * H * kD * sizeof(float);
+  const size_t ml = (size_t)T * sp.n * H * 2 * sizeof(float);
+  return kWsHeader + align256(acc) + align256(ml);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+csa_status_t check_cache(const csa_cache_t* c, const char* name) {
+  if (c == nullptr || c->data == nullptr) return fail(CSA_ERR_INVALID_ARG, "%s: null cache", name);
+  if (!aligned16(c->data)) return fail(CSA_ERR_INVALID_ARG, "%s: data not 16-byte aligned", name);
+  if (c->n_rows <= 0) return fail(CSA_ERR_INVALID_ARG, "%s: n_rows must be > 0", name);
+  if (c->page_table != nullptr) {
+    if (c->page_size <= 0 || c->max_pages <= 0)
+      return fail(CSA_ERR_INVALID_ARG, "%s: page_size and max_pages must be > 0", name);
+  } else if (c->seq_stride < 0) {
+    return fail(CSA_ERR_INVALID_ARG, "%s: seq_stride must be >= 0", name);
+  }
+  return CSA_OK;
+}
+
+CacheRef to_ref(const csa_cache_t* c) {
+  CacheRef r;
+  r.data = static_cast<const __nv_bfloat16*>(c->data);
+  r.n_rows = c->n_rows;
+  r.seq_stride = c->seq_stride;
+  r.page_table = c->page_table;
+  r.page_size = c->page_table ? c->page_size : 1;
+  r.max_pages = c->page_table ? c->max_pages : 0;
+  return r;
+}
+
+csa_status_t check_ws(void* ws, size_t ws_bytes, size_t need, const char* name) {
+  if (need == 0) return CSA_OK;
+  if (ws == nullptr || ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", name, need,
+                ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(CSA_ERR_WORKSPACE, "%s: workspace must be 256-byte aligned", name);
+  return CSA_OK;
+}
+
+}  // namespace
+
+void Launch::begin(int32_t kernel) const {
+  const EventPair& e = g_events[kernel];
+  if (e.begin) cudaEventRecord(e.begin, stream);
+}
+
+cudaError_t Launch::end(int32_t kernel) const {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  cudaError_t err = cudaGetLastError();
+  const EventPair& e = g_events[kernel];
+  if (e.end) cudaEventRecord(e.end, stream);
+  return err;
+}
+
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" {
+
+const char* csa_version(void) { return "csa-b200 0.1 (sm_100a)"; }
+
+const char* csa_last_error(void) { return g_last_error.c_str(); }
+
+uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+csa_status_t csa_set_timing_events(int32_t kernel_id, void* ev_begin, void* ev_end) {
+  if (kernel_id < 0 || kernel_id >= kNumKernelIds)
+    return fail(CSA_ERR_INVALID_ARG, "csa_set_timing_events: kernel_id %d out of range", kernel_id);
+  if ((ev_begin == nullptr) != (ev_end == nullptr))
+    return fail(CSA_ERR_INVALID_ARG, "csa_set_timing_events: give both events or neither");
+  g_events[kernel_id].begin = static_cast<cudaEvent_t>(ev_begin);
+  g_events[kernel_id].end = static_cast<cudaEvent_t>(ev_end);
+  return CSA_OK;
+}
+
+// ---- workspace -------------------------------------------------------------
+size_t csa_indexer_topk_workspace_size(int64_t T, int64_t max_entries, int32_t top_k) {
+  (void)top_k;
+  if (T <= 0 || max_entries < 0) return kWsHeader;
+  const int64_t chunk = indexer_chunk(T, max_entries);
+  return kWsHeader + align256((size_t)chunk * score_stride(max_entries) * sizeof(float));
+}
+
+size_t csa_sparse_attn_decode_workspace_size(int32_t B, int32_t H, int32_t d, int32_t top_k,
+                                             int32_t window) {
+  (void)d;
+  if (B <= 0 || H <= 0) return kWsHeader;
+  return attn_ws_bytes(B, H, (int64_t)top_k + window);
+}
+
+size_t csa_sparse_attn_prefill_workspace_size(int64_t L, int32_t H, int32_t d) {
+  (void)L; (void)H; (void)d;
+  return kWsHeader;   // prefill never splits a query's row list
+}
+
+size_t hca_attn_workspace_size(int64_t T, int32_t H, int32_t d, int64_t max_entries,
+                               int32_t window) {
+  (void)d;
+  if (T <= 0 || H <= 0) return kWsHeader;
+  return attn_ws_bytes(T, H, max_entries + window);
+}
+
+csa_status_t csa_workspace_init(void* ws, size_t ws_bytes, csa_stream_t stream) {
+  if (ws == nullptr || ws_bytes < kWsHeader)
+    return fail(CSA_ERR_WORKSPACE, "csa_workspace_init: workspace smaller than its header");
+  return cuda_status(cudaMemsetAsync(ws, 0, kWsHeader, (cudaStream_t)stream), "cudaMemsetAsync");
+}
+
+csa_status_t csa_workspace_check(void* ws, csa_stream_t stream) {
+  if (ws == nullptr) return fail(CSA_ERR_WORKSPACE, "csa_workspace_check: null workspace");
+  WsHeader h;
+  cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "csa_workspace_check");
+  if (h.code == kErrNone) return CSA_OK;
+  static const char* names[] = {"none", "entry index outside the cache",
+                                "page id outside the pool", "eligible entries above max_entries",
+                                "window length outside [0, window]"};
+  const char* what = (h.code > 0 && h.code <= 4) ? names[h.code] : "unknown";
+  fail(CSA_ERR_DEVICE_CHECK, "device check: %s (query %d, value %lld)", what, h.where,
+       (long long)h.value);
+  e = cudaMemsetAsync(ws, 0, kWsHeader, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  return CSA_ERR_DEVICE_CHECK;
+}
+
+// ---- step 1 ------------------------------------------------------------------
+csa_status_t csa_compress_kv(const csa_bf16* C_a, const csa_bf16* Z_a, const csa_bf16* C_b,
+                             const csa_bf16* Z_b, const float* bias, int64_t n_tokens,
+                             int32_t dim, int32_t m, int32_t overlap, csa_bf16* out,
+                             csa_stream_t stream) {
+  if (C_a == nullptr || Z_a == nullptr || out == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "csa_compress_kv: C_a, Z_a and out are required");
+  if (n_tokens < 0 || m < 1 || dim < 8 || dim % 8 != 0 || (overlap != 0 && overlap != 1))
+    return fail(CSA_ERR_INVALID_ARG,
+                "csa_compress_kv: need n_tokens >= 0, m >= 1, dim a positive multiple of 8, "
+                "overlap in {0,1} (got %lld, %d, %d, %d)",
+                (long long)n_tokens, m, dim, overlap);
+  if (!aligned16(C_a) || !aligned16(Z_a) || !aligned16(out) || (C_b && !aligned16(C_b)) ||
+      (Z_b && !aligned16(Z_b)) || (bias && !aligned16(bias)))
+    return fail(CSA_ERR_INVALID_ARG, "csa_compress_kv: tensors must be 16-byte aligned");
+  Launch L{(cudaStream_t)stream};
+  return cuda_status(
+      launch_compress(L, (const __nv_bfloat16*)C_a, (const __nv_bfloat16*)Z_a,
+                      (const __nv_bfloat16*)C_b, (const __nv_bfloat16*)Z_b, bias, n_tokens, dim, m,
+                      overlap, (__nv_bfloat16*)out),
+      "csa_compress_kv launch");
+}
+
+// ---- steps 2-3 ---------------------------------------------------------------
+csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_cache_t* k_idx,
+                              const int32_t* seq_id, const int64_t* q_pos, int64_t T,
+                              int32_t H_I, int32_t c_I, int32_t m, int64_t max_entries,
+                              int32_t top_k, int32_t* idx_out, int32_t* count_out,
+                              float* score_out, void* ws, size_t ws_bytes, csa_stream_t stream) {
+  if (q_idx == nullptr || w == nullptr || idx_out == nullptr || count_out == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "csa_indexer_topk: q_idx, w, idx_out, count_out required");
+  if (T < 0 || H_I < 1 || m < 1 || top_k < 1 || max_entries < 0)
+    return fail(CSA_ERR_INVALID_ARG,
+                "csa_indexer_topk: need T >= 0, H_I >= 1, m >= 1, top_k >= 1, max_entries >= 0");
+  if (H_I > 64) return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: H_I > 64 not built");
+  if (c_I != 64 && c_I != 128)
+    return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: c_I must be 64 or 128 (got %d)", c_I);
+  if (max_entries > (int64_t(1) << 31) - 1)
+    return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: max_entries >= 2^31");
+  csa_status_t st = check_cache(k_idx, "csa_indexer_topk k_idx");
+  if (st != CSA_OK) return st;
+  if (!aligned16(q_idx)) return fail(CSA_ERR_INVALID_ARG, "csa_indexer_topk: q_idx alignment");
+  const size_t need = csa_indexer_topk_workspace_size(T, max_entries, top_k);
+  if ((st = check_ws(ws, ws_bytes, need, "csa_indexer_topk")) != CSA_OK) return st;
+  if (T == 0) return CSA_OK;
+
+  Launch L{(cudaStream_t)stream};
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeader);
+  const int64_t chunk = indexer_chunk(T, max_entries);
+  for (int64_t t0 = 0; t0 < T; t0 += chunk) {
+    const int64_t n = T - t0 < chunk ? T - t0 : chunk;
+    IndexerArgs ia;
+    ia.q_idx = (const __nv_bfloat16*)q_idx;
+    ia.w = w;
+    ia.keys = to_ref(k_idx);
+    ia.seq_id = seq_id;
+    ia.q_pos = q_pos;
+    ia.T = T;
+    ia.H_I = H_I;
+    ia.c_I = c_I;
+    ia.m = m;
+    ia.max_entries = max_entries;
+    ia.t_begin = t0;
+    ia.scores = scores;
+    ia.score_stride = score_stride(max_entries);
+    ia.err = hdr;
+    cudaError_t e = launch_indexer_scores(L, ia, n);
+    if (e != cudaSuccess) return cuda_status(e, "indexer score launch");
+    SelectArgs sa;
+    sa.scores = scores;
+    sa.score_stride = ia.score_stride;
+    sa.q_pos = q_pos;
+    sa.m = m;
+    sa.max_entries = max_entries;
+    sa.t_begin = t0;
+    sa.top_k = top_k;
+    sa.idx_out = idx_out;
+    sa.count_out = count_out;
+    sa.score_out = score_out;
+    e = launch_topk_select(L, sa, n);
+    if (e != cudaSuccess) return cuda_status(e, "top-k select launch");
+  }
+  return CSA_OK;
+}
+
+// ---- step 4 ------------------------------------------------------------------
+namespace {
+
+csa_status_t check_attn_common(const char* name, const csa_bf16* q, const csa_bf16* out,
+                               int32_t H, int32_t d, int32_t window) {
+  if (q == nullptr || out == nullptr) return fail(CSA_ERR_INVALID_ARG, "%s: q and out required", name);
+  if (H < 1 || window < 0) return fail(CSA_ERR_INVALID_ARG, "%s: need H >= 1, window >= 0", name);
+  if (d != kD) return fail(CSA_ERR_UNSUPPORTED, "%s: head dim %d not built (128 only)", name, d);
+  if (H > 128) return fail(CSA_ERR_UNSUPPORTED, "%s: H > 128 not built", name);
+  if (window > kMaxWindow) return fail(CSA_ERR_UNSUPPORTED, "%s: window > %d", name, kMaxWindow);
+  if (!aligned16(q) || !aligned16(out)) return fail(CSA_ERR_INVALID_ARG, "%s: q/out alignment", name);
+  return CSA_OK;
+}
+
+}  // namespace
+
+csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
+                                     int64_t n_entries, const csa_bf16* kv_raw,
+                                     const int32_t* idx, const int32_t* count, int64_t L,
+                                     int32_t H, int32_t d, int32_t top_k, int32_t window,
+                                     float sm_scale, const float* sink, csa_bf16* out,
+                                     float* lse, void* ws, size_t ws_bytes,
+                                     csa_stream_t stream) {
+  const char* name = "csa_sparse_attn_prefill";
+  csa_status_t st = check_attn_common(name, q, out, H, d, window);
+  if (st != CSA_OK) return st;
+  if (kv_raw == nullptr || idx == nullptr || count == nullptr || L < 0 || top_k < 1 ||
+      n_entries < 0 || (n_entries > 0 && kv_comp == nullptr))
+    return fail(CSA_ERR_INVALID_ARG, "%s: kv_raw, idx, count required; L >= 0, top_k >= 1", name);
+  if (L > 0x7fffffff) return fail(CSA_ERR_UNSUPPORTED, "%s: L >= 2^31", name);
+  if (L == 0) return check_ws(ws, ws_bytes, kWsHeader, name);
+  AttnArgs a{};
+  a.q = (const __nv_bfloat16*)q;
+  a.T = L;
+  a.H = H;
+  a.kv.data = (const __nv_bfloat16*)(kv_comp ? kv_comp : kv_raw);
+  a.kv.n_rows = n_entries;
+  a.kv.seq_stride = 0;
+  a.kv.page_table = nullptr;
+  a.kv.page_size = 1;
+  a.kv.max_pages = 0;
+  a.seq_per_query = 0;
+  a.idx = idx;
+  a.top_k = top_k;
+  a.count = count;
+  a.q_pos = nullptr;
+  a.m = 1;
+  a.max_entries = top_k;
+  a.win = (const __nv_bfloat16*)kv_raw;
+  a.win_len = nullptr;
+  a.window = window;
+  a.sm_scale = sm_scale;
+  a.sink = sink;
+  a.out = (__nv_bfloat16*)out;
+  a.lse = lse;
+  // prefill: one slice per query (many queries fill the GPU)
+  a.n_split = 1;
+  a.split_len = (int)(((int64_t)top_k + window + 63) / 64 * 64);
+  st = check_ws(ws, ws_bytes, kWsHeader, name);
+  if (st != CSA_OK) return st;
+  a.err = static_cast<WsHeader*>(ws);
+  a.part_acc = a.part_ml = nullptr;
+  Launch Lc{(cudaStream_t)stream};
+  return cuda_status(launch_attention(Lc, a), name);
+}
+
+csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_comp,
+                                    const csa_bf16* win, const int32_t* win_len,
+                                    const int32_t* idx, const int32_t* count, int32_t B,
+                                    int32_t H, int32_t d, int32_t top_k, int32_t window,
+                                    float sm_scale, const float* sink, csa_bf16* out,
+                                    float* lse, void* ws, size_t ws_bytes,
+                                    csa_stream_t stream) {
+  const char* name = "csa_sparse_attn_decode";
+  csa_status_t st = check_attn_common(name, q, out, H, d, window);
+  if (st != CSA_OK) return st;
+  if ((st = check_cache(kv_comp, name)) != CSA_OK) return st;
+  if (idx == nullptr || count == nullptr || B < 0 || top_k < 1)
+    return fail(CSA_ERR_INVALID_ARG, "%s: idx, count required; B >= 0, top_k >= 1", name);
+  if (window > 0 && (win == nullptr || win_len == nullptr))
+    return fail(CSA_ERR_INVALID_ARG, "%s: window > 0 needs win and win_len", name);
+  if (B == 0) return check_ws(ws, ws_bytes, kWsHeader, name);
+  AttnArgs a{};
+  a.q = (const __nv_bfloat16*)q;
+  a.T = B;
+  a.H = H;
+  a.kv = to_ref(kv_comp);
+  a.seq_per_query = 1;
+  a.idx = idx;
+  a.top_k = top_k;
+  a.count = count;
+  a.q_pos = nullptr;
+  a.m = 1;
+  a.max_entries = top_k;
+  a.win = (const __nv_bfloat16*)win;
+  a.win_len = win_len;
+  a.window = window;
+  a.sm_scale = sm_scale;
+  a.sink = sink;
+  a.out = (__nv_bfloat16*)out;
+  a.lse = lse;
+  const Split sp = attn_split(B, (int64_t)top_k + window, H);
+  const size_t need = sp.n == 1 ? kWsHeader : attn_ws_bytes(B, H, (int64_t)top_k + window);
+  if ((st = check_ws(ws, ws_bytes, need, name)) != CSA_OK) return st;
+  a.n_split = sp.n;
+  a.split_len = sp.len;
+  a.err = static_cast<WsHeader*>(ws);
+  if (sp.n > 1) {
+    char* p = static_cast<char*>(ws) + kWsHeader;
+    a.part_acc = reinterpret_cast<float*>(p);
+    a.part_ml = reinterpret_cast<float*>(p + align256((size_t)B * sp.n * H * kD * sizeof(float)));
+  }
+  Launch L{(cudaStream_t)stream};
+  return cuda_status(launch_attention(L, a), name);
+}
+
+csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_bf16* kv_win,
+                      const int32_t* win_len, const int64_t* q_pos, int64_t T, int32_t H,
+                      int32_t d, int32_t m, int64_t max_entries, int32_t window,
+                      float sm_scale, const float* sink, csa_bf16* out, float* lse, void* ws,
+                      size_t ws_bytes, csa_stream_t stream) {
+  const char* name = "hca_attn";
+  csa_status_t st = check_attn_common(name, q, out, H, d, window);
+  if (st != CSA_OK) return st;
+  if ((st = check_cache(kv_comp, name)) != CSA_OK) return st;
+  if (T < 0 || m < 1 || max_entries < 0)
+    return fail(CSA_ERR_INVALID_ARG, "%s: need T >= 0, m >= 1, max_entries >= 0", name);
+  if (win_len != nullptr && q_pos == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "%s: decode (win_len given) needs q_pos", name);
+  if (window > 0 && kv_win == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "%s: window > 0 needs kv_win", name);
+  if (T > 0x7fffffff) return fail(CSA_ERR_UNSUPPORTED, "%s: T >= 2^31", name);
+  if (T == 0) return check_ws(ws, ws_bytes, kWsHeader, name);
+  AttnArgs a{};
+  a.q = (const __nv_bfloat16*)q;
+  a.T = T;
+  a.H = H;
+  a.kv = to_ref(kv_comp);
+  a.seq_per_query = win_len != nullptr ? 1 : 0;
+  a.idx = nullptr;
+  a.top_k = 0;
+  a.count = nullptr;
+  a.q_pos = q_pos;
+  a.m = m;
+  a.max_entries = max_entries;
+  a.win = (const __nv_bfloat16*)kv_win;
+  a.win_len = win_len;
+  a.window = window;
+  a.sm_scale = sm_scale;
+  a.sink = sink;
+  a.out = (__nv_bfloat16*)out;
+  a.lse = lse;
+  const Split sp = attn_split(T, max_entries + window, H);
+  const size_t need = sp.n == 1 ? kWsHeader : attn_ws_bytes(T, H, max_entries + window);
+  if ((st = check_ws(ws, ws_bytes, need, name)) != CSA_OK) return st;
+  a.n_split = sp.n;
+  a.split_len = sp.len;
+  a.err = static_cast<WsHeader*>(ws);
+  if (sp.n > 1) {
+    char* p = static_cast<char*>(ws) + kWsHeader;
+    a.part_acc = reinterpret_cast<float*>(p);
+    a.part_ml = reinterpret_cast<float*>(p + align256((size_t)T * sp.n * H * kD * sizeof(float)));
+  }
+  Launch L{(cudaStream_t)stream};
+  return cuda_status(launch_attention(L, a), name);
+}
+
+}  // extern "C"

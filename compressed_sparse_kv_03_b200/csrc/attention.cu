@@ -1,0 +1,319 @@
+// Step 4: shared-KV softmax attention over gathered rows.
+//
+// DeepSeek-V4 book, Ch.6 "Shared key-value MQA" (every head reads the same
+// vectors, each both key and value), Ch.7 "The 128-token uncompressed sliding
+// window" (selected entries and window rows share one softmax), "Dense
+// attention over heavily compressed history" (HCA: all s < floor(t/m)) and
+// "Learned attention sinks" (exp(z'_h) joins the denominator).
+//
+// Each query has a virtual row list: its selected (CSA) or eligible (HCA)
+// compressed entries, then its window rows.  A CTA takes one query, one slice
+// of that list (split-KV) and up to 64 heads (16 per warp).  Rows are
+// gathered 64 at a time with cp.async into a double-buffered, XOR-swizzled
+// shared tile; QK^T and PV run on tensor cores (mma.sync m16n8k16, bf16 in,
+// fp32 accumulate) with an online softmax in the log2 domain.  A slice writes
+// either the final output (one slice) or (acc, max, sum) partials that the
+// merge kernel combines.
+#include "kernels.h"
+
+namespace csa {
+
+namespace {
+
+constexpr int D = 128;
+constexpr int BN = 64;   // rows per tile
+
+__device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) {
+  return *reinterpret_cast<const uint32_t*>(p);
+}
+
+template <int NW>
+__global__ void __launch_bounds__(NW * 32) attn_kernel(AttnArgs a) {
+  constexpr int NTH = NW * 32;
+  __shared__ alignas(128) __nv_bfloat16 sKV[2][BN * D];
+  __shared__ const __nv_bfloat16* sRow[2][BN];
+  __shared__ uint32_t sMask[2][2];
+
+  const int64_t i = blockIdx.x;
+  const int split = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, q4 = lane & 3;
+  const int head0 = (blockIdx.z * NW + warp) * 16;
+
+  // ---- this query's virtual row list ----
+  const int64_t pos = a.q_pos ? __ldg(a.q_pos + i) : i;
+  const int32_t seq = a.seq_per_query ? (int32_t)i : 0;
+  int64_t n_sel;
+  if (a.idx) {
+    n_sel = __ldg(a.count + i);
+    n_sel = n_sel < 0 ? 0 : (n_sel > a.top_k ? a.top_k : n_sel);
+  } else {
+    n_sel = pos / a.m;
+    if (n_sel > a.max_entries) {
+      if (split == 0 && tid == 0 && blockIdx.z == 0) report(a.err, kErrEligible, (int32_t)i, n_sel);
+      n_sel = a.max_entries;
+    }
+  }
+  int64_t n_win, win_first = 0;
+  if (a.win_len) {
+    n_win = __ldg(a.win_len + i);
+    if (n_win < 0 || n_win > a.window) {
+      if (split == 0 && tid == 0 && blockIdx.z == 0) report(a.err, kErrWindow, (int32_t)i, n_win);
+      n_win = n_win < 0 ? 0 : a.window;
+    }
+  } else {
+    n_win = pos + 1 < a.window ? pos + 1 : a.window;
+    win_first = pos - n_win + 1;
+  }
+  const int64_t total = n_sel + n_win;
+  const int64_t v0 = (int64_t)split * a.split_len;
+  const int64_t v1 = total < v0 + a.split_len ? total : v0 + a.split_len;
+  const int ntiles = v1 > v0 ? (int)((v1 - v0 + BN - 1) / BN) : 0;
+
+  auto row_ptr = [&](int64_t v) -> const __nv_bfloat16* {
+    if (v >= v1) return nullptr;
+    if (v < n_sel) {
+      const int64_t e = a.idx ? (int64_t)__ldg(a.idx + i * a.top_k + v) : v;
+      const int64_t r = cache_row(a.kv, seq, e, a.err, (int32_t)i);
+      return r < 0 ? nullptr : a.kv.data + r * D;
+    }
+    const int64_t w = v - n_sel;
+    return a.win_len ? a.win + (i * a.window + w) * D : a.win + (win_first + w) * D;
+  };
+  auto fill_rows = [&](int st, int tt) {
+    for (int r0 = warp * 32; r0 < BN; r0 += NTH) {
+      const int r = r0 + lane;
+      const __nv_bfloat16* p = row_ptr(v0 + (int64_t)tt * BN + r);
+      sRow[st][r] = p;
+      const uint32_t bits = __ballot_sync(0xffffffffu, p != nullptr);
+      if (lane == 0) sMask[st][r0 >> 5] = bits;
+    }
+  };
+  auto issue_tile = [&](int st) {
+    const uint32_t base = smem_u32(sKV[st]);
+#pragma unroll
+    for (int c = tid; c < BN * 16; c += NTH) {
+      const int r = c >> 4, ch = c & 15;
+      const __nv_bfloat16* src = sRow[st][r];
+      const uint32_t dst = base + (uint32_t)(r * D + ((ch ^ (r & 7)) << 3)) * 2u;
+      cp_async_16(dst, src ? src + ch * 8 : a.q, src != nullptr);
+    }
+  };
+
+  // ---- query fragments (A operand, rows = heads) ----
+  uint32_t qa[D / 16][4];
+  {
+    const int h_lo = head0 + g, h_hi = head0 + g + 8;
+    const __nv_bfloat16* qlo = a.q + (i * a.H + h_lo) * D;
+    const __nv_bfloat16* qhi = a.q + (i * a.H + h_hi) * D;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int c = kk * 16 + 2 * q4;
+      qa[kk][0] = h_lo < a.H ? ld_u32(qlo + c) : 0u;
+      qa[kk][1] = h_hi < a.H ? ld_u32(qhi + c) : 0u;
+      qa[kk][2] = h_lo < a.H ? ld_u32(qlo + c + 8) : 0u;
+      qa[kk][3] = h_hi < a.H ? ld_u32(qhi + c + 8) : 0u;
+    }
+  }
+  const float scale = a.sm_scale * kLog2e;
+
+  float acc[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
+
+  if (ntiles > 0) {
+    fill_rows(0, 0);
+    __syncthreads();
+    issue_tile(0);
+    cp_async_commit();
+  }
+  for (int tt = 0; tt < ntiles; ++tt) {
+    const int st = tt & 1;
+    if (tt + 1 < ntiles) fill_rows(st ^ 1, tt + 1);
+    __syncthreads();
+    if (tt + 1 < ntiles) issue_tile(st ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+
+    const uint32_t sbase = smem_u32(sKV[st]);
+    // S = Q K^T  (16 heads x 64 rows per warp)
+    float s[BN / 8][4];
+#pragma unroll
+    for (int j = 0; j < BN / 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+      for (int jp = 0; jp < BN / 16; ++jp) {
+        const int mi = lane >> 3, rr = lane & 7;
+        const int row = 16 * jp + 8 * (mi >> 1) + rr;
+        const int ch = 2 * kk + (mi & 1);
+        uint32_t r[4];
+        ldmatrix_x4(r, sbase + (uint32_t)(row * D + ((ch ^ (row & 7)) << 3)) * 2u);
+        mma_bf16_16816(s[2 * jp], qa[kk], r[0], r[1]);
+        mma_bf16_16816(s[2 * jp + 1], qa[kk], r[2], r[3]);
+      }
+    }
+    // online softmax (log2 domain); rows g (lo) and g+8 (hi) of this warp
+    const uint64_t vmask = (uint64_t)sMask[st][0] | ((uint64_t)sMask[st][1] << 32);
+    float mx_lo = -INFINITY, mx_hi = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < BN / 8; ++j) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const bool ok = (vmask >> (8 * j + 2 * q4 + c)) & 1ull;
+        s[j][c] = ok ? s[j][c] * scale : -INFINITY;
+        s[j][2 + c] = ok ? s[j][2 + c] * scale : -INFINITY;
+        mx_lo = fmaxf(mx_lo, s[j][c]);
+        mx_hi = fmaxf(mx_hi, s[j][2 + c]);
+      }
+    }
+    mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
+    mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
+    mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
+    mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
+    const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
+    const float ref_lo = mn_lo == -INFINITY ? 0.f : mn_lo;
+    const float ref_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
+    const float al_lo = exp2f(m_lo - ref_lo), al_hi = exp2f(m_hi - ref_hi);
+    m_lo = mn_lo;
+    m_hi = mn_hi;
+    l_lo *= al_lo;
+    l_hi *= al_hi;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      acc[n][0] *= al_lo;
+      acc[n][1] *= al_lo;
+      acc[n][2] *= al_hi;
+      acc[n][3] *= al_hi;
+    }
+    uint32_t pa[BN / 16][4];
+#pragma unroll
+    for (int j = 0; j < BN / 8; ++j) {
+      const float p0 = exp2f(s[j][0] - ref_lo), p1 = exp2f(s[j][1] - ref_lo);
+      const float p2 = exp2f(s[j][2] - ref_hi), p3 = exp2f(s[j][3] - ref_hi);
+      l_lo += p0 + p1;
+      l_hi += p2 + p3;
+      pa[j >> 1][(j & 1) * 2 + 0] = pack_bf16(p0, p1);
+      pa[j >> 1][(j & 1) * 2 + 1] = pack_bf16(p2, p3);
+    }
+    // O += P V
+#pragma unroll
+    for (int kk2 = 0; kk2 < BN / 16; ++kk2) {
+#pragma unroll
+      for (int np = 0; np < D / 16; ++np) {
+        const int mi = lane >> 3, rr = lane & 7;
+        const int row = 16 * kk2 + 8 * (mi & 1) + rr;
+        const int ch = 2 * np + (mi >> 1);
+        uint32_t r[4];
+        ldmatrix_x4_trans(r, sbase + (uint32_t)(row * D + ((ch ^ (row & 7)) << 3)) * 2u);
+        mma_bf16_16816(acc[2 * np], pa[kk2], r[0], r[1]);
+        mma_bf16_16816(acc[2 * np + 1], pa[kk2], r[2], r[3]);
+      }
+    }
+    __syncthreads();   // stage st and sRow[st] are refilled two tiles later
+  }
+
+  l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
+  l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
+  l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
+  l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+
+  const int h_lo = head0 + g, h_hi = head0 + g + 8;
+  if (a.n_split == 1) {
+    float f_lo = 1.f, f_hi = 1.f, den_lo = l_lo, den_hi = l_hi;
+    float mm_lo = m_lo, mm_hi = m_hi;
+    if (a.sink) {
+      const float z_lo = h_lo < a.H ? __ldg(a.sink + h_lo) * kLog2e : -INFINITY;
+      const float z_hi = h_hi < a.H ? __ldg(a.sink + h_hi) * kLog2e : -INFINITY;
+      const float M_lo = fmaxf(m_lo, z_lo), M_hi = fmaxf(m_hi, z_hi);
+      const float r_lo = M_lo == -INFINITY ? 0.f : M_lo, r_hi = M_hi == -INFINITY ? 0.f : M_hi;
+      f_lo = exp2f(m_lo - r_lo);
+      f_hi = exp2f(m_hi - r_hi);
+      den_lo = l_lo * f_lo + exp2f(z_lo - r_lo);
+      den_hi = l_hi * f_hi + exp2f(z_hi - r_hi);
+      mm_lo = r_lo;
+      mm_hi = r_hi;
+    }
+    const float inv_lo = den_lo > 0.f ? f_lo / den_lo : 0.f;
+    const float inv_hi = den_hi > 0.f ? f_hi / den_hi : 0.f;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      const int c = 8 * n + 2 * q4;
+      if (h_lo < a.H)
+        *reinterpret_cast<uint32_t*>(a.out + (i * a.H + h_lo) * D + c) =
+            pack_bf16(acc[n][0] * inv_lo, acc[n][1] * inv_lo);
+      if (h_hi < a.H)
+        *reinterpret_cast<uint32_t*>(a.out + (i * a.H + h_hi) * D + c) =
+            pack_bf16(acc[n][2] * inv_hi, acc[n][3] * inv_hi);
+    }
+    if (a.lse && q4 == 0) {
+      if (h_lo < a.H) a.lse[i * a.H + h_lo] = den_lo > 0.f ? (mm_lo + log2f(den_lo)) / kLog2e : -INFINITY;
+      if (h_hi < a.H) a.lse[i * a.H + h_hi] = den_hi > 0.f ? (mm_hi + log2f(den_hi)) / kLog2e : -INFINITY;
+    }
+  } else {
+    const int64_t pbase = (i * a.n_split + split) * a.H;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      const int c = 8 * n + 2 * q4;
+      if (h_lo < a.H)
+        *reinterpret_cast<float2*>(a.part_acc + (pbase + h_lo) * D + c) = make_float2(acc[n][0], acc[n][1]);
+      if (h_hi < a.H)
+        *reinterpret_cast<float2*>(a.part_acc + (pbase + h_hi) * D + c) = make_float2(acc[n][2], acc[n][3]);
+    }
+    if (q4 == 0) {
+      if (h_lo < a.H) *reinterpret_cast<float2*>(a.part_ml + (pbase + h_lo) * 2) = make_float2(m_lo, l_lo);
+      if (h_hi < a.H) *reinterpret_cast<float2*>(a.part_ml + (pbase + h_hi) * 2) = make_float2(m_hi, l_hi);
+    }
+  }
+}
+
+// Combine the split partials of one (query, head): 64 threads, 2 dims each.
+__global__ void __launch_bounds__(64) merge_kernel(AttnArgs a) {
+  const int64_t i = blockIdx.x;
+  const int h = blockIdx.y;
+  const int c = 2 * threadIdx.x;
+  const float* ml = a.part_ml + (i * a.n_split * a.H + h) * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < a.n_split; ++s) M = fmaxf(M, ml[(int64_t)s * a.H * 2]);
+  const float z = a.sink ? __ldg(a.sink + h) * kLog2e : -INFINITY;
+  M = fmaxf(M, z);
+  const float ref = M == -INFINITY ? 0.f : M;
+  float den = exp2f(z - ref), o0 = 0.f, o1 = 0.f;
+  for (int s = 0; s < a.n_split; ++s) {
+    const int64_t ps = (i * a.n_split + s) * a.H + h;
+    const float2 mls = *reinterpret_cast<const float2*>(a.part_ml + ps * 2);
+    const float f = exp2f(mls.x - ref);
+    den = fmaf(mls.y, f, den);
+    const float2 v = *reinterpret_cast<const float2*>(a.part_acc + ps * D + c);
+    o0 = fmaf(v.x, f, o0);
+    o1 = fmaf(v.y, f, o1);
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  *reinterpret_cast<uint32_t*>(a.out + (i * a.H + h) * D + c) = pack_bf16(o0 * inv, o1 * inv);
+  if (a.lse && threadIdx.x == 0) a.lse[i * a.H + h] = den > 0.f ? (ref + log2f(den)) / kLog2e : -INFINITY;
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {
+  if (a.T == 0) return cudaSuccess;
+  const int nw = a.H >= 64 ? 4 : (a.H + 15) / 16;
+  const int hgroups = (a.H + nw * 16 - 1) / (nw * 16);
+  const dim3 grid((unsigned)a.T, (unsigned)a.n_split, (unsigned)hgroups);
+  L.begin(kKernelAttention);
+  switch (nw) {
+    case 1: attn_kernel<1><<<grid, 32, 0, L.stream>>>(a); break;
+    case 2: attn_kernel<2><<<grid, 64, 0, L.stream>>>(a); break;
+    case 3: attn_kernel<3><<<grid, 96, 0, L.stream>>>(a); break;
+    default: attn_kernel<4><<<grid, 128, 0, L.stream>>>(a); break;
+  }
+  cudaError_t e = L.end(kKernelAttention);
+  if (e != cudaSuccess || a.n_split == 1) return e;
+  L.begin(kKernelMerge);
+  merge_kernel<<<dim3((unsigned)a.T, (unsigned)a.H), 64, 0, L.stream>>>(a);
+  return L.end(kKernelMerge);
+}
+
+}  // namespace csa

@@ -1,0 +1,92 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace csa {
+
+enum KernelId : int32_t {
+  kKernelIndexerScore = 0,
+  kKernelTopkSelect = 1,
+  kKernelAttention = 2,
+  kKernelMerge = 3,
+  kKernelCompress = 4,
+  kNumKernelIds = 5,
+};
+
+// Per-call launch context: the stream plus the timing / launch-count hooks.
+struct Launch {
+  cudaStream_t stream;
+  void begin(int32_t kernel) const;              // records the kernel's begin event, if attached
+  cudaError_t end(int32_t kernel) const;         // counts the launch, records the end event, checks
+};
+
+cudaError_t launch_compress(const Launch& L, const __nv_bfloat16* Ca, const __nv_bfloat16* Za,
+                            const __nv_bfloat16* Cb, const __nv_bfloat16* Zb, const float* bias,
+                            int64_t n_tokens, int dim, int m, int overlap, __nv_bfloat16* out);
+
+// Lightning-indexer scores of every eligible entry for every query, written to
+// scores[t * score_stride + s] (fp32).
+struct IndexerArgs {
+  const __nv_bfloat16* q_idx;   // [T, H_I, c_I]
+  const float* w;               // [T, H_I]
+  CacheRef keys;
+  const int32_t* seq_id;        // [T] or null
+  const int64_t* q_pos;         // [T] or null
+  int64_t T;
+  int H_I, c_I, m;
+  int64_t max_entries;
+  int64_t t_begin;              // first query of this launch (chunking)
+  float* scores;                // [T_chunk, score_stride]
+  int64_t score_stride;
+  WsHeader* err;
+};
+cudaError_t launch_indexer_scores(const Launch& L, const IndexerArgs& a, int64_t t_count);
+
+struct SelectArgs {
+  const float* scores;          // [T_chunk, score_stride]
+  int64_t score_stride;
+  const int64_t* q_pos;
+  int m;
+  int64_t max_entries;
+  int64_t t_begin;
+  int top_k;
+  int32_t* idx_out;             // [T, top_k]
+  int32_t* count_out;           // [T]
+  float* score_out;             // [T, top_k] or null
+};
+cudaError_t launch_topk_select(const Launch& L, const SelectArgs& a, int64_t t_count);
+
+// Attention over a virtual row list per query: its selected / eligible
+// compressed entries followed by its window rows.
+struct AttnArgs {
+  const __nv_bfloat16* q;       // [T, H, 128]
+  int64_t T;
+  int H;
+  CacheRef kv;                  // compressed entries
+  int seq_per_query;            // 1: query i reads sequence i; 0: all read sequence 0
+  // entry list: explicit (idx != null) or all s < floor(pos/m)
+  const int32_t* idx;
+  int top_k;
+  const int32_t* count;
+  const int64_t* q_pos;         // null: query i at position i
+  int m;
+  int64_t max_entries;
+  // window: buffer [T, window, 128] with win_len (decode) or raw rows (win_len null)
+  const __nv_bfloat16* win;
+  const int32_t* win_len;
+  int window;
+  float sm_scale;
+  const float* sink;            // [H] or null
+  __nv_bfloat16* out;           // [T, H, 128]
+  float* lse;                   // [T, H] or null
+  // split-KV
+  int n_split;
+  int split_len;                // rows of the virtual list per split (multiple of 64)
+  float* part_acc;              // [T, n_split, H, 128]
+  float* part_ml;               // [T, n_split, H, 2]
+  WsHeader* err;
+};
+cudaError_t launch_attention(const Launch& L, const AttnArgs& a);
+
+}  // namespace csa

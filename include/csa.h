@@ -1,0 +1,228 @@
+/*
+ * csa.h -- C ABI of the CSA / HCA hot-path library for NVIDIA B200 (sm_100a).
+ *
+ * The method (DeepSeek-V4 long-context attention, as described by the
+ * "DeepSeek-V4" book, slop-6tp.pages.dev/papers-html-argon/dsv4.html):
+ *   1. block-compress the KV sequence into one entry per m tokens by
+ *      coordinate-wise softmax pooling        (Ch.5 "How CSA Compresses Memory")
+ *   2. score every eligible compressed entry for each query with the lightning
+ *      indexer                                 (Ch.6 "The lightning indexer")
+ *   3. keep the top-k entries per query        (Ch.6 "Top-k selection ...")
+ *   4. softmax attention over the selected entries plus a window of recent raw
+ *      tokens; HCA attends densely to every eligible heavily compressed entry
+ *                                              (Ch.6 "Shared key-value MQA",
+ *                                               Ch.7 "HCA, Local Attention, and Position")
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; every tensor
+ *     is row-major with the innermost dimension contiguous and 16-byte aligned.
+ *     bf16 tensors are passed as raw bit patterns (csa_bf16).
+ *   - Shared-KV layout: one tensor row is both the key and the value of an
+ *     entry (Ch.6 "Shared key-value MQA").
+ *   - The library allocates no memory and never synchronises, except
+ *     csa_workspace_check(), which synchronises its stream.  Work is enqueued
+ *     on the given stream (NULL = the legacy default stream).
+ *   - Positions are 0-based.  Query position t may read compressed entry s iff
+ *     s < floor(t/m) (Ch.5 "Causal availability and the local sliding window").
+ *     A query's window holds its raw tokens max(0, t-W+1) .. t, itself
+ *     included; duplicates of selected entries are kept (Ch.7 "The 128-token
+ *     uncompressed sliding window").
+ *   - Every call returns a csa_status_t.  Argument errors are detected on the
+ *     host before anything is enqueued.  A kernel that meets a bad index or
+ *     page id records CSA_ERR_DEVICE_CHECK in the workspace header (see
+ *     csa_workspace_check), skips that row and carries on; nothing traps.
+ *   - csa_last_error() returns a thread-local description of the last failure.
+ *
+ * Supported sizes: attention head dim d = 128; indexer key dim c_I in {64, 128};
+ * indexer heads H_I <= 64; attention heads H <= 128; m >= 1; window <= 1024.
+ */
+#ifndef CSA_H
+#define CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t csa_bf16;                 /* raw bf16 bit pattern */
+typedef struct CUstream_st* csa_stream_t;  /* a cudaStream_t */
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1,   /* bad pointer, size or combination; nothing enqueued */
+  CSA_ERR_UNSUPPORTED = 2,   /* legal but not built (e.g. d != 128); nothing enqueued */
+  CSA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+  CSA_ERR_DEVICE_CHECK = 4,  /* a kernel recorded a bad index / page id */
+  CSA_ERR_WORKSPACE = 5      /* workspace missing or smaller than required */
+} csa_status_t;
+
+/*
+ * A per-sequence compressed cache (main KV entries or indexer keys).
+ *   data        device, rows of `dim` bf16 (dim given by the call)
+ *   n_rows      number of physical rows `data` holds (bounds for the checks)
+ *   page_table  NULL: contiguous; sequence b's entry s is row b*seq_stride + s.
+ *               else device int32 [n_seq, max_pages]: entry s of sequence b is
+ *               row page_table[b*max_pages + s/page_size]*page_size + s%page_size
+ *               (a paged-attention style block table; the pages note that the
+ *               compressed cache is kept apart from the raw-token state cache,
+ *               "Decode-time cache state", Ch.5).
+ */
+typedef struct {
+  const void* data;
+  int64_t n_rows;
+  int64_t seq_stride;
+  const int32_t* page_table;
+  int32_t page_size;
+  int32_t max_pages;
+} csa_cache_t;
+
+/* ---- library information ------------------------------------------------ */
+const char* csa_version(void);
+const char* csa_last_error(void);
+/* Number of kernels this library has launched since it was loaded. */
+uint64_t csa_launch_count(void);
+
+/*
+ * Timing hook: when `ev_begin`/`ev_end` (cudaEvent_t, created by the caller)
+ * are non-NULL, the library records them on the call's stream immediately
+ * before and after every launch of kernel `kernel_id`.  Pass NULLs to detach.
+ * kernel_id: 0 = indexer scoring, 1 = top-k selection, 2 = attention,
+ * 3 = split merge, 4 = compression.
+ */
+csa_status_t csa_set_timing_events(int32_t kernel_id, void* ev_begin, void* ev_end);
+
+/* ---- workspace ------------------------------------------------------------ */
+/*
+ * Calls that take `ws` need a caller-allocated device workspace of at least
+ * the size returned by the matching *_workspace_size function (256-byte
+ * aligned).  Its first 256 bytes are a header holding the device-check record;
+ * initialise it once with csa_workspace_init (or zero the buffer).  Calls that
+ * run concurrently on different streams need separate workspaces.
+ */
+size_t csa_indexer_topk_workspace_size(int64_t T, int64_t max_entries, int32_t top_k);
+size_t csa_sparse_attn_decode_workspace_size(int32_t B, int32_t H, int32_t d, int32_t top_k,
+                                             int32_t window);
+size_t csa_sparse_attn_prefill_workspace_size(int64_t L, int32_t H, int32_t d);
+size_t hca_attn_workspace_size(int64_t T, int32_t H, int32_t d, int64_t max_entries,
+                               int32_t window);
+
+/* Zero the header of a workspace (enqueued on `stream`). */
+csa_status_t csa_workspace_init(void* ws, size_t ws_bytes, csa_stream_t stream);
+/*
+ * Synchronise `stream`, read the header and return CSA_OK or
+ * CSA_ERR_DEVICE_CHECK (details in csa_last_error()).  Clears the record.
+ */
+csa_status_t csa_workspace_check(void* ws, csa_stream_t stream);
+
+/* ---- step 1: block compression ------------------------------------------- */
+/*
+ * csa_compress_kv -- coordinate-wise softmax pooling of a token sequence into
+ * floor(n_tokens/m) compressed entries.
+ *   overlap = 0 (BLOCK, HCA's compressor, Ch.7 "HCA's 128:1 non-overlapping
+ *     compressor"): entry i, coordinate r =
+ *       sum_{j=mi}^{mi+m-1} softmax_j(Z_a[j,r] + bias[j-mi,r]) * C_a[j,r]
+ *   overlap = 1 (CSA's compressor, Ch.5 "Coordinate-wise softmax pooling"):
+ *     one softmax over 2m positions: block i with (C_a, Z_a + bias[0]) and
+ *     block i-1 with (C_b, Z_b + bias[1]); entry 0 has no previous block, its
+ *     b branch contributes nothing (content 0, logits -inf).
+ *   C_a, Z_a   [n_tokens, dim] bf16
+ *   C_b, Z_b   [n_tokens, dim] bf16, overlap only; NULL -> use C_a / Z_a
+ *   bias       fp32 [m, dim] (BLOCK) or [2, m, dim] (OVERLAP, a then b), or NULL
+ *   out        [floor(n_tokens/m), dim] bf16; tokens past the last full block
+ *              produce nothing (the window covers them)
+ *   dim % 8 == 0.  Accumulation in fp32, output rounded to nearest bf16.
+ */
+csa_status_t csa_compress_kv(const csa_bf16* C_a, const csa_bf16* Z_a, const csa_bf16* C_b,
+                             const csa_bf16* Z_b, const float* bias, int64_t n_tokens,
+                             int32_t dim, int32_t m, int32_t overlap, csa_bf16* out,
+                             csa_stream_t stream);
+
+/* ---- steps 2-3: lightning indexer + top-k ---------------------------------- */
+/*
+ * csa_indexer_topk -- for every query i at position t_i of sequence b_i:
+ *   I[s] = sum_h w[i,h] * ReLU(q_idx[i,h,:] . K[b_i, s, :]),  s < floor(t_i/m)
+ * (Ch.6 "The lightning indexer"), then the top_k entries by I (Ch.6 "Top-k
+ * selection and asymptotic scaling").  Scores are accumulated and compared in
+ * fp32; equal scores go to the lower entry index; with fewer than top_k
+ * eligible entries all are taken.  The score matrix is never returned.
+ *   q_idx      [T, H_I, c_I] bf16
+ *   w          [T, H_I] fp32
+ *   k_idx      cache of [*, c_I] bf16 indexer keys (host struct)
+ *   seq_id     [T] int32 sequence of each query, or NULL (all sequence 0)
+ *   q_pos      [T] int64 position of each query, or NULL (query i at position i)
+ *   max_entries upper bound of floor(t_i/m) over the queries (workspace layout)
+ *   idx_out    [T, top_k] int32: selected entry ids, ascending, padded with -1
+ *   count_out  [T] int32: number selected = min(top_k, floor(t_i/m))
+ *   score_out  [T, top_k] fp32 score of each selected entry (-inf pad), or NULL
+ */
+csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_cache_t* k_idx,
+                              const int32_t* seq_id, const int64_t* q_pos, int64_t T,
+                              int32_t H_I, int32_t c_I, int32_t m, int64_t max_entries,
+                              int32_t top_k, int32_t* idx_out, int32_t* count_out,
+                              float* score_out, void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* ---- step 4: attention ---------------------------------------------------- */
+/*
+ * csa_sparse_attn_prefill -- CSA attention for the L queries of one sequence,
+ * query t at position t:
+ *   o[t,h] = sum_j softmax_j(sm_scale * q[t,h] . kv_j) kv_j
+ * over j in {kv_comp[idx[t,0..count[t]-1]]} followed by the window rows
+ * kv_raw[max(0,t-W+1) .. t], one softmax (Ch.6 "Shared key-value MQA", Ch.7
+ * "The 128-token uncompressed sliding window").  With `sink` (fp32 [H]) each
+ * head's denominator gains exp(sink[h]) (Ch.7 "Learned attention sinks").
+ *   q        [L, H, d] bf16        kv_comp [n_entries, d] bf16
+ *   kv_raw   [L, d] bf16           idx [L, top_k] int32, count [L] int32
+ *   out      [L, H, d] bf16        lse [L, H] fp32 log of the denominator, or NULL
+ */
+csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
+                                     int64_t n_entries, const csa_bf16* kv_raw,
+                                     const int32_t* idx, const int32_t* count, int64_t L,
+                                     int32_t H, int32_t d, int32_t top_k, int32_t window,
+                                     float sm_scale, const float* sink, csa_bf16* out,
+                                     float* lse, void* ws, size_t ws_bytes,
+                                     csa_stream_t stream);
+
+/*
+ * csa_sparse_attn_decode -- one new token per sequence b (query b belongs to
+ * sequence b of kv_comp): attention over the selected entries
+ * kv_comp[b, idx[b, 0..count[b]-1]] followed by the window buffer rows
+ * win[b, 0..win_len[b]-1] (oldest first, the new token last), one softmax.
+ * The selected set is split over several CTAs and merged (split-KV, which the
+ * DeepSeek-V4 infrastructure video transcript, prism.simon-ai.net, describes
+ * as the way decode keeps every SM busy).
+ *   q [B, H, d] bf16; win [B, window, d] bf16; win_len [B] int32 (<= window)
+ *   idx [B, top_k] int32; count [B] int32; out [B, H, d] bf16; lse [B, H] or NULL
+ */
+csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_comp,
+                                    const csa_bf16* win, const int32_t* win_len,
+                                    const int32_t* idx, const int32_t* count, int32_t B,
+                                    int32_t H, int32_t d, int32_t top_k, int32_t window,
+                                    float sm_scale, const float* sink, csa_bf16* out,
+                                    float* lse, void* ws, size_t ws_bytes,
+                                    csa_stream_t stream);
+
+/*
+ * hca_attn -- dense attention over every eligible heavily compressed entry
+ * s < floor(t_i/m) plus the window, one softmax (Ch.7 "Dense attention over
+ * heavily compressed history").
+ *   Decode (win_len != NULL): query i belongs to sequence i, sits at position
+ *     q_pos[i] (required), and its window is kv_win[i, 0..win_len[i]-1]
+ *     ([T, window, d], oldest first, itself last).
+ *   Prefill (win_len == NULL): all queries belong to sequence 0; query i sits
+ *     at position q_pos[i] (or i if q_pos is NULL); kv_win is the raw token
+ *     sequence [*, d] and the window is rows max(0,t-W+1) .. t.
+ *   max_entries bounds floor(t_i/m) (split layout); q [T, H, d]; out [T, H, d];
+ *   lse [T, H] or NULL; sink [H] or NULL.
+ */
+csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_bf16* kv_win,
+                      const int32_t* win_len, const int64_t* q_pos, int64_t T, int32_t H,
+                      int32_t d, int32_t m, int64_t max_entries, int32_t window,
+                      float sm_scale, const float* sink, csa_bf16* out, float* lse, void* ws,
+                      size_t ws_bytes, csa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H */

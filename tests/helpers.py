@@ -1,0 +1,70 @@
+"""Shared test helpers: device transfer, tolerances and comparisons.
+
+Tolerances (stated once, used by every GPU parity test):
+  * attention outputs and compressed entries: max |gpu - oracle| <= 2e-2 and
+    mean |gpu - oracle| <= 5e-3 (bf16 inputs, fp32 accumulation, bf16 output)
+  * top-k sets: identical, except queries whose differing entries all have
+    oracle scores within the near-tie band of the oracle's k-th score:
+    |s - s_k| <= 1e-3 * max(|s|, |s_k|) + eps, where eps = 2^-20 * sum_h |w_h|
+    * sum_r |q_hr| * max_s |K_sr| bounds the fp32 accumulation error of one
+    score; such queries are reported, not failed
+  * counts and index validity: exact
+"""
+import numpy as np
+import torch
+
+ATTN_MAX_ABS = 2e-2
+ATTN_MEAN_ABS = 5e-3
+TIE_REL = 1e-3
+
+
+def f64(t):
+    """bf16/fp32 torch tensor -> float64 numpy (the same values the GPU sees)."""
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def dev(t, device="cuda"):
+    return t.to(device).contiguous() if t is not None else None
+
+
+def assert_close_attn(gpu, ref, what=""):
+    g = f64(gpu) if isinstance(gpu, torch.Tensor) else np.asarray(gpu, dtype=np.float64)
+    err = np.abs(g - ref)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    mx, mean = float(err.max(initial=0.0)), float(err.mean()) if err.size else 0.0
+    assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, \
+        f"{what}: max-abs {mx:.3g} (<= {ATTN_MAX_ABS}), mean-abs {mean:.3g} (<= {ATTN_MEAN_ABS})"
+    return mx, mean
+
+
+def score_eps(qI, w, KI):
+    """fp32 accumulation bound of one indexer score (see module docstring)."""
+    if KI.shape[0] == 0:
+        return 0.0
+    kmax = np.abs(KI).max(axis=0)                     # [c_I]
+    return 2.0 ** -20 * float(np.abs(w) @ (np.abs(qI) @ kmax))
+
+
+def check_topk(gpu_idx_row, gpu_cnt, ora_scores, k, eps):
+    """Compare one query's GPU selection with the oracle's scores.
+    Returns 'exact' or 'near-tie'; raises AssertionError otherwise."""
+    import oracle
+    n = ora_scores.shape[0]
+    want_cnt = min(k, n)
+    assert int(gpu_cnt) == want_cnt, f"count {int(gpu_cnt)} != {want_cnt}"
+    sel = np.asarray(gpu_idx_row[:want_cnt], dtype=np.int64)
+    assert np.all(np.asarray(gpu_idx_row[want_cnt:]) == -1), "padding must be -1"
+    if want_cnt:
+        assert sel.min() >= 0 and sel.max() < n, "selected index outside the eligible range"
+        assert np.all(np.diff(sel) > 0), "indices must be strictly ascending"
+    ref = oracle.topk_select(ora_scores, k)
+    if np.array_equal(sel, ref):
+        return "exact"
+    kth = np.sort(ora_scores.astype(np.float32).astype(np.float64))[::-1][want_cnt - 1]
+    diff = np.setxor1d(sel, ref)
+    s = ora_scores[diff]
+    band = TIE_REL * np.maximum(np.abs(s), abs(kth)) + eps
+    bad = np.abs(s - kth) > band
+    assert not bad.any(), (f"top-k differs beyond the near-tie band: {diff[bad][:8]} "
+                           f"scores {s[bad][:8]} vs k-th {kth}")
+    return "near-tie"

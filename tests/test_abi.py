@@ -1,0 +1,129 @@
+"""CPU-side checks of the C-ABI library: it loads, exports every symbol the
+header declares, and its host-side validation and workspace sizing behave
+(no kernel is launched; nothing here needs a GPU)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "csa.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while", "for", "sizeof")))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from compressed_sparse_kv_03_b200 import _lib
+    if not os.path.exists(_lib.LIB_PATH):
+        from compressed_sparse_kv_03_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_five_calls():
+    fns = header_functions()
+    for name in ("csa_compress_kv", "csa_indexer_topk", "csa_sparse_attn_prefill",
+                 "csa_sparse_attn_decode", "hca_attn"):
+        assert name in fns
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from compressed_sparse_kv_03_b200 import _lib
+    fns = header_functions()
+    assert fns, "no declarations parsed"
+    for name in fns:
+        assert hasattr(lib, name), f"{name} declared in csa.h but not exported"
+    assert set(fns) == set(_lib.SIGNATURES), "binding signatures differ from the header"
+
+
+def test_version_and_last_error(lib):
+    assert b"sm_100a" in lib.csa_version()
+    assert lib.csa_launch_count() == 0
+
+
+def test_compress_rejects_bad_arguments_without_launching(lib):
+    from compressed_sparse_kv_03_b200._lib import STATUS_NAMES
+    buf = (C.c_uint8 * 64)()
+    p = C.cast(buf, C.c_void_p)
+    # m = 0
+    st = lib.csa_compress_kv(p, p, None, None, None, 16, 8, 0, 0, p, None)
+    assert STATUS_NAMES[st] == "CSA_ERR_INVALID_ARG"
+    assert b"m >= 1" in lib.csa_last_error()
+    # dim not a multiple of 8
+    assert lib.csa_compress_kv(p, p, None, None, None, 16, 12, 4, 0, p, None) == 1
+    # missing output
+    assert lib.csa_compress_kv(p, p, None, None, None, 16, 8, 4, 0, None, None) == 1
+    # overlap flag out of range
+    assert lib.csa_compress_kv(p, p, None, None, None, 16, 8, 4, 2, p, None) == 1
+    assert lib.csa_launch_count() == 0
+
+
+def test_attention_rejects_unsupported_dims(lib):
+    from compressed_sparse_kv_03_b200._lib import CacheT
+    buf = (C.c_uint8 * 4096)()
+    p = C.cast(C.addressof(buf) + (-C.addressof(buf)) % 16, C.c_void_p)
+    cache = CacheT(p.value, 16, 16, None, 0, 0)
+    ws = (C.c_uint8 * 1024)()
+    wsp = C.cast(C.addressof(ws) + (-C.addressof(ws)) % 256, C.c_void_p)
+    # head dim 512 is a legal size the library does not build
+    st = lib.csa_sparse_attn_decode(p, C.byref(cache), p, p, p, p, 1, 8, 512, 4, 8, 1.0, None, p,
+                                    None, wsp, 512, None)
+    assert st == 2 and b"head dim" in lib.csa_last_error()
+    # indexer key dim 96
+    st = lib.csa_indexer_topk(p, p, C.byref(cache), None, None, 4, 2, 96, 4, 16, 2, p, p, None,
+                              wsp, 512, None)
+    assert st == 2
+    # null cache data
+    bad = CacheT(None, 16, 16, None, 0, 0)
+    st = lib.hca_attn(p, C.byref(bad), p, None, None, 4, 8, 128, 4, 16, 8, 1.0, None, p, None,
+                      wsp, 512, None)
+    assert st == 1
+    # decode with a window needs the window buffer
+    st = lib.csa_sparse_attn_decode(p, C.byref(cache), None, None, p, p, 1, 8, 128, 4, 8, 1.0,
+                                    None, p, None, wsp, 512, None)
+    assert st == 1
+    assert lib.csa_launch_count() == 0
+
+
+def test_workspace_sizes(lib):
+    hdr = 256
+    # decode split-KV: 64 queries x 2176 rows -> partials are needed
+    n = lib.csa_sparse_attn_decode_workspace_size(64, 64, 128, 2048, 128)
+    assert n > hdr and n % 256 == 0
+    # prefill never splits
+    assert lib.csa_sparse_attn_prefill_workspace_size(65536, 64, 128) == hdr
+    # indexer scratch: at least one fp32 score per eligible entry of a query
+    n = lib.csa_indexer_topk_workspace_size(64, 32768, 2048)
+    assert n >= hdr + 64 * 32768 * 4
+    # too small a workspace is refused before anything runs
+    from compressed_sparse_kv_03_b200._lib import CacheT
+    buf = (C.c_uint8 * 4096)()
+    p = C.cast(C.addressof(buf) + (-C.addressof(buf)) % 256, C.c_void_p)
+    cache = CacheT(p.value, 16, 16, None, 0, 0)
+    st = lib.csa_indexer_topk(p, p, C.byref(cache), None, None, 64, 8, 64, 4, 32768, 2048, p, p,
+                              None, p, 1024, None)
+    assert st == 5 and b"workspace" in lib.csa_last_error()
+
+
+def test_timing_event_hook_validation(lib):
+    assert lib.csa_set_timing_events(99, None, None) == 1
+    assert lib.csa_set_timing_events(0, C.c_void_p(1), None) == 1
+    assert lib.csa_set_timing_events(0, None, None) == 0
+
+
+def test_product_path_does_not_import_the_oracle():
+    """The package and the bench's timed path never touch oracle/."""
+    pkg = os.path.join(ROOT, "compressed_sparse_kv_03_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f

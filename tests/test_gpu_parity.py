@@ -1,0 +1,324 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle on
+the same seeded inputs.  Small cases span several tiles plus ragged tails;
+the five long-context workloads run at full size with sampled outputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import assert_close_attn, check_topk, dev, f64, score_eps
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import compressed_sparse_kv_03_b200 as csa
+    csa.load()
+    yield csa
+    torch.cuda.synchronize()
+
+
+class LazySeq:
+    """Per-sequence float64 views of a device/host tensor, made on demand."""
+
+    def __init__(self, fn):
+        self.fn = fn
+
+    def __getitem__(self, b):
+        return self.fn(b)
+
+
+def _csa():
+    import compressed_sparse_kv_03_b200 as csa
+    return csa
+
+
+# ---------------------------------------------------------------------------
+# step 1: compression
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N,dim,m,bias", [(1000, 128, 4, False), (1003, 64, 4, True),
+                                          (517, 512, 5, True), (4096, 128, 128, True),
+                                          (37, 8, 1, False), (3, 128, 4, False)])
+def test_compress_block(N, dim, m, bias):
+    csa = _csa()
+    g = synth.generator(10 + N + m)
+    Cc, Z = synth.normal(g, (N, dim)), synth.normal(g, (N, dim))
+    B = synth.normal(g, (m, dim), dtype=torch.float32) if bias else None
+    out = csa.compress_kv(dev(Cc), dev(Z), m, bias=dev(B))
+    assert out.shape == (N // m, dim)
+    ref = oracle.pool_block(f64(Cc), f64(Z), m, None if B is None else f64(B))
+    assert_close_attn(out, ref, "compress block")
+
+
+@pytest.mark.parametrize("N,dim,m,bias,separate", [(1000, 128, 4, True, True),
+                                                   (999, 64, 4, False, False),
+                                                   (260, 128, 2, True, True),
+                                                   (300, 256, 16, True, True)])
+def test_compress_overlap(N, dim, m, bias, separate):
+    csa = _csa()
+    g = synth.generator(20 + N)
+    Ca, Za = synth.normal(g, (N, dim)), synth.normal(g, (N, dim))
+    Cb, Zb = (synth.normal(g, (N, dim)), synth.normal(g, (N, dim))) if separate else (None, None)
+    B = synth.normal(g, (2, m, dim), dtype=torch.float32) if bias else None
+    out = csa.compress_kv(dev(Ca), dev(Za), m, C_b=dev(Cb), Z_b=dev(Zb), bias=dev(B), overlap=True)
+    ref = oracle.pool_overlap(f64(Ca), f64(Za), f64(Cb if separate else Ca),
+                              f64(Zb if separate else Za), m,
+                              None if B is None else f64(B[0]), None if B is None else f64(B[1]))
+    assert_close_attn(out, ref, "compress overlap")
+
+
+# ---------------------------------------------------------------------------
+# steps 2-3: indexer + top-k
+# ---------------------------------------------------------------------------
+def _check_queries(idx, cnt, qI, w, key_of_query, elig_of_query, k, queries, scores=None):
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    sc = scores.cpu().numpy() if scores is not None else None
+    stats = {"exact": 0, "near-tie": 0}
+    for t in queries:
+        n = elig_of_query(t)
+        KI = key_of_query(t)[:n]
+        s = oracle.indexer_scores(f64(qI[t]), f64(w[t]), KI)
+        eps = score_eps(f64(qI[t]), f64(w[t]), KI)
+        stats[check_topk(idx[t], cnt[t], s, k, eps)] += 1
+        if sc is not None and cnt[t]:
+            sel = idx[t, :cnt[t]]
+            np.testing.assert_allclose(sc[t, :cnt[t]], s[sel], rtol=1e-5, atol=10 * eps + 1e-6)
+    return stats
+
+
+@pytest.mark.parametrize("H_I,c_I,wdist", [(8, 64, "uniform"), (4, 64, "normal"),
+                                           (16, 128, "uniform"), (1, 64, "uniform"),
+                                           (12, 64, "normal"), (64, 128, "uniform")])
+def test_indexer_topk_decode_ragged(H_I, c_I, wdist):
+    csa = _csa()
+    g = synth.generator(30 + H_I + c_I)
+    m, k = 4, 64
+    pos = torch.tensor([0, 3, 4, 100, 257, 259, 1000, 9001], dtype=torch.int64)
+    B, S = pos.shape[0], int(pos.max()) // m
+    qI = synth.normal(g, (B, H_I, c_I))
+    w = synth.head_weights(g, (B, H_I), wdist)
+    KI = synth.normal(g, (B, S, c_I))
+    seq = torch.arange(B, dtype=torch.int32)
+    idx, cnt, sc = csa.indexer_topk(dev(qI), dev(w), csa.Cache.contiguous(dev(KI)), m, k,
+                                    seq_id=dev(seq), q_pos=dev(pos), max_entries=S,
+                                    return_scores=True)
+    _check_queries(idx, cnt, qI, w, lambda t: f64(KI[t]), lambda t: int(pos[t]) // m, k,
+                   range(B), sc)
+
+
+@pytest.mark.parametrize("T,m,k,H_I", [(700, 4, 32, 4), (1500, 2, 100, 8), (300, 1, 300, 8)])
+def test_indexer_topk_prefill_causal(T, m, k, H_I):
+    csa = _csa()
+    g = synth.generator(40 + T)
+    S = (T - 1) // m
+    qI = synth.normal(g, (T, H_I, 64))
+    w = synth.uniform(g, (T, H_I))
+    KI = synth.normal(g, (S, 64))
+    idx, cnt = csa.indexer_topk(dev(qI), dev(w), csa.Cache(dev(KI)), m, k)
+    KI64 = f64(KI)
+    stats = _check_queries(idx, cnt, qI, w, lambda t: KI64, lambda t: t // m, k, range(T))
+    assert stats["exact"] >= 0.99 * T, stats
+
+
+def test_indexer_topk_exact_ties():
+    """Integer-valued keys and queries make integer scores with many exact
+    ties: the lower index must win, bit-exactly."""
+    csa = _csa()
+    g = synth.generator(50)
+    T, S, H_I, k, m = 64, 3000, 4, 200, 4
+    qI = torch.randint(-1, 2, (T, H_I, 64), generator=g).to(torch.bfloat16)
+    KI = torch.randint(-1, 2, (S, 64), generator=g).to(torch.bfloat16)
+    w = torch.ones((T, H_I), dtype=torch.float32)
+    pos = torch.randint(0, S * m, (T,), generator=g, dtype=torch.int64)
+    idx, cnt = csa.indexer_topk(dev(qI), dev(w), csa.Cache(dev(KI)), m, k, q_pos=dev(pos),
+                                seq_id=dev(torch.zeros(T, dtype=torch.int32)), max_entries=S)
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    for t in range(T):
+        n = int(pos[t]) // m
+        s = oracle.indexer_scores(f64(qI[t]), f64(w[t]), f64(KI[:n]))
+        ref = oracle.topk_select(s, k)
+        assert cnt[t] == ref.shape[0]
+        np.testing.assert_array_equal(idx[t, :cnt[t]], ref)
+
+
+def test_indexer_topk_all_zero_scores():
+    """Every head negative -> every score is exactly 0: the first k win."""
+    csa = _csa()
+    T, S, k = 4, 500, 37
+    qI = torch.ones((T, 2, 64), dtype=torch.bfloat16)
+    KI = -torch.ones((S, 64), dtype=torch.bfloat16)
+    w = torch.rand((T, 2))
+    pos = torch.full((T,), 4 * S, dtype=torch.int64)
+    idx, cnt = csa.indexer_topk(dev(qI), dev(w), csa.Cache(dev(KI)), 4, k, q_pos=dev(pos),
+                                max_entries=S)
+    assert torch.equal(idx.cpu(), torch.arange(k, dtype=torch.int32).expand(T, k))
+    assert torch.all(cnt.cpu() == k)
+
+
+@pytest.mark.parametrize("page_size", [64, 16])
+def test_indexer_topk_paged(page_size):
+    csa = _csa()
+    g = synth.generator(60 + page_size)
+    m, k, H_I = 4, 128, 8
+    pos = torch.tensor([77, 2048, 4097, 30000, 12345], dtype=torch.int64)
+    S = [int(p) // m for p in pos]
+    pool, table = synth.paged_pool(g, S, 64, page_size)
+    B = len(S)
+    qI, w = synth.normal(g, (B, H_I, 64)), synth.uniform(g, (B, H_I))
+    cache = csa.Cache(dev(pool), page_table=dev(table), page_size=page_size)
+    idx, cnt = csa.indexer_topk(dev(qI), dev(w), cache, m, k, seq_id=dev(torch.arange(B, dtype=torch.int32)),
+                                q_pos=dev(pos), max_entries=max(S))
+    _check_queries(idx, cnt, qI, w,
+                   lambda b: f64(synth.unpage(pool, table[b], S[b], page_size)),
+                   lambda b: S[b], k, range(B))
+
+
+# ---------------------------------------------------------------------------
+# step 4: attention
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("L,H,W,k,sink", [(300, 64, 128, 64, False), (257, 8, 16, 40, True),
+                                          (130, 20, 1, 33, False), (200, 128, 64, 100, True)])
+def test_sparse_attn_prefill(L, H, W, k, sink):
+    csa = _csa()
+    g = synth.generator(70 + L + H)
+    m = 4
+    S = max(L // m, 1)
+    q = synth.normal(g, (L, H, 128), 1 / math.sqrt(128))
+    kv_comp, kv_raw = synth.normal(g, (S, 128)), synth.normal(g, (L, 128))
+    idx, cnt = synth.random_topk_lists(g, L, k, [t // m for t in range(L)])
+    z = synth.normal(g, (H,), dtype=torch.float32) if sink else None
+    out, lse = csa.sparse_attn_prefill(dev(q), dev(kv_comp), dev(kv_raw), dev(idx), dev(cnt), W,
+                                       1.0, sink=dev(z), return_lse=True)
+    ref, ref_lse = oracle.csa_prefill_attention(f64(q), f64(kv_comp), f64(kv_raw), idx.numpy(),
+                                                cnt.numpy(), W, 1.0, None if z is None else f64(z))
+    assert_close_attn(out, ref, "sparse prefill")
+    np.testing.assert_allclose(f64(lse), ref_lse, atol=1e-3, rtol=1e-4)
+
+
+@pytest.mark.parametrize("B,H,k,paged,sink", [(5, 64, 2048, False, False), (3, 64, 300, True, True),
+                                              (7, 16, 100, False, True), (2, 128, 513, True, False)])
+def test_sparse_attn_decode(B, H, k, paged, sink):
+    csa = _csa()
+    g = synth.generator(80 + B + k)
+    W = 128
+    S = [5000 + 977 * b for b in range(B)]
+    q = synth.normal(g, (B, H, 128))
+    win = synth.normal(g, (B, W, 128))
+    win_len = torch.tensor([W, 1, 77, W, 5, 128, 0][:B], dtype=torch.int32)
+    cnt_want = [min(k, s) for s in S]
+    cnt_want[0] = 0 if B > 2 else cnt_want[0]          # an empty selection
+    idx = torch.full((B, k), -1, dtype=torch.int32)
+    for b in range(B):
+        c = cnt_want[b]
+        idx[b, :c] = torch.randperm(S[b], generator=g)[:c].sort().values.to(torch.int32)
+    cnt = torch.tensor(cnt_want, dtype=torch.int32)
+    if paged:
+        pool, table = synth.paged_pool(g, S, 128, 64)
+        cache = csa.Cache(dev(pool), page_table=dev(table), page_size=64)
+        logical = lambda b: f64(synth.unpage(pool, table[b], S[b], 64))
+    else:
+        Smax = max(S)
+        kvc = synth.normal(g, (B, Smax, 128))
+        cache = csa.Cache.contiguous(dev(kvc))
+        logical = lambda b: f64(kvc[b])
+    z = synth.normal(g, (H,), dtype=torch.float32) if sink else None
+    lam = 1 / math.sqrt(128)
+    out, lse = csa.sparse_attn_decode(dev(q), cache, dev(win), dev(win_len), dev(idx), dev(cnt), lam,
+                                      sink=dev(z), return_lse=True)
+    out = f64(out)
+    for b in range(B):
+        rows = np.concatenate([logical(b)[idx[b, :cnt[b]].numpy()], f64(win[b, :win_len[b]])])
+        if rows.shape[0] == 0 and z is None:
+            assert np.all(out[b] == 0)
+            continue
+        ref, ref_lse = oracle.attend_shared_kv(f64(q[b]), rows, lam, None if z is None else f64(z))
+        assert_close_attn(out[b], ref, f"decode seq {b}")
+        np.testing.assert_allclose(f64(lse[b]), ref_lse, atol=1e-3, rtol=1e-4)
+
+
+@pytest.mark.parametrize("B,H,m,paged", [(3, 64, 128, False), (4, 24, 4, True), (1, 64, 16, False)])
+def test_hca_decode(B, H, m, paged):
+    csa = _csa()
+    g = synth.generator(90 + B + m)
+    W = 128
+    pos = torch.tensor([70000, 127, 128, 5000][:B], dtype=torch.int64)
+    S = [int(p) // m for p in pos]
+    q = synth.normal(g, (B, H, 128))
+    win = synth.normal(g, (B, W, 128))
+    win_len = torch.clamp(pos + 1, max=W).to(torch.int32)
+    if paged:
+        pool, table = synth.paged_pool(g, [max(s, 1) for s in S], 128, 64)
+        cache = csa.Cache(dev(pool), page_table=dev(table), page_size=64)
+        logical = lambda b: f64(synth.unpage(pool, table[b], S[b], 64))
+    else:
+        kvc = synth.normal(g, (B, max(S), 128))
+        cache = csa.Cache.contiguous(dev(kvc))
+        logical = lambda b: f64(kvc[b])
+    lam = 1 / math.sqrt(128)
+    out = csa.hca_attn(dev(q), cache, dev(win), m, W, lam, win_len=dev(win_len), q_pos=dev(pos),
+                       max_entries=max(S))
+    ref, _ = oracle.hca_decode(f64(q), LazySeq(logical), f64(win), win_len.numpy(), pos.numpy(), m,
+                               lam)
+    assert_close_attn(out, ref, "hca decode")
+
+
+def test_hca_prefill():
+    csa = _csa()
+    g = synth.generator(95)
+    L, H, m, W = 1100, 64, 16, 128
+    q = synth.normal(g, (L, H, 128), 1 / math.sqrt(128))
+    kv_raw, Z = synth.normal(g, (L, 128)), synth.normal(g, (L, 128))
+    kv_comp = csa.compress_kv(dev(kv_raw), dev(Z), m)
+    out = csa.hca_attn(dev(q), csa.Cache(kv_comp), dev(kv_raw), m, W, 1.0)
+    ref, _ = oracle.hca_prefill(f64(q), oracle.bf16_round(oracle.pool_block(f64(kv_raw), f64(Z), m)),
+                                f64(kv_raw), m, W, 1.0)
+    assert_close_attn(out, ref, "hca prefill")
+
+
+def test_attention_device_check_reports_bad_index():
+    """An entry id outside the cache is skipped and reported through the
+    workspace header; the other queries are unaffected."""
+    csa = _csa()
+    g = synth.generator(99)
+    B, H, k, S = 3, 16, 8, 100
+    q, win = synth.normal(g, (B, H, 128)), synth.normal(g, (B, 4, 128))
+    kvc = synth.normal(g, (B, S, 128))
+    idx = torch.arange(k, dtype=torch.int32).repeat(B, 1)
+    idx[1, 3] = S + 5                          # outside sequence 1's rows
+    cnt = torch.full((B,), k, dtype=torch.int32)
+    wl = torch.full((B,), 4, dtype=torch.int32)
+    ws = csa.Workspace()
+    out = csa.sparse_attn_decode(dev(q), csa.Cache(dev(kvc.reshape(-1, 128)), seq_stride=S),
+                                 dev(win), dev(wl), dev(idx), dev(cnt), 0.1, ws=ws)
+    with pytest.raises(csa.CsaError, match="device check"):
+        ws.check()
+    ws.check()                                   # the record was cleared
+    out = f64(out)
+    for b in (0, 2):
+        rows = np.concatenate([f64(kvc[b, :k]), f64(win[b])])
+        ref, _ = oracle.attend_shared_kv(f64(q[b]), rows, 0.1)
+        assert_close_attn(out[b], ref, "unaffected query")
+
+
+def test_decode_is_deterministic():
+    csa = _csa()
+    g = synth.generator(101)
+    cfg = synth.CsaDecode("t", B=4, N=40000, H=64, d=128, H_I=8, c_I=64, m=4, k=512, W=128,
+                          lam=1 / math.sqrt(128))
+    x = {k_: dev(v) for k_, v in synth.csa_decode_inputs(cfg).items()}
+    S = cfg.N // cfg.m
+
+    def run():
+        idx, cnt = csa.indexer_topk(x["qI"], x["w"], csa.Cache.contiguous(x["kI_comp"]), cfg.m, cfg.k,
+                                    seq_id=torch.arange(cfg.B, dtype=torch.int32, device="cuda"),
+                                    q_pos=x["pos"], max_entries=S)
+        return idx, csa.sparse_attn_decode(x["q"], csa.Cache.contiguous(x["kv_comp"]), x["win"],
+                                           x["win_len"], idx, cnt, cfg.lam)
+    i1, o1 = run()
+    i2, o2 = run()
+    assert torch.equal(i1, i2) and torch.equal(o1, o2)

@@ -19,6 +19,7 @@ on the host cores instead (bounded samples of the same workload).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -458,6 +459,10 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
     torch.cuda.set_device(local_rank)
     cls, cfg = RUNNERS[args.workload]
+    if args.batch and hasattr(cfg, "B"):
+        cfg = dataclasses.replace(cfg, B=args.batch, name=f"{cfg.name}_B{args.batch}")
+    if args.seq_len and hasattr(cfg, "L"):
+        cfg = dataclasses.replace(cfg, L=args.seq_len, name=f"{cfg.name}_L{args.seq_len}")
     W = cls(cfg, seed_offset=rank)
     pk = peaks()
     stream = torch.cuda.current_stream()
@@ -476,48 +481,57 @@ def run_ours(args, rank, world, local_rank):
         between()
     torch.cuda.synchronize()
 
-    # capture K steps into one graph, with per-step events around the dominant kernel
+    # one CUDA graph per timed step, each with its own events around the
+    # dominant kernel; L2 flushes (where a workload needs them) run between
+    # the step events, outside the timed time
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    st = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for pair in ev + st:     # torch creates the CUDA events lazily, on first record
+        pair[0].record(stream)
+        pair[1].record(stream)
+    torch.cuda.synchronize()
     use_graph = not args.no_graph
     launches_before = csa.launch_count()
+    graphs = []
     if use_graph:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for i in range(K):
+        for i in range(K):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
                 csa.set_timing_events(W.dominant, ev[i][0], ev[i][1])
                 W.step()
                 csa.set_timing_events(W.dominant)
-                between()
+            graphs.append(g)
         launches = csa.launch_count() - launches_before
-        g.replay()                       # one more untimed warm pass
+        for g in graphs[:2]:         # untimed warm replays
+            g.replay()
+            between()
         torch.cuda.synchronize()
     clocks = Clocks(local_rank)
     clocks.start()
     barrier()
     torch.cuda.synchronize()
-    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_begin.record(stream)
-    if use_graph:
-        g.replay()
-    else:
-        launches_before = csa.launch_count()
-        for i in range(K):
+    launches_before = csa.launch_count()
+    for i in range(K):
+        st[i][0].record(stream)
+        if use_graph:
+            graphs[i].replay()
+        else:
             csa.set_timing_events(W.dominant, ev[i][0], ev[i][1])
             W.step()
             csa.set_timing_events(W.dominant)
-            between()
+        st[i][1].record(stream)
+        between()
+    if not use_graph:
         launches = csa.launch_count() - launches_before
-    t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    ms = t_begin.elapsed_time(t_end)
+    ms = sum(b.elapsed_time(e) for b, e in st)
     dom_ms = [b.elapsed_time(e) for b, e in ev]
-    if use_graph:
-        del g
+    del graphs
     if world > 1:
-        t = torch.tensor([ms, max(dom_ms)], device="cuda")
+        t = torch.tensor([ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t[0])
     ms_per_step = ms / K
@@ -567,7 +581,8 @@ def run_ours(args, rank, world, local_rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded torch CPU generator, N(0,1) / U(0,1))",
             "config": {**W.config(), "parallelism": f"dp{world}" + flush_note,
-                       "timing": "one CUDA graph of K steps" if use_graph else "eager"},
+                       "timing": "one CUDA graph per step, CUDA events per step" if use_graph
+                       else "eager launches, CUDA events per step"},
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": W.h2d,
                     "d2h_bytes_per_step": W.d2h},
@@ -588,6 +603,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(RUNNERS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of a graph")
+    ap.add_argument("--batch", type=int, default=0, help="override the decode batch (profiling runs)")
+    ap.add_argument("--seq-len", type=int, default=0, help="override the prefill length (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work (cpu_baseline)")
     ap.add_argument("--step-budget", type=float, default=4.0, help="seconds per reference-arm step")

@@ -46,12 +46,32 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int64_t score_stride(int64_t max_entries) { return (max_entries + 63) / 64 * 64; }
 
-int64_t indexer_chunk(int64_t T, int64_t max_entries) {
-  const int64_t per_query = score_stride(max_entries) * (int64_t)sizeof(float);
+// Indexer workspace: header | keys [chunk, stride] u32 | hist [chunk, 4096] u32
+// (bitmap mode only) | 256 B pad.  Queries are processed in chunks
+// so that the key scratch stays bounded.
+struct IndexerLayout {
+  bool bitmap;
+  int64_t chunk, stride;
+  size_t keys_off, hist_off, counter_off, total;
+};
+
+IndexerLayout indexer_layout(int64_t T, int64_t max_entries) {
+  IndexerLayout l;
+  l.stride = score_stride(max_entries);
+  l.bitmap = T <= kBitmapSelectMaxQueries || max_entries > kRadixSelectMaxEntries;
+  const int64_t per_query = l.stride * (int64_t)sizeof(uint32_t) +
+                            (l.bitmap ? kHistBins * (int64_t)sizeof(uint32_t) : 0);
   int64_t c = per_query > 0 ? (int64_t)(kIndexerChunkBytes / per_query) : T;
   if (c < 1) c = 1;
   if (c > 65535) c = 65535;
-  return c < T ? c : T;
+  if (l.bitmap && c > kBitmapSelectMaxQueries) c = kBitmapSelectMaxQueries;
+  l.chunk = c < T ? c : T;
+  if (l.chunk < 1) l.chunk = 1;
+  l.keys_off = kWsHeader;
+  l.hist_off = l.keys_off + align256((size_t)l.chunk * l.stride * sizeof(uint32_t));
+  l.counter_off = l.hist_off + (l.bitmap ? align256((size_t)l.chunk * kHistBins * sizeof(uint32_t)) : 0);
+  l.total = l.counter_off + 256;
+  return l;
 }
 
 struct Split {
@@ -120,16 +140,29 @@ csa_status_t check_ws(void* ws, size_t ws_bytes, size_t need, const char* name) 
 
 }  // namespace
 
+namespace {
+// Inside stream capture an event becomes a graph node only when recorded as
+// an external event; outside capture this is a plain record.
+void record_event(cudaEvent_t ev, cudaStream_t stream) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(stream, &cs);
+  if (cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, stream);
+}
+}  // namespace
+
 void Launch::begin(int32_t kernel) const {
   const EventPair& e = g_events[kernel];
-  if (e.begin) cudaEventRecord(e.begin, stream);
+  if (e.begin) record_event(e.begin, stream);
 }
 
 cudaError_t Launch::end(int32_t kernel) const {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   cudaError_t err = cudaGetLastError();
   const EventPair& e = g_events[kernel];
-  if (e.end) cudaEventRecord(e.end, stream);
+  if (e.end) record_event(e.end, stream);
   return err;
 }
 
@@ -159,8 +192,7 @@ csa_status_t csa_set_timing_events(int32_t kernel_id, void* ev_begin, void* ev_e
 size_t csa_indexer_topk_workspace_size(int64_t T, int64_t max_entries, int32_t top_k) {
   (void)top_k;
   if (T <= 0 || max_entries < 0) return kWsHeader;
-  const int64_t chunk = indexer_chunk(T, max_entries);
-  return kWsHeader + align256((size_t)chunk * score_stride(max_entries) * sizeof(float));
+  return indexer_layout(T, max_entries).total;
 }
 
 size_t csa_sparse_attn_decode_workspace_size(int32_t B, int32_t H, int32_t d, int32_t top_k,
@@ -197,8 +229,10 @@ csa_status_t csa_workspace_check(void* ws, csa_stream_t stream) {
   if (h.code == kErrNone) return CSA_OK;
   static const char* names[] = {"none", "entry index outside the cache",
                                 "page id outside the pool", "eligible entries above max_entries",
-                                "window length outside [0, window]"};
-  const char* what = (h.code > 0 && h.code <= 4) ? names[h.code] : "unknown";
+                                "window length outside [0, window]",
+                                "a bounded pipeline wait timed out",
+                                "top-k scratch inconsistent"};
+  const char* what = (h.code > 0 && h.code <= 6) ? names[h.code] : "unknown";
   fail(CSA_ERR_DEVICE_CHECK, "device check: %s (query %d, value %lld)", what, h.where,
        (long long)h.value);
   e = cudaMemsetAsync(ws, 0, kWsHeader, (cudaStream_t)stream);
@@ -211,13 +245,14 @@ csa_status_t csa_compress_kv(const csa_bf16* C_a, const csa_bf16* Z_a, const csa
                              const csa_bf16* Z_b, const float* bias, int64_t n_tokens,
                              int32_t dim, int32_t m, int32_t overlap, csa_bf16* out,
                              csa_stream_t stream) {
-  if (C_a == nullptr || Z_a == nullptr || out == nullptr)
-    return fail(CSA_ERR_INVALID_ARG, "csa_compress_kv: C_a, Z_a and out are required");
   if (n_tokens < 0 || m < 1 || dim < 8 || dim % 8 != 0 || (overlap != 0 && overlap != 1))
     return fail(CSA_ERR_INVALID_ARG,
                 "csa_compress_kv: need n_tokens >= 0, m >= 1, dim a positive multiple of 8, "
                 "overlap in {0,1} (got %lld, %d, %d, %d)",
                 (long long)n_tokens, m, dim, overlap);
+  if (n_tokens / m == 0) return CSA_OK;   // no complete block: nothing to write
+  if (C_a == nullptr || Z_a == nullptr || out == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "csa_compress_kv: C_a, Z_a and out are required");
   if (!aligned16(C_a) || !aligned16(Z_a) || !aligned16(out) || (C_b && !aligned16(C_b)) ||
       (Z_b && !aligned16(Z_b)) || (bias && !aligned16(bias)))
     return fail(CSA_ERR_INVALID_ARG, "csa_compress_kv: tensors must be 16-byte aligned");
@@ -235,16 +270,18 @@ csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_c
                               int32_t H_I, int32_t c_I, int32_t m, int64_t max_entries,
                               int32_t top_k, int32_t* idx_out, int32_t* count_out,
                               float* score_out, void* ws, size_t ws_bytes, csa_stream_t stream) {
-  if (q_idx == nullptr || w == nullptr || idx_out == nullptr || count_out == nullptr)
-    return fail(CSA_ERR_INVALID_ARG, "csa_indexer_topk: q_idx, w, idx_out, count_out required");
   if (T < 0 || H_I < 1 || m < 1 || top_k < 1 || max_entries < 0)
     return fail(CSA_ERR_INVALID_ARG,
                 "csa_indexer_topk: need T >= 0, H_I >= 1, m >= 1, top_k >= 1, max_entries >= 0");
+  if (T == 0) return CSA_OK;
+  if (q_idx == nullptr || w == nullptr || idx_out == nullptr || count_out == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "csa_indexer_topk: q_idx, w, idx_out, count_out required");
   if (H_I > 64) return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: H_I > 64 not built");
   if (c_I != 64 && c_I != 128)
     return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: c_I must be 64 or 128 (got %d)", c_I);
-  if (max_entries > (int64_t(1) << 31) - 1)
-    return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: max_entries >= 2^31");
+  if (max_entries > kBitmapSelectMaxEntries)
+    return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: max_entries > %lld not built",
+                (long long)kBitmapSelectMaxEntries);
   csa_status_t st = check_cache(k_idx, "csa_indexer_topk k_idx");
   if (st != CSA_OK) return st;
   if (!aligned16(q_idx)) return fail(CSA_ERR_INVALID_ARG, "csa_indexer_topk: q_idx alignment");
@@ -253,11 +290,19 @@ csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_c
   if (T == 0) return CSA_OK;
 
   Launch L{(cudaStream_t)stream};
+  const IndexerLayout lay = indexer_layout(T, max_entries);
+  char* wsb = static_cast<char*>(ws);
   WsHeader* hdr = static_cast<WsHeader*>(ws);
-  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeader);
-  const int64_t chunk = indexer_chunk(T, max_entries);
-  for (int64_t t0 = 0; t0 < T; t0 += chunk) {
-    const int64_t n = T - t0 < chunk ? T - t0 : chunk;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(wsb + lay.keys_off);
+  uint32_t* hist = lay.bitmap ? reinterpret_cast<uint32_t*>(wsb + lay.hist_off) : nullptr;
+  for (int64_t t0 = 0; t0 < T; t0 += lay.chunk) {
+    const int64_t n = T - t0 < lay.chunk ? T - t0 : lay.chunk;
+    // zero the histogram of this chunk (decode mode)
+    cudaError_t e = cudaSuccess;
+    if (lay.bitmap) {
+      e = cudaMemsetAsync(wsb + lay.hist_off, 0, (size_t)n * kHistBins * sizeof(uint32_t), L.stream);
+      if (e != cudaSuccess) return cuda_status(e, "indexer histogram memset");
+    }
     IndexerArgs ia;
     ia.q_idx = (const __nv_bfloat16*)q_idx;
     ia.w = w;
@@ -270,14 +315,16 @@ csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_c
     ia.m = m;
     ia.max_entries = max_entries;
     ia.t_begin = t0;
-    ia.scores = scores;
-    ia.score_stride = score_stride(max_entries);
+    ia.keys_out = keys;
+    ia.key_stride = lay.stride;
+    ia.hist = hist;
     ia.err = hdr;
-    cudaError_t e = launch_indexer_scores(L, ia, n);
+    e = launch_indexer_scores(L, ia, n);
     if (e != cudaSuccess) return cuda_status(e, "indexer score launch");
     SelectArgs sa;
-    sa.scores = scores;
-    sa.score_stride = ia.score_stride;
+    sa.keys = keys;
+    sa.key_stride = lay.stride;
+    sa.hist = hist;
     sa.q_pos = q_pos;
     sa.m = m;
     sa.max_entries = max_entries;
@@ -286,6 +333,7 @@ csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_c
     sa.idx_out = idx_out;
     sa.count_out = count_out;
     sa.score_out = score_out;
+    sa.err = hdr;
     e = launch_topk_select(L, sa, n);
     if (e != cudaSuccess) return cuda_status(e, "top-k select launch");
   }
@@ -316,6 +364,7 @@ csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
                                      float* lse, void* ws, size_t ws_bytes,
                                      csa_stream_t stream) {
   const char* name = "csa_sparse_attn_prefill";
+  if (L == 0) return CSA_OK;
   csa_status_t st = check_attn_common(name, q, out, H, d, window);
   if (st != CSA_OK) return st;
   if (kv_raw == nullptr || idx == nullptr || count == nullptr || L < 0 || top_k < 1 ||
@@ -366,6 +415,7 @@ csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_com
                                     float* lse, void* ws, size_t ws_bytes,
                                     csa_stream_t stream) {
   const char* name = "csa_sparse_attn_decode";
+  if (B == 0) return CSA_OK;
   csa_status_t st = check_attn_common(name, q, out, H, d, window);
   if (st != CSA_OK) return st;
   if ((st = check_cache(kv_comp, name)) != CSA_OK) return st;
@@ -414,6 +464,7 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
                       float sm_scale, const float* sink, csa_bf16* out, float* lse, void* ws,
                       size_t ws_bytes, csa_stream_t stream) {
   const char* name = "hca_attn";
+  if (T == 0) return CSA_OK;
   csa_status_t st = check_attn_common(name, q, out, H, d, window);
   if (st != CSA_OK) return st;
   if ((st = check_cache(kv_comp, name)) != CSA_OK) return st;

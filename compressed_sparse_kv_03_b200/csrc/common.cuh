@@ -27,6 +27,8 @@ enum DevErr : int32_t {
   kErrPageId = 2,        // page table entry outside the pool
   kErrEligible = 3,      // eligible entries exceed the workspace layout bound
   kErrWindow = 4,        // window length outside [0, window]
+  kErrTimeout = 5,       // a bounded wait on a pipeline barrier gave up
+  kErrSelect = 6,        // top-k scratch inconsistent (histogram below k)
 };
 
 __device__ __forceinline__ void report(WsHeader* h, int32_t code, int32_t where, int64_t value) {
@@ -56,7 +58,7 @@ __device__ __forceinline__ int64_t cache_row(const CacheRef& c, int32_t seq, int
   int64_t row;
   if (c.page_table == nullptr) {
     row = (int64_t)seq * c.seq_stride + e;
-    if (e < 0 || row < 0 || row >= c.n_rows) {
+    if (e < 0 || (c.seq_stride > 0 && e >= c.seq_stride) || row >= c.n_rows) {
       report(err, kErrEntryIndex, where, e);
       return -1;
     }
@@ -146,5 +148,66 @@ __device__ __forceinline__ float key_score(uint32_t k) {
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk-copy (TMA, non-tensor) helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase of `bar` with the given parity to complete, giving up
+// after about `limit_cycles` SM cycles.  Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          long long limit_cycles = 2000000000ll) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > limit_cycles) return false;
+  return true;
+}
+// Same, backing off with nanosleep between polls: for waiters that are not on
+// the critical path, so that they leave issue slots to the producer threads.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, unsigned ns = 256,
+                                                long long limit_cycles = 2000000000ll) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > limit_cycles) return false;
+    __nanosleep(ns);
+  }
+  return true;
+}
+// global -> shared bulk copy completing on an mbarrier (both addresses 16-byte
+// aligned, size a multiple of 16)
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
 
 }  // namespace csa

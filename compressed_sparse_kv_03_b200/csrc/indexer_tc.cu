@@ -1,0 +1,324 @@
+// Step 2 on tcgen05 tensor cores: lightning-indexer scores streamed from HBM.
+//
+// DeepSeek-V4 book, Ch.6 "The lightning indexer": I[t,s] = sum_h w[t,h] *
+// ReLU(qI[t,h] . K[s]) over the eligible s < floor(t/m).
+//
+// Persistent kernel, one CTA per SM, three roles:
+//   warp 0     TMA producer: items of 256 keys of one query (one 256-row
+//              box, or four 64-row boxes for a paged cache; 128-byte swizzle)
+//              plus the query's head rows, into a
+//              6-stage shared-memory ring (one mbarrier per stage and
+//              direction);
+//   warp 1     allocates TMEM and issues tcgen05.mma: two M = 128 key tiles
+//              per item against the 16 (padded) indexer heads on N, key dim 64
+//              as K in four steps, into one of four 32-column TMEM sets;
+//   warps 2-9  epilogue, two groups of four warps taking alternate items:
+//              tcgen05.ld of their 32 TMEM lanes (one key per tile), ReLU,
+//              the head-weighted sum, the order-preserving score key,
+//              coalesced stores and (decode mode) the query's 12-bit histogram
+//              through warp-aggregated atomics.
+// Each CTA owns a contiguous range of the valid (query, 256-key chunk) pairs,
+// found from a prefix sum over the queries' chunk counts, so ragged lengths
+// stay balanced; every role walks the same range, so no metadata crosses the
+// ring.  Every wait is bounded; a timeout is reported in the workspace header.
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace csa {
+
+namespace {
+
+constexpr int kStages = 6;
+constexpr int kTileRows = 128;                     // MMA M
+constexpr int kItemRows = 2 * kTileRows;           // keys per pipeline item
+constexpr int kBoxRows = 64;                       // TMA box height (page granule)
+constexpr int kKeyTileBytes = kTileRows * 128;     // 64 bf16 per row
+constexpr int kStageKeyBytes = 2 * kKeyTileBytes;
+constexpr int kQTileBytes = 16 * 128;              // 16 head rows (MMA N)
+constexpr int kEpiWarps = 8;                       // two groups of four
+constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr int kAcc = 4;                            // TMEM accumulator sets (32 columns each)
+constexpr uint32_t kIdesc = tc::idesc_bf16(128, 16);
+constexpr int kTmemCols = 128;
+constexpr int kMaxQueries = 2048;
+
+struct TcIndexerParams {
+  IndexerArgs a;
+  int64_t t_count;
+};
+
+// Walks this CTA's contiguous range of (query, 256-key chunk) pairs in
+// increasing order, skipping queries without chunks.
+struct ItemCursor {
+  const int32_t* prefix;   // [t_count + 1] exclusive prefix of chunk counts
+  int t;
+  int32_t v, v_end;
+  __device__ __forceinline__ void init(const int32_t* pre, int t_count, int32_t lo, int32_t hi) {
+    prefix = pre;
+    v = lo;
+    v_end = hi;
+    int l = 0, r = t_count;   // last t with prefix[t] <= lo
+    while (r - l > 1) {
+      const int mid = (l + r) >> 1;
+      if (pre[mid] <= lo) l = mid; else r = mid;
+    }
+    t = l;
+    while (t < t_count && pre[t + 1] <= v) ++t;
+  }
+  __device__ __forceinline__ bool valid() const { return v < v_end; }
+  __device__ __forceinline__ int32_t chunk() const { return v - prefix[t]; }
+  __device__ __forceinline__ void next() {
+    ++v;
+    while (v < v_end && prefix[t + 1] <= v) ++t;
+  }
+};
+
+__device__ __forceinline__ int64_t eligible(const IndexerArgs& a, int64_t t) {
+  const int64_t pos = a.q_pos ? __ldg(a.q_pos + t) : t;
+  const int64_t n = pos / a.m;
+  return n < a.max_entries ? n : a.max_entries;
+}
+
+template <bool HIST>
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
+                        const __grid_constant__ CUtensorMap tmap_q, TcIndexerParams p) {
+  const IndexerArgs& a = p.a;
+  const int T = (int)p.t_count;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t tfull_bar[kAcc], tempty_bar[kAcc];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int32_t prefix[kMaxQueries + 1];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t keys_sm = base;                                // kStages x 32 KB
+  const uint32_t q_sm = base + kStages * kStageKeyBytes;        // kStages x 2 KB
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&full_bar[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), 1);
+    }
+    for (int i = 0; i < kAcc; ++i) {
+      mbar_init(smem_u32(&tfull_bar[i]), 1);
+      mbar_init(smem_u32(&tempty_bar[i]), 4);
+    }
+    mbar_fence_init();
+  }
+  if (warp == 1) tc::tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
+  // chunk counts and their exclusive prefix (warp 0; T <= kMaxQueries)
+  if (warp == 0) {
+    const int per = (T + 31) / 32;
+    const int t0 = lane * per, t1 = min(T, t0 + per);
+    int32_t sum = 0;
+    for (int t = t0; t < t1; ++t) {
+      const int64_t pos = a.q_pos ? __ldg(a.q_pos + a.t_begin + t) : a.t_begin + t;
+      if (pos / a.m > a.max_entries && blockIdx.x == 0)
+        report(a.err, kErrEligible, (int32_t)(a.t_begin + t), pos / a.m);
+      const int64_t n = eligible(a, a.t_begin + t);
+      prefix[t] = (int32_t)((n + kItemRows - 1) / kItemRows);
+      sum += prefix[t];
+    }
+    int32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int32_t run = incl - sum;
+    for (int t = t0; t < t1; ++t) {
+      const int32_t c = prefix[t];
+      prefix[t] = run;
+      run += c;
+    }
+    if (lane == 31) prefix[T] = incl;
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = tmem_base_sh;
+  const int32_t V = prefix[T];
+  const int32_t lo = (int32_t)((int64_t)V * blockIdx.x / gridDim.x);
+  const int32_t hi = (int32_t)((int64_t)V * (blockIdx.x + 1) / gridDim.x);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tmap_keys);
+      tc::prefetch_tmap(&tmap_q);
+      ItemCursor c;
+      c.init(prefix, T, lo, hi);
+      int64_t issued = 0;
+      for (; c.valid(); c.next(), ++issued) {
+        const int64_t t = a.t_begin + c.t;
+        const int64_t s0 = (int64_t)c.chunk() * kItemRows;
+        const int slot = (int)(issued % kStages);
+        if (!mbar_wait(smem_u32(&empty_bar[slot]), (uint32_t)(((issued / kStages) & 1) ^ 1))) {
+          report(a.err, kErrTimeout, (int32_t)t, 10);
+          break;
+        }
+        const uint32_t fb = smem_u32(&full_bar[slot]);
+        mbar_arrive_expect_tx(fb, kStageKeyBytes + kQTileBytes);
+        const int32_t seq = a.seq_id ? __ldg(a.seq_id + t) : 0;
+        if (a.keys.page_table == nullptr) {
+          // contiguous: the item's 256 keys are one 256-row box
+          tc::tma_load_2d(keys_sm + slot * kStageKeyBytes, &tmap_keys, 0,
+                          (int32_t)((int64_t)seq * a.keys.seq_stride + s0), fb);
+        } else {
+#pragma unroll
+        for (int h = 0; h < kItemRows / kBoxRows; ++h) {
+          const int64_t s = s0 + h * kBoxRows;
+          int64_t row;
+          {
+            const int64_t pi = s / a.keys.page_size;
+            const int32_t page = pi < a.keys.max_pages
+                                     ? __ldg(a.keys.page_table + (int64_t)seq * a.keys.max_pages + pi)
+                                     : -1;
+            row = (int64_t)page * a.keys.page_size + (s - pi * a.keys.page_size);
+            if (page < 0 || row >= a.keys.n_rows) {
+              if (s < eligible(a, t)) report(a.err, kErrPageId, (int32_t)t, page);
+              row = 0;
+            }
+          }
+          tc::tma_load_2d(keys_sm + slot * kStageKeyBytes + h * kBoxRows * 128, &tmap_keys, 0,
+                          (int32_t)row, fb);
+        }
+        }
+        tc::tma_load_2d(q_sm + slot * kQTileBytes, &tmap_q, 0, (int32_t)(t * a.H_I), fb);
+      }
+      // every copy must land before the CTA can exit: the last kStages
+      // issued stages hold the latest phase of every slot
+      const int64_t first = issued > kStages ? issued - kStages : 0;
+      for (int64_t d = first; d < issued; ++d)
+        mbar_wait(smem_u32(&full_bar[d % kStages]), (uint32_t)((d / kStages) & 1), 200000000ll);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      for (int64_t j = 0; j < hi - lo; ++j) {
+        const int slot = (int)(j % kStages);
+        const int acc = (int)(j % kAcc);
+        if (!mbar_wait(smem_u32(&full_bar[slot]), (uint32_t)((j / kStages) & 1))) {
+          report(a.err, kErrTimeout, (int32_t)j, 11);
+          break;
+        }
+        if (!mbar_wait(smem_u32(&tempty_bar[acc]), (uint32_t)(((j / kAcc) & 1) ^ 1))) {
+          report(a.err, kErrTimeout, (int32_t)j, 12);
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t qa = q_sm + slot * kQTileBytes;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t ka = keys_sm + slot * kStageKeyBytes + h * kKeyTileBytes;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc::mma_bf16_ss(tmem_base + acc * 32 + h * 16, tc::smem_desc_sw128(ka + 32 * k),
+                            tc::smem_desc_sw128(qa + 32 * k), kIdesc, k > 0);
+        }
+        tc::mma_commit(smem_u32(&empty_bar[slot]));   // smem stage free when the MMAs finish
+        tc::mma_commit(smem_u32(&tfull_bar[acc]));    // accumulators ready
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int group = ew >> 2;                 // handles items j with j % 2 == group
+    const int quarter = warp & 3;              // TMEM lanes this warp may read
+    const int row = quarter * 32 + lane;       // key within a 128-key tile
+    ItemCursor c;
+    c.init(prefix, T, lo, hi);
+    int t_cached = -1;
+    float wv[16];
+    int64_t n_elig = 0;
+    uint32_t* out = nullptr;
+    uint32_t* gh = nullptr;
+    for (int64_t j = 0; c.valid(); c.next(), ++j) {
+      if ((j & 1) != group) continue;
+      const int acc = (int)(j % kAcc);
+      if (c.t != t_cached) {
+        t_cached = c.t;
+        const int64_t t = a.t_begin + c.t;
+#pragma unroll
+        for (int h = 0; h < 16; ++h) wv[h] = h < a.H_I ? __ldg(a.w + t * a.H_I + h) : 0.f;
+        n_elig = eligible(a, t);
+        out = a.keys_out + (int64_t)c.t * a.key_stride;
+        gh = HIST ? a.hist + (int64_t)c.t * kHistBins : nullptr;
+      }
+      if (!mbar_wait(smem_u32(&tfull_bar[acc]), (uint32_t)((j / kAcc) & 1))) {
+        if (lane == 0) report(a.err, kErrTimeout, (int32_t)j, 13);
+        break;
+      }
+      tc::fence_after_sync();
+      uint32_t r0[16], r1[16];
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * 32;
+      tc::tmem_ld16(taddr, r0);
+      tc::tmem_ld16(taddr + 16, r1);
+      tc::tmem_wait_ld();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[acc]));
+      const int64_t s0 = (int64_t)c.chunk() * kItemRows;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t* r = h ? r1 : r0;
+        float sc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) sc = fmaf(wv[k], fmaxf(__uint_as_float(r[k]), 0.f), sc);
+        const int64_t s = s0 + h * kTileRows + row;
+        const bool valid = s < n_elig;
+        const uint32_t key = score_key(sc);
+        if (valid) out[s] = key;
+        if (HIST) {
+          const uint32_t bin = valid ? key >> 20 : 0xffffffffu;
+          const uint32_t same = __match_any_sync(0xffffffffu, bin);
+          if (valid && lane == __ffs(same) - 1) atomicAdd(gh + bin, (uint32_t)__popc(same));
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem_base, kTmemCols);
+}
+
+}  // namespace
+
+bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count) {
+  if (a.c_I != 64 || a.H_I > 16 || t_count > kMaxQueries) return false;
+  if ((a.max_entries + kItemRows - 1) / kItemRows * t_count > INT32_MAX) return false;
+  if (a.keys.page_table != nullptr && a.keys.page_size % kBoxRows != 0) return false;
+  if (a.keys.n_rows > INT32_MAX || a.T * a.H_I > INT32_MAX) return false;
+  return true;
+}
+
+cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int64_t t_count) {
+  CUtensorMap tk, tq;
+  const uint32_t box_rows = a.keys.page_table == nullptr ? kItemRows : kBoxRows;
+  if (!make_tmap_bf16_2d(&tk, a.keys.data, 64, (uint64_t)a.keys.n_rows, 64, 64, box_rows))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tq, a.q_idx, 64, (uint64_t)(a.T * a.H_I), 64, 64, 16))
+    return cudaErrorInvalidValue;
+  TcIndexerParams p;
+  p.a = a;
+  p.t_count = t_count;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = sms;
+  const int smem = kStages * (kStageKeyBytes + kQTileBytes) + 1024;
+  L.begin(kKernelIndexerScore);
+  if (a.hist != nullptr) {
+    cudaFuncSetAttribute(indexer_score_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    indexer_score_tc_kernel<true><<<(unsigned)grid, kThreads, smem, L.stream>>>(tk, tq, p);
+  } else {
+    cudaFuncSetAttribute(indexer_score_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    indexer_score_tc_kernel<false><<<(unsigned)grid, kThreads, smem, L.stream>>>(tk, tq, p);
+  }
+  return L.end(kKernelIndexerScore);
+}
+
+}  // namespace csa

@@ -25,8 +25,18 @@ cudaError_t launch_compress(const Launch& L, const __nv_bfloat16* Ca, const __nv
                             const __nv_bfloat16* Cb, const __nv_bfloat16* Zb, const float* bias,
                             int64_t n_tokens, int dim, int m, int overlap, __nv_bfloat16* out);
 
-// Lightning-indexer scores of every eligible entry for every query, written to
-// scores[t * score_stride + s] (fp32).
+// Indexer scratch limits.  Few-query (decode) mode keeps a 4096-bin histogram
+// of the top 12 score-key bits per query and selects through a bitmap in
+// shared memory; many-query (prefill) mode holds a query's keys in shared
+// memory for a radix select.
+constexpr int kHistBins = 4096;
+constexpr int64_t kBitmapSelectMaxEntries = int64_t(1) << 19;
+constexpr int64_t kBitmapSelectMaxQueries = 2048;
+constexpr int64_t kRadixSelectMaxEntries = 48 * 1024;
+
+// Lightning-indexer scores of every eligible entry for every query of one
+// chunk of queries, written as order-preserving keys to
+// keys_out[(t - t_begin) * key_stride + s].
 struct IndexerArgs {
   const __nv_bfloat16* q_idx;   // [T, H_I, c_I]
   const float* w;               // [T, H_I]
@@ -37,15 +47,20 @@ struct IndexerArgs {
   int H_I, c_I, m;
   int64_t max_entries;
   int64_t t_begin;              // first query of this launch (chunking)
-  float* scores;                // [T_chunk, score_stride]
-  int64_t score_stride;
+  uint32_t* keys_out;           // [T_chunk, key_stride]
+  int64_t key_stride;
+  uint32_t* hist;               // [T_chunk, kHistBins] (zeroed) or null
   WsHeader* err;
 };
 cudaError_t launch_indexer_scores(const Launch& L, const IndexerArgs& a, int64_t t_count);
+// tcgen05 + TMA scoring path (c_I = 64, H_I <= 16, pages a multiple of 64 rows)
+bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count);
+cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int64_t t_count);
 
 struct SelectArgs {
-  const float* scores;          // [T_chunk, score_stride]
-  int64_t score_stride;
+  const uint32_t* keys;         // [T_chunk, key_stride]
+  int64_t key_stride;
+  const uint32_t* hist;         // decode mode: histogram from the scoring launch; else null
   const int64_t* q_pos;
   int m;
   int64_t max_entries;
@@ -54,8 +69,10 @@ struct SelectArgs {
   int32_t* idx_out;             // [T, top_k]
   int32_t* count_out;           // [T]
   float* score_out;             // [T, top_k] or null
+  WsHeader* err;
 };
 cudaError_t launch_topk_select(const Launch& L, const SelectArgs& a, int64_t t_count);
+bool select_uses_bitmap(int64_t t_count, int64_t max_entries);
 
 // Attention over a virtual row list per query: its selected / eligible
 // compressed entries followed by its window rows.

@@ -296,6 +296,31 @@ RUNNERS = {
 
 
 # ---------------------------------------------------------------------------
+# multi-rank aggregation (weak scaling: every rank runs its own batch)
+# ---------------------------------------------------------------------------
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity when the
+    process group is not initialised)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(units_per_rank, world, ms_per_step):
+    """Whole-job units per second: every rank processed units_per_rank in
+    (at most) the slowest rank's step time."""
+    return units_per_rank * world / (ms_per_step / 1e3)
+
+
+def rank_seed_offset(rank):
+    """Each rank draws its own batch."""
+    return int(rank)
+
+
+# ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class Clocks:
@@ -463,7 +488,7 @@ def run_ours(args, rank, world, local_rank):
         cfg = dataclasses.replace(cfg, B=args.batch, name=f"{cfg.name}_B{args.batch}")
     if args.seq_len and hasattr(cfg, "L"):
         cfg = dataclasses.replace(cfg, L=args.seq_len, name=f"{cfg.name}_L{args.seq_len}")
-    W = cls(cfg, seed_offset=rank)
+    W = cls(cfg, seed_offset=rank_seed_offset(rank))
     pk = peaks()
     stream = torch.cuda.current_stream()
 
@@ -530,13 +555,10 @@ def run_ours(args, rank, world, local_rank):
     ms = sum(b.elapsed_time(e) for b, e in st)
     dom_ms = [b.elapsed_time(e) for b, e in ev]
     del graphs
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
+    ms = max_over_ranks([ms], device="cuda")[0]
     ms_per_step = ms / K
     flush_note = ""
-    value = W.units * world / (ms_per_step / 1e3)
+    value = job_throughput(W.units, world, ms_per_step)
 
     # end to end through the public API: host inputs in, result out, every step
     W.e2e_setup()
@@ -551,12 +573,8 @@ def run_ours(args, rank, world, local_rank):
         between()
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t[0])
-    e2e_value = W.units * world / (e_ms / K / 1e3)
+    e_ms = max_over_ranks([e0.elapsed_time(e1)], device="cuda")[0]
+    e2e_value = job_throughput(W.units, world, e_ms / K)
 
     dom_avg = sum(dom_ms) / len(dom_ms)
     if W.bound == "hbm":

@@ -153,6 +153,8 @@ void record_event(cudaEvent_t ev, cudaStream_t stream) {
 }
 }  // namespace
 
+void set_last_error(const char* msg) { g_last_error = msg; }
+
 void Launch::begin(int32_t kernel) const {
   const EventPair& e = g_events[kernel];
   if (e.begin) record_event(e.begin, stream);

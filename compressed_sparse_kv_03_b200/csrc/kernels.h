@@ -106,4 +106,7 @@ struct AttnArgs {
 };
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a);
 
+// Text returned by csa_last_error() for this thread.
+void set_last_error(const char* msg);
+
 }  // namespace csa

@@ -204,6 +204,35 @@ csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_com
                                     csa_stream_t stream);
 
 /*
+ * csa_sparse_attn_decode_noalloc -- csa_sparse_attn_decode for callers that
+ * cannot allocate device memory (no counterpart in the paper: it only changes
+ * where the scratch lives).  Some callers never get to call cudaMalloc: a
+ * plugin inside a serving engine that owns all device memory and hands its
+ * plugins only a stream, or latency-critical code that must not call
+ * cudaMalloc because it can synchronise the device.  This form takes the same
+ * arguments minus the workspace and keeps its split-KV partials in a 16 MiB
+ * array in the library's own device memory (every GPU that loads the library
+ * holds it until exit).  It allocates nothing.
+ *   - Calls needing more than 16 MiB of scratch (see
+ *     csa_sparse_attn_decode_workspace_size) fail with CSA_ERR_WORKSPACE and
+ *     enqueue nothing; e.g. B = 64, H = 64, top_k = 2048, window = 128 needs
+ *     about 10.6 MB.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current; make that first call before any stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents:
+ *     calls that overlap on the GPU (other streams, other host threads) race.
+ *     Each call clears the array's device-check header first; that record is
+ *     not readable by the caller, so bad indices are skipped but not reported
+ *     by this form.
+ */
+csa_status_t csa_sparse_attn_decode_noalloc(const csa_bf16* q, const csa_cache_t* kv_comp,
+                                            const csa_bf16* win, const int32_t* win_len,
+                                            const int32_t* idx, const int32_t* count, int32_t B,
+                                            int32_t H, int32_t d, int32_t top_k, int32_t window,
+                                            float sm_scale, const float* sink, csa_bf16* out,
+                                            float* lse, csa_stream_t stream);
+
+/*
  * hca_attn -- dense attention over every eligible heavily compressed entry
  * s < floor(t_i/m) plus the window, one softmax (Ch.7 "Dense attention over
  * heavily compressed history").

@@ -265,6 +265,14 @@ def launch_count():
     return int(load().csa_launch_count())
 
 
+ATTENTION_KERNELS = {"auto": 0, "tcgen05": 1, "mma_sync": 2}
+
+
+def set_attention_kernel(name):
+    """Choose the attention kernel: "auto" (default), "tcgen05" or "mma_sync"."""
+    check(load().csa_set_attention_kernel(ATTENTION_KERNELS[name]))
+
+
 def set_timing_events(kernel_id, begin=None, end=None):
     """Attach torch.cuda.Event objects (enable_timing=True) around every launch
     of one library kernel; pass None to detach."""

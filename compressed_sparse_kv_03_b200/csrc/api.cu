@@ -16,6 +16,7 @@ namespace {
 
 thread_local std::string g_last_error;
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int32_t> g_attn_kernel{0};
 struct EventPair {
   cudaEvent_t begin = nullptr, end = nullptr;
 };
@@ -81,14 +82,14 @@ struct Split {
 Split attn_split(int64_t T, int64_t total_max, int H) {
   const int64_t hgroups = (H + 63) / 64;
   const int64_t ctas = T * hgroups;
-  int64_t max_split = (total_max + 63) / 64;
+  int64_t max_split = (total_max + 127) / 128;
   if (max_split < 1) max_split = 1;
   int64_t n = (kAttnTargetCtas + ctas - 1) / ctas;
   if (n > max_split) n = max_split;
   if (n < 1) n = 1;
   int64_t len = (total_max + n - 1) / n;
-  len = (len + 63) / 64 * 64;
-  if (len < 64) len = 64;
+  len = (len + 127) / 128 * 128;
+  if (len < 128) len = 128;
   n = (total_max + len - 1) / len;
   if (n < 1) n = 1;
   return Split{(int)n, (int)len};
@@ -155,6 +156,8 @@ void record_event(cudaEvent_t ev, cudaStream_t stream) {
 
 void set_last_error(const char* msg) { g_last_error = msg; }
 
+int32_t attention_kernel_choice() { return g_attn_kernel.load(std::memory_order_relaxed); }
+
 void Launch::begin(int32_t kernel) const {
   const EventPair& e = g_events[kernel];
   if (e.begin) record_event(e.begin, stream);
@@ -179,6 +182,13 @@ const char* csa_version(void) { return "csa-b200 0.1 (sm_100a)"; }
 const char* csa_last_error(void) { return g_last_error.c_str(); }
 
 uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+csa_status_t csa_set_attention_kernel(int32_t choice) {
+  if (choice < 0 || choice > 2)
+    return fail(CSA_ERR_INVALID_ARG, "csa_set_attention_kernel: choice %d out of range", choice);
+  g_attn_kernel.store(choice, std::memory_order_relaxed);
+  return CSA_OK;
+}
 
 csa_status_t csa_set_timing_events(int32_t kernel_id, void* ev_begin, void* ev_end) {
   if (kernel_id < 0 || kernel_id >= kNumKernelIds)
@@ -394,6 +404,7 @@ csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
   a.win = (const __nv_bfloat16*)kv_raw;
   a.win_len = nullptr;
   a.window = window;
+  a.win_rows = L;
   a.sm_scale = sm_scale;
   a.sink = sink;
   a.out = (__nv_bfloat16*)out;
@@ -493,6 +504,7 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
   a.win = (const __nv_bfloat16*)kv_win;
   a.win_len = win_len;
   a.window = window;
+  a.win_rows = (win_len == nullptr && q_pos == nullptr) ? T : 0;
   a.sm_scale = sm_scale;
   a.sink = sink;
   a.out = (__nv_bfloat16*)out;

@@ -270,35 +270,78 @@ __global__ void __launch_bounds__(NW * 32) attn_kernel(AttnArgs a) {
 }
 
 // Combine the split partials of one (query, head): 64 threads, 2 dims each.
-__global__ void __launch_bounds__(64) merge_kernel(AttnArgs a) {
+// One warp per (query, head): lane s holds split s's weight 2^(m_s - M), the
+// warp sums the weighted denominators, then accumulates the 128-dim partial
+// outputs (4 dims per lane) over the splits with independent loads.
+constexpr int kMergeHeads = 4;   // warps per block
+
+__global__ void __launch_bounds__(32 * kMergeHeads) merge_kernel(AttnArgs a) {
   const int64_t i = blockIdx.x;
-  const int h = blockIdx.y;
-  const int c = 2 * threadIdx.x;
-  const float* ml = a.part_ml + (i * a.n_split * a.H + h) * 2;
-  float M = -INFINITY;
-  for (int s = 0; s < a.n_split; ++s) M = fmaxf(M, ml[(int64_t)s * a.H * 2]);
-  const float z = a.sink ? __ldg(a.sink + h) * kLog2e : -INFINITY;
-  M = fmaxf(M, z);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * kMergeHeads + warp;
+  if (h >= a.H) return;
+  const int ns = a.n_split;
+  const float* const ml = a.part_ml + (i * ns * a.H + h) * 2;
+  const float* const acc = a.part_acc + (i * ns * a.H + h) * D + 4 * lane;
+  float M = a.sink ? __ldg(a.sink + h) * kLog2e : -INFINITY;
+  const float z = M;
+  for (int s = lane; s < ns; s += 32) M = fmaxf(M, ml[(int64_t)s * a.H * 2]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   const float ref = M == -INFINITY ? 0.f : M;
-  float den = exp2f(z - ref), o0 = 0.f, o1 = 0.f;
-  for (int s = 0; s < a.n_split; ++s) {
-    const int64_t ps = (i * a.n_split + s) * a.H + h;
-    const float2 mls = *reinterpret_cast<const float2*>(a.part_ml + ps * 2);
-    const float f = exp2f(mls.x - ref);
-    den = fmaf(mls.y, f, den);
-    const float2 v = *reinterpret_cast<const float2*>(a.part_acc + ps * D + c);
-    o0 = fmaf(v.x, f, o0);
-    o1 = fmaf(v.y, f, o1);
+  float den = 0.f;
+  for (int s = lane; s < ns; s += 32) {
+    const float2 mls = *reinterpret_cast<const float2*>(ml + (int64_t)s * a.H * 2);
+    den = fmaf(mls.y, exp2f(mls.x - ref), den);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  den += exp2f(z - ref);
+  float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    const int s_l = s0 + lane;
+    const float f_l = s_l < ns ? exp2f(ml[(int64_t)s_l * a.H * 2] - ref) : 0.f;
+    const int n = ns - s0 < 32 ? ns - s0 : 32;
+#pragma unroll 4
+    for (int j = 0; j < n; ++j) {
+      const float f = __shfl_sync(0xffffffffu, f_l, j);
+      const float4 v = *reinterpret_cast<const float4*>(acc + (int64_t)(s0 + j) * a.H * D);
+      out.x = fmaf(v.x, f, out.x);
+      out.y = fmaf(v.y, f, out.y);
+      out.z = fmaf(v.z, f, out.z);
+      out.w = fmaf(v.w, f, out.w);
+    }
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  *reinterpret_cast<uint32_t*>(a.out + (i * a.H + h) * D + c) = pack_bf16(o0 * inv, o1 * inv);
-  if (a.lse && threadIdx.x == 0) a.lse[i * a.H + h] = den > 0.f ? (ref + log2f(den)) / kLog2e : -INFINITY;
+  uint2 pk;
+  pk.x = pack_bf16(out.x * inv, out.y * inv);
+  pk.y = pack_bf16(out.z * inv, out.w * inv);
+  *reinterpret_cast<uint2*>(a.out + (i * a.H + h) * D + 4 * lane) = pk;
+  if (a.lse && lane == 0) a.lse[i * a.H + h] = den > 0.f ? (ref + log2f(den)) / kLog2e : -INFINITY;
+}
+
+cudaError_t launch_merge(const Launch& L, const AttnArgs& a) {
+  L.begin(kKernelMerge);
+  const dim3 grid((unsigned)a.T, (unsigned)((a.H + kMergeHeads - 1) / kMergeHeads));
+  merge_kernel<<<grid, 32 * kMergeHeads, 0, L.stream>>>(a);
+  return L.end(kKernelMerge);
 }
 
 }  // namespace
 
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {
   if (a.T == 0) return cudaSuccess;
+#ifndef CSA_NO_TC_ATTENTION
+  const int32_t choice = attention_kernel_choice();
+  if (choice != 2 && tc_attention_supported(a) && (choice == 1 || tc_attention_preferred(a))) {
+    L.begin(kKernelAttention);
+    cudaError_t e = launch_attention_tc(L, a);
+    if (e != cudaSuccess) return e;
+    e = L.end(kKernelAttention);
+    if (e != cudaSuccess || a.n_split == 1) return e;
+    return launch_merge(L, a);
+  }
+#endif
   const int nw = a.H >= 64 ? 4 : (a.H + 15) / 16;
   const int hgroups = (a.H + nw * 16 - 1) / (nw * 16);
   const dim3 grid((unsigned)a.T, (unsigned)a.n_split, (unsigned)hgroups);
@@ -311,9 +354,7 @@ cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {
   }
   cudaError_t e = L.end(kKernelAttention);
   if (e != cudaSuccess || a.n_split == 1) return e;
-  L.begin(kKernelMerge);
-  merge_kernel<<<dim3((unsigned)a.T, (unsigned)a.H), 64, 0, L.stream>>>(a);
-  return L.end(kKernelMerge);
+  return launch_merge(L, a);
 }
 
 }  // namespace csa

@@ -1,0 +1,706 @@
+// Step 4 on tcgen05 tensor cores: shared-KV attention over gathered rows.
+//
+// DeepSeek-V4 book, Ch.6 "Shared key-value MQA" (every head reads the same
+// rows, each both key and value) and Ch.7 "The 128-token uncompressed sliding
+// window" (selected entries and window rows share one softmax), "Dense
+// attention over heavily compressed history", "Learned attention sinks".
+//
+// Rows sit on the MMA M dimension and heads on N, so one 128-row tile of the
+// shared KV feeds both products without a transpose:
+//   S^T [128 rows x 64 heads] = KV [128 x 128 dims] . Q^T      (A K-major)
+//   O^T [128 dims x 64 heads] += KV^T [dims x rows] . P^T       (A and B MN-major)
+// The gathered tile is stored once in the 128-byte swizzled layout; read as a
+// K-major operand it is KV, read as an MN-major operand it is KV^T.  P^T is
+// written by the softmax threads (thread = row, 64 heads = one 128-byte row).
+//
+// Warp roles (persistent CTAs over (query, split, head group) work items):
+//   warps 9-10 producers: selected rows gathered with 16-byte cp.async into
+//              their swizzled slots (through the page table when paged),
+//              contiguous rows (HCA, window) with 128-row TMA boxes; the
+//              item's query heads once per item
+//   warp 8     TMEM allocation and tcgen05.mma issue
+//   warps 0-7  online softmax in two warpgroups that split the 64 heads of
+//              every tile (thread = row of S^T): per-head tile maxima with
+//              redux.sync, a lazily rescaled running max (O^T is rescaled in
+//              TMEM only when a head's max grows by more than 2^8), exp2,
+//              per-thread partial row sums, bf16 P^T to shared memory; at the
+//              end of an item the epilogue (thread = dim of O^T) writes the
+//              normalised output or the split partials.
+// Every wait is bounded (the workspace header records a timeout).
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace csa {
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kNP = 64;                         // heads per CTA (MMA N)
+constexpr int kRows = 128;                      // rows per tile (MMA M of S^T)
+#ifndef CSA_ATTN_STAGES
+#define CSA_ATTN_STAGES 4
+#endif
+constexpr int kStages = CSA_ATTN_STAGES;
+constexpr int kKvTile = kRows * kD * 2;         // 32 KB: two 64-dim blocks of 16 KB
+constexpr int kKBlock = kRows * 128;            // 16 KB
+constexpr int kQTile = kNP * kD * 2;            // 16 KB: two 64-dim blocks of 8 KB
+constexpr int kPTile = kRows * kNP * 2;         // 16 KB
+constexpr int kSmWarps = 8;                     // two softmax warpgroups
+constexpr int kHW = kNP / 2;                    // heads per softmax warpgroup
+constexpr int kMmaWarp = kSmWarps, kProducerWarp = kSmWarps + 1;
+constexpr int kProducerWarps = 2;
+constexpr int kProducerThreads = kProducerWarps * 32;
+// kv_full arrivals per tile: one cp.async completion per producer thread plus
+// one release arrive per producer warp (after its row-validity words)
+constexpr uint32_t kKvFullCount = kProducerThreads + kProducerWarps;
+constexpr int kThreads = (kSmWarps + 1 + kProducerWarps) * 32;
+constexpr float kRescale = 8.f;                 // log2 units
+constexpr int kTmemCols = 256;                  // S^T x2 (64 each) + O^T (64)
+constexpr uint32_t kIdescS = tc::idesc_bf16(128, kNP, false, false);
+constexpr uint32_t kIdescPV = tc::idesc_bf16(128, kNP, true, true);
+
+// smem descriptor for the MN-major 128-byte swizzled operands: 8-row atoms
+// (1024 B) along K at SBO = 1024, 64-element blocks along M/N at LBO.
+__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3fffu);
+  d |= (uint64_t)((lbo >> 4) & 0x3fffu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+struct TcAttnParams {
+  AttnArgs a;
+  int hgroups;
+  int64_t items;
+};
+
+// Row list of one (query, split): selected / eligible entries [v0, min(v1, n_sel)),
+// then window rows [max(v0, n_sel), v1) (virtual indices).
+struct ItemInfo {
+  int64_t i;        // query
+  int split, hg;
+  int64_t pos;
+  int32_t seq;
+  int64_t n_sel, n_win, win_first;
+  int64_t v0, v1;
+  int n_sel_tiles, n_tiles;
+};
+
+__device__ __forceinline__ ItemInfo item_info(const AttnArgs& a, int hgroups, int64_t item,
+                                              bool do_report) {
+  ItemInfo it;
+  it.hg = (int)(item % hgroups);
+  const int64_t rest = item / hgroups;
+  it.split = (int)(rest % a.n_split);
+  it.i = rest / a.n_split;
+  it.pos = a.q_pos ? __ldg(a.q_pos + it.i) : it.i;
+  it.seq = a.seq_per_query ? (int32_t)it.i : 0;
+  if (a.idx) {
+    int64_t c = __ldg(a.count + it.i);
+    it.n_sel = c < 0 ? 0 : (c > a.top_k ? a.top_k : c);
+  } else {
+    it.n_sel = it.pos / a.m;
+    if (it.n_sel > a.max_entries) {
+      if (do_report && it.split == 0 && it.hg == 0) report(a.err, kErrEligible, (int32_t)it.i, it.n_sel);
+      it.n_sel = a.max_entries;
+    }
+  }
+  it.win_first = 0;
+  if (a.win_len) {
+    it.n_win = __ldg(a.win_len + it.i);
+    if (it.n_win < 0 || it.n_win > a.window) {
+      if (do_report && it.split == 0 && it.hg == 0) report(a.err, kErrWindow, (int32_t)it.i, it.n_win);
+      it.n_win = it.n_win < 0 ? 0 : a.window;
+    }
+  } else {
+    it.n_win = it.pos + 1 < a.window ? it.pos + 1 : a.window;
+    it.win_first = it.pos - it.n_win + 1;
+  }
+  const int64_t total = it.n_sel + it.n_win;
+  it.v0 = (int64_t)it.split * a.split_len;
+  it.v1 = total < it.v0 + a.split_len ? total : it.v0 + a.split_len;
+  if (it.v1 < it.v0) it.v1 = it.v0;
+  const int64_t s_end = it.v1 < it.n_sel ? it.v1 : it.n_sel;
+  const int64_t w_beg = it.v0 > it.n_sel ? it.v0 : it.n_sel;
+  it.n_sel_tiles = s_end > it.v0 ? (int)((s_end - it.v0 + kRows - 1) / kRows) : 0;
+  const int n_win_tiles = it.v1 > w_beg ? (int)((it.v1 - w_beg + kRows - 1) / kRows) : 0;
+  it.n_tiles = it.n_sel_tiles + n_win_tiles;
+  return it;
+}
+
+// Tile t of an item: first virtual row and number of rows.
+__device__ __forceinline__ void tile_span(const ItemInfo& it, int t, int64_t& v, int& n) {
+  if (t < it.n_sel_tiles) {
+    v = it.v0 + (int64_t)t * kRows;
+    const int64_t e = it.v1 < it.n_sel ? it.v1 : it.n_sel;
+    n = (int)(e - v < kRows ? e - v : kRows);
+  } else {
+    const int64_t w_beg = it.v0 > it.n_sel ? it.v0 : it.n_sel;
+    v = w_beg + (int64_t)(t - it.n_sel_tiles) * kRows;
+    n = (int)(it.v1 - v < kRows ? it.v1 - v : kRows);
+  }
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float redux_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;\n" : "=f"(r) : "f"(v));
+  return r;
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+// Softmax-warp group barrier on an mbarrier (count 4): bounded, so that a
+// warp that gave up elsewhere cannot strand the others.
+__device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase);
+  phase ^= 1u;
+  return ok;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
+               const __grid_constant__ CUtensorMap tm_win,
+               const __grid_constant__ CUtensorMap tm_q, TcAttnParams p) {
+  const AttnArgs& a = p.a;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages];
+  __shared__ __align__(8) uint64_t q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2];
+  __shared__ __align__(8) uint64_t o_full, o_empty, o_step, red_bar[2];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ uint32_t row_ok[kStages][kRows / 32];   // bit b of word w: row 32w + b is valid
+  __shared__ float red_max[2][kSmWarps][kHW];   // per-warp tile maxima, by tile parity
+  __shared__ float red_l[kSmWarps][kHW];        // per-warp row sums at the end of an item
+  __shared__ __align__(16) float w_bcast[kSmWarps][2 * kHW];   // per warp: exponent offsets, factors
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t q_sm = base;                                 // 2 x 16 KB
+  const uint32_t kv_sm = base + 2 * kQTile;                   // kStages x 32 KB
+  const uint32_t p_sm = kv_sm + kStages * kKvTile;            // 2 x 16 KB
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&kv_full[s]), kKvFullCount);
+      mbar_init(smem_u32(&kv_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&q_full[s]), 1);
+      mbar_init(smem_u32(&q_empty[s]), 1);
+      mbar_init(smem_u32(&s_full[s]), 1);
+      mbar_init(smem_u32(&s_empty[s]), kSmWarps);
+      mbar_init(smem_u32(&p_full[s]), kSmWarps);
+      mbar_init(smem_u32(&p_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&o_full), 1);
+    mbar_init(smem_u32(&o_empty), kSmWarps);
+    mbar_init(smem_u32(&o_step), 1);
+    mbar_init(smem_u32(&red_bar[0]), 4);
+    mbar_init(smem_u32(&red_bar[1]), 4);
+    mbar_fence_init();
+  }
+  if (warp == kMmaWarp) tc::tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = tmem_base_sh;
+  const uint32_t tm_s = tmem_base;              // two 64-column S^T buffers
+  const uint32_t tm_o = tmem_base + 2 * kNP;    // O^T
+  const int64_t n_items = p.items;
+
+  if (warp >= kProducerWarp) {
+    // ================================================================ producer
+    // Two warps.  Gathered rows: thread pt copies rows pt and pt + 64 with
+    // 16-byte cp.async into their swizzled slots.  Contiguous rows: thread 0
+    // issues two 128-row TMA boxes.
+    const int pt = threadIdx.x - kProducerWarp * 32;   // 0 .. 63
+    if (pt == 0) {
+      tc::prefetch_tmap(&tm_kv_tile);
+      tc::prefetch_tmap(&tm_win);
+      tc::prefetch_tmap(&tm_q);
+    }
+    int64_t tiles_done = 0, items_done = 0;
+    bool ok = true;
+    for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const ItemInfo it = item_info(a, p.hgroups, item, pt == 0);
+      if (it.n_tiles == 0) continue;
+      if (pt == 0) {   // the query's heads, once per item
+        const int qb = (int)(items_done & 1);
+        if (!mbar_wait(smem_u32(&q_empty[qb]), (uint32_t)(((items_done >> 1) & 1) ^ 1))) {
+          report(a.err, kErrTimeout, (int32_t)it.i, 20);
+          ok = false;
+        } else {
+          mbar_arrive_expect_tx(smem_u32(&q_full[qb]), kQTile);
+          const int32_t qrow = (int32_t)(it.i * a.H + it.hg * kNP);
+          const uint32_t qd = q_sm + qb * kQTile;
+          tc::tma_load_2d(qd, &tm_q, 0, qrow, smem_u32(&q_full[qb]));
+          tc::tma_load_2d(qd + kQTile / 2, &tm_q, 64, qrow, smem_u32(&q_full[qb]));
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);   // keep each warp's control flow uniform
+      if (!ok) break;
+      ++items_done;
+      for (int t = 0; t < it.n_tiles && ok; ++t, ++tiles_done) {
+        const int slot = (int)(tiles_done % kStages);
+        const bool got =
+            mbar_wait(smem_u32(&kv_empty[slot]), (uint32_t)(((tiles_done / kStages) & 1) ^ 1));
+        if (!__all_sync(0xffffffffu, got)) {
+          if (pt == 0) report(a.err, kErrTimeout, (int32_t)it.i, 21);
+          ok = false;
+          break;
+        }
+        int64_t v;
+        int n;
+        tile_span(it, t, v, n);
+        const uint32_t dst = kv_sm + slot * kKvTile;
+        const uint32_t fb = smem_u32(&kv_full[slot]);
+        const bool sel = t < it.n_sel_tiles;
+        if (sel && (a.idx != nullptr || a.kv.page_table != nullptr)) {
+          // both rows' entry indices are loaded before either is used
+          int64_t e[2];
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int r = pt + 64 * half;
+            e[half] = r >= n ? -1 : (a.idx ? (int64_t)__ldg(a.idx + it.i * a.top_k + v + r) : v + r);
+          }
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int r = pt + 64 * half;
+            const int64_t row = r < n ? cache_row(a.kv, it.seq, e[half], a.err, (int32_t)it.i) : -1;
+            const uint32_t okb = __ballot_sync(0xffffffffu, row >= 0);
+            if (lane == 0) row_ok[slot][r >> 5] = okb;
+            const char* src = reinterpret_cast<const char*>(a.kv.data + (row >= 0 ? row : 0) * kD);
+            const uint32_t rdst = dst + (uint32_t)r * 128;
+#pragma unroll
+            for (int ch = 0; ch < 16; ++ch) {
+              const int kb = ch >> 3, c = ch & 7;
+              cp_async_16(rdst + kb * kKBlock + (uint32_t)(((c ^ (r & 7)) & 7) << 4), src + ch * 16,
+                          row >= 0);
+            }
+          }
+          cp_async_mbar_arrive_noinc(fb);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(fb);   // releases this warp's row_ok words
+        } else if (pt == 0) {
+          // contiguous rows: eligible entries of a contiguous cache, or the window
+          int64_t row0;
+          const CUtensorMap* map;
+          if (sel) {
+            row0 = (int64_t)it.seq * a.kv.seq_stride + v;
+            map = &tm_kv_tile;
+            // rows past this sequence's stride or past the cache are masked
+            int64_t lim = a.kv.n_rows - row0;
+            if (a.kv.seq_stride > 0 && a.kv.seq_stride - v < lim) lim = a.kv.seq_stride - v;
+            if (lim < n) {
+              report(a.err, kErrEntryIndex, (int32_t)it.i, v + (lim > 0 ? lim : 0));
+              n = lim > 0 ? (int)lim : 0;
+            }
+          } else {
+            const int64_t w = v - it.n_sel;
+            row0 = a.win_len ? it.i * a.window + w : it.win_first + w;
+            map = &tm_win;
+          }
+#pragma unroll
+          for (int w = 0; w < kRows / 32; ++w) {
+            const int lo = w * 32;
+            row_ok[slot][w] = n >= lo + 32 ? 0xffffffffu : (n > lo ? (1u << (n - lo)) - 1u : 0u);
+          }
+          mbar_expect_tx(fb, kKvTile);
+          tc::tma_load_2d(dst, map, 0, (int32_t)row0, fb);
+          tc::tma_load_2d(dst + kKBlock, map, 64, (int32_t)row0, fb);
+          mbar_arrive_cnt(fb, kKvFullCount);   // releases the row_ok words
+        }
+      }
+    }
+    // no copy of this thread may still be landing when the CTA exits
+    cp_async_commit();
+    cp_async_wait<0>();
+    if (!ok && pt == 0) {
+      const int64_t first = tiles_done > kStages ? tiles_done - kStages : 0;
+      for (int64_t d = first; d < tiles_done; ++d)
+        mbar_wait(smem_u32(&kv_full[d % kStages]), (uint32_t)((d / kStages) & 1), 200000000ll);
+      if (items_done > 0)
+        mbar_wait(smem_u32(&q_full[(items_done - 1) & 1]), (uint32_t)(((items_done - 1) >> 1) & 1),
+                  200000000ll);
+    }
+  } else if (warp == kMmaWarp) {
+    // ================================================================ MMA
+    if (lane == 0) {
+      int64_t tiles_done = 0, items_done = 0, pv_done = 0;
+      bool ok = true;
+      auto do_pv = [&](int64_t gtile, bool first) -> bool {
+        const int pb = (int)(gtile & 1);
+        if (!mbar_wait(smem_u32(&p_full[pb]), (uint32_t)((gtile >> 1) & 1))) return false;
+        // the previous item's epilogue must have read O^T before it is overwritten
+        if (first && !mbar_wait(smem_u32(&o_empty), (uint32_t)((items_done & 1) ^ 1))) return false;
+        tc::fence_after_sync();
+        const uint32_t kv = kv_sm + (int)(gtile % kStages) * kKvTile;
+        const uint32_t pt = p_sm + pb * kPTile;
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          tc::mma_bf16_ss(tm_o, desc_mn(kv + kk * 2048, kKBlock), desc_mn(pt + kk * 2048, kPTile),
+                          kIdescPV, !(first && kk == 0));
+        tc::mma_commit(smem_u32(&kv_empty[gtile % kStages]));
+        tc::mma_commit(smem_u32(&p_empty[pb]));
+        tc::mma_commit(smem_u32(&o_step));
+        ++pv_done;
+        return true;
+      };
+      for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const ItemInfo it = item_info(a, p.hgroups, item, false);
+        if (it.n_tiles == 0) continue;
+        const int qb = (int)(items_done & 1);
+        const uint32_t qs = q_sm + qb * kQTile;
+        if (!mbar_wait(smem_u32(&q_full[qb]), (uint32_t)((items_done >> 1) & 1))) {
+          report(a.err, kErrTimeout, (int32_t)it.i, 22);
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const int64_t first_tile = tiles_done;
+        for (int t = 0; t < it.n_tiles; ++t, ++tiles_done) {
+          const int slot = (int)(tiles_done % kStages);
+          const int sb = (int)(tiles_done & 1);
+          if (!mbar_wait(smem_u32(&kv_full[slot]), (uint32_t)((tiles_done / kStages) & 1)) ||
+              !mbar_wait(smem_u32(&s_empty[sb]), (uint32_t)(((tiles_done >> 1) & 1) ^ 1))) {
+            report(a.err, kErrTimeout, (int32_t)it.i, 23);
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t kv = kv_sm + slot * kKvTile;
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kKBlock + (kk & 3) * 32;
+            const uint32_t qoff = (kk >> 2) * (kQTile / 2) + (kk & 3) * 32;
+            tc::mma_bf16_ss(tm_s + sb * kNP, tc::smem_desc_sw128(kv + off),
+                            tc::smem_desc_sw128(qs + qoff), kIdescS, kk > 0);
+          }
+          tc::mma_commit(smem_u32(&s_full[sb]));
+          if (t == it.n_tiles - 1) tc::mma_commit(smem_u32(&q_empty[qb]));
+          if (t > 0 && !do_pv(tiles_done - 1, tiles_done - 1 == first_tile)) {
+            report(a.err, kErrTimeout, (int32_t)it.i, 24);
+            ok = false;
+            break;
+          }
+        }
+        if (!ok) break;
+        if (!do_pv(tiles_done - 1, tiles_done - 1 == first_tile)) {
+          report(a.err, kErrTimeout, (int32_t)it.i, 25);
+          ok = false;
+          break;
+        }
+        tc::mma_commit(smem_u32(&o_full));
+        ++items_done;
+      }
+    }
+  } else {
+    // ================================================================ softmax + epilogue
+    // Warpgroup wg (warps 4wg .. 4wg+3) owns heads [32 wg, 32 wg + 32) of every
+    // tile: thread = row of S^T in the tile loop, = dim of O^T in the epilogue.
+    // The four warps exchange only their per-head tile maxima; each warp then
+    // derives the same running maxima itself (lane h holds head 32 wg + h).
+    const int wg = warp >> 2, wq = warp & 3;
+    const int hoff = wg * kHW;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+    const uint32_t rbar = smem_u32(&red_bar[wg]);
+    const float scale = a.sm_scale * kLog2e;
+    float* const my_bc = w_bcast[warp];   // this warp's per-head broadcast row
+    uint32_t red_phase = 0;
+    int64_t tiles_done = 0, items_done = 0, pv_seen = 0;
+    for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const ItemInfo it = item_info(a, p.hgroups, item, false);
+      const int h_base = it.hg * kNP;
+      const int nh = a.H - h_base < kNP ? a.H - h_base : kNP;
+      if (it.n_tiles == 0) {
+        // no rows: an empty partial for the merge, or a zero output
+        for (int hl = 0; hl < kHW; ++hl) {
+          const int h = hoff + hl;
+          if (h >= nh) break;
+          const int hh = h_base + h;
+          if (a.n_split == 1) {
+            a.out[(it.i * a.H + hh) * kD + row] = __float2bfloat16_rn(0.f);
+            if (a.lse && row == 0) a.lse[it.i * a.H + hh] = a.sink ? __ldg(a.sink + hh) : -INFINITY;
+          } else {
+            const int64_t pb = (it.i * a.n_split + it.split) * a.H + hh;
+            a.part_acc[pb * kD + row] = 0.f;
+            if (row == 0) *reinterpret_cast<float2*>(a.part_ml + pb * 2) = make_float2(-INFINITY, 0.f);
+          }
+        }
+        continue;
+      }
+      float m_run = -INFINITY;   // lane h: running max of head hoff + h, log2 units
+      float lpart[kHW];
+#pragma unroll
+      for (int h = 0; h < kHW; ++h) lpart[h] = 0.f;
+      bool ok = true;
+      for (int t = 0; t < it.n_tiles && ok; ++t, ++tiles_done) {
+        const int slot = (int)(tiles_done % kStages);
+        const int sb = (int)(tiles_done & 1);
+        ok = mbar_wait(smem_u32(&s_full[sb]), (uint32_t)((tiles_done >> 1) & 1)) &&
+             mbar_wait(smem_u32(&kv_full[slot]), (uint32_t)((tiles_done / kStages) & 1));
+        if (!ok) break;
+        tc::fence_after_sync();
+        float x[kHW];
+        {
+          uint32_t r0[16], r1[16];
+          tc::tmem_ld16(tm_s + sb * kNP + hoff + lane_base, r0);
+          tc::tmem_ld16(tm_s + sb * kNP + hoff + 16 + lane_base, r1);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            x[j] = __uint_as_float(r0[j]);
+            x[16 + j] = __uint_as_float(r1[j]);
+          }
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&s_empty[sb]));
+        const bool valid = (row_ok[slot][row >> 5] >> (row & 31)) & 1u;
+        // per-head tile maxima of the raw logits across this warp's 32 rows
+        float mine = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < kHW; ++h) {
+          if (!valid) x[h] = -INFINITY;
+          const float mx = redux_max(x[h]);
+          if (lane == h) mine = mx;
+        }
+        float (*const rm)[kHW] = red_max[sb];
+        rm[warp][lane] = mine;
+        if (!(ok = group_sync(rbar, red_phase, lane))) break;
+        float tmax = fmaxf(fmaxf(rm[4 * wg][lane], rm[4 * wg + 1][lane]),
+                           fmaxf(rm[4 * wg + 2][lane], rm[4 * wg + 3][lane]));
+        tmax *= scale;   // scale > 0: the max commutes with it
+        float f = 1.f;
+        bool grew = false;
+        if (tmax > m_run + kRescale || (m_run == -INFINITY && tmax > -INFINITY)) {
+          f = m_run == -INFINITY ? 0.f : exp2f(m_run - tmax);
+          grew = m_run != -INFINITY;
+          m_run = tmax;
+        }
+        const bool rescale = __any_sync(0xffffffffu, grew);
+        my_bc[lane] = m_run == -INFINITY ? 0.f : m_run;
+        if (rescale) my_bc[kHW + lane] = f;
+        __syncwarp();
+        if (rescale) {
+          // this warp's 32 dims of O^T for the group's heads, when a running max moved
+          if (pv_seen < tiles_done) {   // every earlier PV must have completed
+            if (!(ok = mbar_wait(smem_u32(&o_step), (uint32_t)((tiles_done - 1) & 1)))) break;
+            pv_seen = tiles_done;
+          }
+          tc::fence_after_sync();
+#pragma unroll
+          for (int c = 0; c < kHW / 16; ++c) {
+            uint32_t r[16];
+            tc::tmem_ld16(tm_o + hoff + c * 16 + lane_base, r);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              r[j] = __float_as_uint(__uint_as_float(r[j]) * my_bc[kHW + c * 16 + j]);
+            tmem_st16(tm_o + hoff + c * 16 + lane_base, r);
+          }
+          tmem_wait_st();
+          tc::fence_before_sync();
+        }
+        // probabilities, partial sums, bf16 P^T (this group's 64 bytes of the row)
+        if (!(ok = mbar_wait(smem_u32(&p_empty[sb]), (uint32_t)(((tiles_done >> 1) & 1) ^ 1)))) break;
+        const uint32_t prow = p_sm + sb * kPTile + (uint32_t)row * 128;
+#pragma unroll
+        for (int c = 0; c < kHW / 8; ++c) {
+          const float4 me0 = *reinterpret_cast<const float4*>(my_bc + c * 8);
+          const float4 me1 = *reinterpret_cast<const float4*>(my_bc + c * 8 + 4);
+          const float me[8] = {me0.x, me0.y, me0.z, me0.w, me1.x, me1.y, me1.z, me1.w};
+          uint32_t pk[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int hl = c * 8 + 2 * j;
+            const float p0 = ex2_approx(fmaf(x[hl], scale, -me[2 * j]));
+            const float p1 = ex2_approx(fmaf(x[hl + 1], scale, -me[2 * j + 1]));
+            if (rescale) {
+              lpart[hl] = fmaf(lpart[hl], my_bc[kHW + hl], p0);
+              lpart[hl + 1] = fmaf(lpart[hl + 1], my_bc[kHW + hl + 1], p1);
+            } else {
+              lpart[hl] += p0;
+              lpart[hl + 1] += p1;
+            }
+            pk[j] = pack_bf16(p0, p1);
+          }
+          const int chunk = hoff / 8 + c;
+          const uint32_t dst = prow + (uint32_t)(((chunk ^ (row & 7)) & 7) << 4);
+          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
+                       "r"(pk[2]), "r"(pk[3])
+                       : "memory");
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&p_full[sb]));
+      }
+      if (!ok) {
+        if (lane == 0) report(a.err, kErrTimeout, (int32_t)it.i, 26);
+        break;
+      }
+      // ------------------------------------------------------------ epilogue
+      // Compact on purpose: it runs once per item, so it is cold in the
+      // instruction cache; rolled loops keep it short.
+      // Row sums: a butterfly leaves lane h with this warp's sum for head h,
+      // the four warps' sums meet in shared memory.
+#pragma unroll
+      for (int sh = kHW / 2; sh >= 1; sh >>= 1) {
+        const bool upper = (lane & sh) != 0;
+#pragma unroll
+        for (int j = 0; j < sh; ++j) {
+          const float send = upper ? lpart[j] : lpart[j + sh];
+          const float keep = upper ? lpart[j + sh] : lpart[j];
+          lpart[j] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
+        }
+      }
+      red_l[warp][lane] = lpart[0];
+      if (!mbar_wait(smem_u32(&o_full), (uint32_t)(items_done & 1)) ||
+          !group_sync(rbar, red_phase, lane)) {
+        if (lane == 0) report(a.err, kErrTimeout, (int32_t)it.i, 28);
+        break;
+      }
+      pv_seen = tiles_done;
+      {
+        const int h = hoff + lane;
+        const float l = (red_l[4 * wg][lane] + red_l[4 * wg + 1][lane]) +
+                        (red_l[4 * wg + 2][lane] + red_l[4 * wg + 3][lane]);
+        const float m = m_run;
+        float nrm = 1.f;
+        if (a.n_split == 1) {
+          // normaliser (with the sink in the denominator) and log-sum-exp
+          float den = l, f = 1.f, mm = m;
+          if (a.sink != nullptr && h < nh) {
+            const float z = __ldg(a.sink + h_base + h) * kLog2e;
+            const float M = fmaxf(m, z);
+            const float rr = M == -INFINITY ? 0.f : M;
+            f = exp2f(m - rr);
+            den = l * f + exp2f(z - rr);
+            mm = rr;
+          }
+          nrm = den > 0.f ? __fdividef(f, den) : 0.f;
+          if (wq == 0 && a.lse != nullptr && h < nh)
+            a.lse[it.i * a.H + h_base + h] = den > 0.f ? (mm + log2f(den)) / kLog2e : -INFINITY;
+        } else if (wq == 0 && h < nh) {
+          *reinterpret_cast<float2*>(a.part_ml + ((it.i * a.n_split + it.split) * a.H + h_base + h) * 2) =
+              make_float2(m, l);
+        }
+        my_bc[kHW + lane] = nrm;
+      }
+      __syncwarp();
+      tc::fence_after_sync();
+      const int d = row;   // O^T lane = output dim
+      if (a.n_split == 1) {
+        __nv_bfloat16* const outp = a.out + (it.i * a.H + h_base) * kD + d;
+#pragma unroll 1
+        for (int c = 0; c < kHW / 16; ++c) {
+          uint32_t r[16];
+          tc::tmem_ld16(tm_o + hoff + c * 16 + lane_base, r);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int h = hoff + c * 16 + j;
+            if (h < nh) outp[(int64_t)h * kD] = __float2bfloat16_rn(__uint_as_float(r[j]) * my_bc[kHW + c * 16 + j]);
+          }
+        }
+      } else {
+        float* const accp = a.part_acc + ((it.i * a.n_split + it.split) * a.H + h_base) * kD + d;
+#pragma unroll 1
+        for (int c = 0; c < kHW / 16; ++c) {
+          uint32_t r[16];
+          tc::tmem_ld16(tm_o + hoff + c * 16 + lane_base, r);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int h = hoff + c * 16 + j;
+            if (h < nh) accp[(int64_t)h * kD] = __uint_as_float(r[j]);
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&o_empty));
+      ++items_done;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == kMmaWarp) tc::tmem_dealloc(tmem_base, kTmemCols);
+}
+
+}  // namespace
+
+bool tc_attention_supported(const AttnArgs& a) {
+  if (a.T * (int64_t)a.H > INT32_MAX || a.kv.n_rows > INT32_MAX) return false;
+  if (a.win_len == nullptr && a.window > 0 && a.win_rows <= 0) return false;   // raw rows unknown
+  if (a.win_len && a.T * (int64_t)a.window > INT32_MAX) return false;
+  return true;
+}
+
+// The persistent tensor-core kernel pays a pipeline fill and an epilogue per
+// work item; it wins once every SM has several items to stream through.  With
+// fewer queries (decode batches) the one-CTA-per-item mma.sync kernel, many
+// CTAs per SM, hides latency better.
+bool tc_attention_preferred(const AttnArgs& a) {
+#ifdef CSA_TC_ATTN_ALWAYS
+  return true;
+#else
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return a.T * (int64_t)((a.H + kNP - 1) / kNP) >= 4 * (int64_t)sms;
+#endif
+}
+
+cudaError_t launch_attention_tc(const Launch& L, const AttnArgs& a) {
+  CUtensorMap t, w, q;
+  const uint64_t kv_rows = (uint64_t)a.kv.n_rows;
+  if (!make_tmap_bf16_2d(&t, a.kv.data, kD, kv_rows, kD, 64, kRows)) return cudaErrorInvalidValue;
+  const uint64_t win_rows = a.win_len ? (uint64_t)(a.T * a.window) : (uint64_t)a.win_rows;
+  if (a.window > 0 && win_rows > 0) {
+    if (!make_tmap_bf16_2d(&w, a.win, kD, win_rows, kD, 64, kRows)) return cudaErrorInvalidValue;
+  } else {
+    w = t;   // no window rows are ever read
+  }
+  if (!make_tmap_bf16_2d(&q, a.q, kD, (uint64_t)(a.T * a.H), kD, 64, kNP)) return cudaErrorInvalidValue;
+  TcAttnParams p;
+  p.a = a;
+  p.hgroups = (a.H + kNP - 1) / kNP;
+  p.items = a.T * a.n_split * p.hgroups;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = p.items < sms ? p.items : sms;
+  if (grid < 1) return cudaSuccess;
+  const int smem = 2 * kQTile + kStages * kKvTile + 2 * kPTile + 1024;
+  cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  attn_tc_kernel<<<(unsigned)grid, kThreads, smem, L.stream>>>(t, w, q, p);
+  return cudaSuccess;
+}
+
+}  // namespace csa

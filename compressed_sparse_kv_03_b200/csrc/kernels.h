@@ -93,6 +93,7 @@ struct AttnArgs {
   const __nv_bfloat16* win;
   const int32_t* win_len;
   int window;
+  int64_t win_rows;             // raw rows of `win` when win_len is null (0 = unknown)
   float sm_scale;
   const float* sink;            // [H] or null
   __nv_bfloat16* out;           // [T, H, 128]
@@ -105,6 +106,12 @@ struct AttnArgs {
   WsHeader* err;
 };
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a);
+// tcgen05 path (d = 128; any H, in groups of 64 heads)
+bool tc_attention_supported(const AttnArgs& a);
+bool tc_attention_preferred(const AttnArgs& a);
+// 0 automatic, 1 tensor-core kernel, 2 mma.sync kernel
+int32_t attention_kernel_choice();
+cudaError_t launch_attention_tc(const Launch& L, const AttnArgs& a);
 
 // Text returned by csa_last_error() for this thread.
 void set_last_error(const char* msg);

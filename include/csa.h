@@ -93,6 +93,17 @@ uint64_t csa_launch_count(void);
  */
 csa_status_t csa_set_timing_events(int32_t kernel_id, void* ev_begin, void* ev_end);
 
+/*
+ * Attention kernel choice for csa_sparse_attn_prefill, csa_sparse_attn_decode
+ * and hca_attn (process-wide; a library setting with no counterpart in the
+ * method).  0 = automatic (default): the tcgen05 tensor-core kernel when the
+ * call has at least four 64-head work items per SM, else the mma.sync kernel;
+ * 1 = always the tcgen05 kernel where it supports the call; 2 = always the
+ * mma.sync kernel.  Both compute the same attention within the same
+ * tolerance.  Returns CSA_ERR_INVALID_ARG for any other value.
+ */
+csa_status_t csa_set_attention_kernel(int32_t choice);
+
 /* ---- workspace ------------------------------------------------------------ */
 /*
  * Calls that take `ws` need a caller-allocated device workspace of at least

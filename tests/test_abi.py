@@ -119,6 +119,13 @@ def test_timing_event_hook_validation(lib):
     assert lib.csa_set_timing_events(0, None, None) == 0
 
 
+def test_attention_kernel_choice_validation(lib):
+    assert lib.csa_set_attention_kernel(3) == 1 and b"out of range" in lib.csa_last_error()
+    assert lib.csa_set_attention_kernel(-1) == 1
+    for choice in (1, 2, 0):
+        assert lib.csa_set_attention_kernel(choice) == 0
+
+
 def test_product_path_does_not_import_the_oracle():
     """The package and the bench's timed path never touch oracle/."""
     pkg = os.path.join(ROOT, "compressed_sparse_kv_03_b200")

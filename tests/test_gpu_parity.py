@@ -38,6 +38,15 @@ def _csa():
     return csa
 
 
+@pytest.fixture(params=["tcgen05", "mma_sync"])
+def attn_kernel(request):
+    """Run an attention test once per attention kernel."""
+    csa = _csa()
+    csa.set_attention_kernel(request.param)
+    yield request.param
+    csa.set_attention_kernel("auto")
+
+
 # ---------------------------------------------------------------------------
 # step 1: compression
 # ---------------------------------------------------------------------------
@@ -181,6 +190,7 @@ def test_indexer_topk_paged(page_size):
 # ---------------------------------------------------------------------------
 # step 4: attention
 # ---------------------------------------------------------------------------
+@pytest.mark.usefixtures("attn_kernel")
 @pytest.mark.parametrize("L,H,W,k,sink", [(300, 64, 128, 64, False), (257, 8, 16, 40, True),
                                           (130, 20, 1, 33, False), (200, 128, 64, 100, True)])
 def test_sparse_attn_prefill(L, H, W, k, sink):
@@ -200,6 +210,7 @@ def test_sparse_attn_prefill(L, H, W, k, sink):
     np.testing.assert_allclose(f64(lse), ref_lse, atol=1e-3, rtol=1e-4)
 
 
+@pytest.mark.usefixtures("attn_kernel")
 @pytest.mark.parametrize("B,H,k,paged,sink", [(5, 64, 2048, False, False), (3, 64, 300, True, True),
                                               (7, 16, 100, False, True), (2, 128, 513, True, False)])
 def test_sparse_attn_decode(B, H, k, paged, sink):
@@ -241,6 +252,7 @@ def test_sparse_attn_decode(B, H, k, paged, sink):
         np.testing.assert_allclose(f64(lse[b]), ref_lse, atol=1e-3, rtol=1e-4)
 
 
+@pytest.mark.usefixtures("attn_kernel")
 @pytest.mark.parametrize("B,H,m,paged", [(3, 64, 128, False), (4, 24, 4, True), (1, 64, 16, False)])
 def test_hca_decode(B, H, m, paged):
     csa = _csa()
@@ -267,6 +279,7 @@ def test_hca_decode(B, H, m, paged):
     assert_close_attn(out, ref, "hca decode")
 
 
+@pytest.mark.usefixtures("attn_kernel")
 def test_hca_prefill():
     csa = _csa()
     g = synth.generator(95)
@@ -280,6 +293,7 @@ def test_hca_prefill():
     assert_close_attn(out, ref, "hca prefill")
 
 
+@pytest.mark.usefixtures("attn_kernel")
 def test_attention_device_check_reports_bad_index():
     """An entry id outside the cache is skipped and reported through the
     workspace header; the other queries are unaffected."""
@@ -305,6 +319,7 @@ def test_attention_device_check_reports_bad_index():
         assert_close_attn(out[b], ref, "unaffected query")
 
 
+@pytest.mark.usefixtures("attn_kernel")
 def test_decode_is_deterministic():
     csa = _csa()
     g = synth.generator(101)

@@ -286,6 +286,8 @@ class MixedDecode:
                 "l2": f"inputs larger than L2: {self.step_bytes / 1e6:.0f} MB streamed per step"}
 
 
+KERNEL_NAMES = {0: "indexer_score", 1: "topk_select", 2: "attention", 3: "merge", 4: "compress"}
+
 RUNNERS = {
     synth.CFG_DECODE_128K.name: (CsaDecode, synth.CFG_DECODE_128K),
     synth.CFG_HCA_1M.name: (HcaDecode, synth.CFG_HCA_1M),
@@ -510,16 +512,33 @@ def run_ours(args, rank, world, local_rank):
     # dominant kernel; L2 flushes (where a workload needs them) run between
     # the step events, outside the timed time
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    kids = list(KERNEL_NAMES)
+    kev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)] for k in kids}
+    ev = kev[W.dominant]
     st = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for pair in ev + st:     # torch creates the CUDA events lazily, on first record
+    for pair in st:              # torch creates CUDA events lazily, on first record
         pair[0].record(stream)
         pair[1].record(stream)
+    for pair in [p for k in kids for p in kev[k]]:
+        pair[1].record(stream)   # end before begin: a kernel that never runs in the step
+        pair[0].record(stream)   # keeps a negative interval and is left out
     torch.cuda.synchronize()
+
+    def attach(i):
+        for k in kids:
+            csa.set_timing_events(k, kev[k][i][0], kev[k][i][1])
+
+    def detach():
+        for k in kids:
+            csa.set_timing_events(k)
     use_graph = not args.no_graph
     launches_before = csa.launch_count()
-    graphs = []
+    graphs, bgraphs = [], []
     if use_graph:
+        # timed graphs carry events around the dominant kernel only (each
+        # event node costs the step a little); the per-kernel breakdown comes
+        # from separate, untimed replays of graphs with events around every kernel
         for i in range(K):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
@@ -528,6 +547,13 @@ def run_ours(args, rank, world, local_rank):
                 csa.set_timing_events(W.dominant)
             graphs.append(g)
         launches = csa.launch_count() - launches_before
+        for i in range(K):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                attach(i)
+                W.step()
+                detach()
+            bgraphs.append(g)
         for g in graphs[:2]:         # untimed warm replays
             g.replay()
             between()
@@ -554,7 +580,22 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     ms = sum(b.elapsed_time(e) for b, e in st)
     dom_ms = [b.elapsed_time(e) for b, e in ev]
-    del graphs
+    # per-kernel breakdown, outside the timed region
+    for i in range(K):
+        if use_graph:
+            bgraphs[i].replay()
+        else:
+            attach(i)
+            W.step()
+            detach()
+        between()
+    torch.cuda.synchronize()
+    kernels_us = {}
+    for k in kids:
+        t = statistics.median(b.elapsed_time(e) for b, e in kev[k]) * 1e3
+        if t > 0.05:
+            kernels_us[KERNEL_NAMES[k]] = round(t, 2)
+    del graphs, bgraphs
     ms = max_over_ranks([ms], device="cuda")[0]
     ms_per_step = ms / K
     flush_note = ""
@@ -605,7 +646,12 @@ def run_ours(args, rank, world, local_rank):
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": W.h2d,
                     "d2h_bytes_per_step": W.d2h},
-            "clocks": clk, "gpu_launches": int(launches)}
+            "clocks": clk, "gpu_launches": int(launches),
+            "kernels_us": {"median_per_step": kernels_us,
+                           "note": "CUDA events around each library kernel in untimed replays "
+                                   "of the step (event nodes add about a microsecond or two to "
+                                   "each); for a kernel launched more than once in a step, its "
+                                   "last launch"}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         u, s, desc, threads = oracle_sample(args.workload, args.cpu_budget)
         line["cpu_baseline"] = {"value": u / s if s else 0.0, "unit": "tokens/s", "cores": threads,

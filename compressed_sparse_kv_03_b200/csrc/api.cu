@@ -95,6 +95,20 @@ Split attn_split(int64_t T, int64_t total_max, int H) {
   return Split{(int)n, (int)len};
 }
 
+// Split for the persistent tensor-core kernel: at most one work item per SM
+// (a 64-head group of one query over one slice), slices of whole 128-row tiles
+// as even as possible.  Never more slices than `ws` (the workspace layout).
+Split attn_split_tc(int64_t T, int64_t total_max, int H, const Split& ws) {
+  const int64_t q_items = T * ((H + 63) / 64);
+  const int64_t tiles = (total_max + 127) / 128;
+  int64_t n_max = q_items >= kNumSMs ? 1 : kNumSMs / q_items;
+  if (n_max > ws.n) n_max = ws.n;
+  if (n_max <= 1 || tiles <= 1) return Split{1, (int)(tiles * 128 > 128 ? tiles * 128 : 128)};
+  const int64_t len_tiles = (tiles + n_max - 1) / n_max;
+  const int64_t n = (tiles + len_tiles - 1) / len_tiles;
+  return Split{(int)n, (int)(len_tiles * 128)};
+}
+
 size_t attn_ws_bytes(int64_t T, int H, int64_t total_max) {
   const Split sp = attn_split(T, total_max, H);
   if (sp.n == 1) return kWsHeader;
@@ -410,6 +424,7 @@ csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
   a.out = (__nv_bfloat16*)out;
   a.lse = lse;
   // prefill: one slice per query (many queries fill the GPU)
+  a.use_tc = attention_uses_tc(a);
   a.n_split = 1;
   a.split_len = (int)(((int64_t)top_k + window + 63) / 64 * 64);
   st = check_ws(ws, ws_bytes, kWsHeader, name);
@@ -456,9 +471,11 @@ csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_com
   a.sink = sink;
   a.out = (__nv_bfloat16*)out;
   a.lse = lse;
-  const Split sp = attn_split(B, (int64_t)top_k + window, H);
-  const size_t need = sp.n == 1 ? kWsHeader : attn_ws_bytes(B, H, (int64_t)top_k + window);
+  const Split sp_ws = attn_split(B, (int64_t)top_k + window, H);
+  const size_t need = sp_ws.n == 1 ? kWsHeader : attn_ws_bytes(B, H, (int64_t)top_k + window);
   if ((st = check_ws(ws, ws_bytes, need, name)) != CSA_OK) return st;
+  a.use_tc = attention_uses_tc(a);
+  const Split sp = a.use_tc ? attn_split_tc(B, (int64_t)top_k + window, H, sp_ws) : sp_ws;
   a.n_split = sp.n;
   a.split_len = sp.len;
   a.err = static_cast<WsHeader*>(ws);
@@ -509,9 +526,11 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
   a.sink = sink;
   a.out = (__nv_bfloat16*)out;
   a.lse = lse;
-  const Split sp = attn_split(T, max_entries + window, H);
-  const size_t need = sp.n == 1 ? kWsHeader : attn_ws_bytes(T, H, max_entries + window);
+  const Split sp_ws = attn_split(T, max_entries + window, H);
+  const size_t need = sp_ws.n == 1 ? kWsHeader : attn_ws_bytes(T, H, max_entries + window);
   if ((st = check_ws(ws, ws_bytes, need, name)) != CSA_OK) return st;
+  a.use_tc = attention_uses_tc(a);
+  const Split sp = a.use_tc ? attn_split_tc(T, max_entries + window, H, sp_ws) : sp_ws;
   a.n_split = sp.n;
   a.split_len = sp.len;
   a.err = static_cast<WsHeader*>(ws);

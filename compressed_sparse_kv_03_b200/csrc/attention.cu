@@ -329,11 +329,14 @@ cudaError_t launch_merge(const Launch& L, const AttnArgs& a) {
 
 }  // namespace
 
+bool attention_uses_tc(const AttnArgs& a) {
+  const int32_t choice = attention_kernel_choice();
+  return choice != 2 && tc_attention_supported(a);
+}
+
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {
   if (a.T == 0) return cudaSuccess;
-#ifndef CSA_NO_TC_ATTENTION
-  const int32_t choice = attention_kernel_choice();
-  if (choice != 2 && tc_attention_supported(a) && (choice == 1 || tc_attention_preferred(a))) {
+  if (a.use_tc) {
     L.begin(kKernelAttention);
     cudaError_t e = launch_attention_tc(L, a);
     if (e != cudaSuccess) return e;
@@ -341,7 +344,6 @@ cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {
     if (e != cudaSuccess || a.n_split == 1) return e;
     return launch_merge(L, a);
   }
-#endif
   const int nw = a.H >= 64 ? 4 : (a.H + 15) / 16;
   const int hgroups = (a.H + nw * 16 - 1) / (nw * 16);
   const dim3 grid((unsigned)a.T, (unsigned)a.n_split, (unsigned)hgroups);

@@ -14,7 +14,7 @@
 // written by the softmax threads (thread = row, 64 heads = one 128-byte row).
 //
 // Warp roles (persistent CTAs over (query, split, head group) work items):
-//   warps 9-10 producers: selected rows gathered with 16-byte cp.async into
+//   warps 9-15 producers: selected rows gathered with 16-byte cp.async into
 //              their swizzled slots (through the page table when paged),
 //              contiguous rows (HCA, window) with 128-row TMA boxes; the
 //              item's query heads once per item
@@ -48,7 +48,7 @@ constexpr int kPTile = kRows * kNP * 2;         // 16 KB
 constexpr int kSmWarps = 8;                     // two softmax warpgroups
 constexpr int kHW = kNP / 2;                    // heads per softmax warpgroup
 constexpr int kMmaWarp = kSmWarps, kProducerWarp = kSmWarps + 1;
-constexpr int kProducerWarps = 2;
+constexpr int kProducerWarps = 7;
 constexpr int kProducerThreads = kProducerWarps * 32;
 // kv_full arrivals per tile: one cp.async completion per producer thread plus
 // one release arrive per producer warp (after its row-validity words)
@@ -191,7 +191,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
   __shared__ __align__(8) uint64_t q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2];
   __shared__ __align__(8) uint64_t o_full, o_empty, o_step, red_bar[2];
   __shared__ uint32_t tmem_base_sh;
-  __shared__ uint32_t row_ok[kStages][kRows / 32];   // bit b of word w: row 32w + b is valid
+  // validity of the tile's rows, one word per producer warp: bit 2j + s of
+  // word k is row 2 (k + 7 j) + s
+  __shared__ uint32_t row_ok[kStages][8];
   __shared__ float red_max[2][kSmWarps][kHW];   // per-warp tile maxima, by tile parity
   __shared__ float red_l[kSmWarps][kHW];        // per-warp row sums at the end of an item
   __shared__ __align__(16) float w_bcast[kSmWarps][2 * kHW];   // per warp: exponent offsets, factors
@@ -231,12 +233,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
   const uint32_t tm_o = tmem_base + 2 * kNP;    // O^T
   const int64_t n_items = p.items;
 
+  // Registers: the MMA and producer warpgroups give theirs down to 72 per
+  // thread, the softmax warpgroups take 184 (2 x 128 x (72 + 184) = the
+  // 512 x 128 the block is launched with).
+  if (warp >= kMmaWarp) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
   if (warp >= kProducerWarp) {
     // ================================================================ producer
-    // Two warps.  Gathered rows: thread pt copies rows pt and pt + 64 with
-    // 16-byte cp.async into their swizzled slots.  Contiguous rows: thread 0
-    // issues two 128-row TMA boxes.
-    const int pt = threadIdx.x - kProducerWarp * 32;   // 0 .. 63
+    // Seven warps.  Gathered rows: the tile's 64 row pairs are dealt round
+    // robin (pair p to warp p mod 7); lane l of a warp resolves the row
+    // 2 (pk + 7 (l >> 1)) + (l & 1) and the warp copies its rows with 16-byte
+    // cp.async, 16 lanes per 256-byte row, two rows per instruction.  Several
+    // warps keep enough copies in flight to stream the gather.  Contiguous
+    // rows: one thread issues two 128-row TMA boxes.
+    const int pk = warp - kProducerWarp;              // 0 .. kProducerWarps - 1
+    const int pt = threadIdx.x - kProducerWarp * 32;
+    const int my_pairs = (kRows / 2 - pk + kProducerWarps - 1) / kProducerWarps;
+    const bool lane_has_row = (lane >> 1) < my_pairs;
+    const int my_row = 2 * (pk + kProducerWarps * (lane >> 1)) + (lane & 1);
     if (pt == 0) {
       tc::prefetch_tmap(&tm_kv_tile);
       tc::prefetch_tmap(&tm_win);
@@ -263,6 +277,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
       ok = __shfl_sync(0xffffffffu, ok, 0);   // keep each warp's control flow uniform
       if (!ok) break;
       ++items_done;
+      int64_t e_next = -1;   // this lane's entry id in the item's next gathered tile
+      bool have_next = false;
       for (int t = 0; t < it.n_tiles && ok; ++t, ++tiles_done) {
         const int slot = (int)(tiles_done % kStages);
         const bool got =
@@ -279,32 +295,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         const uint32_t fb = smem_u32(&kv_full[slot]);
         const bool sel = t < it.n_sel_tiles;
         if (sel && (a.idx != nullptr || a.kv.page_table != nullptr)) {
-          // both rows' entry indices are loaded before either is used
-          int64_t e[2];
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int r = pt + 64 * half;
-            e[half] = r >= n ? -1 : (a.idx ? (int64_t)__ldg(a.idx + it.i * a.top_k + v + r) : v + r);
+          const bool mine = lane_has_row && my_row < n;
+          const int64_t e = have_next ? e_next
+                                      : (!mine ? -1 : (a.idx ? (int64_t)__ldg(a.idx + it.i * a.top_k + v + my_row)
+                                                             : v + my_row));
+          // the next gathered tile's entry id loads while this tile is copied
+          have_next = t + 1 < it.n_sel_tiles;
+          if (have_next) {
+            int64_t v2;
+            int n2;
+            tile_span(it, t + 1, v2, n2);
+            const bool mine2 = lane_has_row && my_row < n2;
+            e_next = !mine2 ? -1 : (a.idx ? (int64_t)__ldg(a.idx + it.i * a.top_k + v2 + my_row) : v2 + my_row);
           }
+          const int64_t row = mine ? cache_row(a.kv, it.seq, e, a.err, (int32_t)it.i) : -1;
+          const uint32_t okb = __ballot_sync(0xffffffffu, row >= 0);   // bit l: lane l's row
+          if (lane == 0) row_ok[slot][pk] = okb;
+          const int c = lane & 15, sub = lane >> 4;
+          const uint32_t cdst = dst + (c >> 3) * kKBlock;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int r = pt + 64 * half;
-            const int64_t row = r < n ? cache_row(a.kv, it.seq, e[half], a.err, (int32_t)it.i) : -1;
-            const uint32_t okb = __ballot_sync(0xffffffffu, row >= 0);
-            if (lane == 0) row_ok[slot][r >> 5] = okb;
-            const char* src = reinterpret_cast<const char*>(a.kv.data + (row >= 0 ? row : 0) * kD);
-            const uint32_t rdst = dst + (uint32_t)r * 128;
-#pragma unroll
-            for (int ch = 0; ch < 16; ++ch) {
-              const int kb = ch >> 3, c = ch & 7;
-              cp_async_16(rdst + kb * kKBlock + (uint32_t)(((c ^ (r & 7)) & 7) << 4), src + ch * 16,
-                          row >= 0);
+          for (int j = 0; j < (kRows / 2 + kProducerWarps - 1) / kProducerWarps; ++j) {
+            if (j < my_pairs) {
+              const int64_t rr = __shfl_sync(0xffffffffu, row, 2 * j + sub);
+              const int r = 2 * (pk + kProducerWarps * j) + sub;
+              const char* src = reinterpret_cast<const char*>(a.kv.data + (rr >= 0 ? rr : 0) * kD) + c * 16;
+              cp_async_16(cdst + (uint32_t)r * 128 + (uint32_t)((((c & 7) ^ (r & 7)) & 7) << 4), src,
+                          rr >= 0);
             }
           }
           cp_async_mbar_arrive_noinc(fb);
           __syncwarp();
-          if (lane == 0) mbar_arrive(fb);   // releases this warp's row_ok words
-        } else if (pt == 0) {
+          if (lane == 0) mbar_arrive(fb);   // releases this warp's row_ok word
+        } else if (pk == 0) {
           // contiguous rows: eligible entries of a contiguous cache, or the window
           int64_t row0;
           const CUtensorMap* map;
@@ -315,7 +337,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
             int64_t lim = a.kv.n_rows - row0;
             if (a.kv.seq_stride > 0 && a.kv.seq_stride - v < lim) lim = a.kv.seq_stride - v;
             if (lim < n) {
-              report(a.err, kErrEntryIndex, (int32_t)it.i, v + (lim > 0 ? lim : 0));
+              if (lane == 0) report(a.err, kErrEntryIndex, (int32_t)it.i, v + (lim > 0 ? lim : 0));
               n = lim > 0 ? (int)lim : 0;
             }
           } else {
@@ -323,15 +345,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
             row0 = a.win_len ? it.i * a.window + w : it.win_first + w;
             map = &tm_win;
           }
-#pragma unroll
-          for (int w = 0; w < kRows / 32; ++w) {
-            const int lo = w * 32;
-            row_ok[slot][w] = n >= lo + 32 ? 0xffffffffu : (n > lo ? (1u << (n - lo)) - 1u : 0u);
+          if (lane < kProducerWarps) {   // the validity word of producer warp `lane`
+            uint32_t word = 0;
+            for (int j = 0; lane + kProducerWarps * j < kRows / 2; ++j) {
+              const int r = 2 * (lane + kProducerWarps * j);
+              if (r < n) word |= 1u << (2 * j);
+              if (r + 1 < n) word |= 2u << (2 * j);
+            }
+            row_ok[slot][lane] = word;
+            if (lane > 0) mbar_arrive(fb);   // releases its word
           }
-          mbar_expect_tx(fb, kKvTile);
-          tc::tma_load_2d(dst, map, 0, (int32_t)row0, fb);
-          tc::tma_load_2d(dst + kKBlock, map, 64, (int32_t)row0, fb);
-          mbar_arrive_cnt(fb, kKvFullCount);   // releases the row_ok words
+          if (lane == 0) {
+            mbar_expect_tx(fb, kKvTile);
+            tc::tma_load_2d(dst, map, 0, (int32_t)row0, fb);
+            tc::tma_load_2d(dst + kKBlock, map, 64, (int32_t)row0, fb);
+            mbar_arrive_cnt(fb, kKvFullCount - (kProducerWarps - 1));
+          }
         }
       }
     }
@@ -346,7 +375,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         mbar_wait(smem_u32(&q_full[(items_done - 1) & 1]), (uint32_t)(((items_done - 1) >> 1) & 1),
                   200000000ll);
     }
-  } else if (warp == kMmaWarp) {
+  } else {
     // ================================================================ MMA
     if (lane == 0) {
       int64_t tiles_done = 0, items_done = 0, pv_done = 0;
@@ -417,7 +446,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         ++items_done;
       }
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 184;\n" ::: "memory");
     // ================================================================ softmax + epilogue
     // Warpgroup wg (warps 4wg .. 4wg+3) owns heads [32 wg, 32 wg + 32) of every
     // tile: thread = row of S^T in the tile loop, = dim of O^T in the epilogue.
@@ -426,6 +457,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
     const int wg = warp >> 2, wq = warp & 3;
     const int hoff = wg * kHW;
     const int row = wq * 32 + lane;
+    const int ok_word = (row >> 1) % kProducerWarps, ok_bit = 2 * ((row >> 1) / kProducerWarps) + (row & 1);
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const uint32_t rbar = smem_u32(&red_bar[wg]);
     const float scale = a.sm_scale * kLog2e;
@@ -480,9 +512,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&s_empty[sb]));
-        const bool valid = (row_ok[slot][row >> 5] >> (row & 31)) & 1u;
+        const bool valid = (row_ok[slot][ok_word] >> ok_bit) & 1u;
         // per-head tile maxima of the raw logits across this warp's 32 rows
-        float mine = -INFINITY;
+        float mine;
+        mine = -INFINITY;
 #pragma unroll
         for (int h = 0; h < kHW; ++h) {
           if (!valid) x[h] = -INFINITY;
@@ -660,21 +693,6 @@ bool tc_attention_supported(const AttnArgs& a) {
   if (a.win_len == nullptr && a.window > 0 && a.win_rows <= 0) return false;   // raw rows unknown
   if (a.win_len && a.T * (int64_t)a.window > INT32_MAX) return false;
   return true;
-}
-
-// The persistent tensor-core kernel pays a pipeline fill and an epilogue per
-// work item; it wins once every SM has several items to stream through.  With
-// fewer queries (decode batches) the one-CTA-per-item mma.sync kernel, many
-// CTAs per SM, hides latency better.
-bool tc_attention_preferred(const AttnArgs& a) {
-#ifdef CSA_TC_ATTN_ALWAYS
-  return true;
-#else
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return a.T * (int64_t)((a.H + kNP - 1) / kNP) >= 4 * (int64_t)sms;
-#endif
 }
 
 cudaError_t launch_attention_tc(const Launch& L, const AttnArgs& a) {

@@ -104,13 +104,16 @@ struct AttnArgs {
   float* part_acc;              // [T, n_split, H, 128]
   float* part_ml;               // [T, n_split, H, 2]
   WsHeader* err;
+  int use_tc;                   // tcgen05 kernel (else mma.sync); see attention_uses_tc
 };
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a);
 // tcgen05 path (d = 128; any H, in groups of 64 heads)
 bool tc_attention_supported(const AttnArgs& a);
-bool tc_attention_preferred(const AttnArgs& a);
 // 0 automatic, 1 tensor-core kernel, 2 mma.sync kernel
 int32_t attention_kernel_choice();
+// Which attention kernel a call with these arguments runs (fields other than
+// the split / workspace ones must be set).
+bool attention_uses_tc(const AttnArgs& a);
 cudaError_t launch_attention_tc(const Launch& L, const AttnArgs& a);
 
 // Text returned by csa_last_error() for this thread.

@@ -323,12 +323,11 @@ csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_c
   uint32_t* hist = lay.bitmap ? reinterpret_cast<uint32_t*>(wsb + lay.hist_off) : nullptr;
   for (int64_t t0 = 0; t0 < T; t0 += lay.chunk) {
     const int64_t n = T - t0 < lay.chunk ? T - t0 : lay.chunk;
-    // zero the histogram of this chunk (decode mode)
-    cudaError_t e = cudaSuccess;
-    if (lay.bitmap) {
-      e = cudaMemsetAsync(wsb + lay.hist_off, 0, (size_t)n * kHistBins * sizeof(uint32_t), L.stream);
-      if (e != cudaSuccess) return cuda_status(e, "indexer histogram memset");
-    }
+    // zero the histogram of this chunk (decode mode) and the scorer's work
+    // counter (they are adjacent: one memset)
+    const size_t zero_off = lay.bitmap ? lay.hist_off : lay.counter_off;
+    cudaError_t e = cudaMemsetAsync(wsb + zero_off, 0, lay.counter_off + sizeof(uint32_t) - zero_off, L.stream);
+    if (e != cudaSuccess) return cuda_status(e, "indexer workspace memset");
     IndexerArgs ia;
     ia.q_idx = (const __nv_bfloat16*)q_idx;
     ia.w = w;
@@ -344,6 +343,7 @@ csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_c
     ia.keys_out = keys;
     ia.key_stride = lay.stride;
     ia.hist = hist;
+    ia.work = reinterpret_cast<uint32_t*>(wsb + lay.counter_off);
     ia.err = hdr;
     e = launch_indexer_scores(L, ia, n);
     if (e != cudaSuccess) return cuda_status(e, "indexer score launch");

@@ -270,10 +270,12 @@ __global__ void __launch_bounds__(NW * 32) attn_kernel(AttnArgs a) {
 }
 
 // Combine the split partials of one (query, head): 64 threads, 2 dims each.
-// One warp per (query, head): lane s holds split s's weight 2^(m_s - M), the
-// warp sums the weighted denominators, then accumulates the 128-dim partial
-// outputs (4 dims per lane) over the splits with independent loads.
+// One warp per (query, head), 4 dims per lane.  Splits are taken in chunks
+// of 16 whose loads are all issued before any is used (one memory round trip
+// per chunk); the running maximum, denominator and output are rescaled between
+// chunks.  The sink enters as one more term with logit z and no value.
 constexpr int kMergeHeads = 4;   // warps per block
+constexpr int kMergeChunk = 16;
 
 __global__ void __launch_bounds__(32 * kMergeHeads) merge_kernel(AttnArgs a) {
   const int64_t i = blockIdx.x;
@@ -283,35 +285,46 @@ __global__ void __launch_bounds__(32 * kMergeHeads) merge_kernel(AttnArgs a) {
   const int ns = a.n_split;
   const float* const ml = a.part_ml + (i * ns * a.H + h) * 2;
   const float* const acc = a.part_acc + (i * ns * a.H + h) * D + 4 * lane;
-  float M = a.sink ? __ldg(a.sink + h) * kLog2e : -INFINITY;
-  const float z = M;
-  for (int s = lane; s < ns; s += 32) M = fmaxf(M, ml[(int64_t)s * a.H * 2]);
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float ref = M == -INFINITY ? 0.f : M;
-  float den = 0.f;
-  for (int s = lane; s < ns; s += 32) {
-    const float2 mls = *reinterpret_cast<const float2*>(ml + (int64_t)s * a.H * 2);
-    den = fmaf(mls.y, exp2f(mls.x - ref), den);
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-  den += exp2f(z - ref);
+  const float z = a.sink ? __ldg(a.sink + h) * kLog2e : -INFINITY;
+  float M = z, den = z == -INFINITY ? 0.f : 1.f;   // relative to 2^M
   float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < ns; s0 += 32) {
-    const int s_l = s0 + lane;
-    const float f_l = s_l < ns ? exp2f(ml[(int64_t)s_l * a.H * 2] - ref) : 0.f;
-    const int n = ns - s0 < 32 ? ns - s0 : 32;
-#pragma unroll 4
-    for (int j = 0; j < n; ++j) {
+  for (int s0 = 0; s0 < ns; s0 += kMergeChunk) {
+    const int cnt = ns - s0 < kMergeChunk ? ns - s0 : kMergeChunk;
+    float2 mls = make_float2(-INFINITY, 0.f);
+    if (lane < cnt) mls = *reinterpret_cast<const float2*>(ml + (int64_t)(s0 + lane) * a.H * 2);
+    float4 v[kMergeChunk];
+#pragma unroll
+    for (int j = 0; j < kMergeChunk; ++j)
+      if (j < cnt) v[j] = *reinterpret_cast<const float4*>(acc + (int64_t)(s0 + j) * a.H * D);
+    float cm = mls.x;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+    const float nM = fmaxf(M, cm);
+    const float ref = nM == -INFINITY ? 0.f : nM;
+    const float fo = exp2f(M - ref);
+    den *= fo;
+    out.x *= fo;
+    out.y *= fo;
+    out.z *= fo;
+    out.w *= fo;
+    const float f_l = lane < cnt ? exp2f(mls.x - ref) : 0.f;
+    float dl = f_l * mls.y;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
+    den += dl;
+#pragma unroll
+    for (int j = 0; j < kMergeChunk; ++j) {
       const float f = __shfl_sync(0xffffffffu, f_l, j);
-      const float4 v = *reinterpret_cast<const float4*>(acc + (int64_t)(s0 + j) * a.H * D);
-      out.x = fmaf(v.x, f, out.x);
-      out.y = fmaf(v.y, f, out.y);
-      out.z = fmaf(v.z, f, out.z);
-      out.w = fmaf(v.w, f, out.w);
+      if (j < cnt) {
+        out.x = fmaf(v[j].x, f, out.x);
+        out.y = fmaf(v[j].y, f, out.y);
+        out.z = fmaf(v[j].z, f, out.z);
+        out.w = fmaf(v[j].w, f, out.w);
+      }
     }
+    M = nM;
   }
+  const float ref = M == -INFINITY ? 0.f : M;
   const float inv = den > 0.f ? 1.f / den : 0.f;
   uint2 pk;
   pk.x = pack_bf16(out.x * inv, out.y * inv);

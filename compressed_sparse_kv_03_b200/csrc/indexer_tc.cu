@@ -17,10 +17,13 @@
 //              the head-weighted sum, the order-preserving score key,
 //              coalesced stores and (decode mode) the query's 12-bit histogram
 //              through warp-aggregated atomics.
-// Each CTA owns a contiguous range of the valid (query, 256-key chunk) pairs,
-// found from a prefix sum over the queries' chunk counts, so ragged lengths
-// stay balanced; every role walks the same range, so no metadata crosses the
-// ring.  Every wait is bounded; a timeout is reported in the workspace header.
+// The valid (query, 256-key chunk) pairs are numbered through a prefix sum
+// over the queries' chunk counts; the producers of all CTAs take them two at a
+// time from one launch-wide counter, so SMs that stream faster take more (on
+// B200 some SMs see ~20% less bandwidth than others).  The producer passes
+// each item's query, chunk and head weights to the MMA warp and the epilogue
+// through a 16-entry ring with its own full / empty barriers.  Every wait is
+// bounded; a timeout is reported in the workspace header.
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -41,36 +44,23 @@ constexpr int kAcc = 4;                            // TMEM accumulator sets (32 
 constexpr uint32_t kIdesc = tc::idesc_bf16(128, 16);
 constexpr int kTmemCols = 128;
 constexpr int kMaxQueries = 2048;
+constexpr int kRing = 16;                          // item metadata ring (> kStages + kAcc)
+constexpr int kGrab = 2;                           // items taken from the work counter at once
+#ifndef CSA_SCORE_STATIC_PCT
+#define CSA_SCORE_STATIC_PCT 70
+#endif
+constexpr int kStaticPct = CSA_SCORE_STATIC_PCT;   // items dealt out statically, percent
+
+// What the producer tells the MMA warp and the epilogue about item j: the
+// query (-1 ends the stream), the 256-key chunk and the query's head weights.
+struct __align__(16) ItemMeta {
+  float w[16];
+  int32_t t, chunk, pad0, pad1;
+};
 
 struct TcIndexerParams {
   IndexerArgs a;
   int64_t t_count;
-};
-
-// Walks this CTA's contiguous range of (query, 256-key chunk) pairs in
-// increasing order, skipping queries without chunks.
-struct ItemCursor {
-  const int32_t* prefix;   // [t_count + 1] exclusive prefix of chunk counts
-  int t;
-  int32_t v, v_end;
-  __device__ __forceinline__ void init(const int32_t* pre, int t_count, int32_t lo, int32_t hi) {
-    prefix = pre;
-    v = lo;
-    v_end = hi;
-    int l = 0, r = t_count;   // last t with prefix[t] <= lo
-    while (r - l > 1) {
-      const int mid = (l + r) >> 1;
-      if (pre[mid] <= lo) l = mid; else r = mid;
-    }
-    t = l;
-    while (t < t_count && pre[t + 1] <= v) ++t;
-  }
-  __device__ __forceinline__ bool valid() const { return v < v_end; }
-  __device__ __forceinline__ int32_t chunk() const { return v - prefix[t]; }
-  __device__ __forceinline__ void next() {
-    ++v;
-    while (v < v_end && prefix[t + 1] <= v) ++t;
-  }
 };
 
 __device__ __forceinline__ int64_t eligible(const IndexerArgs& a, int64_t t) {
@@ -90,6 +80,9 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
   __shared__ __align__(8) uint64_t tfull_bar[kAcc], tempty_bar[kAcc];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int32_t prefix[kMaxQueries + 1];
+  __shared__ int32_t nelig[kMaxQueries];
+  __shared__ ItemMeta ring[kRing];
+  __shared__ __align__(8) uint64_t ring_full[kRing], ring_empty[kRing];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -105,6 +98,10 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
       mbar_init(smem_u32(&tfull_bar[i]), 1);
       mbar_init(smem_u32(&tempty_bar[i]), 4);
     }
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(smem_u32(&ring_full[i]), 1);
+      mbar_init(smem_u32(&ring_empty[i]), 5);   // the MMA warp + one epilogue group
+    }
     mbar_fence_init();
   }
   if (warp == 1) tc::tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
@@ -118,6 +115,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
       if (pos / a.m > a.max_entries && blockIdx.x == 0)
         report(a.err, kErrEligible, (int32_t)(a.t_begin + t), pos / a.m);
       const int64_t n = eligible(a, a.t_begin + t);
+      nelig[t] = (int32_t)n;
       prefix[t] = (int32_t)((n + kItemRows - 1) / kItemRows);
       sum += prefix[t];
     }
@@ -140,28 +138,87 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
   tc::fence_after_sync();
   const uint32_t tmem_base = tmem_base_sh;
   const int32_t V = prefix[T];
-  const int32_t lo = (int32_t)((int64_t)V * blockIdx.x / gridDim.x);
-  const int32_t hi = (int32_t)((int64_t)V * (blockIdx.x + 1) / gridDim.x);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tc::prefetch_tmap(&tmap_keys);
       tc::prefetch_tmap(&tmap_q);
-      ItemCursor c;
-      c.init(prefix, T, lo, hi);
       int64_t issued = 0;
-      for (; c.valid(); c.next(), ++issued) {
-        const int64_t t = a.t_begin + c.t;
-        const int64_t s0 = (int64_t)c.chunk() * kItemRows;
+      bool ok = true;
+      // Items come from the work counter kGrab at a time; the grab after the
+      // current one is requested as soon as the current one starts, and the
+      // next item's query and head weights load while this item's keys are
+      // issued, so neither latency sits between two items.
+      // The first kStaticPct percent of the items are dealt out statically
+      // (a contiguous range per CTA, streamed in order); the rest go through
+      // the work counter.
+      const int32_t Vs = (int32_t)((int64_t)V * kStaticPct / 100);
+      const int32_t s_lo = (int32_t)((int64_t)Vs * blockIdx.x / gridDim.x);
+      const int32_t s_hi = (int32_t)((int64_t)Vs * (blockIdx.x + 1) / gridDim.x);
+      int32_t g_next = s_lo < s_hi ? s_lo : Vs + (int32_t)atomicAdd(a.work, (uint32_t)kGrab);
+      bool in_static = s_lo < s_hi;
+      int32_t nxt = 0, lim = 0;
+      int tq = 0;
+      auto take = [&]() -> int32_t {
+        if (nxt >= lim) {
+          if (g_next >= V) return -1;
+          nxt = g_next;
+          if (in_static) {
+            lim = s_hi;
+            in_static = false;
+          } else {
+            lim = g_next + kGrab < V ? g_next + kGrab : V;
+          }
+          g_next = Vs + (int32_t)atomicAdd(a.work, (uint32_t)kGrab);
+          int l = 0, r = T;   // the query: last tq with prefix[tq] <= nxt
+          while (r - l > 1) {
+            const int mid = (l + r) >> 1;
+            if (prefix[mid] <= nxt) l = mid; else r = mid;
+          }
+          tq = l;
+        }
+        while (prefix[tq + 1] <= nxt) ++tq;
+        return nxt++;
+      };
+      float wreg[16];
+      int32_t seq_reg = 0;
+      int w_tq = -1;
+      auto load_w = [&]() {   // the query's head weights and sequence
+        if (tq == w_tq) return;
+        w_tq = tq;
+        const int64_t t = a.t_begin + tq;
+#pragma unroll
+        for (int h = 0; h < 16; ++h) wreg[h] = h < a.H_I ? __ldg(a.w + t * a.H_I + h) : 0.f;
+        seq_reg = a.seq_id ? __ldg(a.seq_id + t) : 0;
+      };
+      int32_t item = take();
+      if (item >= 0) load_w();
+      while (item >= 0) {
+        const int32_t chunk = item - prefix[tq];
+        const int64_t t = a.t_begin + tq;
+        const int64_t s0 = (int64_t)chunk * kItemRows;
+        const int rs = (int)(issued % kRing);
+        if (!mbar_wait(smem_u32(&ring_empty[rs]), (uint32_t)(((issued / kRing) & 1) ^ 1))) {
+          report(a.err, kErrTimeout, (int32_t)t, 16);
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int h = 0; h < 16; ++h) ring[rs].w[h] = wreg[h];
+        ring[rs].t = tq;
+        ring[rs].chunk = chunk;
+        mbar_arrive(smem_u32(&ring_full[rs]));
+        const int cur_tq = tq;
+        const int32_t seq = seq_reg;
         const int slot = (int)(issued % kStages);
         if (!mbar_wait(smem_u32(&empty_bar[slot]), (uint32_t)(((issued / kStages) & 1) ^ 1))) {
           report(a.err, kErrTimeout, (int32_t)t, 10);
+          ok = false;
           break;
         }
         const uint32_t fb = smem_u32(&full_bar[slot]);
         mbar_arrive_expect_tx(fb, kStageKeyBytes + kQTileBytes);
-        const int32_t seq = a.seq_id ? __ldg(a.seq_id + t) : 0;
         if (a.keys.page_table == nullptr) {
           // contiguous: the item's 256 keys are one 256-row box
           tc::tma_load_2d(keys_sm + slot * kStageKeyBytes, &tmap_keys, 0,
@@ -178,7 +235,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
                                      : -1;
             row = (int64_t)page * a.keys.page_size + (s - pi * a.keys.page_size);
             if (page < 0 || row >= a.keys.n_rows) {
-              if (s < eligible(a, t)) report(a.err, kErrPageId, (int32_t)t, page);
+              if (s < nelig[cur_tq]) report(a.err, kErrPageId, (int32_t)t, page);
               row = 0;
             }
           }
@@ -187,6 +244,21 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
         }
         }
         tc::tma_load_2d(q_sm + slot * kQTileBytes, &tmap_q, 0, (int32_t)(t * a.H_I), fb);
+        ++issued;
+        item = take();
+        if (item >= 0) load_w();
+      }
+      // two end markers: the MMA warp stops at the first, each epilogue
+      // group (alternate items) at the one that falls to it
+      for (int e = 0; ok && e < 2; ++e) {
+        const int64_t j = issued + e;
+        const int rs = (int)(j % kRing);
+        if (!mbar_wait(smem_u32(&ring_empty[rs]), (uint32_t)(((j / kRing) & 1) ^ 1))) {
+          report(a.err, kErrTimeout, 0, 17);
+          break;
+        }
+        ring[rs].t = -1;
+        mbar_arrive(smem_u32(&ring_full[rs]));
       }
       // every copy must land before the CTA can exit: the last kStages
       // issued stages hold the latest phase of every slot
@@ -197,7 +269,15 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      for (int64_t j = 0; j < hi - lo; ++j) {
+      for (int64_t j = 0;; ++j) {
+        const int rs = (int)(j % kRing);
+        if (!mbar_wait(smem_u32(&ring_full[rs]), (uint32_t)((j / kRing) & 1))) {
+          report(a.err, kErrTimeout, (int32_t)j, 18);
+          break;
+        }
+        const bool end = ring[rs].t < 0;
+        mbar_arrive(smem_u32(&ring_empty[rs]));
+        if (end) break;
         const int slot = (int)(j % kStages);
         const int acc = (int)(j % kAcc);
         if (!mbar_wait(smem_u32(&full_bar[slot]), (uint32_t)((j / kStages) & 1))) {
@@ -228,24 +308,36 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
     const int group = ew >> 2;                 // handles items j with j % 2 == group
     const int quarter = warp & 3;              // TMEM lanes this warp may read
     const int row = quarter * 32 + lane;       // key within a 128-key tile
-    ItemCursor c;
-    c.init(prefix, T, lo, hi);
     int t_cached = -1;
-    float wv[16];
     int64_t n_elig = 0;
     uint32_t* out = nullptr;
     uint32_t* gh = nullptr;
-    for (int64_t j = 0; c.valid(); c.next(), ++j) {
-      if ((j & 1) != group) continue;
-      const int acc = (int)(j % kAcc);
-      if (c.t != t_cached) {
-        t_cached = c.t;
-        const int64_t t = a.t_begin + c.t;
+    for (int64_t j = group;; j += 2) {
+      const int rs = (int)(j % kRing);
+      if (!mbar_wait(smem_u32(&ring_full[rs]), (uint32_t)((j / kRing) & 1))) {
+        if (lane == 0) report(a.err, kErrTimeout, (int32_t)j, 19);
+        break;
+      }
+      const int tq = ring[rs].t;
+      const int32_t chunk = ring[rs].chunk;
+      float wv[16];
 #pragma unroll
-        for (int h = 0; h < 16; ++h) wv[h] = h < a.H_I ? __ldg(a.w + t * a.H_I + h) : 0.f;
-        n_elig = eligible(a, t);
-        out = a.keys_out + (int64_t)c.t * a.key_stride;
-        gh = HIST ? a.hist + (int64_t)c.t * kHistBins : nullptr;
+      for (int h = 0; h < 16; h += 4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(&ring[rs].w[h]);
+        wv[h] = w4.x;
+        wv[h + 1] = w4.y;
+        wv[h + 2] = w4.z;
+        wv[h + 3] = w4.w;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ring_empty[rs]));
+      if (tq < 0) break;
+      const int acc = (int)(j % kAcc);
+      if (tq != t_cached) {
+        t_cached = tq;
+        n_elig = nelig[tq];
+        out = a.keys_out + (int64_t)tq * a.key_stride;
+        gh = HIST ? a.hist + (int64_t)tq * kHistBins : nullptr;
       }
       if (!mbar_wait(smem_u32(&tfull_bar[acc]), (uint32_t)((j / kAcc) & 1))) {
         if (lane == 0) report(a.err, kErrTimeout, (int32_t)j, 13);
@@ -260,7 +352,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[acc]));
-      const int64_t s0 = (int64_t)c.chunk() * kItemRows;
+      const int64_t s0 = (int64_t)chunk * kItemRows;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const uint32_t* r = h ? r1 : r0;
@@ -292,6 +384,7 @@ bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count) {
   if ((a.max_entries + kItemRows - 1) / kItemRows * t_count > INT32_MAX) return false;
   if (a.keys.page_table != nullptr && a.keys.page_size % kBoxRows != 0) return false;
   if (a.keys.n_rows > INT32_MAX || a.T * a.H_I > INT32_MAX) return false;
+  if (a.work == nullptr) return false;
   return true;
 }
 

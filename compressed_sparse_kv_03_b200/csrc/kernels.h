@@ -50,6 +50,7 @@ struct IndexerArgs {
   uint32_t* keys_out;           // [T_chunk, key_stride]
   int64_t key_stride;
   uint32_t* hist;               // [T_chunk, kHistBins] (zeroed) or null
+  uint32_t* work;               // zeroed work counter of the tcgen05 scorer
   WsHeader* err;
 };
 cudaError_t launch_indexer_scores(const Launch& L, const IndexerArgs& a, int64_t t_count);

@@ -194,7 +194,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
   // validity of the tile's rows, one word per producer warp: bit 2j + s of
   // word k is row 2 (k + 7 j) + s
   __shared__ uint32_t row_ok[kStages][8];
-  __shared__ float red_max[2][kSmWarps][kHW];   // per-warp tile maxima, by tile parity
+  __shared__ __align__(16) float red_max[2][kSmWarps][kHW];   // per-warp tile maxima, by tile parity
   __shared__ float red_l[kSmWarps][kHW];        // per-warp row sums at the end of an item
   __shared__ __align__(16) float w_bcast[kSmWarps][2 * kHW];   // per warp: exponent offsets, factors
 
@@ -513,17 +513,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&s_empty[sb]));
         const bool valid = (row_ok[slot][ok_word] >> ok_bit) & 1u;
-        // per-head tile maxima of the raw logits across this warp's 32 rows
-        float mine;
-        mine = -INFINITY;
+        if (!__all_sync(0xffffffffu, valid)) {   // rows past the list or without an entry
 #pragma unroll
-        for (int h = 0; h < kHW; ++h) {
-          if (!valid) x[h] = -INFINITY;
-          const float mx = redux_max(x[h]);
-          if (lane == h) mine = mx;
+          for (int h = 0; h < kHW; ++h)
+            if (!valid) x[h] = -INFINITY;
         }
+        // per-head tile maxima of the raw logits across this warp's 32 rows
+        // (warp-uniform after the reduction; lane 0 publishes them)
         float (*const rm)[kHW] = red_max[sb];
-        rm[warp][lane] = mine;
+        {
+          float mx[kHW];
+#pragma unroll
+          for (int h = 0; h < kHW; ++h) mx[h] = redux_max(x[h]);
+          if (lane == 0) {
+#pragma unroll
+            for (int h = 0; h < kHW; h += 4)
+              *reinterpret_cast<float4*>(&rm[warp][h]) = make_float4(mx[h], mx[h + 1], mx[h + 2], mx[h + 3]);
+          }
+        }
         if (!(ok = group_sync(rbar, red_phase, lane))) break;
         float tmax = fmaxf(fmaxf(rm[4 * wg][lane], rm[4 * wg + 1][lane]),
                            fmaxf(rm[4 * wg + 2][lane], rm[4 * wg + 3][lane]));

@@ -490,6 +490,8 @@ def run_ours(args, rank, world, local_rank):
         cfg = dataclasses.replace(cfg, B=args.batch, name=f"{cfg.name}_B{args.batch}")
     if args.seq_len and hasattr(cfg, "L"):
         cfg = dataclasses.replace(cfg, L=args.seq_len, name=f"{cfg.name}_L{args.seq_len}")
+    if args.batch_invariant:
+        csa.set_batch_invariant(True)
     W = cls(cfg, seed_offset=rank_seed_offset(rank))
     pk = peaks()
     stream = torch.cuda.current_stream()
@@ -641,6 +643,7 @@ def run_ours(args, rank, world, local_rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded torch CPU generator, N(0,1) / U(0,1))",
             "config": {**W.config(), "parallelism": f"dp{world}" + flush_note,
+                       **({"batch_invariant": True} if args.batch_invariant else {}),
                        "timing": "one CUDA graph per step, CUDA events per step" if use_graph
                        else "eager launches, CUDA events per step"},
             "roofline": roof,
@@ -697,6 +700,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work (cpu_baseline)")
     ap.add_argument("--step-budget", type=float, default=4.0, help="seconds per reference-arm step")
+    ap.add_argument("--batch-invariant", action="store_true",
+                    help="decode attention in batch-invariant mode (fixed 512-row slices)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the dominant kernel, if captured for this build")
     args = ap.parse_args()

@@ -273,6 +273,11 @@ def set_attention_kernel(name):
     check(load().csa_set_attention_kernel(ATTENTION_KERNELS[name]))
 
 
+def set_batch_invariant(on):
+    """Batch-invariant decode attention on or off (see csa_set_batch_invariant)."""
+    check(load().csa_set_batch_invariant(1 if on else 0))
+
+
 def set_timing_events(kernel_id, begin=None, end=None):
     """Attach torch.cuda.Event objects (enable_timing=True) around every launch
     of one library kernel; pass None to detach."""

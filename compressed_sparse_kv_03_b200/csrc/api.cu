@@ -17,6 +17,7 @@ namespace {
 thread_local std::string g_last_error;
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int32_t> g_attn_kernel{0};
+std::atomic<int32_t> g_batch_invariant{0};
 struct EventPair {
   cudaEvent_t begin = nullptr, end = nullptr;
 };
@@ -109,12 +110,30 @@ Split attn_split_tc(int64_t T, int64_t total_max, int H, const Split& ws) {
   return Split{(int)n, (int)(len_tiles * 128)};
 }
 
-size_t attn_ws_bytes(int64_t T, int H, int64_t total_max) {
-  const Split sp = attn_split(T, total_max, H);
-  if (sp.n == 1) return kWsHeader;
-  const size_t acc = (size_t)T * sp.n * H * kD * sizeof(float);
-  const size_t ml = (size_t)T * sp.n * H * 2 * sizeof(float);
+// Batch-invariant decode: fixed 512-row slices of every query's row list.
+constexpr int kInvariantSliceRows = 512;
+Split attn_split_invariant(int64_t total_max) {
+  int64_t n = (total_max + kInvariantSliceRows - 1) / kInvariantSliceRows;
+  if (n < 1) n = 1;
+  return Split{(int)n, kInvariantSliceRows};
+}
+
+size_t attn_partials_bytes(int64_t T, int H, int n) {
+  if (n == 1) return kWsHeader;
+  const size_t acc = (size_t)T * n * H * kD * sizeof(float);
+  const size_t ml = (size_t)T * n * H * 2 * sizeof(float);
   return kWsHeader + align256(acc) + align256(ml);
+}
+
+// Workspace of a decode call: the mma.sync split (which bounds the tcgen05
+// one) and, in batch-invariant mode, the fixed slices.
+size_t attn_ws_bytes(int64_t T, int H, int64_t total_max) {
+  size_t b = attn_partials_bytes(T, H, attn_split(T, total_max, H).n);
+  if (g_batch_invariant.load(std::memory_order_relaxed)) {
+    const size_t bi = attn_partials_bytes(T, H, attn_split_invariant(total_max).n);
+    if (bi > b) b = bi;
+  }
+  return b;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -201,6 +220,13 @@ csa_status_t csa_set_attention_kernel(int32_t choice) {
   if (choice < 0 || choice > 2)
     return fail(CSA_ERR_INVALID_ARG, "csa_set_attention_kernel: choice %d out of range", choice);
   g_attn_kernel.store(choice, std::memory_order_relaxed);
+  return CSA_OK;
+}
+
+csa_status_t csa_set_batch_invariant(int32_t on) {
+  if (on != 0 && on != 1)
+    return fail(CSA_ERR_INVALID_ARG, "csa_set_batch_invariant: on must be 0 or 1, got %d", on);
+  g_batch_invariant.store(on, std::memory_order_relaxed);
   return CSA_OK;
 }
 
@@ -472,10 +498,13 @@ csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_com
   a.out = (__nv_bfloat16*)out;
   a.lse = lse;
   const Split sp_ws = attn_split(B, (int64_t)top_k + window, H);
-  const size_t need = sp_ws.n == 1 ? kWsHeader : attn_ws_bytes(B, H, (int64_t)top_k + window);
-  if ((st = check_ws(ws, ws_bytes, need, name)) != CSA_OK) return st;
+  const bool invariant = g_batch_invariant.load(std::memory_order_relaxed) != 0;
+  const Split sp_inv = attn_split_invariant((int64_t)top_k + window);
+  const int n_need = invariant && sp_inv.n > sp_ws.n ? sp_inv.n : sp_ws.n;
+  if ((st = check_ws(ws, ws_bytes, attn_partials_bytes(B, H, n_need), name)) != CSA_OK) return st;
   a.use_tc = attention_uses_tc(a);
-  const Split sp = a.use_tc ? attn_split_tc(B, (int64_t)top_k + window, H, sp_ws) : sp_ws;
+  const Split sp = invariant ? sp_inv
+                             : (a.use_tc ? attn_split_tc(B, (int64_t)top_k + window, H, sp_ws) : sp_ws);
   a.n_split = sp.n;
   a.split_len = sp.len;
   a.err = static_cast<WsHeader*>(ws);
@@ -527,10 +556,13 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
   a.out = (__nv_bfloat16*)out;
   a.lse = lse;
   const Split sp_ws = attn_split(T, max_entries + window, H);
-  const size_t need = sp_ws.n == 1 ? kWsHeader : attn_ws_bytes(T, H, max_entries + window);
-  if ((st = check_ws(ws, ws_bytes, need, name)) != CSA_OK) return st;
+  const bool invariant = win_len != nullptr && g_batch_invariant.load(std::memory_order_relaxed) != 0;
+  const Split sp_inv = attn_split_invariant(max_entries + window);
+  const int n_need = invariant && sp_inv.n > sp_ws.n ? sp_inv.n : sp_ws.n;
+  if ((st = check_ws(ws, ws_bytes, attn_partials_bytes(T, H, n_need), name)) != CSA_OK) return st;
   a.use_tc = attention_uses_tc(a);
-  const Split sp = a.use_tc ? attn_split_tc(T, max_entries + window, H, sp_ws) : sp_ws;
+  const Split sp = invariant ? sp_inv
+                             : (a.use_tc ? attn_split_tc(T, max_entries + window, H, sp_ws) : sp_ws);
   a.n_split = sp.n;
   a.split_len = sp.len;
   a.err = static_cast<WsHeader*>(ws);

@@ -105,6 +105,20 @@ csa_status_t csa_set_timing_events(int32_t kernel_id, void* ev_begin, void* ev_e
  */
 csa_status_t csa_set_attention_kernel(int32_t choice);
 
+/*
+ * Batch-invariant decode (process-wide; off by default).  When on, the split
+ * of each query's row list (selected entries, then window rows) for
+ * csa_sparse_attn_decode and for decode calls of hca_attn is fixed slices of
+ * 512 rows, merged in slice order, whatever the batch: a query's output and
+ * log-sum-exp are then bit-identical whether it is decoded alone or in any
+ * batch, at some cost in speed for small batches.  The decode and HCA
+ * workspace-size queries account for the mode in force when they are called.
+ * DeepSeek-V4 infrastructure notes, "batch invariance": split-KV decoding
+ * otherwise makes the accumulation order, and so the bits, depend on the
+ * batch.  Returns CSA_ERR_INVALID_ARG unless `on` is 0 or 1.
+ */
+csa_status_t csa_set_batch_invariant(int32_t on);
+
 /* ---- workspace ------------------------------------------------------------ */
 /*
  * Calls that take `ws` need a caller-allocated device workspace of at least

@@ -126,6 +126,19 @@ def test_attention_kernel_choice_validation(lib):
         assert lib.csa_set_attention_kernel(choice) == 0
 
 
+def test_batch_invariant_mode_validation_and_sizing(lib):
+    assert lib.csa_set_batch_invariant(2) == 1 and b"0 or 1" in lib.csa_last_error()
+    # B=400 queries fill the GPU without splitting; fixed 512-row slices need partials
+    plain = lib.csa_sparse_attn_decode_workspace_size(400, 64, 128, 2048, 128)
+    assert lib.csa_set_batch_invariant(1) == 0
+    try:
+        inv = lib.csa_sparse_attn_decode_workspace_size(400, 64, 128, 2048, 128)
+    finally:
+        assert lib.csa_set_batch_invariant(0) == 0
+    n = (2048 + 128 + 511) // 512
+    assert inv >= 400 * n * 64 * (128 + 2) * 4 > plain
+
+
 def test_product_path_does_not_import_the_oracle():
     """The package and the bench's timed path never touch oracle/."""
     pkg = os.path.join(ROOT, "compressed_sparse_kv_03_b200")

@@ -337,3 +337,92 @@ def test_decode_is_deterministic():
     i1, o1 = run()
     i2, o2 = run()
     assert torch.equal(i1, i2) and torch.equal(o1, o2)
+
+
+@pytest.mark.usefixtures("attn_kernel")
+@pytest.mark.parametrize("paged", [False, True])
+def test_batch_invariant_decode(paged):
+    """In batch-invariant mode a sequence's decode step (indexer, top-k and
+    attention) gives the same bits alone, in the full batch and in a
+    reordered sub-batch; the outputs still match the oracle."""
+    csa = _csa()
+    g = synth.generator(120 + int(paged))
+    B, H, k, W, m = 6, 64, 300, 128, 4
+    S = [900 + 517 * b for b in range(B)]
+    q = synth.normal(g, (B, H, 128))
+    qI = synth.normal(g, (B, 8, 64))
+    w = synth.uniform(g, (B, 8))
+    win = synth.normal(g, (B, W, 128))
+    win_len = torch.tensor([W, 40, 1, W, 77, W], dtype=torch.int32)
+    pos = torch.tensor([s * m + 3 for s in S], dtype=torch.int64)
+    if paged:
+        pool, table = synth.paged_pool(g, S, 128, 64)
+        kpool = synth.normal(g, (pool.shape[0], 64))
+        cache = lambda sel: csa.Cache(dev(pool), page_table=dev(table[sel]), page_size=64)
+        kcache = lambda sel: csa.Cache(dev(kpool), page_table=dev(table[sel]), page_size=64)
+        logical = lambda b: f64(synth.unpage(pool, table[b], S[b], 64))
+    else:
+        kvc, kI = synth.normal(g, (B, max(S), 128)), synth.normal(g, (B, max(S), 64))
+        cache = lambda sel: csa.Cache.contiguous(dev(kvc[sel]))
+        kcache = lambda sel: csa.Cache.contiguous(dev(kI[sel]))
+        logical = lambda b: f64(kvc[b])
+    lam = 1 / math.sqrt(128)
+
+    def step(sel):
+        n = len(sel)
+        idx, cnt = csa.indexer_topk(dev(qI[sel]), dev(w[sel]), kcache(sel), m, k,
+                                    seq_id=torch.arange(n, dtype=torch.int32, device="cuda"),
+                                    q_pos=dev(pos[sel]), max_entries=max(S))
+        out, lse = csa.sparse_attn_decode(dev(q[sel]), cache(sel), dev(win[sel]), dev(win_len[sel]),
+                                          idx, cnt, lam, return_lse=True)
+        return idx.cpu(), out.cpu(), lse.cpu()
+
+    csa.set_batch_invariant(True)
+    try:
+        full = step(list(range(B)))
+        subsets = [[b] for b in range(B)] + [[4, 1, 3]]
+        for sel in subsets:
+            part = step(sel)
+            for j, b in enumerate(sel):
+                assert torch.equal(part[0][j], full[0][b]), ("idx", sel, b)
+                assert torch.equal(part[1][j], full[1][b]), ("out", sel, b)
+                assert torch.equal(part[2][j], full[2][b]), ("lse", sel, b)
+    finally:
+        csa.set_batch_invariant(False)
+    idx, out = full[0], f64(full[1])
+    for b in range(B):
+        c = int((idx[b] >= 0).sum())
+        rows = np.concatenate([logical(b)[idx[b, :c].numpy()], f64(win[b, :win_len[b]])])
+        ref, _ = oracle.attend_shared_kv(f64(q[b]), rows, lam)
+        assert_close_attn(out[b], ref, f"batch-invariant decode seq {b}")
+
+
+@pytest.mark.usefixtures("attn_kernel")
+def test_batch_invariant_hca_decode():
+    csa = _csa()
+    g = synth.generator(125)
+    B, H, m, W = 5, 64, 16, 128
+    pos = torch.tensor([20000, 130, 9000, 4097, 16], dtype=torch.int64)
+    S = [int(p) // m for p in pos]
+    q = synth.normal(g, (B, H, 128))
+    kvc = synth.normal(g, (B, max(S), 128))
+    win = synth.normal(g, (B, W, 128))
+    win_len = torch.clamp(pos + 1, max=W).to(torch.int32)
+    lam = 1 / math.sqrt(128)
+
+    def step(sel):
+        return csa.hca_attn(dev(q[sel]), csa.Cache.contiguous(dev(kvc[sel])), dev(win[sel]), m, W, lam,
+                            win_len=dev(win_len[sel]), q_pos=dev(pos[sel]), max_entries=max(S)).cpu()
+
+    csa.set_batch_invariant(True)
+    try:
+        full = step(list(range(B)))
+        for sel in [[b] for b in range(B)] + [[3, 0]]:
+            part = step(sel)
+            for j, b in enumerate(sel):
+                assert torch.equal(part[j], full[b]), (sel, b)
+    finally:
+        csa.set_batch_invariant(False)
+    ref, _ = oracle.hca_decode(f64(q), LazySeq(lambda b: f64(kvc[b])), f64(win), win_len.numpy(),
+                               pos.numpy(), m, lam)
+    assert_close_attn(full, ref, "batch-invariant hca decode")

@@ -377,6 +377,349 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
   if (warp == 1) tc::tmem_dealloc(tmem_base, kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// Many-query mode: every query reads the same sequence (prefill), so a block
+// of QB = 128 / H_I consecutive queries shares each key tile.  The block's
+// (query, head) rows fill the MMA N side (128), keys the M side: one 256-key
+// item is two 128 x 128 x 64 products into 256 TMEM columns, 16x fewer key
+// reads per score than the one-query decode mode.  The epilogue thread owns
+// a key and sums the ReLU-weighted heads of each query of the block from its
+// own TMEM row, so no cross-thread reduction is needed.  Items (block, chunk)
+// follow the same hybrid static / work-counter schedule as decode mode.
+// ---------------------------------------------------------------------------
+constexpr int kPStages = 4;
+constexpr int kPQTileBytes = 128 * 128;                  // 128 rows x 64 bf16
+constexpr int kPStageBytes = kStageKeyBytes + kPQTileBytes;
+constexpr int kPAcc = 2;                                 // one per epilogue group
+constexpr int kPTmemCols = 512;
+constexpr uint32_t kPIdesc = tc::idesc_bf16(128, 128);
+constexpr int kMaxBlocks = 2048;
+constexpr int kPRing = 16;
+constexpr int kPEpiWarps = 16;                 // four groups: (item parity, key tile)
+constexpr int kPThreads = (2 + kPEpiWarps) * 32;
+
+struct __align__(16) BlockMeta {
+  float w[128];       // the block's head weights in (query, head) order
+  int32_t nel[32];    // eligible entries of each of the block's queries (0 past the chunk)
+  int32_t b, chunk, pad0, pad1;
+};
+
+template <bool HIST, int HI>
+__global__ void __launch_bounds__(kPThreads, 1)
+indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
+                                const __grid_constant__ CUtensorMap tmap_q, TcIndexerParams p) {
+  const IndexerArgs& a = p.a;
+  const int T = (int)p.t_count;
+  constexpr int QB = 128 / HI;
+  const int NB = (T + QB - 1) / QB;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kPStages], empty_bar[kPStages];
+  __shared__ __align__(8) uint64_t tfull_bar[kPAcc], tempty_bar[kPAcc];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int32_t prefix[kMaxBlocks + 1];
+  __shared__ BlockMeta ring[kPRing];
+  __shared__ __align__(8) uint64_t ring_full[kPRing], ring_empty[kPRing];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;   // kPStages x (32 + 16) KB
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPStages; ++i) {
+      mbar_init(smem_u32(&full_bar[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), 1);
+    }
+    for (int i = 0; i < kPAcc; ++i) {
+      mbar_init(smem_u32(&tfull_bar[i]), 1);
+      mbar_init(smem_u32(&tempty_bar[i]), 8);   // the two groups reading the set
+    }
+    for (int i = 0; i < kPRing; ++i) {
+      mbar_init(smem_u32(&ring_full[i]), 1);
+      mbar_init(smem_u32(&ring_empty[i]), 9);   // the MMA warp + two epilogue groups
+    }
+    mbar_fence_init();
+  }
+  // chunks per block: the most eligible entries of any of its queries
+  for (int b = threadIdx.x; b < NB; b += kPThreads) prefix[b] = 0;
+  if (warp == 1) tc::tmem_alloc(smem_u32(&tmem_base_sh), kPTmemCols);
+  __syncthreads();
+  for (int t = threadIdx.x; t < T; t += kPThreads) {
+    const int64_t pos = a.q_pos ? __ldg(a.q_pos + a.t_begin + t) : a.t_begin + t;
+    if (pos / a.m > a.max_entries && blockIdx.x == 0)
+      report(a.err, kErrEligible, (int32_t)(a.t_begin + t), pos / a.m);
+    const int64_t n = eligible(a, a.t_begin + t);
+    atomicMax(&prefix[t / QB], (int32_t)((n + kItemRows - 1) / kItemRows));
+  }
+  __syncthreads();
+  if (warp == 0) {   // exclusive prefix over the blocks
+    const int per = (NB + 31) / 32;
+    const int b0 = lane * per, b1 = min(NB, b0 + per);
+    int32_t sum = 0;
+    for (int b = b0; b < b1; ++b) sum += prefix[b];
+    int32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int32_t run = incl - sum;
+    for (int b = b0; b < b1; ++b) {
+      const int32_t c = prefix[b];
+      prefix[b] = run;
+      run += c;
+    }
+    if (lane == 31) prefix[NB] = incl;
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = tmem_base_sh;
+  const int32_t V = prefix[NB];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    // The whole warp: lane 0 takes items, waits and issues the copies; the
+    // lanes fill the ring entry together (one float4 of weights and at most
+    // one query length each).
+    if (lane == 0) {
+      tc::prefetch_tmap(&tmap_keys);
+      tc::prefetch_tmap(&tmap_q);
+    }
+    int64_t issued = 0;
+    bool ok = true;
+    const int32_t Vs = (int32_t)((int64_t)V * kStaticPct / 100);
+    const int32_t s_lo = (int32_t)((int64_t)Vs * blockIdx.x / gridDim.x);
+    const int32_t s_hi = (int32_t)((int64_t)Vs * (blockIdx.x + 1) / gridDim.x);
+    int32_t g_next = 0;
+    if (lane == 0) g_next = s_lo < s_hi ? s_lo : Vs + (int32_t)atomicAdd(a.work, (uint32_t)kGrab);
+    bool in_static = s_lo < s_hi;
+    int32_t nxt = 0, lim = 0;
+    int bq = 0, bq_meta = -1;
+    // lane 0's view of the item sequence (the other lanes receive it by shuffle)
+    auto take = [&]() -> int32_t {
+      if (nxt >= lim) {
+        if (g_next >= V) return -1;
+        nxt = g_next;
+        if (in_static) {
+          lim = s_hi;
+          in_static = false;
+        } else {
+          lim = g_next + kGrab < V ? g_next + kGrab : V;
+        }
+        g_next = Vs + (int32_t)atomicAdd(a.work, (uint32_t)kGrab);
+        int l = 0, r = NB;   // the block: last bq with prefix[bq] <= nxt
+        while (r - l > 1) {
+          const int mid = (l + r) >> 1;
+          if (prefix[mid] <= nxt) l = mid; else r = mid;
+        }
+        bq = l;
+      }
+      while (prefix[bq + 1] <= nxt) ++bq;
+      return nxt++;
+    };
+    for (;;) {
+      int32_t item = -1;
+      if (lane == 0) item = take();
+      item = __shfl_sync(0xffffffffu, item, 0);
+      const int b_now = __shfl_sync(0xffffffffu, bq, 0);
+      if (item < 0) break;
+      const int32_t chunk = item - prefix[b_now];
+      const int64_t t0 = (int64_t)b_now * QB;           // first query of the block (chunk-local)
+      const int64_t s0 = (int64_t)chunk * kItemRows;
+      const int rs = (int)(issued % kPRing);
+      bool got = true;
+      if (lane == 0) got = mbar_wait(smem_u32(&ring_empty[rs]), (uint32_t)(((issued / kPRing) & 1) ^ 1));
+      __syncwarp();
+      if (!__shfl_sync(0xffffffffu, got, 0)) {
+        if (lane == 0) report(a.err, kErrTimeout, (int32_t)(a.t_begin + t0), 16);
+        ok = false;
+        break;
+      }
+      BlockMeta& mt = ring[rs];
+      const int64_t nq = T - t0 < QB ? T - t0 : QB;
+      if (b_now != bq_meta) {
+        // the block's weights (128 consecutive floats, 16-byte aligned) and lengths
+        const float4* wsrc = reinterpret_cast<const float4*>(a.w + (a.t_begin + t0) * HI);
+        reinterpret_cast<float4*>(mt.w)[lane] =
+            lane * 4 < nq * HI ? __ldg(wsrc + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane < QB) mt.nel[lane] = lane < nq ? (int32_t)eligible(a, a.t_begin + t0 + lane) : 0;
+        bq_meta = b_now;
+      } else {
+        const BlockMeta& pm = ring[(issued - 1) % kPRing];
+        reinterpret_cast<float4*>(mt.w)[lane] = reinterpret_cast<const float4*>(pm.w)[lane];
+        if (lane < QB) mt.nel[lane] = pm.nel[lane];
+      }
+      if (lane == 0) {
+        mt.b = b_now;
+        mt.chunk = chunk;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ring_full[rs]));   // releases the lanes' writes (after the warp sync)
+      if (lane == 0) {
+        const int slot = (int)(issued % kPStages);
+        if (!mbar_wait(smem_u32(&empty_bar[slot]), (uint32_t)(((issued / kPStages) & 1) ^ 1))) {
+          report(a.err, kErrTimeout, (int32_t)(a.t_begin + t0), 10);
+          got = false;
+        } else {
+          const uint32_t fb = smem_u32(&full_bar[slot]);
+          const uint32_t st = base + slot * kPStageBytes;
+          mbar_arrive_expect_tx(fb, kPStageBytes);
+          if (a.keys.page_table == nullptr) {
+            tc::tma_load_2d(st, &tmap_keys, 0, (int32_t)s0, fb);
+          } else {
+#pragma unroll
+            for (int h = 0; h < kItemRows / kBoxRows; ++h) {
+              const int64_t s = s0 + h * kBoxRows;
+              const int64_t pi = s / a.keys.page_size;
+              const int32_t page = pi < a.keys.max_pages ? __ldg(a.keys.page_table + pi) : -1;
+              int64_t row = (int64_t)page * a.keys.page_size + (s - pi * a.keys.page_size);
+              if (page < 0 || row >= a.keys.n_rows) {
+                if (s < mt.nel[0] || s < mt.nel[QB - 1]) report(a.err, kErrPageId, (int32_t)(a.t_begin + t0), page);
+                row = 0;
+              }
+              tc::tma_load_2d(st + h * kBoxRows * 128, &tmap_keys, 0, (int32_t)row, fb);
+            }
+          }
+          tc::tma_load_2d(st + kStageKeyBytes, &tmap_q, 0, (int32_t)((a.t_begin + t0) * HI), fb);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, got, 0)) {
+        ok = false;
+        break;
+      }
+      ++issued;
+    }
+    if (lane == 0) {
+      for (int e = 0; ok && e < 2; ++e) {   // end markers, as in decode mode
+        const int64_t j = issued + e;
+        const int rs = (int)(j % kPRing);
+        if (!mbar_wait(smem_u32(&ring_empty[rs]), (uint32_t)(((j / kPRing) & 1) ^ 1))) {
+          report(a.err, kErrTimeout, 0, 17);
+          break;
+        }
+        ring[rs].b = -1;
+        mbar_arrive(smem_u32(&ring_full[rs]));
+      }
+      const int64_t first = issued > kPStages ? issued - kPStages : 0;
+      for (int64_t d = first; d < issued; ++d)
+        mbar_wait(smem_u32(&full_bar[d % kPStages]), (uint32_t)((d / kPStages) & 1), 200000000ll);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      for (int64_t j = 0;; ++j) {
+        const int rs = (int)(j % kPRing);
+        if (!mbar_wait(smem_u32(&ring_full[rs]), (uint32_t)((j / kPRing) & 1))) {
+          report(a.err, kErrTimeout, (int32_t)j, 18);
+          break;
+        }
+        const bool end = ring[rs].b < 0;
+        mbar_arrive(smem_u32(&ring_empty[rs]));
+        if (end) break;
+        const int slot = (int)(j % kPStages);
+        const int acc = (int)(j % kPAcc);
+        if (!mbar_wait(smem_u32(&full_bar[slot]), (uint32_t)((j / kPStages) & 1)) ||
+            !mbar_wait(smem_u32(&tempty_bar[acc]), (uint32_t)(((j / kPAcc) & 1) ^ 1))) {
+          report(a.err, kErrTimeout, (int32_t)j, 11);
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t st = base + slot * kPStageBytes;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc::mma_bf16_ss(tmem_base + acc * 256 + h * 128, tc::smem_desc_sw128(st + h * kKeyTileBytes + 32 * k),
+                            tc::smem_desc_sw128(st + kStageKeyBytes + 32 * k), kPIdesc, k > 0);
+        }
+        tc::mma_commit(smem_u32(&empty_bar[slot]));
+        tc::mma_commit(smem_u32(&tfull_bar[acc]));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int eg = (warp - 2) >> 2;            // 0..3
+    const int group = eg >> 1;                 // items j with j % 2 == group, accumulator set `group`
+    const int h = eg & 1;                      // the key tile of the item this group scores
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;       // key within a 128-key tile
+    constexpr int qpc = 32 / HI;               // queries per 32 TMEM columns
+    for (int64_t j = group;; j += 2) {
+      const int rs = (int)(j % kPRing);
+      if (!mbar_wait(smem_u32(&ring_full[rs]), (uint32_t)((j / kPRing) & 1))) {
+        if (lane == 0) report(a.err, kErrTimeout, (int32_t)j, 19);
+        break;
+      }
+      const BlockMeta& mt = ring[rs];
+      const int bq = mt.b;
+      if (bq < 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ring_empty[rs]));
+        break;
+      }
+      const int acc = group;
+      if (!mbar_wait(smem_u32(&tfull_bar[acc]), (uint32_t)((j / kPAcc) & 1))) {
+        if (lane == 0) report(a.err, kErrTimeout, (int32_t)j, 13);
+        break;
+      }
+      tc::fence_after_sync();
+      const int64_t s0 = (int64_t)mt.chunk * kItemRows;
+      const int64_t t0 = (int64_t)bq * QB;
+      {
+        const int64_t s = s0 + h * kTileRows + row;
+        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * 256 + h * 128;
+#pragma unroll 2
+        for (int c = 0; c < 4; ++c) {   // 32 (query, head) columns at a time
+          uint32_t r0[16], r1[16];
+          tc::tmem_ld16(taddr + c * 32, r0);
+          tc::tmem_ld16(taddr + c * 32 + 16, r1);
+          tc::tmem_wait_ld();
+          float x[32], wq[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            x[i] = fmaxf(__uint_as_float(r0[i]), 0.f);
+            x[16 + i] = fmaxf(__uint_as_float(r1[i]), 0.f);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {   // this chunk's 32 head weights
+            const float4 w4 = *reinterpret_cast<const float4*>(&mt.w[c * 32 + i]);
+            wq[i] = w4.x;
+            wq[i + 1] = w4.y;
+            wq[i + 2] = w4.z;
+            wq[i + 3] = w4.w;
+          }
+#pragma unroll
+          for (int qq = 0; qq < qpc; ++qq) {
+            const int q = c * qpc + qq;
+            float sc = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < HI; ++hh) sc = fmaf(wq[qq * HI + hh], x[qq * HI + hh], sc);
+            const bool valid = s < mt.nel[q];
+            const uint32_t key = score_key(sc);
+            const int64_t tl = t0 + q;
+            if (valid) a.keys_out[tl * a.key_stride + s] = key;
+            if (HIST) {
+              const uint32_t bin = valid ? key >> 20 : 0xffffffffu;
+              const uint32_t same = __match_any_sync(0xffffffffu, bin);
+              if (valid && lane == __ffs(same) - 1)
+                atomicAdd(a.hist + tl * kHistBins + bin, (uint32_t)__popc(same));
+            }
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&tempty_bar[acc]));
+        mbar_arrive(smem_u32(&ring_empty[rs]));
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem_base, kPTmemCols);
+}
+
 }  // namespace
 
 bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count) {
@@ -386,6 +729,50 @@ bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count) {
   if (a.keys.n_rows > INT32_MAX || a.T * a.H_I > INT32_MAX) return false;
   if (a.work == nullptr) return false;
   return true;
+}
+
+bool tc_indexer_prefill_supported(const IndexerArgs& a, int64_t t_count) {
+  if (a.seq_id != nullptr || a.c_I != 64 || a.work == nullptr) return false;
+  if (a.H_I != 4 && a.H_I != 8 && a.H_I != 16) return false;
+  // the producer reads a block's 128 head weights as 32 aligned float4
+  if ((reinterpret_cast<uintptr_t>(a.w) & 15u) != 0 || ((a.t_begin * a.H_I) & 3) != 0) return false;
+  const int64_t qb = 128 / a.H_I;
+  const int64_t nb = (t_count + qb - 1) / qb;
+  if (nb > kMaxBlocks || (a.max_entries + kItemRows - 1) / kItemRows * nb > INT32_MAX) return false;
+  if (a.keys.page_table != nullptr && a.keys.page_size % kBoxRows != 0) return false;
+  if (a.keys.n_rows > INT32_MAX || a.T * a.H_I > INT32_MAX) return false;
+  return true;
+}
+
+cudaError_t launch_indexer_scores_tc_prefill(const Launch& L, const IndexerArgs& a, int64_t t_count) {
+  CUtensorMap tk, tq;
+  const uint32_t box_rows = a.keys.page_table == nullptr ? kItemRows : kBoxRows;
+  if (!make_tmap_bf16_2d(&tk, a.keys.data, 64, (uint64_t)a.keys.n_rows, 64, 64, box_rows))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tq, a.q_idx, 64, (uint64_t)(a.T * a.H_I), 64, 64, 128))
+    return cudaErrorInvalidValue;
+  TcIndexerParams p;
+  p.a = a;
+  p.t_count = t_count;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int smem = kPStages * kPStageBytes + 1024;
+  L.begin(kKernelIndexerScore);
+#define CSA_PREFILL_CASE(H_, HIST_)                                                               \
+  if (a.H_I == H_ && (a.hist != nullptr) == HIST_) {                                               \
+    cudaFuncSetAttribute(indexer_score_tc_prefill_kernel<HIST_, H_>,                               \
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                       \
+    indexer_score_tc_prefill_kernel<HIST_, H_><<<(unsigned)sms, kPThreads, smem, L.stream>>>(tk, tq, p); \
+  }
+  CSA_PREFILL_CASE(4, false)
+  CSA_PREFILL_CASE(8, false)
+  CSA_PREFILL_CASE(16, false)
+  CSA_PREFILL_CASE(4, true)
+  CSA_PREFILL_CASE(8, true)
+  CSA_PREFILL_CASE(16, true)
+#undef CSA_PREFILL_CASE
+  return L.end(kKernelIndexerScore);
 }
 
 cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int64_t t_count) {

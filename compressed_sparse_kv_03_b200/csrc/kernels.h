@@ -57,6 +57,10 @@ cudaError_t launch_indexer_scores(const Launch& L, const IndexerArgs& a, int64_t
 // tcgen05 + TMA scoring path (c_I = 64, H_I <= 16, pages a multiple of 64 rows)
 bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count);
 cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int64_t t_count);
+// tcgen05 many-query path: all queries on one sequence (seq_id null), c_I = 64,
+// H_I in {4, 8, 16}; blocks of 128 / H_I queries share each key tile
+bool tc_indexer_prefill_supported(const IndexerArgs& a, int64_t t_count);
+cudaError_t launch_indexer_scores_tc_prefill(const Launch& L, const IndexerArgs& a, int64_t t_count);
 
 struct SelectArgs {
   const uint32_t* keys;         // [T_chunk, key_stride]

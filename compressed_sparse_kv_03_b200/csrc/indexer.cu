@@ -459,6 +459,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_bitmap_kernel(SelectA
 // many-query (prefill) selection: radix select over keys in shared memory
 // ---------------------------------------------------------------------------
 constexpr int kBins = 2048;
+constexpr int64_t kCommonPrefixMin = 8192;   // list length from which the common prefix is found first
 
 __global__ void __launch_bounds__(kSelThreads) topk_select_radix_kernel(SelectArgs a) {
   extern __shared__ uint32_t skeys[];
@@ -484,26 +485,67 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_radix_kernel(SelectAr
     if (threadIdx.x == 0) a.count_out[t] = (int32_t)n;
     return;
   }
-  for (int64_t j = threadIdx.x; j < n; j += kSelThreads) skeys[j] = keys[j];
+  {
+    // whole 16-byte vectors (rows are 256-byte aligned), several loads in flight
+    const int64_t nv = (n + 3) >> 2;
+    const uint4* kv = reinterpret_cast<const uint4*>(keys);
+    uint4* sv = reinterpret_cast<uint4*>(skeys);
+#pragma unroll 4
+    for (int64_t v = threadIdx.x; v < nv; v += kSelThreads) sv[v] = kv[v];
+  }
   __syncthreads();
 
-  uint32_t prefix = 0, mask = 0;
+  // the keys' common leading bits first (a min / max reduction), so that the
+  // first radix digit spreads the keys instead of piling them into the few
+  // bins of one exponent range; short lists skip it (it would cost more
+  // than the atomics it saves)
+  uint32_t kmin = 0u, kmax = 0xffffffffu;   // no common prefix assumed
+  if (n >= kCommonPrefixMin) {                // uniform over the block
+    kmin = 0xffffffffu;
+    kmax = 0u;
+    for (int64_t j = threadIdx.x; j < n; j += kSelThreads) {
+      const uint32_t key = skeys[j];
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    __shared__ uint32_t s_min[32], s_max[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) {
+      s_min[warp] = kmin;
+      s_max[warp] = kmax;
+    }
+    __syncthreads();
+    kmin = lane < kSelThreads / 32 ? s_min[lane] : 0xffffffffu;
+    kmax = lane < kSelThreads / 32 ? s_max[lane] : 0u;
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+  }
+  const int cpl = __clz(kmin ^ kmax);   // 32 when every key is equal
+  uint32_t mask = cpl >= 32 ? 0xffffffffu : ~(0xffffffffu >> cpl);
+  uint32_t prefix = kmin & mask;
   int remaining = k;
-  const int shifts[3] = {21, 10, 0};
-  const uint32_t digit_mask[3] = {0x7ffu, 0x7ffu, 0x3ffu};
+  int shift = 32 - cpl;   // bits below `shift` are still open
 #pragma unroll 1
-  for (int p = 0; p < 3; ++p) {
-    for (int b = threadIdx.x; b < kBins; b += kSelThreads) hist[b] = 0;
+  while (shift > 0) {
+    // an 11-bit digit; the last one is widened to 10 bits (find_bin takes
+    // whole multiples of the block size), its upper bits then already fixed
+    const int lo = shift > 11 ? shift - 11 : 0;
+    const int dig = shift - lo >= 10 ? shift - lo : 10;
+    const uint32_t dmask = (1u << dig) - 1u;
+    for (int b = threadIdx.x; b < (1 << dig); b += kSelThreads) hist[b] = 0;
     __syncthreads();
     for (int64_t j = threadIdx.x; j < n; j += kSelThreads) {
       const uint32_t key = skeys[j];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shifts[p]) & digit_mask[p]], 1);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> lo) & dmask], 1);
     }
     __syncthreads();
-    find_bin(hist, kBins, remaining, warp_sums, &s_bin, &s_above, &s_ok);
-    prefix |= s_bin << shifts[p];
-    mask |= digit_mask[p] << shifts[p];
+    find_bin(hist, 1 << dig, remaining, warp_sums, &s_bin, &s_above, &s_ok);
+    prefix |= s_bin << lo;
+    mask |= dmask << lo;
     remaining -= s_above;
+    shift = lo;
     __syncthreads();
   }
   const uint32_t kth = prefix;
@@ -614,7 +656,7 @@ cudaError_t launch_topk_select(const Launch& L, const SelectArgs& a, int64_t t_c
                          (2 * kCandCap + 2 * (int)(kBitmapSelectMaxEntries / 32)) * (int)sizeof(uint32_t));
     topk_select_bitmap_kernel<<<(unsigned)t_count, kSelThreads, bytes, L.stream>>>(a);
   } else {
-    const size_t bytes = (size_t)a.max_entries * sizeof(uint32_t);
+    const size_t bytes = (size_t)((a.max_entries + 3) & ~int64_t(3)) * sizeof(uint32_t);   // whole uint4 stores
     cudaFuncSetAttribute(topk_select_radix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kRadixSelectMaxEntries * (int)sizeof(uint32_t));
     topk_select_radix_kernel<<<(unsigned)t_count, kSelThreads, bytes, L.stream>>>(a);

@@ -137,6 +137,50 @@ def compress_kv(C_a, Z_a, m, *, C_b=None, Z_b=None, bias=None, overlap=False, ou
     return out
 
 
+@dataclass
+class AppendState:
+    """Per-sequence decode-time cache state for `cache_append`: the unfinished
+    block's a-branch rows, the b-branch rows by block parity (overlap mode) and
+    the window ring."""
+    blk_c: torch.Tensor
+    blk_z: torch.Tensor
+    bb_c: Optional[torch.Tensor]
+    bb_z: Optional[torch.Tensor]
+    win: Optional[torch.Tensor]
+
+    @staticmethod
+    def new(B, dim, m, window, overlap, device="cuda"):
+        z = lambda *shape: torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        return AppendState(z(B, m, dim), z(B, m, dim), z(B, 2, m, dim) if overlap else None,
+                           z(B, 2, m, dim) if overlap else None,
+                           z(B, window, dim) if window > 0 else None)
+
+
+def cache_append(C_a, Z_a, pos, cache: Cache, m, state: AppendState, max_entries, *, C_b=None,
+                 Z_b=None, bias=None, overlap=False, ws=None, stream=None):
+    """Decode-time cache maintenance: append one token per sequence (C_a, Z_a
+    [B, dim] at positions pos [B]); every m-th token completes a block, whose
+    entry is written into `cache`.  `state` persists between calls."""
+    _need(C_a, "C_a", torch.bfloat16, 2)
+    dev = C_a.device
+    B, dim = C_a.shape
+    _need(Z_a, "Z_a", torch.bfloat16, 2, dev)
+    _need(pos, "pos", torch.int64, 1, dev)
+    for name, t in (("C_b", C_b), ("Z_b", Z_b)):
+        if t is not None:
+            _need(t, name, torch.bfloat16, 2, dev)
+    if bias is not None:
+        _need(bias, "bias", torch.float32, None, dev)
+    window = state.win.shape[1] if state.win is not None else 0
+    lib = load()
+    wsp, wsb = _ws(ws, dev).get(256)
+    kc = cache.c()
+    check(lib.csa_cache_append(_ptr(C_a), _ptr(Z_a), _ptr(C_b), _ptr(Z_b), _ptr(bias), _ptr(pos), B,
+                               dim, m, int(bool(overlap)), _ptr(state.blk_c), _ptr(state.blk_z),
+                               _ptr(state.bb_c), _ptr(state.bb_z), _ptr(state.win), window,
+                               C.byref(kc), max_entries, wsp, wsb, _stream(stream)))
+
+
 def indexer_topk(q_idx, w, keys: Cache, m, top_k, *, seq_id=None, q_pos=None, max_entries=None,
                  return_scores=False, ws=None, stream=None, out=None):
     """Steps 2-3: lightning-indexer scores and exact top-k per query.

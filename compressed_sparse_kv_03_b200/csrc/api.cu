@@ -316,6 +316,55 @@ csa_status_t csa_compress_kv(const csa_bf16* C_a, const csa_bf16* Z_a, const csa
       "csa_compress_kv launch");
 }
 
+csa_status_t csa_cache_append(const csa_bf16* C_a, const csa_bf16* Z_a, const csa_bf16* C_b,
+                              const csa_bf16* Z_b, const float* bias, const int64_t* pos,
+                              int32_t B, int32_t dim, int32_t m, int32_t overlap,
+                              csa_bf16* blk_c, csa_bf16* blk_z, csa_bf16* bb_c, csa_bf16* bb_z,
+                              csa_bf16* win, int32_t window, const csa_cache_t* cache,
+                              int64_t max_entries, void* ws, size_t ws_bytes, csa_stream_t stream) {
+  const char* name = "csa_cache_append";
+  if (B < 0 || m < 1 || dim < 8 || dim % 8 != 0 || dim > 2048 || window < 0 || max_entries < 0 ||
+      (overlap != 0 && overlap != 1))
+    return fail(CSA_ERR_INVALID_ARG,
+                "%s: need B >= 0, m >= 1, dim a multiple of 8 in [8, 2048], window >= 0, "
+                "max_entries >= 0, overlap in {0,1}", name);
+  if (B == 0) return CSA_OK;
+  if (C_a == nullptr || Z_a == nullptr || pos == nullptr || blk_c == nullptr || blk_z == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "%s: C_a, Z_a, pos, blk_c and blk_z are required", name);
+  if (overlap && (bb_c == nullptr || bb_z == nullptr))
+    return fail(CSA_ERR_INVALID_ARG, "%s: overlap mode needs bb_c and bb_z", name);
+  if (window > 0 && win == nullptr) return fail(CSA_ERR_INVALID_ARG, "%s: window > 0 needs win", name);
+  csa_status_t st = check_cache(cache, name);
+  if (st != CSA_OK) return st;
+  if (!aligned16(C_a) || !aligned16(Z_a) || (C_b && !aligned16(C_b)) || (Z_b && !aligned16(Z_b)) ||
+      (bias && !aligned16(bias)) || !aligned16(blk_c) || !aligned16(blk_z) ||
+      (bb_c && !aligned16(bb_c)) || (bb_z && !aligned16(bb_z)) || (win && !aligned16(win)))
+    return fail(CSA_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", name);
+  if ((st = check_ws(ws, ws_bytes, kWsHeader, name)) != CSA_OK) return st;
+  CacheAppendArgs a{};
+  a.Ca = (const __nv_bfloat16*)C_a;
+  a.Za = (const __nv_bfloat16*)Z_a;
+  a.Cb = (const __nv_bfloat16*)C_b;
+  a.Zb = (const __nv_bfloat16*)Z_b;
+  a.bias = bias;
+  a.pos = pos;
+  a.B = B;
+  a.dim = dim;
+  a.m = m;
+  a.overlap = overlap;
+  a.blk_c = (__nv_bfloat16*)blk_c;
+  a.blk_z = (__nv_bfloat16*)blk_z;
+  a.bb_c = (__nv_bfloat16*)bb_c;
+  a.bb_z = (__nv_bfloat16*)bb_z;
+  a.win = (__nv_bfloat16*)win;
+  a.window = window;
+  a.cache = to_ref(cache);
+  a.max_entries = max_entries;
+  a.err = static_cast<WsHeader*>(ws);
+  Launch L{(cudaStream_t)stream};
+  return cuda_status(launch_cache_append(L, a), "csa_cache_append launch");
+}
+
 // ---- steps 2-3 ---------------------------------------------------------------
 csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_cache_t* k_idx,
                               const int32_t* seq_id, const int64_t* q_pos, int64_t T,

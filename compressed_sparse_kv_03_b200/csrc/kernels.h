@@ -25,6 +25,22 @@ cudaError_t launch_compress(const Launch& L, const __nv_bfloat16* Ca, const __nv
                             const __nv_bfloat16* Cb, const __nv_bfloat16* Zb, const float* bias,
                             int64_t n_tokens, int dim, int m, int overlap, __nv_bfloat16* out);
 
+// Decode-time cache append (one token per sequence): see cache.cu.
+struct CacheAppendArgs {
+  const __nv_bfloat16 *Ca, *Za, *Cb, *Zb;   // [B, dim] the new tokens (Cb / Zb null: Ca / Za)
+  const float* bias;                         // [m, dim] or [2, m, dim] or null
+  const int64_t* pos;                        // [B] position t of each new token
+  int B, dim, m, overlap;
+  __nv_bfloat16 *blk_c, *blk_z;              // [B, m, dim] the unfinished block's a-branch rows
+  __nv_bfloat16 *bb_c, *bb_z;                // [B, 2, m, dim] b-branch rows by block parity (overlap)
+  __nv_bfloat16* win;                        // [B, window, dim] ring of raw rows, slot t mod window
+  int window;
+  CacheRef cache;                            // compressed entries, written at entry t / m
+  int64_t max_entries;
+  WsHeader* err;
+};
+cudaError_t launch_cache_append(const Launch& L, const CacheAppendArgs& a);
+
 // Indexer scratch limits.  Few-query (decode) mode keeps a 4096-bin histogram
 // of the top 12 score-key bits per query and selects through a bitmap in
 // shared memory; many-query (prefill) mode holds a query's keys in shared

@@ -165,6 +165,42 @@ csa_status_t csa_compress_kv(const csa_bf16* C_a, const csa_bf16* Z_a, const csa
                              int32_t dim, int32_t m, int32_t overlap, csa_bf16* out,
                              csa_stream_t stream);
 
+/*
+ * csa_cache_append -- decode-time cache maintenance, one new token per
+ * sequence (Book Ch.5 "Decode-time cache state"; Ch.8 "Quantization scales
+ * and bounded tail buffers").  For sequence b, with t = pos[b] (the number of
+ * tokens before the new one):
+ *   - its raw row C_a[b] goes to the window ring: win[b, t mod window]
+ *     (the decode attention reads the ring's first min(t+1, window) slots;
+ *     their order does not matter to the softmax);
+ *   - its a-branch rows (C_a, Z_a) go to the unfinished-block buffers at row
+ *     t mod m, and in overlap mode its b-branch rows (C_b, Z_b) to the buffer
+ *     of block parity (t / m) mod 2;
+ *   - when it completes block i = t / m (t mod m == m - 1), entry i of the
+ *     compressed cache is written: the csa_compress_kv pooling of block i
+ *     (and of block i-1's b-branch rows in overlap mode), bit for bit the
+ *     entry csa_compress_kv gives for the whole sequence.
+ * Call once per decode step, in order of t, for every sequence; the buffers
+ * are the per-sequence state and must persist between calls.
+ *   C_a, Z_a      [B, dim] bf16;  C_b, Z_b [B, dim] bf16 (overlap; NULL -> C_a / Z_a)
+ *   bias          fp32 [m, dim] or [2, m, dim] (as csa_compress_kv), or NULL
+ *   pos           int64 [B], >= 0
+ *   blk_c, blk_z  [B, m, dim] bf16 state
+ *   bb_c, bb_z    [B, 2, m, dim] bf16 state (overlap only, else NULL)
+ *   win           [B, window, dim] bf16 ring (NULL when window == 0)
+ *   cache         compressed entries [.., dim]; sequence b's entry i at its row
+ *   max_entries   entries each sequence's cache can hold; a completed block past
+ *                 it, or a bad page id, is skipped and recorded in the workspace
+ *   ws            device workspace of at least 256 bytes (the device-check header)
+ * dim % 8 == 0, dim <= 2048; all buffers 16-byte aligned.
+ */
+csa_status_t csa_cache_append(const csa_bf16* C_a, const csa_bf16* Z_a, const csa_bf16* C_b,
+                              const csa_bf16* Z_b, const float* bias, const int64_t* pos,
+                              int32_t B, int32_t dim, int32_t m, int32_t overlap,
+                              csa_bf16* blk_c, csa_bf16* blk_z, csa_bf16* bb_c, csa_bf16* bb_z,
+                              csa_bf16* win, int32_t window, const csa_cache_t* cache,
+                              int64_t max_entries, void* ws, size_t ws_bytes, csa_stream_t stream);
+
 /* ---- steps 2-3: lightning indexer + top-k ---------------------------------- */
 /*
  * csa_indexer_topk -- for every query i at position t_i of sequence b_i:

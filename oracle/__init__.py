@@ -13,6 +13,7 @@ from .csa_oracle import (  # noqa: F401
     bf16_round,
     pool_block,
     pool_overlap,
+    DecodeCacheState,
     eligible_entries,
     indexer_scores,
     topk_select,

@@ -110,6 +110,48 @@ def pool_overlap(Ca, Za, Cb, Zb, m, Ba=None, Bb=None):
     return out
 
 
+class DecodeCacheState:
+    """Decode-time cache state of one sequence (Ch.5 "Decode-time cache state";
+    Ch.8 "Quantization scales and bounded tail buffers"): the growing list of
+    compressed entries, the window of the last W raw rows, the rows of the
+    unfinished block and, in overlap mode, the b-branch rows of the last
+    completed block.  `append` takes one decode token; the entry of a block is
+    made when its last token arrives, from the block (and the previous block's
+    b-branch rows) alone, with the same pooling definition as the bulk
+    compressor."""
+
+    def __init__(self, m, W, overlap, Ba=None, Bb=None):
+        self.m, self.W, self.overlap = int(m), int(W), bool(overlap)
+        self.Ba, self.Bb = Ba, Bb
+        self.t = 0
+        self.entries = []
+        self.window = []        # raw rows, oldest first, at most W
+        self.block = []         # (c_a, z_a, c_b, z_b) of the unfinished block
+        self.prev_b = None      # (C_b rows, Z_b rows) of the last completed block
+
+    def append(self, c_a, z_a, c_b=None, z_b=None):
+        c_a, z_a = np.asarray(c_a, dtype=np.float64), np.asarray(z_a, dtype=np.float64)
+        c_b = c_a if c_b is None else np.asarray(c_b, dtype=np.float64)
+        z_b = z_a if z_b is None else np.asarray(z_b, dtype=np.float64)
+        if self.W > 0:
+            self.window = (self.window + [c_a])[-self.W:]
+        self.block.append((c_a, z_a, c_b, z_b))
+        self.t += 1
+        if len(self.block) == self.m:
+            Ca, Za, Cb, Zb = (np.stack([r[k] for r in self.block]) for k in range(4))
+            if not self.overlap:
+                self.entries.append(pool_block(Ca, Za, self.m, self.Ba)[0])
+            elif self.prev_b is None:        # block 0: no previous block
+                self.entries.append(pool_overlap(Ca, Za, Cb, Zb, self.m, self.Ba, self.Bb)[0])
+            else:                            # blocks i-1 (b branch only) and i
+                pCb, pZb = self.prev_b
+                two = lambda p, q: np.concatenate([p, q])
+                self.entries.append(pool_overlap(two(Ca, Ca), two(Za, Za), two(pCb, Cb), two(pZb, Zb),
+                                                 self.m, self.Ba, self.Bb)[1])
+            self.prev_b = (Cb, Zb)
+            self.block = []
+
+
 # ---------------------------------------------------------------------------
 # steps 2-3: lightning indexer and top-k
 # ---------------------------------------------------------------------------

@@ -81,6 +81,64 @@ def test_compress_overlap(N, dim, m, bias, separate):
     assert_close_attn(out, ref, "compress overlap")
 
 
+@pytest.mark.parametrize("overlap,paged,dim", [(True, False, 128), (False, True, 128), (True, True, 64)])
+def test_cache_append_matches_bulk_compression(overlap, paged, dim):
+    """Decode-time appends, one token per sequence per call: entry for entry the
+    bits of csa_compress_kv on the whole sequence, within tolerance of the
+    oracle's DecodeCacheState, and the window ring holds the last W raw rows."""
+    csa = _csa()
+    g = synth.generator(140 + dim + int(overlap) + 2 * int(paged))
+    B, N, m, W = 3, 37, 4, 16
+    S = N // m
+    Ca, Za, Cb, Zb = (synth.normal(g, (B, N, dim)) for _ in range(4))
+    bias = synth.normal(g, ((2, m, dim) if overlap else (m, dim)), dtype=torch.float32)
+    if paged:
+        pool, table = synth.paged_pool(g, [S + 3] * B, dim, 4)
+        cache = csa.Cache(dev(torch.zeros_like(pool)), page_table=dev(table), page_size=4)
+        read = lambda b: synth.unpage(cache.data.cpu(), table[b], S, 4)
+    else:
+        buf = torch.zeros((B, S + 3, dim), dtype=torch.bfloat16)
+        cache = csa.Cache.contiguous(dev(buf))
+        read = lambda b: cache.data.cpu().reshape(B, S + 3, dim)[b, :S]
+    st = csa.AppendState.new(B, dim, m, W, overlap)
+    ws = csa.Workspace()
+    for t in range(N):
+        pos = torch.full((B,), t, dtype=torch.int64, device="cuda")
+        csa.cache_append(dev(Ca[:, t].contiguous()), dev(Za[:, t].contiguous()), pos, cache, m, st,
+                         S + 3, C_b=dev(Cb[:, t].contiguous()) if overlap else None,
+                         Z_b=dev(Zb[:, t].contiguous()) if overlap else None, bias=dev(bias),
+                         overlap=overlap, ws=ws)
+    ws.check()
+    for b in range(B):
+        got = read(b)
+        bulk = csa.compress_kv(dev(Ca[b]), dev(Za[b]), m, C_b=dev(Cb[b]) if overlap else None,
+                               Z_b=dev(Zb[b]) if overlap else None, bias=dev(bias), overlap=overlap).cpu()
+        assert torch.equal(got, bulk), f"seq {b}: append differs from csa_compress_kv"
+        ref = oracle.DecodeCacheState(m, W, overlap, f64(bias[0] if overlap else bias),
+                                      f64(bias[1]) if overlap else None)
+        for t in range(N):
+            ref.append(f64(Ca[b, t]), f64(Za[b, t]), f64(Cb[b, t]), f64(Zb[b, t]))
+        assert_close_attn(got, np.array(ref.entries), f"cache append seq {b}")
+        ring = st.win[b].cpu()
+        for t in range(N - W, N):
+            assert torch.equal(ring[t % W], Ca[b, t]), (b, t)
+
+
+def test_cache_append_reports_full_cache():
+    """A block completed past max_entries is skipped and recorded."""
+    csa = _csa()
+    g = synth.generator(150)
+    B, dim, m = 2, 64, 2
+    cache = csa.Cache.contiguous(dev(torch.zeros((B, 1, dim), dtype=torch.bfloat16)))
+    st = csa.AppendState.new(B, dim, m, 0, False)
+    ws = csa.Workspace()
+    for t in range(4):   # blocks 0 and 1; only entry 0 fits
+        x = dev(synth.normal(g, (B, dim)))
+        csa.cache_append(x, x, torch.full((B,), t, dtype=torch.int64, device="cuda"), cache, m, st, 1, ws=ws)
+    with pytest.raises(csa.CsaError, match="device check"):
+        ws.check()
+
+
 # ---------------------------------------------------------------------------
 # steps 2-3: indexer + top-k
 # ---------------------------------------------------------------------------

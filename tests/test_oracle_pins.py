@@ -145,6 +145,49 @@ def _toy_indexer():
     return g, names, qI, KI
 
 
+@pytest.mark.parametrize("overlap", [True, False])
+def test_decode_cache_state_equals_bulk_pooling(overlap):
+    """Appending a sequence token by token (Ch.5 "Decode-time cache state")
+    yields, entry for entry, the bulk pooling of the whole sequence; one entry
+    appears every m tokens; the window holds the last W raw rows in order."""
+    rng = np.random.default_rng(31)
+    N, d, m, W = 27, 6, 4, 5
+    Ca, Za, Cb, Zb = (rng.standard_normal((N, d)) for _ in range(4))
+    Ba, Bb = rng.standard_normal((m, d)), rng.standard_normal((m, d))
+    st = oracle.DecodeCacheState(m, W, overlap, Ba, Bb if overlap else None)
+    for t in range(N):
+        st.append(Ca[t], Za[t], Cb[t], Zb[t])
+        assert len(st.entries) == (t + 1) // m
+        assert np.array_equal(np.array(st.window), Ca[max(0, t + 1 - W):t + 1])
+    ref = oracle.pool_overlap(Ca, Za, Cb, Zb, m, Ba, Bb) if overlap else oracle.pool_block(Ca, Za, m, Ba)
+    np.testing.assert_allclose(np.array(st.entries), ref, rtol=0, atol=1e-12)
+
+
+def test_decode_cache_state_entry_reads_only_its_blocks():
+    """Overlap entry i depends on tokens m(i-1) .. m(i+1)-1 only: changing any
+    other token leaves it unchanged (and changing one inside changes it)."""
+    rng = np.random.default_rng(32)
+    N, d, m = 24, 4, 4
+    X = [rng.standard_normal((N, d)) for _ in range(4)]
+
+    def entries(X):
+        st = oracle.DecodeCacheState(m, 0, True)
+        for t in range(N):
+            st.append(*(x[t] for x in X))
+        return np.array(st.entries)
+
+    base = entries(X)
+    i = 3
+    for t, same in ((m * (i - 1) - 1, True), (m * (i + 1), True), (m * (i - 1), False), (m * i + 1, False)):
+        Y = [x.copy() for x in X]
+        Y[0][t] += 1.0          # content of token t (a branch of its block, b branch of the next)
+        Y[1][t] += 1.0
+        Y[2][t] += 1.0
+        Y[3][t] += 1.0
+        changed = not np.allclose(entries(Y)[i], base[i])
+        assert changed != same, (t, same)
+
+
 def test_indexer_toy_scores():
     g, names, qI, KI = _toy_indexer()
     w = np.array([float(x) for x in g["w_second"][0]])

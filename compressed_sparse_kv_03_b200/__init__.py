@@ -7,9 +7,9 @@ include/csa.h); this package is its thin Python binding.
 from ._lib import (CsaError, KERNEL_ATTENTION, KERNEL_COMPRESS, KERNEL_INDEXER_SCORE,  # noqa: F401
                    KERNEL_MERGE, KERNEL_TOPK_SELECT, load)
 from .api import (AppendState, Cache, Workspace, cache_append, compress_kv, hca_attn,  # noqa: F401
-                  indexer_topk, launch_count, set_attention_kernel, set_batch_invariant,
+                  indexer_topk, launch_count, norm_rope, set_attention_kernel, set_batch_invariant,
                   set_timing_events, sparse_attn_decode, sparse_attn_prefill)
 
-__all__ = ["Cache", "Workspace", "CsaError", "compress_kv", "cache_append", "AppendState",
+__all__ = ["Cache", "Workspace", "CsaError", "compress_kv", "cache_append", "AppendState", "norm_rope",
            "indexer_topk", "sparse_attn_prefill", "sparse_attn_decode", "hca_attn", "launch_count",
            "set_attention_kernel", "set_batch_invariant", "set_timing_events", "load"]

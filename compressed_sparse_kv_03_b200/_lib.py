@@ -54,6 +54,8 @@ SIGNATURES = {
     "csa_workspace_init": (C.c_int, [_vp, _sz, _vp]),
     "csa_workspace_check": (C.c_int, [_vp, _vp]),
     "csa_compress_kv": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp]),
+    "csa_norm_rope": (C.c_int, [_vp, _vp, _i64, _i32, _i32, _vp, _f32, _vp, _i64, _i32, _f32, _i32,
+                                _vp]),
     "csa_cache_append": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp,
                                    _vp, _vp, _vp, _i32, C.POINTER(CacheT), _i64, _vp, _sz, _vp]),
     "csa_indexer_topk": (C.c_int, [_vp, _vp, C.POINTER(CacheT), _vp, _vp, _i64, _i32, _i32, _i32,

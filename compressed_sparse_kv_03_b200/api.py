@@ -137,6 +137,30 @@ def compress_kv(C_a, Z_a, m, *, C_b=None, Z_b=None, bias=None, overlap=False, ou
     return out
 
 
+def norm_rope(x, *, gain=None, eps=1e-6, pos=None, pos_mul=1, rope_dims=64, rope_base=10000.0,
+              inverse=False, out=None, stream=None):
+    """RMSNorm (eps >= 0; eps=None skips it) and partial RoPE (rope_dims > 0)
+    of [T, H, dim] or [T, dim] bf16 vectors at positions (pos or row) * pos_mul;
+    inverse=True applies the output de-rotation R_{-t} (use eps=None)."""
+    _need(x, "x", torch.bfloat16)
+    dev = x.device
+    if x.dim() not in (2, 3):
+        raise ValueError("x must be [T, dim] or [T, H, dim]")
+    T, dim = x.shape[0], x.shape[-1]
+    H = x.shape[1] if x.dim() == 3 else 1
+    if gain is not None:
+        _need(gain, "gain", torch.float32, 1, dev)
+    if pos is not None:
+        _need(pos, "pos", torch.int64, 1, dev)
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", torch.bfloat16, None, dev)
+    check(load().csa_norm_rope(_ptr(x), _ptr(out), T, H, dim, _ptr(gain),
+                               -1.0 if eps is None else float(eps), _ptr(pos), int(pos_mul),
+                               int(rope_dims), float(rope_base), int(bool(inverse)), _stream(stream)))
+    return out
+
+
 @dataclass
 class AppendState:
     """Per-sequence decode-time cache state for `cache_append`: the unfinished

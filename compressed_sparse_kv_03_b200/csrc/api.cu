@@ -365,6 +365,38 @@ csa_status_t csa_cache_append(const csa_bf16* C_a, const csa_bf16* Z_a, const cs
   return cuda_status(launch_cache_append(L, a), "csa_cache_append launch");
 }
 
+csa_status_t csa_norm_rope(const csa_bf16* x, csa_bf16* out, int64_t T, int32_t H, int32_t dim,
+                           const float* gain, float eps, const int64_t* pos, int64_t pos_mul,
+                           int32_t rope_dims, float rope_base, int32_t inverse,
+                           csa_stream_t stream) {
+  const char* name = "csa_norm_rope";
+  if (T < 0 || H < 1 || (dim != 64 && dim != 128 && dim != 256) || rope_dims < 0 ||
+      rope_dims > dim || rope_dims % 8 != 0 || (inverse != 0 && inverse != 1) ||
+      (rope_dims > 0 && !(rope_base > 1.f)) || !(eps == eps))
+    return fail(CSA_ERR_INVALID_ARG,
+                "%s: need T >= 0, H >= 1, dim in {64,128,256}, rope_dims a multiple of 8 <= dim, "
+                "rope_base > 1, inverse in {0,1}", name);
+  if (T == 0) return CSA_OK;
+  if (x == nullptr || out == nullptr) return fail(CSA_ERR_INVALID_ARG, "%s: x and out are required", name);
+  if (!aligned16(x) || !aligned16(out) || (gain && !aligned16(gain)))
+    return fail(CSA_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", name);
+  NormRopeArgs a{};
+  a.x = (const __nv_bfloat16*)x;
+  a.out = (__nv_bfloat16*)out;
+  a.T = T;
+  a.H = H;
+  a.dim = dim;
+  a.gain = gain;
+  a.eps = eps;
+  a.pos = pos;
+  a.pos_mul = pos_mul;
+  a.rope_dims = rope_dims;
+  a.rope_base = rope_base;
+  a.inverse = inverse;
+  Launch L{(cudaStream_t)stream};
+  return cuda_status(launch_norm_rope(L, a), "csa_norm_rope launch");
+}
+
 // ---- steps 2-3 ---------------------------------------------------------------
 csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_cache_t* k_idx,
                               const int32_t* seq_id, const int64_t* q_pos, int64_t T,

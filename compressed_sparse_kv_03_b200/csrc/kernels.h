@@ -41,6 +41,24 @@ struct CacheAppendArgs {
 };
 cudaError_t launch_cache_append(const Launch& L, const CacheAppendArgs& a);
 
+// RMSNorm (eps >= 0) and / or partial RoPE (rope_dims > 0) of [T, H, dim]
+// vectors: see normrope.cu.
+struct NormRopeArgs {
+  const __nv_bfloat16* x;
+  __nv_bfloat16* out;                        // may equal x
+  int64_t T;
+  int H, dim;
+  const float* gain;                         // [dim] or null
+  float eps;                                 // < 0: no RMSNorm
+  const int64_t* pos;                        // [T] or null (row index)
+  int64_t pos_mul;                           // position = (pos ? pos[t] : t) * pos_mul
+  int rope_dims;                             // rotated trailing coordinates (0: none)
+  float rope_base;
+  int inverse;                               // 1: R_{-t}
+  double theta[128];                         // pair frequencies base^(-2j / rope_dims) (host-filled)
+};
+cudaError_t launch_norm_rope(const Launch& L, const NormRopeArgs& a);
+
 // Indexer scratch limits.  Few-query (decode) mode keeps a 4096-bin histogram
 // of the top 12 score-key bits per query and selects through a bitmap in
 // shared memory; many-query (prefill) mode holds a query's keys in shared

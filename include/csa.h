@@ -201,6 +201,29 @@ csa_status_t csa_cache_append(const csa_bf16* C_a, const csa_bf16* Z_a, const cs
                               csa_bf16* win, int32_t window, const csa_cache_t* cache,
                               int64_t max_entries, void* ws, size_t ws_bytes, csa_stream_t stream);
 
+/*
+ * csa_norm_rope -- the attention prologue / epilogue on [T, H, dim] bf16
+ * vectors (Book Ch.2 "Normalization and rotary position embeddings"; Ch.7
+ * "Query and KV RMSNorm", "Partial RoPE and output de-rotation"):
+ *   eps >= 0: RMSNorm, x / sqrt(mean(x^2) + eps) * gain (gain [dim] fp32 or
+ *             NULL for 1); eps < 0 skips it;
+ *   rope_dims > 0: the last rope_dims coordinates are rotated by R_p, pairs
+ *             (2j, 2j+1) of that slice by angle p * rope_base^(-2j/rope_dims),
+ *             at position p = (pos ? pos[t] : t) * pos_mul; inverse = 1 applies
+ *             R_{-p} (the output de-rotation with the query position).
+ * Queries: eps, rope at the token position.  Compressed entries: pos_mul = m
+ * (entry i at position i*m, the first token of its block; a reading, the
+ * pages do not say which token).  Window rows: their token positions.
+ * Attention outputs: eps < 0, inverse = 1, the query positions.
+ *   out may equal x (in place).  dim in {64, 128, 256}; rope_dims a multiple
+ *   of 8 and <= dim; 16-byte aligned buffers.  fp32 arithmetic (angles reduced
+ *   modulo 2 pi in fp64), output rounded to nearest bf16.
+ */
+csa_status_t csa_norm_rope(const csa_bf16* x, csa_bf16* out, int64_t T, int32_t H, int32_t dim,
+                           const float* gain, float eps, const int64_t* pos, int64_t pos_mul,
+                           int32_t rope_dims, float rope_base, int32_t inverse,
+                           csa_stream_t stream);
+
 /* ---- steps 2-3: lightning indexer + top-k ---------------------------------- */
 /*
  * csa_indexer_topk -- for every query i at position t_i of sequence b_i:

@@ -14,6 +14,8 @@ from .csa_oracle import (  # noqa: F401
     pool_block,
     pool_overlap,
     DecodeCacheState,
+    rmsnorm,
+    rope_rotate,
     eligible_entries,
     indexer_scores,
     topk_select,

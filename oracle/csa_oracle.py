@@ -153,6 +153,40 @@ class DecodeCacheState:
 
 
 # ---------------------------------------------------------------------------
+# attention prologue / epilogue: RMSNorm, partial RoPE, output de-rotation
+# ---------------------------------------------------------------------------
+def rmsnorm(x, gain=None, eps=1e-6):
+    """RMSNorm over the last axis (Ch.2 "Normalization and rotary position
+    embeddings"; Ch.7 "Query and KV RMSNorm"): x / sqrt(mean(x^2) + eps),
+    times a per-coordinate gain.  eps is not printed; 1e-6 is the reading."""
+    x = np.asarray(x, dtype=np.float64)
+    y = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return y if gain is None else y * np.asarray(gain, dtype=np.float64)
+
+
+def rope_rotate(x, pos, rope_dims=64, base=10000.0, inverse=False):
+    """Partial RoPE (Ch.7 "Partial RoPE and output de-rotation"): the last
+    `rope_dims` coordinates of every vector are rotated by R_t, block-diagonal
+    with 2x2 rotations of the pairs (2j, 2j+1) of the rotary slice by angle
+    t * base^(-2j / rope_dims); inverse applies R_{-t} = R_t^T.  The pairing
+    and the base are not printed; interleaved pairs and base 10000 are the
+    reading.  x: [..., d]; pos: broadcastable to x.shape[:-1]."""
+    x = np.array(x, dtype=np.float64)
+    d = x.shape[-1]
+    r0 = d - rope_dims
+    j = np.arange(rope_dims // 2)
+    theta = base ** (-2.0 * j / rope_dims)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * theta
+    if inverse:
+        ang = -ang
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[..., r0::2].copy(), x[..., r0 + 1::2].copy()
+    x[..., r0::2] = a * c - b * s
+    x[..., r0 + 1::2] = a * s + b * c
+    return x
+
+
+# ---------------------------------------------------------------------------
 # steps 2-3: lightning indexer and top-k
 # ---------------------------------------------------------------------------
 def eligible_entries(t, m):

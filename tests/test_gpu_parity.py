@@ -81,6 +81,40 @@ def test_compress_overlap(N, dim, m, bias, separate):
     assert_close_attn(out, ref, "compress overlap")
 
 
+@pytest.mark.parametrize("T,H,dim,rope,gain", [(300, 64, 128, 64, True), (1000, 1, 128, 64, False),
+                                               (77, 8, 64, 32, True), (50, 4, 256, 64, True)])
+def test_norm_rope_prologue(T, H, dim, rope, gain):
+    """Query / KV prologue: RMSNorm with a gain, then partial RoPE at large
+    positions; compressed entries at position i*m."""
+    csa = _csa()
+    g = synth.generator(160 + T + dim)
+    x = synth.normal(g, (T, H, dim), 2.5)
+    gn = (1.0 + 0.2 * synth.normal(g, (dim,), dtype=torch.float32)) if gain else None
+    pos = torch.randint(0, 1 << 20, (T,), generator=g, dtype=torch.int64)
+    use_pos = H > 1
+    out = csa.norm_rope(dev(x), gain=dev(gn), pos=dev(pos) if use_pos else None, pos_mul=1 if use_pos else 4,
+                        rope_dims=rope)
+    p = f64(pos) if use_pos else np.arange(T) * 4.0
+    ref = oracle.rope_rotate(oracle.rmsnorm(f64(x), None if gn is None else f64(gn)),
+                             p[:, None] if H > 1 else p[:, None], rope_dims=rope)
+    assert_close_attn(out, ref, "norm + rope")
+
+
+def test_norm_rope_output_derotation_in_place():
+    csa = _csa()
+    g = synth.generator(170)
+    T, H = 200, 64
+    o = synth.normal(g, (T, H, 128))
+    pos = torch.randint(0, 1 << 22, (T,), generator=g, dtype=torch.int64)
+    od = dev(o)
+    got = csa.norm_rope(od, eps=None, pos=dev(pos), inverse=True, out=od)
+    assert got.data_ptr() == od.data_ptr()
+    ref = oracle.rope_rotate(f64(o), f64(pos)[:, None], inverse=True)
+    assert_close_attn(got, ref, "de-rotation")
+    # the content coordinates pass through unchanged
+    assert torch.equal(got[:, :, :64].cpu(), o[:, :, :64])
+
+
 @pytest.mark.parametrize("overlap,paged,dim", [(True, False, 128), (False, True, 128), (True, True, 64)])
 def test_cache_append_matches_bulk_compression(overlap, paged, dim):
     """Decode-time appends, one token per sequence per call: entry for entry the

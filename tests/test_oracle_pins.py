@@ -188,6 +188,57 @@ def test_decode_cache_state_entry_reads_only_its_blocks():
         assert changed != same, (t, same)
 
 
+def test_rmsnorm_closed_forms():
+    """Ch.2 "Normalization and rotary position embeddings": unit RMS without a
+    gain, invariant to a positive scale, gain per coordinate, zeros stay zero."""
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((5, 128)) * 3.0
+    y = oracle.rmsnorm(x, eps=0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(y * y, axis=-1)), 1.0, rtol=1e-12)
+    np.testing.assert_allclose(oracle.rmsnorm(7.5 * x, eps=0.0), y, rtol=1e-12)
+    g = rng.standard_normal(128)
+    np.testing.assert_allclose(oracle.rmsnorm(x, g, eps=0.0), y * g, rtol=1e-12)
+    assert np.all(oracle.rmsnorm(np.zeros((2, 64))) == 0.0)
+
+
+def test_rope_closed_forms():
+    """Ch.7 "Partial RoPE and output de-rotation": only the last 64
+    coordinates move; pair j of the slice turns by t * 10000^(-2j/64); R_t is
+    orthogonal with inverse R_{-t}; q.k after rotation depends only on s - t."""
+    rng = np.random.default_rng(42)
+    d, r0 = 128, 64
+    t = 1234567
+    for j in (0, 5, 31):
+        e = np.zeros(d)
+        e[r0 + 2 * j] = 1.0
+        y = oracle.rope_rotate(e, t)
+        ang = t * 10000.0 ** (-2.0 * j / 64)
+        np.testing.assert_allclose(y[r0 + 2 * j:r0 + 2 * j + 2], [np.cos(ang), np.sin(ang)], atol=1e-9)
+        assert np.count_nonzero(np.abs(y) > 1e-12) <= 2
+    x = rng.standard_normal((4, d))
+    y = oracle.rope_rotate(x, [3, 70, 9000, 2 ** 20])
+    np.testing.assert_array_equal(y[:, :r0], x[:, :r0])
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-12)
+    np.testing.assert_allclose(oracle.rope_rotate(y, [3, 70, 9000, 2 ** 20], inverse=True), x, atol=1e-9)
+    q, k = rng.standard_normal(d), rng.standard_normal(d)
+    dot = lambda tq, ts: oracle.rope_rotate(q, tq) @ oracle.rope_rotate(k, ts)
+    np.testing.assert_allclose(dot(500, 120), dot(500 + 4099, 120 + 4099), rtol=1e-9)
+
+
+def test_output_derotation_gives_relative_positions():
+    """Applying R_{-t} to an attention output over values rotated by R_s gives
+    the sum of values rotated by R_{s-t} (the pages' de-rotation identity)."""
+    rng = np.random.default_rng(43)
+    d, n, t = 128, 6, 777
+    v = rng.standard_normal((n, d))
+    s = np.array([3, 100, 640, 701, 760, 777])
+    p = rng.dirichlet(np.ones(n))
+    o = (p[:, None] * oracle.rope_rotate(v, s)).sum(0)
+    lhs = oracle.rope_rotate(o, t, inverse=True)
+    rhs = (p[:, None] * oracle.rope_rotate(v, s - t)).sum(0)
+    np.testing.assert_allclose(lhs, rhs, atol=1e-9)
+
+
 def test_indexer_toy_scores():
     g, names, qI, KI = _toy_indexer()
     w = np.array([float(x) for x in g["w_second"][0]])

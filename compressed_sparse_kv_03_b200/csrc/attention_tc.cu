@@ -45,8 +45,18 @@ constexpr int kKvTile = kRows * kD * 2;         // 32 KB: two 64-dim blocks of 1
 constexpr int kKBlock = kRows * 128;            // 16 KB
 constexpr int kQTile = kNP * kD * 2;            // 16 KB: two 64-dim blocks of 8 KB
 constexpr int kPTile = kRows * kNP * 2;         // 16 KB
-constexpr int kSmWarps = 8;                     // two softmax warpgroups
-constexpr int kHW = kNP / 2;                    // heads per softmax warpgroup
+#ifndef CSA_ATTN_GROUPS
+#define CSA_ATTN_GROUPS 2
+#endif
+constexpr int kSmGroups = CSA_ATTN_GROUPS;      // softmax warpgroups (2 or 4)
+constexpr int kSmWarps = 4 * kSmGroups;
+constexpr int kHW = kNP / kSmGroups;            // heads per softmax warpgroup
+// registers per thread after setmaxnreg: softmax / the rest.  The block is
+// launched with 65536 / kThreads (rounded down to 8) per thread, and the split
+// must add up to no more than that: 2 groups: 256 x 184 + 256 x 72 = 512 x 128;
+// 4 groups: 512 x 88 + 256 x 64 = 768 x 80.
+constexpr int kSmRegs = kSmGroups == 2 ? 184 : 88;
+constexpr int kOtherRegs = kSmGroups == 2 ? 72 : 64;
 constexpr int kMmaWarp = kSmWarps, kProducerWarp = kSmWarps + 1;
 constexpr int kProducerWarps = 7;
 constexpr int kProducerThreads = kProducerWarps * 32;
@@ -189,7 +199,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages];
   __shared__ __align__(8) uint64_t q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2];
-  __shared__ __align__(8) uint64_t o_full, o_empty, o_step, red_bar[2];
+  __shared__ __align__(8) uint64_t o_full, o_empty, o_step, red_bar[kSmGroups];
   __shared__ uint32_t tmem_base_sh;
   // validity of the tile's rows, one word per producer warp: bit 2j + s of
   // word k is row 2 (k + 7 j) + s
@@ -220,8 +230,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
     mbar_init(smem_u32(&o_full), 1);
     mbar_init(smem_u32(&o_empty), kSmWarps);
     mbar_init(smem_u32(&o_step), 1);
-    mbar_init(smem_u32(&red_bar[0]), 4);
-    mbar_init(smem_u32(&red_bar[1]), 4);
+    for (int g = 0; g < kSmGroups; ++g) mbar_init(smem_u32(&red_bar[g]), 4);
     mbar_fence_init();
   }
   if (warp == kMmaWarp) tc::tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
@@ -237,7 +246,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
   // thread, the softmax warpgroups take 184 (2 x 128 x (72 + 184) = the
   // 512 x 128 the block is launched with).
   if (warp >= kMmaWarp) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs) : "memory");
   if (warp >= kProducerWarp) {
     // ================================================================ producer
     // Seven warps.  Gathered rows: the tile's 64 row pairs are dealt round
@@ -448,7 +457,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
     }
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 184;\n" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSmRegs) : "memory");
     // ================================================================ softmax + epilogue
     // Warpgroup wg (warps 4wg .. 4wg+3) owns heads [32 wg, 32 wg + 32) of every
     // tile: thread = row of S^T in the tile loop, = dim of O^T in the epilogue.
@@ -456,6 +465,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
     // derives the same running maxima itself (lane h holds head 32 wg + h).
     const int wg = warp >> 2, wq = warp & 3;
     const int hoff = wg * kHW;
+    const int hl = lane & (kHW - 1);
     const int row = wq * 32 + lane;
     const int ok_word = (row >> 1) % kProducerWarps, ok_bit = 2 * ((row >> 1) / kProducerWarps) + (row & 1);
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
@@ -499,15 +509,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         tc::fence_after_sync();
         float x[kHW];
         {
-          uint32_t r0[16], r1[16];
-          tc::tmem_ld16(tm_s + sb * kNP + hoff + lane_base, r0);
-          tc::tmem_ld16(tm_s + sb * kNP + hoff + 16 + lane_base, r1);
+          uint32_t rr[kHW / 16][16];
+#pragma unroll
+          for (int c = 0; c < kHW / 16; ++c) tc::tmem_ld16(tm_s + sb * kNP + hoff + 16 * c + lane_base, rr[c]);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            x[j] = __uint_as_float(r0[j]);
-            x[16 + j] = __uint_as_float(r1[j]);
-          }
+          for (int c = 0; c < kHW / 16; ++c)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) x[16 * c + j] = __uint_as_float(rr[c][j]);
         }
         tc::fence_before_sync();
         __syncwarp();
@@ -532,8 +541,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
           }
         }
         if (!(ok = group_sync(rbar, red_phase, lane))) break;
-        float tmax = fmaxf(fmaxf(rm[4 * wg][lane], rm[4 * wg + 1][lane]),
-                           fmaxf(rm[4 * wg + 2][lane], rm[4 * wg + 3][lane]));
+        // lane hl = lane mod kHW stands for head hoff + hl (lanes past kHW repeat them)
+        float tmax = fmaxf(fmaxf(rm[4 * wg][hl], rm[4 * wg + 1][hl]),
+                           fmaxf(rm[4 * wg + 2][hl], rm[4 * wg + 3][hl]));
         tmax *= scale;   // scale > 0: the max commutes with it
         float f = 1.f;
         bool grew = false;
@@ -543,8 +553,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
           m_run = tmax;
         }
         const bool rescale = __any_sync(0xffffffffu, grew);
-        my_bc[lane] = m_run == -INFINITY ? 0.f : m_run;
-        if (rescale) my_bc[kHW + lane] = f;
+        if (lane < kHW) {
+          my_bc[lane] = m_run == -INFINITY ? 0.f : m_run;
+          if (rescale) my_bc[kHW + lane] = f;
+        }
         __syncwarp();
         if (rescale) {
           // this warp's 32 dims of O^T for the group's heads, when a running max moved
@@ -618,7 +630,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
           lpart[j] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
         }
       }
-      red_l[warp][lane] = lpart[0];
+      for (int o = kHW; o < 32; o <<= 1) lpart[0] += __shfl_xor_sync(0xffffffffu, lpart[0], o);
+      if (lane < kHW) red_l[warp][lane] = lpart[0];
       if (!mbar_wait(smem_u32(&o_full), (uint32_t)(items_done & 1)) ||
           !group_sync(rbar, red_phase, lane)) {
         if (lane == 0) report(a.err, kErrTimeout, (int32_t)it.i, 28);
@@ -626,9 +639,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
       }
       pv_seen = tiles_done;
       {
-        const int h = hoff + lane;
-        const float l = (red_l[4 * wg][lane] + red_l[4 * wg + 1][lane]) +
-                        (red_l[4 * wg + 2][lane] + red_l[4 * wg + 3][lane]);
+        const int h = hoff + hl;
+        const float l = (red_l[4 * wg][hl] + red_l[4 * wg + 1][hl]) +
+                        (red_l[4 * wg + 2][hl] + red_l[4 * wg + 3][hl]);
         const float m = m_run;
         float nrm = 1.f;
         if (a.n_split == 1) {
@@ -643,13 +656,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
             mm = rr;
           }
           nrm = den > 0.f ? __fdividef(f, den) : 0.f;
-          if (wq == 0 && a.lse != nullptr && h < nh)
+          if (wq == 0 && lane < kHW && a.lse != nullptr && h < nh)
             a.lse[it.i * a.H + h_base + h] = den > 0.f ? (mm + log2f(den)) / kLog2e : -INFINITY;
-        } else if (wq == 0 && h < nh) {
+        } else if (wq == 0 && lane < kHW && h < nh) {
           *reinterpret_cast<float2*>(a.part_ml + ((it.i * a.n_split + it.split) * a.H + h_base + h) * 2) =
               make_float2(m, l);
         }
-        my_bc[kHW + lane] = nrm;
+        if (lane < kHW) my_bc[kHW + lane] = nrm;
       }
       __syncwarp();
       tc::fence_after_sync();

@@ -29,3 +29,4 @@ from .csa_oracle import (  # noqa: F401
     hca_prefill,
 )
 from . import cost_model  # noqa: F401
+from . import mxfp4  # noqa: F401

@@ -453,3 +453,108 @@ def test_cost_model_matches_pages():
             assert v == want, name
         else:
             assert abs(v - want) <= tol * abs(want), (name, v, want)
+
+
+# ---------------------------------------------------------------------------
+# 4-bit indexer storage (Ch.8 "V4 compressed-entry payload" and "Quantization
+# scales and bounded tail buffers")
+# ---------------------------------------------------------------------------
+from oracle import mxfp4 as ofp4   # noqa: E402
+
+
+def test_e2m1_values_are_the_fp4_grid():
+    # the eight E2M1 magnitudes as the OCP MX format tabulates them, +/- by bit 3
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    got = ofp4.e2m1_value(np.arange(16))
+    assert got[:8].tolist() == mags
+    assert (-got[8:]).tolist() == mags
+    assert np.signbit(got[8])   # code 8 is -0
+
+
+def test_e2m1_encode_matches_library_rounding():
+    import ml_dtypes
+    # every midpoint and every grid value, both signs, plus random values over
+    # and beyond the range (saturation)
+    mags = ofp4.e2m1_value(np.arange(8))
+    mids = (mags[1:] + mags[:-1]) / 2
+    y = np.concatenate([mags, mids, mids * (1 + 2.0 ** -20), mids * (1 - 2.0 ** -20),
+                        rng.uniform(-9, 9, 4000), [6.5, 7.99, 1e6, -1e6]])
+    y = np.concatenate([y, -y]).astype(np.float32)
+    lib = y.astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+    assert np.array_equal(ofp4.e2m1_encode(y.astype(np.float64)), lib)
+
+
+def test_e2m1_ties_go_to_even_codes():
+    # midpoints of adjacent magnitudes -> the neighbour with mantissa bit 0
+    assert ofp4.e2m1_encode([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]).tolist() == [0, 2, 2, 4, 4, 6, 6]
+
+
+def test_mxfp4_scale_puts_block_max_in_top_binade():
+    # X = floor(log2 amax) - 2, so amax / 2^X lies in [4, 8)
+    for _ in range(200):
+        blk = rng.standard_normal(32) * 2.0 ** rng.integers(-30, 30)
+        X = ofp4.mxfp4_scale_exponent(blk)
+        r = np.abs(blk).max() / 2.0 ** X
+        assert 4.0 <= r < 8.0
+    assert ofp4.mxfp4_scale_exponent(np.zeros(32)) == -127
+    assert ofp4.mxfp4_scale_exponent(np.full(32, 2.0 ** -200)) == -127   # clamped
+    assert ofp4.mxfp4_scale_exponent(np.full(32, 6.0)) == 0
+    assert ofp4.mxfp4_scale_exponent(np.full(32, 4.0)) == 0
+    assert ofp4.mxfp4_scale_exponent(np.full(32, 3.99)) == -1
+
+
+def test_mxfp4_roundtrip_and_error_bound():
+    x = oracle.bf16_round(rng.standard_normal((64, 128)))
+    packed, scales = ofp4.mxfp4_quantize(x)
+    assert packed.shape == (64, 64) and scales.shape == (64, 4)
+    y = ofp4.mxfp4_dequantize(packed, scales)
+    # representable values survive unchanged
+    p2, s2 = ofp4.mxfp4_quantize(y)
+    assert np.array_equal(p2, packed) and np.array_equal(s2, scales)
+    # the error of an element is at most half the grid step at its magnitude,
+    # except above 6 (saturation), where it is below 2 * 2^X
+    X = np.repeat(scales.astype(np.int64) - 127, 32, axis=1)
+    u = np.abs(x) / 2.0 ** X
+    half_step = np.where(u < 2, 0.25, np.where(u < 4, 0.5, 1.0))
+    bound = np.where(u > 6, 2.0, half_step) * 2.0 ** X
+    assert np.all(np.abs(y - x) <= bound)
+
+
+def test_mxfp4_packing_order():
+    # element 2i in the low nibble of byte i, element 2i+1 in the high nibble
+    x = np.zeros(32)
+    x[0], x[1], x[30], x[31] = 4.0, -1.0, 0.5, 6.0     # amax 6 -> X = 0
+    packed, scales = ofp4.mxfp4_quantize(x)
+    assert scales.tolist() == [127]
+    assert packed[0] == (0x6 | (0xA << 4)) and packed[15] == (0x1 | (0x7 << 4))
+
+
+def test_mxfp4_key_bytes_match_pages():
+    # a 128-dim FP4 indexer key is 64 bytes; one scale byte per 32 elements adds
+    # 4 bytes, +6.25 % (Ch.8 "Quantization scales and bounded tail buffers")
+    packed, scales = ofp4.mxfp4_quantize(rng.standard_normal(128))
+    assert packed.nbytes == 64 and scales.nbytes == 4
+    assert scales.nbytes / packed.nbytes == 0.0625
+
+
+def test_mxfp4_indexer_scores_brute_force():
+    # scores from codes decoded by the printed grid, in plain loops
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    H, c, n = 3, 64, 5
+    qp, qs = ofp4.mxfp4_quantize(rng.standard_normal((H, c)))
+    kp, ks = ofp4.mxfp4_quantize(rng.standard_normal((n, c)))
+    w = rng.uniform(0, 1, H)
+
+    def val(packed, scales, r):
+        b = int(packed[r // 2])
+        code = (b & 0xF) if r % 2 == 0 else (b >> 4)
+        v = grid[code & 7] * (-1.0 if code & 8 else 1.0)
+        return v * 2.0 ** (int(scales[r // 32]) - 127)
+
+    got = ofp4.indexer_scores_mxfp4(qp, qs, w, kp, ks)
+    for s in range(n):
+        want = 0.0
+        for h in range(H):
+            dot = sum(val(qp[h], qs[h], r) * val(kp[s], ks[s], r) for r in range(c))
+            want += w[h] * max(dot, 0.0)
+        assert got[s] == pytest.approx(want, rel=1e-12, abs=1e-12)

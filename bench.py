@@ -8,7 +8,9 @@ input already resident in HBM.  The default workload is CSA decode (batch 64,
 128K context each, 64 heads x 128 on one shared KV head, m = 4, indexer
 8 x 64, top-k 2048, window 128): step = indexer + top-k + sparse attention.
 Other workloads: csa_prefill_L4096, csa_prefill_L65536,
-hca_decode_B8_N1048576, mixed_decode_B16_N256K_1M.
+hca_decode_B8_N1048576, mixed_decode_B16_N256K_1M, and
+csa_decode_B64_N131072_mxfp4_indexer (the default decode with the indexer keys
+and queries in 4-bit storage).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch (weak
 scaling, no data-path collective); the step time is the max over ranks.
@@ -109,6 +111,40 @@ class CsaDecode:
         return {"workload": c.name, "batch": c.B, "context": c.N, "heads": c.H, "head_dim": c.d,
                 "m": c.m, "indexer_heads": c.H_I, "indexer_dim": c.c_I, "top_k": c.k, "window": c.W,
                 "l2": f"inputs larger than L2: {self.step_bytes / 1e6:.0f} MB streamed per step"}
+
+
+class CsaDecodeMxfp4(CsaDecode):
+    """CSA decode with the 4-bit indexer: the indexer-key cache holds E2M1
+    codes plus one scale byte per 32 elements (quantized once, when the cache
+    is built); a step quantizes the new indexer queries, scores and selects
+    from the codes (csa_indexer_topk_mxfp4), then attends as the bf16 step."""
+
+    def __init__(self, cfg, seed_offset=0):
+        super().__init__(cfg, seed_offset)
+        csa = self.csa
+        kc, ks = csa.quantize_mxfp4(self.d.pop("kI_comp"))
+        self.kI = csa.Cache(kc.view(-1, kc.shape[-1]), seq_stride=self.S)
+        self.kI_scales = ks.view(-1, ks.shape[-1])
+        self.qc, self.qs = csa.quantize_mxfp4(self.d["qI"])
+        torch.cuda.synchronize()
+        sel_rows = min(cfg.k, self.S) + min(cfg.W, cfg.N + 1)
+        self.dominant_bytes = cfg.B * self.S * (cfg.c_I // 2 + cfg.c_I // 32)
+        self.step_bytes = (self.dominant_bytes + cfg.B * sel_rows * cfg.d * 2
+                           + cfg.B * (2 * cfg.H * cfg.d * 2 + cfg.H_I * cfg.c_I * 2 + cfg.H_I * 4))
+
+    def step(self):
+        csa, cfg, d = self.csa, self.cfg, self.d
+        csa.quantize_mxfp4(d["qI"], out=(self.qc, self.qs))
+        csa.indexer_topk_mxfp4(self.qc, self.qs, d["w"], self.kI, self.kI_scales, cfg.m, cfg.k,
+                               seq_id=self.seq_id, q_pos=d["pos"], max_entries=self.S, ws=self.ws_i,
+                               out=(self.idx, self.cnt, None))
+        csa.sparse_attn_decode(d["q"], self.kv, d["win"], d["win_len"], self.idx, self.cnt, cfg.lam,
+                               ws=self.ws_a, out=self.out)
+
+    def config(self):
+        c = super().config()
+        c["indexer_storage"] = "E2M1 codes + one power-of-two scale byte per 32 (34 B per key)"
+        return c
 
 
 class HcaDecode:
@@ -286,7 +322,8 @@ class MixedDecode:
                 "l2": f"inputs larger than L2: {self.step_bytes / 1e6:.0f} MB streamed per step"}
 
 
-KERNEL_NAMES = {0: "indexer_score", 1: "topk_select", 2: "attention", 3: "merge", 4: "compress"}
+KERNEL_NAMES = {0: "indexer_score", 1: "topk_select", 2: "attention", 3: "merge", 4: "compress",
+                5: "quantize"}
 
 RUNNERS = {
     synth.CFG_DECODE_128K.name: (CsaDecode, synth.CFG_DECODE_128K),
@@ -294,6 +331,7 @@ RUNNERS = {
     synth.CFG_PREFILL_4K.name: (CsaPrefill, synth.CFG_PREFILL_4K),
     synth.CFG_PREFILL_64K.name: (CsaPrefill, synth.CFG_PREFILL_64K),
     synth.CFG_MIXED.name: (MixedDecode, synth.CFG_MIXED),
+    synth.CFG_DECODE_128K_MXFP4.name: (CsaDecodeMxfp4, synth.CFG_DECODE_128K_MXFP4),
 }
 
 
@@ -383,6 +421,24 @@ def oracle_sample(name, budget_s):
         threads = 1
     cls, cfg = RUNNERS[name]
     f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+    if cls is CsaDecodeMxfp4:
+        from oracle import mxfp4 as ofp4
+        host = synth.csa_decode_inputs(cfg, B=min(cfg.B, 16))
+        done, secs = 0, 0.0
+        while done < host["q"].shape[0] and secs < budget_s:
+            b = done
+            kc, ks = ofp4.mxfp4_quantize(f(host["kI_comp"][b]))   # cache contents: not timed
+            t0 = time.perf_counter()
+            qc, qs = ofp4.mxfp4_quantize(f(host["qI"][b]))
+            n = oracle.eligible_entries(int(host["pos"][b]), cfg.m)
+            sel = oracle.topk_select(ofp4.indexer_scores_mxfp4(qc, qs, f(host["w"][b]), kc[:n], ks[:n]),
+                                     cfg.k)
+            rows = np.concatenate([f(host["kv_comp"][b])[sel], f(host["win"][b])[:int(host["win_len"][b])]])
+            oracle.attend_shared_kv(f(host["q"][b]), rows, cfg.lam)
+            secs += time.perf_counter() - t0
+            done += 1
+        return (done, secs, f"{done} of {cfg.B} sequences, full decode step each "
+                f"(key quantization of the cache not timed)", threads)
     if cls is CsaDecode:
         host = synth.csa_decode_inputs(synth.CsaDecode(**{**cfg.__dict__, "B": min(cfg.B, 64)}))
         done, t0 = 0, time.perf_counter()

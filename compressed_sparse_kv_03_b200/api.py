@@ -5,6 +5,8 @@ the current torch stream.  Shapes follow the header:
 
     compress_kv          (step 1)    C, Z [N, dim] -> [N // m, dim]
     indexer_topk         (steps 2-3) q_idx [T, H_I, c_I], w [T, H_I], keys -> idx [T, k], count [T]
+    quantize_mxfp4       x [..., dim] bf16 -> 4-bit codes [..., dim/2] + scale bytes [..., dim/32]
+    indexer_topk_mxfp4   (steps 2-3) on 4-bit queries and keys
     sparse_attn_prefill  (step 4)    q [L, H, 128] over kv_comp[idx] + raw window
     sparse_attn_decode   (step 4)    q [B, H, 128] over cache[idx] + window buffer
     hca_attn             (step 4)    q [T, H, 128] over all eligible entries + window
@@ -65,8 +67,8 @@ class Cache:
     def dim(self):
         return self.data.shape[-1]
 
-    def c(self):
-        _need(self.data, "cache.data", torch.bfloat16, 2)
+    def c(self, dtype=torch.bfloat16):
+        _need(self.data, "cache.data", dtype, 2)
         if self.page_table is not None:
             _need(self.page_table, "cache.page_table", torch.int32, 2)
             return CacheT(self.data.data_ptr(), self.data.shape[0], 0, self.page_table.data_ptr(),
@@ -238,6 +240,71 @@ def indexer_topk(q_idx, w, keys: Cache, m, top_k, *, seq_id=None, q_pos=None, ma
     check(lib.csa_indexer_topk(_ptr(q_idx), _ptr(w), C.byref(kc), _ptr(seq_id), _ptr(q_pos), T,
                                H_I, c_I, m, max_entries, top_k, _ptr(idx), _ptr(cnt), _ptr(sco),
                                wsp, wsb, _stream(stream)))
+    return (idx, cnt, sco) if return_scores else (idx, cnt)
+
+
+def quantize_mxfp4(x, *, stream=None, out=None):
+    """4-bit storage of bf16 vectors (E2M1 codes, one power-of-two scale byte
+    per 32 elements; see include/csa.h): x [..., dim] -> (codes [..., dim/2]
+    uint8, scales [..., dim/32] uint8)."""
+    _need(x, "x", torch.bfloat16)
+    dim = x.shape[-1]
+    if dim % 32 != 0 or dim == 0:
+        raise ValueError("the last dim must be a positive multiple of 32")
+    n = x.numel() // dim
+    if out is None:
+        codes = torch.empty(x.shape[:-1] + (dim // 2,), dtype=torch.uint8, device=x.device)
+        scales = torch.empty(x.shape[:-1] + (dim // 32,), dtype=torch.uint8, device=x.device)
+    else:
+        codes, scales = out
+    check(load().csa_quantize_mxfp4(_ptr(x), n, dim, _ptr(codes), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def indexer_topk_mxfp4(q_codes, q_scales, w, keys: Cache, k_scales, m, top_k, *, seq_id=None,
+                       q_pos=None, max_entries=None, return_scores=False, ws=None, stream=None,
+                       out=None):
+    """Steps 2-3 on 4-bit operands: q_codes [T, H_I, c_I/2] / q_scales
+    [T, H_I, c_I/32] from quantize_mxfp4, keys.data [rows, c_I/2] uint8 codes
+    with k_scales [rows, c_I/32] uint8 (same rows, same paging).
+    Returns (idx [T, top_k] int32, count [T] int32[, scores [T, top_k] fp32])."""
+    _need(q_codes, "q_codes", torch.uint8, 3)
+    T, H_I, half = q_codes.shape
+    c_I = 2 * half
+    dev = q_codes.device
+    _need(q_scales, "q_scales", torch.uint8, 3, dev)
+    if tuple(q_scales.shape) != (T, H_I, c_I // 32):
+        raise ValueError("q_scales must be [T, H_I, c_I/32]")
+    _need(w, "w", torch.float32, 2, dev)
+    if tuple(w.shape) != (T, H_I):
+        raise ValueError("w must be [T, H_I]")
+    if keys.dim != half:
+        raise ValueError("key code rows must hold c_I/2 bytes")
+    _need(k_scales, "k_scales", torch.uint8, 2, dev)
+    if tuple(k_scales.shape) != (keys.data.shape[0], c_I // 32):
+        raise ValueError("k_scales must be [rows of keys.data, c_I/32]")
+    if seq_id is not None:
+        _need(seq_id, "seq_id", torch.int32, 1, dev)
+    if q_pos is not None:
+        _need(q_pos, "q_pos", torch.int64, 1, dev)
+    if max_entries is None:
+        if q_pos is None:
+            max_entries = max(T - 1, 0) // m
+        else:
+            raise ValueError("max_entries is required with q_pos")
+    if out is None:
+        idx = torch.empty((T, top_k), dtype=torch.int32, device=dev)
+        cnt = torch.empty((T,), dtype=torch.int32, device=dev)
+        sco = torch.empty((T, top_k), dtype=torch.float32, device=dev) if return_scores else None
+    else:
+        idx, cnt, sco = out
+    lib = load()
+    wsp, wsb = _ws(ws, dev).get(lib.csa_indexer_topk_workspace_size(T, max_entries, top_k))
+    kc = keys.c(torch.uint8)
+    check(lib.csa_indexer_topk_mxfp4(_ptr(q_codes), _ptr(q_scales), _ptr(w), C.byref(kc),
+                                     _ptr(k_scales), _ptr(seq_id), _ptr(q_pos), T, H_I, c_I, m,
+                                     max_entries, top_k, _ptr(idx), _ptr(cnt), _ptr(sco), wsp, wsb,
+                                     _stream(stream)))
     return (idx, cnt, sco) if return_scores else (idx, cnt)
 
 

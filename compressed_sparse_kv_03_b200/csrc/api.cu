@@ -398,30 +398,13 @@ csa_status_t csa_norm_rope(const csa_bf16* x, csa_bf16* out, int64_t T, int32_t 
 }
 
 // ---- steps 2-3 ---------------------------------------------------------------
-csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_cache_t* k_idx,
-                              const int32_t* seq_id, const int64_t* q_pos, int64_t T,
-                              int32_t H_I, int32_t c_I, int32_t m, int64_t max_entries,
-                              int32_t top_k, int32_t* idx_out, int32_t* count_out,
-                              float* score_out, void* ws, size_t ws_bytes, csa_stream_t stream) {
-  if (T < 0 || H_I < 1 || m < 1 || top_k < 1 || max_entries < 0)
-    return fail(CSA_ERR_INVALID_ARG,
-                "csa_indexer_topk: need T >= 0, H_I >= 1, m >= 1, top_k >= 1, max_entries >= 0");
-  if (T == 0) return CSA_OK;
-  if (q_idx == nullptr || w == nullptr || idx_out == nullptr || count_out == nullptr)
-    return fail(CSA_ERR_INVALID_ARG, "csa_indexer_topk: q_idx, w, idx_out, count_out required");
-  if (H_I > 64) return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: H_I > 64 not built");
-  if (c_I != 64 && c_I != 128)
-    return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: c_I must be 64 or 128 (got %d)", c_I);
-  if (max_entries > kBitmapSelectMaxEntries)
-    return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: max_entries > %lld not built",
-                (long long)kBitmapSelectMaxEntries);
-  csa_status_t st = check_cache(k_idx, "csa_indexer_topk k_idx");
-  if (st != CSA_OK) return st;
-  if (!aligned16(q_idx)) return fail(CSA_ERR_INVALID_ARG, "csa_indexer_topk: q_idx alignment");
-  const size_t need = csa_indexer_topk_workspace_size(T, max_entries, top_k);
-  if ((st = check_ws(ws, ws_bytes, need, "csa_indexer_topk")) != CSA_OK) return st;
-  if (T == 0) return CSA_OK;
+namespace {
 
+// Score + select, one chunk of queries at a time (the workspace holds the
+// keys of one chunk).  `base` carries the query / key operands.
+csa_status_t run_indexer_topk(IndexerArgs base, const int64_t* q_pos, int64_t T, int32_t m,
+                              int64_t max_entries, int32_t top_k, int32_t* idx_out,
+                              int32_t* count_out, float* score_out, void* ws, csa_stream_t stream) {
   Launch L{(cudaStream_t)stream};
   const IndexerLayout lay = indexer_layout(T, max_entries);
   char* wsb = static_cast<char*>(ws);
@@ -435,15 +418,9 @@ csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_c
     const size_t zero_off = lay.bitmap ? lay.hist_off : lay.counter_off;
     cudaError_t e = cudaMemsetAsync(wsb + zero_off, 0, lay.counter_off + sizeof(uint32_t) - zero_off, L.stream);
     if (e != cudaSuccess) return cuda_status(e, "indexer workspace memset");
-    IndexerArgs ia;
-    ia.q_idx = (const __nv_bfloat16*)q_idx;
-    ia.w = w;
-    ia.keys = to_ref(k_idx);
-    ia.seq_id = seq_id;
+    IndexerArgs ia = base;
     ia.q_pos = q_pos;
     ia.T = T;
-    ia.H_I = H_I;
-    ia.c_I = c_I;
     ia.m = m;
     ia.max_entries = max_entries;
     ia.t_begin = t0;
@@ -471,6 +448,101 @@ csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_c
     if (e != cudaSuccess) return cuda_status(e, "top-k select launch");
   }
   return CSA_OK;
+}
+
+// Checks shared by the bf16 and 4-bit indexer calls.
+csa_status_t check_indexer_args(const char* name, int64_t T, int32_t H_I, int32_t c_I, int32_t m,
+                                int64_t max_entries, int32_t top_k, const float* w,
+                                const int32_t* idx_out, const int32_t* count_out,
+                                const csa_cache_t* k_idx) {
+  if (T < 0 || H_I < 1 || m < 1 || top_k < 1 || max_entries < 0)
+    return fail(CSA_ERR_INVALID_ARG,
+                "%s: need T >= 0, H_I >= 1, m >= 1, top_k >= 1, max_entries >= 0", name);
+  if (T == 0) return CSA_OK;
+  if (w == nullptr || idx_out == nullptr || count_out == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "%s: w, idx_out and count_out are required", name);
+  if (H_I > 64) return fail(CSA_ERR_UNSUPPORTED, "%s: H_I > 64 not built", name);
+  if (c_I != 64 && c_I != 128)
+    return fail(CSA_ERR_UNSUPPORTED, "%s: c_I must be 64 or 128 (got %d)", name, c_I);
+  if (max_entries > kBitmapSelectMaxEntries)
+    return fail(CSA_ERR_UNSUPPORTED, "%s: max_entries > %lld not built", name,
+                (long long)kBitmapSelectMaxEntries);
+  return check_cache(k_idx, name);
+}
+
+}  // namespace
+
+csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_cache_t* k_idx,
+                              const int32_t* seq_id, const int64_t* q_pos, int64_t T,
+                              int32_t H_I, int32_t c_I, int32_t m, int64_t max_entries,
+                              int32_t top_k, int32_t* idx_out, int32_t* count_out,
+                              float* score_out, void* ws, size_t ws_bytes, csa_stream_t stream) {
+  const char* name = "csa_indexer_topk";
+  csa_status_t st =
+      check_indexer_args(name, T, H_I, c_I, m, max_entries, top_k, w, idx_out, count_out, k_idx);
+  if (st != CSA_OK || T == 0) return st;
+  if (q_idx == nullptr) return fail(CSA_ERR_INVALID_ARG, "%s: q_idx is required", name);
+  if (!aligned16(q_idx)) return fail(CSA_ERR_INVALID_ARG, "%s: q_idx alignment", name);
+  const size_t need = csa_indexer_topk_workspace_size(T, max_entries, top_k);
+  if ((st = check_ws(ws, ws_bytes, need, name)) != CSA_OK) return st;
+  IndexerArgs ia;
+  ia.q_idx = (const __nv_bfloat16*)q_idx;
+  ia.w = w;
+  ia.keys = to_ref(k_idx);
+  ia.seq_id = seq_id;
+  ia.H_I = H_I;
+  ia.c_I = c_I;
+  return run_indexer_topk(ia, q_pos, T, m, max_entries, top_k, idx_out, count_out, score_out, ws,
+                          stream);
+}
+
+csa_status_t csa_quantize_mxfp4(const csa_bf16* x, int64_t n_vectors, int32_t dim, uint8_t* codes,
+                                uint8_t* scales, csa_stream_t stream) {
+  const char* name = "csa_quantize_mxfp4";
+  if (n_vectors < 0 || dim < 32 || dim % 32 != 0)
+    return fail(CSA_ERR_INVALID_ARG, "%s: need n_vectors >= 0 and dim a positive multiple of 32",
+                name);
+  if (n_vectors == 0) return CSA_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "%s: x, codes and scales are required", name);
+  if (!aligned16(x) || !aligned16(codes))
+    return fail(CSA_ERR_INVALID_ARG, "%s: x and codes must be 16-byte aligned", name);
+  Launch L{(cudaStream_t)stream};
+  return cuda_status(launch_mxfp4_quantize(L, (const __nv_bfloat16*)x, n_vectors * (dim / 32),
+                                           codes, scales),
+                     "csa_quantize_mxfp4 launch");
+}
+
+csa_status_t csa_indexer_topk_mxfp4(const uint8_t* q_codes, const uint8_t* q_scales,
+                                    const float* w, const csa_cache_t* k_codes,
+                                    const uint8_t* k_scales, const int32_t* seq_id,
+                                    const int64_t* q_pos, int64_t T, int32_t H_I, int32_t c_I,
+                                    int32_t m, int64_t max_entries, int32_t top_k,
+                                    int32_t* idx_out, int32_t* count_out, float* score_out,
+                                    void* ws, size_t ws_bytes, csa_stream_t stream) {
+  const char* name = "csa_indexer_topk_mxfp4";
+  csa_status_t st =
+      check_indexer_args(name, T, H_I, c_I, m, max_entries, top_k, w, idx_out, count_out, k_codes);
+  if (st != CSA_OK || T == 0) return st;
+  if (q_codes == nullptr || q_scales == nullptr || k_scales == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "%s: q_codes, q_scales and k_scales are required", name);
+  if (!aligned16(q_codes) || !aligned16(k_scales))
+    return fail(CSA_ERR_INVALID_ARG, "%s: q_codes and k_scales must be 16-byte aligned", name);
+  const size_t need = csa_indexer_topk_workspace_size(T, max_entries, top_k);
+  if ((st = check_ws(ws, ws_bytes, need, name)) != CSA_OK) return st;
+  IndexerArgs ia;
+  ia.q_idx = nullptr;
+  ia.w = w;
+  ia.keys = to_ref(k_codes);
+  ia.seq_id = seq_id;
+  ia.H_I = H_I;
+  ia.c_I = c_I;
+  ia.fp4 = 1;
+  ia.q_codes = q_codes;
+  ia.q_scales = q_scales;
+  ia.k_scales = k_scales;
+  return run_indexer_topk(ia, q_pos, T, m, max_entries, top_k, idx_out, count_out, score_out, ws,
+                          stream);
 }
 
 // ---- step 4 ------------------------------------------------------------------

@@ -1,0 +1,333 @@
+// 4-bit lightning indexer: quantization of indexer queries / keys to E2M1
+// codes with one power-of-two scale byte per 32 elements, and indexer scoring
+// straight from those codes.
+//
+// DeepSeek-V4 book, Ch.8 "A Cost Model for Long Context": "V4 compressed-entry
+// payload" (the indexer key is cached in FP4, half a byte per scalar) and
+// "Quantization scales and bounded tail buffers" (one 1-byte scale factor per
+// 32 elements); Ch.6 "Top-k selection and asymptotic scaling" (the indexer
+// scan runs in FP4).  The pages fix neither the element encoding nor the
+// scale rule; the format here is the OCP Microscaling one:
+//   * element: E2M1 (sign, 2 exponent bits with bias 1, 1 mantissa bit):
+//     magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6;
+//   * scale: byte b means 2^(b-127); for a block with largest magnitude amax,
+//     b - 127 = floor(log2 amax) - 2, clamped to [-127, 127] (-127 for an
+//     all-zero block);
+//   * element code: x / 2^(b-127) rounded to the nearest magnitude, ties to
+//     the even code, saturating at 6; the sign bit is x's sign bit;
+//   * packing: byte i holds element 2i (low nibble) and 2i+1 (high nibble);
+//     a vector of n elements is n/2 code bytes and n/32 scale bytes, the
+//     scales in an array of their own with the same row order.
+//
+// Scoring uses the score definition of Ch.6 "The lightning indexer" on the
+// dequantized values.  E2M1 magnitudes are exact fp16 numbers, so a code
+// nibble becomes an fp16 by a byte lookup (prmt); the tensor cores (mma.sync,
+// fp16 inputs, fp32 accumulation) form the dot product of each 32-element
+// scale block exactly (products are multiples of 1/4 below 36, sums below
+// 1152), and the block results are scaled by 2^(b_q - 127) * 2^(b_k - 127)
+// in fp32 before they are added.  The scorer is HBM-bound on the codes: 34
+// bytes per 64-dim key instead of 128.  Keys leave as the same
+// order-preserving 32-bit keys (plus, in decode mode, the same 4096-bin
+// histogram) as the bf16 scorer, so the top-k selection is shared.
+#include "kernels.h"
+
+namespace csa {
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// quantization: one thread per 32-element block
+// ---------------------------------------------------------------------------
+constexpr int kQuantThreads = 256;
+
+__device__ __forceinline__ uint32_t e2m1_code(float y) {
+  const float a = fabsf(y);
+  // nearest magnitude, ties to the even code (0, 1, 1.5 -> 2, 2 -> 4, 4 -> 6)
+  uint32_t c = a <= 0.25f ? 0u
+             : a < 0.75f  ? 1u
+             : a <= 1.25f ? 2u
+             : a < 1.75f  ? 3u
+             : a <= 2.5f  ? 4u
+             : a < 3.5f   ? 5u
+             : a <= 5.0f  ? 6u
+                          : 7u;
+  return c | ((__float_as_uint(y) >> 31) << 3);
+}
+
+__global__ void __launch_bounds__(kQuantThreads) mxfp4_quantize_kernel(
+    const __nv_bfloat16* __restrict__ x, int64_t n_blocks, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales) {
+  const int64_t b = (int64_t)blockIdx.x * kQuantThreads + threadIdx.x;
+  if (b >= n_blocks) return;
+  const uint4* src = reinterpret_cast<const uint4*>(x + b * 32);
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = __ldg(src + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = unpack_bf16(w[j]);
+      v[8 * i + 2 * j] = f.x;
+      v[8 * i + 2 * j + 1] = f.y;
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  // floor(log2 amax) from the exponent field; subnormal or zero amax clamps
+  // to the smallest scale
+  const int ef = (int)((__float_as_uint(amax) >> 23) & 0xffu);
+  int X = ef == 0 ? -127 : ef - 127 - 2;
+  X = X < -127 ? -127 : (X > 127 ? 127 : X);
+  const float inv = __uint_as_float((uint32_t)(127 - X) << 23);   // 2^-X, exact
+  uint32_t out[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) word |= e2m1_code(v[8 * i + j] * inv) << (4 * j);
+    out[i] = word;
+  }
+  *reinterpret_cast<uint4*>(codes + b * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+  scales[b] = (uint8_t)(X + 127);
+}
+
+// ---------------------------------------------------------------------------
+// scoring
+// ---------------------------------------------------------------------------
+constexpr int kFp4Warps = 8;
+constexpr int kFp4Threads = kFp4Warps * 32;
+// 16-key groups in flight per warp: about 16 code bytes per lane per group
+// (c_I = 64), fewer groups where the query fragments take more registers
+constexpr int fp4_unroll(int ci, int nt) { return (ci == 64 ? 8 : 4) / (nt >= 4 ? 2 : 1); }
+
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Eight E2M1 codes (nibble j = element j) -> fp16 pairs (0,1), (2,3), (4,5),
+// (6,7).  Every E2M1 value is an fp16 number whose low byte is zero; its high
+// byte comes from an 8-entry table indexed by the magnitude bits, the sign
+// bit is or-ed in, and the bytes are spread into 16-bit lanes.
+__device__ __forceinline__ uint4 e2m1x8_to_f16(uint32_t x) {
+  constexpr uint32_t kMagLo = 0x3E3C3800u;   // high bytes of 0, 0.5, 1, 1.5
+  constexpr uint32_t kMagHi = 0x46444240u;   // high bytes of 2, 3, 4, 6
+  const uint32_t n0 = x & 0xffffu, n1 = x >> 16;
+  const uint32_t b0 = __byte_perm(kMagLo, kMagHi, n0 & 0x7777u) |
+                      __byte_perm(0x00008000u, 0u, (n0 >> 3) & 0x1111u);
+  const uint32_t b1 = __byte_perm(kMagLo, kMagHi, n1 & 0x7777u) |
+                      __byte_perm(0x00008000u, 0u, (n1 >> 3) & 0x1111u);
+  return make_uint4(__byte_perm(b0, 0u, 0x1404u), __byte_perm(b0, 0u, 0x3424u),
+                    __byte_perm(b1, 0u, 0x1404u), __byte_perm(b1, 0u, 0x3424u));
+}
+
+// 2^(b - 127) for a scale byte b (b = 0: 2^-127, a subnormal)
+__device__ __forceinline__ float e8m0_value(uint32_t b) {
+  return b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);
+}
+
+// Per-lane query data, identical in every warp: lane (g, q) holds, for each
+// group of 8 heads nt and scale block v, the fp16 B fragments of head
+// nt*8 + g over dims [32v + 8q, 32v + 8q + 8), the scale factors of heads
+// nt*8 + 2q and nt*8 + 2q + 1 (the accumulator columns of the lane) and their
+// weights.  Heads >= H_I are zero.
+template <int CI, int NT>
+struct Fp4Query {
+  uint4 frag[NT][CI / 32][32];
+  float2 fac[NT][CI / 32][32];
+  float2 w[NT][32];
+};
+
+// The contraction dimension is permuted so that lane (g, q) of a key row
+// needs only 32-bit word 4v + q of the row's codes for scale block v (dims
+// [32v + 8q, 32v + 8q + 8)); the query fragments use the same permutation,
+// which leaves every dot product unchanged, and every k-column of the two
+// mma of block v falls inside block v.
+template <int CI, int NT, bool HIST>
+__global__ void __launch_bounds__(kFp4Threads) indexer_score_fp4_kernel(IndexerArgs a,
+                                                                        int64_t chunk) {
+  constexpr int KB = CI / 32;                  // scale blocks per vector
+  constexpr int kU = fp4_unroll(CI, NT);       // 16-key groups in flight per warp
+  __shared__ uint32_t sh_hist[HIST ? kHistBins : 1];
+  __shared__ Fp4Query<CI, NT> sq;
+  const int64_t tl = blockIdx.x;
+  const int64_t t = a.t_begin + tl;
+  const int64_t pos = a.q_pos ? __ldg(a.q_pos + t) : t;
+  int64_t n_elig = pos / a.m;
+  if (n_elig > a.max_entries) {
+    if (blockIdx.y == 0 && threadIdx.x == 0) report(a.err, kErrEligible, (int32_t)t, n_elig);
+    n_elig = a.max_entries;
+  }
+  const int64_t s_begin = (int64_t)blockIdx.y * chunk;
+  if (s_begin >= n_elig) return;
+  const int64_t s_end = min(s_begin + chunk, n_elig);
+  const int32_t seq = a.seq_id ? __ldg(a.seq_id + t) : 0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, q4 = lane & 3;
+
+  if (HIST)
+    for (int b = threadIdx.x; b < kHistBins; b += kFp4Threads) sh_hist[b] = 0;
+  for (int i = threadIdx.x; i < NT * KB * 32; i += kFp4Threads) {
+    const int L = i & 31, v = (i >> 5) % KB, nt = (i >> 5) / KB;
+    const int hg = nt * 8 + (L >> 2), h0 = nt * 8 + 2 * (L & 3);
+    uint32_t word = 0;
+    if (hg < a.H_I)
+      word = __ldg(reinterpret_cast<const uint32_t*>(a.q_codes + ((t * a.H_I + hg) * CI) / 2) +
+                   4 * v + (L & 3));
+    sq.frag[nt][v][L] = e2m1x8_to_f16(word);
+    const float f0 = h0 < a.H_I ? e8m0_value(__ldg(a.q_scales + (t * a.H_I + h0) * KB + v)) : 0.f;
+    const float f1 =
+        h0 + 1 < a.H_I ? e8m0_value(__ldg(a.q_scales + (t * a.H_I + h0 + 1) * KB + v)) : 0.f;
+    sq.fac[nt][v][L] = make_float2(f0, f1);
+    if (v == 0)
+      sq.w[nt][L] = make_float2(h0 < a.H_I ? __ldg(a.w + t * a.H_I + h0) : 0.f,
+                                h0 + 1 < a.H_I ? __ldg(a.w + t * a.H_I + h0 + 1) : 0.f);
+  }
+  __syncthreads();
+
+  const uint8_t* codes = reinterpret_cast<const uint8_t*>(a.keys.data);
+  uint32_t* out = a.keys_out + tl * a.key_stride;
+
+  for (int64_t s0 = s_begin + (int64_t)warp * 16 * kU; s0 < s_end;
+       s0 += (int64_t)kFp4Warps * 16 * kU) {
+    uint32_t kw[kU][2][KB];   // code words of rows g (h = 0) and g + 8 (h = 1)
+    uint32_t ks[kU][2];       // their scale bytes, KB per row
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t s = s0 + u * 16 + g + 8 * h;
+        int64_t row = -1;
+        if (s < s_end) row = cache_row(a.keys, seq, s, a.err, (int32_t)t);
+        const uint32_t* rw =
+            reinterpret_cast<const uint32_t*>(codes + (row >= 0 ? row : 0) * (CI / 2));
+#pragma unroll
+        for (int v = 0; v < KB; ++v) kw[u][h][v] = row >= 0 ? __ldg(rw + 4 * v + q4) : 0u;
+        if (CI == 64)
+          ks[u][h] = row >= 0 ? (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(a.k_scales) + row)
+                              : 0u;
+        else
+          ks[u][h] = row >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(a.k_scales) + row) : 0u;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      uint4 ka[2][KB];
+      float fk[2][KB];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int v = 0; v < KB; ++v) {
+          ka[h][v] = e2m1x8_to_f16(kw[u][h][v]);
+          fk[h][v] = e8m0_value((ks[u][h] >> (8 * v)) & 0xffu);
+        }
+      float sg = 0.f, s8 = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float dg0 = 0.f, dg1 = 0.f, d80 = 0.f, d81 = 0.f;   // rows g / g+8, heads h0 / h0+1
+#pragma unroll
+        for (int v = 0; v < KB; ++v) {
+          const uint4 bq = sq.frag[nt][v][lane];
+          float d[4] = {0.f, 0.f, 0.f, 0.f};
+          const uint32_t lo[4] = {ka[0][v].x, ka[1][v].x, ka[0][v].y, ka[1][v].y};
+          mma_f16_16816(d, lo, bq.x, bq.y);
+          const uint32_t hi[4] = {ka[0][v].z, ka[1][v].z, ka[0][v].w, ka[1][v].w};
+          mma_f16_16816(d, hi, bq.z, bq.w);
+          const float2 fq = sq.fac[nt][v][lane];
+          dg0 += d[0] * fq.x * fk[0][v];
+          dg1 += d[1] * fq.y * fk[0][v];
+          d80 += d[2] * fq.x * fk[1][v];
+          d81 += d[3] * fq.y * fk[1][v];
+        }
+        const float2 wv = sq.w[nt][lane];
+        sg = fmaf(wv.x, fmaxf(dg0, 0.f), sg);
+        sg = fmaf(wv.y, fmaxf(dg1, 0.f), sg);
+        s8 = fmaf(wv.x, fmaxf(d80, 0.f), s8);
+        s8 = fmaf(wv.y, fmaxf(d81, 0.f), s8);
+      }
+      sg += __shfl_xor_sync(0xffffffffu, sg, 1);
+      s8 += __shfl_xor_sync(0xffffffffu, s8, 1);
+      sg += __shfl_xor_sync(0xffffffffu, sg, 2);
+      s8 += __shfl_xor_sync(0xffffffffu, s8, 2);
+      const int64_t s = s0 + u * 16 + g + (q4 == 1 ? 8 : 0);
+      const bool valid = q4 < 2 && s < s_end;
+      const uint32_t key = score_key(q4 == 0 ? sg : s8);
+      if (valid) {
+        out[s] = key;
+        if (HIST) atomicAdd(&sh_hist[key >> 20], 1u);
+      }
+    }
+  }
+  if (HIST) {
+    __syncthreads();
+    uint32_t* gh = a.hist + tl * kHistBins;
+    for (int b = threadIdx.x; b < kHistBins; b += kFp4Threads) {
+      const uint32_t v = sh_hist[b];
+      if (v) atomicAdd(gh + b, v);
+    }
+  }
+}
+
+template <int CI, int NT, bool HIST>
+void launch_score_fp4(const Launch& L, const IndexerArgs& a, int64_t t_count) {
+  constexpr int kU = fp4_unroll(CI, NT);
+  int dev = 0, sms = 148, per_sm = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, indexer_score_fp4_kernel<CI, NT, HIST>,
+                                                kFp4Threads, 0);
+  if (per_sm < 1) per_sm = 1;
+  // chunks per query so that the grid fills whole resident waves
+  const int64_t wave = (int64_t)sms * per_sm;
+  int64_t per_q = wave / t_count;
+  if (per_q < 1) per_q = 1;
+  const int64_t min_chunk = 16 * kFp4Warps * kU;   // one pass of the warps
+  int64_t chunk = (a.max_entries + per_q - 1) / per_q;
+  chunk = (chunk + min_chunk - 1) / min_chunk * min_chunk;
+  if (chunk < min_chunk) chunk = min_chunk;
+  per_q = (a.max_entries + chunk - 1) / chunk;
+  const dim3 grid((unsigned)t_count, (unsigned)per_q);
+  indexer_score_fp4_kernel<CI, NT, HIST><<<grid, kFp4Threads, 0, L.stream>>>(a, chunk);
+}
+
+}  // namespace
+
+cudaError_t launch_mxfp4_quantize(const Launch& L, const __nv_bfloat16* x, int64_t n_blocks,
+                                  uint8_t* codes, uint8_t* scales) {
+  if (n_blocks == 0) return cudaSuccess;
+  L.begin(kKernelQuantize);
+  const unsigned blocks = (unsigned)((n_blocks + kQuantThreads - 1) / kQuantThreads);
+  mxfp4_quantize_kernel<<<blocks, kQuantThreads, 0, L.stream>>>(x, n_blocks, codes, scales);
+  return L.end(kKernelQuantize);
+}
+
+cudaError_t launch_indexer_scores_fp4(const Launch& L, const IndexerArgs& a, int64_t t_count) {
+  if (t_count == 0 || a.max_entries == 0) return cudaSuccess;
+  const int nt = (a.H_I + 7) / 8;
+  const int ntb = nt <= 1 ? 1 : nt <= 2 ? 2 : nt <= 4 ? 4 : 8;
+  const bool hist = a.hist != nullptr;
+  L.begin(kKernelIndexerScore);
+#define CSA_FP4_CASE(CI_, NT_)                                             \
+  if (a.c_I == CI_ && ntb == NT_) {                                        \
+    if (hist) launch_score_fp4<CI_, NT_, true>(L, a, t_count);             \
+    else launch_score_fp4<CI_, NT_, false>(L, a, t_count);                 \
+  }
+  CSA_FP4_CASE(64, 1)
+  CSA_FP4_CASE(64, 2)
+  CSA_FP4_CASE(64, 4)
+  CSA_FP4_CASE(64, 8)
+  CSA_FP4_CASE(128, 1)
+  CSA_FP4_CASE(128, 2)
+  CSA_FP4_CASE(128, 4)
+  CSA_FP4_CASE(128, 8)
+#undef CSA_FP4_CASE
+  return L.end(kKernelIndexerScore);
+}
+
+}  // namespace csa

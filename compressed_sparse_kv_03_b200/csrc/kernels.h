@@ -11,7 +11,8 @@ enum KernelId : int32_t {
   kKernelAttention = 2,
   kKernelMerge = 3,
   kKernelCompress = 4,
-  kNumKernelIds = 5,
+  kKernelQuantize = 5,
+  kNumKernelIds = 6,
 };
 
 // Per-call launch context: the stream plus the timing / launch-count hooks.
@@ -86,6 +87,13 @@ struct IndexerArgs {
   uint32_t* hist;               // [T_chunk, kHistBins] (zeroed) or null
   uint32_t* work;               // zeroed work counter of the tcgen05 scorer
   WsHeader* err;
+  // 4-bit mode (fp4 = 1): q_codes [T, H_I, c_I/2] and q_scales [T, H_I, c_I/32]
+  // replace q_idx; keys.data holds rows of c_I/2 code bytes and k_scales rows
+  // of c_I/32 scale bytes at the same physical row index
+  int fp4 = 0;
+  const uint8_t* q_codes = nullptr;
+  const uint8_t* q_scales = nullptr;
+  const uint8_t* k_scales = nullptr;
 };
 cudaError_t launch_indexer_scores(const Launch& L, const IndexerArgs& a, int64_t t_count);
 // tcgen05 + TMA scoring path (c_I = 64, H_I <= 16, pages a multiple of 64 rows)
@@ -95,6 +103,11 @@ cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int6
 // H_I in {4, 8, 16}; blocks of 128 / H_I queries share each key tile
 bool tc_indexer_prefill_supported(const IndexerArgs& a, int64_t t_count);
 cudaError_t launch_indexer_scores_tc_prefill(const Launch& L, const IndexerArgs& a, int64_t t_count);
+// 4-bit scorer (E2M1 codes with one scale byte per 32 elements): see indexer_fp4.cu
+cudaError_t launch_indexer_scores_fp4(const Launch& L, const IndexerArgs& a, int64_t t_count);
+// [n_blocks * 32] bf16 -> n_blocks * 16 code bytes + n_blocks scale bytes
+cudaError_t launch_mxfp4_quantize(const Launch& L, const __nv_bfloat16* x, int64_t n_blocks,
+                                  uint8_t* codes, uint8_t* scales);
 
 struct SelectArgs {
   const uint32_t* keys;         // [T_chunk, key_stride]

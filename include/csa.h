@@ -89,7 +89,7 @@ uint64_t csa_launch_count(void);
  * are non-NULL, the library records them on the call's stream immediately
  * before and after every launch of kernel `kernel_id`.  Pass NULLs to detach.
  * kernel_id: 0 = indexer scoring, 1 = top-k selection, 2 = attention,
- * 3 = split merge, 4 = compression.
+ * 3 = split merge, 4 = compression, 5 = 4-bit quantization.
  */
 csa_status_t csa_set_timing_events(int32_t kernel_id, void* ev_begin, void* ev_end);
 
@@ -247,6 +247,54 @@ csa_status_t csa_indexer_topk(const csa_bf16* q_idx, const float* w, const csa_c
                               int32_t H_I, int32_t c_I, int32_t m, int64_t max_entries,
                               int32_t top_k, int32_t* idx_out, int32_t* count_out,
                               float* score_out, void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/*
+ * 4-bit indexer storage (Ch.8 "A Cost Model for Long Context": "V4
+ * compressed-entry payload" keeps the indexer keys in FP4, half a byte per
+ * scalar; "Quantization scales and bounded tail buffers": one 1-byte scale per
+ * 32 elements; Ch.6 "Top-k selection and asymptotic scaling": the indexer
+ * scan runs in FP4).  The pages fix no encoding; the one used is the OCP
+ * Microscaling (MXFP4) format:
+ *   element  E2M1 code: bit 3 sign, bits 2..1 exponent (bias 1), bit 0
+ *            mantissa; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6
+ *   scale    byte b = X + 127 means 2^X; X = floor(log2 amax) - 2 for the
+ *            block's largest magnitude amax, clamped to [-127, 127]
+ *            (-127 for an all-zero block)
+ *   code     x / 2^X rounded to the nearest magnitude, ties to the even code
+ *            (mantissa bit 0), saturating at 6; sign bit = sign bit of x
+ *   packing  byte i of a vector holds element 2i in its low nibble and
+ *            element 2i+1 in its high nibble; scales in their own array
+ *
+ * csa_quantize_mxfp4 -- quantize n_vectors rows of dim bf16 values:
+ *   x       [n_vectors, dim] bf16 (16-byte aligned); dim % 32 == 0
+ *   codes   [n_vectors, dim/2] uint8 out (16-byte aligned)
+ *   scales  [n_vectors, dim/32] uint8 out
+ * Bit-exact; results for non-finite inputs are unspecified.
+ */
+csa_status_t csa_quantize_mxfp4(const csa_bf16* x, int64_t n_vectors, int32_t dim, uint8_t* codes,
+                                uint8_t* scales, csa_stream_t stream);
+
+/*
+ * csa_indexer_topk_mxfp4 -- csa_indexer_topk on 4-bit queries and keys: the
+ * same score definition applied to the dequantized values (each 32-element
+ * block's dot product is exact; the blocks are scaled and summed, and the
+ * heads weighted and summed, in fp32), the same selection rules, workspace
+ * (csa_indexer_topk_workspace_size) and outputs.
+ *   q_codes   [T, H_I, c_I/2] uint8 (16-byte aligned), q_scales [T, H_I, c_I/32]
+ *   k_codes   cache whose rows are c_I/2 code bytes (data 16-byte aligned)
+ *   k_scales  [k_codes->n_rows, c_I/32] uint8 (16-byte aligned): the scale bytes
+ *             of physical row r of k_codes are row r of k_scales
+ * c_I in {64, 128}; H_I <= 64.  Scale bytes 0 and 255 (2^-127 and the
+ * E8M0 NaN) are outside the supported range: csa_quantize_mxfp4 produces 0
+ * only for blocks whose largest magnitude is below 2^-124.
+ */
+csa_status_t csa_indexer_topk_mxfp4(const uint8_t* q_codes, const uint8_t* q_scales,
+                                    const float* w, const csa_cache_t* k_codes,
+                                    const uint8_t* k_scales, const int32_t* seq_id,
+                                    const int64_t* q_pos, int64_t T, int32_t H_I, int32_t c_I,
+                                    int32_t m, int64_t max_entries, int32_t top_k,
+                                    int32_t* idx_out, int32_t* count_out, float* score_out,
+                                    void* ws, size_t ws_bytes, csa_stream_t stream);
 
 /* ---- step 4: attention ---------------------------------------------------- */
 /*

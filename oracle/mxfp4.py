@@ -79,20 +79,18 @@ def mxfp4_scale_exponent(block):
 
 def mxfp4_quantize(x):
     """Quantize rows of x ([..., n], n a multiple of 32) to packed E2M1 codes
-    [..., n/2] (uint8, reading Q4) and E8M0 scale bytes [..., n/32]."""
+    [..., n/2] (uint8, reading Q4) and E8M0 scale bytes [..., n/32]: per block
+    of 32 the shared exponent of reading Q2, then reading Q3 per element."""
     x = np.asarray(x, dtype=np.float64)
     n = x.shape[-1]
     assert n % BLOCK == 0, "the vector length must be a multiple of 32"
-    flat = x.reshape(-1, n)
-    codes = np.zeros((flat.shape[0], n), dtype=np.uint8)
-    scales = np.zeros((flat.shape[0], n // BLOCK), dtype=np.uint8)
-    for r in range(flat.shape[0]):
-        for b in range(n // BLOCK):
-            blk = flat[r, b * BLOCK:(b + 1) * BLOCK]
-            X = mxfp4_scale_exponent(blk)
-            scales[r, b] = X + 127
-            codes[r, b * BLOCK:(b + 1) * BLOCK] = e2m1_encode(blk / 2.0 ** X)
+    blocks = x.reshape(-1, BLOCK)                            # one row per scale block
+    amax = np.abs(blocks).max(axis=1)
+    _, e = np.frexp(amax)                                    # amax = f * 2^e, f in [0.5, 1)
+    X = np.where(amax == 0.0, -127, np.clip(e - 1 - E2M1_EMAX, -127, 127)).astype(np.int64)
+    codes = e2m1_encode(blocks / np.ldexp(1.0, X)[:, None]).reshape(-1, n)
     packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    scales = (X + 127).astype(np.uint8)
     return packed.reshape(x.shape[:-1] + (n // 2,)), scales.reshape(x.shape[:-1] + (n // BLOCK,))
 
 

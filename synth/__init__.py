@@ -109,8 +109,12 @@ CFG_MIXED = MixedDecode("mixed_decode_B16_N256K_1M", B=16, N_lo=1 << 18, N_hi=1 
                         d=128, H_I=8, c_I=64, m_csa=4, m_hca=128, k=2048, W=128,
                         lam=INV_SQRT_128, page_size=64, seed=4)
 
+# The 128K decode with the indexer keys and queries held in 4-bit storage
+# (same seeded inputs; the keys are quantized when the cache is built).
+CFG_DECODE_128K_MXFP4 = dataclasses.replace(CFG_DECODE_128K, name="csa_decode_B64_N131072_mxfp4_indexer")
+
 WORKLOADS = {c.name: c for c in (CFG_PREFILL_4K, CFG_DECODE_128K, CFG_PREFILL_64K, CFG_HCA_1M,
-                                 CFG_MIXED)}
+                                 CFG_MIXED, CFG_DECODE_128K_MXFP4)}
 
 
 # ---------------------------------------------------------------------------
@@ -261,3 +265,15 @@ def random_topk_lists(g, T, k, n_eligible):
             idx[t, :c] = sel.to(torch.int32)
         cnt[t] = c
     return idx, cnt
+
+
+def fp4_codes(g, rows_shape, dim, scale_lo=124, scale_hi=129):
+    """Random 4-bit storage of vectors of `dim` elements: uniform code bytes
+    (every E2M1 code equally likely in each nibble) [*rows_shape, dim/2] and
+    uniform scale bytes in [scale_lo, scale_hi) [*rows_shape, dim/32]
+    (uint8).  Raw bytes only: both sides decode them."""
+    shape = tuple(rows_shape)
+    codes = torch.randint(0, 256, shape + (dim // 2,), generator=g, dtype=torch.int32).to(torch.uint8)
+    scales = torch.randint(scale_lo, scale_hi, shape + (dim // 32,), generator=g,
+                           dtype=torch.int32).to(torch.uint8)
+    return codes, scales

@@ -147,3 +147,31 @@ def test_product_path_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_mxfp4_calls_reject_bad_arguments_without_launching(lib):
+    from compressed_sparse_kv_03_b200._lib import CacheT
+    before = lib.csa_launch_count()
+    buf = (C.c_uint8 * 4096)()
+    p = C.c_void_p((C.addressof(buf) + 255) // 256 * 256)
+    # quantize: dim not a multiple of 32, missing output, misaligned codes
+    assert lib.csa_quantize_mxfp4(p, 4, 48, p, p, None) == 1
+    assert b"multiple of 32" in lib.csa_last_error()
+    assert lib.csa_quantize_mxfp4(p, 4, 64, None, p, None) == 1
+    assert lib.csa_quantize_mxfp4(p, 4, 64, C.c_void_p(p.value + 4), p, None) == 1
+    assert lib.csa_quantize_mxfp4(p, 0, 64, None, None, None) == 0   # nothing to do
+    cache = CacheT(p.value, 16, 16, None, 0, 0)
+    args = [p, p, p, C.byref(cache), p, None, None, 8, 8, 64, 4, 16, 4, p, p, None, p, 1 << 20, None]
+    # c_I not built
+    a = list(args); a[9] = 96
+    assert lib.csa_indexer_topk_mxfp4(*a) == 2
+    # missing scales
+    a = list(args); a[4] = None
+    assert lib.csa_indexer_topk_mxfp4(*a) == 1 and b"k_scales" in lib.csa_last_error()
+    # H_I above 64
+    a = list(args); a[8] = 65
+    assert lib.csa_indexer_topk_mxfp4(*a) == 2
+    # workspace too small
+    a = list(args); a[17] = 256
+    assert lib.csa_indexer_topk_mxfp4(*a) == 5
+    assert lib.csa_launch_count() == before

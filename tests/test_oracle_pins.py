@@ -558,3 +558,17 @@ def test_mxfp4_indexer_scores_brute_force():
             dot = sum(val(qp[h], qs[h], r) * val(kp[s], ks[s], r) for r in range(c))
             want += w[h] * max(dot, 0.0)
         assert got[s] == pytest.approx(want, rel=1e-12, abs=1e-12)
+
+
+def test_mxfp4_quantize_is_blockwise_definition():
+    # each 32-element block: scale byte from its own maximum, codes of x / 2^X
+    x = oracle.bf16_round(rng.standard_normal((7, 96)) * 2.0 ** rng.integers(-60, 60, (7, 1)))
+    x[0, :32] = 0.0
+    packed, scales = ofp4.mxfp4_quantize(x)
+    for r in range(7):
+        for b in range(3):
+            blk = x[r, 32 * b:32 * b + 32]
+            X = ofp4.mxfp4_scale_exponent(blk)
+            assert scales[r, b] == X + 127
+            codes = ofp4.e2m1_encode(blk / 2.0 ** X)
+            assert np.array_equal(packed[r, 16 * b:16 * b + 16], codes[0::2] | (codes[1::2] << 4))

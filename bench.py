@@ -116,8 +116,9 @@ class CsaDecode:
 class CsaDecodeMxfp4(CsaDecode):
     """CSA decode with the 4-bit indexer: the indexer-key cache holds E2M1
     codes plus one scale byte per 32 elements (quantized once, when the cache
-    is built); a step quantizes the new indexer queries, scores and selects
-    from the codes (csa_indexer_topk_mxfp4), then attends as the bf16 step."""
+    is built); a step scores and selects from the codes with the new bf16
+    indexer queries quantized inside the scorer (csa_indexer_topk_mxfp4),
+    then attends as the bf16 step."""
 
     def __init__(self, cfg, seed_offset=0):
         super().__init__(cfg, seed_offset)
@@ -125,7 +126,6 @@ class CsaDecodeMxfp4(CsaDecode):
         kc, ks = csa.quantize_mxfp4(self.d.pop("kI_comp"))
         self.kI = csa.Cache(kc.view(-1, kc.shape[-1]), seq_stride=self.S)
         self.kI_scales = ks.view(-1, ks.shape[-1])
-        self.qc, self.qs = csa.quantize_mxfp4(self.d["qI"])
         torch.cuda.synchronize()
         sel_rows = min(cfg.k, self.S) + min(cfg.W, cfg.N + 1)
         self.dominant_bytes = cfg.B * self.S * (cfg.c_I // 2 + cfg.c_I // 32)
@@ -134,8 +134,7 @@ class CsaDecodeMxfp4(CsaDecode):
 
     def step(self):
         csa, cfg, d = self.csa, self.cfg, self.d
-        csa.quantize_mxfp4(d["qI"], out=(self.qc, self.qs))
-        csa.indexer_topk_mxfp4(self.qc, self.qs, d["w"], self.kI, self.kI_scales, cfg.m, cfg.k,
+        csa.indexer_topk_mxfp4(d["qI"], d["w"], self.kI, self.kI_scales, cfg.m, cfg.k,
                                seq_id=self.seq_id, q_pos=d["pos"], max_entries=self.S, ws=self.ws_i,
                                out=(self.idx, self.cnt, None))
         csa.sparse_attn_decode(d["q"], self.kv, d["win"], d["win_len"], self.idx, self.cnt, cfg.lam,

@@ -62,9 +62,8 @@ SIGNATURES = {
     "csa_indexer_topk": (C.c_int, [_vp, _vp, C.POINTER(CacheT), _vp, _vp, _i64, _i32, _i32, _i32,
                                    _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "csa_quantize_mxfp4": (C.c_int, [_vp, _i64, _i32, _vp, _vp, _vp]),
-    "csa_indexer_topk_mxfp4": (C.c_int, [_vp, _vp, _vp, C.POINTER(CacheT), _vp, _vp, _vp, _i64,
-                                         _i32, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _sz,
-                                         _vp]),
+    "csa_indexer_topk_mxfp4": (C.c_int, [_vp, _vp, C.POINTER(CacheT), _vp, _vp, _vp, _i64, _i32,
+                                         _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "csa_sparse_attn_prefill": (C.c_int, [_vp, _vp, _i64, _vp, _vp, _vp, _i64, _i32, _i32, _i32,
                                           _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "csa_sparse_attn_decode": (C.c_int, [_vp, C.POINTER(CacheT), _vp, _vp, _vp, _vp, _i32, _i32,

@@ -261,24 +261,20 @@ def quantize_mxfp4(x, *, stream=None, out=None):
     return codes, scales
 
 
-def indexer_topk_mxfp4(q_codes, q_scales, w, keys: Cache, k_scales, m, top_k, *, seq_id=None,
-                       q_pos=None, max_entries=None, return_scores=False, ws=None, stream=None,
-                       out=None):
-    """Steps 2-3 on 4-bit operands: q_codes [T, H_I, c_I/2] / q_scales
-    [T, H_I, c_I/32] from quantize_mxfp4, keys.data [rows, c_I/2] uint8 codes
-    with k_scales [rows, c_I/32] uint8 (same rows, same paging).
+def indexer_topk_mxfp4(q_idx, w, keys: Cache, k_scales, m, top_k, *, seq_id=None, q_pos=None,
+                       max_entries=None, return_scores=False, ws=None, stream=None, out=None):
+    """Steps 2-3 with the indexer keys in 4-bit storage: keys.data [rows,
+    c_I/2] uint8 codes with k_scales [rows, c_I/32] uint8 (same rows, same
+    paging), e.g. from quantize_mxfp4; the bf16 queries q_idx [T, H_I, c_I]
+    are quantized to the same format inside the call.
     Returns (idx [T, top_k] int32, count [T] int32[, scores [T, top_k] fp32])."""
-    _need(q_codes, "q_codes", torch.uint8, 3)
-    T, H_I, half = q_codes.shape
-    c_I = 2 * half
-    dev = q_codes.device
-    _need(q_scales, "q_scales", torch.uint8, 3, dev)
-    if tuple(q_scales.shape) != (T, H_I, c_I // 32):
-        raise ValueError("q_scales must be [T, H_I, c_I/32]")
+    _need(q_idx, "q_idx", torch.bfloat16, 3)
+    T, H_I, c_I = q_idx.shape
+    dev = q_idx.device
     _need(w, "w", torch.float32, 2, dev)
     if tuple(w.shape) != (T, H_I):
         raise ValueError("w must be [T, H_I]")
-    if keys.dim != half:
+    if keys.dim * 2 != c_I:
         raise ValueError("key code rows must hold c_I/2 bytes")
     _need(k_scales, "k_scales", torch.uint8, 2, dev)
     if tuple(k_scales.shape) != (keys.data.shape[0], c_I // 32):
@@ -301,10 +297,9 @@ def indexer_topk_mxfp4(q_codes, q_scales, w, keys: Cache, k_scales, m, top_k, *,
     lib = load()
     wsp, wsb = _ws(ws, dev).get(lib.csa_indexer_topk_workspace_size(T, max_entries, top_k))
     kc = keys.c(torch.uint8)
-    check(lib.csa_indexer_topk_mxfp4(_ptr(q_codes), _ptr(q_scales), _ptr(w), C.byref(kc),
-                                     _ptr(k_scales), _ptr(seq_id), _ptr(q_pos), T, H_I, c_I, m,
-                                     max_entries, top_k, _ptr(idx), _ptr(cnt), _ptr(sco), wsp, wsb,
-                                     _stream(stream)))
+    check(lib.csa_indexer_topk_mxfp4(_ptr(q_idx), _ptr(w), C.byref(kc), _ptr(k_scales),
+                                     _ptr(seq_id), _ptr(q_pos), T, H_I, c_I, m, max_entries, top_k,
+                                     _ptr(idx), _ptr(cnt), _ptr(sco), wsp, wsb, _stream(stream)))
     return (idx, cnt, sco) if return_scores else (idx, cnt)
 
 

@@ -513,33 +513,31 @@ csa_status_t csa_quantize_mxfp4(const csa_bf16* x, int64_t n_vectors, int32_t di
                      "csa_quantize_mxfp4 launch");
 }
 
-csa_status_t csa_indexer_topk_mxfp4(const uint8_t* q_codes, const uint8_t* q_scales,
-                                    const float* w, const csa_cache_t* k_codes,
-                                    const uint8_t* k_scales, const int32_t* seq_id,
-                                    const int64_t* q_pos, int64_t T, int32_t H_I, int32_t c_I,
-                                    int32_t m, int64_t max_entries, int32_t top_k,
-                                    int32_t* idx_out, int32_t* count_out, float* score_out,
-                                    void* ws, size_t ws_bytes, csa_stream_t stream) {
+csa_status_t csa_indexer_topk_mxfp4(const csa_bf16* q_idx, const float* w,
+                                    const csa_cache_t* k_codes, const uint8_t* k_scales,
+                                    const int32_t* seq_id, const int64_t* q_pos, int64_t T,
+                                    int32_t H_I, int32_t c_I, int32_t m, int64_t max_entries,
+                                    int32_t top_k, int32_t* idx_out, int32_t* count_out,
+                                    float* score_out, void* ws, size_t ws_bytes,
+                                    csa_stream_t stream) {
   const char* name = "csa_indexer_topk_mxfp4";
   csa_status_t st =
       check_indexer_args(name, T, H_I, c_I, m, max_entries, top_k, w, idx_out, count_out, k_codes);
   if (st != CSA_OK || T == 0) return st;
-  if (q_codes == nullptr || q_scales == nullptr || k_scales == nullptr)
-    return fail(CSA_ERR_INVALID_ARG, "%s: q_codes, q_scales and k_scales are required", name);
-  if (!aligned16(q_codes) || !aligned16(k_scales))
-    return fail(CSA_ERR_INVALID_ARG, "%s: q_codes and k_scales must be 16-byte aligned", name);
+  if (q_idx == nullptr || k_scales == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "%s: q_idx and k_scales are required", name);
+  if (!aligned16(q_idx) || !aligned16(k_scales))
+    return fail(CSA_ERR_INVALID_ARG, "%s: q_idx and k_scales must be 16-byte aligned", name);
   const size_t need = csa_indexer_topk_workspace_size(T, max_entries, top_k);
   if ((st = check_ws(ws, ws_bytes, need, name)) != CSA_OK) return st;
   IndexerArgs ia;
-  ia.q_idx = nullptr;
+  ia.q_idx = (const __nv_bfloat16*)q_idx;
   ia.w = w;
   ia.keys = to_ref(k_codes);
   ia.seq_id = seq_id;
   ia.H_I = H_I;
   ia.c_I = c_I;
   ia.fp4 = 1;
-  ia.q_codes = q_codes;
-  ia.q_scales = q_scales;
   ia.k_scales = k_scales;
   return run_indexer_topk(ia, q_pos, T, m, max_entries, top_k, idx_out, count_out, score_out, ws,
                           stream);

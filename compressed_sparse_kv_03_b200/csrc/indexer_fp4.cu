@@ -54,16 +54,16 @@ __device__ __forceinline__ uint32_t e2m1_code(float y) {
   return c | ((__float_as_uint(y) >> 31) << 3);
 }
 
-__global__ void __launch_bounds__(kQuantThreads) mxfp4_quantize_kernel(
-    const __nv_bfloat16* __restrict__ x, int64_t n_blocks, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ scales) {
-  const int64_t b = (int64_t)blockIdx.x * kQuantThreads + threadIdx.x;
-  if (b >= n_blocks) return;
-  const uint4* src = reinterpret_cast<const uint4*>(x + b * 32);
+// One 32-element block: its four code words (nibble j of word i = element
+// 8i + j) and its scale byte.  The standalone quantizer and the scorer's
+// query prologue both use this, so their codes are identical.
+__device__ __forceinline__ uint32_t quantize_block(const __nv_bfloat16* __restrict__ src,
+                                                   uint32_t (&out)[4]) {
+  const uint4* p = reinterpret_cast<const uint4*>(src);
   float v[32];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint4 u = __ldg(src + i);
+    const uint4 u = __ldg(p + i);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -81,7 +81,6 @@ __global__ void __launch_bounds__(kQuantThreads) mxfp4_quantize_kernel(
   int X = ef == 0 ? -127 : ef - 127 - 2;
   X = X < -127 ? -127 : (X > 127 ? 127 : X);
   const float inv = __uint_as_float((uint32_t)(127 - X) << 23);   // 2^-X, exact
-  uint32_t out[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     uint32_t word = 0;
@@ -89,8 +88,18 @@ __global__ void __launch_bounds__(kQuantThreads) mxfp4_quantize_kernel(
     for (int j = 0; j < 8; ++j) word |= e2m1_code(v[8 * i + j] * inv) << (4 * j);
     out[i] = word;
   }
+  return (uint32_t)(X + 127);
+}
+
+__global__ void __launch_bounds__(kQuantThreads) mxfp4_quantize_kernel(
+    const __nv_bfloat16* __restrict__ x, int64_t n_blocks, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales) {
+  const int64_t b = (int64_t)blockIdx.x * kQuantThreads + threadIdx.x;
+  if (b >= n_blocks) return;
+  uint32_t out[4];
+  const uint32_t sb = quantize_block(x + b * 32, out);
   *reinterpret_cast<uint4*>(codes + b * 16) = make_uint4(out[0], out[1], out[2], out[3]);
-  scales[b] = (uint8_t)(X + 127);
+  scales[b] = (uint8_t)sb;
 }
 
 // ---------------------------------------------------------------------------
@@ -98,9 +107,10 @@ __global__ void __launch_bounds__(kQuantThreads) mxfp4_quantize_kernel(
 // ---------------------------------------------------------------------------
 constexpr int kFp4Warps = 8;
 constexpr int kFp4Threads = kFp4Warps * 32;
-// 16-key groups in flight per warp: about 16 code bytes per lane per group
-// (c_I = 64), fewer groups where the query fragments take more registers
-constexpr int fp4_unroll(int ci, int nt) { return (ci == 64 ? 8 : 4) / (nt >= 4 ? 2 : 1); }
+// 16-key groups per register batch (two batches in flight per warp): about
+// 16 code bytes per lane per group at c_I = 64, fewer groups where the query
+// fragments take more registers
+constexpr int fp4_unroll(int ci, int nt) { return (ci == 64 ? 4 : 2) / (nt >= 4 ? 2 : 1); }
 
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                               uint32_t b1) {
@@ -144,18 +154,113 @@ struct Fp4Query {
   float2 w[NT][32];
 };
 
+// Code words and scale bytes of kU 16-key groups: rows g (h = 0) and g + 8
+// (h = 1) of each group, for lane (g, q).
+template <int CI, int kU>
+struct KeyBatch {
+  uint32_t kw[kU][2][CI / 32];
+  uint32_t ks[kU][2];
+};
+
+template <int CI, int kU>
+__device__ __forceinline__ void load_batch(KeyBatch<CI, kU>& kb, const IndexerArgs& a,
+                                           const uint8_t* codes, int32_t seq, int64_t s0,
+                                           int64_t s_end, int64_t t, int g, int q4) {
+  constexpr int KB = CI / 32;
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t s = s0 + u * 16 + g + 8 * h;
+      int64_t row = -1;
+      if (s < s_end) row = cache_row(a.keys, seq, s, a.err, (int32_t)t);
+      const uint32_t* rw =
+          reinterpret_cast<const uint32_t*>(codes + (row >= 0 ? row : 0) * (CI / 2));
+#pragma unroll
+      for (int v = 0; v < KB; ++v) kb.kw[u][h][v] = row >= 0 ? __ldg(rw + 4 * v + q4) : 0u;
+      if (CI == 64)
+        kb.ks[u][h] =
+            row >= 0 ? (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(a.k_scales) + row) : 0u;
+      else
+        kb.ks[u][h] = row >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(a.k_scales) + row) : 0u;
+    }
+  }
+}
+
 // The contraction dimension is permuted so that lane (g, q) of a key row
 // needs only 32-bit word 4v + q of the row's codes for scale block v (dims
 // [32v + 8q, 32v + 8q + 8)); the query fragments use the same permutation,
 // which leaves every dot product unchanged, and every k-column of the two
 // mma of block v falls inside block v.
+template <int CI, int NT, bool HIST, int kU>
+__device__ __forceinline__ void score_batch(const KeyBatch<CI, kU>& kb,
+                                            const Fp4Query<CI, NT>& sq, uint32_t* sh_hist,
+                                            uint32_t* out, int64_t s0, int64_t s_end, int lane,
+                                            int g, int q4) {
+  constexpr int KB = CI / 32;
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    uint4 ka[2][KB];
+    float fk[2][KB];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int v = 0; v < KB; ++v) {
+        ka[h][v] = e2m1x8_to_f16(kb.kw[u][h][v]);
+        fk[h][v] = e8m0_value((kb.ks[u][h] >> (8 * v)) & 0xffu);
+      }
+    float sg = 0.f, s8 = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float dg0 = 0.f, dg1 = 0.f, d80 = 0.f, d81 = 0.f;   // rows g / g+8, heads h0 / h0+1
+#pragma unroll
+      for (int v = 0; v < KB; ++v) {
+        const uint4 bq = sq.frag[nt][v][lane];
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t lo[4] = {ka[0][v].x, ka[1][v].x, ka[0][v].y, ka[1][v].y};
+        mma_f16_16816(d, lo, bq.x, bq.y);
+        const uint32_t hi[4] = {ka[0][v].z, ka[1][v].z, ka[0][v].w, ka[1][v].w};
+        mma_f16_16816(d, hi, bq.z, bq.w);
+        const float2 fq = sq.fac[nt][v][lane];
+        dg0 += d[0] * fq.x * fk[0][v];
+        dg1 += d[1] * fq.y * fk[0][v];
+        d80 += d[2] * fq.x * fk[1][v];
+        d81 += d[3] * fq.y * fk[1][v];
+      }
+      const float2 wv = sq.w[nt][lane];
+      sg = fmaf(wv.x, fmaxf(dg0, 0.f), sg);
+      sg = fmaf(wv.y, fmaxf(dg1, 0.f), sg);
+      s8 = fmaf(wv.x, fmaxf(d80, 0.f), s8);
+      s8 = fmaf(wv.y, fmaxf(d81, 0.f), s8);
+    }
+    sg += __shfl_xor_sync(0xffffffffu, sg, 1);
+    s8 += __shfl_xor_sync(0xffffffffu, s8, 1);
+    sg += __shfl_xor_sync(0xffffffffu, sg, 2);
+    s8 += __shfl_xor_sync(0xffffffffu, s8, 2);
+    const int64_t s = s0 + u * 16 + g + (q4 == 1 ? 8 : 0);
+    const bool valid = q4 < 2 && s < s_end;
+    const uint32_t key = score_key(q4 == 0 ? sg : s8);
+    if (valid) {
+      out[s] = key;
+      if (HIST) atomicAdd(&sh_hist[key >> 20], 1u);
+    }
+  }
+}
+
+// One CTA scores a chunk of one query's keys.  The prologue quantizes the
+// query's bf16 heads (the same block quantizer as csa_quantize_mxfp4) and
+// lays out its fragments; each warp then walks batches of kU 16-key groups,
+// loading the next batch's code words into the other register set before it
+// scores the current one.
 template <int CI, int NT, bool HIST>
-__global__ void __launch_bounds__(kFp4Threads) indexer_score_fp4_kernel(IndexerArgs a,
-                                                                        int64_t chunk) {
+__global__ void __launch_bounds__(kFp4Threads, (CI == 64 && NT == 1) ? 3 : 1)
+indexer_score_fp4_kernel(IndexerArgs a, int64_t chunk) {
   constexpr int KB = CI / 32;                  // scale blocks per vector
-  constexpr int kU = fp4_unroll(CI, NT);       // 16-key groups in flight per warp
+  constexpr int kU = fp4_unroll(CI, NT);       // 16-key groups per batch
   __shared__ uint32_t sh_hist[HIST ? kHistBins : 1];
   __shared__ Fp4Query<CI, NT> sq;
+  __shared__ uint32_t qwords[NT * 8][CI / 8];  // the query's codes, head-major
+  __shared__ uint32_t qscale[NT * 8][KB];
   const int64_t tl = blockIdx.x;
   const int64_t t = a.t_begin + tl;
   const int64_t pos = a.q_pos ? __ldg(a.q_pos + t) : t;
@@ -173,17 +278,20 @@ __global__ void __launch_bounds__(kFp4Threads) indexer_score_fp4_kernel(IndexerA
 
   if (HIST)
     for (int b = threadIdx.x; b < kHistBins; b += kFp4Threads) sh_hist[b] = 0;
+  for (int i = threadIdx.x; i < a.H_I * KB; i += kFp4Threads) {
+    const int h = i / KB, v = i - h * KB;
+    uint32_t w4[4];
+    qscale[h][v] = quantize_block(a.q_idx + (t * a.H_I + h) * CI + 32 * v, w4);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) qwords[h][4 * v + j] = w4[j];
+  }
+  __syncthreads();
   for (int i = threadIdx.x; i < NT * KB * 32; i += kFp4Threads) {
     const int L = i & 31, v = (i >> 5) % KB, nt = (i >> 5) / KB;
     const int hg = nt * 8 + (L >> 2), h0 = nt * 8 + 2 * (L & 3);
-    uint32_t word = 0;
-    if (hg < a.H_I)
-      word = __ldg(reinterpret_cast<const uint32_t*>(a.q_codes + ((t * a.H_I + hg) * CI) / 2) +
-                   4 * v + (L & 3));
-    sq.frag[nt][v][L] = e2m1x8_to_f16(word);
-    const float f0 = h0 < a.H_I ? e8m0_value(__ldg(a.q_scales + (t * a.H_I + h0) * KB + v)) : 0.f;
-    const float f1 =
-        h0 + 1 < a.H_I ? e8m0_value(__ldg(a.q_scales + (t * a.H_I + h0 + 1) * KB + v)) : 0.f;
+    sq.frag[nt][v][L] = e2m1x8_to_f16(hg < a.H_I ? qwords[hg][4 * v + (L & 3)] : 0u);
+    const float f0 = h0 < a.H_I ? e8m0_value(qscale[h0][v]) : 0.f;
+    const float f1 = h0 + 1 < a.H_I ? e8m0_value(qscale[h0 + 1][v]) : 0.f;
     sq.fac[nt][v][L] = make_float2(f0, f1);
     if (v == 0)
       sq.w[nt][L] = make_float2(h0 < a.H_I ? __ldg(a.w + t * a.H_I + h0) : 0.f,
@@ -193,76 +301,18 @@ __global__ void __launch_bounds__(kFp4Threads) indexer_score_fp4_kernel(IndexerA
 
   const uint8_t* codes = reinterpret_cast<const uint8_t*>(a.keys.data);
   uint32_t* out = a.keys_out + tl * a.key_stride;
-
-  for (int64_t s0 = s_begin + (int64_t)warp * 16 * kU; s0 < s_end;
-       s0 += (int64_t)kFp4Warps * 16 * kU) {
-    uint32_t kw[kU][2][KB];   // code words of rows g (h = 0) and g + 8 (h = 1)
-    uint32_t ks[kU][2];       // their scale bytes, KB per row
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t s = s0 + u * 16 + g + 8 * h;
-        int64_t row = -1;
-        if (s < s_end) row = cache_row(a.keys, seq, s, a.err, (int32_t)t);
-        const uint32_t* rw =
-            reinterpret_cast<const uint32_t*>(codes + (row >= 0 ? row : 0) * (CI / 2));
-#pragma unroll
-        for (int v = 0; v < KB; ++v) kw[u][h][v] = row >= 0 ? __ldg(rw + 4 * v + q4) : 0u;
-        if (CI == 64)
-          ks[u][h] = row >= 0 ? (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(a.k_scales) + row)
-                              : 0u;
-        else
-          ks[u][h] = row >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(a.k_scales) + row) : 0u;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      uint4 ka[2][KB];
-      float fk[2][KB];
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int v = 0; v < KB; ++v) {
-          ka[h][v] = e2m1x8_to_f16(kw[u][h][v]);
-          fk[h][v] = e8m0_value((ks[u][h] >> (8 * v)) & 0xffu);
-        }
-      float sg = 0.f, s8 = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float dg0 = 0.f, dg1 = 0.f, d80 = 0.f, d81 = 0.f;   // rows g / g+8, heads h0 / h0+1
-#pragma unroll
-        for (int v = 0; v < KB; ++v) {
-          const uint4 bq = sq.frag[nt][v][lane];
-          float d[4] = {0.f, 0.f, 0.f, 0.f};
-          const uint32_t lo[4] = {ka[0][v].x, ka[1][v].x, ka[0][v].y, ka[1][v].y};
-          mma_f16_16816(d, lo, bq.x, bq.y);
-          const uint32_t hi[4] = {ka[0][v].z, ka[1][v].z, ka[0][v].w, ka[1][v].w};
-          mma_f16_16816(d, hi, bq.z, bq.w);
-          const float2 fq = sq.fac[nt][v][lane];
-          dg0 += d[0] * fq.x * fk[0][v];
-          dg1 += d[1] * fq.y * fk[0][v];
-          d80 += d[2] * fq.x * fk[1][v];
-          d81 += d[3] * fq.y * fk[1][v];
-        }
-        const float2 wv = sq.w[nt][lane];
-        sg = fmaf(wv.x, fmaxf(dg0, 0.f), sg);
-        sg = fmaf(wv.y, fmaxf(dg1, 0.f), sg);
-        s8 = fmaf(wv.x, fmaxf(d80, 0.f), s8);
-        s8 = fmaf(wv.y, fmaxf(d81, 0.f), s8);
-      }
-      sg += __shfl_xor_sync(0xffffffffu, sg, 1);
-      s8 += __shfl_xor_sync(0xffffffffu, s8, 1);
-      sg += __shfl_xor_sync(0xffffffffu, sg, 2);
-      s8 += __shfl_xor_sync(0xffffffffu, s8, 2);
-      const int64_t s = s0 + u * 16 + g + (q4 == 1 ? 8 : 0);
-      const bool valid = q4 < 2 && s < s_end;
-      const uint32_t key = score_key(q4 == 0 ? sg : s8);
-      if (valid) {
-        out[s] = key;
-        if (HIST) atomicAdd(&sh_hist[key >> 20], 1u);
-      }
-    }
+  const int64_t stride = (int64_t)kFp4Warps * 16 * kU;
+  KeyBatch<CI, kU> b0, b1;
+  int64_t s0 = s_begin + (int64_t)warp * 16 * kU;
+  if (s0 < s_end) load_batch(b0, a, codes, seq, s0, s_end, t, g, q4);
+  while (s0 < s_end) {
+    int64_t s1 = s0 + stride;
+    if (s1 < s_end) load_batch(b1, a, codes, seq, s1, s_end, t, g, q4);
+    score_batch<CI, NT, HIST>(b0, sq, sh_hist, out, s0, s_end, lane, g, q4);
+    if (s1 >= s_end) break;
+    s0 = s1 + stride;
+    if (s0 < s_end) load_batch(b0, a, codes, seq, s0, s_end, t, g, q4);
+    score_batch<CI, NT, HIST>(b1, sq, sh_hist, out, s1, s_end, lane, g, q4);
   }
   if (HIST) {
     __syncthreads();

@@ -87,12 +87,10 @@ struct IndexerArgs {
   uint32_t* hist;               // [T_chunk, kHistBins] (zeroed) or null
   uint32_t* work;               // zeroed work counter of the tcgen05 scorer
   WsHeader* err;
-  // 4-bit mode (fp4 = 1): q_codes [T, H_I, c_I/2] and q_scales [T, H_I, c_I/32]
-  // replace q_idx; keys.data holds rows of c_I/2 code bytes and k_scales rows
-  // of c_I/32 scale bytes at the same physical row index
+  // 4-bit mode (fp4 = 1): q_idx is quantized to E2M1 codes + scale bytes in
+  // the scorer; keys.data holds rows of c_I/2 code bytes and k_scales rows of
+  // c_I/32 scale bytes at the same physical row index
   int fp4 = 0;
-  const uint8_t* q_codes = nullptr;
-  const uint8_t* q_scales = nullptr;
   const uint8_t* k_scales = nullptr;
 };
 cudaError_t launch_indexer_scores(const Launch& L, const IndexerArgs& a, int64_t t_count);

@@ -275,12 +275,14 @@ csa_status_t csa_quantize_mxfp4(const csa_bf16* x, int64_t n_vectors, int32_t di
                                 uint8_t* scales, csa_stream_t stream);
 
 /*
- * csa_indexer_topk_mxfp4 -- csa_indexer_topk on 4-bit queries and keys: the
- * same score definition applied to the dequantized values (each 32-element
- * block's dot product is exact; the blocks are scaled and summed, and the
- * heads weighted and summed, in fp32), the same selection rules, workspace
- * (csa_indexer_topk_workspace_size) and outputs.
- *   q_codes   [T, H_I, c_I/2] uint8 (16-byte aligned), q_scales [T, H_I, c_I/32]
+ * csa_indexer_topk_mxfp4 -- csa_indexer_topk with the indexer keys in 4-bit
+ * storage: every query's bf16 heads are quantized to the same format inside
+ * the call (codes identical to csa_quantize_mxfp4's), and the score definition
+ * is applied to the dequantized queries and keys (each 32-element block's dot
+ * product is exact; the blocks are scaled and summed, and the heads weighted
+ * and summed, in fp32).  Selection rules, workspace
+ * (csa_indexer_topk_workspace_size) and outputs are those of csa_indexer_topk.
+ *   q_idx     [T, H_I, c_I] bf16 (16-byte aligned)
  *   k_codes   cache whose rows are c_I/2 code bytes (data 16-byte aligned)
  *   k_scales  [k_codes->n_rows, c_I/32] uint8 (16-byte aligned): the scale bytes
  *             of physical row r of k_codes are row r of k_scales
@@ -288,13 +290,13 @@ csa_status_t csa_quantize_mxfp4(const csa_bf16* x, int64_t n_vectors, int32_t di
  * E8M0 NaN) are outside the supported range: csa_quantize_mxfp4 produces 0
  * only for blocks whose largest magnitude is below 2^-124.
  */
-csa_status_t csa_indexer_topk_mxfp4(const uint8_t* q_codes, const uint8_t* q_scales,
-                                    const float* w, const csa_cache_t* k_codes,
-                                    const uint8_t* k_scales, const int32_t* seq_id,
-                                    const int64_t* q_pos, int64_t T, int32_t H_I, int32_t c_I,
-                                    int32_t m, int64_t max_entries, int32_t top_k,
-                                    int32_t* idx_out, int32_t* count_out, float* score_out,
-                                    void* ws, size_t ws_bytes, csa_stream_t stream);
+csa_status_t csa_indexer_topk_mxfp4(const csa_bf16* q_idx, const float* w,
+                                    const csa_cache_t* k_codes, const uint8_t* k_scales,
+                                    const int32_t* seq_id, const int64_t* q_pos, int64_t T,
+                                    int32_t H_I, int32_t c_I, int32_t m, int64_t max_entries,
+                                    int32_t top_k, int32_t* idx_out, int32_t* count_out,
+                                    float* score_out, void* ws, size_t ws_bytes,
+                                    csa_stream_t stream);
 
 /* ---- step 4: attention ---------------------------------------------------- */
 /*

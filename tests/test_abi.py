@@ -161,17 +161,22 @@ def test_mxfp4_calls_reject_bad_arguments_without_launching(lib):
     assert lib.csa_quantize_mxfp4(p, 4, 64, C.c_void_p(p.value + 4), p, None) == 1
     assert lib.csa_quantize_mxfp4(p, 0, 64, None, None, None) == 0   # nothing to do
     cache = CacheT(p.value, 16, 16, None, 0, 0)
-    args = [p, p, p, C.byref(cache), p, None, None, 8, 8, 64, 4, 16, 4, p, p, None, p, 1 << 20, None]
+    # q_idx, w, k_codes, k_scales, seq_id, q_pos, T, H_I, c_I, m, max_entries, top_k,
+    # idx_out, count_out, score_out, ws, ws_bytes, stream
+    args = [p, p, C.byref(cache), p, None, None, 8, 8, 64, 4, 16, 4, p, p, None, p, 1 << 20, None]
     # c_I not built
-    a = list(args); a[9] = 96
+    a = list(args); a[8] = 96
     assert lib.csa_indexer_topk_mxfp4(*a) == 2
     # missing scales
-    a = list(args); a[4] = None
+    a = list(args); a[3] = None
     assert lib.csa_indexer_topk_mxfp4(*a) == 1 and b"k_scales" in lib.csa_last_error()
+    # misaligned queries
+    a = list(args); a[0] = C.c_void_p(p.value + 2)
+    assert lib.csa_indexer_topk_mxfp4(*a) == 1 and b"aligned" in lib.csa_last_error()
     # H_I above 64
-    a = list(args); a[8] = 65
+    a = list(args); a[7] = 65
     assert lib.csa_indexer_topk_mxfp4(*a) == 2
     # workspace too small
-    a = list(args); a[17] = 256
+    a = list(args); a[16] = 256
     assert lib.csa_indexer_topk_mxfp4(*a) == 5
     assert lib.csa_launch_count() == before

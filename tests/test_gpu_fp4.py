@@ -1,6 +1,8 @@
 """GPU parity of the 4-bit indexer (E2M1 codes with one power-of-two scale
 byte per 32 elements): the quantizer bit-exactly against the oracle's, and the
-4-bit scorer + top-k against the oracle's scores of the same codes."""
+4-bit scorer + top-k against the oracle's scores of the same key codes and of
+the oracle's quantization of the same bf16 queries (the scorer quantizes its
+queries itself, with the quantizer checked bit-exact here)."""
 import numpy as np
 import pytest
 import torch
@@ -105,13 +107,13 @@ def test_indexer_topk_mxfp4_decode_ragged(H_I, c_I):
     m, k = 4, 64
     pos = torch.tensor([0, 3, 4, 100, 257, 259, 1000, 9001], dtype=torch.int64)
     B, S = pos.shape[0], int(pos.max()) // m
-    qc, qs = ofp4.mxfp4_quantize(f64(synth.normal(g, (B, H_I, c_I))))
+    qI = synth.normal(g, (B, H_I, c_I))
+    qc, qs = ofp4.mxfp4_quantize(f64(qI))
     kc, ks = ofp4.mxfp4_quantize(f64(synth.normal(g, (B * S, c_I))))
     w = synth.uniform(g, (B, H_I))
     seq = torch.arange(B, dtype=torch.int32)
     cache = csa.Cache(dev(torch.from_numpy(kc)), seq_stride=S)
-    idx, cnt, sc = csa.indexer_topk_mxfp4(dev(torch.from_numpy(qc)), dev(torch.from_numpy(qs)),
-                                          dev(w), cache, dev(torch.from_numpy(ks)), m, k,
+    idx, cnt, sc = csa.indexer_topk_mxfp4(dev(qI), dev(w), cache, dev(torch.from_numpy(ks)), m, k,
                                           seq_id=dev(seq), q_pos=dev(pos), max_entries=S,
                                           return_scores=True)
     kc3, ks3 = kc.reshape(B, S, -1), ks.reshape(B, S, -1)
@@ -126,11 +128,11 @@ def test_indexer_topk_mxfp4_prefill_causal(T, m, k, H_I):
     csa = _csa()
     g = synth.generator(970 + T)
     S = (T - 1) // m
-    qc, qs = ofp4.mxfp4_quantize(f64(synth.normal(g, (T, H_I, 64))))
+    qI = synth.normal(g, (T, H_I, 64))
+    qc, qs = ofp4.mxfp4_quantize(f64(qI))
     kc, ks = ofp4.mxfp4_quantize(f64(synth.normal(g, (S, 64))))
     w = synth.uniform(g, (T, H_I))
-    idx, cnt = csa.indexer_topk_mxfp4(dev(torch.from_numpy(qc)), dev(torch.from_numpy(qs)), dev(w),
-                                      csa.Cache(dev(torch.from_numpy(kc))),
+    idx, cnt = csa.indexer_topk_mxfp4(dev(qI), dev(w), csa.Cache(dev(torch.from_numpy(kc))),
                                       dev(torch.from_numpy(ks)), m, k)
     stats = _check_fp4_queries(idx, cnt, None, lambda t: (qc[t], qs[t]), w, lambda t: (kc, ks),
                                lambda t: t // m, k, range(T))
@@ -146,11 +148,11 @@ def test_indexer_topk_mxfp4_identical_keys_tie_to_lower_index():
     base_c, base_s = synth.fp4_codes(g, (50,), 64)
     pick = torch.randint(0, 50, (S,), generator=g)
     kc, ks = base_c[pick].numpy(), base_s[pick].numpy()
-    qc, qs = (a.numpy() for a in synth.fp4_codes(g, (T, H_I), 64))
+    qI = synth.normal(g, (T, H_I, 64))
+    qc, qs = ofp4.mxfp4_quantize(f64(qI))
     w = synth.uniform(g, (T, H_I))
     pos = torch.randint(0, S * m, (T,), generator=g, dtype=torch.int64)
-    idx, cnt = csa.indexer_topk_mxfp4(dev(torch.from_numpy(qc)), dev(torch.from_numpy(qs)), dev(w),
-                                      csa.Cache(dev(torch.from_numpy(kc))),
+    idx, cnt = csa.indexer_topk_mxfp4(dev(qI), dev(w), csa.Cache(dev(torch.from_numpy(kc))),
                                       dev(torch.from_numpy(ks)), m, k, q_pos=dev(pos),
                                       seq_id=dev(torch.zeros(T, dtype=torch.int32)), max_entries=S)
     idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
@@ -179,13 +181,14 @@ def test_indexer_topk_mxfp4_paged(page_size):
         off += p
     pool_c, pool_s = synth.fp4_codes(g, (sum(pages) * page_size,), 64)
     B = len(S)
-    qc, qs = synth.fp4_codes(g, (B, H_I), 64)
+    qI = synth.normal(g, (B, H_I, 64))
+    qc, qs = ofp4.mxfp4_quantize(f64(qI))
     w = synth.uniform(g, (B, H_I))
     cache = csa.Cache(dev(pool_c), page_table=dev(table), page_size=page_size)
-    idx, cnt = csa.indexer_topk_mxfp4(dev(qc), dev(qs), dev(w), cache, dev(pool_s), m, k,
+    idx, cnt = csa.indexer_topk_mxfp4(dev(qI), dev(w), cache, dev(pool_s), m, k,
                                       seq_id=dev(torch.arange(B, dtype=torch.int32)),
                                       q_pos=dev(pos), max_entries=max(S))
-    _check_fp4_queries(idx, cnt, None, lambda b: (qc[b].numpy(), qs[b].numpy()), w,
+    _check_fp4_queries(idx, cnt, None, lambda b: (qc[b], qs[b]), w,
                        lambda b: (synth.unpage(pool_c, table[b], S[b], page_size).numpy(),
                                   synth.unpage(pool_s, table[b], S[b], page_size).numpy()),
                        lambda b: S[b], k, range(B))
@@ -199,13 +202,13 @@ def test_indexer_topk_mxfp4_decode_full_size_sampled():
     g = synth.generator(999)
     B, S, H_I, k, m = 64, 32768, 8, 2048, 4
     kc, ks = synth.fp4_codes(g, (B * S,), 64)
-    qc, qs = synth.fp4_codes(g, (B, H_I), 64)
+    qI = synth.normal(g, (B, H_I, 64))
+    qc, qs = ofp4.mxfp4_quantize(f64(qI))
     w = synth.uniform(g, (B, H_I))
     pos = torch.full((B,), S * m, dtype=torch.int64)
-    idx, cnt = csa.indexer_topk_mxfp4(dev(qc), dev(qs), dev(w),
-                                      csa.Cache(dev(kc), seq_stride=S), dev(ks), m, k,
-                                      seq_id=dev(torch.arange(B, dtype=torch.int32)),
+    idx, cnt = csa.indexer_topk_mxfp4(dev(qI), dev(w), csa.Cache(dev(kc), seq_stride=S), dev(ks),
+                                      m, k, seq_id=dev(torch.arange(B, dtype=torch.int32)),
                                       q_pos=dev(pos), max_entries=S)
     kc3, ks3 = kc.view(B, S, -1).numpy(), ks.view(B, S, -1).numpy()
-    _check_fp4_queries(idx, cnt, None, lambda b: (qc[b].numpy(), qs[b].numpy()), w,
+    _check_fp4_queries(idx, cnt, None, lambda b: (qc[b], qs[b]), w,
                        lambda b: (kc3[b], ks3[b]), lambda b: S, k, [0, 17, 40, 63])

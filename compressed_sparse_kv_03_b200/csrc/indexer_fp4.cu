@@ -20,8 +20,8 @@
 //     scales in an array of their own with the same row order.
 //
 // Scoring uses the score definition of Ch.6 "The lightning indexer" on the
-// dequantized values.  E2M1 magnitudes are exact fp16 numbers, so a code
-// nibble becomes an fp16 by a byte lookup (prmt); the tensor cores (mma.sync,
+// dequantized values.  E2M1 magnitudes are exact fp16 numbers, so code bytes
+// become fp16 pairs by sm_100a's e2m1x2 conversion; the tensor cores (mma.sync,
 // fp16 inputs, fp32 accumulation) form the dot product of each 32-element
 // scale block exactly (products are multiples of 1/4 below 36, sums below
 // 1152), and the block results are scaled by 2^(b_q - 127) * 2^(b_k - 127)
@@ -122,19 +122,21 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
 }
 
 // Eight E2M1 codes (nibble j = element j) -> fp16 pairs (0,1), (2,3), (4,5),
-// (6,7).  Every E2M1 value is an fp16 number whose low byte is zero; its high
-// byte comes from an 8-entry table indexed by the magnitude bits, the sign
-// bit is or-ed in, and the bytes are spread into 16-bit lanes.
+// (6,7): every E2M1 value is an fp16 number, and sm_100a converts a byte of
+// two codes (low nibble -> low half) in one instruction.
 __device__ __forceinline__ uint4 e2m1x8_to_f16(uint32_t x) {
-  constexpr uint32_t kMagLo = 0x3E3C3800u;   // high bytes of 0, 0.5, 1, 1.5
-  constexpr uint32_t kMagHi = 0x46444240u;   // high bytes of 2, 3, 4, 6
-  const uint32_t n0 = x & 0xffffu, n1 = x >> 16;
-  const uint32_t b0 = __byte_perm(kMagLo, kMagHi, n0 & 0x7777u) |
-                      __byte_perm(0x00008000u, 0u, (n0 >> 3) & 0x1111u);
-  const uint32_t b1 = __byte_perm(kMagLo, kMagHi, n1 & 0x7777u) |
-                      __byte_perm(0x00008000u, 0u, (n1 >> 3) & 0x1111u);
-  return make_uint4(__byte_perm(b0, 0u, 0x1404u), __byte_perm(b0, 0u, 0x3424u),
-                    __byte_perm(b1, 0u, 0x1404u), __byte_perm(b1, 0u, 0x3424u));
+  uint4 r;
+  asm("{\n"
+      ".reg .b8 b0, b1, b2, b3;\n"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n"
+      "}\n"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "r"(x));
+  return r;
 }
 
 // 2^(b - 127) for a scale byte b (b = 0: 2^-127, a subnormal)
@@ -162,10 +164,12 @@ struct KeyBatch {
   uint32_t ks[kU][2];
 };
 
+// base >= 0: contiguous cache whose rows base + [s_begin, s_end) were checked
+// once for the whole chunk; else every row goes through cache_row.
 template <int CI, int kU>
 __device__ __forceinline__ void load_batch(KeyBatch<CI, kU>& kb, const IndexerArgs& a,
-                                           const uint8_t* codes, int32_t seq, int64_t s0,
-                                           int64_t s_end, int64_t t, int g, int q4) {
+                                           const uint8_t* codes, int32_t seq, int64_t base,
+                                           int64_t s0, int64_t s_end, int64_t t, int g, int q4) {
   constexpr int KB = CI / 32;
 #pragma unroll
   for (int u = 0; u < kU; ++u) {
@@ -173,7 +177,7 @@ __device__ __forceinline__ void load_batch(KeyBatch<CI, kU>& kb, const IndexerAr
     for (int h = 0; h < 2; ++h) {
       const int64_t s = s0 + u * 16 + g + 8 * h;
       int64_t row = -1;
-      if (s < s_end) row = cache_row(a.keys, seq, s, a.err, (int32_t)t);
+      if (s < s_end) row = base >= 0 ? base + s : cache_row(a.keys, seq, s, a.err, (int32_t)t);
       const uint32_t* rw =
           reinterpret_cast<const uint32_t*>(codes + (row >= 0 ? row : 0) * (CI / 2));
 #pragma unroll
@@ -302,16 +306,24 @@ indexer_score_fp4_kernel(IndexerArgs a, int64_t chunk) {
   const uint8_t* codes = reinterpret_cast<const uint8_t*>(a.keys.data);
   uint32_t* out = a.keys_out + tl * a.key_stride;
   const int64_t stride = (int64_t)kFp4Warps * 16 * kU;
+  // a contiguous cache whose chunk lies inside the buffer skips the per-row
+  // checks (the same conditions cache_row tests, once for the whole chunk)
+  int64_t base = -1;
+  if (a.keys.page_table == nullptr) {
+    const int64_t b = (int64_t)seq * a.keys.seq_stride;
+    if (b >= 0 && (a.keys.seq_stride == 0 || s_end <= a.keys.seq_stride) && b + s_end <= a.keys.n_rows)
+      base = b;
+  }
   KeyBatch<CI, kU> b0, b1;
   int64_t s0 = s_begin + (int64_t)warp * 16 * kU;
-  if (s0 < s_end) load_batch(b0, a, codes, seq, s0, s_end, t, g, q4);
+  if (s0 < s_end) load_batch(b0, a, codes, seq, base, s0, s_end, t, g, q4);
   while (s0 < s_end) {
     int64_t s1 = s0 + stride;
-    if (s1 < s_end) load_batch(b1, a, codes, seq, s1, s_end, t, g, q4);
+    if (s1 < s_end) load_batch(b1, a, codes, seq, base, s1, s_end, t, g, q4);
     score_batch<CI, NT, HIST>(b0, sq, sh_hist, out, s0, s_end, lane, g, q4);
     if (s1 >= s_end) break;
     s0 = s1 + stride;
-    if (s0 < s_end) load_batch(b0, a, codes, seq, s0, s_end, t, g, q4);
+    if (s0 < s_end) load_batch(b0, a, codes, seq, base, s0, s_end, t, g, q4);
     score_batch<CI, NT, HIST>(b1, sq, sh_hist, out, s1, s_end, lane, g, q4);
   }
   if (HIST) {

@@ -30,3 +30,4 @@ from .csa_oracle import (  # noqa: F401
 )
 from . import cost_model  # noqa: F401
 from . import mxfp4  # noqa: F401
+from . import fp8_entry  # noqa: F401

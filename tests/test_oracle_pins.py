@@ -572,3 +572,89 @@ def test_mxfp4_quantize_is_blockwise_definition():
             assert scales[r, b] == X + 127
             codes = ofp4.e2m1_encode(blk / 2.0 ** X)
             assert np.array_equal(packed[r, 16 * b:16 * b + 16], codes[0::2] | (codes[1::2] << 4))
+
+
+# ---------------------------------------------------------------------------
+# mixed-precision entries: FP8 content + bf16 rotary part (Ch.8 "V4
+# compressed-entry payload")
+# ---------------------------------------------------------------------------
+from oracle import fp8_entry as ofp8   # noqa: E402
+
+
+def test_e4m3_grid_closed_forms():
+    v = ofp8.e4m3_value(np.arange(256))
+    finite = v[np.isfinite(v)]
+    assert np.nanmax(v) == 448.0 and np.nanmin(v) == -448.0          # largest normal
+    assert v[1] == 2.0 ** -9 and v[8] == 2.0 ** -6                     # smallest subnormal / normal
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF]) and finite.size == 254
+    assert np.all(np.diff(v[:0x7F]) > 0)                               # codes ordered by value
+    assert np.signbit(v[0x80]) and v[0x80] == 0.0
+
+
+def test_e4m3_encode_matches_library_rounding():
+    import ml_dtypes
+    mags = ofp8.e4m3_value(np.arange(0x7F))
+    mids = (mags[1:] + mags[:-1]) / 2
+    y = np.concatenate([mags, mids, mids * (1 + 2.0 ** -30), mids * (1 - 2.0 ** -30),
+                        rng.uniform(-448, 448, 6000), rng.standard_normal(3000) * 0.01])
+    y = np.concatenate([y, -y]).astype(np.float32)
+    lib = y.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    assert np.array_equal(ofp8.e4m3_encode(y.astype(np.float64)), lib)
+
+
+def test_e4m3_saturates_and_keeps_sign():
+    assert ofp8.e4m3_encode([449.0, 480.0, 1e9, -1e9]).tolist() == [0x7E, 0x7E, 0x7E, 0xFE]
+    assert ofp8.e4m3_encode([-0.0, -2.0 ** -12]).tolist() == [0x80, 0x80]
+
+
+def test_mxfp8_scale_binade_and_roundtrip():
+    for _ in range(200):
+        blk = rng.standard_normal(32) * 2.0 ** rng.integers(-40, 40)
+        X = ofp8.mxfp8_scale_exponent(blk)
+        assert 256.0 <= np.abs(blk).max() / 2.0 ** X < 512.0
+    x = oracle.bf16_round(rng.standard_normal((20, 64)) * 2.0 ** rng.integers(-20, 20, (20, 1)))
+    codes, scales = ofp8.mxfp8_quantize(x)
+    y = ofp8.mxfp8_dequantize(codes, scales)
+    c2, s2 = ofp8.mxfp8_quantize(y)
+    assert np.array_equal(c2, codes) and np.array_equal(s2, scales)
+    # error at most half a quantum of the element's binade (quantum 2^(e-3),
+    # subnormal quantum 2^-9), in units of 2^X; saturated elements below 64
+    X = np.repeat(scales.astype(np.int64) - 127, 32, axis=1)
+    u = np.abs(x) / 2.0 ** X
+    e = np.floor(np.log2(np.maximum(u, 2.0 ** -6)))
+    bound = np.where(u > 448, 64.0, 2.0 ** (e - 4)) * 2.0 ** X
+    assert np.all(np.abs(y - x) <= bound)
+
+
+def test_mxfp8_quantize_is_blockwise_definition():
+    x = oracle.bf16_round(rng.standard_normal((5, 64)) * 2.0 ** rng.integers(-60, 60, (5, 1)))
+    x[0, 32:] = 0.0
+    codes, scales = ofp8.mxfp8_quantize(x)
+    for r in range(5):
+        for b in range(2):
+            blk = x[r, 32 * b:32 * b + 32]
+            X = ofp8.mxfp8_scale_exponent(blk)
+            assert scales[r, b] == X + 127
+            assert np.array_equal(codes[r, 32 * b:32 * b + 32], ofp8.e4m3_encode(blk / 2.0 ** X))
+
+
+def test_fp8_entry_payload_matches_pages():
+    # c = 512 with the last 64 coordinates rotary: 448 FP8 bytes + 64 bf16 values = 576 B
+    # (Ch.8 "V4 compressed-entry payload"), plus 14 scale bytes of metadata
+    x = oracle.bf16_round(rng.standard_normal(512))
+    codes, scales, rope = ofp8.entry_quantize(x, 64)
+    assert codes.nbytes + 2 * rope.size == 576
+    assert scales.size == 14
+    # the rotary part is kept as given
+    y = ofp8.entry_dequantize(codes, scales, rope)
+    assert np.array_equal(y[448:], x[448:])
+    assert np.array_equal(y[:448], ofp8.mxfp8_dequantize(codes, scales))
+
+
+def test_fp8_entry_values_are_bf16_numbers():
+    # every dequantized content value is exactly representable in bf16 (3
+    # mantissa bits, power-of-two scale), so the dequantized cache is a bf16 cache
+    x = oracle.bf16_round(rng.standard_normal((50, 128)) * 3)
+    codes, scales, rope = ofp8.entry_quantize(x, 64)
+    y = ofp8.entry_dequantize(codes, scales, rope)
+    assert np.array_equal(oracle.bf16_round(y), y)

@@ -10,7 +10,8 @@ input already resident in HBM.  The default workload is CSA decode (batch 64,
 Other workloads: csa_prefill_L4096, csa_prefill_L65536,
 hca_decode_B8_N1048576, mixed_decode_B16_N256K_1M, and
 csa_decode_B64_N131072_mxfp4_indexer (the default decode with the indexer keys
-and queries in 4-bit storage).
+and queries in 4-bit storage) and csa_decode_B64_N131072_lowprec (also the main
+entries in FP8 content + bf16 rotary storage).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch (weak
 scaling, no data-path collective); the step time is the max over ranks.
@@ -143,6 +144,45 @@ class CsaDecodeMxfp4(CsaDecode):
     def config(self):
         c = super().config()
         c["indexer_storage"] = "E2M1 codes + one power-of-two scale byte per 32 (34 B per key)"
+        return c
+
+
+class CsaDecodeLowPrec(CsaDecodeMxfp4):
+    """CSA decode with both low-precision caches: the 4-bit indexer keys of
+    CsaDecodeMxfp4 and main entries stored as E4M3 content with a scale byte
+    per 32 plus the 64 rotary coordinates in bf16 (quantized when the cache is
+    built); a step is csa_indexer_topk_mxfp4 + csa_sparse_attn_decode_fp8."""
+
+    ROPE = 64
+
+    def __init__(self, cfg, seed_offset=0):
+        super().__init__(cfg, seed_offset)
+        csa = self.csa
+        kv = self.d.pop("kv_comp")
+        codes, scales, rope = csa.quantize_entries_fp8(kv.view(-1, kv.shape[-1]), self.ROPE)
+        del kv
+        self.kv = csa.Cache(codes, seq_stride=self.S)
+        self.kv_scales, self.kv_rope = scales, rope
+        torch.cuda.synchronize()
+        sel_rows = min(cfg.k, self.S)
+        win_rows = min(cfg.W, cfg.N + 1)
+        entry_bytes = (cfg.d - self.ROPE) + (cfg.d - self.ROPE) // 32 + 2 * self.ROPE
+        self.step_bytes = (self.dominant_bytes + cfg.B * (sel_rows * entry_bytes + win_rows * cfg.d * 2)
+                           + cfg.B * (2 * cfg.H * cfg.d * 2 + cfg.H_I * cfg.c_I * 2 + cfg.H_I * 4))
+
+    def step(self):
+        csa, cfg, d = self.csa, self.cfg, self.d
+        csa.indexer_topk_mxfp4(d["qI"], d["w"], self.kI, self.kI_scales, cfg.m, cfg.k,
+                               seq_id=self.seq_id, q_pos=d["pos"], max_entries=self.S, ws=self.ws_i,
+                               out=(self.idx, self.cnt, None))
+        csa.sparse_attn_decode_fp8(d["q"], self.kv, self.kv_scales, self.kv_rope, d["win"],
+                                   d["win_len"], self.idx, self.cnt, cfg.lam, ws=self.ws_a,
+                                   out=self.out)
+
+    def config(self):
+        c = super().config()
+        c["entry_storage"] = ("E4M3 content + one power-of-two scale byte per 32 + 64 bf16 rotary "
+                              "coordinates (194 B per entry)")
         return c
 
 
@@ -331,6 +371,7 @@ RUNNERS = {
     synth.CFG_PREFILL_64K.name: (CsaPrefill, synth.CFG_PREFILL_64K),
     synth.CFG_MIXED.name: (MixedDecode, synth.CFG_MIXED),
     synth.CFG_DECODE_128K_MXFP4.name: (CsaDecodeMxfp4, synth.CFG_DECODE_128K_MXFP4),
+    synth.CFG_DECODE_128K_LOWPREC.name: (CsaDecodeLowPrec, synth.CFG_DECODE_128K_LOWPREC),
 }
 
 
@@ -420,19 +461,23 @@ def oracle_sample(name, budget_s):
         threads = 1
     cls, cfg = RUNNERS[name]
     f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
-    if cls is CsaDecodeMxfp4:
+    if cls is CsaDecodeMxfp4 or cls is CsaDecodeLowPrec:
+        from oracle import fp8_entry as ofp8
         from oracle import mxfp4 as ofp4
         host = synth.csa_decode_inputs(cfg, B=min(cfg.B, 16))
         done, secs = 0, 0.0
         while done < host["q"].shape[0] and secs < budget_s:
             b = done
             kc, ks = ofp4.mxfp4_quantize(f(host["kI_comp"][b]))   # cache contents: not timed
+            kv_b = f(host["kv_comp"][b])
+            if cls is CsaDecodeLowPrec:                           # cache contents: not timed
+                kv_b = ofp8.entry_dequantize(*ofp8.entry_quantize(kv_b, CsaDecodeLowPrec.ROPE))
             t0 = time.perf_counter()
             qc, qs = ofp4.mxfp4_quantize(f(host["qI"][b]))
             n = oracle.eligible_entries(int(host["pos"][b]), cfg.m)
             sel = oracle.topk_select(ofp4.indexer_scores_mxfp4(qc, qs, f(host["w"][b]), kc[:n], ks[:n]),
                                      cfg.k)
-            rows = np.concatenate([f(host["kv_comp"][b])[sel], f(host["win"][b])[:int(host["win_len"][b])]])
+            rows = np.concatenate([kv_b[sel], f(host["win"][b])[:int(host["win_len"][b])]])
             oracle.attend_shared_kv(f(host["q"][b]), rows, cfg.lam)
             secs += time.perf_counter() - t0
             done += 1

@@ -7,6 +7,8 @@ the current torch stream.  Shapes follow the header:
     indexer_topk         (steps 2-3) q_idx [T, H_I, c_I], w [T, H_I], keys -> idx [T, k], count [T]
     quantize_mxfp4       x [..., dim] bf16 -> 4-bit codes [..., dim/2] + scale bytes [..., dim/32]
     indexer_topk_mxfp4   (steps 2-3) on 4-bit queries and keys
+    quantize_entries_fp8 entries [..., dim] bf16 -> E4M3 content + scale bytes + bf16 rotary part
+    sparse_attn_decode_fp8 (step 4)  decode over those mixed-precision entries
     sparse_attn_prefill  (step 4)    q [L, H, 128] over kv_comp[idx] + raw window
     sparse_attn_decode   (step 4)    q [B, H, 128] over cache[idx] + window buffer
     hca_attn             (step 4)    q [T, H, 128] over all eligible entries + window
@@ -355,6 +357,63 @@ def sparse_attn_decode(q, kv: Cache, win, win_len, idx, count, sm_scale, *, sink
                                      _ptr(sink), _ptr(out), _ptr(lse), wsp, wsb, _stream(stream)))
     return (out, lse) if return_lse else out
 
+
+def quantize_entries_fp8(x, rope_dims=64, *, stream=None, out=None):
+    """Mixed-precision storage of compressed entries x [..., dim] bf16 (E4M3
+    content with a scale byte per 32, the last rope_dims coordinates kept in
+    bf16; see include/csa.h): returns (codes [..., dim - rope_dims] uint8,
+    scales [..., (dim - rope_dims)/32] uint8, rope [..., rope_dims] bf16)."""
+    _need(x, "x", torch.bfloat16)
+    dim = x.shape[-1]
+    dc = dim - rope_dims
+    if rope_dims < 0 or rope_dims % 8 or dc <= 0 or dc % 32:
+        raise ValueError("need rope_dims a multiple of 8 below dim, dim - rope_dims a multiple of 32")
+    n = x.numel() // dim
+    lead = x.shape[:-1]
+    if out is None:
+        codes = torch.empty(lead + (dc,), dtype=torch.uint8, device=x.device)
+        scales = torch.empty(lead + (dc // 32,), dtype=torch.uint8, device=x.device)
+        rope = torch.empty(lead + (rope_dims,), dtype=torch.bfloat16, device=x.device)
+    else:
+        codes, scales, rope = out
+    check(load().csa_quantize_entries_fp8(_ptr(x), n, dim, rope_dims, _ptr(codes), _ptr(scales),
+                                          _ptr(rope) if rope_dims else None, _stream(stream)))
+    return codes, scales, rope
+
+
+def sparse_attn_decode_fp8(q, codes: Cache, scales, rope, win, win_len, idx, count, sm_scale, *,
+                           sink=None, return_lse=False, ws=None, stream=None, out=None):
+    """Step 4 (CSA decode) over mixed-precision entries: codes.data [rows,
+    128 - r] uint8 (contiguous or paged), scales [rows, (128 - r)/32] uint8,
+    rope [rows, r] bf16 (same rows), from quantize_entries_fp8; the window
+    rows stay bf16.  Arguments otherwise as sparse_attn_decode."""
+    _need(q, "q", torch.bfloat16, 3)
+    B, H, d = q.shape
+    dev = q.device
+    rows = codes.data.shape[0]
+    _need(scales, "scales", torch.uint8, 2, dev)
+    _need(rope, "rope", torch.bfloat16, 2, dev)
+    r = rope.shape[1]
+    if codes.data.shape[1] != d - r or tuple(scales.shape) != (rows, (d - r) // 32) or rope.shape[0] != rows:
+        raise ValueError("codes / scales / rope shapes do not describe the same entries")
+    _need(win, "win", torch.bfloat16, 3, dev)
+    _need(win_len, "win_len", torch.int32, 1, dev)
+    _need(idx, "idx", torch.int32, 2, dev)
+    _need(count, "count", torch.int32, 1, dev)
+    if sink is not None:
+        _need(sink, "sink", torch.float32, 1, dev)
+    top_k, window = idx.shape[1], win.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev) if return_lse else None
+    lib = load()
+    wsp, wsb = _ws(ws, dev).get(lib.csa_sparse_attn_decode_workspace_size(B, H, d, top_k, window))
+    kc = codes.c(torch.uint8)
+    check(lib.csa_sparse_attn_decode_fp8(_ptr(q), C.byref(kc), _ptr(scales), _ptr(rope) if r else None,
+                                         r, _ptr(win), _ptr(win_len), _ptr(idx), _ptr(count), B, H,
+                                         d, top_k, window, float(sm_scale), _ptr(sink), _ptr(out),
+                                         _ptr(lse), wsp, wsb, _stream(stream)))
+    return (out, lse) if return_lse else out
 
 def hca_attn(q, kv: Cache, kv_win, m, window, sm_scale, *, win_len=None, q_pos=None,
              max_entries=None, sink=None, return_lse=False, ws=None, stream=None, out=None):

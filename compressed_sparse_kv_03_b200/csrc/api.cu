@@ -612,28 +612,43 @@ csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
   return cuda_status(launch_attention(Lc, a), name);
 }
 
-csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_comp,
-                                    const csa_bf16* win, const int32_t* win_len,
-                                    const int32_t* idx, const int32_t* count, int32_t B,
-                                    int32_t H, int32_t d, int32_t top_k, int32_t window,
-                                    float sm_scale, const float* sink, csa_bf16* out,
-                                    float* lse, void* ws, size_t ws_bytes,
-                                    csa_stream_t stream) {
-  const char* name = "csa_sparse_attn_decode";
-  if (B == 0) return CSA_OK;
-  csa_status_t st = check_attn_common(name, q, out, H, d, window);
+namespace {
+
+// Split selection, workspace check and launch shared by the decode calls; `a`
+// holds every field but the split / workspace ones.
+csa_status_t run_decode_attention(AttnArgs a, const char* name, int32_t B, int32_t H,
+                                  int32_t top_k, int32_t window, void* ws, size_t ws_bytes,
+                                  csa_stream_t stream) {
+  const Split sp_ws = attn_split(B, (int64_t)top_k + window, H);
+  const bool invariant = g_batch_invariant.load(std::memory_order_relaxed) != 0;
+  const Split sp_inv = attn_split_invariant((int64_t)top_k + window);
+  const int n_need = invariant && sp_inv.n > sp_ws.n ? sp_inv.n : sp_ws.n;
+  csa_status_t st = check_ws(ws, ws_bytes, attn_partials_bytes(B, H, n_need), name);
   if (st != CSA_OK) return st;
-  if ((st = check_cache(kv_comp, name)) != CSA_OK) return st;
-  if (idx == nullptr || count == nullptr || B < 0 || top_k < 1)
-    return fail(CSA_ERR_INVALID_ARG, "%s: idx, count required; B >= 0, top_k >= 1", name);
-  if (window > 0 && (win == nullptr || win_len == nullptr))
-    return fail(CSA_ERR_INVALID_ARG, "%s: window > 0 needs win and win_len", name);
-  if (B == 0) return check_ws(ws, ws_bytes, kWsHeader, name);
+  a.use_tc = attention_uses_tc(a);
+  const Split sp = invariant ? sp_inv
+                             : (a.use_tc ? attn_split_tc(B, (int64_t)top_k + window, H, sp_ws) : sp_ws);
+  a.n_split = sp.n;
+  a.split_len = sp.len;
+  a.err = static_cast<WsHeader*>(ws);
+  if (sp.n > 1) {
+    char* p = static_cast<char*>(ws) + kWsHeader;
+    a.part_acc = reinterpret_cast<float*>(p);
+    a.part_ml = reinterpret_cast<float*>(p + align256((size_t)B * sp.n * H * kD * sizeof(float)));
+  }
+  Launch L{(cudaStream_t)stream};
+  return cuda_status(launch_attention(L, a), name);
+}
+
+AttnArgs decode_args(const csa_bf16* q, const csa_cache_t* kv, const csa_bf16* win,
+                     const int32_t* win_len, const int32_t* idx, const int32_t* count, int32_t B,
+                     int32_t H, int32_t top_k, int32_t window, float sm_scale, const float* sink,
+                     csa_bf16* out, float* lse) {
   AttnArgs a{};
   a.q = (const __nv_bfloat16*)q;
   a.T = B;
   a.H = H;
-  a.kv = to_ref(kv_comp);
+  a.kv = to_ref(kv);
   a.seq_per_query = 1;
   a.idx = idx;
   a.top_k = top_k;
@@ -648,24 +663,91 @@ csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_com
   a.sink = sink;
   a.out = (__nv_bfloat16*)out;
   a.lse = lse;
-  const Split sp_ws = attn_split(B, (int64_t)top_k + window, H);
-  const bool invariant = g_batch_invariant.load(std::memory_order_relaxed) != 0;
-  const Split sp_inv = attn_split_invariant((int64_t)top_k + window);
-  const int n_need = invariant && sp_inv.n > sp_ws.n ? sp_inv.n : sp_ws.n;
-  if ((st = check_ws(ws, ws_bytes, attn_partials_bytes(B, H, n_need), name)) != CSA_OK) return st;
-  a.use_tc = attention_uses_tc(a);
-  const Split sp = invariant ? sp_inv
-                             : (a.use_tc ? attn_split_tc(B, (int64_t)top_k + window, H, sp_ws) : sp_ws);
-  a.n_split = sp.n;
-  a.split_len = sp.len;
-  a.err = static_cast<WsHeader*>(ws);
-  if (sp.n > 1) {
-    char* p = static_cast<char*>(ws) + kWsHeader;
-    a.part_acc = reinterpret_cast<float*>(p);
-    a.part_ml = reinterpret_cast<float*>(p + align256((size_t)B * sp.n * H * kD * sizeof(float)));
-  }
+  return a;
+}
+
+csa_status_t check_decode_args(const char* name, const csa_bf16* q, const csa_cache_t* kv,
+                               const csa_bf16* win, const int32_t* win_len, const int32_t* idx,
+                               const int32_t* count, int32_t B, int32_t H, int32_t d,
+                               int32_t top_k, int32_t window, const csa_bf16* out) {
+  csa_status_t st = check_attn_common(name, q, out, H, d, window);
+  if (st != CSA_OK) return st;
+  if ((st = check_cache(kv, name)) != CSA_OK) return st;
+  if (idx == nullptr || count == nullptr || B < 0 || top_k < 1)
+    return fail(CSA_ERR_INVALID_ARG, "%s: idx, count required; B >= 0, top_k >= 1", name);
+  if (window > 0 && (win == nullptr || win_len == nullptr))
+    return fail(CSA_ERR_INVALID_ARG, "%s: window > 0 needs win and win_len", name);
+  return CSA_OK;
+}
+
+}  // namespace
+
+csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_comp,
+                                    const csa_bf16* win, const int32_t* win_len,
+                                    const int32_t* idx, const int32_t* count, int32_t B,
+                                    int32_t H, int32_t d, int32_t top_k, int32_t window,
+                                    float sm_scale, const float* sink, csa_bf16* out,
+                                    float* lse, void* ws, size_t ws_bytes,
+                                    csa_stream_t stream) {
+  const char* name = "csa_sparse_attn_decode";
+  if (B == 0) return CSA_OK;
+  csa_status_t st =
+      check_decode_args(name, q, kv_comp, win, win_len, idx, count, B, H, d, top_k, window, out);
+  if (st != CSA_OK) return st;
+  const AttnArgs a = decode_args(q, kv_comp, win, win_len, idx, count, B, H, top_k, window,
+                                 sm_scale, sink, out, lse);
+  return run_decode_attention(a, name, B, H, top_k, window, ws, ws_bytes, stream);
+}
+
+csa_status_t csa_quantize_entries_fp8(const csa_bf16* x, int64_t n, int32_t dim, int32_t rope_dims,
+                                      uint8_t* codes, uint8_t* scales, csa_bf16* rope,
+                                      csa_stream_t stream) {
+  const char* name = "csa_quantize_entries_fp8";
+  if (n < 0 || dim < 8 || dim % 8 != 0 || rope_dims < 0 || rope_dims % 8 != 0 ||
+      rope_dims >= dim || (dim - rope_dims) % 32 != 0)
+    return fail(CSA_ERR_INVALID_ARG,
+                "%s: need n >= 0, dim a multiple of 8, rope_dims a multiple of 8 below dim and "
+                "dim - rope_dims a multiple of 32", name);
+  if (n == 0) return CSA_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr || (rope_dims > 0 && rope == nullptr))
+    return fail(CSA_ERR_INVALID_ARG, "%s: x, codes, scales (and rope when rope_dims > 0) required",
+                name);
+  if (!aligned16(x) || !aligned16(codes) || (rope && !aligned16(rope)))
+    return fail(CSA_ERR_INVALID_ARG, "%s: x, codes and rope must be 16-byte aligned", name);
   Launch L{(cudaStream_t)stream};
-  return cuda_status(launch_attention(L, a), name);
+  return cuda_status(launch_fp8_entry_quantize(L, (const __nv_bfloat16*)x, n, dim, rope_dims,
+                                               codes, scales, (__nv_bfloat16*)rope),
+                     name);
+}
+
+csa_status_t csa_sparse_attn_decode_fp8(const csa_bf16* q, const csa_cache_t* kv_codes,
+                                        const uint8_t* kv_scales, const csa_bf16* kv_rope,
+                                        int32_t rope_dims, const csa_bf16* win,
+                                        const int32_t* win_len, const int32_t* idx,
+                                        const int32_t* count, int32_t B, int32_t H, int32_t d,
+                                        int32_t top_k, int32_t window, float sm_scale,
+                                        const float* sink, csa_bf16* out, float* lse, void* ws,
+                                        size_t ws_bytes, csa_stream_t stream) {
+  const char* name = "csa_sparse_attn_decode_fp8";
+  if (B == 0) return CSA_OK;
+  csa_status_t st =
+      check_decode_args(name, q, kv_codes, win, win_len, idx, count, B, H, d, top_k, window, out);
+  if (st != CSA_OK) return st;
+  if (rope_dims < 0 || rope_dims % 8 != 0 || rope_dims >= kD || (kD - rope_dims) % 32 != 0)
+    return fail(CSA_ERR_INVALID_ARG,
+                "%s: rope_dims must be a multiple of 8 below 128 with 128 - rope_dims a multiple "
+                "of 32 (got %d)", name, rope_dims);
+  if (kv_scales == nullptr || (rope_dims > 0 && kv_rope == nullptr))
+    return fail(CSA_ERR_INVALID_ARG, "%s: kv_scales (and kv_rope when rope_dims > 0) required", name);
+  if (kv_rope && !aligned16(kv_rope))
+    return fail(CSA_ERR_INVALID_ARG, "%s: kv_rope must be 16-byte aligned", name);
+  AttnArgs a = decode_args(q, kv_codes, win, win_len, idx, count, B, H, top_k, window, sm_scale,
+                           sink, out, lse);
+  a.kv_fp8 = 1;
+  a.kv_scales = kv_scales;
+  a.kv_rope = (const __nv_bfloat16*)kv_rope;
+  a.rope_dims = rope_dims;
+  return run_decode_attention(a, name, B, H, top_k, window, ws, ws_bytes, stream);
 }
 
 csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_bf16* kv_win,

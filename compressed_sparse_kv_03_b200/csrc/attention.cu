@@ -13,8 +13,12 @@
 // shared tile; QK^T and PV run on tensor cores (mma.sync m16n8k16, bf16 in,
 // fp32 accumulate) with an online softmax in the log2 domain.  A slice writes
 // either the final output (one slice) or (acc, max, sum) partials that the
-// merge kernel combines.
+// merge kernel combines.  With mixed-precision entries (E4M3 content with a
+// scale byte per 32, bf16 rotary part: Ch.8 "V4 compressed-entry payload")
+// the gather expands each entry exactly to bf16 in the tile, so the rest of
+// the kernel is unchanged.
 #include "kernels.h"
+#include "lowprec.cuh"
 
 namespace csa {
 
@@ -32,6 +36,7 @@ __global__ void __launch_bounds__(NW * 32) attn_kernel(AttnArgs a) {
   constexpr int NTH = NW * 32;
   __shared__ alignas(128) __nv_bfloat16 sKV[2][BN * D];
   __shared__ const __nv_bfloat16* sRow[2][BN];
+  __shared__ int64_t sPhys[2][BN];   // mixed-precision entries: physical row, else -1
   __shared__ uint32_t sMask[2][2];
 
   const int64_t i = blockIdx.x;
@@ -70,33 +75,64 @@ __global__ void __launch_bounds__(NW * 32) attn_kernel(AttnArgs a) {
   const int64_t v1 = total < v0 + a.split_len ? total : v0 + a.split_len;
   const int ntiles = v1 > v0 ? (int)((v1 - v0 + BN - 1) / BN) : 0;
 
-  auto row_ptr = [&](int64_t v) -> const __nv_bfloat16* {
-    if (v >= v1) return nullptr;
-    if (v < n_sel) {
-      const int64_t e = a.idx ? (int64_t)__ldg(a.idx + i * a.top_k + v) : v;
-      const int64_t r = cache_row(a.kv, seq, e, a.err, (int32_t)i);
-      return r < 0 ? nullptr : a.kv.data + r * D;
-    }
-    const int64_t w = v - n_sel;
-    return a.win_len ? a.win + (i * a.window + w) * D : a.win + (win_first + w) * D;
-  };
+  // A row of the list is a bf16 row (sRow) or, with mixed-precision entries,
+  // the physical row of an entry (sPhys); invalid rows have neither.
   auto fill_rows = [&](int st, int tt) {
     for (int r0 = warp * 32; r0 < BN; r0 += NTH) {
       const int r = r0 + lane;
-      const __nv_bfloat16* p = row_ptr(v0 + (int64_t)tt * BN + r);
+      const int64_t v = v0 + (int64_t)tt * BN + r;
+      const __nv_bfloat16* p = nullptr;
+      int64_t phys = -1;
+      if (v < v1) {
+        if (v < n_sel) {
+          const int64_t e = a.idx ? (int64_t)__ldg(a.idx + i * a.top_k + v) : v;
+          const int64_t rr = cache_row(a.kv, seq, e, a.err, (int32_t)i);
+          if (rr >= 0) {
+            if (a.kv_fp8) phys = rr;
+            else p = a.kv.data + rr * D;
+          }
+        } else {
+          const int64_t w = v - n_sel;
+          p = a.win_len ? a.win + (i * a.window + w) * D : a.win + (win_first + w) * D;
+        }
+      }
       sRow[st][r] = p;
-      const uint32_t bits = __ballot_sync(0xffffffffu, p != nullptr);
+      sPhys[st][r] = phys;
+      const uint32_t bits = __ballot_sync(0xffffffffu, p != nullptr || phys >= 0);
       if (lane == 0) sMask[st][r0 >> 5] = bits;
     }
   };
+  // bf16 rows (and the rotary part of mixed-precision entries) arrive by
+  // cp.async; an entry's E4M3 content is loaded, scaled and stored as exact
+  // bf16 values in the same swizzled place
+  const int dc8 = (D - a.rope_dims) / 8;   // 16-byte chunks of E4M3 content
+  const uint8_t* kv_codes = reinterpret_cast<const uint8_t*>(a.kv.data);
   auto issue_tile = [&](int st) {
     const uint32_t base = smem_u32(sKV[st]);
 #pragma unroll
     for (int c = tid; c < BN * 16; c += NTH) {
       const int r = c >> 4, ch = c & 15;
       const __nv_bfloat16* src = sRow[st][r];
-      const uint32_t dst = base + (uint32_t)(r * D + ((ch ^ (r & 7)) << 3)) * 2u;
-      cp_async_16(dst, src ? src + ch * 8 : a.q, src != nullptr);
+      const uint32_t off = (uint32_t)(r * D + ((ch ^ (r & 7)) << 3));
+      const int64_t phys = a.kv_fp8 ? sPhys[st][r] : -1;
+      if (phys < 0) {
+        cp_async_16(base + off * 2u, src ? src + ch * 8 : a.q, src != nullptr);
+      } else if (ch < dc8) {
+        const uint2 cw = __ldg(reinterpret_cast<const uint2*>(kv_codes + phys * (8 * dc8) + 8 * ch));
+        const float fs = lowprec::e8m0_to_float(__ldg(a.kv_scales + phys * (dc8 / 4) + (ch >> 2)));
+        uint4 o;
+        o.x = pack_bf16(lowprec::e4m3_to_float(cw.x & 0xffu) * fs,
+                        lowprec::e4m3_to_float((cw.x >> 8) & 0xffu) * fs);
+        o.y = pack_bf16(lowprec::e4m3_to_float((cw.x >> 16) & 0xffu) * fs,
+                        lowprec::e4m3_to_float(cw.x >> 24) * fs);
+        o.z = pack_bf16(lowprec::e4m3_to_float(cw.y & 0xffu) * fs,
+                        lowprec::e4m3_to_float((cw.y >> 8) & 0xffu) * fs);
+        o.w = pack_bf16(lowprec::e4m3_to_float((cw.y >> 16) & 0xffu) * fs,
+                        lowprec::e4m3_to_float(cw.y >> 24) * fs);
+        *reinterpret_cast<uint4*>(&sKV[st][off]) = o;
+      } else {
+        cp_async_16(base + off * 2u, a.kv_rope + phys * a.rope_dims + (ch - dc8) * 8, true);
+      }
     }
   };
 
@@ -344,7 +380,7 @@ cudaError_t launch_merge(const Launch& L, const AttnArgs& a) {
 
 bool attention_uses_tc(const AttnArgs& a) {
   const int32_t choice = attention_kernel_choice();
-  return choice != 2 && tc_attention_supported(a);
+  return choice != 2 && !a.kv_fp8 && tc_attention_supported(a);
 }
 
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {

@@ -155,6 +155,14 @@ struct AttnArgs {
   float* part_ml;               // [T, n_split, H, 2]
   WsHeader* err;
   int use_tc;                   // tcgen05 kernel (else mma.sync); see attention_uses_tc
+  // mixed-precision entries (kv_fp8 = 1, mma.sync kernel only): kv.data holds
+  // rows of 128 - rope_dims E4M3 codes, kv_scales rows of (128 - rope_dims)/32
+  // scale bytes and kv_rope rows of rope_dims bf16, all at the entry's
+  // physical row; window rows stay bf16
+  int kv_fp8 = 0;
+  const uint8_t* kv_scales = nullptr;
+  const __nv_bfloat16* kv_rope = nullptr;
+  int rope_dims = 0;
 };
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a);
 // tcgen05 path (d = 128; any H, in groups of 64 heads)
@@ -165,6 +173,12 @@ int32_t attention_kernel_choice();
 // the split / workspace ones must be set).
 bool attention_uses_tc(const AttnArgs& a);
 cudaError_t launch_attention_tc(const Launch& L, const AttnArgs& a);
+
+// [n, dim] bf16 entries -> E4M3 codes [n, dim - rope] + scale bytes
+// [n, (dim - rope)/32] + rotary part [n, rope] bf16: see fp8_entry.cu
+cudaError_t launch_fp8_entry_quantize(const Launch& L, const __nv_bfloat16* x, int64_t n, int dim,
+                                      int rope, uint8_t* codes, uint8_t* scales,
+                                      __nv_bfloat16* rope_out);
 
 // Text returned by csa_last_error() for this thread.
 void set_last_error(const char* msg);

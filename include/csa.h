@@ -368,6 +368,55 @@ csa_status_t csa_sparse_attn_decode_noalloc(const csa_bf16* q, const csa_cache_t
                                             float* lse, csa_stream_t stream);
 
 /*
+ * Mixed-precision compressed entries (Ch.8 "A Cost Model for Long Context",
+ * "V4 compressed-entry payload": the content channels in FP8, the last 64
+ * rotary channels in BF16, 576 bytes at c = 512; "Quantization scales and
+ * bounded tail buffers": block scale metadata).  The pages fix neither the
+ * FP8 variant nor the scale rule; the ones used:
+ *   element  E4M3 without infinities (sign, 4 exponent bits with bias 7,
+ *            field 0 subnormal, 3 mantissa bits), largest value 448
+ *   scale    one byte per 32 content coordinates, b = X + 127 for 2^X,
+ *            X = floor(log2 amax) - 8, clamped to [-127, 127] (-127 for an
+ *            all-zero block), as in the OCP Microscaling format
+ *   code     x / 2^X rounded to the nearest E4M3 value, ties to the even code,
+ *            saturating at 448; sign bit = sign bit of x
+ *   layout   an entry of dim coordinates, the last rope_dims of them rotary, is
+ *            dim - rope_dims code bytes, (dim - rope_dims)/32 scale bytes and
+ *            rope_dims bf16 values, in three arrays indexed by the same row
+ * Every dequantized value is a bf16 number.
+ *
+ * csa_quantize_entries_fp8 -- store n entries x [n, dim] bf16:
+ *   codes [n, dim - rope_dims] uint8, scales [n, (dim - rope_dims)/32] uint8,
+ *   rope [n, rope_dims] bf16 (NULL when rope_dims == 0)
+ * dim and rope_dims multiples of 8, rope_dims < dim, (dim - rope_dims) % 32 == 0;
+ * x, codes and rope 16-byte aligned.  Bit-exact.
+ */
+csa_status_t csa_quantize_entries_fp8(const csa_bf16* x, int64_t n, int32_t dim, int32_t rope_dims,
+                                      uint8_t* codes, uint8_t* scales, csa_bf16* rope,
+                                      csa_stream_t stream);
+
+/*
+ * csa_sparse_attn_decode_fp8 -- csa_sparse_attn_decode over mixed-precision
+ * entries: the attention of each query over its selected entries
+ * (dequantized, exactly bf16) and its bf16 window rows, with the same
+ * arguments, workspace (csa_sparse_attn_decode_workspace_size) and outputs.
+ *   kv_codes   cache whose rows are 128 - rope_dims code bytes (data 16-byte aligned)
+ *   kv_scales  [kv_codes->n_rows, (128 - rope_dims)/32] uint8
+ *   kv_rope    [kv_codes->n_rows, rope_dims] bf16 (16-byte aligned), or NULL when
+ *              rope_dims == 0; row r of each array belongs to physical row r
+ * d = 128; rope_dims a multiple of 8 with 128 - rope_dims a multiple of 32.  Runs
+ * on the mma.sync attention kernel whatever csa_set_attention_kernel says.
+ */
+csa_status_t csa_sparse_attn_decode_fp8(const csa_bf16* q, const csa_cache_t* kv_codes,
+                                        const uint8_t* kv_scales, const csa_bf16* kv_rope,
+                                        int32_t rope_dims, const csa_bf16* win,
+                                        const int32_t* win_len, const int32_t* idx,
+                                        const int32_t* count, int32_t B, int32_t H, int32_t d,
+                                        int32_t top_k, int32_t window, float sm_scale,
+                                        const float* sink, csa_bf16* out, float* lse, void* ws,
+                                        size_t ws_bytes, csa_stream_t stream);
+
+/*
  * hca_attn -- dense attention over every eligible heavily compressed entry
  * s < floor(t_i/m) plus the window, one softmax (Ch.7 "Dense attention over
  * heavily compressed history").

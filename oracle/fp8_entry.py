@@ -56,16 +56,16 @@ def e4m3_value(code):
 
 
 def e4m3_encode(y):
-    """Nearest E4M3 code of each y (reading F3): brute force over the 127
-    finite magnitudes, ties to the even code, saturation at 448."""
+    """Nearest E4M3 code of each y (reading F3): of the two finite magnitudes
+    that bracket |y| (clamped to 448: saturation) the nearer one, ties to the
+    even code."""
     y = np.asarray(y, dtype=np.float64)
     mags = e4m3_value(np.arange(E4M3_MAX_CODE + 1))         # increasing, 0 .. 448
     a = np.minimum(np.abs(y), mags[-1])
-    dist = np.abs(a[..., None] - mags)
-    best = dist.min(axis=-1, keepdims=True)
-    tied = dist == best
-    even = tied & (np.arange(E4M3_MAX_CODE + 1) % 2 == 0)
-    pick = np.where(even.any(axis=-1), np.argmax(even, axis=-1), np.argmax(tied, axis=-1))
+    hi = np.clip(np.searchsorted(mags, a, side="left"), 0, E4M3_MAX_CODE)   # mags[hi] >= a
+    lo = np.clip(hi - 1, 0, E4M3_MAX_CODE)
+    d_lo, d_hi = a - mags[lo], mags[hi] - a
+    pick = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, np.where(lo % 2 == 0, lo, hi)))
     sign = np.signbit(y).astype(np.int64)
     return (pick + 128 * sign).astype(np.uint8)
 

@@ -112,9 +112,11 @@ CFG_MIXED = MixedDecode("mixed_decode_B16_N256K_1M", B=16, N_lo=1 << 18, N_hi=1 
 # The 128K decode with the indexer keys and queries held in 4-bit storage
 # (same seeded inputs; the keys are quantized when the cache is built).
 CFG_DECODE_128K_MXFP4 = dataclasses.replace(CFG_DECODE_128K, name="csa_decode_B64_N131072_mxfp4_indexer")
+# ... and the main entries in FP8 content + bf16 rotary storage as well.
+CFG_DECODE_128K_LOWPREC = dataclasses.replace(CFG_DECODE_128K, name="csa_decode_B64_N131072_lowprec")
 
 WORKLOADS = {c.name: c for c in (CFG_PREFILL_4K, CFG_DECODE_128K, CFG_PREFILL_64K, CFG_HCA_1M,
-                                 CFG_MIXED, CFG_DECODE_128K_MXFP4)}
+                                 CFG_MIXED, CFG_DECODE_128K_MXFP4, CFG_DECODE_128K_LOWPREC)}
 
 
 # ---------------------------------------------------------------------------

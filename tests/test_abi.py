@@ -180,3 +180,33 @@ def test_mxfp4_calls_reject_bad_arguments_without_launching(lib):
     a = list(args); a[16] = 256
     assert lib.csa_indexer_topk_mxfp4(*a) == 5
     assert lib.csa_launch_count() == before
+
+
+def test_fp8_entry_calls_reject_bad_arguments_without_launching(lib):
+    from compressed_sparse_kv_03_b200._lib import CacheT
+    before = lib.csa_launch_count()
+    buf = (C.c_uint8 * 4096)()
+    p = C.c_void_p((C.addressof(buf) + 255) // 256 * 256)
+    # content part not a multiple of 32, rope not below dim, missing rotary output
+    assert lib.csa_quantize_entries_fp8(p, 4, 128, 48, p, p, p, None) == 1
+    assert b"multiple of 32" in lib.csa_last_error()
+    assert lib.csa_quantize_entries_fp8(p, 4, 128, 128, p, p, p, None) == 1
+    assert lib.csa_quantize_entries_fp8(p, 4, 128, 64, p, p, None, None) == 1
+    assert lib.csa_quantize_entries_fp8(p, 0, 128, 64, None, None, None, None) == 0
+    cache = CacheT(p.value, 16, 16, None, 0, 0)
+    # q, kv_codes, kv_scales, kv_rope, rope_dims, win, win_len, idx, count, B, H, d,
+    # top_k, window, sm_scale, sink, out, lse, ws, ws_bytes, stream
+    args = [p, C.byref(cache), p, p, 64, p, p, p, p, 2, 8, 128, 16, 4, 0.1, None, p, None, p,
+            1 << 20, None]
+    a = list(args); a[4] = 40            # 128 - 40 not a multiple of 32
+    assert lib.csa_sparse_attn_decode_fp8(*a) == 1 and b"rope_dims" in lib.csa_last_error()
+    a = list(args); a[11] = 64           # head dim not built
+    assert lib.csa_sparse_attn_decode_fp8(*a) == 2
+    a = list(args); a[2] = None          # scales missing
+    assert lib.csa_sparse_attn_decode_fp8(*a) == 1 and b"kv_scales" in lib.csa_last_error()
+    # workspace too small: a shape whose split needs partials (so that the
+    # check, not a launch, ends the call)
+    a = list(args); a[10], a[12], a[13], a[19] = 64, 2048, 128, 256
+    assert lib.csa_sparse_attn_decode_workspace_size(2, 64, 128, 2048, 128) > 256
+    assert lib.csa_sparse_attn_decode_fp8(*a) == 5
+    assert lib.csa_launch_count() == before

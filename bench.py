@@ -764,12 +764,13 @@ def run_ours(args, rank, world, local_rank):
 
 
 
-def recorded_traffic(kernel, config):
+def recorded_traffic(kernel, config, root=None):
     """DRAM bytes per launch of `kernel` on this workload from a committed ncu
-    capture (profiles/dram_traffic.json), or None when there is none or the
-    kernel's source changed since it was taken."""
+    capture (profiles/dram_traffic.json under `root`, default this directory),
+    or None when there is none or the kernel's source changed since it was
+    taken."""
     import hashlib
-    here = os.path.dirname(os.path.abspath(__file__))
+    here = root or os.path.dirname(os.path.abspath(__file__))
     try:
         with open(os.path.join(here, "profiles", "dram_traffic.json")) as f:
             entries = json.load(f)["entries"]

@@ -13,7 +13,7 @@ rounded to bf16 (the bytes the GPU sees, widened).  No blocking, fusion or
 reordering beyond the definitions: each function is the formula written out,
 with numpy's matmul / sort as the only library steps.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   R1  causal rule with 0-based positions: query t may use entry s iff
       s < floor(t/m) (Ch.5 "Causal availability and the local sliding window").
   R2  the window holds the raw tokens max(0, t-W+1) .. t, the current token

@@ -14,7 +14,7 @@ Source pages:
   * Ch.7 "Partial RoPE and output de-rotation" (the rotary slice is the last
     64 coordinates).
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   F1  "FP8" is E4M3 without infinities (1 sign, 4 exponent bits with bias 7,
       3 mantissa bits; exponent field 0 is subnormal; the all-ones pattern is
       NaN): largest magnitude 448, smallest 2^-9.

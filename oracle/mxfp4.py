@@ -13,7 +13,7 @@ Source pages:
     versus indexer arithmetic" (the indexer scan runs on four-bit dot
     products).
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   Q1  "FP4" is the E2M1 element type (1 sign, 2 exponent, 1 mantissa bit,
       exponent bias 1, no inf / NaN): magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.
   Q2  the 1-byte scale is a power of two stored as a biased exponent

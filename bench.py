@@ -804,7 +804,7 @@ def main():
     ap.add_argument("--batch-invariant", action="store_true",
                     help="decode attention in batch-invariant mode (fixed 512-row slices)")
     ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu dram bytes per launch of the dominant kernel, if captured for this build")
+                    help="ncu dram bytes per launch of the dominant kernel, if captured for the current kernel source")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -527,9 +527,9 @@ def oracle_sample(name, budget_s):
         b = done
         for lay in host["layers"]:
             S = int(lay["S"][b])
-            kv_b = f(synth.unpage(lay["kv_pool"], lay["page_table"][b], S, cfg.page_size))
+            kv_b = f(oracle.unpage(lay["kv_pool"], lay["page_table"][b], S, cfg.page_size))
             if lay["kind"] == "csa":
-                kI_b = f(synth.unpage(lay["kI_pool"], lay["page_table"][b], S, cfg.page_size))
+                kI_b = f(oracle.unpage(lay["kI_pool"], lay["page_table"][b], S, cfg.page_size))
                 oracle.csa_decode(f(lay["q"][b:b + 1]), [kv_b], [kI_b], f(lay["qI"][b:b + 1]),
                                   f(lay["w"][b:b + 1]), f(lay["win"][b:b + 1]),
                                   lay["win_len"][b:b + 1].numpy(), host["pos"][b:b + 1].numpy(),

@@ -72,7 +72,7 @@ SIGNATURES = {
     "csa_sparse_attn_decode_fp8": (C.c_int, [_vp, C.POINTER(CacheT), _vp, _vp, _i32, _vp, _vp, _vp,
                                              _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp,
                                              _vp, _vp, _sz, _vp]),
-    "hca_attn": (C.c_int, [_vp, C.POINTER(CacheT), _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i64,
+    "hca_attn": (C.c_int, [_vp, C.POINTER(CacheT), _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i64,
                            _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "csa_sparse_attn_decode_noalloc": (C.c_int, [_vp, C.POINTER(CacheT), _vp, _vp, _vp, _vp, _i32,
                                                  _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp,

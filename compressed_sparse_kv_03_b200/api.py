@@ -416,10 +416,13 @@ def sparse_attn_decode_fp8(q, codes: Cache, scales, rope, win, win_len, idx, cou
     return (out, lse) if return_lse else out
 
 def hca_attn(q, kv: Cache, kv_win, m, window, sm_scale, *, win_len=None, q_pos=None,
-             max_entries=None, sink=None, return_lse=False, ws=None, stream=None, out=None):
+             seq_id=None, max_entries=None, sink=None, return_lse=False, ws=None, stream=None,
+             out=None):
     """Step 4 (HCA): dense attention over every entry s < floor(t/m) plus the
-    window.  Decode when `win_len` is given (kv_win [T, window, d]); prefill of
-    sequence 0 otherwise (kv_win = raw tokens [*, d])."""
+    window.  Decode when `win_len` is given (kv_win [T, window, d]; query i
+    reads sequence seq_id[i], default i); prefill otherwise: of sequence 0
+    (kv_win = its raw tokens [*, d]), or, with `seq_id` and `q_pos`, of packed
+    sequences whose raw rows kv_win [T, d] line up with the queries."""
     _need(q, "q", torch.bfloat16, 3)
     T, H, d = q.shape
     dev = q.device
@@ -430,6 +433,10 @@ def hca_attn(q, kv: Cache, kv_win, m, window, sm_scale, *, win_len=None, q_pos=N
         _need(kv_win, "kv_win", torch.bfloat16, 2, dev)
     if q_pos is not None:
         _need(q_pos, "q_pos", torch.int64, 1, dev)
+    if seq_id is not None:
+        _need(seq_id, "seq_id", torch.int32, 1, dev)
+        if win_len is None and q_pos is None:
+            raise ValueError("packed prefill (seq_id without win_len) needs q_pos")
     if sink is not None:
         _need(sink, "sink", torch.float32, 1, dev)
     if max_entries is None:
@@ -443,7 +450,8 @@ def hca_attn(q, kv: Cache, kv_win, m, window, sm_scale, *, win_len=None, q_pos=N
     lib = load()
     wsp, wsb = _ws(ws, dev).get(lib.hca_attn_workspace_size(T, H, d, max_entries, window))
     kc = kv.c()
-    check(lib.hca_attn(_ptr(q), C.byref(kc), _ptr(kv_win), _ptr(win_len), _ptr(q_pos), T, H, d, m,
+    check(lib.hca_attn(_ptr(q), C.byref(kc), _ptr(kv_win), _ptr(win_len), _ptr(seq_id), _ptr(q_pos),
+                       T, H, d, m,
                        max_entries, window, float(sm_scale), _ptr(sink), _ptr(out), _ptr(lse), wsp,
                        wsb, _stream(stream)))
     return (out, lse) if return_lse else out

@@ -682,6 +682,21 @@ csa_status_t check_decode_args(const char* name, const csa_bf16* q, const csa_ca
 
 }  // namespace
 
+}  // extern "C"
+
+// Host-side argument checks of a decode attention call, for the entry points
+// that wrap csa_sparse_attn_decode (internal linkage to the C ABI: not exported
+// under a C name).
+csa_status_t csa::check_decode_call(const char* name, const csa_bf16* q, const csa_cache_t* kv,
+                                    const csa_bf16* win, const int32_t* win_len,
+                                    const int32_t* idx, const int32_t* count, int32_t B,
+                                    int32_t H, int32_t d, int32_t top_k, int32_t window,
+                                    const csa_bf16* out) {
+  return check_decode_args(name, q, kv, win, win_len, idx, count, B, H, d, top_k, window, out);
+}
+
+extern "C" {
+
 csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_comp,
                                     const csa_bf16* win, const int32_t* win_len,
                                     const int32_t* idx, const int32_t* count, int32_t B,
@@ -751,7 +766,8 @@ csa_status_t csa_sparse_attn_decode_fp8(const csa_bf16* q, const csa_cache_t* kv
 }
 
 csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_bf16* kv_win,
-                      const int32_t* win_len, const int64_t* q_pos, int64_t T, int32_t H,
+                      const int32_t* win_len, const int32_t* seq_id, const int64_t* q_pos,
+                      int64_t T, int32_t H,
                       int32_t d, int32_t m, int64_t max_entries, int32_t window,
                       float sm_scale, const float* sink, csa_bf16* out, float* lse, void* ws,
                       size_t ws_bytes, csa_stream_t stream) {
@@ -774,6 +790,7 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
   a.H = H;
   a.kv = to_ref(kv_comp);
   a.seq_per_query = win_len != nullptr ? 1 : 0;
+  a.seq_id = seq_id;
   a.idx = nullptr;
   a.top_k = 0;
   a.count = nullptr;
@@ -783,7 +800,8 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
   a.win = (const __nv_bfloat16*)kv_win;
   a.win_len = win_len;
   a.window = window;
-  a.win_rows = (win_len == nullptr && q_pos == nullptr) ? T : 0;
+  // raw rows known: all T of them when query i is row i (no q_pos, or packed)
+  a.win_rows = (win_len == nullptr && (q_pos == nullptr || seq_id != nullptr)) ? T : 0;
   a.sm_scale = sm_scale;
   a.sink = sink;
   a.out = (__nv_bfloat16*)out;

@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(NW * 32) attn_kernel(AttnArgs a) {
 
   // ---- this query's virtual row list ----
   const int64_t pos = a.q_pos ? __ldg(a.q_pos + i) : i;
-  const int32_t seq = a.seq_per_query ? (int32_t)i : 0;
+  const int32_t seq = attn_seq(a, i);
   int64_t n_sel;
   if (a.idx) {
     n_sel = __ldg(a.count + i);
@@ -67,8 +67,7 @@ __global__ void __launch_bounds__(NW * 32) attn_kernel(AttnArgs a) {
       n_win = n_win < 0 ? 0 : a.window;
     }
   } else {
-    n_win = pos + 1 < a.window ? pos + 1 : a.window;
-    win_first = pos - n_win + 1;
+    win_first = attn_raw_window(a, i, pos, n_win, split == 0 && tid == 0 && blockIdx.z == 0);
   }
   const int64_t total = n_sel + n_win;
   const int64_t v0 = (int64_t)split * a.split_len;

@@ -107,7 +107,7 @@ __device__ __forceinline__ ItemInfo item_info(const AttnArgs& a, int hgroups, in
   it.split = (int)(rest % a.n_split);
   it.i = rest / a.n_split;
   it.pos = a.q_pos ? __ldg(a.q_pos + it.i) : it.i;
-  it.seq = a.seq_per_query ? (int32_t)it.i : 0;
+  it.seq = attn_seq(a, it.i);
   if (a.idx) {
     int64_t c = __ldg(a.count + it.i);
     it.n_sel = c < 0 ? 0 : (c > a.top_k ? a.top_k : c);
@@ -126,8 +126,7 @@ __device__ __forceinline__ ItemInfo item_info(const AttnArgs& a, int hgroups, in
       it.n_win = it.n_win < 0 ? 0 : a.window;
     }
   } else {
-    it.n_win = it.pos + 1 < a.window ? it.pos + 1 : a.window;
-    it.win_first = it.pos - it.n_win + 1;
+    it.win_first = attn_raw_window(a, it.i, it.pos, it.n_win, do_report && it.split == 0 && it.hg == 0);
   }
   const int64_t total = it.n_sel + it.n_win;
   it.v0 = (int64_t)it.split * a.split_len;

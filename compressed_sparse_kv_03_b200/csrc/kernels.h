@@ -132,6 +132,9 @@ struct AttnArgs {
   int H;
   CacheRef kv;                  // compressed entries
   int seq_per_query;            // 1: query i reads sequence i; 0: all read sequence 0
+  const int32_t* seq_id = nullptr;   // [T]: query i reads sequence seq_id[i] (overrides
+                                     // seq_per_query); without win_len the raw rows are
+                                     // packed: query i is raw row i of `win`
   // entry list: explicit (idx != null) or all s < floor(pos/m)
   const int32_t* idx;
   int top_k;
@@ -165,6 +168,27 @@ struct AttnArgs {
   int rope_dims = 0;
 };
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a);
+
+// Sequence whose compressed entries query i reads.
+__device__ __forceinline__ int32_t attn_seq(const AttnArgs& a, int64_t i) {
+  return a.seq_id ? __ldg(a.seq_id + i) : (a.seq_per_query ? (int32_t)i : 0);
+}
+
+// Window of query i at position pos when the window comes from raw rows
+// (win_len null): n_win = min(pos + 1, window) rows ending at the query's own
+// raw row -- row pos of `win`, or row i when the rows are packed (seq_id
+// given).  A packed row list that would start before row 0 is cut there and
+// reported (kErrWindow).  Returns the first row; sets n_win.
+__device__ __forceinline__ int64_t attn_raw_window(const AttnArgs& a, int64_t i, int64_t pos,
+                                                   int64_t& n_win, bool do_report) {
+  n_win = pos + 1 < a.window ? pos + 1 : a.window;
+  const int64_t last = a.seq_id ? i : pos;
+  if (last - n_win + 1 < 0) {
+    if (do_report) report(a.err, kErrWindow, (int32_t)i, pos);
+    n_win = last + 1;
+  }
+  return last - n_win + 1;
+}
 // tcgen05 path (d = 128; any H, in groups of 64 heads)
 bool tc_attention_supported(const AttnArgs& a);
 // 0 automatic, 1 tensor-core kernel, 2 mma.sync kernel
@@ -182,5 +206,12 @@ cudaError_t launch_fp8_entry_quantize(const Launch& L, const __nv_bfloat16* x, i
 
 // Text returned by csa_last_error() for this thread.
 void set_last_error(const char* msg);
+
+// Host-side argument checks of csa_sparse_attn_decode (B > 0): CSA_OK or the
+// status and message that call would return, with nothing enqueued.
+csa_status_t check_decode_call(const char* name, const csa_bf16* q, const csa_cache_t* kv,
+                               const csa_bf16* win, const int32_t* win_len, const int32_t* idx,
+                               const int32_t* count, int32_t B, int32_t H, int32_t d,
+                               int32_t top_k, int32_t window, const csa_bf16* out);
 
 }  // namespace csa

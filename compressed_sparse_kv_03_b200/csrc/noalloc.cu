@@ -27,7 +27,10 @@ std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of the scratch on the current device, looked up once per
-// device (with that device current).
+// device (with that device current) and kept for the life of the process.  A
+// device reset (cudaDeviceReset, or anything else that destroys the primary
+// context) unloads the module; the array may then sit at another address, so
+// this form must not be called again in that process after such a reset.
 csa_status_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -66,6 +69,13 @@ extern "C" csa_status_t csa_sparse_attn_decode_noalloc(
     const int32_t* idx, const int32_t* count, int32_t B, int32_t H, int32_t d, int32_t top_k,
     int32_t window, float sm_scale, const float* sink, csa_bf16* out, float* lse,
     csa_stream_t stream) {
+  const char* name = "csa_sparse_attn_decode_noalloc";
+  // every argument check comes before the scratch is looked up or touched, so
+  // a rejected call enqueues nothing
+  if (B == 0) return CSA_OK;
+  csa_status_t st =
+      check_decode_call(name, q, kv_comp, win, win_len, idx, count, B, H, d, top_k, window, out);
+  if (st != CSA_OK) return st;
   const size_t need = csa_sparse_attn_decode_workspace_size(B, H, d, top_k, window);
   if (need > kNoAllocScratchBytes) {
     char buf[200];
@@ -77,7 +87,7 @@ extern "C" csa_status_t csa_sparse_attn_decode_noalloc(
     return CSA_ERR_WORKSPACE;
   }
   void* scratch = nullptr;
-  csa_status_t st = scratch_address(&scratch);
+  st = scratch_address(&scratch);
   if (st != CSA_OK) return st;
   // the device-check record at the head of the scratch must start clean
   cudaError_t e = cudaMemsetAsync(scratch, 0, kWsHeader, (cudaStream_t)stream);

@@ -27,10 +27,12 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
 
 // Pool rows row0 .. row0+m-1 of (C, Z) into the running accumulator; the bias
 // row for source j is bias[(j - row0) * dim].  kStream: read-only streaming
-// loads (rows not written by the running kernel); else plain loads.
+// loads (rows not written by the running kernel); else plain coherent loads,
+// for rows the calling thread has just written (C and Z are deliberately not
+// __restrict__, which would let the compiler turn those loads into
+// non-coherent read-only ones).
 template <bool kStream>
-__device__ __forceinline__ void pool_rows(Acc8& A, const __nv_bfloat16* __restrict__ C,
-                                          const __nv_bfloat16* __restrict__ Z,
+__device__ __forceinline__ void pool_rows(Acc8& A, const __nv_bfloat16* C, const __nv_bfloat16* Z,
                                           const float* __restrict__ bias, int64_t row0, int m,
                                           int dim, int c0) {
   for (int j0 = 0; j0 < m; j0 += kChunk) {

@@ -352,13 +352,21 @@ csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_com
  *     csa_sparse_attn_decode_workspace_size) fail with CSA_ERR_WORKSPACE and
  *     enqueue nothing; e.g. B = 64, H = 64, top_k = 2048, window = 128 needs
  *     about 10.6 MB.
+ *   - Argument errors (the same checks as csa_sparse_attn_decode) are returned
+ *     before the array is touched; B == 0 returns CSA_OK at once.
  *   - The first call on a device looks up the array's device address with that
- *     device current; make that first call before any stream capture.
+ *     device current and keeps it for the life of the process; make that first
+ *     call before any stream capture.  A device reset (cudaDeviceReset or
+ *     anything else that destroys the primary context) invalidates the kept
+ *     address: do not call this form again in that process after one.
  *   - Every call shares the one array, which keeps the last call's contents:
  *     calls that overlap on the GPU (other streams, other host threads) race.
  *     Each call clears the array's device-check header first; that record is
- *     not readable by the caller, so bad indices are skipped but not reported
- *     by this form.
+ *     not readable by the caller, so what the kernels record there -- bad entry
+ *     indices or page ids (skipped), and a pipeline wait that gave up (output
+ *     incomplete) -- is not reported by this form: a call can return CSA_OK
+ *     after either.  Callers that need those reports use
+ *     csa_sparse_attn_decode with csa_workspace_check.
  */
 csa_status_t csa_sparse_attn_decode_noalloc(const csa_bf16* q, const csa_cache_t* kv_comp,
                                             const csa_bf16* win, const int32_t* win_len,
@@ -420,20 +428,29 @@ csa_status_t csa_sparse_attn_decode_fp8(const csa_bf16* q, const csa_cache_t* kv
  * hca_attn -- dense attention over every eligible heavily compressed entry
  * s < floor(t_i/m) plus the window, one softmax (Ch.7 "Dense attention over
  * heavily compressed history").
- *   Decode (win_len != NULL): query i belongs to sequence i, sits at position
- *     q_pos[i] (required), and its window is kv_win[i, 0..win_len[i]-1]
- *     ([T, window, d], oldest first, itself last).
- *   Prefill (win_len == NULL): all queries belong to sequence 0; query i sits
- *     at position q_pos[i] (or i if q_pos is NULL); kv_win is the raw token
- *     sequence [*, d] and the window is rows max(0,t-W+1) .. t.
+ *   Decode (win_len != NULL): query i sits at position q_pos[i] (required) and
+ *     its window is kv_win[i, 0..win_len[i]-1] ([T, window, d], oldest first,
+ *     itself last); it reads the compressed entries of sequence seq_id[i], or
+ *     of sequence i when seq_id is NULL.
+ *   Prefill (win_len == NULL), one sequence (seq_id NULL): every query reads
+ *     sequence 0; query i sits at position q_pos[i] (or i if q_pos is NULL);
+ *     kv_win is that sequence's raw tokens [*, d] and the window is rows
+ *     max(0,t-W+1) .. t.
+ *   Prefill, packed sequences (seq_id given): the T queries are the tokens of
+ *     several sequences laid end to end; query i reads sequence seq_id[i]'s
+ *     entries, sits at position q_pos[i] within it (required) and is raw row i
+ *     of kv_win [T, d], so its window is rows i-n+1 .. i with
+ *     n = min(W, q_pos[i] + 1).  Those rows must belong to the same sequence
+ *     (the caller's layout); a window that would start before row 0 is cut
+ *     there and recorded in the workspace header.
  *   max_entries bounds floor(t_i/m) (split layout); q [T, H, d]; out [T, H, d];
- *   lse [T, H] or NULL; sink [H] or NULL.
+ *   lse [T, H] or NULL; sink [H] or NULL; seq_id [T] int32 or NULL.
  */
 csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_bf16* kv_win,
-                      const int32_t* win_len, const int64_t* q_pos, int64_t T, int32_t H,
-                      int32_t d, int32_t m, int64_t max_entries, int32_t window,
-                      float sm_scale, const float* sink, csa_bf16* out, float* lse, void* ws,
-                      size_t ws_bytes, csa_stream_t stream);
+                      const int32_t* win_len, const int32_t* seq_id, const int64_t* q_pos,
+                      int64_t T, int32_t H, int32_t d, int32_t m, int64_t max_entries,
+                      int32_t window, float sm_scale, const float* sink, csa_bf16* out,
+                      float* lse, void* ws, size_t ws_bytes, csa_stream_t stream);
 
 #ifdef __cplusplus
 }

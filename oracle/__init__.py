@@ -11,6 +11,8 @@ Every function is written from the DeepSeek-V4 book pages (slop-6tp.pages.dev,
 """
 from .csa_oracle import (  # noqa: F401
     bf16_round,
+    page_rows,
+    unpage,
     pool_block,
     pool_overlap,
     DecodeCacheState,

@@ -50,6 +50,31 @@ def bf16_round(x):
 
 
 # ---------------------------------------------------------------------------
+# paged compressed caches
+# ---------------------------------------------------------------------------
+def page_rows(table_row, n_entries, page_size):
+    """Physical rows of logical entries 0 .. n_entries-1 of one sequence of a
+    paged compressed cache: entry s sits in the page table_row[s // page_size]
+    at offset s % page_size, i.e. at physical row
+    table_row[s // page_size] * page_size + s % page_size.
+
+    The DeepSeek-V4 infrastructure transcript ("KV cache management": the
+    classical KV cache holds the CSA / HCA compressed entries, managed in
+    blocks) leaves the block addressing open; this is the plainest reading,
+    the usual block-table mapping of a paged cache.  Returns int64 [n_entries].
+    """
+    table = np.asarray(table_row, dtype=np.int64)
+    s = np.arange(int(n_entries), dtype=np.int64)
+    return table[s // page_size] * page_size + s % page_size
+
+
+def unpage(pool, table_row, n_entries, page_size):
+    """Logical [n_entries, dim] view of one sequence of a paged pool: the rows
+    page_rows(...) of `pool` (a numpy array or a CPU torch tensor)."""
+    return pool[page_rows(table_row, n_entries, page_size)]
+
+
+# ---------------------------------------------------------------------------
 # step 1: block compression by coordinate-wise softmax pooling
 # ---------------------------------------------------------------------------
 def _softmax_pool(content, logits):

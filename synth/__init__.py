@@ -245,14 +245,6 @@ def mixed_decode_inputs(cfg: MixedDecode, B=None):
     return dict(pos=N, layers=layers)
 
 
-def unpage(pool, table_row, n_entries, page_size):
-    """Logical [n_entries, dim] view of one sequence of a paged pool (a
-    gather, used to hand the oracle plain per-sequence arrays)."""
-    s = torch.arange(int(n_entries))
-    phys = table_row.to(torch.int64)[s // page_size] * page_size + s % page_size
-    return pool[phys]
-
-
 def random_topk_lists(g, T, k, n_eligible):
     """Valid entry lists for attention-only cases: per query a random subset
     of min(k, n_eligible[t]) distinct eligible entries, ascending, padded with

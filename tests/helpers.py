@@ -3,11 +3,20 @@
 Tolerances (stated once, used by every GPU parity test):
   * attention outputs and compressed entries: max |gpu - oracle| <= 2e-2 and
     mean |gpu - oracle| <= 5e-3 (bf16 inputs, fp32 accumulation, bf16 output)
-  * top-k sets: identical, except queries whose differing entries all have
-    oracle scores within the near-tie band of the oracle's k-th score:
-    |s - s_k| <= 1e-3 * max(|s|, |s_k|) + eps, where eps = 2^-20 * sum_h |w_h|
-    * sum_r |q_hr| * max_s |K_sr| bounds the fp32 accumulation error of one
-    score; such queries are reported, not failed
+  * top-k sets: identical, except near-tie queries, which are reported, not
+    failed.  A query counts as a near tie only if both of these hold:
+      (a) its oracle k-th and (k+1)-th scores s_k, s_k1 (rounded to fp32, the
+          precision both sides decide in) lie within 1e-3 relative:
+          |s_k - s_k1| <= 1e-3 * max(|s_k|, |s_k1|) + eps;
+      (b) every entry in the symmetric difference of the two sets has an
+          oracle score within the same band of s_k:
+          |s - s_k| <= 1e-3 * max(|s|, |s_k|) + eps.
+    (a) is the criterion as stated for this path; (b) adds that the sets may
+    differ only among entries at the boundary.  eps = 2^-20 * sum_h |w_h| *
+    sum_r |q_hr| * max_s |K_sr| bounds the fp32 accumulation error of one
+    score, so sign flips of near-zero dot products are not false failures.
+    Each test also bounds how many near-tie queries it accepts
+    (assert_mostly_exact: at most 1% of the queries, and at least one).
   * counts and index validity: exact
 """
 import numpy as np
@@ -60,7 +69,11 @@ def check_topk(gpu_idx_row, gpu_cnt, ora_scores, k, eps):
     ref = oracle.topk_select(ora_scores, k)
     if np.array_equal(sel, ref):
         return "exact"
-    kth = np.sort(ora_scores.astype(np.float32).astype(np.float64))[::-1][want_cnt - 1]
+    assert n > k, "with at most k eligible entries every one is selected: sets must match"
+    s32 = np.sort(ora_scores.astype(np.float32).astype(np.float64))[::-1]
+    kth, k1 = s32[want_cnt - 1], s32[want_cnt]
+    assert abs(kth - k1) <= TIE_REL * max(abs(kth), abs(k1)) + eps, \
+        f"top-k differs although the k-th and (k+1)-th scores are apart: {kth} vs {k1}"
     diff = np.setxor1d(sel, ref)
     s = ora_scores[diff]
     band = TIE_REL * np.maximum(np.abs(s), abs(kth)) + eps
@@ -68,3 +81,11 @@ def check_topk(gpu_idx_row, gpu_cnt, ora_scores, k, eps):
     assert not bad.any(), (f"top-k differs beyond the near-tie band: {diff[bad][:8]} "
                            f"scores {s[bad][:8]} vs k-th {kth}")
     return "near-tie"
+
+
+def assert_mostly_exact(stats, n_queries):
+    """Near-tie queries (see the module docstring) are reported, not failed,
+    but they must stay rare: at most 1% of the queries checked, and at least
+    one is always allowed."""
+    allowed = max(1, int(0.01 * n_queries))
+    assert stats["near-tie"] <= allowed, f"{stats['near-tie']} near-tie queries of {n_queries}: {stats}"

@@ -83,8 +83,8 @@ def test_attention_rejects_unsupported_dims(lib):
     assert st == 2
     # null cache data
     bad = CacheT(None, 16, 16, None, 0, 0)
-    st = lib.hca_attn(p, C.byref(bad), p, None, None, 4, 8, 128, 4, 16, 8, 1.0, None, p, None,
-                      wsp, 512, None)
+    st = lib.hca_attn(p, C.byref(bad), p, None, None, None, 4, 8, 128, 4, 16, 8, 1.0, None, p,
+                      None, wsp, 512, None)
     assert st == 1
     # decode with a window needs the window buffer
     st = lib.csa_sparse_attn_decode(p, C.byref(cache), None, None, p, p, 1, 8, 128, 4, 8, 1.0,
@@ -209,4 +209,32 @@ def test_fp8_entry_calls_reject_bad_arguments_without_launching(lib):
     a = list(args); a[10], a[12], a[13], a[19] = 64, 2048, 128, 256
     assert lib.csa_sparse_attn_decode_workspace_size(2, 64, 128, 2048, 128) > 256
     assert lib.csa_sparse_attn_decode_fp8(*a) == 5
+    assert lib.csa_launch_count() == before
+
+
+def test_noalloc_rejects_bad_arguments_before_touching_its_scratch(lib):
+    """The scratch-free decode form runs the decode call's argument checks
+    before it looks up or clears its static scratch: on a host without a GPU a
+    bad call still returns CSA_ERR_INVALID_ARG / CSA_ERR_UNSUPPORTED (not
+    CSA_ERR_CUDA), and B == 0 returns CSA_OK without loading anything."""
+    from compressed_sparse_kv_03_b200._lib import CacheT
+    before = lib.csa_launch_count()
+    buf = (C.c_uint8 * 4096)()
+    p = C.c_void_p((C.addressof(buf) + 255) // 256 * 256)
+    cache = CacheT(p.value, 16, 16, None, 0, 0)
+    # q, kv_comp, win, win_len, idx, count, B, H, d, top_k, window, sm_scale, sink, out, lse, stream
+    args = [p, C.byref(cache), p, p, p, p, 2, 8, 128, 16, 4, 0.1, None, p, None, None]
+    a = list(args); a[0] = None                  # no queries
+    assert lib.csa_sparse_attn_decode_noalloc(*a) == 1
+    assert b"csa_sparse_attn_decode_noalloc" in lib.csa_last_error()
+    a = list(args); a[4] = None                  # no selection
+    assert lib.csa_sparse_attn_decode_noalloc(*a) == 1
+    a = list(args); a[2] = None                  # window rows missing with window > 0
+    assert lib.csa_sparse_attn_decode_noalloc(*a) == 1
+    a = list(args); a[8] = 64                    # head dim not built
+    assert lib.csa_sparse_attn_decode_noalloc(*a) == 2
+    a = list(args); a[0] = C.c_void_p(p.value + 2)   # misaligned queries
+    assert lib.csa_sparse_attn_decode_noalloc(*a) == 1
+    a = list(args); a[6] = 0                     # nothing to do
+    assert lib.csa_sparse_attn_decode_noalloc(*a) == 0
     assert lib.csa_launch_count() == before

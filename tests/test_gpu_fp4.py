@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import synth
-from helpers import check_topk, dev, f64, score_eps
+from helpers import assert_mostly_exact, check_topk, dev, f64, score_eps
 from oracle import mxfp4 as ofp4
 
 pytestmark = pytest.mark.gpu
@@ -94,6 +94,7 @@ def _check_fp4_queries(idx, cnt, sc, q, w, keys_of, elig_of, k, queries):
         if sc is not None and cnt[t]:
             sel = idx[t, :cnt[t]]
             np.testing.assert_allclose(sc[t, :cnt[t]], s[sel], rtol=1e-5, atol=10 * eps + 1e-6)
+    assert_mostly_exact(stats, len(queries))
     return stats
 
 
@@ -189,8 +190,8 @@ def test_indexer_topk_mxfp4_paged(page_size):
                                       seq_id=dev(torch.arange(B, dtype=torch.int32)),
                                       q_pos=dev(pos), max_entries=max(S))
     _check_fp4_queries(idx, cnt, None, lambda b: (qc[b], qs[b]), w,
-                       lambda b: (synth.unpage(pool_c, table[b], S[b], page_size).numpy(),
-                                  synth.unpage(pool_s, table[b], S[b], page_size).numpy()),
+                       lambda b: (oracle.unpage(pool_c, table[b], S[b], page_size).numpy(),
+                                  oracle.unpage(pool_s, table[b], S[b], page_size).numpy()),
                        lambda b: S[b], k, range(B))
 
 

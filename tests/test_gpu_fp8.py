@@ -78,7 +78,7 @@ def _decode_case(g, B, H, k, paged, rope):
     cnt = torch.tensor(cnt_want, dtype=torch.int32)
     if paged:
         pool, table = synth.paged_pool(g, S, 128, 64)
-        seq_rows = lambda b: synth.unpage(pool, table[b], S[b], 64)   # noqa: E731
+        seq_rows = lambda b: oracle.unpage(pool, table[b], S[b], 64)   # noqa: E731
         store = dict(data=pool, page_table=table, page_size=64)
     else:
         Smax = max(S)

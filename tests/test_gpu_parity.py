@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import synth
-from helpers import assert_close_attn, check_topk, dev, f64, score_eps
+from helpers import assert_close_attn, assert_mostly_exact, check_topk, dev, f64, score_eps
 
 pytestmark = pytest.mark.gpu
 
@@ -129,7 +129,7 @@ def test_cache_append_matches_bulk_compression(overlap, paged, dim):
     if paged:
         pool, table = synth.paged_pool(g, [S + 3] * B, dim, 4)
         cache = csa.Cache(dev(torch.zeros_like(pool)), page_table=dev(table), page_size=4)
-        read = lambda b: synth.unpage(cache.data.cpu(), table[b], S, 4)
+        read = lambda b: oracle.unpage(cache.data.cpu(), table[b], S, 4)
     else:
         buf = torch.zeros((B, S + 3, dim), dtype=torch.bfloat16)
         cache = csa.Cache.contiguous(dev(buf))
@@ -189,6 +189,7 @@ def _check_queries(idx, cnt, qI, w, key_of_query, elig_of_query, k, queries, sco
         if sc is not None and cnt[t]:
             sel = idx[t, :cnt[t]]
             np.testing.assert_allclose(sc[t, :cnt[t]], s[sel], rtol=1e-5, atol=10 * eps + 1e-6)
+    assert_mostly_exact(stats, len(queries))
     return stats
 
 
@@ -275,7 +276,7 @@ def test_indexer_topk_paged(page_size):
     idx, cnt = csa.indexer_topk(dev(qI), dev(w), cache, m, k, seq_id=dev(torch.arange(B, dtype=torch.int32)),
                                 q_pos=dev(pos), max_entries=max(S))
     _check_queries(idx, cnt, qI, w,
-                   lambda b: f64(synth.unpage(pool, table[b], S[b], page_size)),
+                   lambda b: f64(oracle.unpage(pool, table[b], S[b], page_size)),
                    lambda b: S[b], k, range(B))
 
 
@@ -323,7 +324,7 @@ def test_sparse_attn_decode(B, H, k, paged, sink):
     if paged:
         pool, table = synth.paged_pool(g, S, 128, 64)
         cache = csa.Cache(dev(pool), page_table=dev(table), page_size=64)
-        logical = lambda b: f64(synth.unpage(pool, table[b], S[b], 64))
+        logical = lambda b: f64(oracle.unpage(pool, table[b], S[b], 64))
     else:
         Smax = max(S)
         kvc = synth.normal(g, (B, Smax, 128))
@@ -358,7 +359,7 @@ def test_hca_decode(B, H, m, paged):
     if paged:
         pool, table = synth.paged_pool(g, [max(s, 1) for s in S], 128, 64)
         cache = csa.Cache(dev(pool), page_table=dev(table), page_size=64)
-        logical = lambda b: f64(synth.unpage(pool, table[b], S[b], 64))
+        logical = lambda b: f64(oracle.unpage(pool, table[b], S[b], 64))
     else:
         kvc = synth.normal(g, (B, max(S), 128))
         cache = csa.Cache.contiguous(dev(kvc))
@@ -383,6 +384,41 @@ def test_hca_prefill():
     ref, _ = oracle.hca_prefill(f64(q), oracle.bf16_round(oracle.pool_block(f64(kv_raw), f64(Z), m)),
                                 f64(kv_raw), m, W, 1.0)
     assert_close_attn(out, ref, "hca prefill")
+
+
+@pytest.mark.usefixtures("attn_kernel")
+@pytest.mark.parametrize("paged", [False, True])
+def test_hca_prefill_packed_sequences(paged):
+    """Three sequences of 300, 517 and 1 tokens laid end to end: query i
+    reads the compressed entries of sequence seq_id[i] and its window from the
+    packed raw rows; each sequence must equal its own single-sequence HCA
+    prefill in the oracle."""
+    csa = _csa()
+    g = synth.generator(96 + int(paged))
+    lens, H, m, W = [300, 517, 1], 20, 8, 64
+    T = sum(lens)
+    q = synth.normal(g, (T, H, 128), 1 / math.sqrt(128))
+    kv_raw = synth.normal(g, (T, 128))
+    seq_id = torch.cat([torch.full((n,), b, dtype=torch.int32) for b, n in enumerate(lens)])
+    pos = torch.cat([torch.arange(n, dtype=torch.int64) for n in lens])
+    S = [max(n // m, 1) for n in lens]
+    if paged:
+        pool, table = synth.paged_pool(g, S, 128, 16)
+        cache = csa.Cache(dev(pool), page_table=dev(table), page_size=16)
+        logical = lambda b: f64(oracle.unpage(pool, table[b], S[b], 16))
+    else:
+        kvc = synth.normal(g, (len(lens), max(S), 128))
+        cache = csa.Cache.contiguous(dev(kvc))
+        logical = lambda b: f64(kvc[b])
+    out, lse = csa.hca_attn(dev(q), cache, dev(kv_raw), m, W, 1.0, seq_id=dev(seq_id),
+                            q_pos=dev(pos), max_entries=max(S), return_lse=True)
+    off = 0
+    for b, n in enumerate(lens):
+        ref, ref_lse = oracle.hca_prefill(f64(q[off:off + n]), logical(b), f64(kv_raw[off:off + n]),
+                                          m, W, 1.0)
+        assert_close_attn(out[off:off + n], ref, f"packed hca prefill, sequence {b}")
+        np.testing.assert_allclose(f64(lse[off:off + n]), ref_lse, atol=1e-3, rtol=1e-4)
+        off += n
 
 
 @pytest.mark.usefixtures("attn_kernel")
@@ -452,7 +488,7 @@ def test_batch_invariant_decode(paged):
         kpool = synth.normal(g, (pool.shape[0], 64))
         cache = lambda sel: csa.Cache(dev(pool), page_table=dev(table[sel]), page_size=64)
         kcache = lambda sel: csa.Cache(dev(kpool), page_table=dev(table[sel]), page_size=64)
-        logical = lambda b: f64(synth.unpage(pool, table[b], S[b], 64))
+        logical = lambda b: f64(oracle.unpage(pool, table[b], S[b], 64))
     else:
         kvc, kI = synth.normal(g, (B, max(S), 128)), synth.normal(g, (B, max(S), 64))
         cache = lambda sel: csa.Cache.contiguous(dev(kvc[sel]))

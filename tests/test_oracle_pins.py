@@ -658,3 +658,33 @@ def test_fp8_entry_values_are_bf16_numbers():
     codes, scales, rope = ofp8.entry_quantize(x, 64)
     y = ofp8.entry_dequantize(codes, scales, rope)
     assert np.array_equal(oracle.bf16_round(y), y)
+
+
+# ---------------------------------------------------------------------------
+# paged cache addressing (oracle.page_rows / oracle.unpage)
+# ---------------------------------------------------------------------------
+def test_page_rows_hand_mapping():
+    """Three sequences, pages of two rows, page ids written out by hand:
+    seq 0 holds pages (3, 0), seq 1 pages (1, 4), seq 2 page (2) and an unused
+    slot (-1).  Logical entry s of a sequence sits at row page * 2 + s % 2 of
+    the page table[s // 2]; the rows below are counted on paper."""
+    table = np.array([[3, 0], [1, 4], [2, -1]], dtype=np.int32)
+    assert list(oracle.page_rows(table[0], 4, 2)) == [6, 7, 0, 1]
+    assert list(oracle.page_rows(table[1], 3, 2)) == [2, 3, 8]
+    assert list(oracle.page_rows(table[2], 2, 2)) == [4, 5]
+    assert list(oracle.page_rows(table[2], 0, 2)) == []
+    # the sequences' rows never collide, and every used row of the pool is hit once
+    rows = np.concatenate([oracle.page_rows(table[0], 4, 2), oracle.page_rows(table[1], 4, 2),
+                           oracle.page_rows(table[2], 2, 2)])
+    assert sorted(rows) == list(range(10))
+
+
+def test_unpage_gathers_the_mapped_rows():
+    """A pool whose row r holds (r, -r): the logical view of a sequence is the
+    listed rows in logical order (a swapped page or a transposed offset fails).
+    Pages of 4 rows, table (5, 2, 0): entries 0-3 are rows 20-23, entry 4 is
+    row 8."""
+    pool = np.stack([np.arange(24.0), -np.arange(24.0)], axis=1)
+    table = np.array([5, 2, 0], dtype=np.int32)
+    want = np.array([[20, -20], [21, -21], [22, -22], [23, -23], [8, -8]], dtype=np.float64)
+    np.testing.assert_array_equal(oracle.unpage(pool, table, 5, 4), want)

@@ -362,7 +362,7 @@ class MixedDecode:
 
 
 KERNEL_NAMES = {0: "indexer_score", 1: "topk_select", 2: "attention", 3: "merge", 4: "compress",
-                5: "quantize"}
+                5: "quantize", 6: "topk_sample"}
 
 RUNNERS = {
     synth.CFG_DECODE_128K.name: (CsaDecode, synth.CFG_DECODE_128K),
@@ -583,7 +583,6 @@ def run_reference(args, rank, world):
 
 def run_ours(args, rank, world, local_rank):
     import compressed_sparse_kv_03_b200 as csa
-    import torch.distributed as dist
     torch.cuda.set_device(local_rank)
     cls, cfg = RUNNERS[args.workload]
     if args.batch and hasattr(cfg, "B"):
@@ -592,6 +591,34 @@ def run_ours(args, rank, world, local_rank):
         cfg = dataclasses.replace(cfg, L=args.seq_len, name=f"{cfg.name}_L{args.seq_len}")
     if args.batch_invariant:
         csa.set_batch_invariant(True)
+    line = measure(args, args.workload, cls, cfg, args.steps, args.warmup, rank, world, local_rank)
+    # the metric's prefill half: the L=65536 prefill measured in the same run
+    # (one GPU, default decode workload), as a sub-record with its own
+    # roofline (tensor) and oracle baseline
+    if (args.workload == DEFAULT_WORKLOAD and world == 1 and not args.no_prefill
+            and not args.batch and not args.batch_invariant):
+        import gc
+        gc.collect()
+        torch.cuda.empty_cache()
+        pname = synth.CFG_PREFILL_64K.name
+        pcls, pcfg = RUNNERS[pname]
+        sub = measure(args, pname, pcls, pcfg, max(3, min(args.steps, 5)), 3, rank, world,
+                      local_rank)
+        keep = ("metric", "value", "unit", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "dtype", "config", "roofline", "e2e", "clocks", "gpu_launches", "kernels_us",
+                "cpu_baseline")
+        line["prefill"] = {k: sub[k] for k in keep if k in sub}
+        line["prefill"]["metric"] = "CSA prefill tokens/s & tensor-core utilisation"
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measure(args, name, cls, cfg, K, warmup, rank, world, local_rank):
+    """Time one workload (warm-up, K timed graph replays, per-kernel
+    breakdown, end to end, oracle baseline on rank 0 at N=1) and return its
+    JSON record."""
+    import compressed_sparse_kv_03_b200 as csa
+    import torch.distributed as dist
     W = cls(cfg, seed_offset=rank_seed_offset(rank))
     pk = peaks()
     stream = torch.cuda.current_stream()
@@ -605,7 +632,7 @@ def run_ours(args, rank, world, local_rank):
             W.between_steps()
 
     # warm-up (eager)
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         W.step()
         between()
     torch.cuda.synchronize()
@@ -613,7 +640,6 @@ def run_ours(args, rank, world, local_rank):
     # one CUDA graph per timed step, each with its own events around the
     # dominant kernel; L2 flushes (where a workload needs them) run between
     # the step events, outside the timed time
-    K = args.steps
     kids = list(KERNEL_NAMES)
     kev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(K)] for k in kids}
@@ -638,15 +664,14 @@ def run_ours(args, rank, world, local_rank):
     launches_before = csa.launch_count()
     graphs, bgraphs = [], []
     if use_graph:
-        # timed graphs carry events around the dominant kernel only (each
-        # event node costs the step a little); the per-kernel breakdown comes
-        # from separate, untimed replays of graphs with events around every kernel
+        # timed graphs hold the step alone (an event node between two kernels
+        # would also stop them overlapping); the per-kernel times, the dominant
+        # kernel's included, come from separate, untimed replays of graphs with
+        # events around every kernel
         for i in range(K):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                csa.set_timing_events(W.dominant, ev[i][0], ev[i][1])
                 W.step()
-                csa.set_timing_events(W.dominant)
             graphs.append(g)
         launches = csa.launch_count() - launches_before
         for i in range(K):
@@ -681,7 +706,6 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clk = clocks.stop()
     ms = sum(b.elapsed_time(e) for b, e in st)
-    dom_ms = [b.elapsed_time(e) for b, e in ev]
     # per-kernel breakdown, outside the timed region
     for i in range(K):
         if use_graph:
@@ -692,6 +716,9 @@ def run_ours(args, rank, world, local_rank):
             detach()
         between()
     torch.cuda.synchronize()
+    # the dominant kernel: event times of its launches in the breakdown replays
+    # (graph mode) or in the timed eager steps
+    dom_ms = [b.elapsed_time(e) for b, e in ev]
     kernels_us = {}
     for k in kids:
         t = statistics.median(b.elapsed_time(e) for b, e in kev[k]) * 1e3
@@ -739,7 +766,7 @@ def run_ours(args, rank, world, local_rank):
                 "step_tc_frac": W.step_flops / (ms_per_step / 1e3) / 1e12 / peak}
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded torch CPU generator, N(0,1) / U(0,1))",
             "config": {**W.config(), "parallelism": f"dp{world}" + flush_note,
@@ -756,11 +783,11 @@ def run_ours(args, rank, world, local_rank):
                                    "each); for a kernel launched more than once in a step, its "
                                    "last launch"}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        u, s, desc, threads = oracle_sample(args.workload, args.cpu_budget)
+        u, s, desc, threads = oracle_sample(name, args.cpu_budget)
         line["cpu_baseline"] = {"value": u / s if s else 0.0, "unit": "tokens/s", "cores": threads,
                                 "kind": "oracle", "sample": desc}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    del W
+    return line
 
 
 
@@ -799,6 +826,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override the decode batch (profiling runs)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the prefill length (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill sub-record of the default decode run")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work (cpu_baseline)")
     ap.add_argument("--step-budget", type=float, default=4.0, help="seconds per reference-arm step")
     ap.add_argument("--batch-invariant", action="store_true",

@@ -5,7 +5,8 @@ The computation runs in the CUDA library ``_csa_b200.so`` (C ABI:
 include/csa.h); this package is its thin Python binding.
 """
 from ._lib import (CsaError, KERNEL_ATTENTION, KERNEL_COMPRESS, KERNEL_INDEXER_SCORE,  # noqa: F401
-                   KERNEL_MERGE, KERNEL_QUANTIZE, KERNEL_TOPK_SELECT, load)
+                   KERNEL_MERGE, KERNEL_QUANTIZE, KERNEL_TOPK_SAMPLE, KERNEL_TOPK_SELECT,
+                   load)
 from .api import (AppendState, Cache, Workspace, cache_append, compress_kv, hca_attn,  # noqa: F401
                   indexer_topk, indexer_topk_mxfp4, launch_count, norm_rope, quantize_entries_fp8,
                   quantize_mxfp4, set_attention_kernel, set_batch_invariant, set_timing_events,

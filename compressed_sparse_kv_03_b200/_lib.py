@@ -24,6 +24,7 @@ KERNEL_ATTENTION = 2
 KERNEL_MERGE = 3
 KERNEL_COMPRESS = 4
 KERNEL_QUANTIZE = 5
+KERNEL_TOPK_SAMPLE = 6
 
 
 class CsaError(RuntimeError):

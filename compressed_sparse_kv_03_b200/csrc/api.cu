@@ -48,31 +48,42 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int64_t score_stride(int64_t max_entries) { return (max_entries + 63) / 64 * 64; }
 
-// Indexer workspace: header | keys [chunk, stride] u32 | hist [chunk, 4096] u32
-// (bitmap mode only) | 256 B pad.  Queries are processed in chunks
-// so that the key scratch stays bounded.
+// Indexer workspace.  Few-query (fused) mode: header | per query tau and
+// candidate count [chunk][2] u32 | work counter | candidates [chunk, cap]
+// (key, entry) pairs -- O(top_k) per query, no score matrix.  Many-query
+// mode: header | work counter | keys [chunk, stride] u32.  Queries are
+// processed in chunks so that the scratch stays bounded.
 struct IndexerLayout {
-  bool bitmap;
-  int64_t chunk, stride;
-  size_t keys_off, hist_off, counter_off, total;
+  bool fused;
+  int64_t chunk, stride, cap;
+  size_t meta_off, counter_off, data_off, total;
 };
 
-IndexerLayout indexer_layout(int64_t T, int64_t max_entries) {
+// Candidate slots per query: the sample aims at about 2 top_k keys reaching
+// the threshold; twice that (and at least 8192) leaves room for its spread.
+int64_t candidate_cap(int32_t top_k) {
+  int64_t cap = 4 * (int64_t)(top_k > 0 ? top_k : 1);
+  if (cap < 8192) cap = 8192;
+  return (cap + 255) / 256 * 256;
+}
+
+IndexerLayout indexer_layout(int64_t T, int64_t max_entries, int32_t top_k) {
   IndexerLayout l;
+  l.fused = T <= kFusedMaxQueries || max_entries > kRadixSelectMaxEntries;
   l.stride = score_stride(max_entries);
-  l.bitmap = T <= kBitmapSelectMaxQueries || max_entries > kRadixSelectMaxEntries;
-  const int64_t per_query = l.stride * (int64_t)sizeof(uint32_t) +
-                            (l.bitmap ? kHistBins * (int64_t)sizeof(uint32_t) : 0);
+  l.cap = candidate_cap(top_k);
+  const int64_t per_query = l.fused ? l.cap * 8 + 8 : l.stride * (int64_t)sizeof(uint32_t);
   int64_t c = per_query > 0 ? (int64_t)(kIndexerChunkBytes / per_query) : T;
   if (c < 1) c = 1;
   if (c > 65535) c = 65535;
-  if (l.bitmap && c > kBitmapSelectMaxQueries) c = kBitmapSelectMaxQueries;
+  if (l.fused && c > kFusedMaxQueries) c = kFusedMaxQueries;
   l.chunk = c < T ? c : T;
   if (l.chunk < 1) l.chunk = 1;
-  l.keys_off = kWsHeader;
-  l.hist_off = l.keys_off + align256((size_t)l.chunk * l.stride * sizeof(uint32_t));
-  l.counter_off = l.hist_off + (l.bitmap ? align256((size_t)l.chunk * kHistBins * sizeof(uint32_t)) : 0);
-  l.total = l.counter_off + 256;
+  l.meta_off = kWsHeader;
+  l.counter_off = l.meta_off + (l.fused ? align256((size_t)l.chunk * 2 * sizeof(uint32_t)) : 0);
+  l.data_off = l.counter_off + 256;
+  l.total = l.data_off + (l.fused ? align256((size_t)l.chunk * l.cap * 8)
+                                  : align256((size_t)l.chunk * l.stride * sizeof(uint32_t)));
   return l;
 }
 
@@ -242,9 +253,8 @@ csa_status_t csa_set_timing_events(int32_t kernel_id, void* ev_begin, void* ev_e
 
 // ---- workspace -------------------------------------------------------------
 size_t csa_indexer_topk_workspace_size(int64_t T, int64_t max_entries, int32_t top_k) {
-  (void)top_k;
   if (T <= 0 || max_entries < 0) return kWsHeader;
-  return indexer_layout(T, max_entries).total;
+  return indexer_layout(T, max_entries, top_k).total;
 }
 
 size_t csa_sparse_attn_decode_workspace_size(int32_t B, int32_t H, int32_t d, int32_t top_k,
@@ -400,52 +410,65 @@ csa_status_t csa_norm_rope(const csa_bf16* x, csa_bf16* out, int64_t T, int32_t 
 // ---- steps 2-3 ---------------------------------------------------------------
 namespace {
 
-// Score + select, one chunk of queries at a time (the workspace holds the
-// keys of one chunk).  `base` carries the query / key operands.
+// Score + select, one chunk of queries at a time.  Fused mode: sample /
+// threshold, scoring into candidate lists, exact finish.  Many-query mode:
+// every key stored, radix select per query.  `base` carries the query / key
+// operands.
 csa_status_t run_indexer_topk(IndexerArgs base, const int64_t* q_pos, int64_t T, int32_t m,
                               int64_t max_entries, int32_t top_k, int32_t* idx_out,
                               int32_t* count_out, float* score_out, void* ws, csa_stream_t stream) {
   Launch L{(cudaStream_t)stream};
-  const IndexerLayout lay = indexer_layout(T, max_entries);
+  const IndexerLayout lay = indexer_layout(T, max_entries, top_k);
   char* wsb = static_cast<char*>(ws);
   WsHeader* hdr = static_cast<WsHeader*>(ws);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(wsb + lay.keys_off);
-  uint32_t* hist = lay.bitmap ? reinterpret_cast<uint32_t*>(wsb + lay.hist_off) : nullptr;
+  uint32_t* work = reinterpret_cast<uint32_t*>(wsb + lay.counter_off);
   for (int64_t t0 = 0; t0 < T; t0 += lay.chunk) {
     const int64_t n = T - t0 < lay.chunk ? T - t0 : lay.chunk;
-    // zero the histogram of this chunk (decode mode) and the scorer's work
-    // counter (they are adjacent: one memset)
-    const size_t zero_off = lay.bitmap ? lay.hist_off : lay.counter_off;
-    cudaError_t e = cudaMemsetAsync(wsb + zero_off, 0, lay.counter_off + sizeof(uint32_t) - zero_off, L.stream);
-    if (e != cudaSuccess) return cuda_status(e, "indexer workspace memset");
     IndexerArgs ia = base;
     ia.q_pos = q_pos;
     ia.T = T;
     ia.m = m;
     ia.max_entries = max_entries;
     ia.t_begin = t0;
-    ia.keys_out = keys;
-    ia.key_stride = lay.stride;
-    ia.hist = hist;
-    ia.work = reinterpret_cast<uint32_t*>(wsb + lay.counter_off);
+    ia.work = work;
     ia.err = hdr;
-    e = launch_indexer_scores(L, ia, n);
-    if (e != cudaSuccess) return cuda_status(e, "indexer score launch");
-    SelectArgs sa;
-    sa.keys = keys;
-    sa.key_stride = lay.stride;
-    sa.hist = hist;
-    sa.q_pos = q_pos;
-    sa.m = m;
-    sa.max_entries = max_entries;
-    sa.t_begin = t0;
-    sa.top_k = top_k;
-    sa.idx_out = idx_out;
-    sa.count_out = count_out;
-    sa.score_out = score_out;
-    sa.err = hdr;
-    e = launch_topk_select(L, sa, n);
-    if (e != cudaSuccess) return cuda_status(e, "top-k select launch");
+    cudaError_t e;
+    if (lay.fused) {
+      uint32_t* meta = reinterpret_cast<uint32_t*>(wsb + lay.meta_off);
+      ia.tau = meta;
+      ia.cand_count = meta + lay.chunk;
+      ia.cand = reinterpret_cast<uint2*>(wsb + lay.data_off);
+      ia.cand_cap = lay.cap;
+      ia.skip_le = score_out ? 0 : top_k;   // scores of all-selected queries still come from the scorer
+      ia.keys_out = nullptr;
+      // the work counter is zeroed before the sample launch (the scorer may
+      // start while that one runs); the sample launch zeroes the counts
+      e = cudaMemsetAsync(work, 0, sizeof(uint32_t), L.stream);
+      if (e != cudaSuccess) return cuda_status(e, "indexer work counter memset");
+      if ((e = launch_topk_sample(L, ia, top_k, n)) != cudaSuccess) return cuda_status(e, "top-k sample launch");
+      if ((e = launch_indexer_scores(L, ia, n)) != cudaSuccess) return cuda_status(e, "indexer score launch");
+      if ((e = launch_topk_finish(L, ia, top_k, idx_out, count_out, score_out, n)) != cudaSuccess)
+        return cuda_status(e, "top-k finish launch");
+    } else {
+      e = cudaMemsetAsync(work, 0, sizeof(uint32_t), L.stream);
+      if (e != cudaSuccess) return cuda_status(e, "indexer work counter memset");
+      ia.keys_out = reinterpret_cast<uint32_t*>(wsb + lay.data_off);
+      ia.key_stride = lay.stride;
+      if ((e = launch_indexer_scores(L, ia, n)) != cudaSuccess) return cuda_status(e, "indexer score launch");
+      SelectArgs sa;
+      sa.keys = ia.keys_out;
+      sa.key_stride = lay.stride;
+      sa.q_pos = q_pos;
+      sa.m = m;
+      sa.max_entries = max_entries;
+      sa.t_begin = t0;
+      sa.top_k = top_k;
+      sa.idx_out = idx_out;
+      sa.count_out = count_out;
+      sa.score_out = score_out;
+      sa.err = hdr;
+      if ((e = launch_topk_select(L, sa, n)) != cudaSuccess) return cuda_status(e, "top-k select launch");
+    }
   }
   return CSA_OK;
 }
@@ -464,9 +487,10 @@ csa_status_t check_indexer_args(const char* name, int64_t T, int32_t H_I, int32_
   if (H_I > 64) return fail(CSA_ERR_UNSUPPORTED, "%s: H_I > 64 not built", name);
   if (c_I != 64 && c_I != 128)
     return fail(CSA_ERR_UNSUPPORTED, "%s: c_I must be 64 or 128 (got %d)", name, c_I);
-  if (max_entries > kBitmapSelectMaxEntries)
+  if (max_entries > kMaxSelectEntries)
     return fail(CSA_ERR_UNSUPPORTED, "%s: max_entries > %lld not built", name,
-                (long long)kBitmapSelectMaxEntries);
+                (long long)kMaxSelectEntries);
+  if (top_k > 4096) return fail(CSA_ERR_UNSUPPORTED, "%s: top_k > 4096 not built", name);
   return check_cache(k_idx, name);
 }
 

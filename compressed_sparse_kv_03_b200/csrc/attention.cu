@@ -313,6 +313,8 @@ constexpr int kMergeHeads = 4;   // warps per block
 constexpr int kMergeChunk = 16;
 
 __global__ void __launch_bounds__(32 * kMergeHeads) merge_kernel(AttnArgs a) {
+  pdl_wait();   // the partials of the attention launch are complete
+  pdl_trigger();
   const int64_t i = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y * kMergeHeads + warp;
@@ -371,7 +373,9 @@ __global__ void __launch_bounds__(32 * kMergeHeads) merge_kernel(AttnArgs a) {
 cudaError_t launch_merge(const Launch& L, const AttnArgs& a) {
   L.begin(kKernelMerge);
   const dim3 grid((unsigned)a.T, (unsigned)((a.H + kMergeHeads - 1) / kMergeHeads));
-  merge_kernel<<<grid, 32 * kMergeHeads, 0, L.stream>>>(a);
+  prefer_max_shared(merge_kernel);
+  const cudaError_t e = launch_kernel(merge_kernel, grid, dim3(32 * kMergeHeads), 0, L.stream, true, a);
+  if (e != cudaSuccess) return e;
   return L.end(kKernelMerge);
 }
 

@@ -26,6 +26,9 @@
 //              per-thread partial row sums, bf16 P^T to shared memory; at the
 //              end of an item the epilogue (thread = dim of O^T) writes the
 //              normalised output or the split partials.
+// The kernel may start while the previous kernel on the stream finishes
+// (programmatic dependent launch): it sets up its barriers and TMEM and then
+// waits for that kernel before it reads anything.
 // Every wait is bounded (the workspace header records a timeout).
 #include "kernels.h"
 #include "tc.cuh"
@@ -194,6 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
                const __grid_constant__ CUtensorMap tm_win,
                const __grid_constant__ CUtensorMap tm_q, TcAttnParams p) {
+  pdl_trigger();
   const AttnArgs& a = p.a;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages];
@@ -236,6 +240,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  // everything above overlaps the previous kernel's tail; nothing below may
+  // read its outputs (selected entries, counts) before it has completed
+  pdl_wait();
   const uint32_t tmem_base = tmem_base_sh;
   const uint32_t tm_s = tmem_base;              // two 64-column S^T buffers
   const uint32_t tm_o = tmem_base + 2 * kNP;    // O^T
@@ -736,8 +743,9 @@ cudaError_t launch_attention_tc(const Launch& L, const AttnArgs& a) {
   if (grid < 1) return cudaSuccess;
   const int smem = 2 * kQTile + kStages * kKvTile + 2 * kPTile + 1024;
   cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  attn_tc_kernel<<<(unsigned)grid, kThreads, smem, L.stream>>>(t, w, q, p);
-  return cudaSuccess;
+  prefer_max_shared(attn_tc_kernel);
+  return launch_kernel(attn_tc_kernel, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, L.stream,
+                       true, t, w, q, p);
 }
 
 }  // namespace csa

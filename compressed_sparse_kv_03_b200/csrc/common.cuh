@@ -218,6 +218,16 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before its predecessor ends; pdl_wait() blocks until
+// the predecessor has completed and its writes are visible (a no-op in a
+// kernel launched normally), pdl_trigger() lets this kernel's own successor
+// start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
 }

@@ -52,6 +52,7 @@ cudaError_t launch_compress(const Launch& L, const __nv_bfloat16* Ca, const __nv
   const int64_t threads = S * (dim / 8);
   const unsigned blocks = (unsigned)((threads + kThreads - 1) / kThreads);
   L.begin(kKernelCompress);
+  prefer_max_shared(compress_kernel);
   compress_kernel<<<blocks, kThreads, 0, L.stream>>>(Ca, Za, Cb ? Cb : Ca, Zb ? Zb : Za, bias, S,
                                                      dim, m, overlap, out);
   return L.end(kKernelCompress);

@@ -27,9 +27,10 @@
 // 1152), and the block results are scaled by 2^(b_q - 127) * 2^(b_k - 127)
 // in fp32 before they are added.  The scorer is HBM-bound on the codes: 34
 // bytes per 64-dim key instead of 128.  Keys leave as the same
-// order-preserving 32-bit keys (plus, in decode mode, the same 4096-bin
-// histogram) as the bf16 scorer, so the top-k selection is shared.
+// order-preserving 32-bit keys as the bf16 scorer (appended to the candidate
+// lists in fused mode), so the top-k selection is shared.
 #include "kernels.h"
+#include "lowprec.cuh"
 
 namespace csa {
 
@@ -40,56 +41,7 @@ namespace {
 // ---------------------------------------------------------------------------
 constexpr int kQuantThreads = 256;
 
-__device__ __forceinline__ uint32_t e2m1_code(float y) {
-  const float a = fabsf(y);
-  // nearest magnitude, ties to the even code (0, 1, 1.5 -> 2, 2 -> 4, 4 -> 6)
-  uint32_t c = a <= 0.25f ? 0u
-             : a < 0.75f  ? 1u
-             : a <= 1.25f ? 2u
-             : a < 1.75f  ? 3u
-             : a <= 2.5f  ? 4u
-             : a < 3.5f   ? 5u
-             : a <= 5.0f  ? 6u
-                          : 7u;
-  return c | ((__float_as_uint(y) >> 31) << 3);
-}
-
-// One 32-element block: its four code words (nibble j of word i = element
-// 8i + j) and its scale byte.  The standalone quantizer and the scorer's
-// query prologue both use this, so their codes are identical.
-__device__ __forceinline__ uint32_t quantize_block(const __nv_bfloat16* __restrict__ src,
-                                                   uint32_t (&out)[4]) {
-  const uint4* p = reinterpret_cast<const uint4*>(src);
-  float v[32];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 u = __ldg(p + i);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = unpack_bf16(w[j]);
-      v[8 * i + 2 * j] = f.x;
-      v[8 * i + 2 * j + 1] = f.y;
-    }
-  }
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  // floor(log2 amax) from the exponent field; subnormal or zero amax clamps
-  // to the smallest scale
-  const int ef = (int)((__float_as_uint(amax) >> 23) & 0xffu);
-  int X = ef == 0 ? -127 : ef - 127 - 2;
-  X = X < -127 ? -127 : (X > 127 ? 127 : X);
-  const float inv = __uint_as_float((uint32_t)(127 - X) << 23);   // 2^-X, exact
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) word |= e2m1_code(v[8 * i + j] * inv) << (4 * j);
-    out[i] = word;
-  }
-  return (uint32_t)(X + 127);
-}
+using lowprec::quantize_block;
 
 __global__ void __launch_bounds__(kQuantThreads) mxfp4_quantize_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t n_blocks, uint8_t* __restrict__ codes,
@@ -196,11 +148,14 @@ __device__ __forceinline__ void load_batch(KeyBatch<CI, kU>& kb, const IndexerAr
 // [32v + 8q, 32v + 8q + 8)); the query fragments use the same permutation,
 // which leaves every dot product unchanged, and every k-column of the two
 // mma of block v falls inside block v.
-template <int CI, int NT, bool HIST, int kU>
+template <int CI, int NT, bool FUSED, int kU>
 __device__ __forceinline__ void score_batch(const KeyBatch<CI, kU>& kb,
-                                            const Fp4Query<CI, NT>& sq, uint32_t* sh_hist,
-                                            uint32_t* out, int64_t s0, int64_t s_end, int lane,
-                                            int g, int q4) {
+                                            const Fp4Query<CI, NT>& sq, const IndexerArgs& a,
+                                            int64_t tl, uint32_t tau, uint32_t* out,
+                                            CandidateBatch<kU>& pend, int64_t s0, int64_t s_end,
+                                            int lane, int g, int q4) {
+  bool pass[kU];
+  uint32_t keys[kU], ents[kU];
   constexpr int KB = CI / 32;
 #pragma unroll
   for (int u = 0; u < kU; ++u) {
@@ -243,11 +198,16 @@ __device__ __forceinline__ void score_batch(const KeyBatch<CI, kU>& kb,
     s8 += __shfl_xor_sync(0xffffffffu, s8, 2);
     const int64_t s = s0 + u * 16 + g + (q4 == 1 ? 8 : 0);
     const bool valid = q4 < 2 && s < s_end;
-    const uint32_t key = score_key(q4 == 0 ? sg : s8);
-    if (valid) {
-      out[s] = key;
-      if (HIST) atomicAdd(&sh_hist[key >> 20], 1u);
-    }
+    keys[u] = score_key(q4 == 0 ? sg : s8);
+    ents[u] = (uint32_t)s;
+    pass[u] = valid && keys[u] >= tau;
+    if (!FUSED && valid) out[s] = keys[u];
+  }
+  if (FUSED) {
+    CandidateBatch<kU> cur;
+    cur.issue(a, tl, pass, keys, ents);
+    pend.flush(a);
+    pend = cur;
   }
 }
 
@@ -256,12 +216,11 @@ __device__ __forceinline__ void score_batch(const KeyBatch<CI, kU>& kb,
 // lays out its fragments; each warp then walks batches of kU 16-key groups,
 // loading the next batch's code words into the other register set before it
 // scores the current one.
-template <int CI, int NT, bool HIST>
+template <int CI, int NT, bool FUSED>
 __global__ void __launch_bounds__(kFp4Threads, (CI == 64 && NT == 1) ? 3 : 1)
 indexer_score_fp4_kernel(IndexerArgs a, int64_t chunk) {
   constexpr int KB = CI / 32;                  // scale blocks per vector
   constexpr int kU = fp4_unroll(CI, NT);       // 16-key groups per batch
-  __shared__ uint32_t sh_hist[HIST ? kHistBins : 1];
   __shared__ Fp4Query<CI, NT> sq;
   __shared__ uint32_t qwords[NT * 8][CI / 8];  // the query's codes, head-major
   __shared__ uint32_t qscale[NT * 8][KB];
@@ -273,15 +232,13 @@ indexer_score_fp4_kernel(IndexerArgs a, int64_t chunk) {
     if (blockIdx.y == 0 && threadIdx.x == 0) report(a.err, kErrEligible, (int32_t)t, n_elig);
     n_elig = a.max_entries;
   }
+  if (FUSED && n_elig <= a.skip_le) return;
   const int64_t s_begin = (int64_t)blockIdx.y * chunk;
   if (s_begin >= n_elig) return;
   const int64_t s_end = min(s_begin + chunk, n_elig);
   const int32_t seq = a.seq_id ? __ldg(a.seq_id + t) : 0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, q4 = lane & 3;
-
-  if (HIST)
-    for (int b = threadIdx.x; b < kHistBins; b += kFp4Threads) sh_hist[b] = 0;
   for (int i = threadIdx.x; i < a.H_I * KB; i += kFp4Threads) {
     const int h = i / KB, v = i - h * KB;
     uint32_t w4[4];
@@ -304,7 +261,9 @@ indexer_score_fp4_kernel(IndexerArgs a, int64_t chunk) {
   __syncthreads();
 
   const uint8_t* codes = reinterpret_cast<const uint8_t*>(a.keys.data);
-  uint32_t* out = a.keys_out + tl * a.key_stride;
+  uint32_t* out = FUSED ? nullptr : a.keys_out + tl * a.key_stride;
+  const uint32_t tau = FUSED ? __ldg(a.tau + tl) : 0u;
+  CandidateBatch<kU> pend;   // the previous batch's candidates (fused mode)
   const int64_t stride = (int64_t)kFp4Warps * 16 * kU;
   // a contiguous cache whose chunk lies inside the buffer skips the per-row
   // checks (the same conditions cache_row tests, once for the whole chunk)
@@ -320,29 +279,22 @@ indexer_score_fp4_kernel(IndexerArgs a, int64_t chunk) {
   while (s0 < s_end) {
     int64_t s1 = s0 + stride;
     if (s1 < s_end) load_batch(b1, a, codes, seq, base, s1, s_end, t, g, q4);
-    score_batch<CI, NT, HIST>(b0, sq, sh_hist, out, s0, s_end, lane, g, q4);
+    score_batch<CI, NT, FUSED>(b0, sq, a, tl, tau, out, pend, s0, s_end, lane, g, q4);
     if (s1 >= s_end) break;
     s0 = s1 + stride;
     if (s0 < s_end) load_batch(b0, a, codes, seq, base, s0, s_end, t, g, q4);
-    score_batch<CI, NT, HIST>(b1, sq, sh_hist, out, s1, s_end, lane, g, q4);
+    score_batch<CI, NT, FUSED>(b1, sq, a, tl, tau, out, pend, s1, s_end, lane, g, q4);
   }
-  if (HIST) {
-    __syncthreads();
-    uint32_t* gh = a.hist + tl * kHistBins;
-    for (int b = threadIdx.x; b < kHistBins; b += kFp4Threads) {
-      const uint32_t v = sh_hist[b];
-      if (v) atomicAdd(gh + b, v);
-    }
-  }
+  if (FUSED) pend.flush(a);
 }
 
-template <int CI, int NT, bool HIST>
+template <int CI, int NT, bool FUSED>
 void launch_score_fp4(const Launch& L, const IndexerArgs& a, int64_t t_count) {
   constexpr int kU = fp4_unroll(CI, NT);
   int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, indexer_score_fp4_kernel<CI, NT, HIST>,
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, indexer_score_fp4_kernel<CI, NT, FUSED>,
                                                 kFp4Threads, 0);
   if (per_sm < 1) per_sm = 1;
   // chunks per query so that the grid fills whole resident waves
@@ -355,7 +307,8 @@ void launch_score_fp4(const Launch& L, const IndexerArgs& a, int64_t t_count) {
   if (chunk < min_chunk) chunk = min_chunk;
   per_q = (a.max_entries + chunk - 1) / chunk;
   const dim3 grid((unsigned)t_count, (unsigned)per_q);
-  indexer_score_fp4_kernel<CI, NT, HIST><<<grid, kFp4Threads, 0, L.stream>>>(a, chunk);
+  prefer_max_shared(indexer_score_fp4_kernel<CI, NT, FUSED>);
+  indexer_score_fp4_kernel<CI, NT, FUSED><<<grid, kFp4Threads, 0, L.stream>>>(a, chunk);
 }
 
 }  // namespace
@@ -373,11 +326,11 @@ cudaError_t launch_indexer_scores_fp4(const Launch& L, const IndexerArgs& a, int
   if (t_count == 0 || a.max_entries == 0) return cudaSuccess;
   const int nt = (a.H_I + 7) / 8;
   const int ntb = nt <= 1 ? 1 : nt <= 2 ? 2 : nt <= 4 ? 4 : 8;
-  const bool hist = a.hist != nullptr;
+  const bool fused = a.tau != nullptr;
   L.begin(kKernelIndexerScore);
 #define CSA_FP4_CASE(CI_, NT_)                                             \
   if (a.c_I == CI_ && ntb == NT_) {                                        \
-    if (hist) launch_score_fp4<CI_, NT_, true>(L, a, t_count);             \
+    if (fused) launch_score_fp4<CI_, NT_, true>(L, a, t_count);            \
     else launch_score_fp4<CI_, NT_, false>(L, a, t_count);                 \
   }
   CSA_FP4_CASE(64, 1)

@@ -14,9 +14,10 @@
 //              as K in four steps, into one of four 32-column TMEM sets;
 //   warps 2-9  epilogue, two groups of four warps taking alternate items:
 //              tcgen05.ld of their 32 TMEM lanes (one key per tile), ReLU,
-//              the head-weighted sum, the order-preserving score key,
-//              coalesced stores and (decode mode) the query's 12-bit histogram
-//              through warp-aggregated atomics.
+//              the head-weighted sum, the order-preserving score key, and the
+//              fused selection's filter: keys that reach the query's threshold
+//              are appended to its candidate list (one atomic per warp); no
+//              other score leaves the SM.
 // The valid (query, 256-key chunk) pairs are numbered through a prefix sum
 // over the queries' chunk counts; the producers of all CTAs take them two at a
 // time from one launch-wide counter, so SMs that stream faster take more (on
@@ -69,10 +70,10 @@ __device__ __forceinline__ int64_t eligible(const IndexerArgs& a, int64_t t) {
   return n < a.max_entries ? n : a.max_entries;
 }
 
-template <bool HIST>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
                         const __grid_constant__ CUtensorMap tmap_q, TcIndexerParams p) {
+  pdl_trigger();
   const IndexerArgs& a = p.a;
   const int T = (int)p.t_count;
   extern __shared__ uint8_t smem_raw[];
@@ -116,7 +117,8 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
         report(a.err, kErrEligible, (int32_t)(a.t_begin + t), pos / a.m);
       const int64_t n = eligible(a, a.t_begin + t);
       nelig[t] = (int32_t)n;
-      prefix[t] = (int32_t)((n + kItemRows - 1) / kItemRows);
+      // queries that take all of their entries are not scored
+      prefix[t] = n <= a.skip_le ? 0 : (int32_t)((n + kItemRows - 1) / kItemRows);
       sum += prefix[t];
     }
     int32_t incl = sum;
@@ -304,14 +306,18 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // the thresholds and zeroed counts come from the sample pass, which may
+    // still be running when this kernel starts (the producer and the MMA warp
+    // do not need them)
+    pdl_wait();
     const int ew = warp - 2;
     const int group = ew >> 2;                 // handles items j with j % 2 == group
     const int quarter = warp & 3;              // TMEM lanes this warp may read
     const int row = quarter * 32 + lane;       // key within a 128-key tile
     int t_cached = -1;
     int64_t n_elig = 0;
-    uint32_t* out = nullptr;
-    uint32_t* gh = nullptr;
+    uint32_t tau = 0;
+    CandidateBatch<2> pend;   // the previous item's candidates, stored after this item's atomic
     for (int64_t j = group;; j += 2) {
       const int rs = (int)(j % kRing);
       if (!mbar_wait(smem_u32(&ring_full[rs]), (uint32_t)((j / kRing) & 1))) {
@@ -336,8 +342,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
       if (tq != t_cached) {
         t_cached = tq;
         n_elig = nelig[tq];
-        out = a.keys_out + (int64_t)tq * a.key_stride;
-        gh = HIST ? a.hist + (int64_t)tq * kHistBins : nullptr;
+        tau = __ldg(a.tau + tq);
       }
       if (!mbar_wait(smem_u32(&tfull_bar[acc]), (uint32_t)((j / kAcc) & 1))) {
         if (lane == 0) report(a.err, kErrTimeout, (int32_t)j, 13);
@@ -353,6 +358,8 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[acc]));
       const int64_t s0 = (int64_t)chunk * kItemRows;
+      bool pass[2];
+      uint32_t keys[2], ents[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const uint32_t* r = h ? r1 : r0;
@@ -360,16 +367,16 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
 #pragma unroll
         for (int k = 0; k < 16; ++k) sc = fmaf(wv[k], fmaxf(__uint_as_float(r[k]), 0.f), sc);
         const int64_t s = s0 + h * kTileRows + row;
-        const bool valid = s < n_elig;
-        const uint32_t key = score_key(sc);
-        if (valid) out[s] = key;
-        if (HIST) {
-          const uint32_t bin = valid ? key >> 20 : 0xffffffffu;
-          const uint32_t same = __match_any_sync(0xffffffffu, bin);
-          if (valid && lane == __ffs(same) - 1) atomicAdd(gh + bin, (uint32_t)__popc(same));
-        }
+        keys[h] = score_key(sc);
+        ents[h] = (uint32_t)s;
+        pass[h] = s < n_elig && keys[h] >= tau;
       }
+      CandidateBatch<2> cur;
+      cur.issue(a, tq, pass, keys, ents);
+      pend.flush(a);
+      pend = cur;
     }
+    pend.flush(a);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -404,7 +411,7 @@ struct __align__(16) BlockMeta {
   int32_t b, chunk, pad0, pad1;
 };
 
-template <bool HIST, int HI>
+template <int HI>
 __global__ void __launch_bounds__(kPThreads, 1)
 indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
                                 const __grid_constant__ CUtensorMap tmap_q, TcIndexerParams p) {
@@ -697,12 +704,6 @@ indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
             const uint32_t key = score_key(sc);
             const int64_t tl = t0 + q;
             if (valid) a.keys_out[tl * a.key_stride + s] = key;
-            if (HIST) {
-              const uint32_t bin = valid ? key >> 20 : 0xffffffffu;
-              const uint32_t same = __match_any_sync(0xffffffffu, bin);
-              if (valid && lane == __ffs(same) - 1)
-                atomicAdd(a.hist + tl * kHistBins + bin, (uint32_t)__popc(same));
-            }
           }
         }
       }
@@ -723,6 +724,7 @@ indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
 }  // namespace
 
 bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count) {
+  if (a.tau == nullptr) return false;   // fused selection only
   if (a.c_I != 64 || a.H_I > 16 || t_count > kMaxQueries) return false;
   if ((a.max_entries + kItemRows - 1) / kItemRows * t_count > INT32_MAX) return false;
   if (a.keys.page_table != nullptr && a.keys.page_size % kBoxRows != 0) return false;
@@ -732,6 +734,7 @@ bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count) {
 }
 
 bool tc_indexer_prefill_supported(const IndexerArgs& a, int64_t t_count) {
+  if (a.tau != nullptr) return false;   // stores every key (many-query mode)
   if (a.seq_id != nullptr || a.c_I != 64 || a.work == nullptr) return false;
   if (a.H_I != 4 && a.H_I != 8 && a.H_I != 16) return false;
   // the producer reads a block's 128 head weights as 32 aligned float4
@@ -759,18 +762,16 @@ cudaError_t launch_indexer_scores_tc_prefill(const Launch& L, const IndexerArgs&
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int smem = kPStages * kPStageBytes + 1024;
   L.begin(kKernelIndexerScore);
-#define CSA_PREFILL_CASE(H_, HIST_)                                                               \
-  if (a.H_I == H_ && (a.hist != nullptr) == HIST_) {                                               \
-    cudaFuncSetAttribute(indexer_score_tc_prefill_kernel<HIST_, H_>,                               \
+#define CSA_PREFILL_CASE(H_)                                                                      \
+  if (a.H_I == H_) {                                                                               \
+    cudaFuncSetAttribute(indexer_score_tc_prefill_kernel<H_>,                                      \
                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                       \
-    indexer_score_tc_prefill_kernel<HIST_, H_><<<(unsigned)sms, kPThreads, smem, L.stream>>>(tk, tq, p); \
+    prefer_max_shared(indexer_score_tc_prefill_kernel<H_>);                                        \
+    indexer_score_tc_prefill_kernel<H_><<<(unsigned)sms, kPThreads, smem, L.stream>>>(tk, tq, p);  \
   }
-  CSA_PREFILL_CASE(4, false)
-  CSA_PREFILL_CASE(8, false)
-  CSA_PREFILL_CASE(16, false)
-  CSA_PREFILL_CASE(4, true)
-  CSA_PREFILL_CASE(8, true)
-  CSA_PREFILL_CASE(16, true)
+  CSA_PREFILL_CASE(4)
+  CSA_PREFILL_CASE(8)
+  CSA_PREFILL_CASE(16)
 #undef CSA_PREFILL_CASE
   return L.end(kKernelIndexerScore);
 }
@@ -791,13 +792,11 @@ cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int6
   const int64_t grid = sms;
   const int smem = kStages * (kStageKeyBytes + kQTileBytes) + 1024;
   L.begin(kKernelIndexerScore);
-  if (a.hist != nullptr) {
-    cudaFuncSetAttribute(indexer_score_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    indexer_score_tc_kernel<true><<<(unsigned)grid, kThreads, smem, L.stream>>>(tk, tq, p);
-  } else {
-    cudaFuncSetAttribute(indexer_score_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    indexer_score_tc_kernel<false><<<(unsigned)grid, kThreads, smem, L.stream>>>(tk, tq, p);
-  }
+  cudaFuncSetAttribute(indexer_score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  prefer_max_shared(indexer_score_tc_kernel);
+  cudaError_t e = launch_kernel(indexer_score_tc_kernel, dim3((unsigned)grid), dim3(kThreads),
+                                (size_t)smem, L.stream, true, tk, tq, p);
+  if (e != cudaSuccess) return e;
   return L.end(kKernelIndexerScore);
 }
 

@@ -1,6 +1,8 @@
 // Internal launch interface between the C-ABI layer (api.cu) and the kernels.
 #pragma once
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace csa {
@@ -12,7 +14,8 @@ enum KernelId : int32_t {
   kKernelMerge = 3,
   kKernelCompress = 4,
   kKernelQuantize = 5,
-  kNumKernelIds = 6,
+  kKernelTopkSample = 6,   // the fused selection's sampling / threshold pass
+  kNumKernelIds = 7,
 };
 
 // Per-call launch context: the stream plus the timing / launch-count hooks.
@@ -60,18 +63,21 @@ struct NormRopeArgs {
 };
 cudaError_t launch_norm_rope(const Launch& L, const NormRopeArgs& a);
 
-// Indexer scratch limits.  Few-query (decode) mode keeps a 4096-bin histogram
-// of the top 12 score-key bits per query and selects through a bitmap in
-// shared memory; many-query (prefill) mode holds a query's keys in shared
-// memory for a radix select.
-constexpr int kHistBins = 4096;
-constexpr int64_t kBitmapSelectMaxEntries = int64_t(1) << 19;
-constexpr int64_t kBitmapSelectMaxQueries = 2048;
+// Indexer selection modes.  Few-query (decode) mode, at most
+// kFusedMaxQueries queries per launch: the scorer keeps only the (key, entry)
+// pairs that reach a per-query threshold drawn from a sample of the query's
+// scores, and a finishing pass selects exactly among them (no score matrix is
+// stored).  Many-query (prefill) mode holds a query's keys in shared memory
+// for a radix select.
+constexpr int64_t kMaxSelectEntries = int64_t(1) << 19;
+constexpr int64_t kFusedMaxQueries = 2048;
 constexpr int64_t kRadixSelectMaxEntries = 48 * 1024;
 
 // Lightning-indexer scores of every eligible entry for every query of one
-// chunk of queries, written as order-preserving keys to
-// keys_out[(t - t_begin) * key_stride + s].
+// chunk of queries: in many-query mode written as order-preserving keys to
+// keys_out[(t - t_begin) * key_stride + s]; in fused mode (tau != null) only
+// the entries whose key reaches tau[t - t_begin] are appended to the query's
+// candidate list.
 struct IndexerArgs {
   const __nv_bfloat16* q_idx;   // [T, H_I, c_I]
   const float* w;               // [T, H_I]
@@ -82,10 +88,16 @@ struct IndexerArgs {
   int H_I, c_I, m;
   int64_t max_entries;
   int64_t t_begin;              // first query of this launch (chunking)
-  uint32_t* keys_out;           // [T_chunk, key_stride]
+  uint32_t* keys_out;           // [T_chunk, key_stride] (many-query mode)
   int64_t key_stride;
-  uint32_t* hist;               // [T_chunk, kHistBins] (zeroed) or null
   uint32_t* work;               // zeroed work counter of the tcgen05 scorer
+  // fused selection (few-query mode)
+  const uint32_t* tau = nullptr;     // [T_chunk] candidate threshold (a score key)
+  uint32_t* cand_count = nullptr;    // [T_chunk] zeroed; counts every pair that passes
+  uint2* cand = nullptr;             // [T_chunk, cand_cap] (key, entry), first cand_cap kept
+  int64_t cand_cap = 0;
+  int64_t skip_le = 0;               // queries with at most this many eligible entries are
+                                     // not scored (they select all of them)
   WsHeader* err;
   // 4-bit mode (fp4 = 1): q_idx is quantized to E2M1 codes + scale bytes in
   // the scorer; keys.data holds rows of c_I/2 code bytes and k_scales rows of
@@ -94,7 +106,50 @@ struct IndexerArgs {
   const uint8_t* k_scales = nullptr;
 };
 cudaError_t launch_indexer_scores(const Launch& L, const IndexerArgs& a, int64_t t_count);
-// tcgen05 + TMA scoring path (c_I = 64, H_I <= 16, pages a multiple of 64 rows)
+// Fused-selection epilogue of the scorers, one warp at a time: a batch of U
+// keys per lane (entry ids alongside) whose `pass` flags mark the candidates.
+// issue() takes the warp's ballots and reserves slots with one atomic on the
+// query's count; flush() stores the batch into the reserved slots.  A scorer
+// issues batch j and flushes batch j-1 after it, so the atomic's round trip
+// overlaps the next batch instead of stalling the warp.  Slots past cand_cap
+// are counted but not stored.  Every lane of the warp must make each call.
+template <int U>
+struct CandidateBatch {
+  uint32_t key[U], ent[U], m[U];
+  uint32_t base = 0, tot = 0;
+  int64_t tl = 0;
+  __device__ __forceinline__ void issue(const IndexerArgs& a, int64_t tl_, const bool (&pass)[U],
+                                        const uint32_t (&k)[U], const uint32_t (&e)[U]) {
+    uint32_t t = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      m[u] = __ballot_sync(0xffffffffu, pass[u]);
+      key[u] = k[u];
+      ent[u] = e[u];
+      t += (uint32_t)__popc(m[u]);
+    }
+    tot = t;
+    tl = tl_;
+    if (t != 0u && (threadIdx.x & 31) == 0) base = atomicAdd(a.cand_count + tl_, t);
+  }
+  __device__ __forceinline__ void flush(const IndexerArgs& a) {
+    if (tot == 0u) return;   // warp-uniform
+    const int lane = threadIdx.x & 31;
+    uint32_t off = __shfl_sync(0xffffffffu, base, 0);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if ((m[u] >> lane) & 1u) {
+        const uint32_t slot = off + (uint32_t)__popc(m[u] & ((1u << lane) - 1u));
+        if (slot < (uint64_t)a.cand_cap) a.cand[tl * a.cand_cap + slot] = make_uint2(key[u], ent[u]);
+      }
+      off += (uint32_t)__popc(m[u]);
+    }
+    tot = 0u;
+  }
+};
+
+// tcgen05 + TMA scoring path (c_I = 64, H_I <= 16, pages a multiple of 64 rows;
+// fused mode only)
 bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count);
 cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int64_t t_count);
 // tcgen05 many-query path: all queries on one sequence (seq_id null), c_I = 64,
@@ -107,10 +162,10 @@ cudaError_t launch_indexer_scores_fp4(const Launch& L, const IndexerArgs& a, int
 cudaError_t launch_mxfp4_quantize(const Launch& L, const __nv_bfloat16* x, int64_t n_blocks,
                                   uint8_t* codes, uint8_t* scales);
 
+// Many-query selection over stored keys (radix select per query).
 struct SelectArgs {
   const uint32_t* keys;         // [T_chunk, key_stride]
   int64_t key_stride;
-  const uint32_t* hist;         // decode mode: histogram from the scoring launch; else null
   const int64_t* q_pos;
   int m;
   int64_t max_entries;
@@ -122,7 +177,18 @@ struct SelectArgs {
   WsHeader* err;
 };
 cudaError_t launch_topk_select(const Launch& L, const SelectArgs& a, int64_t t_count);
-bool select_uses_bitmap(int64_t t_count, int64_t max_entries);
+
+// Fused selection (few-query mode), around the scoring launch of the same
+// IndexerArgs (tau / cand_count / cand / cand_cap / skip_le / work set):
+//   launch_topk_sample: per query, zeroes its candidate count (and the work
+//     counter), scores a strided sample of its eligible entries and writes a
+//     threshold tau that about 2 top_k of its entries are expected to reach;
+//   launch_topk_finish: per query, the exact top-k -- among the candidates when
+//     top_k <= count <= cand_cap, else by exact recompute passes over every
+//     eligible entry -- written ascending with its count (and scores).
+cudaError_t launch_topk_sample(const Launch& L, const IndexerArgs& a, int top_k, int64_t t_count);
+cudaError_t launch_topk_finish(const Launch& L, const IndexerArgs& a, int top_k, int32_t* idx_out,
+                               int32_t* count_out, float* score_out, int64_t t_count);
 
 // Attention over a virtual row list per query: its selected / eligible
 // compressed entries followed by its window rows.
@@ -203,6 +269,36 @@ cudaError_t launch_attention_tc(const Launch& L, const AttnArgs& a);
 cudaError_t launch_fp8_entry_quantize(const Launch& L, const __nv_bfloat16* x, int64_t n, int dim,
                                       int rope, uint8_t* codes, uint8_t* scales,
                                       __nv_bfloat16* rope_out);
+
+// Every kernel asks for the largest shared-memory carveout, so that the
+// kernels of a step, some of which need nearly all of it, never make the SMs
+// repartition L1 and shared memory between launches.
+template <class K>
+inline void prefer_max_shared(K kernel) {
+  cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                       (int)cudaSharedmemCarveoutMaxShared);
+}
+
+// Launch `kernel`, with programmatic stream serialization when `pdl` (the
+// kernel then must call pdl_wait() before it reads anything a predecessor
+// writes).
+template <class... P, class... A>
+inline cudaError_t launch_kernel(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t stream, bool pdl, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
 
 // Text returned by csa_last_error() for this thread.
 void set_last_error(const char* msg);

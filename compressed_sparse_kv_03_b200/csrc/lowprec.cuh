@@ -42,5 +42,71 @@ __device__ __forceinline__ uint32_t e4m3_code(float y) {
   return c | ((__float_as_uint(y) >> 31) << 7);
 }
 
+
+// Nearest E2M1 code of y (4-bit indexer format): magnitudes 0, 0.5, 1, 1.5,
+// 2, 3, 4, 6, ties to the even code, saturating at 6; the sign bit is y's.
+__device__ __forceinline__ uint32_t e2m1_code(float y) {
+  const float a = fabsf(y);
+  // nearest magnitude, ties to the even code (0, 1, 1.5 -> 2, 2 -> 4, 4 -> 6)
+  uint32_t c = a <= 0.25f ? 0u
+             : a < 0.75f  ? 1u
+             : a <= 1.25f ? 2u
+             : a < 1.75f  ? 3u
+             : a <= 2.5f  ? 4u
+             : a < 3.5f   ? 5u
+             : a <= 5.0f  ? 6u
+                          : 7u;
+  return c | ((__float_as_uint(y) >> 31) << 3);
+}
+
+// One 32-element block of the 4-bit indexer format (E2M1 codes, one
+// power-of-two scale byte): its four code words (nibble j of word i = element
+// 8i + j) and its scale byte.  The standalone quantizer, the scorer's query
+// prologue and the selection's own scoring all use this, so their codes are
+// identical.
+__device__ __forceinline__ uint32_t quantize_block(const __nv_bfloat16* __restrict__ src,
+                                                   uint32_t (&out)[4]) {
+  const uint4* p = reinterpret_cast<const uint4*>(src);
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = __ldg(p + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = unpack_bf16(w[j]);
+      v[8 * i + 2 * j] = f.x;
+      v[8 * i + 2 * j + 1] = f.y;
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  // floor(log2 amax) from the exponent field; subnormal or zero amax clamps
+  // to the smallest scale
+  const int ef = (int)((__float_as_uint(amax) >> 23) & 0xffu);
+  int X = ef == 0 ? -127 : ef - 127 - 2;
+  X = X < -127 ? -127 : (X > 127 ? 127 : X);
+  const float inv = __uint_as_float((uint32_t)(127 - X) << 23);   // 2^-X, exact
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) word |= e2m1_code(v[8 * i + j] * inv) << (4 * j);
+    out[i] = word;
+  }
+  return (uint32_t)(X + 127);
+}
+
+
+// Value of an E2M1 code (sign bit 3, exponent bits 2-1 with bias 1, mantissa
+// bit 0): exactly one of +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+__device__ __forceinline__ float e2m1_to_float(uint32_t c) {
+  const uint32_t E = (c >> 1) & 3u, M = c & 1u;
+  const float v = E ? __uint_as_float(((E + 126u) << 23) | (M << 22))   // (1 + M/2) 2^(E-1)
+                    : 0.5f * (float)M;
+  return (c & 8u) ? -v : v;
+}
+
 }  // namespace lowprec
 }  // namespace csa

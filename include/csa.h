@@ -232,6 +232,16 @@ csa_status_t csa_norm_rope(const csa_bf16* x, csa_bf16* out, int64_t T, int32_t 
  * selection and asymptotic scaling").  Scores are accumulated and compared in
  * fp32; equal scores go to the lower entry index; with fewer than top_k
  * eligible entries all are taken.  The score matrix is never returned.
+ * Up to 2048 queries per call (decode), no score matrix is formed at all: a
+ * small pass scores a strided sample of each query's entries and sets a
+ * threshold that about 2 top_k of them are expected to reach; the scorer keeps
+ * only the (score, entry) pairs at or above it, O(top_k) per query in the
+ * workspace; an exact select over those finishes the job whenever at least
+ * top_k and at most the workspace's slots reached the threshold, and exact
+ * recompute passes over the query's entries handle the other (rare) cases.
+ * Larger calls (prefill) keep every score of a chunk of queries in the
+ * workspace and select per query.  Results are the same either way.
+ * top_k <= 4096; max_entries <= 2^19; c_I in {64, 128}; H_I <= 64.
  *   q_idx      [T, H_I, c_I] bf16
  *   w          [T, H_I] fp32
  *   k_idx      cache of [*, c_I] bf16 indexer keys (host struct)

@@ -100,9 +100,16 @@ def test_workspace_sizes(lib):
     assert n > hdr and n % 256 == 0
     # prefill never splits
     assert lib.csa_sparse_attn_prefill_workspace_size(65536, 64, 128) == hdr
-    # indexer scratch: at least one fp32 score per eligible entry of a query
+    # decode-mode indexer scratch is O(queries x top_k): a threshold, a count and
+    # 4 top_k (at least 8192) candidate (key, entry) pairs per query -- no score
+    # matrix, and independent of the number of entries
     n = lib.csa_indexer_topk_workspace_size(64, 32768, 2048)
-    assert n >= hdr + 64 * 32768 * 4
+    assert hdr + 64 * 8192 * 8 <= n <= hdr + 64 * (8192 * 8 + 8) + 3 * 256
+    assert lib.csa_indexer_topk_workspace_size(64, 1 << 19, 2048) == n
+    assert lib.csa_indexer_topk_workspace_size(64, 32768, 4096) > n
+    # many-query (prefill) mode stores one key per eligible entry, in bounded chunks
+    n = lib.csa_indexer_topk_workspace_size(65536, 16384, 2048)
+    assert hdr + 8192 * 16384 * 4 <= n <= (520 << 20)
     # too small a workspace is refused before anything runs
     from compressed_sparse_kv_03_b200._lib import CacheT
     buf = (C.c_uint8 * 4096)()

@@ -213,3 +213,21 @@ def test_indexer_topk_mxfp4_decode_full_size_sampled():
     kc3, ks3 = kc.view(B, S, -1).numpy(), ks.view(B, S, -1).numpy()
     _check_fp4_queries(idx, cnt, None, lambda b: (qc[b], qs[b]), w,
                        lambda b: (kc3[b], ks3[b]), lambda b: S, k, [0, 17, 40, 63])
+
+
+def test_indexer_topk_mxfp4_all_equal_scores_beyond_the_candidate_slots():
+    """4-bit keys that all score exactly 0 (every code -1 against positive
+    queries) on 20000 entries: more keys reach the threshold than the
+    candidate slots hold, so the selection recomputes from the codes; the
+    first k entries win, bit-exactly."""
+    csa = _csa()
+    T, S, k, m = 2, 20000, 500, 4
+    qI = torch.ones((T, 8, 64), dtype=torch.bfloat16)
+    codes = torch.full((S, 32), 0xAA, dtype=torch.uint8)        # every nibble -1.0
+    scales = torch.full((S, 2), 127, dtype=torch.uint8)
+    w = torch.rand((T, 8), generator=synth.generator(990))
+    pos = torch.full((T,), 4 * S, dtype=torch.int64)
+    idx, cnt = csa.indexer_topk_mxfp4(dev(qI), dev(w), csa.Cache(dev(codes)), dev(scales), m, k,
+                                      q_pos=dev(pos), max_entries=S)
+    assert torch.equal(idx.cpu(), torch.arange(k, dtype=torch.int32).expand(T, k))
+    assert torch.all(cnt.cpu() == k)

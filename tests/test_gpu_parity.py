@@ -213,6 +213,68 @@ def test_indexer_topk_decode_ragged(H_I, c_I, wdist):
                    range(B), sc)
 
 
+@pytest.mark.parametrize("H_I,c_I,k", [(8, 64, 512), (64, 128, 256), (12, 64, 2048), (4, 64, 64)])
+def test_indexer_topk_decode_sampled_threshold(H_I, c_I, k):
+    """Contexts long enough (more than 4096 eligible entries) for the sampled
+    threshold: the selection comes from the candidate lists; scores too."""
+    csa = _csa()
+    g = synth.generator(35 + H_I + c_I + k)
+    m = 4
+    pos = torch.tensor([20000, 40001, 65537, 131072, 77777], dtype=torch.int64)
+    B, S = pos.shape[0], int(pos.max()) // m
+    qI = synth.normal(g, (B, H_I, c_I))
+    w = synth.uniform(g, (B, H_I))
+    KI = synth.normal(g, (B, S, c_I))
+    idx, cnt, sc = csa.indexer_topk(dev(qI), dev(w), csa.Cache.contiguous(dev(KI)), m, k,
+                                    seq_id=dev(torch.arange(B, dtype=torch.int32)), q_pos=dev(pos),
+                                    max_entries=S, return_scores=True)
+    _check_queries(idx, cnt, qI, w, lambda t: f64(KI[t]), lambda t: int(pos[t]) // m, k,
+                   range(B), sc)
+
+
+@pytest.mark.parametrize("return_scores", [False, True])
+def test_indexer_topk_all_equal_scores_beyond_the_candidate_slots(return_scores):
+    """20000 eligible entries whose scores are all exactly 0 (every head
+    negative): every key reaches any threshold, more than the candidate slots
+    hold, so the selection falls back to recomputing the keys.  The first k
+    entries must win (ties to the lower index), bit-exactly."""
+    csa = _csa()
+    T, S, k, m = 3, 20000, 300, 4
+    qI = torch.ones((T, 2, 64), dtype=torch.bfloat16)
+    KI = -torch.ones((S, 64), dtype=torch.bfloat16)
+    w = torch.rand((T, 2), generator=synth.generator(36))
+    pos = torch.tensor([4 * S, 4 * S - 1, 4 * 1000 + 3], dtype=torch.int64)
+    out = csa.indexer_topk(dev(qI), dev(w), csa.Cache(dev(KI)), m, k, q_pos=dev(pos),
+                           max_entries=S, return_scores=return_scores)
+    idx, cnt = out[0].cpu(), out[1].cpu()
+    assert torch.equal(idx, torch.arange(k, dtype=torch.int32).expand(T, k))
+    assert torch.all(cnt == k)
+    if return_scores:
+        assert torch.all(out[2].cpu() == 0)
+
+
+@pytest.mark.parametrize("H_I,c_I", [(8, 64), (16, 128)])
+def test_indexer_topk_sample_misled_by_structure(H_I, c_I):
+    """A cache whose every 32nd row (the sample's stride at this length)
+    scores far above the rest: the threshold drawn from the sample is then too
+    high (fewer than k keys reach it) and the selection recomputes.  Whatever
+    path it takes, the result must be the oracle's."""
+    csa = _csa()
+    g = synth.generator(37 + H_I)
+    B, m, k = 2, 4, 2048
+    S = 40960                               # a multiple of 32: the sample hits rows 0 mod 32
+    qI = synth.normal(g, (B, H_I, c_I))
+    w = synth.uniform(g, (B, H_I))
+    KI = synth.normal(g, (B, S, c_I), 0.05)
+    for b in range(B):                      # rows 0 mod 32 aligned with the query's heads
+        KI[b, ::32] = (qI[b].float().sum(0) / H_I).to(torch.bfloat16)
+    pos = torch.full((B,), S * m, dtype=torch.int64)
+    idx, cnt, sc = csa.indexer_topk(dev(qI), dev(w), csa.Cache.contiguous(dev(KI)), m, k,
+                                    seq_id=dev(torch.arange(B, dtype=torch.int32)), q_pos=dev(pos),
+                                    max_entries=S, return_scores=True)
+    _check_queries(idx, cnt, qI, w, lambda t: f64(KI[t]), lambda t: S, k, range(B), sc)
+
+
 @pytest.mark.parametrize("T,m,k,H_I", [(700, 4, 32, 4), (1500, 2, 100, 8), (300, 1, 300, 8)])
 def test_indexer_topk_prefill_causal(T, m, k, H_I):
     csa = _csa()

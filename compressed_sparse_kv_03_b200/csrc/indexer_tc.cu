@@ -43,7 +43,7 @@ constexpr int kEpiWarps = 8;                       // two groups of four
 constexpr int kThreads = (2 + kEpiWarps) * 32;
 constexpr int kAcc = 4;                            // TMEM accumulator sets (32 columns each)
 constexpr uint32_t kIdesc = tc::idesc_bf16(128, 16);
-constexpr int kTmemCols = 128;
+constexpr int kTmemCols = kAcc * 32;
 constexpr int kMaxQueries = 2048;
 constexpr int kRing = 16;                          // item metadata ring (> kStages + kAcc)
 constexpr int kGrab = 2;                           // items taken from the work counter at once

@@ -183,10 +183,12 @@ __device__ __noinline__ uint32_t recompute_key(const IndexerArgs& a, const float
 // its low 10 bits cleared (two radix levels of 11 bits: bits 31-21, 20-10),
 // r = the expected number of sampled keys at or above the k-th largest key
 // plus six standard deviations and a margin; 0 when r reaches ns.
+// With `built`, hist already holds the first level (bits 31-21 of every
+// sampled key, counted while scoring).
 template <int NT>
 __device__ uint32_t sample_threshold(const uint32_t* skey, int ns, int64_t n, int top_k,
                                      int* hist, int* warp_sums, uint32_t* s_bin, int* s_above,
-                                     int* s_ok) {
+                                     int* s_ok, bool built = false) {
   const double mu = (double)ns * (double)top_k / (double)n;
   const int64_t r = (int64_t)ceil(mu + 6.0 * sqrt(mu) + 8.0);
   if (r >= ns) return 0u;
@@ -195,13 +197,15 @@ __device__ uint32_t sample_threshold(const uint32_t* skey, int ns, int64_t n, in
 #pragma unroll 1
   for (int level = 0; level < 2; ++level) {
     const int lo = level == 0 ? 21 : 10;
-    for (int b = threadIdx.x; b < 2048; b += NT) hist[b] = 0;
-    __syncthreads();
-    for (int j = threadIdx.x; j < ns; j += NT) {
-      const uint32_t key = skey[j];
-      if (level == 0 || (key >> 21) == (prefix >> 21)) atomicAdd(&hist[(key >> lo) & 2047u], 1);
+    if (level > 0 || !built) {
+      for (int b = threadIdx.x; b < 2048; b += NT) hist[b] = 0;
+      __syncthreads();
+      for (int j = threadIdx.x; j < ns; j += NT) {
+        const uint32_t key = skey[j];
+        if (level == 0 || (key >> 21) == (prefix >> 21)) atomicAdd(&hist[(key >> lo) & 2047u], 1);
+      }
+      __syncthreads();
     }
-    __syncthreads();
     sel::find_bin<NT>(hist, 2048, need, warp_sums, s_bin, s_above, s_ok);
     prefix |= *s_bin << lo;
     need -= *s_above;
@@ -235,7 +239,13 @@ __global__ void __launch_bounds__(kSampleThreads) topk_sample_kernel(IndexerArgs
   const int64_t tl = blockIdx.x;
   const int64_t t = a.t_begin + tl;
   if (threadIdx.x == 0) a.cand_count[tl] = 0u;
+  // the query's position, sequence and head fragments load together
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, q4 = lane & 3;
   const int64_t n = eligible_of(a, t);
+  const int32_t seq = a.seq_id ? __ldg(a.seq_id + t) : 0;
+  QueryFrags<CI, NT> Q;
+  Q.load(a, t, g, q4);
   // few entries: every key is a candidate (cand_cap >= 2 top_k), nothing to sample
   if (n <= a.skip_le || 2 * n <= a.cand_cap) {
     if (threadIdx.x == 0) const_cast<uint32_t*>(a.tau)[tl] = 0u;
@@ -243,11 +253,8 @@ __global__ void __launch_bounds__(kSampleThreads) topk_sample_kernel(IndexerArgs
   }
   const int ns = sample_size(n);
   const int ng = ns / 16;
-  const int32_t seq = a.seq_id ? __ldg(a.seq_id + t) : 0;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, q4 = lane & 3;
-  QueryFrags<CI, NT> Q;
-  Q.load(a, t, g, q4);
+  for (int b = threadIdx.x; b < 2048; b += kSampleThreads) hist[b] = 0;
+  __syncthreads();
   for (int g0 = warp * kU; g0 < ng; g0 += (kSampleThreads / 32) * kU) {
     uint4 kr[kU][2][CI / 32];
 #pragma unroll
@@ -268,12 +275,16 @@ __global__ void __launch_bounds__(kSampleThreads) topk_sample_kernel(IndexerArgs
       float sg, s8;
       score_group<CI, NT>(kr[u], Q, sg, s8);
       const int grp = g0 + u;
-      if (grp < ng && q4 < 2) skey[grp * 16 + g + 8 * q4] = score_key(q4 == 0 ? sg : s8);
+      if (grp < ng && q4 < 2) {
+        const uint32_t key = score_key(q4 == 0 ? sg : s8);
+        skey[grp * 16 + g + 8 * q4] = key;
+        atomicAdd(&hist[key >> 21], 1);   // the first radix level
+      }
     }
   }
   __syncthreads();
-  const uint32_t tau =
-      sample_threshold<kSampleThreads>(skey, ns, n, top_k, hist, warp_sums, &s_bin, &s_above, &s_ok);
+  const uint32_t tau = sample_threshold<kSampleThreads>(skey, ns, n, top_k, hist, warp_sums, &s_bin,
+                                                        &s_above, &s_ok, true);
   if (threadIdx.x == 0) const_cast<uint32_t*>(a.tau)[tl] = tau;
 }
 

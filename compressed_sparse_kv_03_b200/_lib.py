@@ -39,7 +39,14 @@ class CacheT(C.Structure):
                 ("page_table", C.c_void_p), ("page_size", C.c_int32), ("max_pages", C.c_int32)]
 
 
+class QRopeT(C.Structure):
+    """Mirror of csa_qrope_t."""
+    _fields_ = [("q_gain", C.c_void_p), ("q_eps", C.c_float), ("rope_dims", C.c_int32),
+                ("rope_base", C.c_float), ("derotate", C.c_int32), ("pos", C.c_void_p)]
+
+
 _vp, _i32, _i64, _f32, _sz = C.c_void_p, C.c_int32, C.c_int64, C.c_float, C.c_size_t
+_qr = C.POINTER(QRopeT)
 
 # name -> (restype, argtypes); the exact list of functions include/csa.h declares
 SIGNATURES = {
@@ -66,15 +73,15 @@ SIGNATURES = {
     "csa_indexer_topk_mxfp4": (C.c_int, [_vp, _vp, C.POINTER(CacheT), _vp, _vp, _vp, _i64, _i32,
                                          _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "csa_sparse_attn_prefill": (C.c_int, [_vp, _vp, _i64, _vp, _vp, _vp, _i64, _i32, _i32, _i32,
-                                          _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+                                          _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp, _qr]),
     "csa_sparse_attn_decode": (C.c_int, [_vp, C.POINTER(CacheT), _vp, _vp, _vp, _vp, _i32, _i32,
-                                         _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+                                         _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp, _qr]),
     "csa_quantize_entries_fp8": (C.c_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp]),
     "csa_sparse_attn_decode_fp8": (C.c_int, [_vp, C.POINTER(CacheT), _vp, _vp, _i32, _vp, _vp, _vp,
                                              _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp,
                                              _vp, _vp, _sz, _vp]),
     "hca_attn": (C.c_int, [_vp, C.POINTER(CacheT), _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i64,
-                           _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+                           _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp, _qr]),
     "csa_sparse_attn_decode_noalloc": (C.c_int, [_vp, C.POINTER(CacheT), _vp, _vp, _vp, _vp, _i32,
                                                  _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
                                                  _vp]),

@@ -22,7 +22,7 @@ from typing import Optional
 import torch
 
 from . import _lib
-from ._lib import CacheT, check, load
+from ._lib import CacheT, QRopeT, check, load
 
 
 def _ptr(t):
@@ -305,10 +305,38 @@ def indexer_topk_mxfp4(q_idx, w, keys: Cache, k_scales, m, top_k, *, seq_id=None
     return (idx, cnt, sco) if return_scores else (idx, cnt)
 
 
+@dataclass
+class QRope:
+    """The attention calls' fused query prologue / output epilogue
+    (csa_qrope_t): every query head becomes R_t . RMSNorm(q) * gain, rounded to
+    bf16, before the dot products; with `derotate` each output head's last
+    rope_dims coordinates are rotated back by R_{-t}.  eps < 0 skips the
+    RMSNorm, rope_dims = 0 the rotation.  pos: int64 [T] query positions
+    (required on decode calls; default: the row index, or q_pos for HCA)."""
+    gain: "torch.Tensor | None" = None
+    eps: float = 1e-6
+    rope_dims: int = 64
+    rope_base: float = 10000.0
+    derotate: bool = True
+    pos: "torch.Tensor | None" = None
+
+
+def _qrope_c(qr, dev):
+    if qr is None:
+        return None
+    if qr.gain is not None:
+        _need(qr.gain, "qrope.gain", torch.float32, 1, dev)
+    if qr.pos is not None:
+        _need(qr.pos, "qrope.pos", torch.int64, 1, dev)
+    return C.byref(QRopeT(_ptr(qr.gain), float(qr.eps), int(qr.rope_dims), float(qr.rope_base),
+                          int(bool(qr.derotate)), _ptr(qr.pos)))
+
+
 def sparse_attn_prefill(q, kv_comp, kv_raw, idx, count, window, sm_scale, *, sink=None,
-                        return_lse=False, ws=None, stream=None, out=None):
+                        qrope=None, return_lse=False, ws=None, stream=None, out=None):
     """Step 4 (CSA prefill): query t attends to kv_comp[idx[t, :count[t]]]
-    and the raw window rows max(0, t-W+1) .. t."""
+    and the raw window rows max(0, t-W+1) .. t; `qrope` (QRope) fuses the
+    query RMSNorm / RoPE and the output de-rotation."""
     _need(q, "q", torch.bfloat16, 3)
     L, H, d = q.shape
     dev = q.device
@@ -327,14 +355,15 @@ def sparse_attn_prefill(q, kv_comp, kv_raw, idx, count, window, sm_scale, *, sin
     check(lib.csa_sparse_attn_prefill(_ptr(q), _ptr(kv_comp), kv_comp.shape[0], _ptr(kv_raw),
                                       _ptr(idx), _ptr(count), L, H, d, top_k, window,
                                       float(sm_scale), _ptr(sink), _ptr(out), _ptr(lse), wsp, wsb,
-                                      _stream(stream)))
+                                      _stream(stream), _qrope_c(qrope, dev)))
     return (out, lse) if return_lse else out
 
 
 def sparse_attn_decode(q, kv: Cache, win, win_len, idx, count, sm_scale, *, sink=None,
-                       return_lse=False, ws=None, stream=None, out=None):
+                       qrope=None, return_lse=False, ws=None, stream=None, out=None):
     """Step 4 (CSA decode): query b attends to entries idx[b, :count[b]] of
-    sequence b of `kv` and its window buffer win[b, :win_len[b]]."""
+    sequence b of `kv` and its window buffer win[b, :win_len[b]]; `qrope`
+    (QRope, pos required) fuses the query prologue / output de-rotation."""
     _need(q, "q", torch.bfloat16, 3)
     B, H, d = q.shape
     dev = q.device
@@ -354,7 +383,8 @@ def sparse_attn_decode(q, kv: Cache, win, win_len, idx, count, sm_scale, *, sink
     kc = kv.c()
     check(lib.csa_sparse_attn_decode(_ptr(q), C.byref(kc), _ptr(win), _ptr(win_len), _ptr(idx),
                                      _ptr(count), B, H, d, top_k, window, float(sm_scale),
-                                     _ptr(sink), _ptr(out), _ptr(lse), wsp, wsb, _stream(stream)))
+                                     _ptr(sink), _ptr(out), _ptr(lse), wsp, wsb, _stream(stream),
+                                     _qrope_c(qrope, dev)))
     return (out, lse) if return_lse else out
 
 
@@ -416,8 +446,8 @@ def sparse_attn_decode_fp8(q, codes: Cache, scales, rope, win, win_len, idx, cou
     return (out, lse) if return_lse else out
 
 def hca_attn(q, kv: Cache, kv_win, m, window, sm_scale, *, win_len=None, q_pos=None,
-             seq_id=None, max_entries=None, sink=None, return_lse=False, ws=None, stream=None,
-             out=None):
+             seq_id=None, max_entries=None, sink=None, qrope=None, return_lse=False, ws=None,
+             stream=None, out=None):
     """Step 4 (HCA): dense attention over every entry s < floor(t/m) plus the
     window.  Decode when `win_len` is given (kv_win [T, window, d]; query i
     reads sequence seq_id[i], default i); prefill otherwise: of sequence 0
@@ -453,7 +483,7 @@ def hca_attn(q, kv: Cache, kv_win, m, window, sm_scale, *, win_len=None, q_pos=N
     check(lib.hca_attn(_ptr(q), C.byref(kc), _ptr(kv_win), _ptr(win_len), _ptr(seq_id), _ptr(q_pos),
                        T, H, d, m,
                        max_entries, window, float(sm_scale), _ptr(sink), _ptr(out), _ptr(lse), wsp,
-                       wsb, _stream(stream)))
+                       wsb, _stream(stream), _qrope_c(qrope, dev)))
     return (out, lse) if return_lse else out
 
 

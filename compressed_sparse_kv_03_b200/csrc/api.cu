@@ -581,6 +581,37 @@ csa_status_t check_attn_common(const char* name, const csa_bf16* q, const csa_bf
   return CSA_OK;
 }
 
+// The fused query prologue / output epilogue: checks and AttnArgs fields.
+csa_status_t apply_qrope(const char* name, const csa_qrope_t* r, bool decode, AttnArgs& a) {
+  if (r == nullptr) return CSA_OK;
+  if (r->rope_dims < 0 || r->rope_dims > kD || r->rope_dims % 8 != 0 ||
+      (r->rope_dims > 0 && !(r->rope_base > 1.f)) || (r->derotate != 0 && r->derotate != 1) ||
+      !(r->q_eps == r->q_eps))
+    return fail(CSA_ERR_INVALID_ARG,
+                "%s: qrope needs rope_dims a multiple of 8 up to %d, rope_base > 1 when rotating, "
+                "derotate in {0,1}", name, kD);
+  if (decode && r->rope_dims > 0 && r->pos == nullptr)
+    return fail(CSA_ERR_INVALID_ARG, "%s: qrope on a decode call needs pos", name);
+  if (r->q_gain != nullptr && !aligned16(r->q_gain))
+    return fail(CSA_ERR_INVALID_ARG, "%s: qrope gain must be 16-byte aligned", name);
+  a.qprologue = (r->q_eps >= 0.f || r->rope_dims > 0) ? 1 : 0;
+  a.q_norm_gain = r->q_gain;
+  a.q_norm_eps = r->q_eps;
+  a.q_rope_dims = r->rope_dims;
+  a.q_rope_base = r->rope_base;
+  a.out_derotate = r->rope_dims > 0 ? r->derotate : 0;
+  a.rope_pos = r->pos;
+  return CSA_OK;
+}
+
+csa_status_t need_tc_for_qrope(const char* name, const AttnArgs& a) {
+  if ((a.qprologue || a.out_derotate) && !a.use_tc)
+    return fail(CSA_ERR_UNSUPPORTED,
+                "%s: the fused query prologue / output de-rotation runs on the tensor-core "
+                "attention kernel only", name);
+  return CSA_OK;
+}
+
 }  // namespace
 
 csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
@@ -589,7 +620,7 @@ csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
                                      int32_t H, int32_t d, int32_t top_k, int32_t window,
                                      float sm_scale, const float* sink, csa_bf16* out,
                                      float* lse, void* ws, size_t ws_bytes,
-                                     csa_stream_t stream) {
+                                     csa_stream_t stream, const csa_qrope_t* qrope) {
   const char* name = "csa_sparse_attn_prefill";
   if (L == 0) return CSA_OK;
   csa_status_t st = check_attn_common(name, q, out, H, d, window);
@@ -624,8 +655,10 @@ csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
   a.sink = sink;
   a.out = (__nv_bfloat16*)out;
   a.lse = lse;
+  if ((st = apply_qrope(name, qrope, false, a)) != CSA_OK) return st;
   // prefill: one slice per query (many queries fill the GPU)
   a.use_tc = attention_uses_tc(a);
+  if ((st = need_tc_for_qrope(name, a)) != CSA_OK) return st;
   a.n_split = 1;
   a.split_len = (int)(((int64_t)top_k + window + 63) / 64 * 64);
   st = check_ws(ws, ws_bytes, kWsHeader, name);
@@ -650,6 +683,7 @@ csa_status_t run_decode_attention(AttnArgs a, const char* name, int32_t B, int32
   csa_status_t st = check_ws(ws, ws_bytes, attn_partials_bytes(B, H, n_need), name);
   if (st != CSA_OK) return st;
   a.use_tc = attention_uses_tc(a);
+  if ((st = need_tc_for_qrope(name, a)) != CSA_OK) return st;
   const Split sp = invariant ? sp_inv
                              : (a.use_tc ? attn_split_tc(B, (int64_t)top_k + window, H, sp_ws) : sp_ws);
   a.n_split = sp.n;
@@ -727,14 +761,15 @@ csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_com
                                     int32_t H, int32_t d, int32_t top_k, int32_t window,
                                     float sm_scale, const float* sink, csa_bf16* out,
                                     float* lse, void* ws, size_t ws_bytes,
-                                    csa_stream_t stream) {
+                                    csa_stream_t stream, const csa_qrope_t* qrope) {
   const char* name = "csa_sparse_attn_decode";
   if (B == 0) return CSA_OK;
   csa_status_t st =
       check_decode_args(name, q, kv_comp, win, win_len, idx, count, B, H, d, top_k, window, out);
   if (st != CSA_OK) return st;
-  const AttnArgs a = decode_args(q, kv_comp, win, win_len, idx, count, B, H, top_k, window,
-                                 sm_scale, sink, out, lse);
+  AttnArgs a = decode_args(q, kv_comp, win, win_len, idx, count, B, H, top_k, window,
+                           sm_scale, sink, out, lse);
+  if ((st = apply_qrope(name, qrope, true, a)) != CSA_OK) return st;
   return run_decode_attention(a, name, B, H, top_k, window, ws, ws_bytes, stream);
 }
 
@@ -794,7 +829,7 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
                       int64_t T, int32_t H,
                       int32_t d, int32_t m, int64_t max_entries, int32_t window,
                       float sm_scale, const float* sink, csa_bf16* out, float* lse, void* ws,
-                      size_t ws_bytes, csa_stream_t stream) {
+                      size_t ws_bytes, csa_stream_t stream, const csa_qrope_t* qrope) {
   const char* name = "hca_attn";
   if (T == 0) return CSA_OK;
   csa_status_t st = check_attn_common(name, q, out, H, d, window);
@@ -830,12 +865,14 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
   a.sink = sink;
   a.out = (__nv_bfloat16*)out;
   a.lse = lse;
+  if ((st = apply_qrope(name, qrope, false, a)) != CSA_OK) return st;   // pos defaults to q_pos
   const Split sp_ws = attn_split(T, max_entries + window, H);
   const bool invariant = win_len != nullptr && g_batch_invariant.load(std::memory_order_relaxed) != 0;
   const Split sp_inv = attn_split_invariant(max_entries + window);
   const int n_need = invariant && sp_inv.n > sp_ws.n ? sp_inv.n : sp_ws.n;
   if ((st = check_ws(ws, ws_bytes, attn_partials_bytes(T, H, n_need), name)) != CSA_OK) return st;
   a.use_tc = attention_uses_tc(a);
+  if ((st = need_tc_for_qrope(name, a)) != CSA_OK) return st;
   const Split sp = invariant ? sp_inv
                              : (a.use_tc ? attn_split_tc(T, max_entries + window, H, sp_ws) : sp_ws);
   a.n_split = sp.n;

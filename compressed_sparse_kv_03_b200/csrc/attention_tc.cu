@@ -30,6 +30,8 @@
 // (programmatic dependent launch): it sets up its barriers and TMEM and then
 // waits for that kernel before it reads anything.
 // Every wait is bounded (the workspace header records a timeout).
+#include <cmath>
+
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -88,7 +90,25 @@ struct TcAttnParams {
   AttnArgs a;
   int hgroups;
   int64_t items;
+  double theta[kD / 2];   // rotary pair frequencies base^(-2j / rope_dims) (host-filled)
 };
+
+// Position of query i for the rotary prologue / epilogue.
+__device__ __forceinline__ int64_t rope_position(const AttnArgs& a, int64_t i) {
+  return a.rope_pos ? __ldg(a.rope_pos + i) : (a.q_pos ? __ldg(a.q_pos + i) : i);
+}
+
+// cos / sin of the rotation of pair j at position p (R_p, or R_{-p} with
+// inverse): the angle is formed and reduced modulo 2 pi in double precision
+// (positions reach 2^20 and more), then sincosf.
+__device__ __forceinline__ void rope_cs(const TcAttnParams& p, int64_t pos, int j, bool inverse,
+                                        float& c, float& s) {
+  const double two_pi = 6.283185307179586476925, inv_two_pi = 0.159154943091895335769;
+  double ang = (double)pos * p.theta[j];
+  ang -= two_pi * floor(ang * inv_two_pi);
+  if (inverse) ang = -ang;
+  sincosf((float)ang, &s, &c);
+}
 
 // Row list of one (query, split): selected / eligible entries [v0, min(v1, n_sel)),
 // then window rows [max(v0, n_sel), v1) (virtual indices).
@@ -203,6 +223,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
   __shared__ __align__(8) uint64_t kv_full[kStages], kv_empty[kStages];
   __shared__ __align__(8) uint64_t q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2];
   __shared__ __align__(8) uint64_t o_full, o_empty, o_step, red_bar[kSmGroups];
+  // query prologue: the tile is normalised / rotated in place before S^T
+  __shared__ __align__(8) uint64_t q_ready[2], pro_bar;
+  __shared__ float2 rope_tab[2][kD / 2];   // cos / sin per pair, by Q buffer
   __shared__ uint32_t tmem_base_sh;
   // validity of the tile's rows, one word per producer warp: bit 2j + s of
   // word k is row 2 (k + 7 j) + s
@@ -233,6 +256,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
     mbar_init(smem_u32(&o_full), 1);
     mbar_init(smem_u32(&o_empty), kSmWarps);
     mbar_init(smem_u32(&o_step), 1);
+    mbar_init(smem_u32(&q_ready[0]), kSmWarps);
+    mbar_init(smem_u32(&q_ready[1]), kSmWarps);
+    mbar_init(smem_u32(&pro_bar), kSmWarps);
     for (int g = 0; g < kSmGroups; ++g) mbar_init(smem_u32(&red_bar[g]), 4);
     mbar_fence_init();
   }
@@ -418,7 +444,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         if (it.n_tiles == 0) continue;
         const int qb = (int)(items_done & 1);
         const uint32_t qs = q_sm + qb * kQTile;
-        if (!mbar_wait(smem_u32(&q_full[qb]), (uint32_t)((items_done >> 1) & 1))) {
+        if (!mbar_wait(smem_u32(a.qprologue ? &q_ready[qb] : &q_full[qb]), (uint32_t)((items_done >> 1) & 1))) {
           report(a.err, kErrTimeout, (int32_t)it.i, 22);
           ok = false;
           break;
@@ -478,7 +504,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
     const uint32_t rbar = smem_u32(&red_bar[wg]);
     const float scale = a.sm_scale * kLog2e;
     float* const my_bc = w_bcast[warp];   // this warp's per-head broadcast row
-    uint32_t red_phase = 0;
+    uint32_t red_phase = 0, pro_phase = 0;
     int64_t tiles_done = 0, items_done = 0, pv_seen = 0;
     for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
       const ItemInfo it = item_info(a, p.hgroups, item, false);
@@ -500,6 +526,77 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
           }
         }
         continue;
+      }
+      if (a.qprologue) {
+        // ---------------------------------------------------- query prologue
+        // RMSNorm (times the gain) and the rotation R_t of every head of this
+        // item's query tile, in place in shared memory: thread = (head,
+        // quarter of the dims), four 16-byte chunks of the swizzled tile.
+        const int qb = (int)(items_done & 1);
+        bool okp = mbar_wait(smem_u32(&q_full[qb]), (uint32_t)((items_done >> 1) & 1));
+        const int r0 = kD - a.q_rope_dims;
+        if (okp && a.q_rope_dims > 0 && (int)threadIdx.x < a.q_rope_dims / 2) {
+          float c, sn;
+          rope_cs(p, rope_position(a, it.i), threadIdx.x, false, c, sn);
+          rope_tab[qb][threadIdx.x] = make_float2(c, sn);
+        }
+        okp = okp && group_sync(smem_u32(&pro_bar), pro_phase, lane);
+        if (!okp) {
+          if (lane == 0) report(a.err, kErrTimeout, (int32_t)it.i, 30);
+          break;
+        }
+        const int head = threadIdx.x >> 2, qq = threadIdx.x & 3;
+        uint8_t* const qtile = smem_raw + (q_sm + qb * kQTile - smem_u32(smem_raw));
+        float x[32];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {   // chunk cc = dims [8 cc, 8 cc + 8)
+          const int cc = 4 * qq + i, blk = cc >> 3, cb = cc & 7;
+          const uint4 v = *reinterpret_cast<const uint4*>(qtile + blk * (kQTile / 2) + head * 128 +
+                                                          ((cb ^ (head & 7)) << 4));
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f2 = unpack_bf16(w4[e]);
+            x[8 * i + 2 * e] = f2.x;
+            x[8 * i + 2 * e + 1] = f2.y;
+          }
+        }
+        if (a.q_norm_eps >= 0.f) {
+          float ss = 0.f;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ss = fmaf(x[e], x[e], ss);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+          const float rn = fminf(rsqrtf(ss / (float)kD + a.q_norm_eps), 3.0e38f);   // zero rows stay zero
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float gv = a.q_norm_gain ? __ldg(a.q_norm_gain + 32 * qq + e) : 1.f;
+            x[e] *= rn * gv;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int dim = 32 * qq + e;
+          if (a.q_rope_dims > 0 && dim >= r0) {
+            const float2 cs = rope_tab[qb][(dim - r0) >> 1];
+            const float u = x[e], w = x[e + 1];
+            x[e] = u * cs.x - w * cs.y;
+            x[e + 1] = u * cs.y + w * cs.x;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int cc = 4 * qq + i, blk = cc >> 3, cb = cc & 7;
+          uint4 v;
+          v.x = pack_bf16(x[8 * i], x[8 * i + 1]);
+          v.y = pack_bf16(x[8 * i + 2], x[8 * i + 3]);
+          v.z = pack_bf16(x[8 * i + 4], x[8 * i + 5]);
+          v.w = pack_bf16(x[8 * i + 6], x[8 * i + 7]);
+          *reinterpret_cast<uint4*>(qtile + blk * (kQTile / 2) + head * 128 + ((cb ^ (head & 7)) << 4)) = v;
+        }
+        fence_async_smem();   // the MMA reads the tile through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&q_ready[qb]));
       }
       float m_run = -INFINITY;   // lane h: running max of head hoff + h, log2 units
       float lpart[kHW];
@@ -673,6 +770,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
       __syncwarp();
       tc::fence_after_sync();
       const int d = row;   // O^T lane = output dim
+      // output de-rotation R_{-t} of the rotary pairs (2j, 2j+1): the pair's
+      // two dims sit in neighbouring lanes; applied before normalisation or to
+      // the split partials alike (both are linear in O)
+      const bool derot = a.out_derotate && d >= kD - a.q_rope_dims;
+      float dc = 1.f, ds = 0.f;
+      if (derot) rope_cs(p, rope_position(a, it.i), (d - (kD - a.q_rope_dims)) >> 1, true, dc, ds);
+      const float dsig = (d & 1) ? ds : -ds;   // even: v c - partner s; odd: v c + partner s
       if (a.n_split == 1) {
         __nv_bfloat16* const outp = a.out + (it.i * a.H + h_base) * kD + d;
 #pragma unroll 1
@@ -683,7 +787,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int h = hoff + c * 16 + j;
-            if (h < nh) outp[(int64_t)h * kD] = __float2bfloat16_rn(__uint_as_float(r[j]) * my_bc[kHW + c * 16 + j]);
+            float v = __uint_as_float(r[j]) * my_bc[kHW + c * 16 + j];
+            const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
+            if (derot) v = fmaf(v, dc, partner * dsig);
+            if (h < nh) outp[(int64_t)h * kD] = __float2bfloat16_rn(v);
           }
         }
       } else {
@@ -696,7 +803,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int h = hoff + c * 16 + j;
-            if (h < nh) accp[(int64_t)h * kD] = __uint_as_float(r[j]);
+            float v = __uint_as_float(r[j]);
+            const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
+            if (derot) v = fmaf(v, dc, partner * dsig);
+            if (h < nh) accp[(int64_t)h * kD] = v;
           }
         }
       }
@@ -736,6 +846,9 @@ cudaError_t launch_attention_tc(const Launch& L, const AttnArgs& a) {
   p.a = a;
   p.hgroups = (a.H + kNP - 1) / kNP;
   p.items = a.T * a.n_split * p.hgroups;
+  for (int j = 0; j < kD / 2; ++j)
+    p.theta[j] = j < a.q_rope_dims / 2
+                     ? std::pow((double)a.q_rope_base, -2.0 * j / (double)a.q_rope_dims) : 0.0;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

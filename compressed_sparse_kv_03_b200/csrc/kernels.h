@@ -232,6 +232,17 @@ struct AttnArgs {
   const uint8_t* kv_scales = nullptr;
   const __nv_bfloat16* kv_rope = nullptr;
   int rope_dims = 0;
+  // query prologue / output epilogue (tcgen05 kernel only): RMSNorm of every
+  // query head (q_norm_eps >= 0, gain q_norm_gain [128] or null), rotation of
+  // its last q_rope_dims coordinates by R_t, and with out_derotate the
+  // output's by R_{-t}; t = rope_pos[i] (or q_pos[i], or i)
+  int qprologue = 0;
+  const float* q_norm_gain = nullptr;
+  float q_norm_eps = -1.f;
+  int q_rope_dims = 0;
+  float q_rope_base = 10000.f;
+  int out_derotate = 0;
+  const int64_t* rope_pos = nullptr;
 };
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a);
 

@@ -96,5 +96,6 @@ extern "C" csa_status_t csa_sparse_attn_decode_noalloc(
     return CSA_ERR_CUDA;
   }
   return csa_sparse_attn_decode(q, kv_comp, win, win_len, idx, count, B, H, d, top_k, window,
-                                sm_scale, sink, out, lse, scratch, kNoAllocScratchBytes, stream);
+                                sm_scale, sink, out, lse, scratch, kNoAllocScratchBytes, stream,
+                                nullptr);
 }

@@ -310,6 +310,34 @@ csa_status_t csa_indexer_topk_mxfp4(const csa_bf16* q_idx, const float* w,
 
 /* ---- step 4: attention ---------------------------------------------------- */
 /*
+ * csa_qrope_t -- the attention layer's query prologue and output epilogue,
+ * fused into the attention calls below (Ch.7 "Query and KV RMSNorm", "Partial
+ * RoPE and output de-rotation"; Ch.2 "Normalization and rotary position
+ * embeddings").  With a non-NULL csa_qrope_t* the call reads the raw queries
+ * and, before the dot products, replaces every query head q by
+ *   R_t . (q / sqrt(mean(q^2) + q_eps) * q_gain)        (q_eps < 0: no RMSNorm)
+ * rounded to bf16, R_t rotating pairs (2j, 2j+1) of the last rope_dims
+ * coordinates by t * rope_base^(-2j / rope_dims) (t the query's position); with
+ * derotate = 1 each output head's last rope_dims coordinates are rotated by
+ * R_{-t} before they are stored.  The compressed entries and window rows are
+ * used as given (normalise and rotate them once with csa_norm_rope).
+ *   q_gain     [d] fp32 gain, or NULL (gain 1)
+ *   rope_dims  a multiple of 8 up to d (0: no rotation); rope_base > 1 when used
+ *   pos        [T] int64 position of each query; NULL means the row index for
+ *              csa_sparse_attn_prefill and q_pos (else the row index) for
+ *              hca_attn; required by csa_sparse_attn_decode
+ * Needs the tensor-core attention kernel (CSA_ERR_UNSUPPORTED otherwise).
+ */
+typedef struct {
+  const float* q_gain;
+  float q_eps;
+  int32_t rope_dims;
+  float rope_base;
+  int32_t derotate;
+  const int64_t* pos;
+} csa_qrope_t;
+
+/*
  * csa_sparse_attn_prefill -- CSA attention for the L queries of one sequence,
  * query t at position t:
  *   o[t,h] = sum_j softmax_j(sm_scale * q[t,h] . kv_j) kv_j
@@ -320,6 +348,7 @@ csa_status_t csa_indexer_topk_mxfp4(const csa_bf16* q_idx, const float* w,
  *   q        [L, H, d] bf16        kv_comp [n_entries, d] bf16
  *   kv_raw   [L, d] bf16           idx [L, top_k] int32, count [L] int32
  *   out      [L, H, d] bf16        lse [L, H] fp32 log of the denominator, or NULL
+ *   qrope    query prologue / output epilogue (see csa_qrope_t), or NULL
  */
 csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
                                      int64_t n_entries, const csa_bf16* kv_raw,
@@ -327,7 +356,7 @@ csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
                                      int32_t H, int32_t d, int32_t top_k, int32_t window,
                                      float sm_scale, const float* sink, csa_bf16* out,
                                      float* lse, void* ws, size_t ws_bytes,
-                                     csa_stream_t stream);
+                                     csa_stream_t stream, const csa_qrope_t* qrope);
 
 /*
  * csa_sparse_attn_decode -- one new token per sequence b (query b belongs to
@@ -339,6 +368,7 @@ csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
  * as the way decode keeps every SM busy).
  *   q [B, H, d] bf16; win [B, window, d] bf16; win_len [B] int32 (<= window)
  *   idx [B, top_k] int32; count [B] int32; out [B, H, d] bf16; lse [B, H] or NULL
+ *   qrope query prologue / output epilogue (csa_qrope_t; its pos is required), or NULL
  */
 csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_comp,
                                     const csa_bf16* win, const int32_t* win_len,
@@ -346,7 +376,7 @@ csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_com
                                     int32_t H, int32_t d, int32_t top_k, int32_t window,
                                     float sm_scale, const float* sink, csa_bf16* out,
                                     float* lse, void* ws, size_t ws_bytes,
-                                    csa_stream_t stream);
+                                    csa_stream_t stream, const csa_qrope_t* qrope);
 
 /*
  * csa_sparse_attn_decode_noalloc -- csa_sparse_attn_decode for callers that
@@ -454,13 +484,15 @@ csa_status_t csa_sparse_attn_decode_fp8(const csa_bf16* q, const csa_cache_t* kv
  *     (the caller's layout); a window that would start before row 0 is cut
  *     there and recorded in the workspace header.
  *   max_entries bounds floor(t_i/m) (split layout); q [T, H, d]; out [T, H, d];
- *   lse [T, H] or NULL; sink [H] or NULL; seq_id [T] int32 or NULL.
+ *   lse [T, H] or NULL; sink [H] or NULL; seq_id [T] int32 or NULL;
+ *   qrope query prologue / output epilogue (csa_qrope_t), or NULL.
  */
 csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_bf16* kv_win,
                       const int32_t* win_len, const int32_t* seq_id, const int64_t* q_pos,
                       int64_t T, int32_t H, int32_t d, int32_t m, int64_t max_entries,
                       int32_t window, float sm_scale, const float* sink, csa_bf16* out,
-                      float* lse, void* ws, size_t ws_bytes, csa_stream_t stream);
+                      float* lse, void* ws, size_t ws_bytes, csa_stream_t stream,
+                      const csa_qrope_t* qrope);
 
 #ifdef __cplusplus
 }

@@ -75,7 +75,7 @@ def test_attention_rejects_unsupported_dims(lib):
     wsp = C.cast(C.addressof(ws) + (-C.addressof(ws)) % 256, C.c_void_p)
     # head dim 512 is a legal size the library does not build
     st = lib.csa_sparse_attn_decode(p, C.byref(cache), p, p, p, p, 1, 8, 512, 4, 8, 1.0, None, p,
-                                    None, wsp, 512, None)
+                                    None, wsp, 512, None, None)
     assert st == 2 and b"head dim" in lib.csa_last_error()
     # indexer key dim 96
     st = lib.csa_indexer_topk(p, p, C.byref(cache), None, None, 4, 2, 96, 4, 16, 2, p, p, None,
@@ -84,12 +84,43 @@ def test_attention_rejects_unsupported_dims(lib):
     # null cache data
     bad = CacheT(None, 16, 16, None, 0, 0)
     st = lib.hca_attn(p, C.byref(bad), p, None, None, None, 4, 8, 128, 4, 16, 8, 1.0, None, p,
-                      None, wsp, 512, None)
+                      None, wsp, 512, None, None)
     assert st == 1
     # decode with a window needs the window buffer
     st = lib.csa_sparse_attn_decode(p, C.byref(cache), None, None, p, p, 1, 8, 128, 4, 8, 1.0,
-                                    None, p, None, wsp, 512, None)
+                                    None, p, None, wsp, 512, None, None)
     assert st == 1
+    assert lib.csa_launch_count() == 0
+
+
+def test_qrope_arguments_are_checked_before_any_launch(lib):
+    """The fused query prologue's arguments (csa_qrope_t) are validated on the
+    host: rotary width a multiple of 8 up to the head dim, a base above 1, a
+    0/1 de-rotation flag, an aligned gain, and a position array on the decode
+    call, which has no other source of positions."""
+    from compressed_sparse_kv_03_b200._lib import CacheT, QRopeT
+    buf = (C.c_uint8 * 4096)()
+    p = C.cast(C.addressof(buf) + (-C.addressof(buf)) % 16, C.c_void_p)
+    cache = CacheT(p.value, 16, 16, None, 0, 0)
+    ws = (C.c_uint8 * 1024)()
+    wsp = C.cast(C.addressof(ws) + (-C.addressof(ws)) % 256, C.c_void_p)
+    odd_gain = C.c_void_p(p.value + 4)
+    bad = [QRopeT(None, 1e-6, 60, 1e4, 1, p.value),        # rope_dims not a multiple of 8
+           QRopeT(None, 1e-6, 136, 1e4, 1, p.value),       # wider than the head
+           QRopeT(None, 1e-6, 64, 1.0, 1, p.value),        # base must exceed 1
+           QRopeT(None, 1e-6, 64, 1e4, 2, p.value),        # derotate not 0/1
+           QRopeT(None, float("nan"), 64, 1e4, 1, p.value),
+           QRopeT(odd_gain, 1e-6, 64, 1e4, 1, p.value),    # misaligned gain
+           QRopeT(None, 1e-6, 64, 1e4, 1, None)]           # decode without positions
+    for r in bad:
+        st = lib.csa_sparse_attn_decode(p, C.byref(cache), p, p, p, p, 1, 8, 128, 4, 8, 1.0, None,
+                                        p, None, wsp, 512, None, C.byref(r))
+        assert st == 1 and b"qrope" in lib.csa_last_error(), (r.rope_dims, lib.csa_last_error())
+    # prefill takes the row index as the position: no pos needed, but the
+    # other checks hold there too
+    st = lib.csa_sparse_attn_prefill(p, p, 16, p, p, p, 4, 8, 128, 4, 8, 1.0, None, p, None, wsp,
+                                     512, None, C.byref(bad[0]))
+    assert st == 1 and b"qrope" in lib.csa_last_error()
     assert lib.csa_launch_count() == 0
 
 

@@ -48,15 +48,15 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int64_t score_stride(int64_t max_entries) { return (max_entries + 63) / 64 * 64; }
 
-// Indexer workspace.  Few-query (fused) mode: header | per query tau and
-// candidate count [chunk][2] u32 | work counter | candidates [chunk, cap]
-// (key, entry) pairs -- O(top_k) per query, no score matrix.  Many-query
-// mode: header | work counter | keys [chunk, stride] u32.  Queries are
-// processed in chunks so that the scratch stays bounded.
+// Indexer workspace: header | per query tau, candidate count and fallback
+// list entry [3][chunk] u32 + the fallback count | work counter | candidates
+// [chunk, cap] (key, entry) pairs | in many-query mode the sampled keys
+// [chunk, kPSampleKeys] u32.  O(top_k) per query: no score matrix is stored.
+// Queries are processed in chunks so that the scratch stays bounded.
 struct IndexerLayout {
-  bool fused;
-  int64_t chunk, stride, cap;
-  size_t meta_off, counter_off, data_off, total;
+  bool many;
+  int64_t chunk, cap;
+  size_t meta_off, counter_off, data_off, sample_off, total;
 };
 
 // Candidate slots per query: the sample aims at about 2 top_k keys reaching
@@ -69,21 +69,21 @@ int64_t candidate_cap(int32_t top_k) {
 
 IndexerLayout indexer_layout(int64_t T, int64_t max_entries, int32_t top_k) {
   IndexerLayout l;
-  l.fused = T <= kFusedMaxQueries || max_entries > kRadixSelectMaxEntries;
-  l.stride = score_stride(max_entries);
+  l.many = T > kFusedMaxQueries && max_entries <= kManyMaxEntries;
   l.cap = candidate_cap(top_k);
-  const int64_t per_query = l.fused ? l.cap * 8 + 8 : l.stride * (int64_t)sizeof(uint32_t);
-  int64_t c = per_query > 0 ? (int64_t)(kIndexerChunkBytes / per_query) : T;
-  if (c < 1) c = 1;
+  const int64_t per_query = l.cap * 8 + 12 + (l.many ? kPSampleKeys * 4 : 0);
+  int64_t c = (int64_t)(kIndexerChunkBytes / per_query);
   if (c > 65535) c = 65535;
-  if (l.fused && c > kFusedMaxQueries) c = kFusedMaxQueries;
+  if (!l.many && c > kFusedMaxQueries) c = kFusedMaxQueries;
+  c &= ~int64_t(255);   // chunk starts stay aligned for the scorers' weight loads
+  if (c < 256) c = 256;
   l.chunk = c < T ? c : T;
   if (l.chunk < 1) l.chunk = 1;
   l.meta_off = kWsHeader;
-  l.counter_off = l.meta_off + (l.fused ? align256((size_t)l.chunk * 2 * sizeof(uint32_t)) : 0);
+  l.counter_off = l.meta_off + align256(((size_t)l.chunk * 3 + 1) * sizeof(uint32_t));
   l.data_off = l.counter_off + 256;
-  l.total = l.data_off + (l.fused ? align256((size_t)l.chunk * l.cap * 8)
-                                  : align256((size_t)l.chunk * l.stride * sizeof(uint32_t)));
+  l.sample_off = l.data_off + align256((size_t)l.chunk * l.cap * 8);
+  l.total = l.sample_off + (l.many ? align256((size_t)l.chunk * kPSampleKeys * 4) : 0);
   return l;
 }
 
@@ -410,10 +410,12 @@ csa_status_t csa_norm_rope(const csa_bf16* x, csa_bf16* out, int64_t T, int32_t 
 // ---- steps 2-3 ---------------------------------------------------------------
 namespace {
 
-// Score + select, one chunk of queries at a time.  Fused mode: sample /
-// threshold, scoring into candidate lists, exact finish.  Many-query mode:
-// every key stored, radix select per query.  `base` carries the query / key
-// operands.
+// Score + select, one chunk of queries at a time: a threshold from a sample
+// of each query's scores, scoring into candidate lists, exact finish.  Few
+// queries (decode): a per-query sample launch and one CTA per query in the
+// finish.  Many queries (prefill): the tcgen05 scorer's own sample pass, a
+// per-warp threshold and finish, when its shapes allow.  `base` carries the
+// query / key operands.
 csa_status_t run_indexer_topk(IndexerArgs base, const int64_t* q_pos, int64_t T, int32_t m,
                               int64_t max_entries, int32_t top_k, int32_t* idx_out,
                               int32_t* count_out, float* score_out, void* ws, csa_stream_t stream) {
@@ -433,14 +435,29 @@ csa_status_t run_indexer_topk(IndexerArgs base, const int64_t* q_pos, int64_t T,
     ia.work = work;
     ia.err = hdr;
     cudaError_t e;
-    if (lay.fused) {
-      uint32_t* meta = reinterpret_cast<uint32_t*>(wsb + lay.meta_off);
-      ia.tau = meta;
-      ia.cand_count = meta + lay.chunk;
-      ia.cand = reinterpret_cast<uint2*>(wsb + lay.data_off);
-      ia.cand_cap = lay.cap;
-      ia.skip_le = score_out ? 0 : top_k;   // scores of all-selected queries still come from the scorer
-      ia.keys_out = nullptr;
+    uint32_t* meta = reinterpret_cast<uint32_t*>(wsb + lay.meta_off);
+    ia.tau = meta;
+    ia.cand_count = meta + lay.chunk;
+    ia.fb_list = meta + 2 * lay.chunk;
+    ia.fb_count = meta + 3 * lay.chunk;
+    ia.cand = reinterpret_cast<uint2*>(wsb + lay.data_off);
+    ia.cand_cap = lay.cap;
+    ia.skip_le = score_out ? 0 : top_k;   // scores of all-selected queries still come from the scorer
+    ia.psample = lay.many ? reinterpret_cast<uint32_t*>(wsb + lay.sample_off) : nullptr;
+    if (ia.psample && tc_indexer_prefill_supported(ia, n) && topk_many_supported(ia)) {
+      // the scorer's sample pass, thresholds (which zero the counts and the
+      // work counter), the scorer's candidate pass, per-warp finish
+      e = cudaMemsetAsync(work, 0, sizeof(uint32_t), L.stream);
+      if (e != cudaSuccess) return cuda_status(e, "indexer work counter memset");
+      if ((e = launch_indexer_scores_tc_prefill(L, ia, n, true)) != cudaSuccess)
+        return cuda_status(e, "indexer sample launch");
+      if ((e = launch_topk_threshold_many(L, ia, top_k, n)) != cudaSuccess)
+        return cuda_status(e, "top-k threshold launch");
+      if ((e = launch_indexer_scores(L, ia, n)) != cudaSuccess) return cuda_status(e, "indexer score launch");
+      if ((e = launch_topk_finish_many(L, ia, top_k, idx_out, count_out, score_out, n)) != cudaSuccess)
+        return cuda_status(e, "top-k finish launch");
+    } else {
+      ia.psample = nullptr;
       // the work counter is zeroed before the sample launch (the scorer may
       // start while that one runs); the sample launch zeroes the counts
       e = cudaMemsetAsync(work, 0, sizeof(uint32_t), L.stream);
@@ -449,25 +466,6 @@ csa_status_t run_indexer_topk(IndexerArgs base, const int64_t* q_pos, int64_t T,
       if ((e = launch_indexer_scores(L, ia, n)) != cudaSuccess) return cuda_status(e, "indexer score launch");
       if ((e = launch_topk_finish(L, ia, top_k, idx_out, count_out, score_out, n)) != cudaSuccess)
         return cuda_status(e, "top-k finish launch");
-    } else {
-      e = cudaMemsetAsync(work, 0, sizeof(uint32_t), L.stream);
-      if (e != cudaSuccess) return cuda_status(e, "indexer work counter memset");
-      ia.keys_out = reinterpret_cast<uint32_t*>(wsb + lay.data_off);
-      ia.key_stride = lay.stride;
-      if ((e = launch_indexer_scores(L, ia, n)) != cudaSuccess) return cuda_status(e, "indexer score launch");
-      SelectArgs sa;
-      sa.keys = ia.keys_out;
-      sa.key_stride = lay.stride;
-      sa.q_pos = q_pos;
-      sa.m = m;
-      sa.max_entries = max_entries;
-      sa.t_begin = t0;
-      sa.top_k = top_k;
-      sa.idx_out = idx_out;
-      sa.count_out = count_out;
-      sa.score_out = score_out;
-      sa.err = hdr;
-      if ((e = launch_topk_select(L, sa, n)) != cudaSuccess) return cuda_status(e, "top-k select launch");
     }
   }
   return CSA_OK;

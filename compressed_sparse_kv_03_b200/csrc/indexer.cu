@@ -278,7 +278,7 @@ cudaError_t launch_indexer_scores(const Launch& L, const IndexerArgs& a, int64_t
   if (t_count == 0 || a.max_entries == 0) return cudaSuccess;
   if (a.fp4) return launch_indexer_scores_fp4(L, a, t_count);
 #ifndef CSA_NO_TC_INDEXER
-  if (tc_indexer_prefill_supported(a, t_count)) return launch_indexer_scores_tc_prefill(L, a, t_count);
+  if (tc_indexer_prefill_supported(a, t_count)) return launch_indexer_scores_tc_prefill(L, a, t_count, false);
   if (tc_indexer_supported(a, t_count)) return launch_indexer_scores_tc(L, a, t_count);
 #endif
   const int nt = (a.H_I + 7) / 8;

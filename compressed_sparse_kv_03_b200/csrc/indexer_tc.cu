@@ -393,6 +393,11 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
 // a key and sums the ReLU-weighted heads of each query of the block from its
 // own TMEM row, so no cross-thread reduction is needed.  Items (block, chunk)
 // follow the same hybrid static / work-counter schedule as decode mode.
+// Two passes use it (no score matrix is stored):
+//   MODE kPSample: only the block's sampled chunks (psample_chunk); every key
+//     goes to the query's sample row psample[t, i * 256 + key];
+//   MODE kPFused: every chunk; keys that reach the query's tau are appended to
+//     its candidate list, one slot reservation per warp and query.
 // ---------------------------------------------------------------------------
 constexpr int kPStages = 4;
 constexpr int kPQTileBytes = 128 * 128;                  // 128 rows x 64 bf16
@@ -408,10 +413,13 @@ constexpr int kPThreads = (2 + kPEpiWarps) * 32;
 struct __align__(16) BlockMeta {
   float w[128];       // the block's head weights in (query, head) order
   int32_t nel[32];    // eligible entries of each of the block's queries (0 past the chunk)
-  int32_t b, chunk, pad0, pad1;
+  uint32_t tau[32];   // their candidate thresholds (fused pass)
+  int32_t b, chunk, sidx, pad1;   // sidx: the chunk's ordinal among the sampled ones
 };
 
-template <int HI>
+constexpr int kPSample = 1, kPFused = 2;
+
+template <int HI, int MODE>
 __global__ void __launch_bounds__(kPThreads, 1)
 indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
                                 const __grid_constant__ CUtensorMap tmap_q, TcIndexerParams p) {
@@ -424,6 +432,7 @@ indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
   __shared__ __align__(8) uint64_t tfull_bar[kPAcc], tempty_bar[kPAcc];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int32_t prefix[kMaxBlocks + 1];
+  __shared__ int32_t bmin[MODE == kPSample ? kMaxBlocks : 1];   // fewest eligible entries per block
   __shared__ BlockMeta ring[kPRing];
   __shared__ __align__(8) uint64_t ring_full[kPRing], ring_empty[kPRing];
 
@@ -445,17 +454,31 @@ indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
     }
     mbar_fence_init();
   }
-  // chunks per block: the most eligible entries of any of its queries
-  for (int b = threadIdx.x; b < NB; b += kPThreads) prefix[b] = 0;
+  // items per block: fused pass, the chunks of its longest query that is
+  // scored; sample pass, its sampled chunks (from its fewest and most
+  // eligible entries)
+  for (int b = threadIdx.x; b < NB; b += kPThreads) {
+    prefix[b] = 0;
+    if (MODE == kPSample) bmin[b] = INT32_MAX;
+  }
   if (warp == 1) tc::tmem_alloc(smem_u32(&tmem_base_sh), kPTmemCols);
   __syncthreads();
   for (int t = threadIdx.x; t < T; t += kPThreads) {
     const int64_t pos = a.q_pos ? __ldg(a.q_pos + a.t_begin + t) : a.t_begin + t;
-    if (pos / a.m > a.max_entries && blockIdx.x == 0)
+    if (MODE == kPFused && pos / a.m > a.max_entries && blockIdx.x == 0)
       report(a.err, kErrEligible, (int32_t)(a.t_begin + t), pos / a.m);
     const int64_t n = eligible(a, a.t_begin + t);
-    atomicMax(&prefix[t / QB], (int32_t)((n + kItemRows - 1) / kItemRows));
+    if (MODE == kPSample) {
+      atomicMax(&prefix[t / QB], (int32_t)n);
+      atomicMin(&bmin[t / QB], (int32_t)n);
+    } else if (n > a.skip_le) {
+      atomicMax(&prefix[t / QB], (int32_t)((n + kItemRows - 1) / kItemRows));
+    }
   }
+  __syncthreads();
+  if (MODE == kPSample)
+    for (int b = threadIdx.x; b < NB; b += kPThreads)
+      prefix[b] = psample_chunks(bmin[b], prefix[b], a.cand_cap, a.skip_le);
   __syncthreads();
   if (warp == 0) {   // exclusive prefix over the blocks
     const int per = (NB + 31) / 32;
@@ -529,7 +552,10 @@ indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
       item = __shfl_sync(0xffffffffu, item, 0);
       const int b_now = __shfl_sync(0xffffffffu, bq, 0);
       if (item < 0) break;
-      const int32_t chunk = item - prefix[b_now];
+      const int32_t sidx = item - prefix[b_now];
+      const int32_t chunk = MODE == kPSample
+                                ? (int32_t)psample_chunk(sidx, prefix[b_now + 1] - prefix[b_now], bmin[b_now])
+                                : sidx;
       const int64_t t0 = (int64_t)b_now * QB;           // first query of the block (chunk-local)
       const int64_t s0 = (int64_t)chunk * kItemRows;
       const int rs = (int)(issued % kPRing);
@@ -548,16 +574,23 @@ indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
         const float4* wsrc = reinterpret_cast<const float4*>(a.w + (a.t_begin + t0) * HI);
         reinterpret_cast<float4*>(mt.w)[lane] =
             lane * 4 < nq * HI ? __ldg(wsrc + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-        if (lane < QB) mt.nel[lane] = lane < nq ? (int32_t)eligible(a, a.t_begin + t0 + lane) : 0;
+        if (lane < QB) {
+          mt.nel[lane] = lane < nq ? (int32_t)eligible(a, a.t_begin + t0 + lane) : 0;
+          mt.tau[lane] = MODE == kPFused && lane < nq ? __ldg(a.tau + t0 + lane) : 0u;
+        }
         bq_meta = b_now;
       } else {
         const BlockMeta& pm = ring[(issued - 1) % kPRing];
         reinterpret_cast<float4*>(mt.w)[lane] = reinterpret_cast<const float4*>(pm.w)[lane];
-        if (lane < QB) mt.nel[lane] = pm.nel[lane];
+        if (lane < QB) {
+          mt.nel[lane] = pm.nel[lane];
+          mt.tau[lane] = pm.tau[lane];
+        }
       }
       if (lane == 0) {
         mt.b = b_now;
         mt.chunk = chunk;
+        mt.sidx = sidx;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ring_full[rs]));   // releases the lanes' writes (after the warp sync)
@@ -674,7 +707,8 @@ indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
       {
         const int64_t s = s0 + h * kTileRows + row;
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * 256 + h * 128;
-#pragma unroll 2
+        uint32_t keys[QB];   // this thread's key for each query of the block
+#pragma unroll
         for (int c = 0; c < 4; ++c) {   // 32 (query, head) columns at a time
           uint32_t r0[16], r1[16];
           tc::tmem_ld16(taddr + c * 32, r0);
@@ -696,14 +730,38 @@ indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
           }
 #pragma unroll
           for (int qq = 0; qq < qpc; ++qq) {
-            const int q = c * qpc + qq;
             float sc = 0.f;
 #pragma unroll
             for (int hh = 0; hh < HI; ++hh) sc = fmaf(wq[qq * HI + hh], x[qq * HI + hh], sc);
-            const bool valid = s < mt.nel[q];
-            const uint32_t key = score_key(sc);
-            const int64_t tl = t0 + q;
-            if (valid) a.keys_out[tl * a.key_stride + s] = key;
+            keys[c * qpc + qq] = score_key(sc);
+          }
+        }
+        if (MODE == kPSample) {
+          // the sampled chunks are readable by every query of the block
+          const int64_t col = (int64_t)mt.sidx * kItemRows + h * kTileRows + row;
+#pragma unroll
+          for (int q = 0; q < QB; ++q)
+            if (t0 + q < T) a.psample[(t0 + q) * kPSampleKeys + col] = keys[q];
+        } else {
+          // candidates: one ballot per query; lane q reserves the warp's slots
+          // for query q, so that all the block's reservations are one round trip
+          uint32_t mym = 0u;
+#pragma unroll
+          for (int q = 0; q < QB; ++q) {
+            const int32_t nq = mt.nel[q];
+            const uint32_t m = __ballot_sync(0xffffffffu, s < nq && nq > a.skip_le && keys[q] >= mt.tau[q]);
+            if (lane == q) mym = m;
+          }
+          const uint32_t mybase = mym ? atomicAdd(a.cand_count + t0 + lane, (uint32_t)__popc(mym)) : 0u;
+#pragma unroll
+          for (int q = 0; q < QB; ++q) {
+            const uint32_t m = __shfl_sync(0xffffffffu, mym, q);
+            const uint32_t b0 = __shfl_sync(0xffffffffu, mybase, q);
+            if ((m >> lane) & 1u) {
+              const uint32_t slot = b0 + (uint32_t)__popc(m & ((1u << lane) - 1u));
+              if (slot < (uint64_t)a.cand_cap)
+                a.cand[(t0 + q) * a.cand_cap + slot] = make_uint2(keys[q], (uint32_t)s);
+            }
           }
         }
       }
@@ -734,7 +792,7 @@ bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count) {
 }
 
 bool tc_indexer_prefill_supported(const IndexerArgs& a, int64_t t_count) {
-  if (a.tau != nullptr) return false;   // stores every key (many-query mode)
+  if (a.tau == nullptr || a.psample == nullptr || a.fp4) return false;   // the sampled fused selection
   if (a.seq_id != nullptr || a.c_I != 64 || a.work == nullptr) return false;
   if (a.H_I != 4 && a.H_I != 8 && a.H_I != 16) return false;
   // the producer reads a block's 128 head weights as 32 aligned float4
@@ -747,7 +805,8 @@ bool tc_indexer_prefill_supported(const IndexerArgs& a, int64_t t_count) {
   return true;
 }
 
-cudaError_t launch_indexer_scores_tc_prefill(const Launch& L, const IndexerArgs& a, int64_t t_count) {
+cudaError_t launch_indexer_scores_tc_prefill(const Launch& L, const IndexerArgs& a, int64_t t_count,
+                                             bool sample) {
   CUtensorMap tk, tq;
   const uint32_t box_rows = a.keys.page_table == nullptr ? kItemRows : kBoxRows;
   if (!make_tmap_bf16_2d(&tk, a.keys.data, 64, (uint64_t)a.keys.n_rows, 64, 64, box_rows))
@@ -762,16 +821,19 @@ cudaError_t launch_indexer_scores_tc_prefill(const Launch& L, const IndexerArgs&
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int smem = kPStages * kPStageBytes + 1024;
   L.begin(kKernelIndexerScore);
-#define CSA_PREFILL_CASE(H_)                                                                      \
-  if (a.H_I == H_) {                                                                               \
-    cudaFuncSetAttribute(indexer_score_tc_prefill_kernel<H_>,                                      \
+#define CSA_PREFILL_CASE(H_, M_)                                                                   \
+  if (a.H_I == H_ && (M_ == kPSample) == sample) {                                                 \
+    cudaFuncSetAttribute(indexer_score_tc_prefill_kernel<H_, M_>,                                  \
                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                       \
-    prefer_max_shared(indexer_score_tc_prefill_kernel<H_>);                                        \
-    indexer_score_tc_prefill_kernel<H_><<<(unsigned)sms, kPThreads, smem, L.stream>>>(tk, tq, p);  \
+    prefer_max_shared(indexer_score_tc_prefill_kernel<H_, M_>);                                    \
+    indexer_score_tc_prefill_kernel<H_, M_><<<(unsigned)sms, kPThreads, smem, L.stream>>>(tk, tq, p); \
   }
-  CSA_PREFILL_CASE(4)
-  CSA_PREFILL_CASE(8)
-  CSA_PREFILL_CASE(16)
+  CSA_PREFILL_CASE(4, kPSample)
+  CSA_PREFILL_CASE(8, kPSample)
+  CSA_PREFILL_CASE(16, kPSample)
+  CSA_PREFILL_CASE(4, kPFused)
+  CSA_PREFILL_CASE(8, kPFused)
+  CSA_PREFILL_CASE(16, kPFused)
 #undef CSA_PREFILL_CASE
   return L.end(kKernelIndexerScore);
 }

@@ -72,6 +72,10 @@ cudaError_t launch_norm_rope(const Launch& L, const NormRopeArgs& a);
 constexpr int64_t kMaxSelectEntries = int64_t(1) << 19;
 constexpr int64_t kFusedMaxQueries = 2048;
 constexpr int64_t kRadixSelectMaxEntries = 48 * 1024;
+// Many-query mode (more than kFusedMaxQueries queries per call): one warp per
+// query in the threshold and finish passes, whose selection bitmaps bound the
+// entries per query.
+constexpr int64_t kManyMaxEntries = 48 * 1024;
 
 // Lightning-indexer scores of every eligible entry for every query of one
 // chunk of queries: in many-query mode written as order-preserving keys to
@@ -98,6 +102,12 @@ struct IndexerArgs {
   int64_t cand_cap = 0;
   int64_t skip_le = 0;               // queries with at most this many eligible entries are
                                      // not scored (they select all of them)
+  // many-query (prefill) selection: the tcgen05 scorer's sample pass writes
+  // each query's sampled keys here ([T_chunk, kPSampleKeys]); queries whose
+  // candidate count misses [top_k, cand_cap] are listed for the exact fallback
+  uint32_t* psample = nullptr;
+  uint32_t* fb_list = nullptr;       // [T_chunk] chunk-local query ids
+  uint32_t* fb_count = nullptr;      // zeroed by the threshold pass
   WsHeader* err;
   // 4-bit mode (fp4 = 1): q_idx is quantized to E2M1 codes + scale bytes in
   // the scorer; keys.data holds rows of c_I/2 code bytes and k_scales rows of
@@ -106,6 +116,24 @@ struct IndexerArgs {
   const uint8_t* k_scales = nullptr;
 };
 cudaError_t launch_indexer_scores(const Launch& L, const IndexerArgs& a, int64_t t_count);
+
+// Many-query sampling: a block of 128 / H_I consecutive queries (the tcgen05
+// scorer's block) shares kPSampleChunks whole 256-key chunks spread evenly
+// over the entries every query of the block can read; a query's sample is
+// those chunks' keys.  Blocks whose queries all keep every key as a candidate
+// (2 n <= cand_cap) or select every entry (n <= skip_le) take no sample.
+constexpr int kPSampleChunks = 4;
+constexpr int kPSampleKeys = kPSampleChunks * 256;
+__host__ __device__ inline int psample_chunks(int64_t nmin, int64_t nmax, int64_t cand_cap,
+                                              int64_t skip_le) {
+  if (nmax <= skip_le || 2 * nmax <= cand_cap) return 0;
+  const int64_t c = nmin / 256;
+  return c < kPSampleChunks ? (int)c : kPSampleChunks;
+}
+// The i-th of sc sampled chunks of a block whose queries all read nmin entries.
+__host__ __device__ inline int64_t psample_chunk(int i, int sc, int64_t nmin) {
+  return ((2 * (int64_t)i + 1) * (nmin / 256)) / (2 * (int64_t)sc);
+}
 // Fused-selection epilogue of the scorers, one warp at a time: a batch of U
 // keys per lane (entry ids alongside) whose `pass` flags mark the candidates.
 // issue() takes the warp's ballots and reserves slots with one atomic on the
@@ -153,9 +181,11 @@ struct CandidateBatch {
 bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count);
 cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int64_t t_count);
 // tcgen05 many-query path: all queries on one sequence (seq_id null), c_I = 64,
-// H_I in {4, 8, 16}; blocks of 128 / H_I queries share each key tile
+// H_I in {4, 8, 16}; blocks of 128 / H_I queries share each key tile.  Its
+// sample pass (sample = true) writes a.psample, its fused pass candidates.
 bool tc_indexer_prefill_supported(const IndexerArgs& a, int64_t t_count);
-cudaError_t launch_indexer_scores_tc_prefill(const Launch& L, const IndexerArgs& a, int64_t t_count);
+cudaError_t launch_indexer_scores_tc_prefill(const Launch& L, const IndexerArgs& a, int64_t t_count,
+                                             bool sample);
 // 4-bit scorer (E2M1 codes with one scale byte per 32 elements): see indexer_fp4.cu
 cudaError_t launch_indexer_scores_fp4(const Launch& L, const IndexerArgs& a, int64_t t_count);
 // [n_blocks * 32] bf16 -> n_blocks * 16 code bytes + n_blocks scale bytes
@@ -189,6 +219,17 @@ cudaError_t launch_topk_select(const Launch& L, const SelectArgs& a, int64_t t_c
 cudaError_t launch_topk_sample(const Launch& L, const IndexerArgs& a, int top_k, int64_t t_count);
 cudaError_t launch_topk_finish(const Launch& L, const IndexerArgs& a, int top_k, int32_t* idx_out,
                                int32_t* count_out, float* score_out, int64_t t_count);
+// Many-query (prefill) selection, one warp per query, after the tcgen05
+// scorer's sample pass and around its fused pass (fb_list / fb_count /
+// psample set):
+//   launch_topk_threshold_many: tau from the sampled keys; zeroes the counts,
+//     the fallback list and the work counter;
+//   launch_topk_finish_many: the exact top-k among the candidates, then the
+//     recompute of the listed queries whose count missed [top_k, cand_cap].
+bool topk_many_supported(const IndexerArgs& a);
+cudaError_t launch_topk_threshold_many(const Launch& L, const IndexerArgs& a, int top_k, int64_t t_count);
+cudaError_t launch_topk_finish_many(const Launch& L, const IndexerArgs& a, int top_k, int32_t* idx_out,
+                                    int32_t* count_out, float* score_out, int64_t t_count);
 
 // Attention over a virtual row list per query: its selected / eligible
 // compressed entries followed by its window rows.

@@ -335,7 +335,9 @@ struct FinishArgs {
   int32_t* idx_out;
   int32_t* count_out;
   float* score_out;
-  int stage_cap;   // candidates that fit the shared-memory staging area
+  int stage_cap;                   // candidates that fit the shared-memory staging area
+  const uint32_t* list = nullptr;  // with list: the queries list[0 .. *list_count) only,
+  const uint32_t* list_count = nullptr;   // each CTA taking every gridDim.x-th
 };
 
 // Dynamic shared memory: sel [Wmax], tie [Wmax] (Wmax = ceil(max_entries/32)
@@ -355,350 +357,675 @@ __global__ void __launch_bounds__(kThreads) topk_finish_kernel(IndexerArgs a, Fi
 
   pdl_wait();      // the scorer's candidate lists are complete
   pdl_trigger();
-  const int64_t tl = blockIdx.x;
+  auto finish_query = [&](const int64_t tl) {
+    const int64_t t = a.t_begin + tl;
+    const int64_t n = eligible_of(a, t);
+    const int k = f.top_k;
+    int32_t* idx = f.idx_out + t * k;
+    float* sco = f.score_out ? f.score_out + t * k : nullptr;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint2* cand = a.cand + tl * a.cand_cap;
+    const int64_t c_all = (int64_t)a.cand_count[tl];
+
+    if (n <= k) {
+      // every eligible entry; when scores are asked for, the scorer listed all
+      // of them (tau = 0, no skipping)
+      for (int64_t j = tid; j < k; j += kThreads) {
+        idx[j] = j < n ? (int32_t)j : -1;
+        if (sco && j >= n) sco[j] = -INFINITY;
+      }
+      if (sco) {
+        const int64_t c = c_all < a.cand_cap ? c_all : a.cand_cap;
+        for (int64_t i = tid; i < c; i += kThreads) {
+          const uint2 e = cand[i];
+          if ((int64_t)e.y < n) sco[e.y] = key_score(e.x);
+        }
+      }
+      if (tid == 0) f.count_out[t] = (int32_t)n;
+      return;
+    }
+
+    const int W = (int)((n + 31) >> 5);
+    const int Wmax = (int)((((a.max_entries + 31) >> 5) + 3) & ~int64_t(3));   // keeps q 16-byte aligned
+    uint32_t* selb = fsm;
+    uint32_t* tieb = fsm + Wmax;
+    uint2* stage = reinterpret_cast<uint2*>(tieb + Wmax);
+    uint32_t* cand_key = reinterpret_cast<uint32_t*>(stage);
+    int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_key + kCandSmem);
+    float* qs = reinterpret_cast<float*>(stage + f.stage_cap);
+    float* ws = qs + a.H_I * CI;
+    for (int w = tid; w < W; w += kThreads) {
+      selb[w] = 0u;
+      tieb[w] = 0u;
+    }
+    bool consistent = true;
+    int need;   // copies of the k-th largest key still to take, lowest index first
+
+    if (c_all >= k && c_all <= a.cand_cap) {
+      // ------------------------------------------------ select among candidates
+      const int c = (int)c_all;
+      // one pass over the list in global memory: staged in shared memory when
+      // it fits (every later pass then stays on chip), and its key range
+      const uint2* src = cand;
+      uint32_t kmin = 0xffffffffu, kmax = 0u;
+      if (c <= f.stage_cap) {
+        // pairs of candidates as 16-byte vectors, four vectors of loads in
+        // flight per thread before any is stored
+        const uint4* g4 = reinterpret_cast<const uint4*>(cand);   // rows of cand_cap pairs: 16-byte aligned
+        uint4* s4 = reinterpret_cast<uint4*>(stage);
+        const int nv = (c + 1) >> 1;
+        for (int i0 = tid; i0 < nv; i0 += 4 * kThreads) {
+          uint4 v[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (i0 + u * kThreads < nv) v[u] = __ldcs(g4 + i0 + u * kThreads);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * kThreads;
+            if (i < nv) {
+              s4[i] = v[u];
+              kmin = min(kmin, v[u].x);
+              kmax = max(kmax, v[u].x);
+              if (2 * i + 1 < c) {
+                kmin = min(kmin, v[u].z);
+                kmax = max(kmax, v[u].z);
+              }
+            }
+          }
+        }
+        src = stage;
+      } else {
+        for (int i = tid; i < c; i += kThreads) {
+          const uint32_t key = cand[i].x;
+          kmin = min(kmin, key);
+          kmax = max(kmax, key);
+        }
+      }
+      for (int b = tid; b < kHist; b += kThreads) hist[b] = 0;
+      if (tid == 0) s_listn = 0;
+      kmin = __reduce_min_sync(0xffffffffu, kmin);
+      kmax = __reduce_max_sync(0xffffffffu, kmax);
+      if (lane == 0) {
+        s_min[warp] = kmin;
+        s_max[warp] = kmax;
+      }
+      __syncthreads();
+      kmin = __reduce_min_sync(0xffffffffu, lane < kThreads / 32 ? s_min[lane] : 0xffffffffu);
+      kmax = __reduce_max_sync(0xffffffffu, lane < kThreads / 32 ? s_max[lane] : 0u);
+      // the candidates' common leading bits are fixed; the next 12 bits are a
+      // digit (widened downwards to at least 512 bins, whose upper bits are then
+      // fixed too)
+      const int cpl = __clz(kmin ^ kmax);   // 32 when all candidates are equal
+      uint32_t mask = cpl >= 32 ? 0xffffffffu : ~(0xffffffffu >> cpl);
+      uint32_t prefix = kmin & mask;
+      need = k;
+      int shift = 32 - cpl;
+      if (shift > 0) {
+        const int lo = shift > 12 ? shift - 12 : 0;
+        const int dig = shift - lo >= 9 ? shift - lo : 9;
+        const uint32_t dmask = (1u << dig) - 1u;
+        for (int i = tid; i < c; i += kThreads) atomicAdd(&hist[(src[i].x >> lo) & dmask], 1);
+        __syncthreads();
+        consistent &= sel::find_bin<kThreads>(hist, 1 << dig, need, warp_sums, &s_bin, &s_above, &s_ok);
+        const uint32_t bsel = s_bin;
+        const int in_bin = hist[bsel];
+        need -= s_above;
+        __syncthreads();   // the bins are read: hist becomes the threshold bin's list
+        uint2* list = reinterpret_cast<uint2*>(hist);
+        // keys above the threshold bin are selected; the bin's keys are listed
+        // when few enough to rank directly
+        const bool rank_list = in_bin <= kRankList;
+        for (int i = tid; i < c; i += kThreads) {
+          const uint2 e = src[i];
+          if ((int64_t)e.y >= n) continue;   // never listed; kept out of the bitmaps
+          const uint32_t dgt = (e.x >> lo) & dmask;
+          if (dgt > bsel) {
+            atomicOr(&selb[e.y >> 5], 1u << (e.y & 31));
+          } else if (dgt == bsel && rank_list) {
+            const int q = atomicAdd(&s_listn, 1);
+            if (q < kRankList) list[q] = e;
+          }
+        }
+        __syncthreads();
+        if (rank_list) {
+          // an entry of the bin is selected iff fewer than `need` entries of the
+          // bin come before it in (key descending, index ascending) order: this
+          // also settles ties at the k-th key by the lower index
+          const int mb = s_listn < kRankList ? s_listn : kRankList;
+          for (int q = tid; q < mb; q += kThreads) {
+            const uint2 e = list[q];
+            int before = 0;
+            for (int j = 0; j < mb; ++j) {
+              const uint2 o = list[j];
+              before += (o.x > e.x) || (o.x == e.x && o.y < e.y);
+            }
+            if (before < need) atomicOr(&selb[e.y >> 5], 1u << (e.y & 31));
+          }
+          need = 0;
+        } else {
+          // a crowded bin: further 11-bit digits over the candidates, then the
+          // k-th key's copies go to the lowest indices
+          prefix |= bsel << lo;
+          mask |= dmask << lo;
+          shift = lo;
+#pragma unroll 1
+          while (shift > 0) {
+            const int lo2 = shift > 11 ? shift - 11 : 0;
+            const int dig2 = shift - lo2 >= 9 ? shift - lo2 : 9;
+            const uint32_t dm2 = (1u << dig2) - 1u;
+            for (int b = tid; b < (1 << dig2); b += kThreads) hist[b] = 0;
+            __syncthreads();
+            for (int i = tid; i < c; i += kThreads) {
+              const uint32_t key = src[i].x;
+              if ((key & mask) == prefix) atomicAdd(&hist[(key >> lo2) & dm2], 1);
+            }
+            __syncthreads();
+            consistent &= sel::find_bin<kThreads>(hist, 1 << dig2, need, warp_sums, &s_bin, &s_above, &s_ok);
+            prefix |= s_bin << lo2;
+            mask |= dm2 << lo2;
+            need -= s_above;
+            shift = lo2;
+            __syncthreads();
+          }
+          for (int i = tid; i < c; i += kThreads) {
+            const uint2 e = src[i];
+            if ((int64_t)e.y >= n) continue;
+            if (e.x > prefix) atomicOr(&selb[e.y >> 5], 1u << (e.y & 31));
+            else if (e.x == prefix) atomicOr(&tieb[e.y >> 5], 1u << (e.y & 31));
+          }
+        }
+      } else {
+        // every candidate has the same key: the lowest indices win
+        for (int i = tid; i < c; i += kThreads) {
+          const uint2 e = src[i];
+          if ((int64_t)e.y < n) atomicOr(&tieb[e.y >> 5], 1u << (e.y & 31));
+        }
+      }
+      __syncthreads();
+    } else {
+      // ------------------------------------------------ fallback: recompute
+      load_query<CI>(a, t, qs, ws);
+      __syncthreads();
+      const int32_t seq = a.seq_id ? __ldg(a.seq_id + t) : 0;
+      auto key_at = [&](int64_t j) -> uint32_t {
+        return recompute_key<CI>(a, qs, ws, seq, j, (int32_t)t);
+      };
+      for (int b = tid; b < kHist; b += kThreads) hist[b] = 0;
+      __syncthreads();
+      for (int64_t j = tid; j < n; j += kThreads) atomicAdd(&hist[key_at(j) >> 20], 1);
+      __syncthreads();
+      consistent &= sel::find_bin<kThreads>(hist, kHist, k, warp_sums, &s_bin, &s_above, &s_ok);
+      uint32_t prefix = s_bin << 20, mask = 0xfff00000u;
+      need = k - s_above;
+      int cnt = hist[s_bin];
+      int shift = 20;
+      __syncthreads();
+      // refine the prefix by one 10-bit digit with a recompute pass
+      auto refine = [&]() {
+        shift -= 10;
+        for (int b = tid; b < 1024; b += kThreads) hist[b] = 0;
+        __syncthreads();
+        for (int64_t j = tid; j < n; j += kThreads) {
+          const uint32_t key = key_at(j);
+          if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 1023u], 1);
+        }
+        __syncthreads();
+        consistent &= sel::find_bin<kThreads>(hist, 1024, need, warp_sums, &s_bin, &s_above, &s_ok);
+        prefix |= s_bin << shift;
+        mask |= 1023u << shift;
+        need -= s_above;
+        cnt = hist[s_bin];
+        __syncthreads();
+      };
+      while (cnt > kCandSmem && shift > 0) refine();
+      constexpr int kWarpCap = kCandSmem / (kThreads / 32);
+      // one pass per warp and word: keys above the prefix go to the bitmap;
+      // keys equal to it are candidates in the warp's slice (or ties when the
+      // prefix is complete); a slice overflow refines and repeats the pass
+      for (;;) {
+        if (tid == 0) s_overflow = 0;
+        __syncthreads();
+        int wcnt = 0;
+        for (int w = warp; w < W; w += kThreads / 32) {
+          const int64_t j = (int64_t)w * 32 + lane;
+          const uint32_t key = j < n ? key_at(j) : 0u;
+          const uint32_t mk = key & mask;
+          const bool gt = j < n && mk > prefix;
+          const bool eq = j < n && mk == prefix;
+          const uint32_t bg = __ballot_sync(0xffffffffu, gt);
+          const uint32_t be = __ballot_sync(0xffffffffu, eq);
+          if (lane == 0) {
+            selb[w] = bg;
+            tieb[w] = shift == 0 ? be : 0u;
+          }
+          if (shift > 0 && be) {
+            if (eq) {
+              const int p = wcnt + __popc(be & ((1u << lane) - 1u));
+              if (p < kWarpCap) {
+                cand_key[warp * kWarpCap + p] = key;
+                cand_idx[warp * kWarpCap + p] = (int32_t)j;
+              }
+            }
+            wcnt += __popc(be);
+          }
+        }
+        if (lane == 0) {
+          s_wcnt[warp] = wcnt;
+          if (wcnt > kWarpCap) s_overflow = 1;
+        }
+        __syncthreads();
+        if (!s_overflow || shift == 0) break;
+        refine();
+      }
+      if (shift > 0) {
+        auto cand_ok = [&](int cc) { return (cc % kWarpCap) < s_wcnt[cc / kWarpCap]; };
+        int nc = 0;
+        for (int w = 0; w < kThreads / 32; ++w) nc += min(s_wcnt[w], kWarpCap);
+        if (need >= nc) {
+          for (int cc = tid; cc < kCandSmem; cc += kThreads)
+            if (cand_ok(cc)) atomicOr(&selb[cand_idx[cc] >> 5], 1u << (cand_idx[cc] & 31));
+          need = 0;
+        } else {
+          // radix select of the need-th largest candidate over the low bits
+          uint32_t cp = prefix, cm = mask;
+          while (shift > 0) {
+            const int dig = shift >= 10 ? 10 : shift;
+            shift -= dig;
+            const uint32_t dm = (1u << dig) - 1u;
+            for (int b = tid; b < 1024; b += kThreads) hist[b] = 0;
+            __syncthreads();
+            for (int cc = tid; cc < kCandSmem; cc += kThreads)
+              if (cand_ok(cc) && (cand_key[cc] & cm) == cp) atomicAdd(&hist[(cand_key[cc] >> shift) & dm], 1);
+            __syncthreads();
+            consistent &= sel::find_bin<kThreads>(hist, 1024, need, warp_sums, &s_bin, &s_above, &s_ok);
+            cp |= s_bin << shift;
+            cm |= dm << shift;
+            need -= s_above;
+            __syncthreads();
+          }
+          for (int cc = tid; cc < kCandSmem; cc += kThreads) {
+            if (!cand_ok(cc)) continue;
+            const uint32_t key = cand_key[cc];
+            const int j = cand_idx[cc];
+            if (key > cp) atomicOr(&selb[j >> 5], 1u << (j & 31));
+            else if (key == cp) atomicOr(&tieb[j >> 5], 1u << (j & 31));
+          }
+        }
+      }
+      __syncthreads();
+      sel::take_lowest_ties<kThreads>(selb, tieb, W, need, warp_sums);
+      sel::compact_ascending<kThreads>(selb, W, k, idx, warp_sums, [&](int o, int64_t j) {
+        if (sco) sco[o] = key_score(key_at(j));
+      });
+      if (tid == 0) {
+        f.count_out[t] = k;
+        if (!consistent) report(a.err, kErrSelect, (int32_t)t, k);
+      }
+      return;
+    }
+
+    // ---------------------------------------------------- candidates: finish
+    if (need > 0) sel::take_lowest_ties<kThreads>(selb, tieb, W, need, warp_sums);
+    sel::compact_ascending<kThreads>(selb, W, k, idx, warp_sums, [](int, int64_t) {});
+    if (sco) {
+      // output position of a selected entry j = set bits of sel below j:
+      // prefix counts per 1024 entries (32 words), then the words in between
+      __syncthreads();
+      int* gpre = hist;   // (W + 31) / 32 <= 512 groups
+      const int G = (W + 31) >> 5;
+      int cg = 0;
+      if (tid < G)
+        for (int w = tid * 32; w < min(W, tid * 32 + 32); ++w) cg += __popc(selb[w]);
+      int tot;
+      const int before = sel::block_exclusive_scan<kThreads>(cg, warp_sums, tot);
+      if (tid < G) gpre[tid] = before;
+      __syncthreads();
+      const int c = (int)c_all;
+      const uint2* src = c <= f.stage_cap ? stage : cand;
+      for (int i = tid; i < c; i += kThreads) {
+        const uint2 e = src[i];
+        const uint32_t j = e.y;
+        if ((int64_t)j >= n || !((selb[j >> 5] >> (j & 31)) & 1u)) continue;
+        int pos = gpre[j >> 10];
+        for (uint32_t w = (j >> 10) << 5; w < (j >> 5); ++w) pos += __popc(selb[w]);
+        pos += __popc(selb[j >> 5] & ((1u << (j & 31)) - 1u));
+        if (pos < k) sco[pos] = key_score(e.x);
+      }
+    }
+    if (tid == 0) {
+      f.count_out[t] = k;
+      if (!consistent) report(a.err, kErrSelect, (int32_t)t, k);
+    }
+  };
+  if (f.list == nullptr) {
+    finish_query(blockIdx.x);
+    return;
+  }
+  const int64_t nl = (int64_t)*f.list_count;
+  for (int64_t i = blockIdx.x; i < nl; i += gridDim.x) {
+    __syncthreads();   // the previous query's shared memory is no longer read
+    finish_query((int64_t)f.list[i]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Many-query mode (prefill): one warp per query in both passes below, so that
+// tens of queries share an SM and no pass waits on a block-wide barrier.
+// ---------------------------------------------------------------------------
+// Warp-level helpers.  Histogram bins are owned from the top, nbins / 32 per
+// lane (nbins a multiple of 32).
+__device__ __forceinline__ int warp_exclusive_scan(int v, int& total) {
+  const int lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  total = __shfl_sync(0xffffffffu, x, 31);
+  return x - v;
+}
+
+// Bin holding the need-th largest counted element: false (bin 0, above 0)
+// when the histogram holds fewer than `need`.
+__device__ __forceinline__ bool warp_find_bin(const int* hist, int nbins, int need, uint32_t& bin,
+                                              int& above) {
+  const int lane = threadIdx.x & 31, per = nbins >> 5;
+  int c = 0;
+  for (int r = 0; r < per; ++r) c += hist[nbins - 1 - (lane * per + r)];
+  int tot;
+  int before = warp_exclusive_scan(c, tot);
+  uint32_t my_bin = 0u;
+  int my_above = 0;
+  const bool mine = before < need && before + c >= need;
+  if (mine) {
+    for (int r = 0; r < per; ++r) {
+      const int b = nbins - 1 - (lane * per + r);
+      const int h = hist[b];
+      if (before + h >= need) {
+        my_bin = (uint32_t)b;
+        my_above = before;
+        break;
+      }
+      before += h;
+    }
+  }
+  const uint32_t who = __ballot_sync(0xffffffffu, mine);
+  if (who == 0u) {
+    bin = 0u;
+    above = 0;
+    return false;
+  }
+  const int src = __ffs(who) - 1;
+  bin = __shfl_sync(0xffffffffu, my_bin, src);
+  above = __shfl_sync(0xffffffffu, my_above, src);
+  return true;
+}
+
+// The first `need` set bits of tie[0 .. W) (index order) join sel.
+__device__ __forceinline__ void warp_take_lowest_ties(uint32_t* sel, const uint32_t* tie, int W, int need) {
+  const int lane = threadIdx.x & 31;
+  const int wpt = (W + 31) >> 5, w0 = lane * wpt, w1 = min(W, w0 + wpt);
+  int c = 0;
+  for (int w = w0; w < w1; ++w) c += __popc(tie[w]);
+  int tot;
+  int before = warp_exclusive_scan(c, tot);
+  for (int w = w0; w < w1; ++w) {
+    uint32_t x = tie[w];
+    const int pc = __popc(x);
+    int take = need - before;
+    take = take < 0 ? 0 : (take > pc ? pc : take);
+    uint32_t kept = 0u;
+    for (int i = 0; i < take; ++i) {
+      const uint32_t low = x & (0u - x);
+      kept |= low;
+      x ^= low;
+    }
+    sel[w] |= kept;
+    before += pc;
+  }
+  __syncwarp();
+}
+
+// Threshold pass: tau of each query from the keys the scorer's sample pass
+// left in psample (the same rank rule and two 11-bit radix levels as the
+// few-query sample pass); also zeroes the candidate counts, the fallback list
+// and the work counter of the scoring pass that follows.
+constexpr int kTWarps = 4;
+__global__ void __launch_bounds__(kTWarps * 32) topk_threshold_many_kernel(IndexerArgs a, int top_k,
+                                                                        int64_t t_count) {
+  __shared__ int hist_all[kTWarps][2048];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *a.fb_count = 0u;
+    *a.work = 0u;
+  }
+  const int64_t tl = (int64_t)blockIdx.x * kTWarps + warp;
+  if (tl >= t_count) return;
+  const int64_t t = a.t_begin + tl;
+  if (lane == 0) a.cand_count[tl] = 0u;
+  const int64_t n = eligible_of(a, t);
+  uint32_t tau = 0u;
+  if (n > a.skip_le && 2 * n > a.cand_cap) {
+    // the block's sampled chunks, by the scorer's rule
+    const int64_t QB = 128 / a.H_I;
+    const int64_t b0 = tl / QB * QB, b1 = b0 + QB < t_count ? b0 + QB : t_count;
+    int64_t nmin = INT64_MAX, nmax = 0;
+    for (int64_t u = b0 + lane; u < b1; u += 32) {
+      const int64_t nu = eligible_of(a, a.t_begin + u);
+      nmin = nu < nmin ? nu : nmin;
+      nmax = nu > nmax ? nu : nmax;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const int64_t x = __shfl_xor_sync(0xffffffffu, nmin, o), y = __shfl_xor_sync(0xffffffffu, nmax, o);
+      nmin = x < nmin ? x : nmin;
+      nmax = y > nmax ? y : nmax;
+    }
+    const int ns = 256 * psample_chunks(nmin, nmax, a.cand_cap, a.skip_le);
+    const double mu = (double)ns * (double)top_k / (double)n;
+    const int64_t r = (int64_t)ceil(mu + 6.0 * sqrt(mu) + 8.0);
+    if (ns > 0 && r < ns) {
+      uint32_t kv[kPSampleKeys / 32];
+      const uint32_t* sk = a.psample + tl * kPSampleKeys;
+#pragma unroll
+      for (int i = 0; i < kPSampleKeys / 32; ++i) kv[i] = 32 * i + lane < ns ? __ldcs(sk + 32 * i + lane) : 0u;
+      int* hist = hist_all[warp];
+      uint32_t prefix = 0u;
+      int need = (int)r;
+#pragma unroll 1
+      for (int level = 0; level < 2; ++level) {
+        const int lo = level == 0 ? 21 : 10;
+        for (int b = lane; b < 2048; b += 32) hist[b] = 0;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kPSampleKeys / 32; ++i)
+          if (32 * i + lane < ns && (level == 0 || (kv[i] >> 21) == (prefix >> 21)))
+            atomicAdd(&hist[(kv[i] >> lo) & 2047u], 1);
+        __syncwarp();
+        uint32_t bin;
+        int above;
+        warp_find_bin(hist, 2048, need, bin, above);
+        prefix |= bin << lo;
+        need -= above;
+        __syncwarp();
+      }
+      tau = prefix;
+    }
+  }
+  if (lane == 0) const_cast<uint32_t*>(a.tau)[tl] = tau;
+}
+
+// Finish pass: the exact top-k among a query's candidates by one warp, when
+// top_k <= count <= cand_cap; other queries are appended to the fallback
+// list for topk_finish_kernel's recompute.  Shared memory per warp: hist
+// [1024] int, sel / tie bitmaps [Wmax] each, the threshold bin's list
+// [kWList] (key, entry) pairs.
+constexpr int kFWarps = 8;
+constexpr int kWList = 128;
+__host__ __device__ inline int finish_many_words(int64_t max_entries) {
+  return (int)((((max_entries + 31) >> 5) + 1) & ~int64_t(1));   // keeps the list 8-byte aligned
+}
+__global__ void __launch_bounds__(kFWarps * 32) topk_finish_many_kernel(IndexerArgs a, FinishArgs f,
+                                                                     int64_t t_count) {
+  extern __shared__ __align__(16) uint32_t msm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t tl = (int64_t)blockIdx.x * kFWarps + warp;
+  if (tl >= t_count) return;   // no block-wide barrier below
+  const int Wmax = finish_many_words(a.max_entries);
+  uint32_t* my = msm + (size_t)warp * (1024 + 2 * Wmax + 2 * kWList);
+  int* hist = reinterpret_cast<int*>(my);
+  uint32_t* selb = my + 1024;
+  uint32_t* tieb = selb + Wmax;
+  uint2* list = reinterpret_cast<uint2*>(tieb + Wmax);
+
   const int64_t t = a.t_begin + tl;
   const int64_t n = eligible_of(a, t);
   const int k = f.top_k;
   int32_t* idx = f.idx_out + t * k;
   float* sco = f.score_out ? f.score_out + t * k : nullptr;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint2* cand = a.cand + tl * a.cand_cap;
   const int64_t c_all = (int64_t)a.cand_count[tl];
-
   if (n <= k) {
-    // every eligible entry; when scores are asked for, the scorer listed all
-    // of them (tau = 0, no skipping)
-    for (int64_t j = tid; j < k; j += kThreads) {
+    for (int64_t j = lane; j < k; j += 32) {
       idx[j] = j < n ? (int32_t)j : -1;
       if (sco && j >= n) sco[j] = -INFINITY;
     }
     if (sco) {
       const int64_t c = c_all < a.cand_cap ? c_all : a.cand_cap;
-      for (int64_t i = tid; i < c; i += kThreads) {
+      for (int64_t i = lane; i < c; i += 32) {
         const uint2 e = cand[i];
         if ((int64_t)e.y < n) sco[e.y] = key_score(e.x);
       }
     }
-    if (tid == 0) f.count_out[t] = (int32_t)n;
+    if (lane == 0) f.count_out[t] = (int32_t)n;
     return;
   }
-
+  if (c_all < k || c_all > a.cand_cap) {
+    if (lane == 0) a.fb_list[atomicAdd(a.fb_count, 1u)] = (uint32_t)tl;
+    return;
+  }
+  const int c = (int)c_all;
   const int W = (int)((n + 31) >> 5);
-  const int Wmax = (int)((((a.max_entries + 31) >> 5) + 3) & ~int64_t(3));   // keeps q 16-byte aligned
-  uint32_t* selb = fsm;
-  uint32_t* tieb = fsm + Wmax;
-  uint2* stage = reinterpret_cast<uint2*>(tieb + Wmax);
-  uint32_t* cand_key = reinterpret_cast<uint32_t*>(stage);
-  int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_key + kCandSmem);
-  float* qs = reinterpret_cast<float*>(stage + f.stage_cap);
-  float* ws = qs + a.H_I * CI;
-  for (int w = tid; w < W; w += kThreads) {
+  for (int w = lane; w < W; w += 32) {
     selb[w] = 0u;
     tieb[w] = 0u;
   }
-  bool consistent = true;
-  int need;   // copies of the k-th largest key still to take, lowest index first
-
-  if (c_all >= k && c_all <= a.cand_cap) {
-    // ------------------------------------------------ select among candidates
-    const int c = (int)c_all;
-    // one pass over the list in global memory: staged in shared memory when
-    // it fits (every later pass then stays on chip), and its key range
-    const uint2* src = cand;
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-    if (c <= f.stage_cap) {
-      // pairs of candidates as 16-byte vectors, four vectors of loads in
-      // flight per thread before any is stored
-      const uint4* g4 = reinterpret_cast<const uint4*>(cand);   // rows of cand_cap pairs: 16-byte aligned
-      uint4* s4 = reinterpret_cast<uint4*>(stage);
-      const int nv = (c + 1) >> 1;
-      for (int i0 = tid; i0 < nv; i0 += 4 * kThreads) {
-        uint4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (i0 + u * kThreads < nv) v[u] = __ldcs(g4 + i0 + u * kThreads);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = i0 + u * kThreads;
-          if (i < nv) {
-            s4[i] = v[u];
-            kmin = min(kmin, v[u].x);
-            kmax = max(kmax, v[u].x);
-            if (2 * i + 1 < c) {
-              kmin = min(kmin, v[u].z);
-              kmax = max(kmax, v[u].z);
-            }
-          }
-        }
-      }
-      src = stage;
-    } else {
-      for (int i = tid; i < c; i += kThreads) {
-        const uint32_t key = cand[i].x;
-        kmin = min(kmin, key);
-        kmax = max(kmax, key);
-      }
-    }
-    for (int b = tid; b < kHist; b += kThreads) hist[b] = 0;
-    if (tid == 0) s_listn = 0;
-    kmin = __reduce_min_sync(0xffffffffu, kmin);
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
-    if (lane == 0) {
-      s_min[warp] = kmin;
-      s_max[warp] = kmax;
-    }
-    __syncthreads();
-    kmin = __reduce_min_sync(0xffffffffu, lane < kThreads / 32 ? s_min[lane] : 0xffffffffu);
-    kmax = __reduce_max_sync(0xffffffffu, lane < kThreads / 32 ? s_max[lane] : 0u);
-    // the candidates' common leading bits are fixed; the next 12 bits are a
-    // digit (widened downwards to at least 512 bins, whose upper bits are then
-    // fixed too)
-    const int cpl = __clz(kmin ^ kmax);   // 32 when all candidates are equal
-    uint32_t mask = cpl >= 32 ? 0xffffffffu : ~(0xffffffffu >> cpl);
-    uint32_t prefix = kmin & mask;
-    need = k;
-    int shift = 32 - cpl;
-    if (shift > 0) {
-      const int lo = shift > 12 ? shift - 12 : 0;
-      const int dig = shift - lo >= 9 ? shift - lo : 9;
-      const uint32_t dmask = (1u << dig) - 1u;
-      for (int i = tid; i < c; i += kThreads) atomicAdd(&hist[(src[i].x >> lo) & dmask], 1);
-      __syncthreads();
-      consistent &= sel::find_bin<kThreads>(hist, 1 << dig, need, warp_sums, &s_bin, &s_above, &s_ok);
-      const uint32_t bsel = s_bin;
-      const int in_bin = hist[bsel];
-      need -= s_above;
-      __syncthreads();   // the bins are read: hist becomes the threshold bin's list
-      uint2* list = reinterpret_cast<uint2*>(hist);
-      // keys above the threshold bin are selected; the bin's keys are listed
-      // when few enough to rank directly
-      const bool rank_list = in_bin <= kRankList;
-      for (int i = tid; i < c; i += kThreads) {
-        const uint2 e = src[i];
-        if ((int64_t)e.y >= n) continue;   // never listed; kept out of the bitmaps
-        const uint32_t dgt = (e.x >> lo) & dmask;
-        if (dgt > bsel) {
-          atomicOr(&selb[e.y >> 5], 1u << (e.y & 31));
-        } else if (dgt == bsel && rank_list) {
-          const int q = atomicAdd(&s_listn, 1);
-          if (q < kRankList) list[q] = e;
-        }
-      }
-      __syncthreads();
-      if (rank_list) {
-        // an entry of the bin is selected iff fewer than `need` entries of the
-        // bin come before it in (key descending, index ascending) order: this
-        // also settles ties at the k-th key by the lower index
-        const int mb = s_listn < kRankList ? s_listn : kRankList;
-        for (int q = tid; q < mb; q += kThreads) {
-          const uint2 e = list[q];
-          int before = 0;
-          for (int j = 0; j < mb; ++j) {
-            const uint2 o = list[j];
-            before += (o.x > e.x) || (o.x == e.x && o.y < e.y);
-          }
-          if (before < need) atomicOr(&selb[e.y >> 5], 1u << (e.y & 31));
-        }
-        need = 0;
-      } else {
-        // a crowded bin: further 11-bit digits over the candidates, then the
-        // k-th key's copies go to the lowest indices
-        prefix |= bsel << lo;
-        mask |= dmask << lo;
-        shift = lo;
-#pragma unroll 1
-        while (shift > 0) {
-          const int lo2 = shift > 11 ? shift - 11 : 0;
-          const int dig2 = shift - lo2 >= 9 ? shift - lo2 : 9;
-          const uint32_t dm2 = (1u << dig2) - 1u;
-          for (int b = tid; b < (1 << dig2); b += kThreads) hist[b] = 0;
-          __syncthreads();
-          for (int i = tid; i < c; i += kThreads) {
-            const uint32_t key = src[i].x;
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> lo2) & dm2], 1);
-          }
-          __syncthreads();
-          consistent &= sel::find_bin<kThreads>(hist, 1 << dig2, need, warp_sums, &s_bin, &s_above, &s_ok);
-          prefix |= s_bin << lo2;
-          mask |= dm2 << lo2;
-          need -= s_above;
-          shift = lo2;
-          __syncthreads();
-        }
-        for (int i = tid; i < c; i += kThreads) {
-          const uint2 e = src[i];
-          if ((int64_t)e.y >= n) continue;
-          if (e.x > prefix) atomicOr(&selb[e.y >> 5], 1u << (e.y & 31));
-          else if (e.x == prefix) atomicOr(&tieb[e.y >> 5], 1u << (e.y & 31));
-        }
-      }
-    } else {
-      // every candidate has the same key: the lowest indices win
-      for (int i = tid; i < c; i += kThreads) {
-        const uint2 e = src[i];
-        if ((int64_t)e.y < n) atomicOr(&tieb[e.y >> 5], 1u << (e.y & 31));
-      }
-    }
-    __syncthreads();
-  } else {
-    // ------------------------------------------------ fallback: recompute
-    load_query<CI>(a, t, qs, ws);
-    __syncthreads();
-    const int32_t seq = a.seq_id ? __ldg(a.seq_id + t) : 0;
-    auto key_at = [&](int64_t j) -> uint32_t {
-      return recompute_key<CI>(a, qs, ws, seq, j, (int32_t)t);
-    };
-    for (int b = tid; b < kHist; b += kThreads) hist[b] = 0;
-    __syncthreads();
-    for (int64_t j = tid; j < n; j += kThreads) atomicAdd(&hist[key_at(j) >> 20], 1);
-    __syncthreads();
-    consistent &= sel::find_bin<kThreads>(hist, kHist, k, warp_sums, &s_bin, &s_above, &s_ok);
-    uint32_t prefix = s_bin << 20, mask = 0xfff00000u;
-    need = k - s_above;
-    int cnt = hist[s_bin];
-    int shift = 20;
-    __syncthreads();
-    // refine the prefix by one 10-bit digit with a recompute pass
-    auto refine = [&]() {
-      shift -= 10;
-      for (int b = tid; b < 1024; b += kThreads) hist[b] = 0;
-      __syncthreads();
-      for (int64_t j = tid; j < n; j += kThreads) {
-        const uint32_t key = key_at(j);
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 1023u], 1);
-      }
-      __syncthreads();
-      consistent &= sel::find_bin<kThreads>(hist, 1024, need, warp_sums, &s_bin, &s_above, &s_ok);
-      prefix |= s_bin << shift;
-      mask |= 1023u << shift;
-      need -= s_above;
-      cnt = hist[s_bin];
-      __syncthreads();
-    };
-    while (cnt > kCandSmem && shift > 0) refine();
-    constexpr int kWarpCap = kCandSmem / (kThreads / 32);
-    // one pass per warp and word: keys above the prefix go to the bitmap;
-    // keys equal to it are candidates in the warp's slice (or ties when the
-    // prefix is complete); a slice overflow refines and repeats the pass
-    for (;;) {
-      if (tid == 0) s_overflow = 0;
-      __syncthreads();
-      int wcnt = 0;
-      for (int w = warp; w < W; w += kThreads / 32) {
-        const int64_t j = (int64_t)w * 32 + lane;
-        const uint32_t key = j < n ? key_at(j) : 0u;
-        const uint32_t mk = key & mask;
-        const bool gt = j < n && mk > prefix;
-        const bool eq = j < n && mk == prefix;
-        const uint32_t bg = __ballot_sync(0xffffffffu, gt);
-        const uint32_t be = __ballot_sync(0xffffffffu, eq);
-        if (lane == 0) {
-          selb[w] = bg;
-          tieb[w] = shift == 0 ? be : 0u;
-        }
-        if (shift > 0 && be) {
-          if (eq) {
-            const int p = wcnt + __popc(be & ((1u << lane) - 1u));
-            if (p < kWarpCap) {
-              cand_key[warp * kWarpCap + p] = key;
-              cand_idx[warp * kWarpCap + p] = (int32_t)j;
-            }
-          }
-          wcnt += __popc(be);
-        }
-      }
-      if (lane == 0) {
-        s_wcnt[warp] = wcnt;
-        if (wcnt > kWarpCap) s_overflow = 1;
-      }
-      __syncthreads();
-      if (!s_overflow || shift == 0) break;
-      refine();
-    }
-    if (shift > 0) {
-      auto cand_ok = [&](int cc) { return (cc % kWarpCap) < s_wcnt[cc / kWarpCap]; };
-      int nc = 0;
-      for (int w = 0; w < kThreads / 32; ++w) nc += min(s_wcnt[w], kWarpCap);
-      if (need >= nc) {
-        for (int cc = tid; cc < kCandSmem; cc += kThreads)
-          if (cand_ok(cc)) atomicOr(&selb[cand_idx[cc] >> 5], 1u << (cand_idx[cc] & 31));
-        need = 0;
-      } else {
-        // radix select of the need-th largest candidate over the low bits
-        uint32_t cp = prefix, cm = mask;
-        while (shift > 0) {
-          const int dig = shift >= 10 ? 10 : shift;
-          shift -= dig;
-          const uint32_t dm = (1u << dig) - 1u;
-          for (int b = tid; b < 1024; b += kThreads) hist[b] = 0;
-          __syncthreads();
-          for (int cc = tid; cc < kCandSmem; cc += kThreads)
-            if (cand_ok(cc) && (cand_key[cc] & cm) == cp) atomicAdd(&hist[(cand_key[cc] >> shift) & dm], 1);
-          __syncthreads();
-          consistent &= sel::find_bin<kThreads>(hist, 1024, need, warp_sums, &s_bin, &s_above, &s_ok);
-          cp |= s_bin << shift;
-          cm |= dm << shift;
-          need -= s_above;
-          __syncthreads();
-        }
-        for (int cc = tid; cc < kCandSmem; cc += kThreads) {
-          if (!cand_ok(cc)) continue;
-          const uint32_t key = cand_key[cc];
-          const int j = cand_idx[cc];
-          if (key > cp) atomicOr(&selb[j >> 5], 1u << (j & 31));
-          else if (key == cp) atomicOr(&tieb[j >> 5], 1u << (j & 31));
-        }
-      }
-    }
-    __syncthreads();
-    sel::take_lowest_ties<kThreads>(selb, tieb, W, need, warp_sums);
-    sel::compact_ascending<kThreads>(selb, W, k, idx, warp_sums, [&](int o, int64_t j) {
-      if (sco) sco[o] = key_score(key_at(j));
-    });
-    if (tid == 0) {
-      f.count_out[t] = k;
-      if (!consistent) report(a.err, kErrSelect, (int32_t)t, k);
-    }
-    return;
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int i = lane; i < c; i += 32) {
+    const uint32_t key = cand[i].x;
+    kmin = min(kmin, key);
+    kmax = max(kmax, key);
   }
-
-  // ---------------------------------------------------- candidates: finish
-  if (need > 0) sel::take_lowest_ties<kThreads>(selb, tieb, W, need, warp_sums);
-  sel::compact_ascending<kThreads>(selb, W, k, idx, warp_sums, [](int, int64_t) {});
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  __syncwarp();
+  const int cpl = __clz(kmin ^ kmax);   // 32 when all candidates are equal
+  uint32_t mask = cpl >= 32 ? 0xffffffffu : ~(0xffffffffu >> cpl);
+  uint32_t prefix = kmin & mask;
+  int need = k;
+  int shift = 32 - cpl;
+  bool consistent = true;
+  // digits of at most 10 bits below the common prefix until the threshold
+  // bin is small enough to rank directly, or the key is complete
+  while (shift > 0) {
+    const int dig = shift < 10 ? shift : 10;
+    const int lo = shift - dig;
+    const uint32_t dm = (1u << dig) - 1u;
+    const int nb = dig < 5 ? 32 : (1 << dig);
+    for (int b = lane; b < nb; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int i = lane; i < c; i += 32) {
+      const uint32_t key = cand[i].x;
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> lo) & dm], 1);
+    }
+    __syncwarp();
+    uint32_t bin;
+    int above;
+    consistent &= warp_find_bin(hist, nb, need, bin, above);
+    const int in_bin = hist[bin];
+    prefix |= bin << lo;
+    mask |= dm << lo;
+    need -= above;
+    shift = lo;
+    __syncwarp();
+    if (in_bin <= kWList) break;
+  }
+  // keys above the threshold bin are selected; its keys are ties (complete
+  // key) or listed for ranking
+  int listn = 0;
+  for (int i0 = 0; i0 < c; i0 += 32) {
+    const int i = i0 + lane;
+    const uint2 e = i < c ? cand[i] : make_uint2(0u, 0u);
+    const bool valid = i < c && (int64_t)e.y < n;
+    const uint32_t mk = e.x & mask;
+    if (valid && mk > prefix) atomicOr(&selb[e.y >> 5], 1u << (e.y & 31));
+    const bool eq = valid && mk == prefix;
+    if (shift == 0) {
+      if (eq) atomicOr(&tieb[e.y >> 5], 1u << (e.y & 31));
+    } else {
+      const uint32_t be = __ballot_sync(0xffffffffu, eq);
+      const int pos = listn + __popc(be & ((1u << lane) - 1u));
+      if (eq && pos < kWList) list[pos] = e;
+      listn += __popc(be);
+    }
+  }
+  __syncwarp();
+  if (shift > 0) {
+    // an entry of the bin is selected iff fewer than `need` entries of the bin
+    // precede it in (key descending, index ascending) order
+    const int mb = listn < kWList ? listn : kWList;
+    consistent &= listn <= kWList;
+    for (int q = lane; q < mb; q += 32) {
+      const uint2 e = list[q];
+      int before = 0;
+      for (int j = 0; j < mb; ++j) {
+        const uint2 o = list[j];
+        before += (o.x > e.x) || (o.x == e.x && o.y < e.y);
+      }
+      if (before < need) atomicOr(&selb[e.y >> 5], 1u << (e.y & 31));
+    }
+    need = 0;
+  }
+  __syncwarp();
+  if (need > 0) warp_take_lowest_ties(selb, tieb, W, need);
+  // ascending compaction: lane-owned runs of words, then (for the scores)
+  // each word's output offset, kept in the tie bitmap's place
+  const int wpt = (W + 31) >> 5, w0 = lane * wpt, w1 = min(W, w0 + wpt);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(selb[w]);
+  int tot;
+  int o = warp_exclusive_scan(cnt, tot);
+  for (int w = w0; w < w1; ++w) {
+    uint32_t x = selb[w];
+    tieb[w] = (uint32_t)o;
+    while (x) {
+      const int b = __ffs(x) - 1;
+      x &= x - 1;
+      if (o < k) idx[o] = w * 32 + b;
+      ++o;
+    }
+  }
+  __syncwarp();
   if (sco) {
-    // output position of a selected entry j = set bits of sel below j:
-    // prefix counts per 1024 entries (32 words), then the words in between
-    __syncthreads();
-    int* gpre = hist;   // (W + 31) / 32 <= 512 groups
-    const int G = (W + 31) >> 5;
-    int cg = 0;
-    if (tid < G)
-      for (int w = tid * 32; w < min(W, tid * 32 + 32); ++w) cg += __popc(selb[w]);
-    int tot;
-    const int before = sel::block_exclusive_scan<kThreads>(cg, warp_sums, tot);
-    if (tid < G) gpre[tid] = before;
-    __syncthreads();
-    const int c = (int)c_all;
-    const uint2* src = c <= f.stage_cap ? stage : cand;
-    for (int i = tid; i < c; i += kThreads) {
-      const uint2 e = src[i];
+    for (int i = lane; i < c; i += 32) {
+      const uint2 e = cand[i];
       const uint32_t j = e.y;
       if ((int64_t)j >= n || !((selb[j >> 5] >> (j & 31)) & 1u)) continue;
-      int pos = gpre[j >> 10];
-      for (uint32_t w = (j >> 10) << 5; w < (j >> 5); ++w) pos += __popc(selb[w]);
-      pos += __popc(selb[j >> 5] & ((1u << (j & 31)) - 1u));
-      if (pos < k) sco[pos] = key_score(e.x);
+      const uint32_t pos = tieb[j >> 5] + (uint32_t)__popc(selb[j >> 5] & ((1u << (j & 31)) - 1u));
+      if (pos < (uint32_t)k) sco[pos] = key_score(e.x);
     }
   }
-  if (tid == 0) {
+  if (lane == 0) {
     f.count_out[t] = k;
-    if (!consistent) report(a.err, kErrSelect, (int32_t)t, k);
+    if (!consistent || tot != k) report(a.err, kErrSelect, (int32_t)t, k);
   }
 }
 
 template <int CI>
 cudaError_t launch_finish(const Launch& L, const IndexerArgs& a, int top_k, int32_t* idx_out,
-                          int32_t* count_out, float* score_out, int64_t t_count) {
+                          int32_t* count_out, float* score_out, int64_t t_count,
+                          const uint32_t* list = nullptr, const uint32_t* list_count = nullptr) {
   const size_t qbytes = (size_t)a.H_I * CI * sizeof(float) + 64 * sizeof(float);
   const size_t wmax = (size_t)((((a.max_entries + 31) >> 5) + 3) & ~int64_t(3));
   // staging area: the whole candidate list when it fits next to the bitmaps
@@ -711,9 +1038,9 @@ cudaError_t launch_finish(const Launch& L, const IndexerArgs& a, int top_k, int3
   const size_t bytes = fixed + stage * 8;
   cudaFuncSetAttribute(topk_finish_kernel<CI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   prefer_max_shared(topk_finish_kernel<CI>);
-  FinishArgs f{top_k, idx_out, count_out, score_out, (int)stage};
+  FinishArgs f{top_k, idx_out, count_out, score_out, (int)stage, list, list_count};
   return launch_kernel(topk_finish_kernel<CI>, dim3((unsigned)t_count), dim3(kThreads), bytes,
-                       L.stream, true, a, f);
+                       L.stream, list == nullptr, a, f);
 }
 
 template <int CI>
@@ -760,6 +1087,40 @@ cudaError_t launch_topk_finish(const Launch& L, const IndexerArgs& a, int top_k,
   L.begin(kKernelTopkSelect);
   if (a.c_I == 64) launch_finish<64>(L, a, top_k, idx_out, count_out, score_out, t_count);
   else launch_finish<128>(L, a, top_k, idx_out, count_out, score_out, t_count);
+  return L.end(kKernelTopkSelect);
+}
+
+bool topk_many_supported(const IndexerArgs& a) {
+  const size_t per_warp = (1024 + 2 * (size_t)finish_many_words(a.max_entries) + 2 * kWList) * 4;
+  return a.fb_list != nullptr && a.fb_count != nullptr && per_warp * kFWarps <= 200 * 1024;
+}
+
+cudaError_t launch_topk_threshold_many(const Launch& L, const IndexerArgs& a, int top_k, int64_t t_count) {
+  if (t_count == 0) return cudaSuccess;
+  L.begin(kKernelTopkSample);
+  prefer_max_shared(topk_threshold_many_kernel);
+  const unsigned grid = (unsigned)((t_count + kTWarps - 1) / kTWarps);
+  topk_threshold_many_kernel<<<grid, kTWarps * 32, 0, L.stream>>>(a, top_k, t_count);
+  return L.end(kKernelTopkSample);
+}
+
+cudaError_t launch_topk_finish_many(const Launch& L, const IndexerArgs& a, int top_k, int32_t* idx_out,
+                                    int32_t* count_out, float* score_out, int64_t t_count) {
+  if (t_count == 0) return cudaSuccess;
+  L.begin(kKernelTopkSelect);
+  const size_t bytes = (1024 + 2 * (size_t)finish_many_words(a.max_entries) + 2 * kWList) * 4 * kFWarps;
+  cudaFuncSetAttribute(topk_finish_many_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  prefer_max_shared(topk_finish_many_kernel);
+  FinishArgs f{top_k, idx_out, count_out, score_out, 0};
+  const unsigned grid = (unsigned)((t_count + kFWarps - 1) / kFWarps);
+  topk_finish_many_kernel<<<grid, kFWarps * 32, bytes, L.stream>>>(a, f, t_count);
+  // the queries whose candidate count missed [top_k, cand_cap]: exact recompute
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t g2 = t_count < sms ? t_count : sms;
+  if (a.c_I == 64) launch_finish<64>(L, a, top_k, idx_out, count_out, score_out, g2, a.fb_list, a.fb_count);
+  else launch_finish<128>(L, a, top_k, idx_out, count_out, score_out, g2, a.fb_list, a.fb_count);
   return L.end(kKernelTopkSelect);
 }
 

@@ -138,9 +138,13 @@ def test_workspace_sizes(lib):
     assert hdr + 64 * 8192 * 8 <= n <= hdr + 64 * (8192 * 8 + 8) + 3 * 256
     assert lib.csa_indexer_topk_workspace_size(64, 1 << 19, 2048) == n
     assert lib.csa_indexer_topk_workspace_size(64, 32768, 4096) > n
-    # many-query (prefill) mode stores one key per eligible entry, in bounded chunks
+    # many-query (prefill) mode: the same O(top_k) candidate lists plus 1024
+    # sampled keys per query, in chunks of a multiple of 256 queries within
+    # about 512 MB -- no score per eligible entry
     n = lib.csa_indexer_topk_workspace_size(65536, 16384, 2048)
-    assert hdr + 8192 * 16384 * 4 <= n <= (520 << 20)
+    per_query = 8192 * 8 + 1024 * 4
+    assert hdr + 256 * per_query <= n <= (520 << 20)
+    assert lib.csa_indexer_topk_workspace_size(65536, 40000, 2048) == n   # independent of the entries
     # too small a workspace is refused before anything runs
     from compressed_sparse_kv_03_b200._lib import CacheT
     buf = (C.c_uint8 * 4096)()

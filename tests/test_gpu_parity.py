@@ -289,6 +289,52 @@ def test_indexer_topk_prefill_causal(T, m, k, H_I):
     assert stats["exact"] >= 0.99 * T, stats
 
 
+@pytest.mark.parametrize("T,m,k,H_I,scores", [(6000, 1, 256, 8, False), (9000, 2, 128, 4, True),
+                                              (5000, 1, 1024, 16, False), (4500, 1, 200, 12, True)])
+def test_indexer_topk_many_queries(T, m, k, H_I, scores):
+    """More than 2048 queries on one sequence (prefill mode): with H_I in
+    {4, 8, 16} the tcgen05 scorer's own sample pass, per-warp thresholds,
+    candidate lists and a per-warp finish; H_I = 12 takes the per-query
+    sample and finish launches.  Contexts pass the 4096 entries from which a
+    threshold is sampled, and T = 9000 spans two chunks of 7680 queries.
+    Checked on the first and last queries, both sides of the sampling and
+    chunk boundaries, and 240 random queries."""
+    csa = _csa()
+    g = synth.generator(45 + T + H_I)
+    S = (T - 1) // m
+    qI = synth.normal(g, (T, H_I, 64))
+    w = synth.uniform(g, (T, H_I))
+    KI = synth.normal(g, (S, 64))
+    out = csa.indexer_topk(dev(qI), dev(w), csa.Cache(dev(KI)), m, k, return_scores=scores)
+    idx, cnt, sc = out if scores else (out[0], out[1], None)
+    picks = {0, 1, T - 2, T - 1} | set(range(4090 * m, 4102 * m)) | set(range(7676, 7685))
+    picks |= set(torch.randint(0, T, (240,), generator=g).tolist())
+    queries = sorted(t for t in picks if t < T)
+    KI64 = f64(KI)
+    stats = _check_queries(idx, cnt, qI, w, lambda t: KI64, lambda t: t // m, k, queries, sc)
+    assert stats["exact"] >= 0.99 * len(queries), stats
+
+
+def test_indexer_topk_many_queries_all_equal_scores():
+    """9000 queries whose scores are all exactly 0: below 4097 entries every
+    key is a candidate, up to 8192 the sampled threshold admits every key, and
+    beyond 8192 entries the count passes the candidate slots so the query is
+    listed for the exact recompute.  Every query must select its first k
+    entries (ties to the lower index), bit for bit."""
+    csa = _csa()
+    T, k, m = 9000, 64, 1
+    S = T - 1
+    qI = torch.ones((T, 8, 64), dtype=torch.bfloat16)
+    KI = -torch.ones((S, 64), dtype=torch.bfloat16)
+    w = torch.rand((T, 8), generator=synth.generator(46))
+    idx, cnt = csa.indexer_topk(dev(qI), dev(w), csa.Cache(dev(KI)), m, k)
+    idx, cnt = idx.cpu(), cnt.cpu()
+    n = torch.clamp(torch.arange(T), max=k)
+    assert torch.equal(cnt, n.to(torch.int32))
+    want = torch.where(torch.arange(k)[None, :] < n[:, None], torch.arange(k)[None, :], -1)
+    assert torch.equal(idx, want.to(torch.int32))
+
+
 def test_indexer_topk_exact_ties():
     """Integer-valued keys and queries make integer scores with many exact
     ties: the lower index must win, bit-exactly."""

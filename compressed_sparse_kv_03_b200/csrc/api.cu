@@ -46,8 +46,6 @@ constexpr size_t kIndexerChunkBytes = size_t(512) << 20;   // score scratch per 
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-int64_t score_stride(int64_t max_entries) { return (max_entries + 63) / 64 * 64; }
-
 // Indexer workspace: header | per query tau, candidate count and fallback
 // list entry [3][chunk] u32 + the fallback count | work counter | candidates
 // [chunk, cap] (key, entry) pairs | in many-query mode the sampled keys

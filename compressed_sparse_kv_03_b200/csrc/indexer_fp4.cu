@@ -28,7 +28,7 @@
 // in fp32 before they are added.  The scorer is HBM-bound on the codes: 34
 // bytes per 64-dim key instead of 128.  Keys leave as the same
 // order-preserving 32-bit keys as the bf16 scorer (appended to the candidate
-// lists in fused mode), so the top-k selection is shared.
+// lists), so the top-k selection is shared.
 #include "kernels.h"
 #include "lowprec.cuh"
 
@@ -148,10 +148,10 @@ __device__ __forceinline__ void load_batch(KeyBatch<CI, kU>& kb, const IndexerAr
 // [32v + 8q, 32v + 8q + 8)); the query fragments use the same permutation,
 // which leaves every dot product unchanged, and every k-column of the two
 // mma of block v falls inside block v.
-template <int CI, int NT, bool FUSED, int kU>
+template <int CI, int NT, int kU>
 __device__ __forceinline__ void score_batch(const KeyBatch<CI, kU>& kb,
                                             const Fp4Query<CI, NT>& sq, const IndexerArgs& a,
-                                            int64_t tl, uint32_t tau, uint32_t* out,
+                                            int64_t tl, uint32_t tau,
                                             CandidateBatch<kU>& pend, int64_t s0, int64_t s_end,
                                             int lane, int g, int q4) {
   bool pass[kU];
@@ -201,14 +201,11 @@ __device__ __forceinline__ void score_batch(const KeyBatch<CI, kU>& kb,
     keys[u] = score_key(q4 == 0 ? sg : s8);
     ents[u] = (uint32_t)s;
     pass[u] = valid && keys[u] >= tau;
-    if (!FUSED && valid) out[s] = keys[u];
   }
-  if (FUSED) {
-    CandidateBatch<kU> cur;
-    cur.issue(a, tl, pass, keys, ents);
-    pend.flush(a);
-    pend = cur;
-  }
+  CandidateBatch<kU> cur;
+  cur.issue(a, tl, pass, keys, ents);
+  pend.flush(a);
+  pend = cur;
 }
 
 // One CTA scores a chunk of one query's keys.  The prologue quantizes the
@@ -216,7 +213,7 @@ __device__ __forceinline__ void score_batch(const KeyBatch<CI, kU>& kb,
 // lays out its fragments; each warp then walks batches of kU 16-key groups,
 // loading the next batch's code words into the other register set before it
 // scores the current one.
-template <int CI, int NT, bool FUSED>
+template <int CI, int NT>
 __global__ void __launch_bounds__(kFp4Threads, (CI == 64 && NT == 1) ? 3 : 1)
 indexer_score_fp4_kernel(IndexerArgs a, int64_t chunk) {
   constexpr int KB = CI / 32;                  // scale blocks per vector
@@ -232,7 +229,7 @@ indexer_score_fp4_kernel(IndexerArgs a, int64_t chunk) {
     if (blockIdx.y == 0 && threadIdx.x == 0) report(a.err, kErrEligible, (int32_t)t, n_elig);
     n_elig = a.max_entries;
   }
-  if (FUSED && n_elig <= a.skip_le) return;
+  if (n_elig <= a.skip_le) return;
   const int64_t s_begin = (int64_t)blockIdx.y * chunk;
   if (s_begin >= n_elig) return;
   const int64_t s_end = min(s_begin + chunk, n_elig);
@@ -261,9 +258,8 @@ indexer_score_fp4_kernel(IndexerArgs a, int64_t chunk) {
   __syncthreads();
 
   const uint8_t* codes = reinterpret_cast<const uint8_t*>(a.keys.data);
-  uint32_t* out = FUSED ? nullptr : a.keys_out + tl * a.key_stride;
-  const uint32_t tau = FUSED ? __ldg(a.tau + tl) : 0u;
-  CandidateBatch<kU> pend;   // the previous batch's candidates (fused mode)
+  const uint32_t tau = __ldg(a.tau + tl);
+  CandidateBatch<kU> pend;   // the previous batch's candidates
   const int64_t stride = (int64_t)kFp4Warps * 16 * kU;
   // a contiguous cache whose chunk lies inside the buffer skips the per-row
   // checks (the same conditions cache_row tests, once for the whole chunk)
@@ -279,22 +275,22 @@ indexer_score_fp4_kernel(IndexerArgs a, int64_t chunk) {
   while (s0 < s_end) {
     int64_t s1 = s0 + stride;
     if (s1 < s_end) load_batch(b1, a, codes, seq, base, s1, s_end, t, g, q4);
-    score_batch<CI, NT, FUSED>(b0, sq, a, tl, tau, out, pend, s0, s_end, lane, g, q4);
+    score_batch<CI, NT>(b0, sq, a, tl, tau, pend, s0, s_end, lane, g, q4);
     if (s1 >= s_end) break;
     s0 = s1 + stride;
     if (s0 < s_end) load_batch(b0, a, codes, seq, base, s0, s_end, t, g, q4);
-    score_batch<CI, NT, FUSED>(b1, sq, a, tl, tau, out, pend, s1, s_end, lane, g, q4);
+    score_batch<CI, NT>(b1, sq, a, tl, tau, pend, s1, s_end, lane, g, q4);
   }
-  if (FUSED) pend.flush(a);
+  pend.flush(a);
 }
 
-template <int CI, int NT, bool FUSED>
+template <int CI, int NT>
 void launch_score_fp4(const Launch& L, const IndexerArgs& a, int64_t t_count) {
   constexpr int kU = fp4_unroll(CI, NT);
   int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, indexer_score_fp4_kernel<CI, NT, FUSED>,
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, indexer_score_fp4_kernel<CI, NT>,
                                                 kFp4Threads, 0);
   if (per_sm < 1) per_sm = 1;
   // chunks per query so that the grid fills whole resident waves
@@ -307,8 +303,8 @@ void launch_score_fp4(const Launch& L, const IndexerArgs& a, int64_t t_count) {
   if (chunk < min_chunk) chunk = min_chunk;
   per_q = (a.max_entries + chunk - 1) / chunk;
   const dim3 grid((unsigned)t_count, (unsigned)per_q);
-  prefer_max_shared(indexer_score_fp4_kernel<CI, NT, FUSED>);
-  indexer_score_fp4_kernel<CI, NT, FUSED><<<grid, kFp4Threads, 0, L.stream>>>(a, chunk);
+  prefer_max_shared(indexer_score_fp4_kernel<CI, NT>);
+  indexer_score_fp4_kernel<CI, NT><<<grid, kFp4Threads, 0, L.stream>>>(a, chunk);
 }
 
 }  // namespace
@@ -326,13 +322,9 @@ cudaError_t launch_indexer_scores_fp4(const Launch& L, const IndexerArgs& a, int
   if (t_count == 0 || a.max_entries == 0) return cudaSuccess;
   const int nt = (a.H_I + 7) / 8;
   const int ntb = nt <= 1 ? 1 : nt <= 2 ? 2 : nt <= 4 ? 4 : 8;
-  const bool fused = a.tau != nullptr;
   L.begin(kKernelIndexerScore);
-#define CSA_FP4_CASE(CI_, NT_)                                             \
-  if (a.c_I == CI_ && ntb == NT_) {                                        \
-    if (fused) launch_score_fp4<CI_, NT_, true>(L, a, t_count);            \
-    else launch_score_fp4<CI_, NT_, false>(L, a, t_count);                 \
-  }
+#define CSA_FP4_CASE(CI_, NT_) \
+  if (a.c_I == CI_ && ntb == NT_) launch_score_fp4<CI_, NT_>(L, a, t_count);
   CSA_FP4_CASE(64, 1)
   CSA_FP4_CASE(64, 2)
   CSA_FP4_CASE(64, 4)

@@ -63,25 +63,21 @@ struct NormRopeArgs {
 };
 cudaError_t launch_norm_rope(const Launch& L, const NormRopeArgs& a);
 
-// Indexer selection modes.  Few-query (decode) mode, at most
-// kFusedMaxQueries queries per launch: the scorer keeps only the (key, entry)
-// pairs that reach a per-query threshold drawn from a sample of the query's
-// scores, and a finishing pass selects exactly among them (no score matrix is
-// stored).  Many-query (prefill) mode holds a query's keys in shared memory
-// for a radix select.
+// Indexer selection: the scorer keeps only the (key, entry) pairs that reach
+// a per-query threshold drawn from a sample of the query's scores, and a
+// finishing pass selects exactly among them (no score matrix is stored).
+// Few-query (decode) mode, at most kFusedMaxQueries queries per launch: a
+// per-query sample launch and one CTA per query to finish.  Many-query mode
+// (more queries per call, at most kManyMaxEntries entries each): the tcgen05
+// scorer samples its own keys, and one warp per query sets the threshold and
+// finishes (its selection bitmaps bound the entries per query).
 constexpr int64_t kMaxSelectEntries = int64_t(1) << 19;
 constexpr int64_t kFusedMaxQueries = 2048;
-constexpr int64_t kRadixSelectMaxEntries = 48 * 1024;
-// Many-query mode (more than kFusedMaxQueries queries per call): one warp per
-// query in the threshold and finish passes, whose selection bitmaps bound the
-// entries per query.
 constexpr int64_t kManyMaxEntries = 48 * 1024;
 
 // Lightning-indexer scores of every eligible entry for every query of one
-// chunk of queries: in many-query mode written as order-preserving keys to
-// keys_out[(t - t_begin) * key_stride + s]; in fused mode (tau != null) only
-// the entries whose key reaches tau[t - t_begin] are appended to the query's
-// candidate list.
+// chunk of queries: the entries whose order-preserving key reaches
+// tau[t - t_begin] are appended to the query's candidate list.
 struct IndexerArgs {
   const __nv_bfloat16* q_idx;   // [T, H_I, c_I]
   const float* w;               // [T, H_I]
@@ -92,10 +88,8 @@ struct IndexerArgs {
   int H_I, c_I, m;
   int64_t max_entries;
   int64_t t_begin;              // first query of this launch (chunking)
-  uint32_t* keys_out;           // [T_chunk, key_stride] (many-query mode)
-  int64_t key_stride;
   uint32_t* work;               // zeroed work counter of the tcgen05 scorer
-  // fused selection (few-query mode)
+  // selection
   const uint32_t* tau = nullptr;     // [T_chunk] candidate threshold (a score key)
   uint32_t* cand_count = nullptr;    // [T_chunk] zeroed; counts every pair that passes
   uint2* cand = nullptr;             // [T_chunk, cand_cap] (key, entry), first cand_cap kept
@@ -192,23 +186,8 @@ cudaError_t launch_indexer_scores_fp4(const Launch& L, const IndexerArgs& a, int
 cudaError_t launch_mxfp4_quantize(const Launch& L, const __nv_bfloat16* x, int64_t n_blocks,
                                   uint8_t* codes, uint8_t* scales);
 
-// Many-query selection over stored keys (radix select per query).
-struct SelectArgs {
-  const uint32_t* keys;         // [T_chunk, key_stride]
-  int64_t key_stride;
-  const int64_t* q_pos;
-  int m;
-  int64_t max_entries;
-  int64_t t_begin;
-  int top_k;
-  int32_t* idx_out;             // [T, top_k]
-  int32_t* count_out;           // [T]
-  float* score_out;             // [T, top_k] or null
-  WsHeader* err;
-};
-cudaError_t launch_topk_select(const Launch& L, const SelectArgs& a, int64_t t_count);
 
-// Fused selection (few-query mode), around the scoring launch of the same
+// Few-query selection, around the scoring launch of the same
 // IndexerArgs (tau / cand_count / cand / cand_cap / skip_le / work set):
 //   launch_topk_sample: per query, zeroes its candidate count (and the work
 //     counter), scores a strided sample of its eligible entries and writes a

@@ -1,5 +1,4 @@
-// Step 3 fused with step 2 (few-query / decode mode): exact top-k without a
-// stored score matrix.
+// Step 3 fused with step 2: exact top-k without a stored score matrix.
 //
 // DeepSeek-V4 book, Ch.6 "The lightning indexer" (scores I[t,s] = sum_h
 // w[t,h] ReLU(qI[t,h] . K[s]) over s < floor(t/m)) and "Top-k selection and
@@ -26,6 +25,14 @@
 //      12-bit histogram, refinements of the threshold bin, then a bitmap pass.
 // Both branches give every key above the k-th largest, then the lowest-index
 // keys equal to it, in ascending index order (bitmap compaction).
+//
+// Many-query mode (prefill, more than kFusedMaxQueries queries on one
+// sequence) takes the same three steps with the per-query launches replaced:
+// the tcgen05 scorer's sample pass scores a few whole key chunks per block of
+// queries, topk_threshold_many_kernel derives tau per query (one warp each),
+// and topk_finish_many_kernel selects among the candidates (one warp each),
+// listing the queries whose count misses [k, cand_cap] for the recompute of
+// topk_finish_kernel.
 //
 // Recomputed keys (sample and fallback) use plain fp32 arithmetic; they can
 // differ from the scorer's in the last bits, which only moves near-ties.  The
@@ -788,13 +795,12 @@ __device__ __forceinline__ void warp_take_lowest_ties(uint32_t* sel, const uint3
 }
 
 // Threshold pass: tau of each query from the keys the scorer's sample pass
-// left in psample (the same rank rule and two 11-bit radix levels as the
-// few-query sample pass); also zeroes the candidate counts, the fallback list
-// and the work counter of the scoring pass that follows.
+// left in psample (the few-query sample pass's rank rule, the same 10 low
+// bits cleared); also zeroes the candidate counts, the fallback list and the
+// work counter of the scoring pass that follows.
 constexpr int kTWarps = 4;
 __global__ void __launch_bounds__(kTWarps * 32) topk_threshold_many_kernel(IndexerArgs a, int top_k,
                                                                         int64_t t_count) {
-  __shared__ int hist_all[kTWarps][2048];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     *a.fb_count = 0u;
@@ -826,29 +832,26 @@ __global__ void __launch_bounds__(kTWarps * 32) topk_threshold_many_kernel(Index
     const double mu = (double)ns * (double)top_k / (double)n;
     const int64_t r = (int64_t)ceil(mu + 6.0 * sqrt(mu) + 8.0);
     if (ns > 0 && r < ns) {
+      // the r-th largest sampled key with its low 10 bits cleared, by a
+      // bitwise radix select over the keys held in registers (32 per lane):
+      // bit by bit from the top, the count of keys in the current prefix
+      // group with that bit set decides the branch
       uint32_t kv[kPSampleKeys / 32];
       const uint32_t* sk = a.psample + tl * kPSampleKeys;
+      const int nv = ns >> 5;   // ns is a multiple of 256: whole rows of 32
 #pragma unroll
-      for (int i = 0; i < kPSampleKeys / 32; ++i) kv[i] = 32 * i + lane < ns ? __ldcs(sk + 32 * i + lane) : 0u;
-      int* hist = hist_all[warp];
+      for (int i = 0; i < kPSampleKeys / 32; ++i) kv[i] = i < nv ? __ldcs(sk + 32 * i + lane) : 0u;
       uint32_t prefix = 0u;
       int need = (int)r;
 #pragma unroll 1
-      for (int level = 0; level < 2; ++level) {
-        const int lo = level == 0 ? 21 : 10;
-        for (int b = lane; b < 2048; b += 32) hist[b] = 0;
-        __syncwarp();
+      for (int bit = 31; bit >= 10; --bit) {
+        const uint32_t want = (prefix >> bit) | 1u;
+        int cnt = 0;
 #pragma unroll
-        for (int i = 0; i < kPSampleKeys / 32; ++i)
-          if (32 * i + lane < ns && (level == 0 || (kv[i] >> 21) == (prefix >> 21)))
-            atomicAdd(&hist[(kv[i] >> lo) & 2047u], 1);
-        __syncwarp();
-        uint32_t bin;
-        int above;
-        warp_find_bin(hist, 2048, need, bin, above);
-        prefix |= bin << lo;
-        need -= above;
-        __syncwarp();
+        for (int i = 0; i < kPSampleKeys / 32; ++i) cnt += (i < nv && (kv[i] >> bit) == want) ? 1 : 0;
+        cnt = __reduce_add_sync(0xffffffffu, cnt);
+        if (cnt >= need) prefix |= 1u << bit;
+        else need -= cnt;
       }
       tau = prefix;
     }
@@ -863,6 +866,7 @@ __global__ void __launch_bounds__(kTWarps * 32) topk_threshold_many_kernel(Index
 // [kWList] (key, entry) pairs.
 constexpr int kFWarps = 8;
 constexpr int kWList = 128;
+constexpr int kFBatch = 8;   // candidates per lane with their loads in flight together
 __host__ __device__ inline int finish_many_words(int64_t max_entries) {
   return (int)((((max_entries + 31) >> 5) + 1) & ~int64_t(1));   // keeps the list 8-byte aligned
 }
@@ -911,12 +915,28 @@ __global__ void __launch_bounds__(kFWarps * 32) topk_finish_many_kernel(IndexerA
     selb[w] = 0u;
     tieb[w] = 0u;
   }
+  // every pass walks the list kFBatch candidates per lane at a time, with all
+  // of their loads issued before any is used; fn(e, in_range) is called by
+  // every lane for each slot of the batch (warp-collective calls allowed)
+  auto for_each_cand = [&](auto&& fn) {
+    for (int i0 = 0; i0 < c; i0 += 32 * kFBatch) {
+      uint2 e[kFBatch];
+#pragma unroll
+      for (int u = 0; u < kFBatch; ++u) {
+        const int i = i0 + 32 * u + lane;
+        e[u] = i < c ? cand[i] : make_uint2(0u, 0xffffffffu);
+      }
+#pragma unroll
+      for (int u = 0; u < kFBatch; ++u) fn(e[u], i0 + 32 * u + lane < c);
+    }
+  };
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int i = lane; i < c; i += 32) {
-    const uint32_t key = cand[i].x;
-    kmin = min(kmin, key);
-    kmax = max(kmax, key);
-  }
+  for_each_cand([&](const uint2 e, bool in) {
+    if (in) {
+      kmin = min(kmin, e.x);
+      kmax = max(kmax, e.x);
+    }
+  });
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   __syncwarp();
@@ -935,10 +955,9 @@ __global__ void __launch_bounds__(kFWarps * 32) topk_finish_many_kernel(IndexerA
     const int nb = dig < 5 ? 32 : (1 << dig);
     for (int b = lane; b < nb; b += 32) hist[b] = 0;
     __syncwarp();
-    for (int i = lane; i < c; i += 32) {
-      const uint32_t key = cand[i].x;
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> lo) & dm], 1);
-    }
+    for_each_cand([&](const uint2 e, bool in) {
+      if (in && (e.x & mask) == prefix) atomicAdd(&hist[(e.x >> lo) & dm], 1);
+    });
     __syncwarp();
     uint32_t bin;
     int above;
@@ -954,10 +973,8 @@ __global__ void __launch_bounds__(kFWarps * 32) topk_finish_many_kernel(IndexerA
   // keys above the threshold bin are selected; its keys are ties (complete
   // key) or listed for ranking
   int listn = 0;
-  for (int i0 = 0; i0 < c; i0 += 32) {
-    const int i = i0 + lane;
-    const uint2 e = i < c ? cand[i] : make_uint2(0u, 0u);
-    const bool valid = i < c && (int64_t)e.y < n;
+  for_each_cand([&](const uint2 e, bool in) {
+    const bool valid = in && (int64_t)e.y < n;
     const uint32_t mk = e.x & mask;
     if (valid && mk > prefix) atomicOr(&selb[e.y >> 5], 1u << (e.y & 31));
     const bool eq = valid && mk == prefix;
@@ -969,7 +986,7 @@ __global__ void __launch_bounds__(kFWarps * 32) topk_finish_many_kernel(IndexerA
       if (eq && pos < kWList) list[pos] = e;
       listn += __popc(be);
     }
-  }
+  });
   __syncwarp();
   if (shift > 0) {
     // an entry of the bin is selected iff fewer than `need` entries of the bin
@@ -1008,13 +1025,12 @@ __global__ void __launch_bounds__(kFWarps * 32) topk_finish_many_kernel(IndexerA
   }
   __syncwarp();
   if (sco) {
-    for (int i = lane; i < c; i += 32) {
-      const uint2 e = cand[i];
+    for_each_cand([&](const uint2 e, bool in) {
       const uint32_t j = e.y;
-      if ((int64_t)j >= n || !((selb[j >> 5] >> (j & 31)) & 1u)) continue;
+      if (!in || (int64_t)j >= n || !((selb[j >> 5] >> (j & 31)) & 1u)) return;
       const uint32_t pos = tieb[j >> 5] + (uint32_t)__popc(selb[j >> 5] & ((1u << (j & 31)) - 1u));
       if (pos < (uint32_t)k) sco[pos] = key_score(e.x);
-    }
+    });
   }
   if (lane == 0) {
     f.count_out[t] = k;

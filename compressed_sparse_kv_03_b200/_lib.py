@@ -56,6 +56,7 @@ SIGNATURES = {
     "csa_set_timing_events": (C.c_int, [_i32, _vp, _vp]),
     "csa_set_attention_kernel": (C.c_int, [_i32]),
     "csa_set_batch_invariant": (C.c_int, [_i32]),
+    "csa_test_attention_timeout": (C.c_int, [_i32]),
     "csa_indexer_topk_workspace_size": (_sz, [_i64, _i64, _i32]),
     "csa_sparse_attn_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "csa_sparse_attn_prefill_workspace_size": (_sz, [_i64, _i32, _i32]),

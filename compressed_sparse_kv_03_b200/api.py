@@ -505,6 +505,13 @@ def set_batch_invariant(on):
     check(load().csa_set_batch_invariant(1 if on else 0))
 
 
+def test_attention_timeout(on=True):
+    """Failure-detection self-test (see csa_test_attention_timeout): the next
+    tensor-core attention launch lets its bounded pipeline waits run out and
+    records the timeout in its workspace header."""
+    check(load().csa_test_attention_timeout(1 if on else 0))
+
+
 def set_timing_events(kernel_id, begin=None, end=None):
     """Attach torch.cuda.Event objects (enable_timing=True) around every launch
     of one library kernel; pass None to detach."""

@@ -18,6 +18,7 @@ thread_local std::string g_last_error;
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int32_t> g_attn_kernel{0};
 std::atomic<int32_t> g_batch_invariant{0};
+std::atomic<int32_t> g_timeout_test{0};
 struct EventPair {
   cudaEvent_t begin = nullptr, end = nullptr;
 };
@@ -200,6 +201,8 @@ void set_last_error(const char* msg) { g_last_error = msg; }
 
 int32_t attention_kernel_choice() { return g_attn_kernel.load(std::memory_order_relaxed); }
 
+bool take_attention_timeout_test() { return g_timeout_test.exchange(0, std::memory_order_relaxed) != 0; }
+
 void Launch::begin(int32_t kernel) const {
   const EventPair& e = g_events[kernel];
   if (e.begin) record_event(e.begin, stream);
@@ -229,6 +232,13 @@ csa_status_t csa_set_attention_kernel(int32_t choice) {
   if (choice < 0 || choice > 2)
     return fail(CSA_ERR_INVALID_ARG, "csa_set_attention_kernel: choice %d out of range", choice);
   g_attn_kernel.store(choice, std::memory_order_relaxed);
+  return CSA_OK;
+}
+
+csa_status_t csa_test_attention_timeout(int32_t on) {
+  if (on != 0 && on != 1)
+    return fail(CSA_ERR_INVALID_ARG, "csa_test_attention_timeout: on must be 0 or 1, got %d", on);
+  g_timeout_test.store(on, std::memory_order_relaxed);
   return CSA_OK;
 }
 

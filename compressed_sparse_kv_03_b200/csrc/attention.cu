@@ -390,7 +390,12 @@ cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {
   if (a.T == 0) return cudaSuccess;
   if (a.use_tc) {
     L.begin(kKernelAttention);
-    cudaError_t e = launch_attention_tc(L, a);
+    AttnArgs b = a;
+    if (take_attention_timeout_test()) {
+      b.withhold_q = 1;
+      b.wait_limit = 1ll << 21;
+    }
+    cudaError_t e = launch_attention_tc(L, b);
     if (e != cudaSuccess) return e;
     e = L.end(kKernelAttention);
     if (e != cudaSuccess || a.n_split == 1) return e;

@@ -205,10 +205,10 @@ __device__ __forceinline__ void fence_async_smem() {
 
 // Softmax-warp group barrier on an mbarrier (count 4): bounded, so that a
 // warp that gave up elsewhere cannot strand the others.
-__device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, int lane) {
+__device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, int lane, long long limit) {
   __syncwarp();
   if (lane == 0) mbar_arrive(bar);
-  const bool ok = mbar_wait(bar, phase);
+  const bool ok = mbar_wait(bar, phase, limit);
   phase ^= 1u;
   return ok;
 }
@@ -304,10 +304,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
       if (it.n_tiles == 0) continue;
       if (pt == 0) {   // the query's heads, once per item
         const int qb = (int)(items_done & 1);
-        if (!mbar_wait(smem_u32(&q_empty[qb]), (uint32_t)(((items_done >> 1) & 1) ^ 1))) {
+        if (!mbar_wait(smem_u32(&q_empty[qb]), (uint32_t)(((items_done >> 1) & 1) ^ 1), a.wait_limit)) {
           report(a.err, kErrTimeout, (int32_t)it.i, 20);
           ok = false;
-        } else {
+        } else if (!(a.withhold_q && items_done == 0)) {   // (test hook: never arrives)
           mbar_arrive_expect_tx(smem_u32(&q_full[qb]), kQTile);
           const int32_t qrow = (int32_t)(it.i * a.H + it.hg * kNP);
           const uint32_t qd = q_sm + qb * kQTile;
@@ -323,7 +323,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
       for (int t = 0; t < it.n_tiles && ok; ++t, ++tiles_done) {
         const int slot = (int)(tiles_done % kStages);
         const bool got =
-            mbar_wait(smem_u32(&kv_empty[slot]), (uint32_t)(((tiles_done / kStages) & 1) ^ 1));
+            mbar_wait(smem_u32(&kv_empty[slot]), (uint32_t)(((tiles_done / kStages) & 1) ^ 1), a.wait_limit);
         if (!__all_sync(0xffffffffu, got)) {
           if (pt == 0) report(a.err, kErrTimeout, (int32_t)it.i, 21);
           ok = false;
@@ -412,7 +412,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
       const int64_t first = tiles_done > kStages ? tiles_done - kStages : 0;
       for (int64_t d = first; d < tiles_done; ++d)
         mbar_wait(smem_u32(&kv_full[d % kStages]), (uint32_t)((d / kStages) & 1), 200000000ll);
-      if (items_done > 0)
+      if (items_done > 0 && !(a.withhold_q && items_done == 1))   // no query copy was issued
         mbar_wait(smem_u32(&q_full[(items_done - 1) & 1]), (uint32_t)(((items_done - 1) >> 1) & 1),
                   200000000ll);
     }
@@ -423,9 +423,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
       bool ok = true;
       auto do_pv = [&](int64_t gtile, bool first) -> bool {
         const int pb = (int)(gtile & 1);
-        if (!mbar_wait(smem_u32(&p_full[pb]), (uint32_t)((gtile >> 1) & 1))) return false;
+        if (!mbar_wait(smem_u32(&p_full[pb]), (uint32_t)((gtile >> 1) & 1), a.wait_limit)) return false;
         // the previous item's epilogue must have read O^T before it is overwritten
-        if (first && !mbar_wait(smem_u32(&o_empty), (uint32_t)((items_done & 1) ^ 1))) return false;
+        if (first && !mbar_wait(smem_u32(&o_empty), (uint32_t)((items_done & 1) ^ 1), a.wait_limit)) return false;
         tc::fence_after_sync();
         const uint32_t kv = kv_sm + (int)(gtile % kStages) * kKvTile;
         const uint32_t pt = p_sm + pb * kPTile;
@@ -444,7 +444,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         if (it.n_tiles == 0) continue;
         const int qb = (int)(items_done & 1);
         const uint32_t qs = q_sm + qb * kQTile;
-        if (!mbar_wait(smem_u32(a.qprologue ? &q_ready[qb] : &q_full[qb]), (uint32_t)((items_done >> 1) & 1))) {
+        if (!mbar_wait(smem_u32(a.qprologue ? &q_ready[qb] : &q_full[qb]), (uint32_t)((items_done >> 1) & 1), a.wait_limit)) {
           report(a.err, kErrTimeout, (int32_t)it.i, 22);
           ok = false;
           break;
@@ -454,8 +454,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         for (int t = 0; t < it.n_tiles; ++t, ++tiles_done) {
           const int slot = (int)(tiles_done % kStages);
           const int sb = (int)(tiles_done & 1);
-          if (!mbar_wait(smem_u32(&kv_full[slot]), (uint32_t)((tiles_done / kStages) & 1)) ||
-              !mbar_wait(smem_u32(&s_empty[sb]), (uint32_t)(((tiles_done >> 1) & 1) ^ 1))) {
+          if (!mbar_wait(smem_u32(&kv_full[slot]), (uint32_t)((tiles_done / kStages) & 1), a.wait_limit) ||
+              !mbar_wait(smem_u32(&s_empty[sb]), (uint32_t)(((tiles_done >> 1) & 1) ^ 1), a.wait_limit)) {
             report(a.err, kErrTimeout, (int32_t)it.i, 23);
             ok = false;
             break;
@@ -533,14 +533,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         // item's query tile, in place in shared memory: thread = (head,
         // quarter of the dims), four 16-byte chunks of the swizzled tile.
         const int qb = (int)(items_done & 1);
-        bool okp = mbar_wait(smem_u32(&q_full[qb]), (uint32_t)((items_done >> 1) & 1));
+        bool okp = mbar_wait(smem_u32(&q_full[qb]), (uint32_t)((items_done >> 1) & 1), a.wait_limit);
         const int r0 = kD - a.q_rope_dims;
         if (okp && a.q_rope_dims > 0 && (int)threadIdx.x < a.q_rope_dims / 2) {
           float c, sn;
           rope_cs(p, rope_position(a, it.i), threadIdx.x, false, c, sn);
           rope_tab[qb][threadIdx.x] = make_float2(c, sn);
         }
-        okp = okp && group_sync(smem_u32(&pro_bar), pro_phase, lane);
+        okp = okp && group_sync(smem_u32(&pro_bar), pro_phase, lane, a.wait_limit);
         if (!okp) {
           if (lane == 0) report(a.err, kErrTimeout, (int32_t)it.i, 30);
           break;
@@ -606,8 +606,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
       for (int t = 0; t < it.n_tiles && ok; ++t, ++tiles_done) {
         const int slot = (int)(tiles_done % kStages);
         const int sb = (int)(tiles_done & 1);
-        ok = mbar_wait(smem_u32(&s_full[sb]), (uint32_t)((tiles_done >> 1) & 1)) &&
-             mbar_wait(smem_u32(&kv_full[slot]), (uint32_t)((tiles_done / kStages) & 1));
+        ok = mbar_wait(smem_u32(&s_full[sb]), (uint32_t)((tiles_done >> 1) & 1), a.wait_limit) &&
+             mbar_wait(smem_u32(&kv_full[slot]), (uint32_t)((tiles_done / kStages) & 1), a.wait_limit);
         if (!ok) break;
         tc::fence_after_sync();
         float x[kHW];
@@ -643,7 +643,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
               *reinterpret_cast<float4*>(&rm[warp][h]) = make_float4(mx[h], mx[h + 1], mx[h + 2], mx[h + 3]);
           }
         }
-        if (!(ok = group_sync(rbar, red_phase, lane))) break;
+        if (!(ok = group_sync(rbar, red_phase, lane, a.wait_limit))) break;
         // lane hl = lane mod kHW stands for head hoff + hl (lanes past kHW repeat them)
         float tmax = fmaxf(fmaxf(rm[4 * wg][hl], rm[4 * wg + 1][hl]),
                            fmaxf(rm[4 * wg + 2][hl], rm[4 * wg + 3][hl]));
@@ -664,7 +664,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         if (rescale) {
           // this warp's 32 dims of O^T for the group's heads, when a running max moved
           if (pv_seen < tiles_done) {   // every earlier PV must have completed
-            if (!(ok = mbar_wait(smem_u32(&o_step), (uint32_t)((tiles_done - 1) & 1)))) break;
+            if (!(ok = mbar_wait(smem_u32(&o_step), (uint32_t)((tiles_done - 1) & 1), a.wait_limit))) break;
             pv_seen = tiles_done;
           }
           tc::fence_after_sync();
@@ -682,7 +682,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
           tc::fence_before_sync();
         }
         // probabilities, partial sums, bf16 P^T (this group's 64 bytes of the row)
-        if (!(ok = mbar_wait(smem_u32(&p_empty[sb]), (uint32_t)(((tiles_done >> 1) & 1) ^ 1)))) break;
+        if (!(ok = mbar_wait(smem_u32(&p_empty[sb]), (uint32_t)(((tiles_done >> 1) & 1) ^ 1), a.wait_limit))) break;
         const uint32_t prow = p_sm + sb * kPTile + (uint32_t)row * 128;
 #pragma unroll
         for (int c = 0; c < kHW / 8; ++c) {
@@ -735,8 +735,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
       }
       for (int o = kHW; o < 32; o <<= 1) lpart[0] += __shfl_xor_sync(0xffffffffu, lpart[0], o);
       if (lane < kHW) red_l[warp][lane] = lpart[0];
-      if (!mbar_wait(smem_u32(&o_full), (uint32_t)(items_done & 1)) ||
-          !group_sync(rbar, red_phase, lane)) {
+      if (!mbar_wait(smem_u32(&o_full), (uint32_t)(items_done & 1), a.wait_limit) ||
+          !group_sync(rbar, red_phase, lane, a.wait_limit)) {
         if (lane == 0) report(a.err, kErrTimeout, (int32_t)it.i, 28);
         break;
       }

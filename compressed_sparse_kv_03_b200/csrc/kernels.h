@@ -263,6 +263,11 @@ struct AttnArgs {
   float q_rope_base = 10000.f;
   int out_derotate = 0;
   const int64_t* rope_pos = nullptr;
+  // cycles a pipeline wait of the tcgen05 kernel may take before it gives up
+  // and records a timeout; withhold_q (failure-detection self-test) skips the
+  // first work item's query-tile copy so that those waits run out
+  long long wait_limit = 2000000000ll;
+  int withhold_q = 0;
 };
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a);
 
@@ -290,6 +295,9 @@ __device__ __forceinline__ int64_t attn_raw_window(const AttnArgs& a, int64_t i,
 bool tc_attention_supported(const AttnArgs& a);
 // 0 automatic, 1 tensor-core kernel, 2 mma.sync kernel
 int32_t attention_kernel_choice();
+// true once after csa_test_attention_timeout(1): the next tensor-core
+// attention launch runs the self-test
+bool take_attention_timeout_test();
 // Which attention kernel a call with these arguments runs (fields other than
 // the split / workspace ones must be set).
 bool attention_uses_tc(const AttnArgs& a);

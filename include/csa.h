@@ -119,6 +119,19 @@ csa_status_t csa_set_attention_kernel(int32_t choice);
  */
 csa_status_t csa_set_batch_invariant(int32_t on);
 
+/*
+ * Failure-detection self-test (process-wide, one shot; a library setting with
+ * no counterpart in the method).  With on = 1 the next launch of the tcgen05
+ * attention kernel never issues its first work item's query-tile copy and
+ * waits at most about 1 ms (2^21 cycles) on each pipeline barrier: its
+ * bounded waits give up, it records "a bounded pipeline wait timed out" in
+ * the workspace header (read it with csa_workspace_check) and returns, and
+ * the device stays usable.  No output of that launch is valid.  The setting
+ * clears itself at that launch; on = 0 clears it before.  Returns
+ * CSA_ERR_INVALID_ARG unless `on` is 0 or 1.
+ */
+csa_status_t csa_test_attention_timeout(int32_t on);
+
 /* ---- workspace ------------------------------------------------------------ */
 /*
  * Calls that take `ws` need a caller-allocated device workspace of at least

@@ -168,6 +168,13 @@ def test_attention_kernel_choice_validation(lib):
         assert lib.csa_set_attention_kernel(choice) == 0
 
 
+def test_timeout_self_test_validation(lib):
+    assert lib.csa_test_attention_timeout(2) == 1 and b"0 or 1" in lib.csa_last_error()
+    assert lib.csa_test_attention_timeout(-1) == 1
+    assert lib.csa_test_attention_timeout(1) == 0
+    assert lib.csa_test_attention_timeout(0) == 0   # cleared before any launch
+
+
 def test_batch_invariant_mode_validation_and_sizing(lib):
     assert lib.csa_set_batch_invariant(2) == 1 and b"0 or 1" in lib.csa_last_error()
     # B=400 queries fill the GPU without splitting; fixed 512-row slices need partials

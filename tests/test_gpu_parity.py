@@ -555,6 +555,44 @@ def test_attention_device_check_reports_bad_index():
         assert_close_attn(out[b], ref, "unaffected query")
 
 
+def test_bounded_wait_timeout_is_reported_and_the_device_stays_usable():
+    """Failure detection without a fault: the self-test withholds the first
+    query tile of one tensor-core attention launch, so its bounded pipeline
+    waits (about 1 ms each) run out.  The launch must end by itself, the
+    workspace header must report the timeout, and the next call must give the
+    same bits as before the test."""
+    import time
+    csa = _csa()
+    g = synth.generator(97)
+    B, H, k, W, S = 4, 64, 256, 128, 5000
+    q = synth.normal(g, (B, H, 128))
+    kvc = synth.normal(g, (B, S, 128))
+    win = synth.normal(g, (B, W, 128))
+    win_len = torch.full((B,), W, dtype=torch.int32)
+    idx = torch.stack([torch.randperm(S, generator=g)[:k].sort().values for _ in range(B)]).to(torch.int32)
+    cnt = torch.full((B,), k, dtype=torch.int32)
+    args = (dev(q), csa.Cache.contiguous(dev(kvc)), dev(win), dev(win_len), dev(idx), dev(cnt), 0.088)
+    csa.set_attention_kernel("tcgen05")
+    ws = csa.Workspace()
+    try:
+        ref = csa.sparse_attn_decode(*args, ws=ws)
+        ws.check()
+        csa.test_attention_timeout(True)
+        t0 = time.time()
+        csa.sparse_attn_decode(*args, ws=ws)
+        torch.cuda.synchronize()
+        took = time.time() - t0
+        with pytest.raises(csa.CsaError, match="timed out"):
+            ws.check()
+        assert took < 30, took
+        again = csa.sparse_attn_decode(*args, ws=ws)
+        ws.check()
+        assert torch.equal(again, ref)
+    finally:
+        csa.test_attention_timeout(False)
+        csa.set_attention_kernel("auto")
+
+
 @pytest.mark.usefixtures("attn_kernel")
 def test_decode_is_deterministic():
     csa = _csa()

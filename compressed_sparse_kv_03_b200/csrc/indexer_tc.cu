@@ -10,8 +10,9 @@
 //              6-stage shared-memory ring (one mbarrier per stage and
 //              direction);
 //   warp 1     allocates TMEM and issues tcgen05.mma: two M = 128 key tiles
-//              per item against the 16 (padded) indexer heads on N, key dim 64
-//              as K in four steps, into one of four 32-column TMEM sets;
+//              per item against the indexer heads (padded to NH = 16, 32 or
+//              64) on N, key dim c_I = 64 or 128 as K in steps of 16, into
+//              one of four 2 NH-column TMEM sets;
 //   warps 2-9  epilogue, two groups of four warps taking alternate items:
 //              tcgen05.ld of their 32 TMEM lanes (one key per tile), ReLU,
 //              the head-weighted sum, the order-preserving score key, and the
@@ -32,20 +33,35 @@ namespace csa {
 
 namespace {
 
-constexpr int kStages = 6;
 constexpr int kTileRows = 128;                     // MMA M
 constexpr int kItemRows = 2 * kTileRows;           // keys per pipeline item
 constexpr int kBoxRows = 64;                       // TMA box height (page granule)
 constexpr int kKeyTileBytes = kTileRows * 128;     // 64 bf16 per row
 constexpr int kStageKeyBytes = 2 * kKeyTileBytes;
-constexpr int kQTileBytes = 16 * 128;              // 16 head rows (MMA N)
 constexpr int kEpiWarps = 8;                       // two groups of four
 constexpr int kThreads = (2 + kEpiWarps) * 32;
-constexpr int kAcc = 4;                            // TMEM accumulator sets (32 columns each)
-constexpr uint32_t kIdesc = tc::idesc_bf16(128, 16);
-constexpr int kTmemCols = kAcc * 32;
+constexpr int kAcc = 4;                            // TMEM accumulator sets
+
+// Decode-mode layout for key dim CI (64 or 128) and NH padded heads: an
+// item's keys are CI / 64 column blocks of 256 rows x 128 bytes (one TMA box
+// of the 128-byte swizzle each), the query's heads as many blocks of NH rows.
+template <int CI, int NH>
+struct ScoreCfg {
+  static constexpr int kKB = CI / 64;
+  static constexpr int kKeyBlk = kItemRows * 128;
+  static constexpr int kStageKey = kKB * kKeyBlk;
+  static constexpr int kQBlk = NH * 128;
+  static constexpr int kQBytes = kKB * kQBlk;
+  // as many stages as fit beside the kernel's static shared memory (<= 6)
+  static constexpr int kFit = (205 * 1024) / (kStageKey + kQBytes);
+  static constexpr int kStages = kFit < 6 ? kFit : 6;
+  static constexpr int kAccCols = 2 * NH;          // two key tiles of NH columns
+  static constexpr int kTmemCols = kAcc * kAccCols;   // 128, 256 or 512
+  static constexpr uint32_t kIdesc = tc::idesc_bf16(128, NH);
+  static constexpr int kSmem = kStages * (kStageKey + kQBytes) + 1024;
+};
 constexpr int kMaxQueries = 2048;
-constexpr int kRing = 16;                          // item metadata ring (> kStages + kAcc)
+constexpr int kRing = 16;                          // item metadata ring (> stages + kAcc)
 constexpr int kGrab = 2;                           // items taken from the work counter at once
 #ifndef CSA_SCORE_STATIC_PCT
 #define CSA_SCORE_STATIC_PCT 70
@@ -55,7 +71,7 @@ constexpr int kStaticPct = CSA_SCORE_STATIC_PCT;   // items dealt out statically
 // What the producer tells the MMA warp and the epilogue about item j: the
 // query (-1 ends the stream), the 256-key chunk and the query's head weights.
 struct __align__(16) ItemMeta {
-  float w[16];
+  float w[64];
   int32_t t, chunk, pad0, pad1;
 };
 
@@ -70,9 +86,12 @@ __device__ __forceinline__ int64_t eligible(const IndexerArgs& a, int64_t t) {
   return n < a.max_entries ? n : a.max_entries;
 }
 
+template <int CI, int NH>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
                         const __grid_constant__ CUtensorMap tmap_q, TcIndexerParams p) {
+  using Cfg = ScoreCfg<CI, NH>;
+  constexpr int kStages = Cfg::kStages, kTmemCols = Cfg::kTmemCols;
   pdl_trigger();
   const IndexerArgs& a = p.a;
   const int T = (int)p.t_count;
@@ -87,8 +106,8 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t keys_sm = base;                                // kStages x 32 KB
-  const uint32_t q_sm = base + kStages * kStageKeyBytes;        // kStages x 2 KB
+  const uint32_t keys_sm = base;                                // kStages x kStageKey
+  const uint32_t q_sm = base + kStages * Cfg::kStageKey;        // kStages x kQBytes
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -183,7 +202,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
         while (prefix[tq + 1] <= nxt) ++tq;
         return nxt++;
       };
-      float wreg[16];
+      float wreg[NH];
       int32_t seq_reg = 0;
       int w_tq = -1;
       auto load_w = [&]() {   // the query's head weights and sequence
@@ -191,7 +210,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
         w_tq = tq;
         const int64_t t = a.t_begin + tq;
 #pragma unroll
-        for (int h = 0; h < 16; ++h) wreg[h] = h < a.H_I ? __ldg(a.w + t * a.H_I + h) : 0.f;
+        for (int h = 0; h < NH; ++h) wreg[h] = h < a.H_I ? __ldg(a.w + t * a.H_I + h) : 0.f;
         seq_reg = a.seq_id ? __ldg(a.seq_id + t) : 0;
       };
       int32_t item = take();
@@ -207,7 +226,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
           break;
         }
 #pragma unroll
-        for (int h = 0; h < 16; ++h) ring[rs].w[h] = wreg[h];
+        for (int h = 0; h < NH; ++h) ring[rs].w[h] = wreg[h];
         ring[rs].t = tq;
         ring[rs].chunk = chunk;
         mbar_arrive(smem_u32(&ring_full[rs]));
@@ -220,11 +239,14 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
           break;
         }
         const uint32_t fb = smem_u32(&full_bar[slot]);
-        mbar_arrive_expect_tx(fb, kStageKeyBytes + kQTileBytes);
+        mbar_arrive_expect_tx(fb, Cfg::kStageKey + Cfg::kQBytes);
+        const uint32_t kst = keys_sm + slot * Cfg::kStageKey;
         if (a.keys.page_table == nullptr) {
-          // contiguous: the item's 256 keys are one 256-row box
-          tc::tma_load_2d(keys_sm + slot * kStageKeyBytes, &tmap_keys, 0,
-                          (int32_t)((int64_t)seq * a.keys.seq_stride + s0), fb);
+          // contiguous: the item's 256 keys are one 256-row box per column block
+#pragma unroll
+          for (int kb = 0; kb < Cfg::kKB; ++kb)
+            tc::tma_load_2d(kst + kb * Cfg::kKeyBlk, &tmap_keys, 64 * kb,
+                            (int32_t)((int64_t)seq * a.keys.seq_stride + s0), fb);
         } else {
 #pragma unroll
         for (int h = 0; h < kItemRows / kBoxRows; ++h) {
@@ -241,11 +263,16 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
               row = 0;
             }
           }
-          tc::tma_load_2d(keys_sm + slot * kStageKeyBytes + h * kBoxRows * 128, &tmap_keys, 0,
-                          (int32_t)row, fb);
+#pragma unroll
+          for (int kb = 0; kb < Cfg::kKB; ++kb)
+            tc::tma_load_2d(kst + kb * Cfg::kKeyBlk + h * kBoxRows * 128, &tmap_keys, 64 * kb,
+                            (int32_t)row, fb);
         }
         }
-        tc::tma_load_2d(q_sm + slot * kQTileBytes, &tmap_q, 0, (int32_t)(t * a.H_I), fb);
+#pragma unroll
+        for (int kb = 0; kb < Cfg::kKB; ++kb)
+          tc::tma_load_2d(q_sm + slot * Cfg::kQBytes + kb * Cfg::kQBlk, &tmap_q, 64 * kb,
+                          (int32_t)(t * a.H_I), fb);
         ++issued;
         item = take();
         if (item >= 0) load_w();
@@ -291,14 +318,18 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
           break;
         }
         tc::fence_after_sync();
-        const uint32_t qa = q_sm + slot * kQTileBytes;
+        const uint32_t qa = q_sm + slot * Cfg::kQBytes;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const uint32_t ka = keys_sm + slot * kStageKeyBytes + h * kKeyTileBytes;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc::mma_bf16_ss(tmem_base + acc * 32 + h * 16, tc::smem_desc_sw128(ka + 32 * k),
-                            tc::smem_desc_sw128(qa + 32 * k), kIdesc, k > 0);
+          for (int kb = 0; kb < Cfg::kKB; ++kb) {
+            const uint32_t ka = keys_sm + slot * Cfg::kStageKey + kb * Cfg::kKeyBlk + h * kKeyTileBytes;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc::mma_bf16_ss(tmem_base + acc * Cfg::kAccCols + h * NH, tc::smem_desc_sw128(ka + 32 * k),
+                              tc::smem_desc_sw128(qa + kb * Cfg::kQBlk + 32 * k), Cfg::kIdesc,
+                              kb > 0 || k > 0);
+          }
         }
         tc::mma_commit(smem_u32(&empty_bar[slot]));   // smem stage free when the MMAs finish
         tc::mma_commit(smem_u32(&tfull_bar[acc]));    // accumulators ready
@@ -326,9 +357,9 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
       }
       const int tq = ring[rs].t;
       const int32_t chunk = ring[rs].chunk;
-      float wv[16];
+      float wv[NH];
 #pragma unroll
-      for (int h = 0; h < 16; h += 4) {
+      for (int h = 0; h < NH; h += 4) {
         const float4 w4 = *reinterpret_cast<const float4*>(&ring[rs].w[h]);
         wv[h] = w4.x;
         wv[h + 1] = w4.y;
@@ -349,11 +380,22 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
         break;
       }
       tc::fence_after_sync();
-      uint32_t r0[16], r1[16];
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * 32;
-      tc::tmem_ld16(taddr, r0);
-      tc::tmem_ld16(taddr + 16, r1);
-      tc::tmem_wait_ld();
+      // this key's ReLU-weighted head sum in each of the two tiles, NH
+      // columns each, 16 columns per TMEM load
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * Cfg::kAccCols;
+      float scs[2] = {0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < NH / 16; ++c) {
+        uint32_t r0[16], r1[16];
+        tc::tmem_ld16(taddr + 16 * c, r0);
+        tc::tmem_ld16(taddr + NH + 16 * c, r1);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          scs[0] = fmaf(wv[16 * c + k], fmaxf(__uint_as_float(r0[k]), 0.f), scs[0]);
+          scs[1] = fmaf(wv[16 * c + k], fmaxf(__uint_as_float(r1[k]), 0.f), scs[1]);
+        }
+      }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[acc]));
@@ -362,10 +404,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
       uint32_t keys[2], ents[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const uint32_t* r = h ? r1 : r0;
-        float sc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) sc = fmaf(wv[k], fmaxf(__uint_as_float(r[k]), 0.f), sc);
+        const float sc = scs[h];
         const int64_t s = s0 + h * kTileRows + row;
         keys[h] = score_key(sc);
         ents[h] = (uint32_t)s;
@@ -783,7 +822,7 @@ indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
 
 bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count) {
   if (a.tau == nullptr) return false;   // fused selection only
-  if (a.c_I != 64 || a.H_I > 16 || t_count > kMaxQueries) return false;
+  if ((a.c_I != 64 && a.c_I != 128) || a.H_I > 64 || t_count > kMaxQueries) return false;
   if ((a.max_entries + kItemRows - 1) / kItemRows * t_count > INT32_MAX) return false;
   if (a.keys.page_table != nullptr && a.keys.page_size % kBoxRows != 0) return false;
   if (a.keys.n_rows > INT32_MAX || a.T * a.H_I > INT32_MAX) return false;
@@ -838,12 +877,16 @@ cudaError_t launch_indexer_scores_tc_prefill(const Launch& L, const IndexerArgs&
   return L.end(kKernelIndexerScore);
 }
 
-cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int64_t t_count) {
+namespace {
+
+template <int CI, int NH>
+cudaError_t launch_score_tc(const Launch& L, const IndexerArgs& a, int64_t t_count) {
+  using Cfg = ScoreCfg<CI, NH>;
   CUtensorMap tk, tq;
   const uint32_t box_rows = a.keys.page_table == nullptr ? kItemRows : kBoxRows;
-  if (!make_tmap_bf16_2d(&tk, a.keys.data, 64, (uint64_t)a.keys.n_rows, 64, 64, box_rows))
+  if (!make_tmap_bf16_2d(&tk, a.keys.data, CI, (uint64_t)a.keys.n_rows, CI, 64, box_rows))
     return cudaErrorInvalidValue;
-  if (!make_tmap_bf16_2d(&tq, a.q_idx, 64, (uint64_t)(a.T * a.H_I), 64, 64, 16))
+  if (!make_tmap_bf16_2d(&tq, a.q_idx, CI, (uint64_t)(a.T * a.H_I), CI, 64, NH))
     return cudaErrorInvalidValue;
   TcIndexerParams p;
   p.a = a;
@@ -851,13 +894,26 @@ cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int6
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t grid = sms;
-  const int smem = kStages * (kStageKeyBytes + kQTileBytes) + 1024;
+  cudaFuncSetAttribute(indexer_score_tc_kernel<CI, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       Cfg::kSmem);
+  prefer_max_shared(indexer_score_tc_kernel<CI, NH>);
+  return launch_kernel(indexer_score_tc_kernel<CI, NH>, dim3((unsigned)sms), dim3(kThreads),
+                       (size_t)Cfg::kSmem, L.stream, true, tk, tq, p);
+}
+
+}  // namespace
+
+cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int64_t t_count) {
   L.begin(kKernelIndexerScore);
-  cudaFuncSetAttribute(indexer_score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  prefer_max_shared(indexer_score_tc_kernel);
-  cudaError_t e = launch_kernel(indexer_score_tc_kernel, dim3((unsigned)grid), dim3(kThreads),
-                                (size_t)smem, L.stream, true, tk, tq, p);
+  const int nh = a.H_I <= 16 ? 16 : a.H_I <= 32 ? 32 : 64;
+  cudaError_t e = cudaSuccess;
+  if (a.c_I == 64) {
+    e = nh == 16 ? launch_score_tc<64, 16>(L, a, t_count)
+        : nh == 32 ? launch_score_tc<64, 32>(L, a, t_count) : launch_score_tc<64, 64>(L, a, t_count);
+  } else {
+    e = nh == 16 ? launch_score_tc<128, 16>(L, a, t_count)
+        : nh == 32 ? launch_score_tc<128, 32>(L, a, t_count) : launch_score_tc<128, 64>(L, a, t_count);
+  }
   if (e != cudaSuccess) return e;
   return L.end(kKernelIndexerScore);
 }

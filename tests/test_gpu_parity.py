@@ -115,11 +115,13 @@ def test_norm_rope_output_derotation_in_place():
     assert torch.equal(got[:, :, :64].cpu(), o[:, :, :64])
 
 
-@pytest.mark.parametrize("overlap,paged,dim", [(True, False, 128), (False, True, 128), (True, True, 64)])
+@pytest.mark.parametrize("overlap,paged,dim", [(True, False, 128), (False, True, 128), (True, True, 64),
+                                              (True, True, 512), (False, False, 512)])
 def test_cache_append_matches_bulk_compression(overlap, paged, dim):
     """Decode-time appends, one token per sequence per call: entry for entry the
     bits of csa_compress_kv on the whole sequence, within tolerance of the
-    oracle's DecodeCacheState, and the window ring holds the last W raw rows."""
+    oracle's DecodeCacheState, and the window ring holds the last W raw rows.
+    dim 512 is the pages' compressed-entry width c."""
     csa = _csa()
     g = synth.generator(140 + dim + int(overlap) + 2 * int(paged))
     B, N, m, W = 3, 37, 4, 16
@@ -213,10 +215,12 @@ def test_indexer_topk_decode_ragged(H_I, c_I, wdist):
                    range(B), sc)
 
 
-@pytest.mark.parametrize("H_I,c_I,k", [(8, 64, 512), (64, 128, 256), (12, 64, 2048), (4, 64, 64)])
+@pytest.mark.parametrize("H_I,c_I,k", [(8, 64, 512), (64, 128, 256), (12, 64, 2048), (4, 64, 64),
+                                       (64, 128, 512), (64, 128, 1024), (32, 128, 2048)])
 def test_indexer_topk_decode_sampled_threshold(H_I, c_I, k):
     """Contexts long enough (more than 4096 eligible entries) for the sampled
-    threshold: the selection comes from the candidate lists; scores too."""
+    threshold: the selection comes from the candidate lists; scores too.
+    H_I = 64 heads of c_I = 128 with k in {512, 1024} is the pages' indexer."""
     csa = _csa()
     g = synth.generator(35 + H_I + c_I + k)
     m = 4

@@ -383,7 +383,7 @@ cudaError_t launch_merge(const Launch& L, const AttnArgs& a) {
 
 bool attention_uses_tc(const AttnArgs& a) {
   const int32_t choice = attention_kernel_choice();
-  return choice != 2 && !a.kv_fp8 && tc_attention_supported(a);
+  return choice != 2 && tc_attention_supported(a);
 }
 
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {

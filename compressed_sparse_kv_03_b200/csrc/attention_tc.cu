@@ -33,6 +33,7 @@
 #include <cmath>
 
 #include "kernels.h"
+#include "lowprec.cuh"
 #include "tc.cuh"
 
 namespace csa {
@@ -213,6 +214,67 @@ __device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, int la
   return ok;
 }
 
+// Producer gather of mixed-precision entries (kept out of line: its registers
+// stay off the bf16 path).  Lane (c = lane & 15, sub = lane >> 4) handles
+// chunk c of row 2 (pk + kProducerWarps j) + sub of each of the warp's pairs
+// j; `row` is lane l's physical row for pair l >> 1 (or -1).  Chunk c < dc8
+// is 8 E4M3 codes and the scale byte of their block, expanded exactly to bf16
+// and stored in the chunk's swizzled place (zeros for a missing row, as the
+// zero fill of a bf16 row); the rotary chunks arrive by cp.async.  A few rows
+// at a time: their loads are all issued before the first expansion.
+__device__ __noinline__ void gather_fp8_rows(const uint8_t* codes, const uint8_t* scales,
+                                             const __nv_bfloat16* rope, int rope_dims, uint32_t cdst,
+                                             int64_t row, int my_pairs, int pk, int lane) {
+  constexpr int kJ = (kRows / 2 + kProducerWarps - 1) / kProducerWarps;
+  constexpr int kFB = 4;   // rows per load batch
+  const int c = lane & 15, sub = lane >> 4;
+  const int dc8 = (kD - rope_dims) / 8;
+#pragma unroll
+  for (int j0 = 0; j0 < kJ; j0 += kFB) {
+    uint2 cw[kFB];
+    uint32_t sbyte[kFB];
+#pragma unroll
+    for (int u = 0; u < kFB; ++u) {
+      const int j = j0 + u;
+      cw[u] = make_uint2(0u, 0u);
+      sbyte[u] = 0u;
+      const int64_t rr = __shfl_sync(0xffffffffu, row, (2 * j + sub) & 31);
+      if (j < kJ && j < my_pairs) {
+        const int r = 2 * (pk + kProducerWarps * j) + sub;
+        if (c < dc8) {
+          if (rr >= 0) {
+            cw[u] = __ldg(reinterpret_cast<const uint2*>(codes + rr * (8 * dc8) + 8 * c));
+            sbyte[u] = __ldg(scales + rr * (dc8 / 4) + (c >> 2));
+          }
+        } else {
+          cp_async_16(cdst + (uint32_t)r * 128 + (uint32_t)((((c & 7) ^ (r & 7)) & 7) << 4),
+                      rope + (rr >= 0 ? rr : 0) * rope_dims + (c - dc8) * 8, rr >= 0);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kFB; ++u) {
+      const int j = j0 + u;
+      if (j < kJ && j < my_pairs && c < dc8) {
+        const int r = 2 * (pk + kProducerWarps * j) + sub;
+        const float fs = lowprec::e8m0_to_float(sbyte[u]);
+        const uint32_t w2[2] = {cw[u].x, cw[u].y};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t wd = w2[q >> 1] >> (16 * (q & 1));
+          o[q] = pack_bf16(lowprec::e4m3_to_float(wd & 0xffu) * fs,
+                           lowprec::e4m3_to_float((wd >> 8) & 0xffu) * fs);
+        }
+        const uint32_t addr = cdst + (uint32_t)r * 128 + (uint32_t)((((c & 7) ^ (r & 7)) & 7) << 4);
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(o[0]), "r"(o[1]),
+                     "r"(o[2]), "r"(o[3])
+                     : "memory");
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
                const __grid_constant__ CUtensorMap tm_win,
@@ -335,7 +397,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         const uint32_t dst = kv_sm + slot * kKvTile;
         const uint32_t fb = smem_u32(&kv_full[slot]);
         const bool sel = t < it.n_sel_tiles;
-        if (sel && (a.idx != nullptr || a.kv.page_table != nullptr)) {
+        if (sel && (a.idx != nullptr || a.kv.page_table != nullptr || a.kv_fp8)) {
           const bool mine = lane_has_row && my_row < n;
           const int64_t e = have_next ? e_next
                                       : (!mine ? -1 : (a.idx ? (int64_t)__ldg(a.idx + it.i * a.top_k + v + my_row)
@@ -354,15 +416,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
           if (lane == 0) row_ok[slot][pk] = okb;
           const int c = lane & 15, sub = lane >> 4;
           const uint32_t cdst = dst + (c >> 3) * kKBlock;
+          constexpr int kJ = (kRows / 2 + kProducerWarps - 1) / kProducerWarps;
+          if (!a.kv_fp8) {
 #pragma unroll
-          for (int j = 0; j < (kRows / 2 + kProducerWarps - 1) / kProducerWarps; ++j) {
-            if (j < my_pairs) {
-              const int64_t rr = __shfl_sync(0xffffffffu, row, 2 * j + sub);
-              const int r = 2 * (pk + kProducerWarps * j) + sub;
-              const char* src = reinterpret_cast<const char*>(a.kv.data + (rr >= 0 ? rr : 0) * kD) + c * 16;
-              cp_async_16(cdst + (uint32_t)r * 128 + (uint32_t)((((c & 7) ^ (r & 7)) & 7) << 4), src,
-                          rr >= 0);
+            for (int j = 0; j < kJ; ++j) {
+              if (j < my_pairs) {
+                const int64_t rr = __shfl_sync(0xffffffffu, row, 2 * j + sub);
+                const int r = 2 * (pk + kProducerWarps * j) + sub;
+                const char* src = reinterpret_cast<const char*>(a.kv.data + (rr >= 0 ? rr : 0) * kD) + c * 16;
+                cp_async_16(cdst + (uint32_t)r * 128 + (uint32_t)((((c & 7) ^ (r & 7)) & 7) << 4), src,
+                            rr >= 0);
+              }
             }
+          } else {
+            gather_fp8_rows(reinterpret_cast<const uint8_t*>(a.kv.data), a.kv_scales, a.kv_rope,
+                            a.rope_dims, cdst, row, my_pairs, pk, lane);
+            fence_async_smem();   // the MMAs read the expanded rows through the async proxy
           }
           cp_async_mbar_arrive_noinc(fb);
           __syncwarp();
@@ -834,7 +903,10 @@ bool tc_attention_supported(const AttnArgs& a) {
 cudaError_t launch_attention_tc(const Launch& L, const AttnArgs& a) {
   CUtensorMap t, w, q;
   const uint64_t kv_rows = (uint64_t)a.kv.n_rows;
-  if (!make_tmap_bf16_2d(&t, a.kv.data, kD, kv_rows, kD, 64, kRows)) return cudaErrorInvalidValue;
+  // (mixed-precision entries are always gathered: no tile of them is a box)
+  if (!make_tmap_bf16_2d(&t, a.kv_fp8 ? (const void*)a.q : (const void*)a.kv.data, kD,
+                         a.kv_fp8 ? (uint64_t)(a.T * a.H) : kv_rows, kD, 64, kRows))
+    return cudaErrorInvalidValue;
   const uint64_t win_rows = a.win_len ? (uint64_t)(a.T * a.window) : (uint64_t)a.win_rows;
   if (a.window > 0 && win_rows > 0) {
     if (!make_tmap_bf16_2d(&w, a.win, kD, win_rows, kD, 64, kRows)) return cudaErrorInvalidValue;

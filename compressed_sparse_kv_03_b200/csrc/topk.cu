@@ -221,6 +221,34 @@ __device__ uint32_t sample_threshold(const uint32_t* skey, int ns, int64_t n, in
   return prefix;
 }
 
+// The same threshold for ns <= kWarpSample keys, by one warp without
+// shared-memory histograms or block barriers: the keys go to registers (32
+// per lane) and a bitwise radix select walks bits 31 .. 10 from the top, each
+// step counting the keys of the current prefix group that have the bit set.
+constexpr int kWarpSample = 1024;
+__device__ uint32_t warp_sample_threshold(const uint32_t* skey, int ns, int64_t n, int top_k) {
+  const double mu = (double)ns * (double)top_k / (double)n;
+  const int64_t r = (int64_t)ceil(mu + 6.0 * sqrt(mu) + 8.0);
+  if (r >= ns) return 0u;
+  const int lane = threadIdx.x & 31;
+  uint32_t kv[kWarpSample / 32];
+#pragma unroll
+  for (int i = 0; i < kWarpSample / 32; ++i) kv[i] = 32 * i + lane < ns ? skey[32 * i + lane] : 0u;
+  uint32_t prefix = 0u;
+  int need = (int)r;
+#pragma unroll 1
+  for (int bit = 31; bit >= 10; --bit) {
+    const uint32_t want = (prefix >> bit) | 1u;
+    int cnt = 0;
+#pragma unroll
+    for (int i = 0; i < kWarpSample / 32; ++i) cnt += (32 * i + lane < ns && (kv[i] >> bit) == want) ? 1 : 0;
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (cnt >= need) prefix |= 1u << bit;
+    else need -= cnt;
+  }
+  return prefix;
+}
+
 // Sampled entries: ns = max(1024, n/32) (at most n, a multiple of 16), as
 // ns / 16 groups of 16 consecutive entries, group i starting at i n / (ns/16).
 __device__ __forceinline__ int sample_size(int64_t n) {
@@ -260,7 +288,9 @@ __global__ void __launch_bounds__(kSampleThreads) topk_sample_kernel(IndexerArgs
   }
   const int ns = sample_size(n);
   const int ng = ns / 16;
-  for (int b = threadIdx.x; b < 2048; b += kSampleThreads) hist[b] = 0;
+  const bool by_warp = ns <= kWarpSample;   // the common case: one warp sets tau
+  if (!by_warp)
+    for (int b = threadIdx.x; b < 2048; b += kSampleThreads) hist[b] = 0;
   __syncthreads();
   for (int g0 = warp * kU; g0 < ng; g0 += (kSampleThreads / 32) * kU) {
     uint4 kr[kU][2][CI / 32];
@@ -285,11 +315,18 @@ __global__ void __launch_bounds__(kSampleThreads) topk_sample_kernel(IndexerArgs
       if (grp < ng && q4 < 2) {
         const uint32_t key = score_key(q4 == 0 ? sg : s8);
         skey[grp * 16 + g + 8 * q4] = key;
-        atomicAdd(&hist[key >> 21], 1);   // the first radix level
+        if (!by_warp) atomicAdd(&hist[key >> 21], 1);   // the first radix level
       }
     }
   }
   __syncthreads();
+  if (by_warp) {
+    if (warp == 0) {
+      const uint32_t tau = warp_sample_threshold(skey, ns, n, top_k);
+      if (lane == 0) const_cast<uint32_t*>(a.tau)[tl] = tau;
+    }
+    return;
+  }
   const uint32_t tau = sample_threshold<kSampleThreads>(skey, ns, n, top_k, hist, warp_sums, &s_bin,
                                                         &s_above, &s_ok, true);
   if (threadIdx.x == 0) const_cast<uint32_t*>(a.tau)[tl] = tau;
@@ -329,6 +366,13 @@ __global__ void __launch_bounds__(kSampleThreads) topk_sample_fp4_kernel(Indexer
     skey[j] = score_key(entry_score<CI>(a, qs, ws, row));
   }
   __syncthreads();
+  if (ns <= kWarpSample) {
+    if (threadIdx.x < 32) {
+      const uint32_t tau = warp_sample_threshold(skey, ns, n, top_k);
+      if (threadIdx.x == 0) const_cast<uint32_t*>(a.tau)[tl] = tau;
+    }
+    return;
+  }
   const uint32_t tau =
       sample_threshold<kSampleThreads>(skey, ns, n, top_k, hist, warp_sums, &s_bin, &s_above, &s_ok);
   if (threadIdx.x == 0) const_cast<uint32_t*>(a.tau)[tl] = tau;

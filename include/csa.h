@@ -465,8 +465,11 @@ csa_status_t csa_quantize_entries_fp8(const csa_bf16* x, int64_t n, int32_t dim,
  *   kv_scales  [kv_codes->n_rows, (128 - rope_dims)/32] uint8
  *   kv_rope    [kv_codes->n_rows, rope_dims] bf16 (16-byte aligned), or NULL when
  *              rope_dims == 0; row r of each array belongs to physical row r
- * d = 128; rope_dims a multiple of 8 with 128 - rope_dims a multiple of 32.  Runs
- * on the mma.sync attention kernel whatever csa_set_attention_kernel says.
+ * d = 128; rope_dims a multiple of 8 with 128 - rope_dims a multiple of 32.  The
+ * attention kernel follows csa_set_attention_kernel: the tcgen05 kernel's
+ * producer warps (or the mma.sync kernel's gather) expand each entry's codes
+ * exactly to bf16 in shared memory, so the result equals that kernel's over a
+ * bf16 cache holding the dequantized entries, bit for bit.
  */
 csa_status_t csa_sparse_attn_decode_fp8(const csa_bf16* q, const csa_cache_t* kv_codes,
                                         const uint8_t* kv_scales, const csa_bf16* kv_rope,

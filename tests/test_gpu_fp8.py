@@ -88,6 +88,16 @@ def _decode_case(g, B, H, k, paged, rope):
     return q, win, win_len, idx, cnt, seq_rows, store
 
 
+@pytest.fixture(params=["tcgen05", "mma_sync"])
+def attn_kernel(request):
+    """Run an attention test once per attention kernel."""
+    csa = _csa()
+    csa.set_attention_kernel(request.param)
+    yield request.param
+    csa.set_attention_kernel("auto")
+
+
+@pytest.mark.usefixtures("attn_kernel")
 @pytest.mark.parametrize("B,H,k,paged,sink,rope", [(5, 64, 2048, False, False, 64),
                                                    (3, 64, 300, True, True, 64),
                                                    (2, 20, 500, False, True, 32),
@@ -116,14 +126,15 @@ def test_sparse_attn_decode_fp8(B, H, k, paged, sink, rope):
         np.testing.assert_allclose(f64(lse[b]), ref_lse, atol=1e-3, rtol=1e-4)
 
 
-def test_sparse_attn_decode_fp8_equals_bf16_on_dequantized_cache():
+@pytest.mark.parametrize("paged", [False, True])
+def test_sparse_attn_decode_fp8_equals_bf16_on_dequantized_cache(attn_kernel, paged):
     """The expansion is exact: attention over the stored entries equals the
-    bf16 kernel over a bf16 cache holding the dequantized entries, bit for bit
-    (both on the mma.sync kernel)."""
+    same kernel's over a bf16 cache holding the dequantized entries, bit for
+    bit (tcgen05: expanded by its producer warps; mma.sync: by its gather)."""
     csa = _csa()
     g = synth.generator(760)
     B, H, k = 4, 64, 600
-    q, win, win_len, idx, cnt, seq_rows, store = _decode_case(g, B, H, k, False, 64)
+    q, win, win_len, idx, cnt, seq_rows, store = _decode_case(g, B, H, k, paged, 64)
     c_np, s_np, r_np = ofp8.entry_quantize(f64(store["data"]), 64)   # the oracle's storage
     deq = ofp8.entry_dequantize(c_np, s_np, r_np)
     deq_bf16 = torch.from_numpy(deq).to(torch.bfloat16)
@@ -132,14 +143,12 @@ def test_sparse_attn_decode_fp8_equals_bf16_on_dequantized_cache():
     scales = dev(torch.from_numpy(s_np))
     rp = dev(torch.from_numpy(r_np).to(torch.bfloat16))
     lam = 1 / math.sqrt(128)
-    a = csa.sparse_attn_decode_fp8(dev(q), csa.Cache(codes, seq_stride=store["seq_stride"]), scales,
-                                   rp, dev(win), dev(win_len), dev(idx), dev(cnt), lam)
-    csa.set_attention_kernel("mma_sync")
-    try:
-        b_ = csa.sparse_attn_decode(dev(q), csa.Cache(dev(deq_bf16), seq_stride=store["seq_stride"]),
-                                    dev(win), dev(win_len), dev(idx), dev(cnt), lam)
-    finally:
-        csa.set_attention_kernel("auto")
+    lay = dict(seq_stride=store.get("seq_stride", 0), page_table=dev(store.get("page_table")),
+               page_size=store.get("page_size", 0))
+    a = csa.sparse_attn_decode_fp8(dev(q), csa.Cache(codes, **lay), scales, rp, dev(win), dev(win_len),
+                                   dev(idx), dev(cnt), lam)
+    b_ = csa.sparse_attn_decode(dev(q), csa.Cache(dev(deq_bf16), **lay), dev(win), dev(win_len),
+                                dev(idx), dev(cnt), lam)
     assert torch.equal(a, b_)
 
 

@@ -49,8 +49,9 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Indexer workspace: header | per query tau, candidate count and fallback
 // list entry [3][chunk] u32 + the fallback count | work counter | candidates
-// [chunk, cap] (key, entry) pairs | in many-query mode the sampled keys
-// [chunk, kPSampleKeys] u32.  O(top_k) per query: no score matrix is stored.
+// [chunk, cap] (key, entry) pairs | sampled keys [chunk, kPSampleKeys] u32 (the
+// tensor-core scorers' sample passes).  O(top_k) per query: no score matrix
+// is stored.
 // Queries are processed in chunks so that the scratch stays bounded.
 struct IndexerLayout {
   bool many;
@@ -70,7 +71,7 @@ IndexerLayout indexer_layout(int64_t T, int64_t max_entries, int32_t top_k) {
   IndexerLayout l;
   l.many = T > kFusedMaxQueries && max_entries <= kManyMaxEntries;
   l.cap = candidate_cap(top_k);
-  const int64_t per_query = l.cap * 8 + 12 + (l.many ? kPSampleKeys * 4 : 0);
+  const int64_t per_query = l.cap * 8 + 12 + kPSampleKeys * 4;
   int64_t c = (int64_t)(kIndexerChunkBytes / per_query);
   if (c > 65535) c = 65535;
   if (!l.many && c > kFusedMaxQueries) c = kFusedMaxQueries;
@@ -82,7 +83,7 @@ IndexerLayout indexer_layout(int64_t T, int64_t max_entries, int32_t top_k) {
   l.counter_off = l.meta_off + align256(((size_t)l.chunk * 3 + 1) * sizeof(uint32_t));
   l.data_off = l.counter_off + 256;
   l.sample_off = l.data_off + align256((size_t)l.chunk * l.cap * 8);
-  l.total = l.sample_off + (l.many ? align256((size_t)l.chunk * kPSampleKeys * 4) : 0);
+  l.total = l.sample_off + align256((size_t)l.chunk * kPSampleKeys * 4);
   return l;
 }
 
@@ -451,18 +452,35 @@ csa_status_t run_indexer_topk(IndexerArgs base, const int64_t* q_pos, int64_t T,
     ia.cand = reinterpret_cast<uint2*>(wsb + lay.data_off);
     ia.cand_cap = lay.cap;
     ia.skip_le = score_out ? 0 : top_k;   // scores of all-selected queries still come from the scorer
-    ia.psample = lay.many ? reinterpret_cast<uint32_t*>(wsb + lay.sample_off) : nullptr;
-    if (ia.psample && tc_indexer_prefill_supported(ia, n) && topk_many_supported(ia)) {
+    ia.psample = reinterpret_cast<uint32_t*>(wsb + lay.sample_off);
+    if (lay.many && tc_indexer_prefill_supported(ia, n) && topk_many_supported(ia)) {
       // the scorer's sample pass, thresholds (which zero the counts and the
       // work counter), the scorer's candidate pass, per-warp finish
       e = cudaMemsetAsync(work, 0, sizeof(uint32_t), L.stream);
       if (e != cudaSuccess) return cuda_status(e, "indexer work counter memset");
       if ((e = launch_indexer_scores_tc_prefill(L, ia, n, true)) != cudaSuccess)
         return cuda_status(e, "indexer sample launch");
-      if ((e = launch_topk_threshold_many(L, ia, top_k, n)) != cudaSuccess)
+      if ((e = launch_topk_threshold_many(L, ia, top_k, n, 128 / ia.H_I)) != cudaSuccess)
         return cuda_status(e, "top-k threshold launch");
       if ((e = launch_indexer_scores(L, ia, n)) != cudaSuccess) return cuda_status(e, "indexer score launch");
       if ((e = launch_topk_finish_many(L, ia, top_k, idx_out, count_out, score_out, n)) != cudaSuccess)
+        return cuda_status(e, "top-k finish launch");
+    } else if (tc_fp4_indexer_supported(ia, n)) {
+      // 4-bit keys on the block-scaled tensor cores: the queries' operand
+      // images (in the tail of the candidate area, whose per-query stride
+      // shrinks by kFp4ImgSlots; this launch also zeroes the work counter),
+      // the scorer's sample pass (whole chunks per query), one-warp
+      // thresholds, its candidate pass
+      ia.cand_cap = lay.cap - kFp4ImgSlots;
+      ia.q_img = reinterpret_cast<uint8_t*>(wsb + lay.data_off) + (size_t)lay.chunk * (size_t)ia.cand_cap * 8;
+      if ((e = launch_fp4_query_images(L, ia, n)) != cudaSuccess) return cuda_status(e, "query image launch");
+      if ((e = launch_indexer_scores_fp4_tc(L, ia, n, true)) != cudaSuccess)
+        return cuda_status(e, "indexer sample launch");
+      if ((e = launch_topk_threshold_many(L, ia, top_k, n, 1)) != cudaSuccess)
+        return cuda_status(e, "top-k threshold launch");
+      if ((e = launch_indexer_scores_fp4_tc(L, ia, n, false)) != cudaSuccess)
+        return cuda_status(e, "indexer score launch");
+      if ((e = launch_topk_finish(L, ia, top_k, idx_out, count_out, score_out, n)) != cudaSuccess)
         return cuda_status(e, "top-k finish launch");
     } else {
       ia.psample = nullptr;

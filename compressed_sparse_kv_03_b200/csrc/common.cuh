@@ -197,6 +197,27 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
     if (clock64() - t0 > limit_cycles) return false;
   return true;
 }
+// Same, with a suspend-time hint: a waiting thread is parked until the phase
+// completes (or the hint, in ns, runs out) instead of polling, so it takes no
+// issue slots or shared-memory bandwidth from the threads doing the work.
+__device__ __forceinline__ bool mbar_try_wait_susp(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_susp(uint32_t bar, uint32_t parity,
+                                               long long limit_cycles = 2000000000ll) {
+  if (mbar_try_wait_susp(bar, parity, 100000u)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait_susp(bar, parity, 100000u))
+    if (clock64() - t0 > limit_cycles) return false;
+  return true;
+}
 // Same, backing off with nanosleep between polls: for waiters that are not on
 // the critical path, so that they leave issue slots to the producer threads.
 __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, unsigned ns = 256,
@@ -208,6 +229,11 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, u
     __nanosleep(ns);
   }
   return true;
+}
+// Orders this thread's generic-proxy shared-memory writes before later reads
+// by the async proxy (TMA, tcgen05.mma / tcgen05.cp operands).
+__device__ __forceinline__ void fence_async_smem_cta() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 // global -> shared bulk copy completing on an mbarrier (both addresses 16-byte
 // aligned, size a multiple of 16)

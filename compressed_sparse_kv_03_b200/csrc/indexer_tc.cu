@@ -27,6 +27,7 @@
 // through a 16-entry ring with its own full / empty barriers.  Every wait is
 // bounded; a timeout is reported in the workspace header.
 #include "kernels.h"
+#include "lowprec.cuh"
 #include "tc.cuh"
 
 namespace csa {
@@ -818,6 +819,569 @@ indexer_score_tc_prefill_kernel(const __grid_constant__ CUtensorMap tmap_keys,
   if (warp == 1) tc::tmem_dealloc(tmem_base, kPTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// 4-bit keys (few-query mode): the same persistent pipeline as the bf16
+// decode scorer, on block-scaled tensor-core MMAs
+// (tcgen05.mma.kind::mxf4.block_scale, M = 128 keys, K = 64 per instruction):
+// the tensor cores apply both scales, so TMEM holds the exact scaled dot
+// products.  An item's key codes (E2M1, 32 bytes per 64-dim block) and scale
+// bytes arrive by 1-D bulk copies (a TMA box of 32-byte rows streams at a
+// fraction of the rate).  The MMA reads operands in the 32-byte-swizzled
+// K-major layout, where rows 4..7 of every 8 have their two 16-byte halves
+// exchanged:
+//  * 64-dim keys land as stored and are read as if swizzled, so those rows
+//    reach the MMA with halves exchanged; the B operand holds every head twice,
+//    as stored (columns 0 .. NH) and with halves exchanged (NH .. 2 NH), each
+//    key's scale bytes are exchanged to match, and the epilogue takes each row's
+//    dot products from the copy that pairs its halves correctly;
+//  * 128-dim keys are moved into the swizzled layout by the MMA warp's lanes.
+// The producer warp quantizes each query's heads (the block quantizer of
+// csa_quantize_mxfp4) once and writes them, with their scale bytes, into the
+// stage; the MMA warp arranges the keys' scale bytes in the layout tcgen05.cp
+// moves to TMEM and one lane issues the MMAs.  The epilogue is the bf16
+// scorer's.  A sample mode (MODE kFp4Sample) scores only psample_chunks whole
+// chunks of each query and writes their keys to psample.
+// ---------------------------------------------------------------------------
+constexpr int kFp4Sample = 1, kFp4Fused = 2;
+constexpr int kFMinItem = 256;                 // the smallest item (keys) of any shape
+
+template <int CI, int NH, bool SAMPLE>
+struct Fp4Cfg {
+  static constexpr bool kSwap = CI == 64;                 // codes used as stored (see above)
+  static constexpr int kN = kSwap ? 2 * NH : NH;          // MMA N: B rows
+  // keys per item (128-key tiles): as many as TMEM holds accumulators for
+  // (the per-item work of the producer and MMA warps is mostly fixed); the
+  // sample pass takes 256-key chunks
+  static constexpr int kItem = SAMPLE || !kSwap ? 256 : kN <= 32 ? 1024 : kN == 64 ? 512 : 256;
+  static constexpr int kTiles = kItem / kTileRows;
+  static constexpr int kKB = CI / 64;                     // 64-element blocks per key (one MMA each)
+  static constexpr int kCodeBlk = kItem * 32;             // one block of an item's key codes
+  static constexpr int kCodes = kKB * kCodeBlk;
+  static constexpr int kQBlk = kN * 32;
+  static constexpr int kQCodes = kKB * kQBlk;
+  static constexpr int kRawSc = kItem * (CI / 32);        // the keys' scale bytes as stored
+  static constexpr int kSfa = kTiles * kKB * 512;         // per (tile, block): 32 rows x 16 B
+  static constexpr int kSfb = kKB * 512;
+  // a query's operand image (B codes, then its SFB blocks): one bulk copy
+  static constexpr int kQImg = kQCodes + kSfb;
+  static constexpr int kQOff = kCodes;
+  static constexpr int kSfbOff = kQOff + kQCodes;
+  static constexpr int kRawOff = kSfbOff + kSfb;
+  static constexpr int kSfaOff = kRawOff + kRawSc;
+  // where the copied codes land: the operand itself (kSwap), else a staging area
+  static constexpr int kRawCodes = kSwap ? 0 : kItem * (CI / 2);
+  static constexpr int kRawCOff = kSwap ? 0 : (kSfaOff + kSfa + 127) / 128 * 128;
+  static constexpr int kStage = ((kSwap ? kSfaOff + kSfa : kRawCOff + kRawCodes) + 1023) / 1024 * 1024;
+  static constexpr int kStages = (200 * 1024) / kStage < 8 ? (200 * 1024) / kStage : 8;
+  static constexpr int kAccCols = kTiles * kN;
+  static constexpr int kSfCols = 4 * (kTiles + 1) * kKB;  // per set: SFA kTiles x kKB, SFB kKB, 4 columns each
+  static constexpr int kAccF = 2 * (kAccCols + kSfCols) <= 512 ? 2 : 1;   // accumulator sets
+  static constexpr int kSfBase = kAccF * kAccCols;
+  static constexpr int kTmemCols = 512;
+  static constexpr uint32_t kIdesc = tc::idesc_mxf4(128, kN);
+  static constexpr int kSmem = kStages * kStage + 1024;
+  static_assert(kN % 16 == 0 && kN <= 128 && NH >= 8, "MMA N");
+  static_assert(kQImg <= kFp4ImgSlots * 8, "query image");
+  static_assert(kSfBase + kAccF * kSfCols <= kTmemCols, "TMEM columns");
+};
+
+// An item's rows in 64-row runs (pages, or the end of a contiguous cache):
+// lane 0 sets the barrier's byte count and issues bulk copies of the codes
+// (any row count) and of the scale bytes of whole multiples of 8 rows; lanes
+// 1 .. 31 load a run's last (rows mod 8) scale bytes themselves.  Rows past
+// the cache's end are not copied (they are never scored valid).
+template <int CI, int ITEM>
+__device__ __noinline__ void fp4_copy_runs(CacheRef keys, const uint8_t* k_scales, WsHeader* err,
+                                           uint32_t codes_sm, uint32_t scales_sm, uint8_t* scales_p,
+                                           uint32_t fb, int32_t seq, int64_t s0, int64_t n_cur, int32_t t,
+                                           int lane) {
+  constexpr int kRuns = ITEM / kBoxRows, cb = CI / 2, nsc = CI / 32;
+  const uint8_t* const kc = reinterpret_cast<const uint8_t*>(keys.data);
+  int64_t row0[kRuns];
+  int nrow[kRuns];
+  uint32_t bytes = 0;
+#pragma unroll
+  for (int hb = 0; hb < kRuns; ++hb) {
+    const int64_t s = s0 + hb * kBoxRows;
+    int64_t row;
+    if (keys.page_table == nullptr) {
+      row = (int64_t)seq * keys.seq_stride + s;
+    } else {
+      const int64_t pi = s / keys.page_size;
+      const int32_t page = pi < keys.max_pages ? __ldg(keys.page_table + (int64_t)seq * keys.max_pages + pi) : -1;
+      row = (int64_t)page * keys.page_size + (s - pi * keys.page_size);
+      if (page < 0 || row >= keys.n_rows) {
+        if (lane == 0 && s < n_cur) report(err, kErrPageId, t, page);
+        row = 0;
+      }
+    }
+    int64_t nr = keys.n_rows - row;
+    nr = nr < 0 ? 0 : (nr > kBoxRows ? kBoxRows : nr);
+    row0[hb] = row;
+    nrow[hb] = (int)nr;
+    bytes += (uint32_t)(nrow[hb] * cb + (nrow[hb] & ~7) * nsc);
+  }
+  if (lane == 0) {
+    mbar_arrive_expect_tx(fb, bytes);
+#pragma unroll
+    for (int hb = 0; hb < kRuns; ++hb) {
+      if (nrow[hb] > 0)
+        bulk_g2s(codes_sm + hb * kBoxRows * cb, kc + row0[hb] * cb, (uint32_t)(nrow[hb] * cb), fb);
+      if ((nrow[hb] & ~7) > 0)
+        bulk_g2s(scales_sm + hb * kBoxRows * nsc, k_scales + row0[hb] * nsc, (uint32_t)((nrow[hb] & ~7) * nsc), fb);
+    }
+  } else {
+    bool wrote = false;
+    const int sl = lane - 1;
+#pragma unroll
+    for (int hb = 0; hb < kRuns; ++hb) {
+      const int nb = nrow[hb] & ~7;
+      if (sl < (nrow[hb] - nb) * nsc) {
+        const int r = nb + sl / nsc, jj = sl % nsc;
+        scales_p[(hb * kBoxRows + r) * nsc + jj] = k_scales[(row0[hb] + r) * nsc + jj];
+        wrote = true;
+      }
+    }
+    if (wrote) fence_async_smem_cta();
+  }
+}
+
+// One warp per query: the block quantizer of csa_quantize_mxfp4 on each head
+// (zero codes for the padded heads), then the stage image of the MMA's B
+// operand: B row r = head r mod NH (rows NH .. 2 NH with halves exchanged when
+// kSwap) in the K-major 32-byte swizzle, and the SFB blocks in the tcgen05.cp
+// layout (row r at byte 4 (r / 32) + k of row r mod 32).
+template <int CI, int NH>
+__global__ void __launch_bounds__(128) fp4_query_image_kernel(IndexerArgs a, int64_t t_count) {
+  using Cfg = Fp4Cfg<CI, NH, false>;
+  __shared__ __align__(16) uint8_t codes[4][NH * CI / 2];
+  __shared__ uint8_t sfs[4][NH * CI / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.work = 0u;
+  const int64_t tl = (int64_t)blockIdx.x * 4 + warp;
+  if (tl >= t_count) return;
+  const int64_t t = a.t_begin + tl;
+  for (int b = lane; b < NH * (CI / 32); b += 32) {
+    const int h = b / (CI / 32), v = b - h * (CI / 32);
+    uint32_t w4[4] = {0u, 0u, 0u, 0u};
+    uint32_t sb = 0u;
+    if (h < a.H_I) sb = lowprec::quantize_block(a.q_idx + (t * a.H_I + h) * CI + 32 * v, w4);
+    *reinterpret_cast<uint4*>(codes[warp] + h * (CI / 2) + 16 * v) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    sfs[warp][h * (CI / 32) + v] = (uint8_t)sb;
+  }
+  __syncwarp();
+  uint8_t* const img = a.q_img + tl * Cfg::kQImg;
+#pragma unroll
+  for (int kb = 0; kb < Cfg::kKB; ++kb) {
+    for (int c = lane; c < Cfg::kN * 2; c += 32) {
+      const int r = c >> 1, half = c & 1, hh = r & (NH - 1), xs = Cfg::kSwap && r >= NH;
+      *reinterpret_cast<uint4*>(img + kb * Cfg::kQBlk + r * 32 + (((half ^ (r >> 2)) & 1) << 4)) =
+          *reinterpret_cast<const uint4*>(codes[warp] + hh * (CI / 2) + kb * 32 + (half ^ xs) * 16);
+    }
+    const int m0 = lane;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int cc = 0; cc < (Cfg::kN + 31) / 32; ++cc) {
+      const int r = m0 + 32 * cc, hh = r & (NH - 1), xs = Cfg::kSwap && r >= NH;
+      if (r < Cfg::kN)
+        w[cc] = (uint32_t)sfs[warp][hh * (CI / 32) + 2 * kb + xs] |
+                ((uint32_t)sfs[warp][hh * (CI / 32) + 2 * kb + (xs ^ 1)] << 8);
+    }
+    *reinterpret_cast<uint4*>(img + Cfg::kQCodes + kb * 512 + m0 * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+template <int CI, int NH, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_score_fp4_tc_kernel(TcIndexerParams p) {
+  using Cfg = Fp4Cfg<CI, NH, MODE == kFp4Sample>;
+  constexpr int kStages = Cfg::kStages, kAccF = Cfg::kAccF;
+  const IndexerArgs& a = p.a;
+  const int T = (int)p.t_count;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t tfull_bar[kAccF], tempty_bar[kAccF];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int32_t prefix[kMaxQueries + 1];
+  __shared__ int32_t nelig[kMaxQueries];
+  __shared__ ItemMeta ring[kRing];
+  __shared__ __align__(8) uint64_t ring_full[kRing], ring_empty[kRing];
+  __shared__ __align__(16) float qc_w[NH];                    // the current query's head weights
+  __shared__ int32_t slot_q[Cfg::kStages];                   // the query whose heads a stage holds
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - smem_u32(smem_raw));
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      slot_q[i] = -1;
+      mbar_init(smem_u32(&full_bar[i]), 2);   // the copies' arrival + the query staging's
+      mbar_init(smem_u32(&empty_bar[i]), 1);
+    }
+    for (int i = 0; i < kAccF; ++i) {
+      mbar_init(smem_u32(&tfull_bar[i]), 1);
+      mbar_init(smem_u32(&tempty_bar[i]), 4);
+    }
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(smem_u32(&ring_full[i]), 1);
+      mbar_init(smem_u32(&ring_empty[i]), 5);   // the MMA warp + one epilogue group
+    }
+    mbar_fence_init();
+  }
+  if (warp == 1) tc::tmem_alloc(smem_u32(&tmem_base_sh), Cfg::kTmemCols);
+  if (warp == 0) {
+    // items per query: its chunks (fused pass) or its sampled chunks
+    const int per = (T + 31) / 32;
+    const int t0 = lane * per, t1 = min(T, t0 + per);
+    int32_t sum = 0;
+    for (int t = t0; t < t1; ++t) {
+      const int64_t pos = a.q_pos ? __ldg(a.q_pos + a.t_begin + t) : a.t_begin + t;
+      if (MODE == kFp4Fused && pos / a.m > a.max_entries && blockIdx.x == 0)
+        report(a.err, kErrEligible, (int32_t)(a.t_begin + t), pos / a.m);
+      const int64_t n = eligible(a, a.t_begin + t);
+      nelig[t] = (int32_t)n;
+      prefix[t] = MODE == kFp4Sample ? psample_chunks(n, n, a.cand_cap, a.skip_le) * 256 / Cfg::kItem
+                                     : (n <= a.skip_le ? 0 : (int32_t)((n + Cfg::kItem - 1) / Cfg::kItem));
+      sum += prefix[t];
+    }
+    int32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int32_t run = incl - sum;
+    for (int t = t0; t < t1; ++t) {
+      const int32_t c = prefix[t];
+      prefix[t] = run;
+      run += c;
+    }
+    if (lane == 31) prefix[T] = incl;
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = tmem_base_sh;
+  const int32_t V = prefix[T];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int64_t issued = 0;
+    bool ok = true;
+    const int32_t Vs = (int32_t)((int64_t)V * kStaticPct / 100);
+    const int32_t s_lo = (int32_t)((int64_t)Vs * blockIdx.x / gridDim.x);
+    const int32_t s_hi = (int32_t)((int64_t)Vs * (blockIdx.x + 1) / gridDim.x);
+    int32_t g_next = 0;
+    if (lane == 0) g_next = s_lo < s_hi ? s_lo : Vs + (int32_t)atomicAdd(a.work, (uint32_t)kGrab);
+    bool in_static = s_lo < s_hi;
+    int32_t nxt = 0, lim = 0;
+    int tq = 0, q_tq = -1;
+    int32_t q_seq = 0;
+    auto take = [&]() -> int32_t {   // lane 0's view of the item sequence
+      if (nxt >= lim) {
+        if (g_next >= V) return -1;
+        nxt = g_next;
+        if (in_static) {
+          lim = s_hi;
+          in_static = false;
+        } else {
+          lim = g_next + kGrab < V ? g_next + kGrab : V;
+        }
+        g_next = Vs + (int32_t)atomicAdd(a.work, (uint32_t)kGrab);
+        int l = 0, r = T;
+        while (r - l > 1) {
+          const int mid = (l + r) >> 1;
+          if (prefix[mid] <= nxt) l = mid; else r = mid;
+        }
+        tq = l;
+      }
+      while (prefix[tq + 1] <= nxt) ++tq;
+      return nxt++;
+    };
+    const int nsc = CI / 32;   // scale bytes per key row
+    const uint8_t* const kc = reinterpret_cast<const uint8_t*>(a.keys.data);   // CI / 2 code bytes per row
+    for (;;) {
+      int32_t item = -1;
+      if (lane == 0) item = take();
+      item = __shfl_sync(0xffffffffu, item, 0);
+      const int cur = __shfl_sync(0xffffffffu, tq, 0);
+      if (item < 0) break;
+      const int32_t sidx = item - prefix[cur];
+      const int64_t n_cur = nelig[cur];
+      const int32_t chunk = MODE == kFp4Sample
+                                ? (int32_t)(((2 * (int64_t)sidx + 1) * (n_cur / Cfg::kItem)) /
+                                            (2 * (int64_t)(prefix[cur + 1] - prefix[cur])))
+                                : sidx;
+      const int64_t t = a.t_begin + cur;
+      const int64_t s0 = (int64_t)chunk * Cfg::kItem;
+      if (cur != q_tq) {
+        for (int h = lane; h < NH; h += 32) qc_w[h] = h < a.H_I ? __ldg(a.w + t * a.H_I + h) : 0.f;
+        q_tq = cur;
+        q_seq = a.seq_id ? __ldg(a.seq_id + t) : 0;
+        __syncwarp();
+      }
+      const int32_t seq = q_seq;
+      const int rs = (int)(issued % kRing);
+      const int slot = (int)(issued % kStages);
+      bool got = true;
+      if (lane == 0) {
+        got = mbar_wait_susp(smem_u32(&ring_empty[rs]), (uint32_t)(((issued / kRing) & 1) ^ 1));
+        if (!got) report(a.err, kErrTimeout, (int32_t)t, 16);
+      }
+      if (!__shfl_sync(0xffffffffu, got, 0)) {
+        ok = false;
+        break;
+      }
+      for (int h = lane; h < NH; h += 32) ring[rs].w[h] = qc_w[h];
+      __syncwarp();
+      if (lane == 0) {
+        ring[rs].t = cur;
+        ring[rs].chunk = MODE == kFp4Sample ? sidx : chunk;
+        mbar_arrive(smem_u32(&ring_full[rs]));   // releases the lanes' weights (after the warp sync)
+        got = mbar_wait_susp(smem_u32(&empty_bar[slot]), (uint32_t)(((issued / kStages) & 1) ^ 1));
+        if (!got) report(a.err, kErrTimeout, (int32_t)t, 10);
+      }
+      if (!__shfl_sync(0xffffffffu, got, 0)) {
+        ok = false;
+        break;
+      }
+      uint8_t* const st = base_ptr + slot * Cfg::kStage;
+      const uint32_t sst = base + slot * Cfg::kStage;
+      const uint32_t fb = smem_u32(&full_bar[slot]);
+      // the item's codes and scale bytes: two bulk copies for a whole item of a
+      // contiguous cache, else page by page (out of line)
+      const int64_t cbase = (int64_t)seq * a.keys.seq_stride + s0;
+      if (a.keys.page_table == nullptr && a.keys.n_rows - cbase >= Cfg::kItem) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(fb, (uint32_t)(Cfg::kItem * (CI / 2 + nsc)));
+          bulk_g2s(sst + Cfg::kRawCOff, kc + cbase * (CI / 2), (uint32_t)(Cfg::kItem * (CI / 2)), fb);
+          bulk_g2s(sst + Cfg::kRawOff, a.k_scales + cbase * nsc, (uint32_t)(Cfg::kItem * nsc), fb);
+        }
+      } else {
+        fp4_copy_runs<CI, Cfg::kItem>(a.keys, a.k_scales, a.err, sst + Cfg::kRawCOff, sst + Cfg::kRawOff,
+                                      st + Cfg::kRawOff, fb, seq, s0, n_cur, (int32_t)t, lane);
+      }
+      // the query's operand image, unless the stage still holds it
+      if (lane == 0 && slot_q[slot] != cur) {
+        mbar_expect_tx(fb, (uint32_t)Cfg::kQImg);
+        bulk_g2s(sst + Cfg::kQOff, a.q_img + (int64_t)cur * Cfg::kQImg, (uint32_t)Cfg::kQImg, fb);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        slot_q[slot] = cur;
+        mbar_arrive(fb);   // the staging's arrival: releases the lanes' writes
+      }
+      ++issued;
+    }
+    if (lane == 0) {
+      for (int e = 0; ok && e < 2; ++e) {   // end markers (the MMA warp stops at the first)
+        const int64_t j = issued + e;
+        const int rs = (int)(j % kRing);
+        if (!mbar_wait_susp(smem_u32(&ring_empty[rs]), (uint32_t)(((j / kRing) & 1) ^ 1))) {
+          report(a.err, kErrTimeout, 0, 17);
+          break;
+        }
+        ring[rs].t = -1;
+        mbar_arrive(smem_u32(&ring_full[rs]));
+      }
+      const int64_t first = issued > kStages ? issued - kStages : 0;
+      for (int64_t d = first; d < issued; ++d)
+        mbar_wait(smem_u32(&full_bar[d % kStages]), (uint32_t)((d / kStages) & 1), 200000000ll);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // (the whole warp: lanes arrange the operands, lane 0 issues)
+    for (int64_t j = 0;; ++j) {
+      const int rs = (int)(j % kRing);
+      bool got = true, end = false;
+      if (lane == 0) {
+        got = mbar_wait_susp(smem_u32(&ring_full[rs]), (uint32_t)((j / kRing) & 1));
+        if (!got) report(a.err, kErrTimeout, (int32_t)j, 18);
+        else {
+          end = ring[rs].t < 0;
+          mbar_arrive(smem_u32(&ring_empty[rs]));
+        }
+      }
+      got = __shfl_sync(0xffffffffu, got, 0);
+      end = __shfl_sync(0xffffffffu, end, 0);
+      if (!got || end) break;
+      const int slot = (int)(j % kStages);
+      const int acc = (int)(j % kAccF);
+      if (lane == 0) {
+        got = mbar_wait_susp(smem_u32(&full_bar[slot]), (uint32_t)((j / kStages) & 1)) &&
+              mbar_wait_susp(smem_u32(&tempty_bar[acc]), (uint32_t)(((j / kAccF) & 1) ^ 1));
+        if (!got) report(a.err, kErrTimeout, (int32_t)j, 11);
+      }
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      tc::fence_after_sync();
+      uint8_t* const st = base_ptr + slot * Cfg::kStage;
+      // 128-dim keys: lanes 1 .. 31 move the codes into the K-major 32-byte
+      // swizzle (row r of block kb at 32 r, its 16-byte halves exchanged when
+      // bit 2 of r is set).  Then every lane m0 writes row m0 of the SFA blocks
+      // (tile h, block kb): bytes 4 c + (0, 1) hold the scale bytes of key
+      // m0 + 32 c, exchanged for the rows whose halves the MMA sees exchanged.
+      if (!Cfg::kSwap && lane > 0) {
+        constexpr int kChunks = Cfg::kItem * Cfg::kKB * 2;
+        const uint8_t* raw = st + Cfg::kRawCOff;
+#pragma unroll 4
+        for (int q = lane - 1; q < kChunks; q += 31) {
+          const int r = q / (Cfg::kKB * 2), kb = (q >> 1) % Cfg::kKB, half = q & 1;
+          const uint4 v = *reinterpret_cast<const uint4*>(raw + r * (CI / 2) + kb * 32 + half * 16);
+          *reinterpret_cast<uint4*>(st + kb * Cfg::kCodeBlk + r * 32 + (((half ^ (r >> 2)) & 1) << 4)) = v;
+        }
+      }
+      {
+        const int m0 = lane;
+        const bool xs = Cfg::kSwap && ((m0 >> 2) & 1);
+        const uint16_t* rsc = reinterpret_cast<const uint16_t*>(st + Cfg::kRawOff);
+#pragma unroll
+        for (int h = 0; h < Cfg::kTiles; ++h)
+#pragma unroll
+          for (int kb = 0; kb < Cfg::kKB; ++kb) {
+            uint32_t w[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint32_t v = rsc[(h * 128 + m0 + 32 * c) * Cfg::kKB + kb];
+              w[c] = xs ? ((v >> 8) | ((v & 0xffu) << 8)) : v;
+            }
+            *reinterpret_cast<uint4*>(st + Cfg::kSfaOff + (h * Cfg::kKB + kb) * 512 + m0 * 16) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        fence_async_smem_cta();
+      }
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_after_sync();
+        const uint32_t sst = base + slot * Cfg::kStage;
+        const uint32_t sf = tmem_base + Cfg::kSfBase + acc * Cfg::kSfCols;
+#pragma unroll
+        for (int i = 0; i < Cfg::kTiles * Cfg::kKB; ++i) tc::copy_scales(sf + 4 * i, sst + Cfg::kSfaOff + i * 512);
+#pragma unroll
+        for (int kb = 0; kb < Cfg::kKB; ++kb)
+          tc::copy_scales(sf + 4 * (Cfg::kTiles * Cfg::kKB + kb), sst + Cfg::kSfbOff + kb * 512);
+#pragma unroll
+        for (int h = 0; h < Cfg::kTiles; ++h)
+#pragma unroll
+          for (int kb = 0; kb < Cfg::kKB; ++kb)
+            tc::mma_mxf4_ss(tmem_base + acc * Cfg::kAccCols + h * Cfg::kN,
+                            tc::smem_desc_sw32(sst + kb * Cfg::kCodeBlk + h * 128 * 32),
+                            tc::smem_desc_sw32(sst + Cfg::kQOff + kb * Cfg::kQBlk), Cfg::kIdesc,
+                            sf + 4 * (h * Cfg::kKB + kb), sf + 4 * (Cfg::kTiles * Cfg::kKB + kb), kb > 0);
+        tc::mma_commit(smem_u32(&empty_bar[slot]));
+        tc::mma_commit(smem_u32(&tfull_bar[acc]));
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int group = ew >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    int t_cached = -1;
+    int64_t n_elig = 0;
+    uint32_t tau = 0;
+    CandidateBatch<Cfg::kTiles> pend;
+    for (int64_t j = group;; j += 2) {
+      const int rs = (int)(j % kRing);
+      if (!mbar_wait_susp(smem_u32(&ring_full[rs]), (uint32_t)((j / kRing) & 1))) {
+        if (lane == 0) report(a.err, kErrTimeout, (int32_t)j, 19);
+        break;
+      }
+      const int tq = ring[rs].t;
+      const int32_t chunk = ring[rs].chunk;   // the sampled chunk's ordinal in sample mode
+      float wv[NH];
+#pragma unroll
+      for (int h = 0; h < NH; h += 4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(&ring[rs].w[h]);
+        wv[h] = w4.x;
+        wv[h + 1] = w4.y;
+        wv[h + 2] = w4.z;
+        wv[h + 3] = w4.w;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ring_empty[rs]));
+      if (tq < 0) break;
+      const int acc = (int)(j % kAccF);
+      if (tq != t_cached) {
+        t_cached = tq;
+        n_elig = nelig[tq];
+        tau = MODE == kFp4Fused ? __ldg(a.tau + tq) : 0u;
+      }
+      if (!mbar_wait_susp(smem_u32(&tfull_bar[acc]), (uint32_t)((j / kAccF) & 1))) {
+        if (lane == 0) report(a.err, kErrTimeout, (int32_t)j, 13);
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * Cfg::kAccCols;
+      // this row's dot products, from the copy that pairs its halves
+      // correctly (columns NH + h for rows 4 .. 7 of every 8 when kSwap, else
+      // h), at most 64 columns loaded per wait: kPass passes of kHP heads
+      constexpr int kPass = Cfg::kN > 64 ? 2 : 1;
+      constexpr int kHP = NH / kPass;
+      constexpr int kChN = (kHP + 15) / 16;   // 16-column loads of a pass's plain columns
+      const bool second = Cfg::kSwap && ((row >> 2) & 1);
+      float scs[Cfg::kTiles];
+#pragma unroll
+      for (int h = 0; h < Cfg::kTiles; ++h) {
+        scs[h] = 0.f;
+#pragma unroll
+        for (int pa = 0; pa < kPass; ++pa) {
+          uint32_t r[4][16];
+          const uint32_t tcol = taddr + h * Cfg::kN + pa * kHP;
+          if (Cfg::kSwap && kHP < 16) {
+            tc::tmem_ld16(tcol, r[0]);   // NH = 8: plain and exchanged copies in one load
+          } else {
+#pragma unroll
+            for (int c = 0; c < kChN; ++c) {
+              tc::tmem_ld16(tcol + 16 * c, r[c]);
+              if (Cfg::kSwap) tc::tmem_ld16(tcol + NH + 16 * c, r[kChN + c]);
+            }
+          }
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int hh = 0; hh < kHP; ++hh) {
+            uint32_t v;
+            if (Cfg::kSwap && kHP < 16) v = second ? r[0][(8 + hh) & 15] : r[0][hh & 15];
+            else if (Cfg::kSwap) v = second ? r[kChN + hh / 16][hh % 16] : r[hh / 16][hh % 16];
+            else v = r[hh / 16][hh % 16];
+            scs[h] = fmaf(wv[pa * kHP + hh], fmaxf(__uint_as_float(v), 0.f), scs[h]);
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[acc]));
+      if (MODE == kFp4Sample) {
+#pragma unroll
+        for (int h = 0; h < Cfg::kTiles; ++h)
+          a.psample[(int64_t)tq * kPSampleKeys + chunk * Cfg::kItem + h * kTileRows + row] = score_key(scs[h]);
+        continue;
+      }
+      const int64_t s0 = (int64_t)chunk * Cfg::kItem;
+      bool pass[Cfg::kTiles];
+      uint32_t keys[Cfg::kTiles], ents[Cfg::kTiles];
+#pragma unroll
+      for (int h = 0; h < Cfg::kTiles; ++h) {
+        const int64_t s = s0 + h * kTileRows + row;
+        keys[h] = score_key(scs[h]);
+        ents[h] = (uint32_t)s;
+        pass[h] = s < n_elig && keys[h] >= tau;
+      }
+      CandidateBatch<Cfg::kTiles> cur;
+      cur.issue(a, tq, pass, keys, ents);
+      pend.flush(a);
+      pend = cur;
+    }
+    if (MODE == kFp4Fused) pend.flush(a);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem_base, Cfg::kTmemCols);
+}
+
 }  // namespace
 
 bool tc_indexer_supported(const IndexerArgs& a, int64_t t_count) {
@@ -902,6 +1466,76 @@ cudaError_t launch_score_tc(const Launch& L, const IndexerArgs& a, int64_t t_cou
 }
 
 }  // namespace
+
+bool tc_fp4_indexer_supported(const IndexerArgs& a, int64_t t_count) {
+  if (!a.fp4 || a.tau == nullptr || a.psample == nullptr || a.work == nullptr) return false;
+  if ((a.c_I != 64 && a.c_I != 128) || a.H_I > 64 || t_count > kMaxQueries) return false;
+  if ((a.max_entries + kFMinItem - 1) / kFMinItem * t_count > INT32_MAX) return false;
+  if (a.keys.page_table != nullptr && a.keys.page_size % kBoxRows != 0) return false;
+  if (a.keys.n_rows > INT32_MAX || a.T * a.H_I > INT32_MAX) return false;
+  // code rows and scale-byte copies must stay 16-byte aligned
+  const int64_t code_row = a.c_I / 2, sc_row = a.c_I / 32;
+  if ((reinterpret_cast<uintptr_t>(a.keys.data) & 15u) || (reinterpret_cast<uintptr_t>(a.k_scales) & 15u))
+    return false;
+  if (a.keys.page_table == nullptr && ((a.keys.seq_stride * sc_row) % 16 != 0 || (a.keys.seq_stride * code_row) % 16 != 0))
+    return false;
+  return true;
+}
+
+namespace {
+
+template <int CI, int NH, int MODE>
+cudaError_t launch_score_fp4_tc(const Launch& L, const IndexerArgs& a, int64_t t_count) {
+  using Cfg = Fp4Cfg<CI, NH, MODE == kFp4Sample>;
+  TcIndexerParams p;
+  p.a = a;
+  p.t_count = t_count;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaFuncSetAttribute(indexer_score_fp4_tc_kernel<CI, NH, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       Cfg::kSmem);
+  prefer_max_shared(indexer_score_fp4_tc_kernel<CI, NH, MODE>);
+  indexer_score_fp4_tc_kernel<CI, NH, MODE><<<(unsigned)sms, kThreads, Cfg::kSmem, L.stream>>>(p);
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_fp4_query_images(const Launch& L, const IndexerArgs& a, int64_t t_count) {
+  L.begin(kKernelIndexerScore);
+  const int nh = a.c_I == 64 && a.H_I <= 8 ? 8 : a.c_I == 64 && a.H_I <= 16 ? 16 : a.H_I <= 32 ? 32 : 64;
+  const unsigned grid = (unsigned)((t_count + 3) / 4);
+#define CSA_FP4IMG(CI_, NH_) fp4_query_image_kernel<CI_, NH_><<<grid, 128, 0, L.stream>>>(a, t_count);
+  if (a.c_I == 64) {
+    if (nh == 8) { CSA_FP4IMG(64, 8) } else if (nh == 16) { CSA_FP4IMG(64, 16) }
+    else if (nh == 32) { CSA_FP4IMG(64, 32) } else { CSA_FP4IMG(64, 64) }
+  } else {
+    if (nh == 32) { CSA_FP4IMG(128, 32) } else { CSA_FP4IMG(128, 64) }
+  }
+#undef CSA_FP4IMG
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return L.end(kKernelIndexerScore);
+}
+
+cudaError_t launch_indexer_scores_fp4_tc(const Launch& L, const IndexerArgs& a, int64_t t_count, bool sample) {
+  L.begin(kKernelIndexerScore);
+  // padded heads: 8 / 16 / 32 / 64 for 64-dim keys (B holds 2 NH rows), 32 / 64 for 128-dim
+  const int nh = a.c_I == 64 && a.H_I <= 8 ? 8 : a.c_I == 64 && a.H_I <= 16 ? 16 : a.H_I <= 32 ? 32 : 64;
+  cudaError_t e;
+#define CSA_FP4TC(CI_, NH_) \
+  e = sample ? launch_score_fp4_tc<CI_, NH_, kFp4Sample>(L, a, t_count) : launch_score_fp4_tc<CI_, NH_, kFp4Fused>(L, a, t_count);
+  if (a.c_I == 64) {
+    if (nh == 8) { CSA_FP4TC(64, 8) } else if (nh == 16) { CSA_FP4TC(64, 16) }
+    else if (nh == 32) { CSA_FP4TC(64, 32) } else { CSA_FP4TC(64, 64) }
+  } else {
+    if (nh == 32) { CSA_FP4TC(128, 32) } else { CSA_FP4TC(128, 64) }
+  }
+#undef CSA_FP4TC
+  if (e != cudaSuccess) return e;
+  return L.end(kKernelIndexerScore);
+}
 
 cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int64_t t_count) {
   L.begin(kKernelIndexerScore);

@@ -100,6 +100,9 @@ struct IndexerArgs {
   // each query's sampled keys here ([T_chunk, kPSampleKeys]); queries whose
   // candidate count misses [top_k, cand_cap] are listed for the exact fallback
   uint32_t* psample = nullptr;
+  // tcgen05 4-bit scorer: per chunk query, its quantized heads as the MMA's B
+  // operand image (written by launch_fp4_query_images, read by both passes)
+  uint8_t* q_img = nullptr;
   uint32_t* fb_list = nullptr;       // [T_chunk] chunk-local query ids
   uint32_t* fb_count = nullptr;      // zeroed by the threshold pass
   WsHeader* err;
@@ -180,6 +183,17 @@ cudaError_t launch_indexer_scores_tc(const Launch& L, const IndexerArgs& a, int6
 bool tc_indexer_prefill_supported(const IndexerArgs& a, int64_t t_count);
 cudaError_t launch_indexer_scores_tc_prefill(const Launch& L, const IndexerArgs& a, int64_t t_count,
                                              bool sample);
+// tcgen05 4-bit scorer (few-query mode, c_I in {64, 128}, H_I <= 64, pages a
+// multiple of 64 rows): block-scaled MMAs on the stored codes; its sample pass
+// (sample = true) writes a.psample for topk_threshold_many, its fused pass the
+// candidate lists
+bool tc_fp4_indexer_supported(const IndexerArgs& a, int64_t t_count);
+cudaError_t launch_indexer_scores_fp4_tc(const Launch& L, const IndexerArgs& a, int64_t t_count, bool sample);
+// Quantizes each chunk query's heads into its operand image at a.q_img (at
+// most kFp4ImgSlots * 8 bytes per query) and zeroes the work counter; runs
+// before the tcgen05 4-bit scorer's passes.
+constexpr int kFp4ImgSlots = 640;
+cudaError_t launch_fp4_query_images(const Launch& L, const IndexerArgs& a, int64_t t_count);
 // 4-bit scorer (E2M1 codes with one scale byte per 32 elements): see indexer_fp4.cu
 cudaError_t launch_indexer_scores_fp4(const Launch& L, const IndexerArgs& a, int64_t t_count);
 // [n_blocks * 32] bf16 -> n_blocks * 16 code bytes + n_blocks scale bytes
@@ -201,12 +215,15 @@ cudaError_t launch_topk_finish(const Launch& L, const IndexerArgs& a, int top_k,
 // Many-query (prefill) selection, one warp per query, after the tcgen05
 // scorer's sample pass and around its fused pass (fb_list / fb_count /
 // psample set):
-//   launch_topk_threshold_many: tau from the sampled keys; zeroes the counts,
-//     the fallback list and the work counter;
+//   launch_topk_threshold_many: tau from the sampled keys (the sample of a block
+//     of qb consecutive queries: 128 / H_I for the prefill scorer, 1 for the
+//     4-bit decode scorer); zeroes the counts, the fallback list and the work
+//     counter;
 //   launch_topk_finish_many: the exact top-k among the candidates, then the
 //     recompute of the listed queries whose count missed [top_k, cand_cap].
 bool topk_many_supported(const IndexerArgs& a);
-cudaError_t launch_topk_threshold_many(const Launch& L, const IndexerArgs& a, int top_k, int64_t t_count);
+cudaError_t launch_topk_threshold_many(const Launch& L, const IndexerArgs& a, int top_k, int64_t t_count,
+                                      int qb);
 cudaError_t launch_topk_finish_many(const Launch& L, const IndexerArgs& a, int top_k, int32_t* idx_out,
                                     int32_t* count_out, float* score_out, int64_t t_count);
 

@@ -30,6 +30,60 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of a K-major operand whose rows are 32
+// bytes (64 4-bit elements) in the 32-byte swizzle: 8-row groups 256 bytes
+// apart.
+__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3fffu);
+  d |= (uint64_t)(16u >> 4) << 16;
+  d |= (uint64_t)(256u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)6 << 61;
+  return d;
+}
+
+// Descriptor of a 32-row x 16-byte source of tcgen05.cp (no swizzle: rows 16
+// bytes apart, 8-row groups 128 bytes apart).
+__device__ __forceinline__ uint64_t smem_desc_cp32x16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3fffu);
+  d |= (uint64_t)(128u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// Instruction descriptor of kind::mxf4 with block scaling (E2M1 A and B, E8M0
+// scale bytes, K = 64 per instruction, fp32 accumulator), both K-major.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) {
+  return (1u << 7)                       // A format: E2M1
+         | (1u << 10)                    // B format: E2M1
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | (1u << 23)                    // scale format: E8M0
+         | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// D (+)= (A * 2^(sfa - 127)) (B * 2^(sfb - 127))^T over one K = 64 block pair,
+// the scale bytes of A's rows and B's rows in TMEM at sfa / sfb (one byte per
+// 32 elements, bytes 0 and 1 of the row's column; see copy_scales).
+__device__ __forceinline__ void mma_mxf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa, uint32_t sfb, bool acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)acc), "r"(sfa), "r"(sfb));
+}
+
+// Copy a 32-row x 16-byte block from shared memory to TMEM columns
+// taddr .. taddr + 3 of all four 32-lane quarters (row r to lanes r, 32 + r,
+// 64 + r, 96 + r): the layout block-scaled MMAs read their scale bytes in
+// (row m of a 128-row operand: lane m mod 32, column m / 32; a 32-row operand:
+// column 0).
+__device__ __forceinline__ void copy_scales(uint32_t taddr, uint32_t saddr) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n" ::"r"(taddr),
+               "l"(smem_desc_cp32x16(saddr)));
+}
+
 // Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator, both
 // operands K-major unless *_mn is set, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn = false,
@@ -118,5 +172,6 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 // out-of-bounds rows read as zero.  Returns false on failure.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                        uint64_t pitch_elems, uint32_t box_cols, uint32_t box_rows);
+
 
 }  // namespace csa

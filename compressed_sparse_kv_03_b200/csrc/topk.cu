@@ -844,7 +844,7 @@ __device__ __forceinline__ void warp_take_lowest_ties(uint32_t* sel, const uint3
 // work counter of the scoring pass that follows.
 constexpr int kTWarps = 4;
 __global__ void __launch_bounds__(kTWarps * 32) topk_threshold_many_kernel(IndexerArgs a, int top_k,
-                                                                        int64_t t_count) {
+                                                                        int64_t t_count, int qb) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     *a.fb_count = 0u;
@@ -857,8 +857,8 @@ __global__ void __launch_bounds__(kTWarps * 32) topk_threshold_many_kernel(Index
   const int64_t n = eligible_of(a, t);
   uint32_t tau = 0u;
   if (n > a.skip_le && 2 * n > a.cand_cap) {
-    // the block's sampled chunks, by the scorer's rule
-    const int64_t QB = 128 / a.H_I;
+    // the sampled chunks of the query's block of qb queries, by the scorer's rule
+    const int64_t QB = qb;
     const int64_t b0 = tl / QB * QB, b1 = b0 + QB < t_count ? b0 + QB : t_count;
     int64_t nmin = INT64_MAX, nmax = 0;
     for (int64_t u = b0 + lane; u < b1; u += 32) {
@@ -1155,12 +1155,13 @@ bool topk_many_supported(const IndexerArgs& a) {
   return a.fb_list != nullptr && a.fb_count != nullptr && per_warp * kFWarps <= 200 * 1024;
 }
 
-cudaError_t launch_topk_threshold_many(const Launch& L, const IndexerArgs& a, int top_k, int64_t t_count) {
+cudaError_t launch_topk_threshold_many(const Launch& L, const IndexerArgs& a, int top_k, int64_t t_count,
+                                      int qb) {
   if (t_count == 0) return cudaSuccess;
   L.begin(kKernelTopkSample);
   prefer_max_shared(topk_threshold_many_kernel);
   const unsigned grid = (unsigned)((t_count + kTWarps - 1) / kTWarps);
-  topk_threshold_many_kernel<<<grid, kTWarps * 32, 0, L.stream>>>(a, top_k, t_count);
+  topk_threshold_many_kernel<<<grid, kTWarps * 32, 0, L.stream>>>(a, top_k, t_count, qb);
   return L.end(kKernelTopkSample);
 }
 

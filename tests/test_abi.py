@@ -131,11 +131,13 @@ def test_workspace_sizes(lib):
     assert n > hdr and n % 256 == 0
     # prefill never splits
     assert lib.csa_sparse_attn_prefill_workspace_size(65536, 64, 128) == hdr
-    # decode-mode indexer scratch is O(queries x top_k): a threshold, a count and
-    # 4 top_k (at least 8192) candidate (key, entry) pairs per query -- no score
-    # matrix, and independent of the number of entries
+    # decode-mode indexer scratch is O(queries x top_k): a threshold, a count, a
+    # fallback slot, 4 top_k (at least 8192) candidate (key, entry) pairs and
+    # 1024 sampled keys per query -- no score matrix, and independent of the
+    # number of entries
     n = lib.csa_indexer_topk_workspace_size(64, 32768, 2048)
-    assert hdr + 64 * 8192 * 8 <= n <= hdr + 64 * (8192 * 8 + 8) + 3 * 256
+    per_query = 8192 * 8 + 1024 * 4
+    assert hdr + 64 * per_query <= n <= hdr + 64 * (per_query + 12) + 4 * 256
     assert lib.csa_indexer_topk_workspace_size(64, 1 << 19, 2048) == n
     assert lib.csa_indexer_topk_workspace_size(64, 32768, 4096) > n
     # many-query (prefill) mode: the same O(top_k) candidate lists plus 1024

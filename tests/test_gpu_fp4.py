@@ -98,7 +98,7 @@ def _check_fp4_queries(idx, cnt, sc, q, w, keys_of, elig_of, k, queries):
     return stats
 
 
-@pytest.mark.parametrize("H_I,c_I", [(8, 64), (16, 128), (1, 64), (12, 64), (64, 128), (40, 64)])
+@pytest.mark.parametrize("H_I,c_I", [(8, 64), (16, 128), (1, 64), (12, 64), (64, 128), (40, 64), (24, 64)])
 def test_indexer_topk_mxfp4_decode_ragged(H_I, c_I):
     """Few-query (histogram + bitmap select) mode, one sequence per query,
     ragged eligible counts; the codes are the oracle's quantization of normal

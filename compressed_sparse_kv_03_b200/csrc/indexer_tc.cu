@@ -991,15 +991,19 @@ __global__ void __launch_bounds__(128) fp4_query_image_kernel(IndexerArgs a, int
   }
 }
 
+// producer, MMA issuer, kEpiWarps epilogue warps, then the operand warp
+constexpr int kFThreads = kThreads + 32;
+constexpr int kOpWarp = kThreads / 32;
+
 template <int CI, int NH, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFThreads, 1)
 indexer_score_fp4_tc_kernel(TcIndexerParams p) {
   using Cfg = Fp4Cfg<CI, NH, MODE == kFp4Sample>;
   constexpr int kStages = Cfg::kStages, kAccF = Cfg::kAccF;
   const IndexerArgs& a = p.a;
   const int T = (int)p.t_count;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], opnd_bar[kStages];
   __shared__ __align__(8) uint64_t tfull_bar[kAccF], tempty_bar[kAccF];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int32_t prefix[kMaxQueries + 1];
@@ -1018,6 +1022,7 @@ indexer_score_fp4_tc_kernel(TcIndexerParams p) {
       slot_q[i] = -1;
       mbar_init(smem_u32(&full_bar[i]), 2);   // the copies' arrival + the query staging's
       mbar_init(smem_u32(&empty_bar[i]), 1);
+      mbar_init(smem_u32(&opnd_bar[i]), 1);   // the operand warp's arrival
     }
     for (int i = 0; i < kAccF; ++i) {
       mbar_init(smem_u32(&tfull_bar[i]), 1);
@@ -1025,7 +1030,7 @@ indexer_score_fp4_tc_kernel(TcIndexerParams p) {
     }
     for (int i = 0; i < kRing; ++i) {
       mbar_init(smem_u32(&ring_full[i]), 1);
-      mbar_init(smem_u32(&ring_empty[i]), 5);   // the MMA warp + one epilogue group
+      mbar_init(smem_u32(&ring_empty[i]), 6);   // the MMA warp, one epilogue group, the operand warp
     }
     mbar_fence_init();
   }
@@ -1191,12 +1196,12 @@ indexer_score_fp4_tc_kernel(TcIndexerParams p) {
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // (the whole warp: lanes arrange the operands, lane 0 issues)
-    for (int64_t j = 0;; ++j) {
+    // (lane 0 issues; the operand warp has arranged the stage's operands)
+    for (uint32_t j = 0;; ++j) {
       const int rs = (int)(j % kRing);
       bool got = true, end = false;
       if (lane == 0) {
-        got = mbar_wait_susp(smem_u32(&ring_full[rs]), (uint32_t)((j / kRing) & 1));
+        got = mbar_wait_susp(smem_u32(&ring_full[rs]), (j / kRing) & 1u);
         if (!got) report(a.err, kErrTimeout, (int32_t)j, 18);
         else {
           end = ring[rs].t < 0;
@@ -1209,69 +1214,90 @@ indexer_score_fp4_tc_kernel(TcIndexerParams p) {
       const int slot = (int)(j % kStages);
       const int acc = (int)(j % kAccF);
       if (lane == 0) {
-        got = mbar_wait_susp(smem_u32(&full_bar[slot]), (uint32_t)((j / kStages) & 1)) &&
-              mbar_wait_susp(smem_u32(&tempty_bar[acc]), (uint32_t)(((j / kAccF) & 1) ^ 1));
+        got = mbar_wait_susp(smem_u32(&full_bar[slot]), (j / kStages) & 1u) &&
+              mbar_wait_susp(smem_u32(&opnd_bar[slot]), (j / kStages) & 1u) &&
+              mbar_wait_susp(smem_u32(&tempty_bar[acc]), ((j / kAccF) & 1u) ^ 1u);
         if (!got) report(a.err, kErrTimeout, (int32_t)j, 11);
+        else {
+          tc::fence_after_sync();
+          const uint32_t sst = base + slot * Cfg::kStage;
+          const uint32_t sf = tmem_base + Cfg::kSfBase + acc * Cfg::kSfCols;
+#pragma unroll
+          for (int i = 0; i < Cfg::kTiles * Cfg::kKB; ++i) tc::copy_scales(sf + 4 * i, sst + Cfg::kSfaOff + i * 512);
+#pragma unroll
+          for (int kb = 0; kb < Cfg::kKB; ++kb)
+            tc::copy_scales(sf + 4 * (Cfg::kTiles * Cfg::kKB + kb), sst + Cfg::kSfbOff + kb * 512);
+#pragma unroll
+          for (int h = 0; h < Cfg::kTiles; ++h)
+#pragma unroll
+            for (int kb = 0; kb < Cfg::kKB; ++kb)
+              tc::mma_mxf4_ss(tmem_base + acc * Cfg::kAccCols + h * Cfg::kN,
+                              tc::smem_desc_sw32(sst + kb * Cfg::kCodeBlk + h * 128 * 32),
+                              tc::smem_desc_sw32(sst + Cfg::kQOff + kb * Cfg::kQBlk), Cfg::kIdesc,
+                              sf + 4 * (h * Cfg::kKB + kb), sf + 4 * (Cfg::kTiles * Cfg::kKB + kb), kb > 0);
+          tc::mma_commit(smem_u32(&empty_bar[slot]));
+          tc::mma_commit(smem_u32(&tfull_bar[acc]));
+        }
       }
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
-      tc::fence_after_sync();
+    }
+  } else if (warp == kOpWarp) {
+    // ------------------------------------------------------------ operands
+    // Once a stage's copies land: for 128-dim keys the codes into the K-major
+    // 32-byte swizzle (row r of block kb at 32 r, its 16-byte halves exchanged
+    // when bit 2 of r is set); then lane m0 writes row m0 of every SFA block
+    // (tile h, block kb): bytes 4 c + (0, 1) hold the scale bytes of key
+    // m0 + 32 c, exchanged for the rows whose halves the MMA sees exchanged.
+    for (uint32_t j = 0;; ++j) {
+      const int rs = (int)(j % kRing);
+      bool got = true, end = false;
+      if (lane == 0) {
+        got = mbar_wait_susp(smem_u32(&ring_full[rs]), (j / kRing) & 1u);
+        if (!got) report(a.err, kErrTimeout, (int32_t)j, 20);
+        else {
+          end = ring[rs].t < 0;
+          mbar_arrive(smem_u32(&ring_empty[rs]));
+        }
+      }
+      got = __shfl_sync(0xffffffffu, got, 0);
+      end = __shfl_sync(0xffffffffu, end, 0);
+      if (!got || end) break;
+      const int slot = (int)(j % kStages);
+      if (lane == 0) {
+        got = mbar_wait_susp(smem_u32(&full_bar[slot]), (j / kStages) & 1u);
+        if (!got) report(a.err, kErrTimeout, (int32_t)j, 21);
+      }
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
       uint8_t* const st = base_ptr + slot * Cfg::kStage;
-      // 128-dim keys: lanes 1 .. 31 move the codes into the K-major 32-byte
-      // swizzle (row r of block kb at 32 r, its 16-byte halves exchanged when
-      // bit 2 of r is set).  Then every lane m0 writes row m0 of the SFA blocks
-      // (tile h, block kb): bytes 4 c + (0, 1) hold the scale bytes of key
-      // m0 + 32 c, exchanged for the rows whose halves the MMA sees exchanged.
-      if (!Cfg::kSwap && lane > 0) {
+      if (!Cfg::kSwap) {
         constexpr int kChunks = Cfg::kItem * Cfg::kKB * 2;
         const uint8_t* raw = st + Cfg::kRawCOff;
 #pragma unroll 4
-        for (int q = lane - 1; q < kChunks; q += 31) {
+        for (int q = lane; q < kChunks; q += 32) {
           const int r = q / (Cfg::kKB * 2), kb = (q >> 1) % Cfg::kKB, half = q & 1;
           const uint4 v = *reinterpret_cast<const uint4*>(raw + r * (CI / 2) + kb * 32 + half * 16);
           *reinterpret_cast<uint4*>(st + kb * Cfg::kCodeBlk + r * 32 + (((half ^ (r >> 2)) & 1) << 4)) = v;
         }
       }
-      {
-        const int m0 = lane;
-        const bool xs = Cfg::kSwap && ((m0 >> 2) & 1);
-        const uint16_t* rsc = reinterpret_cast<const uint16_t*>(st + Cfg::kRawOff);
+      const int m0 = lane;
+      const bool xs = Cfg::kSwap && ((m0 >> 2) & 1);
+      const uint16_t* rsc = reinterpret_cast<const uint16_t*>(st + Cfg::kRawOff);
 #pragma unroll
-        for (int h = 0; h < Cfg::kTiles; ++h)
+      for (int h = 0; h < Cfg::kTiles; ++h)
 #pragma unroll
-          for (int kb = 0; kb < Cfg::kKB; ++kb) {
-            uint32_t w[4];
+        for (int kb = 0; kb < Cfg::kKB; ++kb) {
+          uint32_t w[4];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint32_t v = rsc[(h * 128 + m0 + 32 * c) * Cfg::kKB + kb];
-              w[c] = xs ? ((v >> 8) | ((v & 0xffu) << 8)) : v;
-            }
-            *reinterpret_cast<uint4*>(st + Cfg::kSfaOff + (h * Cfg::kKB + kb) * 512 + m0 * 16) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t v = rsc[(h * 128 + m0 + 32 * c) * Cfg::kKB + kb];
+            w[c] = xs ? ((v >> 8) | ((v & 0xffu) << 8)) : v;
           }
-        fence_async_smem_cta();
-      }
+          *reinterpret_cast<uint4*>(st + Cfg::kSfaOff + (h * Cfg::kKB + kb) * 512 + m0 * 16) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      fence_async_smem_cta();
       __syncwarp();
-      if (lane == 0) {
-        tc::fence_after_sync();
-        const uint32_t sst = base + slot * Cfg::kStage;
-        const uint32_t sf = tmem_base + Cfg::kSfBase + acc * Cfg::kSfCols;
-#pragma unroll
-        for (int i = 0; i < Cfg::kTiles * Cfg::kKB; ++i) tc::copy_scales(sf + 4 * i, sst + Cfg::kSfaOff + i * 512);
-#pragma unroll
-        for (int kb = 0; kb < Cfg::kKB; ++kb)
-          tc::copy_scales(sf + 4 * (Cfg::kTiles * Cfg::kKB + kb), sst + Cfg::kSfbOff + kb * 512);
-#pragma unroll
-        for (int h = 0; h < Cfg::kTiles; ++h)
-#pragma unroll
-          for (int kb = 0; kb < Cfg::kKB; ++kb)
-            tc::mma_mxf4_ss(tmem_base + acc * Cfg::kAccCols + h * Cfg::kN,
-                            tc::smem_desc_sw32(sst + kb * Cfg::kCodeBlk + h * 128 * 32),
-                            tc::smem_desc_sw32(sst + Cfg::kQOff + kb * Cfg::kQBlk), Cfg::kIdesc,
-                            sf + 4 * (h * Cfg::kKB + kb), sf + 4 * (Cfg::kTiles * Cfg::kKB + kb), kb > 0);
-        tc::mma_commit(smem_u32(&empty_bar[slot]));
-        tc::mma_commit(smem_u32(&tfull_bar[acc]));
-      }
-      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&opnd_bar[slot]));
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -1283,9 +1309,9 @@ indexer_score_fp4_tc_kernel(TcIndexerParams p) {
     int64_t n_elig = 0;
     uint32_t tau = 0;
     CandidateBatch<Cfg::kTiles> pend;
-    for (int64_t j = group;; j += 2) {
+    for (uint32_t j = group;; j += 2) {
       const int rs = (int)(j % kRing);
-      if (!mbar_wait_susp(smem_u32(&ring_full[rs]), (uint32_t)((j / kRing) & 1))) {
+      if (!mbar_wait_susp(smem_u32(&ring_full[rs]), (j / kRing) & 1u)) {
         if (lane == 0) report(a.err, kErrTimeout, (int32_t)j, 19);
         break;
       }
@@ -1496,7 +1522,7 @@ cudaError_t launch_score_fp4_tc(const Launch& L, const IndexerArgs& a, int64_t t
   cudaFuncSetAttribute(indexer_score_fp4_tc_kernel<CI, NH, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        Cfg::kSmem);
   prefer_max_shared(indexer_score_fp4_tc_kernel<CI, NH, MODE>);
-  indexer_score_fp4_tc_kernel<CI, NH, MODE><<<(unsigned)sms, kThreads, Cfg::kSmem, L.stream>>>(p);
+  indexer_score_fp4_tc_kernel<CI, NH, MODE><<<(unsigned)sms, kFThreads, Cfg::kSmem, L.stream>>>(p);
   return cudaSuccess;
 }
 

@@ -120,14 +120,10 @@ __global__ void __launch_bounds__(NW * 32) attn_kernel(AttnArgs a) {
         const uint2 cw = __ldg(reinterpret_cast<const uint2*>(kv_codes + phys * (8 * dc8) + 8 * ch));
         const float fs = lowprec::e8m0_to_float(__ldg(a.kv_scales + phys * (dc8 / 4) + (ch >> 2)));
         uint4 o;
-        o.x = pack_bf16(lowprec::e4m3_to_float(cw.x & 0xffu) * fs,
-                        lowprec::e4m3_to_float((cw.x >> 8) & 0xffu) * fs);
-        o.y = pack_bf16(lowprec::e4m3_to_float((cw.x >> 16) & 0xffu) * fs,
-                        lowprec::e4m3_to_float(cw.x >> 24) * fs);
-        o.z = pack_bf16(lowprec::e4m3_to_float(cw.y & 0xffu) * fs,
-                        lowprec::e4m3_to_float((cw.y >> 8) & 0xffu) * fs);
-        o.w = pack_bf16(lowprec::e4m3_to_float((cw.y >> 16) & 0xffu) * fs,
-                        lowprec::e4m3_to_float(cw.y >> 24) * fs);
+        o.x = lowprec::e4m3x2_scaled_bf16x2(cw.x, fs);
+        o.y = lowprec::e4m3x2_scaled_bf16x2(cw.x >> 16, fs);
+        o.z = lowprec::e4m3x2_scaled_bf16x2(cw.y, fs);
+        o.w = lowprec::e4m3x2_scaled_bf16x2(cw.y >> 16, fs);
         *reinterpret_cast<uint4*>(&sKV[st][off]) = o;
       } else {
         cp_async_16(base + off * 2u, a.kv_rope + phys * a.rope_dims + (ch - dc8) * 8, true);

@@ -226,7 +226,7 @@ __device__ __noinline__ void gather_fp8_rows(const uint8_t* codes, const uint8_t
                                              const __nv_bfloat16* rope, int rope_dims, uint32_t cdst,
                                              int64_t row, int my_pairs, int pk, int lane) {
   constexpr int kJ = (kRows / 2 + kProducerWarps - 1) / kProducerWarps;
-  constexpr int kFB = 4;   // rows per load batch
+  constexpr int kFB = kJ;   // all of the warp's rows in one batch: one round trip per tile
   const int c = lane & 15, sub = lane >> 4;
   const int dc8 = (kD - rope_dims) / 8;
 #pragma unroll
@@ -261,11 +261,7 @@ __device__ __noinline__ void gather_fp8_rows(const uint8_t* codes, const uint8_t
         const uint32_t w2[2] = {cw[u].x, cw[u].y};
         uint32_t o[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t wd = w2[q >> 1] >> (16 * (q & 1));
-          o[q] = pack_bf16(lowprec::e4m3_to_float(wd & 0xffu) * fs,
-                           lowprec::e4m3_to_float((wd >> 8) & 0xffu) * fs);
-        }
+        for (int q = 0; q < 4; ++q) o[q] = lowprec::e4m3x2_scaled_bf16x2(w2[q >> 1] >> (16 * (q & 1)), fs);
         const uint32_t addr = cdst + (uint32_t)r * 128 + (uint32_t)((((c & 7) ^ (r & 7)) & 7) << 4);
         asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(o[0]), "r"(o[1]),
                      "r"(o[2]), "r"(o[3])

@@ -6,6 +6,8 @@
 // largest value 448.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace csa {
@@ -22,6 +24,17 @@ __device__ __forceinline__ float e4m3_to_float(uint32_t c) {
   const float v = E ? __uint_as_float(((E + 120u) << 23) | (M << 20))   // (1 + M/8) 2^(E-7)
                     : (float)M * 0.001953125f;                            // M 2^-9
   return (c & 0x80u) ? -v : v;
+}
+
+// Two E4M3 codes (bits 0-7 and 8-15 of `two`) times fs, rounded to a bf16
+// pair (low half = the first code): the hardware pair conversion to f16 is
+// exact, so is the fp32 product with a power of two, and the bf16 rounding
+// equals that of e4m3_to_float(c) * fs.
+__device__ __forceinline__ uint32_t e4m3x2_scaled_bf16x2(uint32_t two, float fs) {
+  uint32_t h2;
+  asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}\n" : "=r"(h2) : "r"(two));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+  return pack_bf16(f.x * fs, f.y * fs);
 }
 
 // Nearest E4M3 code of y, ties to the even code, saturating at 448; the sign

@@ -41,28 +41,34 @@ constexpr int kKeyTileBytes = kTileRows * 128;     // 64 bf16 per row
 constexpr int kStageKeyBytes = 2 * kKeyTileBytes;
 constexpr int kEpiWarps = 8;                       // two groups of four
 constexpr int kThreads = (2 + kEpiWarps) * 32;
-constexpr int kAcc = 4;                            // TMEM accumulator sets
 
 // Decode-mode layout for key dim CI (64 or 128) and NH padded heads: an
-// item's keys are CI / 64 column blocks of 256 rows x 128 bytes (one TMA box
-// of the 128-byte swizzle each), the query's heads as many blocks of NH rows.
+// item's keys are CI / 64 column blocks of kItem rows x 128 bytes (256-row TMA
+// boxes of the 128-byte swizzle), the query's heads as many blocks of NH rows.
+// An item is 512 keys for CI = 64 (the issuing threads' work per item is
+// mostly fixed, so larger items stream closer to the memory bound) and 256
+// for CI = 128 (so that several stages still fit).
 template <int CI, int NH>
 struct ScoreCfg {
+  static constexpr int kItem = CI == 64 ? 512 : 256;
+  static constexpr int kTiles = kItem / kTileRows;
   static constexpr int kKB = CI / 64;
-  static constexpr int kKeyBlk = kItemRows * 128;
+  static constexpr int kKeyBlk = kItem * 128;
   static constexpr int kStageKey = kKB * kKeyBlk;
   static constexpr int kQBlk = NH * 128;
   static constexpr int kQBytes = kKB * kQBlk;
   // as many stages as fit beside the kernel's static shared memory (<= 6)
   static constexpr int kFit = (205 * 1024) / (kStageKey + kQBytes);
   static constexpr int kStages = kFit < 6 ? kFit : 6;
-  static constexpr int kAccCols = 2 * NH;          // two key tiles of NH columns
-  static constexpr int kTmemCols = kAcc * kAccCols;   // 128, 256 or 512
+  static constexpr int kAccCols = kTiles * NH;     // kTiles key tiles of NH columns
+  static constexpr int kAccSets = 4 * kAccCols <= 512 ? 4 : 2;   // TMEM accumulator sets
+  static constexpr int kTmemCols = kAccSets * kAccCols <= 128 ? 128 : kAccSets * kAccCols <= 256 ? 256 : 512;
   static constexpr uint32_t kIdesc = tc::idesc_bf16(128, NH);
   static constexpr int kSmem = kStages * (kStageKey + kQBytes) + 1024;
+  static_assert(kAccSets * kAccCols <= 512 && kStages >= 2, "decode scorer layout");
 };
 constexpr int kMaxQueries = 2048;
-constexpr int kRing = 16;                          // item metadata ring (> stages + kAcc)
+constexpr int kRing = 16;                          // item metadata ring (> stages + accumulator sets)
 constexpr int kGrab = 2;                           // items taken from the work counter at once
 #ifndef CSA_SCORE_STATIC_PCT
 #define CSA_SCORE_STATIC_PCT 70
@@ -92,7 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
                         const __grid_constant__ CUtensorMap tmap_q, TcIndexerParams p) {
   using Cfg = ScoreCfg<CI, NH>;
-  constexpr int kStages = Cfg::kStages, kTmemCols = Cfg::kTmemCols;
+  constexpr int kStages = Cfg::kStages, kTmemCols = Cfg::kTmemCols, kAcc = Cfg::kAccSets;
   pdl_trigger();
   const IndexerArgs& a = p.a;
   const int T = (int)p.t_count;
@@ -138,7 +144,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
       const int64_t n = eligible(a, a.t_begin + t);
       nelig[t] = (int32_t)n;
       // queries that take all of their entries are not scored
-      prefix[t] = n <= a.skip_le ? 0 : (int32_t)((n + kItemRows - 1) / kItemRows);
+      prefix[t] = n <= a.skip_le ? 0 : (int32_t)((n + Cfg::kItem - 1) / Cfg::kItem);
       sum += prefix[t];
     }
     int32_t incl = sum;
@@ -219,7 +225,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
       while (item >= 0) {
         const int32_t chunk = item - prefix[tq];
         const int64_t t = a.t_begin + tq;
-        const int64_t s0 = (int64_t)chunk * kItemRows;
+        const int64_t s0 = (int64_t)chunk * Cfg::kItem;
         const int rs = (int)(issued % kRing);
         if (!mbar_wait(smem_u32(&ring_empty[rs]), (uint32_t)(((issued / kRing) & 1) ^ 1))) {
           report(a.err, kErrTimeout, (int32_t)t, 16);
@@ -243,14 +249,16 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
         mbar_arrive_expect_tx(fb, Cfg::kStageKey + Cfg::kQBytes);
         const uint32_t kst = keys_sm + slot * Cfg::kStageKey;
         if (a.keys.page_table == nullptr) {
-          // contiguous: the item's 256 keys are one 256-row box per column block
+          // contiguous: 256-row boxes per column block
 #pragma unroll
           for (int kb = 0; kb < Cfg::kKB; ++kb)
-            tc::tma_load_2d(kst + kb * Cfg::kKeyBlk, &tmap_keys, 64 * kb,
-                            (int32_t)((int64_t)seq * a.keys.seq_stride + s0), fb);
+#pragma unroll
+            for (int hh = 0; hh < Cfg::kItem / kItemRows; ++hh)
+              tc::tma_load_2d(kst + kb * Cfg::kKeyBlk + hh * kItemRows * 128, &tmap_keys, 64 * kb,
+                              (int32_t)((int64_t)seq * a.keys.seq_stride + s0 + hh * kItemRows), fb);
         } else {
 #pragma unroll
-        for (int h = 0; h < kItemRows / kBoxRows; ++h) {
+        for (int h = 0; h < Cfg::kItem / kBoxRows; ++h) {
           const int64_t s = s0 + h * kBoxRows;
           int64_t row;
           {
@@ -321,7 +329,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
         tc::fence_after_sync();
         const uint32_t qa = q_sm + slot * Cfg::kQBytes;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < Cfg::kTiles; ++h) {
 #pragma unroll
           for (int kb = 0; kb < Cfg::kKB; ++kb) {
             const uint32_t ka = keys_sm + slot * Cfg::kStageKey + kb * Cfg::kKeyBlk + h * kKeyTileBytes;
@@ -349,7 +357,7 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
     int t_cached = -1;
     int64_t n_elig = 0;
     uint32_t tau = 0;
-    CandidateBatch<2> pend;   // the previous item's candidates, stored after this item's atomic
+    CandidateBatch<Cfg::kTiles> pend;   // the previous item's candidates, stored after this item's atomic
     for (int64_t j = group;; j += 2) {
       const int rs = (int)(j % kRing);
       if (!mbar_wait(smem_u32(&ring_full[rs]), (uint32_t)((j / kRing) & 1))) {
@@ -381,37 +389,38 @@ indexer_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys,
         break;
       }
       tc::fence_after_sync();
-      // this key's ReLU-weighted head sum in each of the two tiles, NH
-      // columns each, 16 columns per TMEM load
+      // this key's ReLU-weighted head sum in each tile, NH columns each, 16
+      // columns per TMEM load, every tile's load of a column group before one wait
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * Cfg::kAccCols;
-      float scs[2] = {0.f, 0.f};
+      float scs[Cfg::kTiles];
+#pragma unroll
+      for (int h = 0; h < Cfg::kTiles; ++h) scs[h] = 0.f;
 #pragma unroll
       for (int c = 0; c < NH / 16; ++c) {
-        uint32_t r0[16], r1[16];
-        tc::tmem_ld16(taddr + 16 * c, r0);
-        tc::tmem_ld16(taddr + NH + 16 * c, r1);
+        uint32_t r[Cfg::kTiles][16];
+#pragma unroll
+        for (int h = 0; h < Cfg::kTiles; ++h) tc::tmem_ld16(taddr + h * NH + 16 * c, r[h]);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          scs[0] = fmaf(wv[16 * c + k], fmaxf(__uint_as_float(r0[k]), 0.f), scs[0]);
-          scs[1] = fmaf(wv[16 * c + k], fmaxf(__uint_as_float(r1[k]), 0.f), scs[1]);
-        }
+        for (int h = 0; h < Cfg::kTiles; ++h)
+#pragma unroll
+          for (int k = 0; k < 16; ++k) scs[h] = fmaf(wv[16 * c + k], fmaxf(__uint_as_float(r[h][k]), 0.f), scs[h]);
       }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[acc]));
-      const int64_t s0 = (int64_t)chunk * kItemRows;
-      bool pass[2];
-      uint32_t keys[2], ents[2];
+      const int64_t s0 = (int64_t)chunk * Cfg::kItem;
+      bool pass[Cfg::kTiles];
+      uint32_t keys[Cfg::kTiles], ents[Cfg::kTiles];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < Cfg::kTiles; ++h) {
         const float sc = scs[h];
         const int64_t s = s0 + h * kTileRows + row;
         keys[h] = score_key(sc);
         ents[h] = (uint32_t)s;
         pass[h] = s < n_elig && keys[h] >= tau;
       }
-      CandidateBatch<2> cur;
+      CandidateBatch<Cfg::kTiles> cur;
       cur.issue(a, tq, pass, keys, ents);
       pend.flush(a);
       pend = cur;

@@ -1009,6 +1009,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
 indexer_score_fp4_tc_kernel(TcIndexerParams p) {
   using Cfg = Fp4Cfg<CI, NH, MODE == kFp4Sample>;
   constexpr int kStages = Cfg::kStages, kAccF = Cfg::kAccF;
+  pdl_trigger();   // the next launch may set itself up; it waits for this one's results
   const IndexerArgs& a = p.a;
   const int T = (int)p.t_count;
   extern __shared__ uint8_t smem_raw[];
@@ -1081,6 +1082,9 @@ indexer_score_fp4_tc_kernel(TcIndexerParams p) {
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // the work counter and the query images come from the preceding launch,
+    // which may still run while this kernel sets itself up
+    pdl_wait();
     int64_t issued = 0;
     bool ok = true;
     const int32_t Vs = (int32_t)((int64_t)V * kStaticPct / 100);
@@ -1310,6 +1314,7 @@ indexer_score_fp4_tc_kernel(TcIndexerParams p) {
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    pdl_wait();   // tau and the zeroed candidate counts (fused pass) come from the preceding launch
     const int ew = warp - 2;
     const int group = ew >> 2;
     const int quarter = warp & 3;
@@ -1531,8 +1536,8 @@ cudaError_t launch_score_fp4_tc(const Launch& L, const IndexerArgs& a, int64_t t
   cudaFuncSetAttribute(indexer_score_fp4_tc_kernel<CI, NH, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        Cfg::kSmem);
   prefer_max_shared(indexer_score_fp4_tc_kernel<CI, NH, MODE>);
-  indexer_score_fp4_tc_kernel<CI, NH, MODE><<<(unsigned)sms, kFThreads, Cfg::kSmem, L.stream>>>(p);
-  return cudaSuccess;
+  return launch_kernel(indexer_score_fp4_tc_kernel<CI, NH, MODE>, dim3((unsigned)sms), dim3(kFThreads),
+                       (size_t)Cfg::kSmem, L.stream, true, p);
 }
 
 }  // namespace

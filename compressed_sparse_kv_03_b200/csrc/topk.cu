@@ -845,6 +845,8 @@ __device__ __forceinline__ void warp_take_lowest_ties(uint32_t* sel, const uint3
 constexpr int kTWarps = 4;
 __global__ void __launch_bounds__(kTWarps * 32) topk_threshold_many_kernel(IndexerArgs a, int top_k,
                                                                         int64_t t_count, int qb) {
+  pdl_wait();      // the sample pass's keys are complete (and it no longer uses the work counter)
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     *a.fb_count = 0u;
@@ -1161,7 +1163,9 @@ cudaError_t launch_topk_threshold_many(const Launch& L, const IndexerArgs& a, in
   L.begin(kKernelTopkSample);
   prefer_max_shared(topk_threshold_many_kernel);
   const unsigned grid = (unsigned)((t_count + kTWarps - 1) / kTWarps);
-  topk_threshold_many_kernel<<<grid, kTWarps * 32, 0, L.stream>>>(a, top_k, t_count, qb);
+  const cudaError_t e = launch_kernel(topk_threshold_many_kernel, dim3(grid), dim3(kTWarps * 32), 0, L.stream,
+                                      true, a, top_k, t_count, qb);
+  if (e != cudaSuccess) return e;
   return L.end(kKernelTopkSample);
 }
 

@@ -37,6 +37,8 @@
 // Recomputed keys (sample and fallback) use plain fp32 arithmetic; they can
 // differ from the scorer's in the last bits, which only moves near-ties.  The
 // sample never affects the result, only how many candidates are kept.
+#include <cooperative_groups.h>
+
 #include "kernels.h"
 #include "lowprec.cuh"
 #include "score_mma.cuh"
@@ -251,18 +253,26 @@ __device__ uint32_t warp_sample_threshold(const uint32_t* skey, int ns, int64_t 
 
 // Sampled entries: ns = max(1024, n/32) (at most n, a multiple of 16), as
 // ns / 16 groups of 16 consecutive entries, group i starting at i n / (ns/16).
-__device__ __forceinline__ int sample_size(int64_t n) {
+__host__ __device__ __forceinline__ int sample_size(int64_t n) {
   int64_t ns = n / 32 > kSampleMin ? n / 32 : kSampleMin;
   if (ns > n) ns = n;
   if (ns > kSampleMax) ns = kSampleMax;
   return (int)(ns & ~int64_t(15));
 }
 
-// bf16 keys: each warp scores groups of 16 entries with mma.sync, kU groups
-// with their loads in flight at a time.
-// Dynamic shared memory: sample keys [kSampleMax].
-template <int CI, int NT>
+// bf16 keys: C CTAs per query (a thread-block cluster when C > 1), each
+// scoring its share of the groups of 16 entries with mma.sync (kU groups with
+// their loads in flight at a time) into its own shared memory; with C > 1 the
+// first CTA gathers the keys through distributed shared memory.  The first CTA
+// sets tau: one warp's register select for samples of up to kWarpSample keys
+// on one CTA, else the block-wide select.  C = 1 leaves most SMs to the scorer
+// that overlaps this pass; large samples (long contexts) take C = 4.
+// Dynamic shared memory: sample keys [kSampleMax] (each CTA fills the slots of
+// its groups).
+constexpr int kSampleCluster = 4;
+template <int CI, int NT, int C>
 __global__ void __launch_bounds__(kSampleThreads) topk_sample_kernel(IndexerArgs a, int top_k) {
+  namespace cg = cooperative_groups;
   constexpr int kU = (CI == 128 && NT >= 4) ? 2 : (CI == 128 || NT >= 4) ? 4 : 8;
   extern __shared__ uint32_t skey[];
   __shared__ int hist[2048];
@@ -271,9 +281,11 @@ __global__ void __launch_bounds__(kSampleThreads) topk_sample_kernel(IndexerArgs
   __shared__ int s_above, s_ok;
 
   pdl_trigger();   // the scorer may start streaming keys; it waits before it reads tau
-  const int64_t tl = blockIdx.x;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = C > 1 ? (int)cluster.block_rank() : 0;
+  const int64_t tl = blockIdx.x / C;
   const int64_t t = a.t_begin + tl;
-  if (threadIdx.x == 0) a.cand_count[tl] = 0u;
+  if (threadIdx.x == 0 && rank == 0) a.cand_count[tl] = 0u;
   // the query's position, sequence and head fragments load together
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, q4 = lane & 3;
@@ -281,18 +293,16 @@ __global__ void __launch_bounds__(kSampleThreads) topk_sample_kernel(IndexerArgs
   const int32_t seq = a.seq_id ? __ldg(a.seq_id + t) : 0;
   QueryFrags<CI, NT> Q;
   Q.load(a, t, g, q4);
-  // few entries: every key is a candidate (cand_cap >= 2 top_k), nothing to sample
+  // few entries: every key is a candidate (cand_cap >= 2 top_k), nothing to
+  // sample (the same for every CTA of the cluster: none waits at its barriers)
   if (n <= a.skip_le || 2 * n <= a.cand_cap) {
-    if (threadIdx.x == 0) const_cast<uint32_t*>(a.tau)[tl] = 0u;
+    if (threadIdx.x == 0 && rank == 0) const_cast<uint32_t*>(a.tau)[tl] = 0u;
     return;
   }
   const int ns = sample_size(n);
   const int ng = ns / 16;
-  const bool by_warp = ns <= kWarpSample;   // the common case: one warp sets tau
-  if (!by_warp)
-    for (int b = threadIdx.x; b < 2048; b += kSampleThreads) hist[b] = 0;
-  __syncthreads();
-  for (int g0 = warp * kU; g0 < ng; g0 += (kSampleThreads / 32) * kU) {
+  const int g_hi = (rank + 1) * ng / C;   // this CTA's groups: [rank ng / C, g_hi)
+  for (int g0 = rank * ng / C + warp * kU; g0 < g_hi; g0 += (kSampleThreads / 32) * kU) {
     uint4 kr[kU][2][CI / 32];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
@@ -300,7 +310,7 @@ __global__ void __launch_bounds__(kSampleThreads) topk_sample_kernel(IndexerArgs
       const int64_t e0 = (int64_t)grp * n / ng;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int64_t row = grp < ng ? cache_row(a.keys, seq, e0 + g + 8 * h, nullptr, 0) : -1;
+        const int64_t row = grp < g_hi ? cache_row(a.keys, seq, e0 + g + 8 * h, nullptr, 0) : -1;
 #pragma unroll
         for (int v = 0; v < CI / 32; ++v)
           kr[u][h][v] = row >= 0 ? ld_stream_16(a.keys.data + row * CI + 32 * v + 8 * q4)
@@ -312,23 +322,32 @@ __global__ void __launch_bounds__(kSampleThreads) topk_sample_kernel(IndexerArgs
       float sg, s8;
       score_group<CI, NT>(kr[u], Q, sg, s8);
       const int grp = g0 + u;
-      if (grp < ng && q4 < 2) {
-        const uint32_t key = score_key(q4 == 0 ? sg : s8);
-        skey[grp * 16 + g + 8 * q4] = key;
-        if (!by_warp) atomicAdd(&hist[key >> 21], 1);   // the first radix level
+      if (grp < g_hi && q4 < 2) skey[grp * 16 + g + 8 * q4] = score_key(q4 == 0 ? sg : s8);
+    }
+  }
+  if (C > 1) {
+    cluster.sync();   // every CTA's keys are in its shared memory
+    if (rank == 0) {
+      for (int r = 1; r < C; ++r) {
+        const uint32_t* rk = cluster.map_shared_rank(skey, r);
+        const int lo = (r * ng / C) * 16, hi = ((r + 1) * ng / C) * 16;
+        for (int i = lo + (int)threadIdx.x; i < hi; i += kSampleThreads) skey[i] = rk[i];
       }
     }
-  }
-  __syncthreads();
-  if (by_warp) {
-    if (warp == 0) {
-      const uint32_t tau = warp_sample_threshold(skey, ns, n, top_k);
-      if (lane == 0) const_cast<uint32_t*>(a.tau)[tl] = tau;
+    cluster.sync();   // the other CTAs' keys have been read before any of them exits
+    if (rank != 0) return;
+  } else {
+    __syncthreads();
+    if (ns <= kWarpSample) {   // the common case: one warp sets tau
+      if (warp == 0) {
+        const uint32_t tau = warp_sample_threshold(skey, ns, n, top_k);
+        if (lane == 0) const_cast<uint32_t*>(a.tau)[tl] = tau;
+      }
+      return;
     }
-    return;
   }
   const uint32_t tau = sample_threshold<kSampleThreads>(skey, ns, n, top_k, hist, warp_sums, &s_bin,
-                                                        &s_above, &s_ok, true);
+                                                        &s_above, &s_ok);
   if (threadIdx.x == 0) const_cast<uint32_t*>(a.tau)[tl] = tau;
 }
 
@@ -1105,6 +1124,25 @@ cudaError_t launch_finish(const Launch& L, const IndexerArgs& a, int top_k, int3
                        L.stream, list == nullptr, a, f);
 }
 
+// A sample kernel as clusters of kSampleCluster CTAs per query.
+template <class K>
+void launch_sample_cluster(K kernel, int64_t t_count, size_t smem, cudaStream_t stream, const IndexerArgs& a,
+                           int top_k) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(t_count * kSampleCluster));
+  cfg.blockDim = dim3(kSampleThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSampleCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, a, top_k);
+}
+
 template <int CI>
 void launch_sample(const Launch& L, const IndexerArgs& a, int top_k, int64_t t_count) {
   if (a.fp4) {
@@ -1118,12 +1156,22 @@ void launch_sample(const Launch& L, const IndexerArgs& a, int top_k, int64_t t_c
   }
   const int nt = (a.H_I + 7) / 8;
   constexpr size_t kBytes = kSampleMax * sizeof(uint32_t);
+  // one CTA per query while the largest sample fits one warp's select, else
+  // clusters of kSampleCluster CTAs
+  const bool clustered = sample_size(a.max_entries) > kWarpSample;
 #define CSA_SAMPLE_CASE(NT_)                                                                   \
   if (nt <= NT_) {                                                                             \
-    prefer_max_shared(topk_sample_kernel<CI, NT_>);                                          \
-    cudaFuncSetAttribute(topk_sample_kernel<CI, NT_>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                         (int)kBytes);                                                         \
-    topk_sample_kernel<CI, NT_><<<(unsigned)t_count, kSampleThreads, kBytes, L.stream>>>(a, top_k); \
+    if (!clustered) {                                                                          \
+      prefer_max_shared(topk_sample_kernel<CI, NT_, 1>);                                     \
+      cudaFuncSetAttribute(topk_sample_kernel<CI, NT_, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                           (int)kBytes);                                                       \
+      topk_sample_kernel<CI, NT_, 1><<<(unsigned)t_count, kSampleThreads, kBytes, L.stream>>>(a, top_k); \
+    } else {                                                                                   \
+      prefer_max_shared(topk_sample_kernel<CI, NT_, kSampleCluster>);                        \
+      cudaFuncSetAttribute(topk_sample_kernel<CI, NT_, kSampleCluster>,                      \
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBytes);          \
+      launch_sample_cluster(topk_sample_kernel<CI, NT_, kSampleCluster>, t_count, kBytes, L.stream, a, top_k); \
+    }                                                                                          \
     return;                                                                                    \
   }
   CSA_SAMPLE_CASE(1)

@@ -236,6 +236,26 @@ def test_indexer_topk_decode_sampled_threshold(H_I, c_I, k):
                    range(B), sc)
 
 
+@pytest.mark.parametrize("H_I,c_I", [(8, 64), (16, 128)])
+def test_indexer_topk_decode_long_context_clustered_sample(H_I, c_I):
+    """More than 32768 eligible entries for some query: the sample of each
+    query is scored by a cluster of CTAs and gathered through distributed
+    shared memory before the threshold is set."""
+    csa = _csa()
+    g = synth.generator(38 + H_I)
+    m, k = 4, 2048
+    pos = torch.tensor([4 * 70000, 4 * 33000 + 3, 50000], dtype=torch.int64)
+    B, S = pos.shape[0], int(pos.max()) // m
+    qI = synth.normal(g, (B, H_I, c_I))
+    w = synth.uniform(g, (B, H_I))
+    KI = synth.normal(g, (B, S, c_I))
+    idx, cnt, sc = csa.indexer_topk(dev(qI), dev(w), csa.Cache.contiguous(dev(KI)), m, k,
+                                    seq_id=dev(torch.arange(B, dtype=torch.int32)), q_pos=dev(pos),
+                                    max_entries=S, return_scores=True)
+    _check_queries(idx, cnt, qI, w, lambda t: f64(KI[t]), lambda t: int(pos[t]) // m, k,
+                   range(B), sc)
+
+
 @pytest.mark.parametrize("return_scores", [False, True])
 def test_indexer_topk_all_equal_scores_beyond_the_candidate_slots(return_scores):
     """20000 eligible entries whose scores are all exactly 0 (every head

@@ -883,7 +883,8 @@ struct Fp4Cfg {
   static constexpr int kStage = ((kSwap ? kSfaOff + kSfa : kRawCOff + kRawCodes) + 1023) / 1024 * 1024;
   static constexpr int kStages = (200 * 1024) / kStage < 8 ? (200 * 1024) / kStage : 8;
   static constexpr int kAccCols = kTiles * kN;
-  static constexpr int kSfCols = 4 * (kTiles + 1) * kKB;  // per set: SFA kTiles x kKB, SFB kKB, 4 columns each
+  // per set: SFA kTiles x kKB, then one SFB copy per issuing warp (kKB each), 4 columns each
+  static constexpr int kSfCols = 4 * (kTiles + 2) * kKB;
   static constexpr int kAccF = 2 * (kAccCols + kSfCols) <= 512 ? 2 : 1;   // accumulator sets
   static constexpr int kSfBase = kAccF * kAccCols;
   static constexpr int kTmemCols = 512;
@@ -1000,9 +1001,11 @@ __global__ void __launch_bounds__(128) fp4_query_image_kernel(IndexerArgs a, int
   }
 }
 
-// producer, MMA issuer, kEpiWarps epilogue warps, then the operand warp
-constexpr int kFThreads = kThreads + 32;
+// producer, MMA issuer, kEpiWarps epilogue warps, the operand warp, a second
+// MMA issuer (the two take alternate halves of an item's tiles)
+constexpr int kFThreads = kThreads + 64;
 constexpr int kOpWarp = kThreads / 32;
+constexpr int kMma2Warp = kOpWarp + 1;
 
 template <int CI, int NH, int MODE>
 __global__ void __launch_bounds__(kFThreads, 1)
@@ -1031,16 +1034,16 @@ indexer_score_fp4_tc_kernel(TcIndexerParams p) {
     for (int i = 0; i < kStages; ++i) {
       slot_q[i] = -1;
       mbar_init(smem_u32(&full_bar[i]), 2);   // the copies' arrival + the query staging's
-      mbar_init(smem_u32(&empty_bar[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), 2);   // both MMA issuers' commits
       mbar_init(smem_u32(&opnd_bar[i]), 1);   // the operand warp's arrival
     }
     for (int i = 0; i < kAccF; ++i) {
-      mbar_init(smem_u32(&tfull_bar[i]), 1);
+      mbar_init(smem_u32(&tfull_bar[i]), 2);   // both MMA issuers' commits
       mbar_init(smem_u32(&tempty_bar[i]), 4);
     }
     for (int i = 0; i < kRing; ++i) {
       mbar_init(smem_u32(&ring_full[i]), 1);
-      mbar_init(smem_u32(&ring_empty[i]), 6);   // the MMA warp, one epilogue group, the operand warp
+      mbar_init(smem_u32(&ring_empty[i]), 7);   // two MMA issuers, one epilogue group, the operand warp
     }
     mbar_fence_init();
   }
@@ -1207,9 +1210,12 @@ indexer_score_fp4_tc_kernel(TcIndexerParams p) {
       for (int64_t d = first; d < issued; ++d)
         mbar_wait(smem_u32(&full_bar[d % kStages]), (uint32_t)((d / kStages) & 1), 200000000ll);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // (lane 0 issues; the operand warp has arranged the stage's operands)
+  } else if (warp == 1 || warp == kMma2Warp) {
+    // ------------------------------------------------------------ MMA issuers
+    // (lane 0 of each issues half of an item's tiles, with its own copy of the
+    // query's scale factors; the operand warp has arranged the stage's operands)
+    const int half = warp == 1 ? 0 : 1;
+    constexpr int kHalf = Cfg::kTiles / 2;
     for (uint32_t j = 0;; ++j) {
       const int rs = (int)(j % kRing);
       bool got = true, end = false;
@@ -1235,19 +1241,20 @@ indexer_score_fp4_tc_kernel(TcIndexerParams p) {
           tc::fence_after_sync();
           const uint32_t sst = base + slot * Cfg::kStage;
           const uint32_t sf = tmem_base + Cfg::kSfBase + acc * Cfg::kSfCols;
+          const uint32_t sfb = sf + 4 * (Cfg::kTiles + half) * Cfg::kKB;   // this issuer's SFB copy
 #pragma unroll
-          for (int i = 0; i < Cfg::kTiles * Cfg::kKB; ++i) tc::copy_scales(sf + 4 * i, sst + Cfg::kSfaOff + i * 512);
+          for (int i = half * kHalf * Cfg::kKB; i < (half + 1) * kHalf * Cfg::kKB; ++i)
+            tc::copy_scales(sf + 4 * i, sst + Cfg::kSfaOff + i * 512);
 #pragma unroll
-          for (int kb = 0; kb < Cfg::kKB; ++kb)
-            tc::copy_scales(sf + 4 * (Cfg::kTiles * Cfg::kKB + kb), sst + Cfg::kSfbOff + kb * 512);
+          for (int kb = 0; kb < Cfg::kKB; ++kb) tc::copy_scales(sfb + 4 * kb, sst + Cfg::kSfbOff + kb * 512);
 #pragma unroll
-          for (int h = 0; h < Cfg::kTiles; ++h)
+          for (int h = half * kHalf; h < (half + 1) * kHalf; ++h)
 #pragma unroll
             for (int kb = 0; kb < Cfg::kKB; ++kb)
               tc::mma_mxf4_ss(tmem_base + acc * Cfg::kAccCols + h * Cfg::kN,
                               tc::smem_desc_sw32(sst + kb * Cfg::kCodeBlk + h * 128 * 32),
                               tc::smem_desc_sw32(sst + Cfg::kQOff + kb * Cfg::kQBlk), Cfg::kIdesc,
-                              sf + 4 * (h * Cfg::kKB + kb), sf + 4 * (Cfg::kTiles * Cfg::kKB + kb), kb > 0);
+                              sf + 4 * (h * Cfg::kKB + kb), sfb + 4 * kb, kb > 0);
           tc::mma_commit(smem_u32(&empty_bar[slot]));
           tc::mma_commit(smem_u32(&tfull_bar[acc]));
         }

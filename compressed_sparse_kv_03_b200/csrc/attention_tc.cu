@@ -183,6 +183,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// a * b + c and a + b on two fp32 lanes per instruction (fma.rn / add.rn
+// .f32x2: each lane rounds as fmaf / fadd do)
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n mov.b64 rc, {%6, %7};\n"
+      " fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 __device__ __forceinline__ float redux_max(float v) {
   float r;
   asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;\n" : "=f"(r) : "f"(v));
@@ -722,7 +741,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         }
         const bool rescale = __any_sync(0xffffffffu, grew);
         if (lane < kHW) {
-          my_bc[lane] = m_run == -INFINITY ? 0.f : m_run;
+          my_bc[lane] = m_run == -INFINITY ? 0.f : -m_run;   // negated: the exponent is s scale + this
           if (rescale) my_bc[kHW + lane] = f;
         }
         __syncwarp();
@@ -753,21 +772,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
         for (int c = 0; c < kHW / 8; ++c) {
           const float4 me0 = *reinterpret_cast<const float4*>(my_bc + c * 8);
           const float4 me1 = *reinterpret_cast<const float4*>(my_bc + c * 8 + 4);
-          const float me[8] = {me0.x, me0.y, me0.z, me0.w, me1.x, me1.y, me1.z, me1.w};
+          const float nme[8] = {me0.x, me0.y, me0.z, me0.w, me1.x, me1.y, me1.z, me1.w};
           uint32_t pk[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int hl = c * 8 + 2 * j;
-            const float p0 = ex2_approx(fmaf(x[hl], scale, -me[2 * j]));
-            const float p1 = ex2_approx(fmaf(x[hl + 1], scale, -me[2 * j + 1]));
-            if (rescale) {
-              lpart[hl] = fmaf(lpart[hl], my_bc[kHW + hl], p0);
-              lpart[hl + 1] = fmaf(lpart[hl + 1], my_bc[kHW + hl + 1], p1);
-            } else {
-              lpart[hl] += p0;
-              lpart[hl + 1] += p1;
-            }
-            pk[j] = pack_bf16(p0, p1);
+            // two heads per instruction: exponent, then the running row sums
+            const float2 e2 = fma2(make_float2(x[hl], x[hl + 1]), make_float2(scale, scale),
+                                   make_float2(nme[2 * j], nme[2 * j + 1]));
+            const float2 p = make_float2(ex2_approx(e2.x), ex2_approx(e2.y));
+            const float2 lp = rescale ? fma2(make_float2(lpart[hl], lpart[hl + 1]),
+                                             make_float2(my_bc[kHW + hl], my_bc[kHW + hl + 1]), p)
+                                      : add2(make_float2(lpart[hl], lpart[hl + 1]), p);
+            lpart[hl] = lp.x;
+            lpart[hl + 1] = lp.y;
+            pk[j] = pack_bf16(p.x, p.y);
           }
           const int chunk = hoff / 8 + c;
           const uint32_t dst = prow + (uint32_t)(((chunk ^ (row & 7)) & 7) << 4);

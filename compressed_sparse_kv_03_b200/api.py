@@ -9,9 +9,10 @@ the current torch stream.  Shapes follow the header:
     indexer_topk_mxfp4   (steps 2-3) on 4-bit queries and keys
     quantize_entries_fp8 entries [..., dim] bf16 -> E4M3 content + scale bytes + bf16 rotary part
     sparse_attn_decode_fp8 (step 4)  decode over those mixed-precision entries
-    sparse_attn_prefill  (step 4)    q [L, H, 128] over kv_comp[idx] + raw window
-    sparse_attn_decode   (step 4)    q [B, H, 128] over cache[idx] + window buffer
-    hca_attn             (step 4)    q [T, H, 128] over all eligible entries + window
+    sparse_attn_prefill  (step 4)    q [L, H, d] over kv_comp[idx] + raw window
+    sparse_attn_decode   (step 4)    q [B, H, d] over cache[idx] + window buffer
+    hca_attn             (step 4)    q [T, H, d] over all eligible entries + window
+                                     (d = 128, or 512: the pages' entry width)
 """
 from __future__ import annotations
 

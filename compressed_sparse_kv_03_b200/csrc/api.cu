@@ -129,19 +129,19 @@ Split attn_split_invariant(int64_t total_max) {
   return Split{(int)n, kInvariantSliceRows};
 }
 
-size_t attn_partials_bytes(int64_t T, int H, int n) {
+size_t attn_partials_bytes(int64_t T, int H, int n, int d = kD) {
   if (n == 1) return kWsHeader;
-  const size_t acc = (size_t)T * n * H * kD * sizeof(float);
+  const size_t acc = (size_t)T * n * H * d * sizeof(float);
   const size_t ml = (size_t)T * n * H * 2 * sizeof(float);
   return kWsHeader + align256(acc) + align256(ml);
 }
 
 // Workspace of a decode call: the mma.sync split (which bounds the tcgen05
 // one) and, in batch-invariant mode, the fixed slices.
-size_t attn_ws_bytes(int64_t T, int H, int64_t total_max) {
-  size_t b = attn_partials_bytes(T, H, attn_split(T, total_max, H).n);
+size_t attn_ws_bytes(int64_t T, int H, int64_t total_max, int d = kD) {
+  size_t b = attn_partials_bytes(T, H, attn_split(T, total_max, H).n, d);
   if (g_batch_invariant.load(std::memory_order_relaxed)) {
-    const size_t bi = attn_partials_bytes(T, H, attn_split_invariant(total_max).n);
+    const size_t bi = attn_partials_bytes(T, H, attn_split_invariant(total_max).n, d);
     if (bi > b) b = bi;
   }
   return b;
@@ -268,9 +268,8 @@ size_t csa_indexer_topk_workspace_size(int64_t T, int64_t max_entries, int32_t t
 
 size_t csa_sparse_attn_decode_workspace_size(int32_t B, int32_t H, int32_t d, int32_t top_k,
                                              int32_t window) {
-  (void)d;
   if (B <= 0 || H <= 0) return kWsHeader;
-  return attn_ws_bytes(B, H, (int64_t)top_k + window);
+  return attn_ws_bytes(B, H, (int64_t)top_k + window, d == 512 ? 512 : kD);
 }
 
 size_t csa_sparse_attn_prefill_workspace_size(int64_t L, int32_t H, int32_t d) {
@@ -280,9 +279,8 @@ size_t csa_sparse_attn_prefill_workspace_size(int64_t L, int32_t H, int32_t d) {
 
 size_t hca_attn_workspace_size(int64_t T, int32_t H, int32_t d, int64_t max_entries,
                                int32_t window) {
-  (void)d;
   if (T <= 0 || H <= 0) return kWsHeader;
-  return attn_ws_bytes(T, H, max_entries + window);
+  return attn_ws_bytes(T, H, max_entries + window, d == 512 ? 512 : kD);
 }
 
 csa_status_t csa_workspace_init(void* ws, size_t ws_bytes, csa_stream_t stream) {
@@ -598,7 +596,8 @@ csa_status_t check_attn_common(const char* name, const csa_bf16* q, const csa_bf
                                int32_t H, int32_t d, int32_t window) {
   if (q == nullptr || out == nullptr) return fail(CSA_ERR_INVALID_ARG, "%s: q and out required", name);
   if (H < 1 || window < 0) return fail(CSA_ERR_INVALID_ARG, "%s: need H >= 1, window >= 0", name);
-  if (d != kD) return fail(CSA_ERR_UNSUPPORTED, "%s: head dim %d not built (128 only)", name, d);
+  if (d != kD && d != 512)
+    return fail(CSA_ERR_UNSUPPORTED, "%s: head dim %d not built (128 or 512)", name, d);
   if (H > 128) return fail(CSA_ERR_UNSUPPORTED, "%s: H > 128 not built", name);
   if (window > kMaxWindow) return fail(CSA_ERR_UNSUPPORTED, "%s: window > %d", name, kMaxWindow);
   if (!aligned16(q) || !aligned16(out)) return fail(CSA_ERR_INVALID_ARG, "%s: q/out alignment", name);
@@ -655,6 +654,7 @@ csa_status_t csa_sparse_attn_prefill(const csa_bf16* q, const csa_bf16* kv_comp,
   if (L > 0x7fffffff) return fail(CSA_ERR_UNSUPPORTED, "%s: L >= 2^31", name);
   if (L == 0) return check_ws(ws, ws_bytes, kWsHeader, name);
   AttnArgs a{};
+  a.d = d;
   a.q = (const __nv_bfloat16*)q;
   a.T = L;
   a.H = H;
@@ -704,7 +704,7 @@ csa_status_t run_decode_attention(AttnArgs a, const char* name, int32_t B, int32
   const bool invariant = g_batch_invariant.load(std::memory_order_relaxed) != 0;
   const Split sp_inv = attn_split_invariant((int64_t)top_k + window);
   const int n_need = invariant && sp_inv.n > sp_ws.n ? sp_inv.n : sp_ws.n;
-  csa_status_t st = check_ws(ws, ws_bytes, attn_partials_bytes(B, H, n_need), name);
+  csa_status_t st = check_ws(ws, ws_bytes, attn_partials_bytes(B, H, n_need, a.d), name);
   if (st != CSA_OK) return st;
   a.use_tc = attention_uses_tc(a);
   if ((st = need_tc_for_qrope(name, a)) != CSA_OK) return st;
@@ -716,7 +716,7 @@ csa_status_t run_decode_attention(AttnArgs a, const char* name, int32_t B, int32
   if (sp.n > 1) {
     char* p = static_cast<char*>(ws) + kWsHeader;
     a.part_acc = reinterpret_cast<float*>(p);
-    a.part_ml = reinterpret_cast<float*>(p + align256((size_t)B * sp.n * H * kD * sizeof(float)));
+    a.part_ml = reinterpret_cast<float*>(p + align256((size_t)B * sp.n * H * a.d * sizeof(float)));
   }
   Launch L{(cudaStream_t)stream};
   return cuda_status(launch_attention(L, a), name);
@@ -793,6 +793,7 @@ csa_status_t csa_sparse_attn_decode(const csa_bf16* q, const csa_cache_t* kv_com
   if (st != CSA_OK) return st;
   AttnArgs a = decode_args(q, kv_comp, win, win_len, idx, count, B, H, top_k, window,
                            sm_scale, sink, out, lse);
+  a.d = d;
   if ((st = apply_qrope(name, qrope, true, a)) != CSA_OK) return st;
   return run_decode_attention(a, name, B, H, top_k, window, ws, ws_bytes, stream);
 }
@@ -831,6 +832,7 @@ csa_status_t csa_sparse_attn_decode_fp8(const csa_bf16* q, const csa_cache_t* kv
   csa_status_t st =
       check_decode_args(name, q, kv_codes, win, win_len, idx, count, B, H, d, top_k, window, out);
   if (st != CSA_OK) return st;
+  if (d != kD) return fail(CSA_ERR_UNSUPPORTED, "%s: mixed-precision entries at head dim 128 only", name);
   if (rope_dims < 0 || rope_dims % 8 != 0 || rope_dims >= kD || (kD - rope_dims) % 32 != 0)
     return fail(CSA_ERR_INVALID_ARG,
                 "%s: rope_dims must be a multiple of 8 below 128 with 128 - rope_dims a multiple "
@@ -868,6 +870,7 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
   if (T > 0x7fffffff) return fail(CSA_ERR_UNSUPPORTED, "%s: T >= 2^31", name);
   if (T == 0) return check_ws(ws, ws_bytes, kWsHeader, name);
   AttnArgs a{};
+  a.d = d;
   a.q = (const __nv_bfloat16*)q;
   a.T = T;
   a.H = H;
@@ -894,7 +897,7 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
   const bool invariant = win_len != nullptr && g_batch_invariant.load(std::memory_order_relaxed) != 0;
   const Split sp_inv = attn_split_invariant(max_entries + window);
   const int n_need = invariant && sp_inv.n > sp_ws.n ? sp_inv.n : sp_ws.n;
-  if ((st = check_ws(ws, ws_bytes, attn_partials_bytes(T, H, n_need), name)) != CSA_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, attn_partials_bytes(T, H, n_need, d), name)) != CSA_OK) return st;
   a.use_tc = attention_uses_tc(a);
   if ((st = need_tc_for_qrope(name, a)) != CSA_OK) return st;
   const Split sp = invariant ? sp_inv
@@ -905,7 +908,7 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
   if (sp.n > 1) {
     char* p = static_cast<char*>(ws) + kWsHeader;
     a.part_acc = reinterpret_cast<float*>(p);
-    a.part_ml = reinterpret_cast<float*>(p + align256((size_t)T * sp.n * H * kD * sizeof(float)));
+    a.part_ml = reinterpret_cast<float*>(p + align256((size_t)T * sp.n * H * d * sizeof(float)));
   }
   Launch L{(cudaStream_t)stream};
   return cuda_status(launch_attention(L, a), name);

@@ -316,53 +316,58 @@ __global__ void __launch_bounds__(32 * kMergeHeads) merge_kernel(AttnArgs a) {
   const int h = blockIdx.y * kMergeHeads + warp;
   if (h >= a.H) return;
   const int ns = a.n_split;
+  const int dd = a.d;   // 128 or 512: blocks of 128 dims, 4 per lane
   const float* const ml = a.part_ml + (i * ns * a.H + h) * 2;
-  const float* const acc = a.part_acc + (i * ns * a.H + h) * D + 4 * lane;
-  const float z = a.sink ? __ldg(a.sink + h) * kLog2e : -INFINITY;
-  float M = z, den = z == -INFINITY ? 0.f : 1.f;   // relative to 2^M
-  float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < ns; s0 += kMergeChunk) {
-    const int cnt = ns - s0 < kMergeChunk ? ns - s0 : kMergeChunk;
-    float2 mls = make_float2(-INFINITY, 0.f);
-    if (lane < cnt) mls = *reinterpret_cast<const float2*>(ml + (int64_t)(s0 + lane) * a.H * 2);
-    float4 v[kMergeChunk];
+  float M = 0.f, den = 0.f;   // the same for every block; the last one's is kept for the LSE
+  for (int d0 = 0; d0 < dd; d0 += D) {
+    const float* const acc = a.part_acc + (i * ns * a.H + h) * dd + d0 + 4 * lane;
+    const float z = a.sink ? __ldg(a.sink + h) * kLog2e : -INFINITY;
+    M = z;
+    den = z == -INFINITY ? 0.f : 1.f;   // relative to 2^M
+    float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < ns; s0 += kMergeChunk) {
+      const int cnt = ns - s0 < kMergeChunk ? ns - s0 : kMergeChunk;
+      float2 mls = make_float2(-INFINITY, 0.f);
+      if (lane < cnt) mls = *reinterpret_cast<const float2*>(ml + (int64_t)(s0 + lane) * a.H * 2);
+      float4 v[kMergeChunk];
 #pragma unroll
-    for (int j = 0; j < kMergeChunk; ++j)
-      if (j < cnt) v[j] = *reinterpret_cast<const float4*>(acc + (int64_t)(s0 + j) * a.H * D);
-    float cm = mls.x;
+      for (int j = 0; j < kMergeChunk; ++j)
+        if (j < cnt) v[j] = *reinterpret_cast<const float4*>(acc + (int64_t)(s0 + j) * a.H * dd);
+      float cm = mls.x;
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
-    const float nM = fmaxf(M, cm);
-    const float ref = nM == -INFINITY ? 0.f : nM;
-    const float fo = exp2f(M - ref);
-    den *= fo;
-    out.x *= fo;
-    out.y *= fo;
-    out.z *= fo;
-    out.w *= fo;
-    const float f_l = lane < cnt ? exp2f(mls.x - ref) : 0.f;
-    float dl = f_l * mls.y;
+      for (int o = 16; o >= 1; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+      const float nM = fmaxf(M, cm);
+      const float ref = nM == -INFINITY ? 0.f : nM;
+      const float fo = exp2f(M - ref);
+      den *= fo;
+      out.x *= fo;
+      out.y *= fo;
+      out.z *= fo;
+      out.w *= fo;
+      const float f_l = lane < cnt ? exp2f(mls.x - ref) : 0.f;
+      float dl = f_l * mls.y;
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
-    den += dl;
+      for (int o = 16; o >= 1; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
+      den += dl;
 #pragma unroll
-    for (int j = 0; j < kMergeChunk; ++j) {
-      const float f = __shfl_sync(0xffffffffu, f_l, j);
-      if (j < cnt) {
-        out.x = fmaf(v[j].x, f, out.x);
-        out.y = fmaf(v[j].y, f, out.y);
-        out.z = fmaf(v[j].z, f, out.z);
-        out.w = fmaf(v[j].w, f, out.w);
+      for (int j = 0; j < kMergeChunk; ++j) {
+        const float f = __shfl_sync(0xffffffffu, f_l, j);
+        if (j < cnt) {
+          out.x = fmaf(v[j].x, f, out.x);
+          out.y = fmaf(v[j].y, f, out.y);
+          out.z = fmaf(v[j].z, f, out.z);
+          out.w = fmaf(v[j].w, f, out.w);
+        }
       }
+      M = nM;
     }
-    M = nM;
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    uint2 pk;
+    pk.x = pack_bf16(out.x * inv, out.y * inv);
+    pk.y = pack_bf16(out.z * inv, out.w * inv);
+    *reinterpret_cast<uint2*>(a.out + (i * a.H + h) * dd + d0 + 4 * lane) = pk;
   }
   const float ref = M == -INFINITY ? 0.f : M;
-  const float inv = den > 0.f ? 1.f / den : 0.f;
-  uint2 pk;
-  pk.x = pack_bf16(out.x * inv, out.y * inv);
-  pk.y = pack_bf16(out.z * inv, out.w * inv);
-  *reinterpret_cast<uint2*>(a.out + (i * a.H + h) * D + 4 * lane) = pk;
   if (a.lse && lane == 0) a.lse[i * a.H + h] = den > 0.f ? (ref + log2f(den)) / kLog2e : -INFINITY;
 }
 
@@ -384,6 +389,14 @@ bool attention_uses_tc(const AttnArgs& a) {
 
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {
   if (a.T == 0) return cudaSuccess;
+  if (a.d == 512) {   // the pages' entry width (attention512.cu)
+    L.begin(kKernelAttention);
+    cudaError_t e = launch_attention512(L, a);
+    if (e != cudaSuccess) return e;
+    e = L.end(kKernelAttention);
+    if (e != cudaSuccess || a.n_split == 1) return e;
+    return launch_merge(L, a);
+  }
   if (a.use_tc) {
     L.begin(kKernelAttention);
     AttnArgs b = a;

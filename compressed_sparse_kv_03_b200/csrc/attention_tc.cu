@@ -909,6 +909,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv_tile,
 }  // namespace
 
 bool tc_attention_supported(const AttnArgs& a) {
+  if (a.d != kD) return false;
   if (a.T * (int64_t)a.H > INT32_MAX || a.kv.n_rows > INT32_MAX) return false;
   if (a.win_len == nullptr && a.window > 0 && a.win_rows <= 0) return false;   // raw rows unknown
   if (a.win_len && a.T * (int64_t)a.window > INT32_MAX) return false;

@@ -230,7 +230,8 @@ cudaError_t launch_topk_finish_many(const Launch& L, const IndexerArgs& a, int t
 // Attention over a virtual row list per query: its selected / eligible
 // compressed entries followed by its window rows.
 struct AttnArgs {
-  const __nv_bfloat16* q;       // [T, H, 128]
+  int d = 128;                  // head dim: 128, or 512 (attention512.cu, mma.sync only)
+  const __nv_bfloat16* q;       // [T, H, d]
   int64_t T;
   int H;
   CacheRef kv;                  // compressed entries
@@ -319,6 +320,8 @@ bool take_attention_timeout_test();
 // the split / workspace ones must be set).
 bool attention_uses_tc(const AttnArgs& a);
 cudaError_t launch_attention_tc(const Launch& L, const AttnArgs& a);
+// head dim 512: one CTA per (query, slice, 16 heads), warps split the dims
+cudaError_t launch_attention512(const Launch& L, const AttnArgs& a);
 
 // [n, dim] bf16 entries -> E4M3 codes [n, dim - rope] + scale bytes
 // [n, (dim - rope)/32] + rotary part [n, rope] bf16: see fp8_entry.cu

@@ -33,8 +33,11 @@
  *     csa_workspace_check), skips that row and carries on; nothing traps.
  *   - csa_last_error() returns a thread-local description of the last failure.
  *
- * Supported sizes: attention head dim d = 128; indexer key dim c_I in {64, 128};
- * indexer heads H_I <= 64; attention heads H <= 128; m >= 1; window <= 1024.
+ * Supported sizes: attention head dim d in {128, 512} (512, the pages' entry
+ * width, runs on an mma.sync kernel whose four warps split the dims; the
+ * mixed-precision entries and the fused query prologue / output de-rotation
+ * need d = 128); indexer key dim c_I in {64, 128}; indexer heads H_I <= 64;
+ * attention heads H <= 128; m >= 1; window <= 1024.
  */
 #ifndef CSA_H
 #define CSA_H

@@ -73,8 +73,8 @@ def test_attention_rejects_unsupported_dims(lib):
     cache = CacheT(p.value, 16, 16, None, 0, 0)
     ws = (C.c_uint8 * 1024)()
     wsp = C.cast(C.addressof(ws) + (-C.addressof(ws)) % 256, C.c_void_p)
-    # head dim 512 is a legal size the library does not build
-    st = lib.csa_sparse_attn_decode(p, C.byref(cache), p, p, p, p, 1, 8, 512, 4, 8, 1.0, None, p,
+    # head dim 256 is a legal size the library does not build (128 and 512 are)
+    st = lib.csa_sparse_attn_decode(p, C.byref(cache), p, p, p, p, 1, 8, 256, 4, 8, 1.0, None, p,
                                     None, wsp, 512, None, None)
     assert st == 2 and b"head dim" in lib.csa_last_error()
     # indexer key dim 96

@@ -121,6 +121,22 @@ Split attn_split_tc(int64_t T, int64_t total_max, int H, const Split& ws) {
   return Split{(int)n, (int)(len_tiles * 128)};
 }
 
+// Split for the head-dim-512 kernel (CTAs of 32 heads, one resident per SM):
+// slices of whole 64-row tiles, as many as fit in one wave of CTAs and never
+// more than `ws`.  Each slice costs a partial O of 2 KB per head written and
+// merged, which measured slower than leaving SMs idle (B = 64, H = 64, 1152
+// rows: 164 us unsplit against 185-191 us at one to four waves of slices).
+Split attn_split_512(int64_t T, int64_t total_max, int H, const Split& ws) {
+  const int64_t ctas = T * ((H + 31) / 32);
+  const int64_t tiles = (total_max + 63) / 64;
+  int64_t n = kNumSMs / ctas;
+  if (n > ws.n) n = ws.n;
+  if (n > tiles) n = tiles;
+  if (n <= 1 || tiles <= 1) return Split{1, (int)(tiles * 64 > 64 ? tiles * 64 : 64)};
+  const int64_t len_tiles = (tiles + n - 1) / n;
+  return Split{(int)((tiles + len_tiles - 1) / len_tiles), (int)(len_tiles * 64)};
+}
+
 // Batch-invariant decode: fixed 512-row slices of every query's row list.
 constexpr int kInvariantSliceRows = 512;
 Split attn_split_invariant(int64_t total_max) {
@@ -709,7 +725,8 @@ csa_status_t run_decode_attention(AttnArgs a, const char* name, int32_t B, int32
   a.use_tc = attention_uses_tc(a);
   if ((st = need_tc_for_qrope(name, a)) != CSA_OK) return st;
   const Split sp = invariant ? sp_inv
-                             : (a.use_tc ? attn_split_tc(B, (int64_t)top_k + window, H, sp_ws) : sp_ws);
+                   : a.use_tc ? attn_split_tc(B, (int64_t)top_k + window, H, sp_ws)
+                   : a.d == 512 ? attn_split_512(B, (int64_t)top_k + window, H, sp_ws) : sp_ws;
   a.n_split = sp.n;
   a.split_len = sp.len;
   a.err = static_cast<WsHeader*>(ws);
@@ -901,7 +918,8 @@ csa_status_t hca_attn(const csa_bf16* q, const csa_cache_t* kv_comp, const csa_b
   a.use_tc = attention_uses_tc(a);
   if ((st = need_tc_for_qrope(name, a)) != CSA_OK) return st;
   const Split sp = invariant ? sp_inv
-                             : (a.use_tc ? attn_split_tc(T, max_entries + window, H, sp_ws) : sp_ws);
+                   : a.use_tc ? attn_split_tc(T, max_entries + window, H, sp_ws)
+                   : a.d == 512 ? attn_split_512(T, max_entries + window, H, sp_ws) : sp_ws;
   a.n_split = sp.n;
   a.split_len = sp.len;
   a.err = static_cast<WsHeader*>(ws);

@@ -5,12 +5,15 @@
 //
 // The same virtual row list, split-KV slices and online softmax as the d = 128
 // mma.sync kernel (attention.cu), laid out for 512-dim rows.  A CTA takes one
-// query, one slice and 16 heads; warp w owns dims [128 w, 128 w + 128): it
+// query, one slice and 32 heads in two groups of 16; warp w of a group owns
+// dims [128 w, 128 w + 128): it
 // contracts its quarter of Q K^T for the tile (mma.sync m16n8k16, bf16 in,
 // fp32 accumulate), the four partial score tiles are summed through shared
 // memory in a fixed order (every warp then holds the same scores and runs the
-// same online softmax), and it accumulates O for its own dims.  Rows arrive 64
-// at a time by cp.async into a double-buffered, XOR-swizzled tile (2 x 64 KB).
+// same online softmax), and it accumulates O for its own dims.  A CTA holds two
+// such groups of four warps (32 heads), which share each tile of rows.  Rows
+// arrive 64 at a time by cp.async into a double-buffered, XOR-swizzled tile
+// (2 x 64 KB).
 #include "kernels.h"
 
 namespace csa {
@@ -19,9 +22,11 @@ namespace {
 
 constexpr int kD5 = 512;         // head dim
 constexpr int kBN5 = 64;         // rows per tile
-constexpr int kW5 = 4;           // warps; warp w owns dims [kDW5 w, kDW5 (w + 1))
-constexpr int kDW5 = kD5 / kW5;  // 128
-constexpr int kHeads5 = 16;      // heads per CTA
+constexpr int kQ5 = 4;           // warps per head group; warp w owns dims [kDW5 w, kDW5 (w + 1))
+constexpr int kG5 = 2;           // head groups of 16 per CTA
+constexpr int kW5 = kQ5 * kG5;   // warps
+constexpr int kDW5 = kD5 / kQ5;  // 128
+constexpr int kHeads5 = 16 * kG5;   // heads per CTA
 constexpr size_t kSmem5 = 2 * kBN5 * kD5 * sizeof(__nv_bfloat16) + kW5 * 32 * 32 * sizeof(float);
 
 __global__ void __launch_bounds__(kW5 * 32) attn512_kernel(AttnArgs a) {
@@ -36,8 +41,9 @@ __global__ void __launch_bounds__(kW5 * 32) attn512_kernel(AttnArgs a) {
   const int split = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, q4 = lane & 3;
-  const int head0 = blockIdx.z * kHeads5;
-  const int dw0 = warp * kDW5;
+  const int hgrp = warp / kQ5, dq = warp % kQ5;
+  const int head0 = blockIdx.z * kHeads5 + 16 * hgrp;
+  const int dw0 = dq * kDW5;
   const bool reporter = split == 0 && tid == 0 && blockIdx.z == 0;
 
   // ---- this query's virtual row list ----
@@ -166,10 +172,10 @@ __global__ void __launch_bounds__(kW5 * 32) attn512_kernel(AttnArgs a) {
       __syncthreads();
 #pragma unroll
       for (int j = 0; j < kBN5 / 8; ++j) {
-        float4 t = *reinterpret_cast<const float4*>(sS + (0 * 32 + lane) * 32 + 4 * j);
+        float4 t = *reinterpret_cast<const float4*>(sS + ((hgrp * kQ5 + 0) * 32 + lane) * 32 + 4 * j);
 #pragma unroll
-        for (int w2 = 1; w2 < kW5; ++w2) {
-          const float4 u = *reinterpret_cast<const float4*>(sS + (w2 * 32 + lane) * 32 + 4 * j);
+        for (int w2 = 1; w2 < kQ5; ++w2) {
+          const float4 u = *reinterpret_cast<const float4*>(sS + ((hgrp * kQ5 + w2) * 32 + lane) * 32 + 4 * j);
           t.x += u.x;
           t.y += u.y;
           t.z += u.z;
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(kW5 * 32) attn512_kernel(AttnArgs a) {
         *reinterpret_cast<uint32_t*>(a.out + (i * a.H + h_hi) * kD5 + c) =
             pack_bf16(acc[n][2] * inv_hi, acc[n][3] * inv_hi);
     }
-    if (a.lse && q4 == 0 && warp == 0) {
+    if (a.lse && q4 == 0 && dq == 0) {
       if (h_lo < a.H) a.lse[i * a.H + h_lo] = den_lo > 0.f ? (mm_lo + log2f(den_lo)) / kLog2e : -INFINITY;
       if (h_hi < a.H) a.lse[i * a.H + h_hi] = den_hi > 0.f ? (mm_hi + log2f(den_hi)) / kLog2e : -INFINITY;
     }
@@ -288,7 +294,7 @@ __global__ void __launch_bounds__(kW5 * 32) attn512_kernel(AttnArgs a) {
       if (h_hi < a.H)
         *reinterpret_cast<float2*>(a.part_acc + (pbase + h_hi) * kD5 + c) = make_float2(acc[n][2], acc[n][3]);
     }
-    if (q4 == 0 && warp == 0) {
+    if (q4 == 0 && dq == 0) {
       if (h_lo < a.H) *reinterpret_cast<float2*>(a.part_ml + (pbase + h_lo) * 2) = make_float2(m_lo, l_lo);
       if (h_hi < a.H) *reinterpret_cast<float2*>(a.part_ml + (pbase + h_hi) * 2) = make_float2(m_hi, l_hi);
     }

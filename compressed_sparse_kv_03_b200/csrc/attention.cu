@@ -382,9 +382,21 @@ cudaError_t launch_merge(const Launch& L, const AttnArgs& a) {
 
 }  // namespace
 
+// Short row lists favour the mma.sync kernel: the tensor-core kernel's fixed
+// cost per (query, slice) item (query tile, first scores, epilogue: about
+// 4 us) then outweighs its tiles.  Measured at L = 4096, m = 4, W = 128 with
+// H from 8 to 64: k = 64 (at most 192 rows) 100-164 us against 179-182 us;
+// k = 512 (640 rows) 236-369 us against 250-254 us, and decode at k = 2048
+// 38-66 us against 32-36 us.  The automatic choice keeps the tensor-core
+// kernel for the fused query prologue and output de-rotation, which only it
+// implements.
+constexpr int64_t kTcMinRows = 257;
 bool attention_uses_tc(const AttnArgs& a) {
   const int32_t choice = attention_kernel_choice();
-  return choice != 2 && tc_attention_supported(a);
+  if (choice == 2 || !tc_attention_supported(a)) return false;
+  if (choice == 1) return true;
+  const int64_t rows = (a.idx ? (int64_t)a.top_k : a.max_entries) + a.window;
+  return rows >= kTcMinRows || a.qprologue || a.out_derotate;
 }
 
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {

@@ -121,15 +121,15 @@ Split attn_split_tc(int64_t T, int64_t total_max, int H, const Split& ws) {
   return Split{(int)n, (int)(len_tiles * 128)};
 }
 
-// Split for the head-dim-512 kernel (CTAs of 32 heads, one resident per SM):
-// slices of whole 64-row tiles, as many as fit in one wave of CTAs and never
+// Split for the head-dim-512 kernel (CTAs of 32 heads, two resident per SM):
+// slices of whole 64-row spans, as many as fit in one wave of CTAs and never
 // more than `ws`.  Each slice costs a partial O of 2 KB per head written and
-// merged, which measured slower than leaving SMs idle (B = 64, H = 64, 1152
-// rows: 164 us unsplit against 185-191 us at one to four waves of slices).
+// merged, so the split stops at one wave (B = 64, H = 64, 1152 rows: 134 us
+// at two slices against 150 us unsplit).
 Split attn_split_512(int64_t T, int64_t total_max, int H, const Split& ws) {
   const int64_t ctas = T * ((H + 31) / 32);
   const int64_t tiles = (total_max + 63) / 64;
-  int64_t n = kNumSMs / ctas;
+  int64_t n = 2 * kNumSMs / ctas;
   if (n > ws.n) n = ws.n;
   if (n > tiles) n = tiles;
   if (n <= 1 || tiles <= 1) return Split{1, (int)(tiles * 64 > 64 ? tiles * 64 : 64)};

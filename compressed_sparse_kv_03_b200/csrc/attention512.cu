@@ -12,8 +12,10 @@
 // memory in a fixed order (every warp then holds the same scores and runs the
 // same online softmax), and it accumulates O for its own dims.  A CTA holds two
 // such groups of four warps (32 heads), which share each tile of rows.  Rows
-// arrive 64 at a time by cp.async into a double-buffered, XOR-swizzled tile
-// (2 x 64 KB).
+// arrive 32 at a time by cp.async into a double-buffered, XOR-swizzled tile
+// (2 x 32 KB); the query's heads sit in shared memory (32 KB) and are read
+// as MMA fragments per step, so that a thread stays within 128 registers and
+// two CTAs share an SM.
 #include "kernels.h"
 
 namespace csa {
@@ -21,19 +23,23 @@ namespace csa {
 namespace {
 
 constexpr int kD5 = 512;         // head dim
-constexpr int kBN5 = 64;         // rows per tile
+constexpr int kBN5 = 32;         // rows per tile
 constexpr int kQ5 = 4;           // warps per head group; warp w owns dims [kDW5 w, kDW5 (w + 1))
 constexpr int kG5 = 2;           // head groups of 16 per CTA
 constexpr int kW5 = kQ5 * kG5;   // warps
 constexpr int kDW5 = kD5 / kQ5;  // 128
 constexpr int kHeads5 = 16 * kG5;   // heads per CTA
-constexpr size_t kSmem5 = 2 * kBN5 * kD5 * sizeof(__nv_bfloat16) + kW5 * 32 * 32 * sizeof(float);
+constexpr int kSw5 = kBN5 / 2;   // floats per lane in the score exchange (kBN5 / 8 fragments of 4)
+constexpr size_t kQOff5 = 2 * kBN5 * kD5 * sizeof(__nv_bfloat16);
+constexpr size_t kSOff5 = kQOff5 + kHeads5 * kD5 * sizeof(__nv_bfloat16);
+constexpr size_t kSmem5 = kSOff5 + kW5 * 32 * kSw5 * sizeof(float);   // 112 KB: two CTAs per SM
 
-__global__ void __launch_bounds__(kW5 * 32) attn512_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(kW5 * 32, 2) attn512_kernel(AttnArgs a) {
   constexpr int NTH = kW5 * 32;
   extern __shared__ __align__(128) uint8_t smem5[];
   __nv_bfloat16* const sKV = reinterpret_cast<__nv_bfloat16*>(smem5);                   // 2 x kBN5 x kD5
-  float* const sS = reinterpret_cast<float*>(smem5 + 2 * kBN5 * kD5 * sizeof(__nv_bfloat16));
+  __nv_bfloat16* const sQ = reinterpret_cast<__nv_bfloat16*>(smem5 + kQOff5);          // kHeads5 x kD5
+  float* const sS = reinterpret_cast<float*>(smem5 + kSOff5);
   __shared__ const __nv_bfloat16* sRow[2][kBN5];
   __shared__ uint32_t sMask[2][2];
 
@@ -92,7 +98,7 @@ __global__ void __launch_bounds__(kW5 * 32) attn512_kernel(AttnArgs a) {
       }
       sRow[st][r] = p;
       const uint32_t bits = __ballot_sync(0xffffffffu, p != nullptr);
-      if (lane == 0) sMask[st][r0 >> 5] = bits;
+      if (lane == 0) sMask[st][r0 >> 5] = bits;   // kBN5 = 32: word 0
     }
   };
   // row r's 16-byte chunk ch at r * kD5 + 8 (ch ^ (r mod 8)) elements
@@ -106,20 +112,14 @@ __global__ void __launch_bounds__(kW5 * 32) attn512_kernel(AttnArgs a) {
     }
   };
 
-  // ---- this warp's quarter of the query fragments (A operand, rows = heads) ----
-  uint32_t qa[kDW5 / 16][4];
-  {
-    const int h_lo = head0 + g, h_hi = head0 + g + 8;
-    const __nv_bfloat16* qlo = a.q + (i * a.H + h_lo) * kD5 + dw0;
-    const __nv_bfloat16* qhi = a.q + (i * a.H + h_hi) * kD5 + dw0;
-#pragma unroll
-    for (int kk = 0; kk < kDW5 / 16; ++kk) {
-      const int c = kk * 16 + 2 * q4;
-      qa[kk][0] = h_lo < a.H ? *reinterpret_cast<const uint32_t*>(qlo + c) : 0u;
-      qa[kk][1] = h_hi < a.H ? *reinterpret_cast<const uint32_t*>(qhi + c) : 0u;
-      qa[kk][2] = h_lo < a.H ? *reinterpret_cast<const uint32_t*>(qlo + c + 8) : 0u;
-      qa[kk][3] = h_hi < a.H ? *reinterpret_cast<const uint32_t*>(qhi + c + 8) : 0u;
-    }
+  // ---- the CTA's 32 heads of the query in shared memory: head h's 16-byte
+  // chunk ch at h * kD5 + 8 (ch ^ (h mod 8)) elements (zeros past H) ----
+  for (int c = tid; c < kHeads5 * (kD5 / 8); c += NTH) {
+    const int hh = c / (kD5 / 8), ch = c % (kD5 / 8);
+    const int h = blockIdx.z * kHeads5 + hh;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (h < a.H) v = *reinterpret_cast<const uint4*>(a.q + (i * a.H + h) * kD5 + ch * 8);
+    *reinterpret_cast<uint4*>(sQ + hh * kD5 + ((ch ^ (hh & 7)) << 3)) = v;
   }
   const float scale = a.sm_scale * kLog2e;
 
@@ -148,8 +148,15 @@ __global__ void __launch_bounds__(kW5 * 32) attn512_kernel(AttnArgs a) {
     float s[kBN5 / 8][4];
 #pragma unroll
     for (int j = 0; j < kBN5 / 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+    const uint32_t qbase = smem_u32(sQ);
 #pragma unroll
     for (int kk = 0; kk < kDW5 / 16; ++kk) {
+      uint32_t qa[4];   // heads 16 hgrp + (0..15) x dims dw0 + 16 kk + (0..15)
+      {
+        const int hr = 16 * hgrp + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int ch = dw0 / 8 + 2 * kk + (lane >> 4);
+        ldmatrix_x4(qa, qbase + (uint32_t)(hr * kD5 + ((ch ^ (hr & 7)) << 3)) * 2u);
+      }
 #pragma unroll
       for (int jp = 0; jp < kBN5 / 16; ++jp) {
         const int mi = lane >> 3, rr = lane & 7;
@@ -157,25 +164,25 @@ __global__ void __launch_bounds__(kW5 * 32) attn512_kernel(AttnArgs a) {
         const int ch = dw0 / 8 + 2 * kk + (mi & 1);
         uint32_t r[4];
         ldmatrix_x4(r, sbase + (uint32_t)(row * kD5 + ((ch ^ (row & 7)) << 3)) * 2u);
-        mma_bf16_16816(s[2 * jp], qa[kk], r[0], r[1]);
-        mma_bf16_16816(s[2 * jp + 1], qa[kk], r[2], r[3]);
+        mma_bf16_16816(s[2 * jp], qa, r[0], r[1]);
+        mma_bf16_16816(s[2 * jp + 1], qa, r[2], r[3]);
       }
     }
     // the four quarters meet in shared memory (the same fragment layout in
     // every warp); every warp sums them in the same order, so all four hold
     // the same scores bit for bit
     {
-      float* const mine = sS + (warp * 32 + lane) * 32;
+      float* const mine = sS + (warp * 32 + lane) * kSw5;
 #pragma unroll
       for (int j = 0; j < kBN5 / 8; ++j)
         *reinterpret_cast<float4*>(mine + 4 * j) = make_float4(s[j][0], s[j][1], s[j][2], s[j][3]);
       __syncthreads();
 #pragma unroll
       for (int j = 0; j < kBN5 / 8; ++j) {
-        float4 t = *reinterpret_cast<const float4*>(sS + ((hgrp * kQ5 + 0) * 32 + lane) * 32 + 4 * j);
+        float4 t = *reinterpret_cast<const float4*>(sS + ((hgrp * kQ5 + 0) * 32 + lane) * kSw5 + 4 * j);
 #pragma unroll
         for (int w2 = 1; w2 < kQ5; ++w2) {
-          const float4 u = *reinterpret_cast<const float4*>(sS + ((hgrp * kQ5 + w2) * 32 + lane) * 32 + 4 * j);
+          const float4 u = *reinterpret_cast<const float4*>(sS + ((hgrp * kQ5 + w2) * 32 + lane) * kSw5 + 4 * j);
           t.x += u.x;
           t.y += u.y;
           t.z += u.z;
@@ -188,13 +195,13 @@ __global__ void __launch_bounds__(kW5 * 32) attn512_kernel(AttnArgs a) {
       }
     }
     // online softmax (log2 domain); rows g (lo) and g + 8 (hi) are heads
-    const uint64_t vmask = (uint64_t)sMask[st][0] | ((uint64_t)sMask[st][1] << 32);
+    const uint32_t vmask = sMask[st][0];
     float mx_lo = -INFINITY, mx_hi = -INFINITY;
 #pragma unroll
     for (int j = 0; j < kBN5 / 8; ++j) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const bool ok = (vmask >> (8 * j + 2 * q4 + c)) & 1ull;
+        const bool ok = (vmask >> (8 * j + 2 * q4 + c)) & 1u;
         s[j][c] = ok ? s[j][c] * scale : -INFINITY;
         s[j][2 + c] = ok ? s[j][2 + c] * scale : -INFINITY;
         mx_lo = fmaxf(mx_lo, s[j][c]);

@@ -25,14 +25,16 @@ namespace csa {
 namespace {
 
 constexpr int D = 128;
-constexpr int BN = 64;   // rows per tile
 
 __device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) {
   return *reinterpret_cast<const uint32_t*>(p);
 }
 
-template <int NW>
+// BN rows per tile (32 or 64): with few warps per CTA the 2 x BN x 256 B of
+// row tiles is what limits the CTAs resident on an SM.
+template <int NW, int BN>
 __global__ void __launch_bounds__(NW * 32) attn_kernel(AttnArgs a) {
+  static_assert(BN == 32 || BN == 64, "row tiles of 32 or 64");
   constexpr int NTH = NW * 32;
   __shared__ alignas(128) __nv_bfloat16 sKV[2][BN * D];
   __shared__ const __nv_bfloat16* sRow[2][BN];
@@ -382,21 +384,30 @@ cudaError_t launch_merge(const Launch& L, const AttnArgs& a) {
 
 }  // namespace
 
-// Short row lists favour the mma.sync kernel: the tensor-core kernel's fixed
-// cost per (query, slice) item (query tile, first scores, epilogue: about
-// 4 us) then outweighs its tiles.  Measured at L = 4096, m = 4, W = 128 with
-// H from 8 to 64: k = 64 (at most 192 rows) 100-164 us against 179-182 us;
-// k = 512 (640 rows) 236-369 us against 250-254 us, and decode at k = 2048
-// 38-66 us against 32-36 us.  The automatic choice keeps the tensor-core
-// kernel for the fused query prologue and output de-rotation, which only it
-// implements.
+// The automatic choice.  Short row lists favour the mma.sync kernel: the
+// tensor-core kernel's fixed cost per (query, slice) item (query tile, first
+// scores, epilogue: about 4 us) then outweighs its tiles.  Measured at
+// L = 4096, m = 4, W = 128 with H from 8 to 64: k = 64 (at most 192 rows)
+// 72-150 us against 179-182 us.  So do few heads over many queries: the
+// tensor-core kernel still runs 64-head tiles, while the mma.sync kernel
+// takes one warp (and 32-row tiles) per 16 heads: with H = 8 or 16, k = 512
+// to 2048 and 4096 to 16384 queries, 195-1837 us against 252-2338 us.  With
+// few queries the split tensor-core kernel stays ahead (decode, 64 or 256
+// sequences, k = 512 or 2048: 21-32 us against 21-48 us).  The fused query
+// prologue and output de-rotation exist only in the tensor-core kernel.
 constexpr int64_t kTcMinRows = 257;
+constexpr int kFewHeads = 16;
+constexpr int64_t kManyQueries = 2048;
+// CTAs of at most this many warps use 32-row tiles
+constexpr int kSmallTileMaxWarps = 1;
 bool attention_uses_tc(const AttnArgs& a) {
   const int32_t choice = attention_kernel_choice();
   if (choice == 2 || !tc_attention_supported(a)) return false;
   if (choice == 1) return true;
+  if (a.qprologue || a.out_derotate) return true;
   const int64_t rows = (a.idx ? (int64_t)a.top_k : a.max_entries) + a.window;
-  return rows >= kTcMinRows || a.qprologue || a.out_derotate;
+  if (rows < kTcMinRows) return false;
+  return !(a.H <= kFewHeads && a.T >= kManyQueries);
 }
 
 cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {
@@ -425,12 +436,25 @@ cudaError_t launch_attention(const Launch& L, const AttnArgs& a) {
   const int nw = a.H >= 64 ? 4 : (a.H + 15) / 16;
   const int hgroups = (a.H + nw * 16 - 1) / (nw * 16);
   const dim3 grid((unsigned)a.T, (unsigned)a.n_split, (unsigned)hgroups);
+  const bool small = nw <= kSmallTileMaxWarps;
   L.begin(kKernelAttention);
   switch (nw) {
-    case 1: attn_kernel<1><<<grid, 32, 0, L.stream>>>(a); break;
-    case 2: attn_kernel<2><<<grid, 64, 0, L.stream>>>(a); break;
-    case 3: attn_kernel<3><<<grid, 96, 0, L.stream>>>(a); break;
-    default: attn_kernel<4><<<grid, 128, 0, L.stream>>>(a); break;
+    case 1:
+      if (small) attn_kernel<1, 32><<<grid, 32, 0, L.stream>>>(a);
+      else attn_kernel<1, 64><<<grid, 32, 0, L.stream>>>(a);
+      break;
+    case 2:
+      if (small) attn_kernel<2, 32><<<grid, 64, 0, L.stream>>>(a);
+      else attn_kernel<2, 64><<<grid, 64, 0, L.stream>>>(a);
+      break;
+    case 3:
+      if (small) attn_kernel<3, 32><<<grid, 96, 0, L.stream>>>(a);
+      else attn_kernel<3, 64><<<grid, 96, 0, L.stream>>>(a);
+      break;
+    default:
+      if (small) attn_kernel<4, 32><<<grid, 128, 0, L.stream>>>(a);
+      else attn_kernel<4, 64><<<grid, 128, 0, L.stream>>>(a);
+      break;
   }
   cudaError_t e = L.end(kKernelAttention);
   if (e != cudaSuccess || a.n_split == 1) return e;

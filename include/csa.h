@@ -100,10 +100,12 @@ csa_status_t csa_set_timing_events(int32_t kernel_id, void* ev_begin, void* ev_e
  * Attention kernel choice for csa_sparse_attn_prefill, csa_sparse_attn_decode
  * and hca_attn (process-wide; a library setting with no counterpart in the
  * method).  0 = automatic (default): the tcgen05 tensor-core kernel wherever
- * it supports the call and a query's row list may hold more than 256 rows
- * (top_k, or max_entries for hca_attn, plus window) or the call asks for the
- * fused query prologue / output de-rotation, else the mma.sync kernel (faster
- * on short row lists); 1 = the tcgen05 kernel wherever it supports the
+ * it supports the call and the call asks for the fused query prologue /
+ * output de-rotation, or a query's row list may hold more than 256 rows
+ * (top_k, or max_entries for hca_attn, plus window) and the call is not one
+ * of at most 16 heads over at least 2048 queries; else the mma.sync kernel
+ * (faster on short row lists and on few heads over many queries); 1 = the
+ * tcgen05 kernel wherever it supports the
  * call, else the mma.sync kernel; 2 = always the mma.sync kernel.  Both compute the same attention within the same
  * tolerance; the split-KV slicing of a decode call may differ between them
  * (within the same workspace size).  Returns CSA_ERR_INVALID_ARG for any other

@@ -38,30 +38,34 @@ def _csa():
     return csa
 
 
-def test_auto_attention_kernel_follows_row_list_length(cuda_lib):
+def test_auto_attention_kernel_choice(cuda_lib):
     """The automatic choice runs the mma.sync kernel when a query's row list
-    holds at most 256 rows (top_k + window) and the tensor-core kernel above
-    that: its output equals, bit for bit, that of the kernel it names, and
-    matches the oracle."""
+    holds at most 256 rows (top_k + window) or when at most 16 heads cover at
+    least 2048 queries, and the tensor-core kernel otherwise: its output
+    equals, bit for bit, that of the kernel it names, and matches the
+    oracle."""
     csa = _csa()
     g = synth.generator(777)
-    L, m = 300, 4
-    kv_comp, kv_raw = synth.normal(g, (L // m, 128)), synth.normal(g, (L, 128))
+    m = 4
+    cases = [(300, 64, 64, 8, "mma_sync"), (300, 64, 64, 64, "mma_sync"),
+             (300, 128, 128, 64, "mma_sync"), (300, 129, 128, 8, "tcgen05"),
+             (300, 512, 64, 64, "tcgen05"), (2048, 512, 64, 8, "mma_sync"),
+             (2048, 512, 64, 16, "mma_sync"), (2048, 512, 64, 17, "tcgen05"),
+             (2047, 512, 64, 8, "tcgen05")]
     try:
-        for k, W, named in ((64, 64, "mma_sync"), (128, 128, "mma_sync"), (129, 128, "tcgen05"),
-                            (512, 64, "tcgen05")):
+        for L, k, W, H, named in cases:
+            kv_comp, kv_raw = synth.normal(g, (L // m, 128)), synth.normal(g, (L, 128))
             idx, cnt = synth.random_topk_lists(g, L, k, [t // m for t in range(L)])
-            for H in (8, 64):
-                q = synth.normal(g, (L, H, 128))
-                outs = {}
-                for kern in ("auto", named):
-                    csa.set_attention_kernel(kern)
-                    outs[kern] = csa.sparse_attn_prefill(dev(q), dev(kv_comp), dev(kv_raw), dev(idx), dev(cnt),
-                                                         W, 0.088)
-                assert torch.equal(outs["auto"], outs[named]), (k, W, H)
-                ref, _ = oracle.csa_prefill_attention(f64(q), f64(kv_comp), f64(kv_raw), idx.numpy(),
-                                                      cnt.numpy(), W, 0.088)
-                assert_close_attn(outs["auto"], ref, f"auto kernel k={k} W={W} H={H}")
+            q = synth.normal(g, (L, H, 128))
+            outs = {}
+            for kern in ("auto", named):
+                csa.set_attention_kernel(kern)
+                outs[kern] = csa.sparse_attn_prefill(dev(q), dev(kv_comp), dev(kv_raw), dev(idx), dev(cnt),
+                                                     W, 0.088)
+            assert torch.equal(outs["auto"], outs[named]), (L, k, W, H)
+            ref, _ = oracle.csa_prefill_attention(f64(q), f64(kv_comp), f64(kv_raw), idx.numpy(),
+                                                  cnt.numpy(), W, 0.088)
+            assert_close_attn(outs["auto"], ref, f"auto kernel L={L} k={k} W={W} H={H}")
     finally:
         csa.set_attention_kernel("auto")
 

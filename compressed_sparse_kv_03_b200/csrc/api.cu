@@ -470,9 +470,11 @@ csa_status_t run_indexer_topk(IndexerArgs base, const int64_t* q_pos, int64_t T,
     if (lay.many && tc_indexer_prefill_supported(ia, n) && topk_many_supported(ia)) {
       // the scorer's sample pass, thresholds (which zero the counts and the
       // work counter), the scorer's candidate pass, per-warp finish
+      // (no sample pass when every query's entries fit its candidate list:
+      // the thresholds are then all zero)
       e = cudaMemsetAsync(work, 0, sizeof(uint32_t), L.stream);
       if (e != cudaSuccess) return cuda_status(e, "indexer work counter memset");
-      if ((e = launch_indexer_scores_tc_prefill(L, ia, n, true)) != cudaSuccess)
+      if (2 * max_entries > ia.cand_cap && (e = launch_indexer_scores_tc_prefill(L, ia, n, true)) != cudaSuccess)
         return cuda_status(e, "indexer sample launch");
       if ((e = launch_topk_threshold_many(L, ia, top_k, n, 128 / ia.H_I)) != cudaSuccess)
         return cuda_status(e, "top-k threshold launch");

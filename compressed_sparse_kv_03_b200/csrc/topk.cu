@@ -1103,6 +1103,154 @@ __global__ void __launch_bounds__(kFWarps * 32) topk_finish_many_kernel(IndexerA
   }
 }
 
+// The same selection for entry lists of at most kSmallList entries (every
+// query's candidates then fit in registers: 32 per lane): one load of the
+// list, then a bitwise radix select over the keys in registers, from the
+// highest bit on which the keys differ, bit by bit: it stops as soon as the
+// keys at or above the current prefix are exactly k (then no tie is left),
+// else it ends with the exact k-th largest key T and how many keys equal to T
+// are taken (lowest entries first).  Selected keys and ties go to the
+// bitmaps, then the same ascending compaction.  No shared-memory histograms
+// and no second pass over the list in memory.
+constexpr int kSWarps = 4;         // queries (warps) per CTA
+constexpr int kSmallList = 1024;   // longest entry list of this form
+__global__ void __launch_bounds__(kSWarps * 32) topk_finish_small_kernel(IndexerArgs a, FinishArgs f,
+                                                                       int64_t t_count) {
+  __shared__ uint32_t sbits[kSWarps][2][kSmallList / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t tl = (int64_t)blockIdx.x * kSWarps + warp;
+  if (tl >= t_count) return;   // no block-wide barrier below
+  const int64_t t = a.t_begin + tl;
+  const int64_t n = eligible_of(a, t);
+  const int k = f.top_k;
+  int32_t* idx = f.idx_out + t * k;
+  float* sco = f.score_out ? f.score_out + t * k : nullptr;
+  const uint2* cand = a.cand + tl * a.cand_cap;
+  const int64_t c_all = (int64_t)a.cand_count[tl];
+  if (n <= k) {
+    for (int64_t j = lane; j < k; j += 32) {
+      idx[j] = j < n ? (int32_t)j : -1;
+      if (sco && j >= n) sco[j] = -INFINITY;
+    }
+    if (sco) {
+      const int64_t c = c_all < a.cand_cap ? c_all : a.cand_cap;
+      for (int64_t i = lane; i < c; i += 32) {
+        const uint2 e = cand[i];
+        if ((int64_t)e.y < n) sco[e.y] = key_score(e.x);
+      }
+    }
+    if (lane == 0) f.count_out[t] = (int32_t)n;
+    return;
+  }
+  if (c_all < k || c_all > a.cand_cap || c_all > kSmallList || n > kSmallList) {
+    if (lane == 0) a.fb_list[atomicAdd(a.fb_count, 1u)] = (uint32_t)tl;
+    return;
+  }
+  const int c = (int)c_all;
+  const int W = (int)((n + 31) >> 5);
+  uint32_t* selb = sbits[warp][0];
+  uint32_t* tieb = sbits[warp][1];
+  for (int w = lane; w < W; w += 32) {
+    selb[w] = 0u;
+    tieb[w] = 0u;
+  }
+  // candidate 32 j + lane in e[j]; a slot past the list, or an entry past
+  // the eligible range, holds entry 0xffffffff (never valid)
+  uint2 e[kSmallList / 32];
+  uint32_t vm = 0u;   // bit j: e[j] is a candidate of an eligible entry
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int j = 0; j < kSmallList / 32; ++j) {
+    const int i = 32 * j + lane;
+    e[j] = i < c ? cand[i] : make_uint2(0u, 0xffffffffu);
+    if (i < c && (int64_t)e[j].y < n) {
+      vm |= 1u << j;
+      kmin = min(kmin, e[j].x);
+      kmax = max(kmax, e[j].x);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  // every eligible key shares the bits above hb; the loop walks bit hb down
+  int need = k;
+  uint32_t prefix = kmin;
+  int stop = 0;          // lowest bit examined
+  bool early = false;    // the keys whose bits stop.. match the prefix or more are exactly k
+  if (kmin != kmax) {
+    const int hb = 31 - __clz(kmin ^ kmax);
+    prefix = hb == 31 ? 0u : kmin & (0xffffffffu << (hb + 1));
+#pragma unroll 1
+    for (int bit = hb; bit >= 0; --bit) {
+      const uint32_t want = (prefix >> bit) | 1u;
+      int cnt = 0;
+#pragma unroll
+      for (int j = 0; j < kSmallList / 32; ++j) cnt += ((vm >> j) & 1u) && (e[j].x >> bit) == want ? 1 : 0;
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      stop = bit;
+      if (cnt >= need) {
+        prefix |= 1u << bit;
+        if (cnt == need) {
+          early = true;
+          break;
+        }
+      } else {
+        need -= cnt;
+      }
+    }
+  }
+  __syncwarp();
+  // early: keys with (key >> stop) >= (prefix >> stop) are the k selected.
+  // Else T = prefix: keys above it are selected, and `need` of the keys
+  // equal to it (1 <= need <= their number), the lowest entries.
+  const uint32_t thr = prefix >> stop;
+  int ties = 0;
+#pragma unroll
+  for (int j = 0; j < kSmallList / 32; ++j) {
+    if (!((vm >> j) & 1u)) continue;
+    const uint32_t y = e[j].y, hi = e[j].x >> stop;
+    if (hi > thr || (early && hi == thr)) atomicOr(&selb[y >> 5], 1u << (y & 31));
+    else if (hi == thr) {
+      atomicOr(&tieb[y >> 5], 1u << (y & 31));
+      ++ties;
+    }
+  }
+  ties = __reduce_add_sync(0xffffffffu, ties);
+  bool consistent = early || (need >= 1 && need <= ties);
+  if (early) need = 0;
+  __syncwarp();
+  if (need > 0) warp_take_lowest_ties(selb, tieb, W, need);
+  // ascending compaction (n <= kSmallList: one bitmap word per lane), then
+  // each word's output offset kept in the tie bitmap's place for the scores
+  const uint32_t x0 = lane < W ? selb[lane] : 0u;
+  int tot;
+  const int o0 = warp_exclusive_scan(__popc(x0), tot);
+  if (lane < W) tieb[lane] = (uint32_t)o0;
+  {
+    uint32_t x = x0;
+    int o = o0;
+    while (x) {
+      const int b = __ffs(x) - 1;
+      x &= x - 1;
+      if (o < k) idx[o] = lane * 32 + b;
+      ++o;
+    }
+  }
+  __syncwarp();
+  if (sco) {
+#pragma unroll
+    for (int j = 0; j < kSmallList / 32; ++j) {
+      const uint32_t y = e[j].y;
+      if (!((vm >> j) & 1u) || !((selb[y >> 5] >> (y & 31)) & 1u)) continue;
+      const uint32_t pos = tieb[y >> 5] + (uint32_t)__popc(selb[y >> 5] & ((1u << (y & 31)) - 1u));
+      if (pos < (uint32_t)k) sco[pos] = key_score(e[j].x);
+    }
+  }
+  if (lane == 0) {
+    f.count_out[t] = k;
+    if (!consistent || tot != k) report(a.err, kErrSelect, (int32_t)t, k);
+  }
+}
+
 template <int CI>
 cudaError_t launch_finish(const Launch& L, const IndexerArgs& a, int top_k, int32_t* idx_out,
                           int32_t* count_out, float* score_out, int64_t t_count,
@@ -1225,8 +1373,13 @@ cudaError_t launch_topk_finish_many(const Launch& L, const IndexerArgs& a, int t
   cudaFuncSetAttribute(topk_finish_many_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   prefer_max_shared(topk_finish_many_kernel);
   FinishArgs f{top_k, idx_out, count_out, score_out, 0};
-  const unsigned grid = (unsigned)((t_count + kFWarps - 1) / kFWarps);
-  topk_finish_many_kernel<<<grid, kFWarps * 32, bytes, L.stream>>>(a, f, t_count);
+  if (a.max_entries <= kSmallList) {   // every list fits in registers
+    const unsigned grid = (unsigned)((t_count + kSWarps - 1) / kSWarps);
+    topk_finish_small_kernel<<<grid, kSWarps * 32, 0, L.stream>>>(a, f, t_count);
+  } else {
+    const unsigned grid = (unsigned)((t_count + kFWarps - 1) / kFWarps);
+    topk_finish_many_kernel<<<grid, kFWarps * 32, bytes, L.stream>>>(a, f, t_count);
+  }
   // the queries whose candidate count missed [top_k, cand_cap]: exact recompute
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

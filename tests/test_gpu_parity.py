@@ -391,6 +391,60 @@ def test_indexer_topk_many_queries_all_equal_scores():
     assert torch.equal(idx, want.to(torch.int32))
 
 
+@pytest.mark.parametrize("T,m,k,H_I,scores", [(4096, 4, 64, 4, True), (3000, 3, 256, 8, False),
+                                              (2500, 4, 600, 16, True)])
+def test_indexer_topk_many_queries_short_lists(T, m, k, H_I, scores):
+    """More than 2048 queries whose entry lists hold at most 1024 entries:
+    every key is a candidate and the per-warp finish selects among them in
+    registers (exact k-th key by a bitwise radix select, ties to the lower
+    index).  Checked on the first and last queries, the k boundary and 240
+    random queries, with the scores when returned."""
+    csa = _csa()
+    g = synth.generator(61 + T + k)
+    S = (T - 1) // m
+    qI = synth.normal(g, (T, H_I, 64))
+    w = synth.uniform(g, (T, H_I))
+    KI = synth.normal(g, (S, 64))
+    out = csa.indexer_topk(dev(qI), dev(w), csa.Cache(dev(KI)), m, k, return_scores=scores)
+    idx, cnt, sc = out if scores else (out[0], out[1], None)
+    picks = {0, 1, T - 2, T - 1} | set(range(k * m - 3, k * m + 4))
+    picks |= set(torch.randint(0, T, (240,), generator=g).tolist())
+    queries = sorted(t for t in picks if t < T)
+    KI64 = f64(KI)
+    stats = _check_queries(idx, cnt, qI, w, lambda t: KI64, lambda t: t // m, k, queries, sc)
+    assert stats["exact"] >= 0.99 * len(queries), stats
+
+
+def test_indexer_topk_many_queries_short_lists_exact_ties():
+    """Integer-valued keys and queries over 3000 queries with at most 749
+    entries each (the register finish): integer scores with many exact ties,
+    the lower index winning, bit for bit on 200 queries; and all-zero scores,
+    where every query takes its first k entries."""
+    csa = _csa()
+    g = synth.generator(62)
+    T, m, k, H_I = 3000, 4, 100, 8
+    S = (T - 1) // m
+    qI = torch.randint(-1, 2, (T, H_I, 64), generator=g).to(torch.bfloat16)
+    KI = torch.randint(-1, 2, (S, 64), generator=g).to(torch.bfloat16)
+    w = torch.ones((T, H_I), dtype=torch.float32)
+    idx, cnt = csa.indexer_topk(dev(qI), dev(w), csa.Cache(dev(KI)), m, k)
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    for t in sorted({0, 5, k * m, k * m + 1, T - 1} | set(torch.randint(0, T, (195,), generator=g).tolist())):
+        n = t // m
+        s = oracle.indexer_scores(f64(qI[t]), f64(w[t]), f64(KI[:n]))
+        ref = oracle.topk_select(s, k)
+        assert cnt[t] == ref.shape[0], t
+        np.testing.assert_array_equal(idx[t, :cnt[t]], ref)
+    qz = torch.ones((T, H_I, 64), dtype=torch.bfloat16)
+    kz = -torch.ones((S, 64), dtype=torch.bfloat16)
+    idx, cnt = csa.indexer_topk(dev(qz), dev(w), csa.Cache(dev(kz)), m, k)
+    idx, cnt = idx.cpu(), cnt.cpu()
+    nn = torch.clamp(torch.arange(T) // m, max=k)
+    assert torch.equal(cnt, nn.to(torch.int32))
+    want = torch.where(torch.arange(k)[None, :] < nn[:, None], torch.arange(k)[None, :], -1)
+    assert torch.equal(idx, want.to(torch.int32))
+
+
 def test_indexer_topk_exact_ties():
     """Integer-valued keys and queries make integer scores with many exact
     ties: the lower index must win, bit-exactly."""

@@ -938,6 +938,8 @@ __host__ __device__ inline int finish_many_words(int64_t max_entries) {
 __global__ void __launch_bounds__(kFWarps * 32) topk_finish_many_kernel(IndexerArgs a, FinishArgs f,
                                                                      int64_t t_count) {
   extern __shared__ __align__(16) uint32_t msm[];
+  pdl_wait();      // the scorer's candidate lists are complete
+  pdl_trigger();   // the recompute launch may start; it waits for this one
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t tl = (int64_t)blockIdx.x * kFWarps + warp;
   if (tl >= t_count) return;   // no block-wide barrier below
@@ -1117,6 +1119,8 @@ constexpr int kSmallList = 1024;   // longest entry list of this form
 __global__ void __launch_bounds__(kSWarps * 32) topk_finish_small_kernel(IndexerArgs a, FinishArgs f,
                                                                        int64_t t_count) {
   __shared__ uint32_t sbits[kSWarps][2][kSmallList / 32];
+  pdl_wait();      // the scorer's candidate lists are complete
+  pdl_trigger();   // the recompute launch may start; it waits for this one
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t tl = (int64_t)blockIdx.x * kSWarps + warp;
   if (tl >= t_count) return;   // no block-wide barrier below
@@ -1375,10 +1379,14 @@ cudaError_t launch_topk_finish_many(const Launch& L, const IndexerArgs& a, int t
   FinishArgs f{top_k, idx_out, count_out, score_out, 0};
   if (a.max_entries <= kSmallList) {   // every list fits in registers
     const unsigned grid = (unsigned)((t_count + kSWarps - 1) / kSWarps);
-    topk_finish_small_kernel<<<grid, kSWarps * 32, 0, L.stream>>>(a, f, t_count);
+    const cudaError_t e = launch_kernel(topk_finish_small_kernel, dim3(grid), dim3(kSWarps * 32), 0, L.stream,
+                                        true, a, f, t_count);
+    if (e != cudaSuccess) return e;
   } else {
     const unsigned grid = (unsigned)((t_count + kFWarps - 1) / kFWarps);
-    topk_finish_many_kernel<<<grid, kFWarps * 32, bytes, L.stream>>>(a, f, t_count);
+    const cudaError_t e = launch_kernel(topk_finish_many_kernel, dim3(grid), dim3(kFWarps * 32), bytes,
+                                        L.stream, true, a, f, t_count);
+    if (e != cudaSuccess) return e;
   }
   // the queries whose candidate count missed [top_k, cand_cap]: exact recompute
   int dev = 0, sms = 148;

@@ -31,9 +31,11 @@ __device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) {
 }
 
 // BN rows per tile (32 or 64): with few warps per CTA the 2 x BN x 256 B of
-// row tiles is what limits the CTAs resident on an SM.
+// row tiles is what limits the CTAs resident on an SM.  One-warp CTAs are
+// held to 168 registers so that 12 fit on an SM (L = 4096, H = 8, k = 64:
+// 70.2 -> 68.0 us; 16 per SM, at 128 registers, spilled: 80.4 us).
 template <int NW, int BN>
-__global__ void __launch_bounds__(NW * 32) attn_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(NW * 32, NW == 1 ? 12 : 1) attn_kernel(AttnArgs a) {
   static_assert(BN == 32 || BN == 64, "row tiles of 32 or 64");
   constexpr int NTH = NW * 32;
   __shared__ alignas(128) __nv_bfloat16 sKV[2][BN * D];

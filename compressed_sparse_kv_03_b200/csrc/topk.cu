@@ -410,6 +410,30 @@ struct FinishArgs {
   const uint32_t* list_count = nullptr;   // each CTA taking every gridDim.x-th
 };
 
+// A query with at most k eligible entries selects every one (ascending,
+// padded with -1); when scores are asked for, the scorer listed all of them
+// (tau = 0, no skipping).  Threads r, r + step, ... of the calling group.
+__device__ __forceinline__ void finish_all_eligible(const IndexerArgs& a, const FinishArgs& f, int64_t t,
+                                                    int64_t tl, int64_t n, int r, int step) {
+  const int k = f.top_k;
+  int32_t* idx = f.idx_out + t * k;
+  float* sco = f.score_out ? f.score_out + t * k : nullptr;
+  for (int64_t j = r; j < k; j += step) {
+    idx[j] = j < n ? (int32_t)j : -1;
+    if (sco && j >= n) sco[j] = -INFINITY;
+  }
+  if (sco) {
+    const uint2* cand = a.cand + tl * a.cand_cap;
+    const int64_t c_all = (int64_t)a.cand_count[tl];
+    const int64_t c = c_all < a.cand_cap ? c_all : a.cand_cap;
+    for (int64_t i = r; i < c; i += step) {
+      const uint2 e = cand[i];
+      if ((int64_t)e.y < n) sco[e.y] = key_score(e.x);
+    }
+  }
+  if (r == 0) f.count_out[t] = (int32_t)n;
+}
+
 // Dynamic shared memory: sel [Wmax], tie [Wmax] (Wmax = ceil(max_entries/32)
 // rounded up to a multiple of 4), a staging area of stage_cap (key, entry)
 // pairs (the candidates, or the fallback's keys and ids [kCandSmem] each), q
@@ -438,20 +462,7 @@ __global__ void __launch_bounds__(kThreads) topk_finish_kernel(IndexerArgs a, Fi
     const int64_t c_all = (int64_t)a.cand_count[tl];
 
     if (n <= k) {
-      // every eligible entry; when scores are asked for, the scorer listed all
-      // of them (tau = 0, no skipping)
-      for (int64_t j = tid; j < k; j += kThreads) {
-        idx[j] = j < n ? (int32_t)j : -1;
-        if (sco && j >= n) sco[j] = -INFINITY;
-      }
-      if (sco) {
-        const int64_t c = c_all < a.cand_cap ? c_all : a.cand_cap;
-        for (int64_t i = tid; i < c; i += kThreads) {
-          const uint2 e = cand[i];
-          if ((int64_t)e.y < n) sco[e.y] = key_score(e.x);
-        }
-      }
-      if (tid == 0) f.count_out[t] = (int32_t)n;
+      finish_all_eligible(a, f, t, tl, n, tid, kThreads);
       return;
     }
 
@@ -958,18 +969,7 @@ __global__ void __launch_bounds__(kFWarps * 32) topk_finish_many_kernel(IndexerA
   const uint2* cand = a.cand + tl * a.cand_cap;
   const int64_t c_all = (int64_t)a.cand_count[tl];
   if (n <= k) {
-    for (int64_t j = lane; j < k; j += 32) {
-      idx[j] = j < n ? (int32_t)j : -1;
-      if (sco && j >= n) sco[j] = -INFINITY;
-    }
-    if (sco) {
-      const int64_t c = c_all < a.cand_cap ? c_all : a.cand_cap;
-      for (int64_t i = lane; i < c; i += 32) {
-        const uint2 e = cand[i];
-        if ((int64_t)e.y < n) sco[e.y] = key_score(e.x);
-      }
-    }
-    if (lane == 0) f.count_out[t] = (int32_t)n;
+    finish_all_eligible(a, f, t, tl, n, lane, 32);
     return;
   }
   if (c_all < k || c_all > a.cand_cap) {
@@ -1132,18 +1132,7 @@ __global__ void __launch_bounds__(kSWarps * 32) topk_finish_small_kernel(Indexer
   const uint2* cand = a.cand + tl * a.cand_cap;
   const int64_t c_all = (int64_t)a.cand_count[tl];
   if (n <= k) {
-    for (int64_t j = lane; j < k; j += 32) {
-      idx[j] = j < n ? (int32_t)j : -1;
-      if (sco && j >= n) sco[j] = -INFINITY;
-    }
-    if (sco) {
-      const int64_t c = c_all < a.cand_cap ? c_all : a.cand_cap;
-      for (int64_t i = lane; i < c; i += 32) {
-        const uint2 e = cand[i];
-        if ((int64_t)e.y < n) sco[e.y] = key_score(e.x);
-      }
-    }
-    if (lane == 0) f.count_out[t] = (int32_t)n;
+    finish_all_eligible(a, f, t, tl, n, lane, 32);
     return;
   }
   if (c_all < k || c_all > a.cand_cap || c_all > kSmallList || n > kSmallList) {

@@ -5,17 +5,16 @@
 //
 // The same virtual row list, split-KV slices and online softmax as the d = 128
 // mma.sync kernel (attention.cu), laid out for 512-dim rows.  A CTA takes one
-// query, one slice and 32 heads in two groups of 16; warp w of a group owns
-// dims [128 w, 128 w + 128): it
-// contracts its quarter of Q K^T for the tile (mma.sync m16n8k16, bf16 in,
-// fp32 accumulate), the four partial score tiles are summed through shared
-// memory in a fixed order (every warp then holds the same scores and runs the
-// same online softmax), and it accumulates O for its own dims.  A CTA holds two
-// such groups of four warps (32 heads), which share each tile of rows.  Rows
-// arrive 32 at a time by cp.async into a double-buffered, XOR-swizzled tile
-// (2 x 32 KB); the query's heads sit in shared memory (32 KB) and are read
-// as MMA fragments per step, so that a thread stays within 128 registers and
-// two CTAs share an SM.
+// query, one slice and 32 heads: two groups of 16 heads, four warps each,
+// sharing every tile of rows.  Warp w of a group owns dims [128 w, 128 w +
+// 128): it contracts its quarter of Q K^T for the tile (mma.sync m16n8k16,
+// bf16 in, fp32 accumulate), the group's four partial score tiles are summed
+// through shared memory in a fixed order (all four warps then hold the same
+// scores and run the same online softmax), and it accumulates O for its own
+// dims.  Rows arrive 32 at a time by cp.async into a double-buffered,
+// XOR-swizzled tile (2 x 32 KB); the query's heads sit in shared memory
+// (32 KB) and are read as MMA fragments per step, so that a thread stays
+// within 128 registers and two CTAs share an SM.
 #include "kernels.h"
 
 namespace csa {
@@ -24,6 +23,7 @@ namespace {
 
 constexpr int kD5 = 512;         // head dim
 constexpr int kBN5 = 32;         // rows per tile
+static_assert(kBN5 == 32, "one 32-bit validity word per stage; fragments of kBN5 / 8 n-tiles");
 constexpr int kQ5 = 4;           // warps per head group; warp w owns dims [kDW5 w, kDW5 (w + 1))
 constexpr int kG5 = 2;           // head groups of 16 per CTA
 constexpr int kW5 = kQ5 * kG5;   // warps
@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(kW5 * 32, 2) attn512_kernel(AttnArgs a) {
   __nv_bfloat16* const sQ = reinterpret_cast<__nv_bfloat16*>(smem5 + kQOff5);          // kHeads5 x kD5
   float* const sS = reinterpret_cast<float*>(smem5 + kSOff5);
   __shared__ const __nv_bfloat16* sRow[2][kBN5];
-  __shared__ uint32_t sMask[2][2];
+  __shared__ uint32_t sMask[2][kBN5 / 32];   // row validity bits of each stage
 
   const int64_t i = blockIdx.x;
   const int split = blockIdx.y;
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kW5 * 32, 2) attn512_kernel(AttnArgs a) {
       }
       sRow[st][r] = p;
       const uint32_t bits = __ballot_sync(0xffffffffu, p != nullptr);
-      if (lane == 0) sMask[st][r0 >> 5] = bits;   // kBN5 = 32: word 0
+      if (lane == 0) sMask[st][r0 >> 5] = bits;
     }
   };
   // row r's 16-byte chunk ch at r * kD5 + 8 (ch ^ (r mod 8)) elements

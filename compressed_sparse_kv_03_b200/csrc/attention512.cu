@@ -172,17 +172,20 @@ __global__ void __launch_bounds__(kW5 * 32, 2) attn512_kernel(AttnArgs a) {
     // every warp); every warp sums them in the same order, so all four hold
     // the same scores bit for bit
     {
+      // lane l's four float4 slots in the order j ^ ((l >> 1) & 3): the eight
+      // lanes of a 16-byte access phase then meet eight different banks
+      const int xs = (lane >> 1) & 3;
       float* const mine = sS + (warp * 32 + lane) * kSw5;
 #pragma unroll
       for (int j = 0; j < kBN5 / 8; ++j)
-        *reinterpret_cast<float4*>(mine + 4 * j) = make_float4(s[j][0], s[j][1], s[j][2], s[j][3]);
+        *reinterpret_cast<float4*>(mine + 4 * (j ^ xs)) = make_float4(s[j][0], s[j][1], s[j][2], s[j][3]);
       __syncthreads();
 #pragma unroll
       for (int j = 0; j < kBN5 / 8; ++j) {
-        float4 t = *reinterpret_cast<const float4*>(sS + ((hgrp * kQ5 + 0) * 32 + lane) * kSw5 + 4 * j);
+        float4 t = *reinterpret_cast<const float4*>(sS + ((hgrp * kQ5 + 0) * 32 + lane) * kSw5 + 4 * (j ^ xs));
 #pragma unroll
         for (int w2 = 1; w2 < kQ5; ++w2) {
-          const float4 u = *reinterpret_cast<const float4*>(sS + ((hgrp * kQ5 + w2) * 32 + lane) * kSw5 + 4 * j);
+          const float4 u = *reinterpret_cast<const float4*>(sS + ((hgrp * kQ5 + w2) * 32 + lane) * kSw5 + 4 * (j ^ xs));
           t.x += u.x;
           t.y += u.y;
           t.z += u.z;
